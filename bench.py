@@ -1,0 +1,447 @@
+"""Benchmark of the sparse-convolution hot path on B200.
+
+One step is one pass of every stage of the path over the LiDAR-shaped
+SubmConv3d workload (batch 2 x 100k voxels in a 1440x1440x41 grid, fp16,
+64 channels), all through the C ABI:
+
+  hash build -> submanifold kernel map (probe, pairs, mask sort, tile masks)
+  -> SubmConv3d fwd 64->64 -> dgrad -> per-offset wgrad
+  -> strided support (k=2 s=2) -> strided + transposed kernel maps
+  -> strided Conv3d fwd 64->128 -> ConvTranspose3d fwd 128->64.
+
+value = effective TFLOP/s of the step (sum over the five convolution passes
+of 2 * pairs * Cin * Cout, divided by the step's device time); the kernel-map
+rate (voxels / (hash + query time)) is reported beside it.  L2 is flushed
+(256 MB write) before every timed step, outside the step's events.
+
+--impl reference times the CPU oracle on the same workload (a bounded sample
+of steps on the host cores).  Under torchrun every rank runs its own batch
+(weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+WORKLOAD = "lidar_subm"
+METRIC = "sparse-conv effective TFLOP/s + kmap Mvoxels/s at 1 B200, % of roofline"
+CIN, CMID = 64, 128
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# --------------------------------------------------------------------------- inputs
+def make_inputs(rank: int):
+    wl = synthetic.WORKLOADS[WORKLOAD]
+    seed = wl.seed + 1000 * rank
+    coords = synthetic.lidar(seed=seed, **wl.gen_args)
+    n = len(coords)
+    x = torch.from_numpy(synthetic.features(n, CIN, seed)).half()
+    g = torch.from_numpy(synthetic.features(n, CIN, seed, 1)).half()
+    w = torch.from_numpy(synthetic.weights(27, CIN, CIN, seed)).half()
+    wd = torch.from_numpy(synthetic.weights(8, CIN, CMID, seed, 1)).half()
+    wu = torch.from_numpy(synthetic.weights(8, CMID, CIN, seed, 2)).half()
+    return dict(coords=torch.from_numpy(coords), x=x, g=g, w=w, wd=wd, wu=wu)
+
+
+# --------------------------------------------------------------------------- GPU pipeline
+class Pipeline:
+    """Preallocated buffers + the sequence of C-ABI calls of one step."""
+
+    PHASES = ["hash", "kmap", "fwd", "dgrad", "wgrad", "downsample", "down_maps", "down_fwd", "up_fwd"]
+
+    def __init__(self, host: dict, dev: torch.device):
+        import sparse_convolution_voxel_b200 as scv
+        self.scv = scv
+        self.dev = dev
+        self.d = {k: v.to(dev) for k, v in host.items()}
+        n = self.n = host["coords"].shape[0]
+        self.status = scv.new_status(dev)
+        self.ws = scv.Workspace(dev)
+        self.table = torch.empty(scv.lat_hash_bytes(n, 2.0) // 8, dtype=torch.int64, device=dev)
+        self.km = scv.KernelMap(n, n, 27, dev)
+        self.y = torch.empty((n, CIN), dtype=torch.half, device=dev)
+        self.dx = torch.empty((n, CIN), dtype=torch.half, device=dev)
+        self.dw = torch.empty((27, CIN, CIN), dtype=torch.float32, device=dev)
+        self.coarse_buf = torch.empty((n, 4), dtype=torch.int32, device=dev)
+        self.z = torch.empty((n, CIN), dtype=torch.half, device=dev)
+        self.g_sub, self.g_down, self.g_up = scv.subm_geom(3), scv.strided_geom(2, 2, 0), scv.transposed_geom(2, 2, 0)
+        # the coarse support size is fixed for a fixed input: size the coarse buffers once
+        self.nc = scv.lat_downsample_coords(self.d["coords"], self.g_down, self.coarse_buf,
+                                            self.ws.get(scv.lat_downsample_ws_bytes(n, self.g_down)), self.status)
+        nc = self.nc
+        self.ctable = torch.empty(scv.lat_hash_bytes(nc, 2.0) // 8, dtype=torch.int64, device=dev)
+        self.km_down = scv.KernelMap(n, nc, 8, dev)
+        self.km_up = scv.KernelMap(nc, n, 8, dev)
+        self.yc = torch.empty((nc, CMID), dtype=torch.half, device=dev)
+        self.ws_bytes = max(scv.lat_kmap_ws_bytes(n, 27), scv.lat_kmap_ws_bytes(n, 8),
+                            scv.lat_downsample_ws_bytes(n, self.g_down),
+                            scv.lat_sconv_ws_bytes(2, CIN, CIN, self.km.c, torch.half),
+                            scv.lat_sconv_ws_bytes(0, CIN, CIN, self.km.c, torch.half),
+                            scv.lat_sconv_ws_bytes(1, CIN, CIN, self.km.c, torch.half),
+                            scv.lat_sconv_ws_bytes(0, CIN, CMID, self.km_down.c, torch.half),
+                            scv.lat_sconv_ws_bytes(0, CMID, CIN, self.km_up.c, torch.half))
+        self.wsb = self.ws.get(self.ws_bytes)
+        self.pairs = None
+
+    def step(self, ev=None):
+        """Run one step; if `ev` is a list of events, record one before each phase and one at the end."""
+        scv, d, s = self.scv, self.d, self.status
+        rec = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
+        rec(0)
+        scv.lat_hash_build(d["coords"], self.table, s)
+        rec(1)
+        scv.lat_kmap_query(self.table, d["coords"], self.g_sub, self.km.c, self.wsb, s)
+        rec(2)
+        scv.lat_sconv_fwd(d["x"], d["w"], self.km.c, self.y, self.wsb, s)
+        rec(3)
+        scv.lat_sconv_dgrad(d["g"], d["w"], self.km.c, True, self.dx, self.wsb, s)
+        rec(4)
+        scv.lat_sconv_wgrad(d["x"], d["g"], self.km.c, self.dw, self.wsb, s)
+        rec(5)
+        nc = scv.lat_downsample_coords(d["coords"], self.g_down, self.coarse_buf, self.wsb, s)
+        assert nc == self.nc
+        coarse = self.coarse_buf[:nc]
+        rec(6)
+        scv.lat_kmap_query(self.table, coarse, self.g_down, self.km_down.c, self.wsb, s)
+        scv.lat_hash_build(coarse, self.ctable, s)
+        scv.lat_kmap_query(self.ctable, d["coords"], self.g_up, self.km_up.c, self.wsb, s)
+        rec(7)
+        scv.lat_sconv_fwd(d["x"], d["wd"], self.km_down.c, self.yc, self.wsb, s)
+        rec(8)
+        scv.lat_sconv_fwd(self.yc, d["wu"], self.km_up.c, self.z, self.wsb, s)
+        rec(9)
+
+    def pair_count(self) -> int:
+        if self.pairs is None:
+            self.pairs = int(self.km.pair_off[27].item())
+        return self.pairs
+
+    def flops(self) -> float:
+        p = self.pair_count()
+        return 2.0 * (3 * p * CIN * CIN + self.n * CIN * CMID + self.n * CMID * CIN)
+
+    def phase_bytes(self) -> dict:
+        """Algorithmic bytes per phase (fp16 features, int32 indices)."""
+        n, p, nc, e = self.n, self.pair_count(), self.nc, 2
+        w = 27 * CIN * CIN * e
+        return {
+            "hash": n * 16 + n * 16,
+            "kmap": n * 16 + n * 27 * 4 + n * 4 + 8 * p,
+            "fwd": p * CIN * e + n * CIN * e + w + 8 * p,
+            "dgrad": p * CIN * e + n * CIN * e + w + 8 * p,
+            "wgrad": p * 2 * CIN * e + 27 * CIN * CIN * 4 + 8 * p,
+            "down_fwd": n * CIN * e + nc * CMID * e + 8 * CIN * CMID * e + 8 * n,
+            "up_fwd": n * CMID * e + n * CIN * e + 8 * CIN * CMID * e + 8 * n,
+        }
+
+
+def flush_l2(buf: torch.Tensor):
+    buf.add_(1)
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv") if os.path.isdir(
+            os.path.join(ROOT, "gpurun_out")) else f"/tmp/lattice_clocks_{os.getpid()}.csv"
+
+    def __enter__(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self) -> dict:
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [t.strip() for t in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def count_launches(pipe: Pipeline) -> int:
+    """Kernels one step launches, counted with the CUDA profiler (outside timing)."""
+    from torch.profiler import ProfilerActivity, profile
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        pipe.step()
+        torch.cuda.synchronize()
+    n = 0
+    for e in prof.events():
+        if e.device_type == torch.autograd.DeviceType.CUDA and "memset" not in e.name.lower() \
+                and "memcpy" not in e.name.lower():
+            n += 1
+    return n
+
+
+# --------------------------------------------------------------------------- CPU oracle arm
+def oracle_step(host: dict, nthreads: int = 0) -> float:
+    """One step of the oracle on the same input; returns its effective flops."""
+    import oracle
+    c = host["coords"].numpy()
+    x = host["x"].double().numpy()
+    g = host["g"].double().numpy()
+    w = host["w"].double().numpy()
+    nbr = oracle.kmap(c, c, 3, 1, 1, oracle.SUBM, nthreads)
+    oracle.conv_fwd(x, w, nbr, nthreads)
+    oracle.conv_dgrad(g, w, nbr, len(c), nthreads)
+    oracle.conv_wgrad(x, g, nbr, nthreads)
+    coarse = oracle.downsample(c, 2, 2, 0)
+    down = oracle.kmap(c, coarse, 2, 2, 0, oracle.STRIDED, nthreads)
+    up = oracle.kmap(coarse, c, 2, 2, 0, oracle.TRANSPOSED, nthreads)
+    yc = oracle.conv_fwd(x, host["wd"].double().numpy(), down, nthreads)
+    oracle.conv_fwd(yc, host["wu"].double().numpy(), up, nthreads)
+    p = int((nbr >= 0).sum())
+    n = len(c)
+    return 2.0 * (3 * p * CIN * CIN + n * CIN * CMID + n * CMID * CIN)
+
+
+def cpu_baseline(host: dict, budget_s: float = 15.0) -> dict:
+    import oracle
+    cores = oracle.max_threads()
+    times, flops = [], 0.0
+    t_all = time.perf_counter()
+    while True:
+        t0 = time.perf_counter()
+        flops = oracle_step(host)
+        times.append(time.perf_counter() - t0)
+        if time.perf_counter() - t_all > budget_s or len(times) >= 5:
+            break
+    t = statistics.median(times)
+    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{len(times)} full oracle steps of the {WORKLOAD} workload (median {t:.2f} s per step)"}
+
+
+def run_reference(args):
+    world, rank, local = dist_env()
+    if rank != 0:
+        return
+    host = make_inputs(0)
+    import oracle
+    cores = oracle.max_threads()
+    for _ in range(args.warmup):
+        oracle_step(host)
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        flops = oracle_step(host)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = flops * args.steps / total / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(host["coords"].shape[0], world),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{args.steps} full oracle steps of the {WORKLOAD} workload"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(n, world):
+    return {"workload": f"{WORKLOAD}: LiDAR-shaped SubmConv3d k=3 (batch 2 x 100k voxels, 1440x1440x41 grid, fp16, "
+                        f"64->64) + dgrad + wgrad + strided Conv3d k2s2 64->128 + ConvTranspose3d 128->64 on the "
+                        f"same support",
+            "voxels_per_gpu": int(n), "global_batch": 2 * world, "parallelism": f"replicas x{world}",
+            "l2": "flushed (256 MB write) before every timed step"}
+
+
+# --------------------------------------------------------------------------- main GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--lean", action="store_true",
+                    help="skip launch counting, the end-to-end pass and the CPU baseline (for profiler runs)")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+    import sparse_convolution_voxel_b200 as scv
+    try:
+        scv.load()
+    except ImportError:
+        from sparse_convolution_voxel_b200 import build as b
+        b.build()
+        scv.load()
+
+    host = make_inputs(rank)
+    pipe = Pipeline(host, dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        pipe.step()
+    torch.cuda.synchronize()
+    st = scv.lat_status_fetch(pipe.status)
+    if st:
+        raise scv.LatticeError(st, "device status after warm-up")
+    launches_per_step = None if args.lean else count_launches(pipe)
+
+    nph = len(Pipeline.PHASES)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nph + 1)] for _ in range(args.steps)]
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush_l2(flush)
+            pipe.step(evs[i])
+        torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    step_ms = [e[0].elapsed_time(e[nph]) for e in evs]
+    phase_ms = {p: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, p in enumerate(Pipeline.PHASES)}
+    total_ms = sum(step_ms)
+    if pg:
+        t = torch.tensor([total_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms = float(t.item())
+    flops = pipe.flops()
+    value = flops * world * args.steps / (total_ms * 1e-3) / 1e12
+    kmap_ms = phase_ms["hash"] + phase_ms["kmap"]
+
+    # end to end through the public API: host inputs in, results back to the host
+    e2e = None
+    if rank == 0 and not args.lean:
+        e2e = measure_e2e(host, dev, steps=max(3, min(args.steps, 10)))
+
+    if rank == 0:
+        hbm, tc, src = load_peaks()
+        pb = pipe.phase_bytes()
+        dominant = max(pb, key=lambda p: phase_ms[p])
+        achieved = pb[dominant] / (phase_ms[dominant] * 1e-3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "config": config_dict(pipe.n, world),
+            "kmap_mvoxels_per_s": pipe.n / (kmap_ms * 1e-3) / 1e6,
+            "pairs": pipe.pair_count(), "coarse_voxels": pipe.nc,
+            "phase_ms": {k: round(v, 4) for k, v in phase_ms.items()},
+            "roofline": {"kernel": dominant, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                         "frac": achieved / hbm, "traffic": None, "peak_source": f"{src} hbm_gbs",
+                         "per_phase_frac": {p: round(pb[p] / (phase_ms[p] * 1e-3) / 1e9 / hbm, 4) for p in pb}},
+            "gpu_launches": None if launches_per_step is None else launches_per_step * args.steps,
+            "e2e": e2e,
+            "clocks": clk.summary(),
+        }
+        if not args.no_cpu_baseline and not args.lean and world == 1:
+            line["cpu_baseline"] = cpu_baseline(host)
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def measure_e2e(host: dict, dev: torch.device, steps: int) -> dict:
+    """Same step through the public API with inputs copied from pinned host memory and
+    the results copied back, copies inside the timed region."""
+    pinned = {k: v.pin_memory() for k, v in host.items()}
+    pipe = Pipeline(host, dev)
+    outs = {"y": torch.empty(pipe.y.shape, dtype=torch.half).pin_memory(),
+            "dx": torch.empty(pipe.dx.shape, dtype=torch.half).pin_memory(),
+            "dw": torch.empty(pipe.dw.shape, dtype=torch.float32).pin_memory(),
+            "z": torch.empty(pipe.z.shape, dtype=torch.half).pin_memory()}
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = sum(v.numel() * v.element_size() for v in outs.values())
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def one():
+        for k, v in pinned.items():
+            pipe.d[k].copy_(v, non_blocking=True)
+        pipe.step()
+        outs["y"].copy_(pipe.y, non_blocking=True)
+        outs["dx"].copy_(pipe.dx, non_blocking=True)
+        outs["dw"].copy_(pipe.dw, non_blocking=True)
+        outs["z"].copy_(pipe.z, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
+        flush_l2(flush)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        one()
+        b.record()
+        torch.cuda.synchronize()
+        ms.append(a.elapsed_time(b))
+    t = sum(ms) / len(ms)
+    return {"value": pipe.flops() / (t * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": t}
+
+
+if __name__ == "__main__":
+    main()

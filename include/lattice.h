@@ -1,0 +1,240 @@
+/*
+ * lattice.h -- C ABI of the B200 sparse-convolution library (liblattice.so).
+ *
+ * Sparse convolution over coordinate-indexed feature rows: a sparse tensor is
+ * an int32 (N, 4) array of coordinate rows (batch, x, y, z) plus an (N, C)
+ * feature array, where coordinate row i owns feature row i and batch is the
+ * first column (Torch Lattice docs, "Migrating from TorchSparse", section
+ * "Sparse tensor expectations").  The library covers the three convolution
+ * families of that page's "Convolution mapping" table:
+ *   - SubmConv3d       preserves the input support;
+ *   - Conv3d, strided  generates a downsampled support;
+ *   - ConvTranspose3d  consumes an existing relation back onto a known support;
+ * and the hashing, kernel-map construction and coordinate query that feed
+ * them ("What remains familiar": CUDA kernels cover sparse convolution,
+ * hashing and coordinate query).  Forward, data-gradient and per-offset
+ * weight-gradient passes are provided, since models train with standard
+ * optimizers (same page) and TorchSparse++ targets training as well as
+ * inference (TorchSparse++ abstract).
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer is a DEVICE pointer to a caller-allocated, contiguous,
+ *     row-major buffer, unless documented as host.  The library never
+ *     allocates or frees memory and keeps no state between calls except
+ *     per-device kernel attributes set on first use.
+ *   - Work is enqueued on `stream` (NULL = legacy default stream) and is
+ *     asynchronous, except lat_downsample_coords and lat_status_fetch,
+ *     which synchronise `stream` because they return a device-computed value.
+ *   - Argument errors are detected on the host and returned synchronously;
+ *     nothing is enqueued then.  Errors found by a kernel (range, duplicate,
+ *     table full, capacity, malformed map) are OR-ed into the caller's int32
+ *     status word `d_status` (device memory, may be NULL to ignore) and read
+ *     back with lat_status_fetch.
+ *   - Scratch memory (`ws`, `ws_bytes`) is supplied by the caller; each op
+ *     has a *_ws_bytes query returning the size it needs.  A NULL `ws` with a
+ *     zero size is valid when the query returns 0.
+ *   - Feature / weight / output arrays share one element type (lat_dtype),
+ *     except the weight gradient, which is always fp32.
+ *
+ * Readings taken where the pages are silent (the same readings drive the
+ * CPU oracle used by the tests):
+ *   - cross-correlation: y(q) = sum_k x(in(q, k)) * W[k], like dense conv3d;
+ *   - offset index k = (ix*Ky + iy)*Kz + iz for offset vector (ix, iy, iz);
+ *   - input coordinate of output q at offset k: stride*q + (ix,iy,iz) - pad
+ *     (SubmConv3d: stride 1, pad (K-1)/2);
+ *   - weights are (K^3, Cin, Cout) row-major; no bias;
+ *   - the transposed relation links fine output p to coarse input q when
+ *     stride*q + (ix,iy,iz) - pad == p;
+ *   - a 16-bit output is the fp32 accumulator rounded to nearest even once.
+ */
+#ifndef LATTICE_H
+#define LATTICE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; NULL selects the legacy default stream. */
+typedef struct CUstream_st *lat_stream;
+
+/* Status codes.  Values are bit flags so a device status word can hold several. */
+typedef enum {
+    LAT_OK = 0,
+    LAT_ERR_ARG = 1,          /* invalid argument (host check)                          */
+    LAT_ERR_COORD_RANGE = 2,  /* coordinate outside the packable key range (device)     */
+    LAT_ERR_DUPLICATE = 4,    /* two coordinate rows are equal (device)                 */
+    LAT_ERR_TABLE_FULL = 8,   /* hash probing visited every slot (device)               */
+    LAT_ERR_CAPACITY = 16,    /* an output buffer is smaller than the result (device)   */
+    LAT_ERR_UNSUPPORTED = 32, /* shape / dtype combination not implemented (host)       */
+    LAT_ERR_CUDA = 64,        /* a CUDA runtime call failed (host)                      */
+    LAT_ERR_WORKSPACE = 128,  /* ws_bytes smaller than the *_ws_bytes query (host)      */
+    LAT_ERR_BAD_MAP = 256     /* a kernel map holds a row index outside [0, n_in) (device) */
+} lat_status;
+
+typedef enum { LAT_F32 = 0, LAT_F16 = 1, LAT_BF16 = 2 } lat_dtype;
+
+/* Support semantics ("Convolution mapping" table of the migration page). */
+typedef enum {
+    LAT_SUBM = 0,       /* SubmConv3d: output coords are the input coords themselves  */
+    LAT_STRIDED = 1,    /* Conv3d with stride: output coords from lat_downsample_coords */
+    LAT_TRANSPOSED = 2  /* ConvTranspose3d: fine outputs, coarse inputs               */
+} lat_mode;
+
+/* Convolution geometry.  K^3 = ksize[0]*ksize[1]*ksize[2] must be in [1, 32]. */
+typedef struct {
+    int32_t ksize[3];
+    int32_t stride[3]; /* all 1 for LAT_SUBM                                  */
+    int32_t pad[3];    /* LAT_SUBM: (K-1)/2 per axis, K odd                    */
+    int32_t mode;      /* lat_mode                                             */
+} lat_geom;
+
+/* Rows per output tile of the convolution kernels (and of tile_mask). */
+#define LAT_TILE_ROWS 128
+
+/*
+ * Kernel map ("relation" in the migration page's "Backend and configuration
+ * differences" section): for every output row j and offset k, the input row
+ * found at the offset coordinate.  All arrays are caller-allocated device
+ * buffers that lat_kmap_query fills:
+ *   nbr       int32  [k3][n_out]  nbr[k*n_out + j] = input row, or -1
+ *   mask      uint32 [n_out]      bit k set iff nbr[k*n_out + j] >= 0
+ *   perm      int32  [n_out]      output rows sorted by mask (stable: ties keep
+ *                                 ascending row order)
+ *   tile_mask uint32 [ceil(n_out/LAT_TILE_ROWS)]  OR of mask over each run of
+ *                                 LAT_TILE_ROWS consecutive entries of perm
+ *   pair_off  int64  [k3 + 1]     pair_off[k] = first pair of offset k
+ *   pair_in   int32  [pair_capacity]  input row of each pair
+ *   pair_out  int32  [pair_capacity]  output row of each pair
+ * Pairs are grouped by offset (ascending k) and, within an offset, sorted by
+ * ascending output row, so the lists are deterministic.  n_in, n_out and k3
+ * are set by the caller before lat_kmap_query; mode records the geometry's
+ * mode (written by the query).
+ */
+typedef struct {
+    int32_t *nbr;
+    uint32_t *mask;
+    int32_t *perm;
+    uint32_t *tile_mask;
+    int64_t *pair_off;
+    int32_t *pair_in;
+    int32_t *pair_out;
+    int64_t pair_capacity;
+    int64_t n_in;
+    int64_t n_out;
+    int32_t k3;
+    int32_t mode;
+} lat_kmap;
+
+/* ---------------------------------------------------------------- hashing --
+ * GPU open-addressing hash of packed 64-bit coordinate keys ("hashing" in
+ * the CUDA kernel list of the migration page; capacity knob
+ * torch_lattice.backends.hash_rsv_ratio of "Backend and configuration
+ * differences").
+ *
+ * Key packing: key = b<<48 | (x+2^15)<<32 | (y+2^15)<<16 | (z+2^15), so the
+ * unsigned key order is the lexicographic (b, x, y, z) order.  b must lie in
+ * [0, 65534] and x, y, z in [-32768, 32767]; rows outside are skipped and
+ * flag LAT_ERR_COORD_RANGE.  The table is an array of 16-byte slots
+ * {uint64 key; int32 row; int32 unused} with a power-of-two slot count; an
+ * empty slot holds key 0xFFFF...F.  Keys are placed with the SplitMix64
+ * output function and linear probing.
+ */
+
+/* Bytes of a table for n rows: 16 * next_pow2(max(ceil(rsv_ratio*n), 64)).
+ * rsv_ratio must be >= 1 (default 2).  Returns 0 on invalid input. */
+size_t lat_hash_bytes(int64_t n, float rsv_ratio);
+
+/* Insert coords[0..n) (int32 (n,4)) into `table` (table_bytes from
+ * lat_hash_bytes; clears it first).  A duplicate coordinate keeps the lowest
+ * row and flags LAT_ERR_DUPLICATE; a full table flags LAT_ERR_TABLE_FULL. */
+lat_status lat_hash_build(const int32_t *coords, int64_t n, void *table, size_t table_bytes,
+                          int32_t *d_status, lat_stream stream);
+
+/* ------------------------------------------------------ kernel-map query --
+ * For every output row and each of the K^3 offsets, probe the input table
+ * (built by lat_hash_build over the n_in input rows) and fill `map` (see
+ * lat_kmap).  Coordinate query + kernel-map construction of the migration
+ * page ("What remains familiar"; "Sparse tensor expectations").
+ *   LAT_SUBM       out_coords must be the input coordinate rows themselves.
+ *   LAT_STRIDED    out_coords come from lat_downsample_coords (same geom).
+ *   LAT_TRANSPOSED table holds the coarse rows, out_coords the fine rows.
+ * pair_capacity may be as large as n_out*k3; pairs beyond it are dropped and
+ * flag LAT_ERR_CAPACITY (pair_off is still exact). */
+size_t lat_kmap_ws_bytes(int64_t n_out, int32_t k3);
+lat_status lat_kmap_query(const void *table, size_t table_bytes, const int32_t *out_coords,
+                          const lat_geom *geom, lat_kmap *map, void *ws, size_t ws_bytes,
+                          int32_t *d_status, lat_stream stream);
+
+/* --------------------------------------------------- support generation --
+ * Output support of a strided Conv3d ("Convolution mapping": strided forward
+ * convolution creates a downsampled support): every coarse q whose window
+ * {stride*q + (ix,iy,iz) - pad} holds at least one active input, batch
+ * unchanged.  Written to out_coords (int32 (out_capacity, 4)) sorted by packed
+ * key, i.e. in canonical (b, x, y, z) order, so the result is deterministic.
+ * geom->mode must be LAT_STRIDED.  Synchronises `stream` and writes the row
+ * count to *n_out (HOST pointer).  out_capacity >= n_in is enough when
+ * ksize == stride and pad == 0; in general n_in * prod(ceil(ksize/stride))
+ * bounds the count.  Too small a capacity returns LAT_ERR_CAPACITY with the
+ * needed count in *n_out. */
+size_t lat_downsample_ws_bytes(int64_t n_in, const lat_geom *geom);
+lat_status lat_downsample_coords(const int32_t *coords, int64_t n_in, const lat_geom *geom,
+                                 int32_t *out_coords, int64_t out_capacity, int64_t *n_out,
+                                 void *ws, size_t ws_bytes, int32_t *d_status, lat_stream stream);
+
+/* ------------------------------------------------------------ convolution --
+ * y[j] = sum over k with nbr[k][j] >= 0 of x[nbr[k][j]] . W[k]
+ * x (map->n_in, cin), w (k3, cin, cout), y (map->n_out, cout), all `dtype`;
+ * accumulation in fp32; every output row is written exactly once (rows with
+ * no neighbour get zeros).  Implicit-GEMM dataflow (TorchSparse++ abstract;
+ * the migration page requires every dataflow to give the same result for a
+ * fixed relation and weight tensor).  cin and cout must be multiples of 8 and
+ * at most 256 (fp32) / 128 (fp16, bf16 on tensor cores). */
+size_t lat_sconv_ws_bytes(int32_t op, int32_t cin, int32_t cout, const lat_kmap *map,
+                          lat_dtype dtype);
+#define LAT_OP_FWD 0
+#define LAT_OP_DGRAD 1
+#define LAT_OP_WGRAD 2
+lat_status lat_sconv_fwd(const void *x, int32_t cin, const void *w, int32_t cout,
+                         const lat_kmap *map, void *y, lat_dtype dtype, void *ws, size_t ws_bytes,
+                         int32_t *d_status, lat_stream stream);
+
+/* Data gradient: dx[i] = sum over pairs (i, j, k) of dy[j] . W[k]^T.
+ * `map` is the relation seen from dx's rows:
+ *   SubmConv3d        pass the forward map and flip_offsets = 1 (the pair
+ *                     (i, j, k) is found at nbr[k3-1-k][i]);
+ *   strided Conv3d    pass the LAT_TRANSPOSED map of the same geometry
+ *                     (fine rows as outputs), flip_offsets = 0;
+ *   ConvTranspose3d   pass the LAT_STRIDED map, flip_offsets = 0.
+ * dy (map->n_in... rows of the forward output, cout), w (k3, cin, cout) as in
+ * the forward pass, dx (map->n_out, cin). */
+lat_status lat_sconv_dgrad(const void *dy, int32_t cout, const void *w, int32_t cin,
+                           const lat_kmap *map, int32_t flip_offsets, void *dx, lat_dtype dtype,
+                           void *ws, size_t ws_bytes, int32_t *d_status, lat_stream stream);
+
+/* Per-offset weight gradient: dW[k] = sum over pairs (i, j) of offset k of
+ * x[i]^T dy[j], fp32 (k3, cin, cout), from the forward map's pair lists.
+ * Deterministic: fixed chunks of pairs, each reduced into a partial in fp32,
+ * partials summed in a fixed order (no atomics). */
+lat_status lat_sconv_wgrad(const void *x, int32_t cin, const void *dy, int32_t cout,
+                           const lat_kmap *map, float *dw, lat_dtype dtype, void *ws,
+                           size_t ws_bytes, int32_t *d_status, lat_stream stream);
+
+/* ---------------------------------------------------------------- misc --- */
+
+/* Synchronise `stream`, then return the status word at d_status (device). */
+int32_t lat_status_fetch(const int32_t *d_status, lat_stream stream);
+
+/* Static description of a status value (bit flags are listed by lowest bit). */
+const char *lat_status_string(int32_t status);
+
+/* Library ABI version (major*100 + minor). */
+int32_t lat_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LATTICE_H */

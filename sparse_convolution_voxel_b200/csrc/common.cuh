@@ -1,0 +1,115 @@
+// Device helpers shared by the liblattice kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "lattice.h"
+
+namespace lat {
+
+constexpr uint64_t kEmptyKey = ~0ull;
+
+// One hash slot: 16 bytes so a single vector load resolves a probe.
+struct __align__(16) Slot {
+    unsigned long long key;
+    unsigned int row;  // unsigned so atomicMin keeps the lowest row; 0xFFFFFFFF = none
+    unsigned int unused;
+};
+
+// Packed key of (b, x, y, z); returns false when a field is outside the key range.
+__device__ __forceinline__ bool pack_key(int b, int x, int y, int z, uint64_t &key) {
+    if (b < 0 || b > 65534 || x < -32768 || x > 32767 || y < -32768 || y > 32767 || z < -32768 ||
+        z > 32767)
+        return false;
+    key = (uint64_t(b) << 48) | (uint64_t(x + 32768) << 32) | (uint64_t(y + 32768) << 16) |
+          uint64_t(z + 32768);
+    return true;
+}
+
+__device__ __forceinline__ void unpack_key(uint64_t key, int4 &c) {
+    c.x = int(key >> 48);
+    c.y = int((key >> 32) & 0xFFFF) - 32768;
+    c.z = int((key >> 16) & 0xFFFF) - 32768;
+    c.w = int(key & 0xFFFF) - 32768;
+}
+
+// SplitMix64 output function (Steele, Lea & Flood, OOPSLA 2014): a full-avalanche
+// 64-bit mixer, so consecutive voxels land in unrelated slots.
+__device__ __forceinline__ uint64_t mix64(uint64_t z) {
+    z += 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+// Look a key up; returns the row or -1.  Probing is bounded by the slot count.
+__device__ __forceinline__ int hash_find(const Slot *__restrict__ slots, uint64_t cap_mask,
+                                         uint64_t key) {
+    uint64_t s = mix64(key) & cap_mask;
+    for (uint64_t probe = 0; probe <= cap_mask; ++probe) {
+        const ulonglong2 v = __ldg(reinterpret_cast<const ulonglong2 *>(slots + s));
+        if (v.x == key) return int(unsigned(v.y));
+        if (v.x == kEmptyKey) return -1;
+        s = (s + 1) & cap_mask;
+    }
+    return -1;
+}
+
+__device__ __forceinline__ void flag(int32_t *d_status, int32_t bits) {
+    if (d_status) atomicOr(d_status, bits);
+}
+
+// floor division by a positive divisor
+__device__ __forceinline__ int floordiv(int a, int b) {
+    int q = a / b;
+    return (a % b != 0 && a < 0) ? q - 1 : q;
+}
+
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+    static __device__ __forceinline__ float to_f(float v) { return v; }
+    static __device__ __forceinline__ float from_f(float v) { return v; }
+};
+template <> struct Elem<__half> {
+    static __device__ __forceinline__ float to_f(__half v) { return __half2float(v); }
+    static __device__ __forceinline__ __half from_f(float v) { return __float2half_rn(v); }
+};
+template <> struct Elem<__nv_bfloat16> {
+    static __device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+    static __device__ __forceinline__ __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
+};
+
+}  // namespace lat
+
+// Host-side error plumbing.
+#define LAT_CUDA_TRY(expr)                                   \
+    do {                                                     \
+        cudaError_t _e = (expr);                             \
+        if (_e != cudaSuccess) return LAT_ERR_CUDA;          \
+    } while (0)
+
+namespace lat {
+inline int num_sms() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+inline bool pow2(uint64_t v) { return v && !(v & (v - 1)); }
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Carves consecutive 256-byte aligned sub-buffers out of a caller workspace.
+struct Carver {
+    char *base;
+    size_t used = 0;
+    explicit Carver(void *b) : base(static_cast<char *>(b)) {}
+    template <typename T> T *take(size_t count) {
+        used = align_up(used, 256);
+        T *p = base ? reinterpret_cast<T *>(base + used) : nullptr;
+        used += count * sizeof(T);
+        return p;
+    }
+};
+}  // namespace lat

@@ -1,0 +1,72 @@
+// GPU open-addressing hash of packed coordinate keys (lat_hash_bytes, lat_hash_build).
+//
+// Torch Lattice docs, "Migrating from TorchSparse": hashing is one of the CUDA
+// kernels of the library ("What remains familiar") and its capacity knob is
+// torch_lattice.backends.hash_rsv_ratio ("Backend and configuration
+// differences").  Design: 16-byte slots {key, row}, SplitMix64 placement,
+// linear probing bounded by the slot count, 64-bit atomicCAS to claim a slot
+// and an unsigned atomicMin on the row so that duplicates keep the lowest row
+// deterministically.
+#include "common.cuh"
+
+namespace lat {
+
+__global__ void __launch_bounds__(256) hash_insert_kernel(const int4 *__restrict__ coords, int64_t n,
+                                                          Slot *__restrict__ slots, uint64_t cap_mask,
+                                                          int32_t *d_status) {
+    int32_t bad = 0;
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const int4 c = __ldg(coords + i);
+        uint64_t key;
+        if (!pack_key(c.x, c.y, c.z, c.w, key)) {
+            bad |= LAT_ERR_COORD_RANGE;
+            continue;
+        }
+        uint64_t s = mix64(key) & cap_mask;
+        bool placed = false;
+        for (uint64_t probe = 0; probe <= cap_mask; ++probe) {
+            unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(&slots[s].key);
+            if (cur == kEmptyKey)
+                cur = atomicCAS(&slots[s].key, (unsigned long long)kEmptyKey, (unsigned long long)key);
+            if (cur == kEmptyKey || cur == key) {
+                atomicMin(&slots[s].row, unsigned(i));
+                if (cur == key) bad |= LAT_ERR_DUPLICATE;
+                placed = true;
+                break;
+            }
+            s = (s + 1) & cap_mask;
+        }
+        if (!placed) bad |= LAT_ERR_TABLE_FULL;
+    }
+    if (bad) flag(d_status, bad);
+}
+
+}  // namespace lat
+
+extern "C" size_t lat_hash_bytes(int64_t n, float rsv_ratio) {
+    if (n < 0 || !(rsv_ratio >= 1.0f) || n > (int64_t(1) << 31)) return 0;
+    double want = double(rsv_ratio) * double(n);
+    uint64_t cap = 64;
+    while (double(cap) < want) cap <<= 1;
+    return size_t(cap) * sizeof(lat::Slot);
+}
+
+extern "C" lat_status lat_hash_build(const int32_t *coords, int64_t n, void *table, size_t table_bytes,
+                                     int32_t *d_status, lat_stream stream) {
+    using namespace lat;
+    if (n < 0 || n >= (int64_t(1) << 31) || (n > 0 && !coords) || !table) return LAT_ERR_ARG;
+    if (table_bytes % sizeof(Slot) || !pow2(table_bytes / sizeof(Slot)) || table_bytes / sizeof(Slot) < 64)
+        return LAT_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(coords) % 16 || reinterpret_cast<uintptr_t>(table) % 16) return LAT_ERR_ARG;
+    const uint64_t cap = table_bytes / sizeof(Slot);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    LAT_CUDA_TRY(cudaMemsetAsync(table, 0xFF, table_bytes, s));
+    if (n == 0) return LAT_OK;
+    const int threads = 256;
+    const int64_t blocks = (n + threads - 1) / threads;
+    hash_insert_kernel<<<unsigned(blocks), threads, 0, s>>>(reinterpret_cast<const int4 *>(coords), n,
+                                                             static_cast<Slot *>(table), cap - 1, d_status);
+    LAT_CUDA_TRY(cudaGetLastError());
+    return LAT_OK;
+}

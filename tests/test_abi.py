@@ -1,0 +1,73 @@
+"""The C-ABI library loads and exports every symbol include/lattice.h declares (CPU only).
+
+Only host-side behaviour is exercised here: size queries, status strings and
+argument checks that return before anything is enqueued on a GPU.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_convolution_voxel_b200 as scv
+from sparse_convolution_voxel_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_convolution_voxel_b200 import build
+    build.build()
+    return _lib.load()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "lattice.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lat_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert _declared() == sorted(_lib.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_size_queries(lib):
+    assert scv.lat_hash_bytes(1000, 2.0) == 16 * 2048
+    assert scv.lat_hash_bytes(10, 2.0) == 16 * 64
+    assert scv.lat_hash_bytes(1000, 0.5) == 0
+    assert scv.lat_kmap_ws_bytes(200_000, 27) > 0
+    assert scv.lat_kmap_ws_bytes(10, 33) == 0
+    g = scv.strided_geom(2, 2, 0)
+    assert scv.lat_downsample_ws_bytes(1000, g) > 0
+    assert scv.lat_downsample_ws_bytes(1000, scv.subm_geom(3)) == 0
+
+
+def test_status_strings_and_version(lib):
+    assert scv.lat_status_string(0) == "ok"
+    assert "duplicate" in scv.lat_status_string(4)
+    assert scv.lat_version() >= 100
+
+
+def test_host_argument_checks_return_without_gpu(lib):
+    P = ctypes.c_void_p
+    # null coords with n > 0
+    assert lib.lat_hash_build(None, 10, P(16), 16 * 64, None, None) == 1
+    # table size not a power of two
+    assert lib.lat_hash_build(P(16), 10, P(16), 16 * 65, None, None) == 1
+    km = _lib.lat_kmap()
+    km.k3 = 27
+    km.n_out = 10
+    km.n_in = 10
+    bad = scv.make_geom(3, 1, 0, scv.LAT_SUBM)       # submanifold pad must be (K-1)/2
+    assert lib.lat_kmap_query(P(16), 16 * 64, P(16), ctypes.byref(bad), ctypes.byref(km), None, 0, None, None) == 1
+    km.k3 = 40
+    assert lib.lat_sconv_fwd(P(16), 16, P(16), 16, ctypes.byref(km), P(16), 0, None, 0, None, None) == 1
+    km.k3 = 27
+    # channel counts must be multiples of 8
+    assert lib.lat_sconv_fwd(P(16), 12, P(16), 16, ctypes.byref(km), P(16), 0, None, 0, None, None) == 1

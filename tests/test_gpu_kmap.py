@@ -1,0 +1,178 @@
+"""Hash table, kernel-map query and support generation on the GPU against the oracle.
+
+Integer results are compared bit-exactly: neighbour tables, masks, pair
+lists (canonical order: offset, then output row), the stable mask sort, tile
+masks and generated coordinates.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from tests.util import check_kmap, rand_coords, u32
+
+pytestmark = pytest.mark.gpu
+
+scv = pytest.importorskip("sparse_convolution_voxel_b200")
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def _subm(coords, ks=(3, 3, 3), d_status=None):
+    c = _dev(coords)
+    table = scv.hash_table(c, 2.0, d_status)
+    g = scv.subm_geom(ks)
+    return scv.kernel_map(table, len(coords), c, g, d_status=d_status), table
+
+
+# --------------------------------------------------------------------------- hash table
+def test_hash_table_places_every_key_reachably():
+    rng = np.random.default_rng(0)
+    coords = rand_coords(rng, 3000, -40, 40, batch=3)
+    st = scv.new_status()
+    table = scv.hash_table(_dev(coords), 2.0, st)
+    scv.check_status(st)
+    t = table.cpu().numpy().view(np.uint64).reshape(-1, 2)
+    keys, rows = t[:, 0], (t[:, 1] & np.uint64(0xFFFFFFFF)).astype(np.int64)
+    cap = len(keys)
+    empty = np.uint64(0xFFFFFFFFFFFFFFFF)
+    occupied = np.nonzero(keys != empty)[0]
+    assert len(occupied) == len(coords)
+    want = {oracle.pack_key(*map(int, r)): i for i, r in enumerate(coords)}
+    for s in occupied:
+        k = int(keys[s])
+        assert want[k] == rows[s]
+        home = oracle.splitmix64(k) & (cap - 1)
+        d = (s - home) % cap                       # linear probing: no empty slot between home and s
+        assert all(keys[(home + e) % cap] != empty for e in range(d))
+
+
+def test_hash_flags_duplicates_and_keeps_lowest_row():
+    coords = np.array([[0, 1, 2, 3], [0, 5, 5, 5], [0, 1, 2, 3], [0, 1, 2, 3]], np.int32)
+    st = scv.new_status()
+    table = scv.hash_table(_dev(coords), 2.0, st)
+    assert scv.lat_status_fetch(st) & 4
+    t = table.cpu().numpy().view(np.uint64).reshape(-1, 2)
+    k = np.uint64(oracle.pack_key(0, 1, 2, 3))
+    assert int(t[t[:, 0] == k, 1][0] & np.uint64(0xFFFFFFFF)) == 0
+
+
+def test_hash_flags_out_of_range_coordinates():
+    coords = np.array([[0, 40000, 0, 0], [0, 1, 1, 1], [70000, 0, 0, 0]], np.int32)
+    st = scv.new_status()
+    scv.hash_table(_dev(coords), 2.0, st)
+    assert scv.lat_status_fetch(st) & 2
+
+
+def test_hash_flags_full_table():
+    rng = np.random.default_rng(1)
+    coords = rand_coords(rng, 100, 0, 10)
+    table = torch.empty(2 * 64, dtype=torch.int64, device="cuda")   # 64 slots < 100 rows
+    st = scv.new_status()
+    scv.lat_hash_build(_dev(coords), table, st)
+    assert scv.lat_status_fetch(st) & 8
+
+
+# --------------------------------------------------------------------------- submanifold maps
+@pytest.mark.parametrize("n,batch,lo,hi", [(1, 1, 0, 4), (127, 1, 0, 8), (129, 2, -5, 5), (1000, 3, -12, 12)])
+def test_subm_kmap_small_ragged(n, batch, lo, hi):
+    rng = np.random.default_rng(n)
+    coords = rand_coords(rng, n, lo, hi, batch)
+    st = scv.new_status()
+    km, _ = _subm(coords, d_status=st)
+    scv.check_status(st)
+    check_kmap(km, oracle.kmap(coords, coords, 3, 1, 1, oracle.SUBM))
+
+
+def test_subm_kmap_empty():
+    coords = np.zeros((0, 4), np.int32)
+    km, _ = _subm(coords)
+    torch.cuda.synchronize()
+    assert km.pair_off.cpu().numpy().tolist() == [0] * 28
+
+
+@pytest.mark.parametrize("ks", [(5, 3, 1), (1, 1, 1), (3, 3, 1), (5, 5, 1)])
+def test_subm_kmap_other_kernels(ks):
+    rng = np.random.default_rng(3)
+    coords = rand_coords(rng, 700, -9, 9, 2)
+    km, _ = _subm(coords, ks)
+    check_kmap(km, oracle.kmap(coords, coords, ks, 1, oracle.subm_pad(ks), oracle.SUBM))
+
+
+@pytest.mark.parametrize("name", ["subm_small", "lidar_subm", "images_subm", "lidar_train"])
+def test_subm_kmap_full_workloads(name):
+    w = synthetic.WORKLOADS[name]
+    coords = w.coords()
+    st = scv.new_status()
+    km, _ = _subm(coords, w.ksize, st)
+    scv.check_status(st)
+    check_kmap(km, oracle.kmap(coords, coords, w.ksize, 1, oracle.subm_pad(w.ksize), oracle.SUBM))
+
+
+def test_kmap_runs_are_deterministic():
+    coords = synthetic.WORKLOADS["lidar_subm"].coords()
+    a, _ = _subm(coords)
+    b, _ = _subm(coords)
+    P = int(a.pair_off[-1].item())
+    n, k3 = a.n_out, a.k3
+    for f, m in (("nbr", n * k3), ("mask", n), ("perm", n), ("tile_mask", a.ntiles), ("pair_off", k3 + 1),
+                 ("pair_in", P), ("pair_out", P)):
+        assert torch.equal(getattr(a, f)[:m], getattr(b, f)[:m]), f
+
+
+def test_kmap_flags_small_pair_capacity():
+    rng = np.random.default_rng(5)
+    coords = rand_coords(rng, 500, 0, 9)
+    c = _dev(coords)
+    st = scv.new_status()
+    table = scv.hash_table(c, 2.0, st)
+    km = scv.kernel_map(table, len(coords), c, scv.subm_geom(3), d_status=st, pair_capacity=100)
+    assert scv.lat_status_fetch(st) & 16
+    ref = oracle.kmap(coords, coords, 3, 1, 1, oracle.SUBM)
+    assert np.array_equal(km.pair_off.cpu().numpy(), oracle.pairs(ref)[0])
+
+
+# --------------------------------------------------------------------------- strided / transposed
+@pytest.mark.parametrize("ks,st_,pd", [((2, 2, 2), (2, 2, 2), (0, 0, 0)), ((3, 3, 3), (2, 2, 2), (1, 1, 1)),
+                                       ((3, 2, 1), (2, 1, 3), (0, 1, 0))])
+def test_downsample_and_strided_maps_small(ks, st_, pd):
+    rng = np.random.default_rng(11)
+    coords = rand_coords(rng, 900, -10, 10, 2)
+    c = _dev(coords)
+    st = scv.new_status()
+    g = scv.strided_geom(ks, st_, pd)
+    coarse = scv.downsample(c, g, d_status=st)
+    ref_coarse = oracle.downsample(coords, ks, st_, pd)
+    assert np.array_equal(coarse.cpu().numpy(), ref_coarse)
+    table = scv.hash_table(c, 2.0, st)
+    down = scv.kernel_map(table, len(coords), coarse.contiguous(), g, d_status=st)
+    check_kmap(down, oracle.kmap(coords, ref_coarse, ks, st_, pd, oracle.STRIDED))
+    ctable = scv.hash_table(coarse.contiguous(), 2.0, st)
+    up = scv.kernel_map(ctable, len(ref_coarse), c, scv.transposed_geom(ks, st_, pd), d_status=st)
+    check_kmap(up, oracle.kmap(ref_coarse, coords, ks, st_, pd, oracle.TRANSPOSED))
+    scv.check_status(st)
+
+
+def test_downsample_full_workload():
+    coords = synthetic.WORKLOADS["lidar_down_up"].coords()
+    c = _dev(coords)
+    g = scv.strided_geom(2, 2, 0)
+    coarse = scv.downsample(c, g)
+    ref = oracle.downsample(coords, 2, 2, 0)
+    assert np.array_equal(coarse.cpu().numpy(), ref)
+    table = scv.hash_table(c)
+    check_kmap(scv.kernel_map(table, len(coords), coarse.contiguous(), g),
+               oracle.kmap(coords, ref, 2, 2, 0, oracle.STRIDED))
+    ctable = scv.hash_table(coarse.contiguous())
+    check_kmap(scv.kernel_map(ctable, len(ref), c, scv.transposed_geom(2, 2, 0)),
+               oracle.kmap(ref, coords, 2, 2, 0, oracle.TRANSPOSED))
+
+
+def test_downsample_capacity_error():
+    rng = np.random.default_rng(2)
+    coords = rand_coords(rng, 300, 0, 20)
+    with pytest.raises(scv.LatticeError):
+        scv.downsample(_dev(coords), scv.strided_geom(2, 2, 0), capacity=10)
