@@ -222,6 +222,37 @@ lat_status lat_sconv_wgrad(const void *x, int32_t cin, const void *dy, int32_t c
                            const lat_kmap *map, float *dw, lat_dtype dtype, void *ws,
                            size_t ws_bytes, int32_t *d_status, lat_stream stream);
 
+/* Weight gradient for callers that cannot allocate.  No counterpart in the
+ * papers or docs: this exists for users of the library, not for the method.
+ *
+ * Some callers cannot call cudaMalloc or hand over a scratch buffer: code
+ * that runs while a stream is captured into a CUDA graph without memory
+ * nodes, real-time loops that must not allocate (cudaMalloc / cudaFree can
+ * synchronise the whole device) once running, or hosts whose device
+ * allocator belongs to another runtime.  This entry point computes the same
+ * dW as lat_sconv_wgrad (same kernels, same chunking, same summation order)
+ * but takes no `ws`: its scratch is one static device array of
+ * LAT_WGRAD_STATIC_SCRATCH_BYTES (32 MiB) inside the library, which every
+ * GPU that loads the library keeps until the process exits.  It allocates
+ * nothing and calls no allocating routine.
+ *   - Limit: the scratch must hold (k3 + 1) int32 plus
+ *     (ceil(pair_capacity / 1024) + k3) fp32 partials of cin*cout; larger
+ *     problems return LAT_ERR_WORKSPACE before anything is enqueued (e.g.
+ *     cin = cout = 64 allows about 2.07 million pair slots, 128 x 128
+ *     about 496 thousand).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture begins.
+ *   - All calls share the one array and it keeps the last call's contents;
+ *     every byte a call reads is written earlier by the same call, so no
+ *     clearing is needed.  Calls whose work overlaps on the GPU (different
+ *     streams, or host threads racing on one device) race on the array:
+ *     order them on one stream. */
+#define LAT_WGRAD_STATIC_SCRATCH_BYTES (32u << 20)
+lat_status lat_sconv_wgrad_static(const void *x, int32_t cin, const void *dy, int32_t cout,
+                                  const lat_kmap *map, float *dw, lat_dtype dtype,
+                                  int32_t *d_status, lat_stream stream);
+
 /* ---------------------------------------------------------------- misc --- */
 
 /* Synchronise `stream`, then return the status word at d_status (device). */

@@ -19,7 +19,7 @@ from ._lib import (  # noqa: F401  (re-exported C entry points and constants)
     EXPORTS, LAT_BF16, LAT_F16, LAT_F32, LAT_OK, LAT_OP_DGRAD, LAT_OP_FWD, LAT_OP_WGRAD, LAT_STRIDED, LAT_SUBM,
     LAT_TILE_ROWS, LAT_TRANSPOSED, LIB_PATH, LatticeError, lat_downsample_coords, lat_downsample_ws_bytes, lat_geom,
     lat_hash_build, lat_hash_bytes, lat_kmap, lat_kmap_query, lat_kmap_ws_bytes, lat_sconv_dgrad, lat_sconv_fwd,
-    lat_sconv_wgrad, lat_sconv_ws_bytes, lat_status_fetch, lat_status_string, lat_version, load, make_geom,
+    lat_sconv_wgrad, lat_sconv_wgrad_static, lat_sconv_ws_bytes, lat_status_fetch, lat_status_string, lat_version, load, make_geom,
 )
 
 __all__ = [

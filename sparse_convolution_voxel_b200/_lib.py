@@ -32,7 +32,7 @@ STATUS_BITS = {
 EXPORTS = [
     "lat_hash_bytes", "lat_hash_build", "lat_kmap_ws_bytes", "lat_kmap_query",
     "lat_downsample_ws_bytes", "lat_downsample_coords", "lat_sconv_ws_bytes", "lat_sconv_fwd",
-    "lat_sconv_dgrad", "lat_sconv_wgrad", "lat_status_fetch", "lat_status_string", "lat_version",
+    "lat_sconv_dgrad", "lat_sconv_wgrad", "lat_sconv_wgrad_static", "lat_status_fetch", "lat_status_string", "lat_version",
 ]
 
 
@@ -80,6 +80,7 @@ def load() -> ctypes.CDLL:
         "lat_sconv_fwd": (I32, [P, I32, P, I32, K, P, I32, P, SZ, P, P]),
         "lat_sconv_dgrad": (I32, [P, I32, P, I32, K, I32, P, I32, P, SZ, P, P]),
         "lat_sconv_wgrad": (I32, [P, I32, P, I32, K, P, I32, P, SZ, P, P]),
+        "lat_sconv_wgrad_static": (I32, [P, I32, P, I32, K, P, I32, P, P]),
         "lat_status_fetch": (I32, [P, P]),
         "lat_status_string": (ctypes.c_char_p, [I32]),
         "lat_version": (I32, []),
@@ -194,6 +195,13 @@ def lat_sconv_wgrad(x, dy, kmap: lat_kmap, dw, ws=None, d_status=None, stream=No
     rc = load().lat_sconv_wgrad(_ptr(x), cin, _ptr(dy), cout, ctypes.byref(kmap), _ptr(dw), dtype_code(x.dtype), p, n,
                                 _ptr(d_status), _stream(stream))
     _check(rc, "lat_sconv_wgrad")
+
+
+def lat_sconv_wgrad_static(x, dy, kmap: lat_kmap, dw, d_status=None, stream=None):
+    """Weight gradient with the library's own static scratch (no workspace argument)."""
+    rc = load().lat_sconv_wgrad_static(_ptr(x), x.shape[1], _ptr(dy), dy.shape[1], ctypes.byref(kmap), _ptr(dw),
+                                       dtype_code(x.dtype), _ptr(d_status), _stream(stream))
+    _check(rc, "lat_sconv_wgrad_static")
 
 
 def lat_status_fetch(d_status: torch.Tensor, stream=None) -> int:

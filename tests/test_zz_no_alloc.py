@@ -1,0 +1,68 @@
+"""The weight gradient that uses the library's static scratch instead of a caller buffer.
+
+Callers that cannot allocate device memory (code running under stream
+capture without memory nodes, real-time loops that must not call cudaMalloc
+or cudaFree once running, hosts whose allocator belongs to another runtime)
+use lat_sconv_wgrad_static.  It must give the same dW as lat_sconv_wgrad,
+call after call, since every call reuses the one static array.  This file
+is named so pytest collects it last.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from tests.util import assert_close, feats, rand_coords
+
+pytestmark = pytest.mark.gpu
+
+scv = pytest.importorskip("sparse_convolution_voxel_b200")
+
+
+def _map(coords):
+    c = torch.from_numpy(coords).cuda()
+    st = scv.new_status()
+    km = scv.kernel_map(scv.hash_table(c, 2.0, st), len(coords), c, scv.subm_geom(3), d_status=st)
+    scv.check_status(st)
+    return km
+
+
+@pytest.mark.parametrize("dtype,cin,cout", [(torch.float16, 64, 64), (torch.bfloat16, 128, 128),
+                                            (torch.float32, 16, 32)])
+def test_static_scratch_wgrad_matches_workspace_wgrad_twice(dtype, cin, cout):
+    scv.load()
+    rng = np.random.default_rng(cin + cout)
+    coords = rand_coords(rng, 4000, -12, 12, 2)
+    km = _map(coords)
+    x, _ = feats(len(coords), cin, dtype, seed=41)
+    g, _ = feats(len(coords), cout, dtype, seed=41, stream=1)
+    ref = scv.conv_wgrad(x, g, km).double().cpu().numpy()
+    lib = scv.load()
+    outs = []
+    for _ in range(2):
+        dw = torch.full((27, cin, cout), float("nan"), dtype=torch.float32, device="cuda")
+        st = scv.new_status()
+        rc = lib.lat_sconv_wgrad_static(ctypes.c_void_p(x.data_ptr()), cin, ctypes.c_void_p(g.data_ptr()), cout,
+                                        ctypes.byref(km.c), ctypes.c_void_p(dw.data_ptr()),
+                                        scv._lib.dtype_code(dtype), ctypes.c_void_p(st.data_ptr()),
+                                        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        assert rc == 0, scv.lat_status_string(rc)
+        scv.check_status(st)
+        outs.append(dw.double().cpu().numpy())
+        assert_close(outs[-1], ref, dtype, "static-scratch wgrad")
+    assert_close(outs[1], outs[0], dtype, "second call")
+
+
+def test_static_scratch_wgrad_rejects_problems_above_its_limit():
+    scv.load()
+    rng = np.random.default_rng(3)
+    coords = rand_coords(rng, 200, 0, 8)
+    km = _map(coords)
+    big = scv.lat_kmap.from_buffer_copy(km.c)
+    big.pair_capacity = 3_000_000                     # 64 x 64 partials for 3M pair slots exceed 32 MiB
+    x = torch.zeros((len(coords), 64), dtype=torch.float16, device="cuda")
+    dw = torch.zeros((27, 64, 64), dtype=torch.float32, device="cuda")
+    rc = scv.load().lat_sconv_wgrad_static(ctypes.c_void_p(x.data_ptr()), 64, ctypes.c_void_p(x.data_ptr()), 64,
+                                           ctypes.byref(big), ctypes.c_void_p(dw.data_ptr()), 1, None, None)
+    assert rc == 128                                  # LAT_ERR_WORKSPACE, nothing enqueued
