@@ -71,7 +71,8 @@ typedef enum {
     LAT_ERR_UNSUPPORTED = 32, /* shape / dtype combination not implemented (host)       */
     LAT_ERR_CUDA = 64,        /* a CUDA runtime call failed (host)                      */
     LAT_ERR_WORKSPACE = 128,  /* ws_bytes smaller than the *_ws_bytes query (host)      */
-    LAT_ERR_BAD_MAP = 256     /* a kernel map holds a row index outside [0, n_in) (device) */
+    LAT_ERR_BAD_MAP = 256,    /* a kernel map holds a row index outside [0, n_in) (device) */
+    LAT_ERR_TIMEOUT = 512     /* a bounded in-kernel wait gave up; the kernel drained and exited */
 } lat_status;
 
 typedef enum { LAT_F32 = 0, LAT_F16 = 1, LAT_BF16 = 2 } lat_dtype;
@@ -191,7 +192,9 @@ lat_status lat_downsample_coords(const int32_t *coords, int64_t n_in, const lat_
  * no neighbour get zeros).  Implicit-GEMM dataflow (TorchSparse++ abstract;
  * the migration page requires every dataflow to give the same result for a
  * fixed relation and weight tensor).  cin and cout must be multiples of 8 and
- * at most 256 (fp32) / 128 (fp16, bf16 on tensor cores). */
+ * at most 256.  fp16 / bf16 with cin, cout in {64, 128} run on the tcgen05
+ * tensor cores (fp32 accumulate in TMEM); other shapes and fp32 run on CUDA
+ * cores (FFMA, no TF32). */
 size_t lat_sconv_ws_bytes(int32_t op, int32_t cin, int32_t cout, const lat_kmap *map,
                           lat_dtype dtype);
 #define LAT_OP_FWD 0

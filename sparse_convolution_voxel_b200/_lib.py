@@ -25,7 +25,7 @@ LAT_TILE_ROWS = 128
 STATUS_BITS = {
     1: "LAT_ERR_ARG", 2: "LAT_ERR_COORD_RANGE", 4: "LAT_ERR_DUPLICATE", 8: "LAT_ERR_TABLE_FULL",
     16: "LAT_ERR_CAPACITY", 32: "LAT_ERR_UNSUPPORTED", 64: "LAT_ERR_CUDA", 128: "LAT_ERR_WORKSPACE",
-    256: "LAT_ERR_BAD_MAP",
+    256: "LAT_ERR_BAD_MAP", 512: "LAT_ERR_TIMEOUT",
 }
 
 # every symbol include/lattice.h declares

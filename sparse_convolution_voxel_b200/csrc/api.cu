@@ -33,9 +33,10 @@ static lat_status by_dtype(lat_dtype dt, F &&f) {
 }  // namespace lat
 
 extern "C" size_t lat_sconv_ws_bytes(int32_t op, int32_t cin, int32_t cout, const lat_kmap *map, lat_dtype dtype) {
-    (void)dtype;
     if (!lat::map_ok(map)) return 0;
-    if (op == LAT_OP_WGRAD) return lat::wgrad_simt_ws_bytes(cin, cout, map);
+    if (op == LAT_OP_WGRAD)
+        return (dtype != LAT_F32 && lat::wgrad_tc_supported(cin, cout)) ? lat::wgrad_tc_ws_bytes(cin, cout, map)
+                                                                        : lat::wgrad_simt_ws_bytes(cin, cout, map);
     return 0;
 }
 
@@ -50,6 +51,8 @@ extern "C" lat_status lat_sconv_fwd(const void *x, int32_t cin, const void *w, i
     if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return LAT_ERR_ARG;
     const MapView mv = make_view(map, false);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype != LAT_F32 && conv_tc_supported(cin, cout))
+        return launch_conv_tc(dtype == LAT_BF16, x, cin, w, cout, map->k3, mv, false, y, d_status, s);
     return by_dtype(dtype, [&](auto t) {
         using T = decltype(t);
         return launch_conv_simt<T>(x, cin, w, cout, mv, false, y, d_status, s);
@@ -69,6 +72,8 @@ extern "C" lat_status lat_sconv_dgrad(const void *dy, int32_t cout, const void *
     const MapView mv = make_view(map, flip_offsets != 0);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // the pass gathers dy rows (cout channels) and produces dx rows (cin channels) with W[k]^T
+    if (dtype != LAT_F32 && conv_tc_supported(cout, cin))
+        return launch_conv_tc(dtype == LAT_BF16, dy, cout, w, cin, map->k3, mv, true, dx, d_status, s);
     return by_dtype(dtype, [&](auto t) {
         using T = decltype(t);
         return launch_conv_simt<T>(dy, cout, w, cin, mv, true, dx, d_status, s);
@@ -82,9 +87,11 @@ extern "C" lat_status lat_sconv_wgrad(const void *x, int32_t cin, const void *dy
     if (!map_ok(map) || !chan_ok(cin, dtype) || !chan_ok(cout, dtype) || !dw || !map->pair_off) return LAT_ERR_ARG;
     if (map->pair_capacity > 0 && (!map->pair_in || !map->pair_out)) return LAT_ERR_ARG;
     if (!aligned16(x) || !aligned16(dy) || !aligned16(dw)) return LAT_ERR_ARG;
-    const size_t need = wgrad_simt_ws_bytes(cin, cout, map);
+    const bool tc = dtype != LAT_F32 && wgrad_tc_supported(cin, cout);
+    const size_t need = tc ? wgrad_tc_ws_bytes(cin, cout, map) : wgrad_simt_ws_bytes(cin, cout, map);
     if (ws_bytes < need || !ws) return LAT_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (tc) return launch_wgrad_tc(dtype == LAT_BF16, x, cin, dy, cout, map, dw, ws, d_status, s);
     return by_dtype(dtype, [&](auto t) {
         using T = decltype(t);
         return launch_wgrad_simt<T>(x, cin, dy, cout, map, dw, ws, d_status, s);
@@ -111,6 +118,7 @@ extern "C" const char *lat_status_string(int32_t status) {
     if (status & LAT_ERR_CUDA) return "CUDA runtime error";
     if (status & LAT_ERR_WORKSPACE) return "workspace too small";
     if (status & LAT_ERR_BAD_MAP) return "kernel map row index out of range";
+    if (status & LAT_ERR_TIMEOUT) return "bounded in-kernel wait timed out";
     return "unknown status";
 }
 

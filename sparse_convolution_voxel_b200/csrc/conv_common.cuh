@@ -52,4 +52,12 @@ lat_status launch_wgrad_simt(const void *x, int cin, const void *dy, int cout, c
                              void *ws, int32_t *d_status, cudaStream_t s);
 size_t wgrad_simt_ws_bytes(int cin, int cout, const lat_kmap *map);
 
+bool conv_tc_supported(int kc, int n);
+bool wgrad_tc_supported(int cin, int cout);
+size_t wgrad_tc_ws_bytes(int cin, int cout, const lat_kmap *map);
+lat_status launch_wgrad_tc(bool bf16, const void *x, int cin, const void *dy, int cout, const lat_kmap *map, float *dw,
+                           void *ws, int32_t *d_status, cudaStream_t s);
+lat_status launch_conv_tc(bool bf16, const void *x, int kc, const void *w, int n, int k3, const MapView &mv, bool wt,
+                          void *y, int32_t *d_status, cudaStream_t s);
+
 }  // namespace lat

@@ -1,0 +1,352 @@
+// tcgen05 implicit-GEMM sparse convolution: fp16 / bf16 in, fp32 accumulate in TMEM.
+//
+// Output-stationary implicit GEMM (TorchSparse++ abstract: implicit GEMM
+// overlaps computation and memory access; the migration page's "Backend and
+// configuration differences" requires every dataflow to give the same result
+// for a fixed relation and weight tensor).  One persistent CTA per SM walks
+// 128-row tiles of the mask-sorted output order; for every offset in a
+// tile's mask union and every 64-channel K block it
+//   - gathers the 128 neighbour rows with 16-byte cp.async into a 128-byte
+//     swizzled K-major tile (absent neighbours are zero-filled, no read),
+//   - loads the W[k] slab with TMA (128-byte swizzle, no multicast),
+//   - issues 4 tcgen05.mma (M=128, N=Cout, K=16) into a TMEM accumulator.
+// Epilogue warps read the accumulator with tcgen05.ld, round once to the
+// output type and write each output row exactly once -- no atomics.  The
+// accumulator is double buffered in TMEM so the epilogue of tile t overlaps
+// the main loop of tile t+1.
+//
+// Roles (288 threads): warps 0-3 gather (thread 0 also issues TMA), warps 4-7
+// epilogue (warp w reads TMEM lanes 32*(w%4)..+31), warp 8 lane 0 issues MMAs.
+// Every mbarrier wait is bounded; a wait that gives up flags LAT_ERR_TIMEOUT
+// and the CTA drains and exits, releasing its TMEM.
+//
+// The same kernel computes the data gradient: the gathered operand is dy, the
+// B operand is W[k]^T (K-major view of the same weight slab), and a
+// submanifold map is walked with flipped offsets.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "conv_common.cuh"
+#include "tc_ptx.cuh"
+
+namespace lat {
+namespace tc {
+
+constexpr int kM = 128;          // tile rows = MMA M
+constexpr int kProdWarps = 4;    // gather warps
+constexpr int kEpiWarps = 4;     // epilogue warps
+constexpr int kMmaWarp = kProdWarps + kEpiWarps;
+constexpr int kThreads = (kMmaWarp + 1) * 32;
+constexpr int kLag = 3;          // cp.async groups a gather thread keeps in flight
+constexpr uint32_t kABytes = kM * 128;  // 128 rows x 64 channels x 2 bytes
+constexpr uint64_t kWaitNs = 2000000000ull;
+
+template <int N>
+struct Cfg {
+    static constexpr uint32_t kBBytes = uint32_t(N) * 128;  // 64 K x N (or N x 64) x 2 bytes
+    static constexpr uint32_t kStage = kABytes + kBBytes;
+    static constexpr int kStages = N == 64 ? 8 : 6;
+    static constexpr uint32_t kBarBytes = 256;
+    static constexpr uint32_t kSmem = kStages * kStage + kBarBytes + 1024;
+    static constexpr uint32_t kTmemCols = 2 * N;
+};
+
+template <typename T> constexpr bool is_bf16() { return sizeof(T) == 2 && !std::is_same<T, __half>::value; }
+
+// Instruction descriptor, kind::f16: fp32 D, A/B fp16 or bf16, A K-major,
+// B MN-major (forward: W[k] is (Cin x Cout), Cout contiguous) or K-major
+// (data gradient: W[k]^T viewed as (N=Cin) x (K=Cout) rows), M=128, N.
+template <typename T, int N, bool BMN>
+__host__ __device__ constexpr uint32_t make_idesc() {
+    return (1u << 4) | ((is_bf16<T>() ? 1u : 0u) << 7) | ((is_bf16<T>() ? 1u : 0u) << 10) |
+           ((BMN ? 1u : 0u) << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(kM >> 4) << 24);
+}
+
+__device__ __forceinline__ uint32_t pack2(float a, float b, __half) {
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+__device__ __forceinline__ uint32_t pack2(float a, float b, __nv_bfloat16) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// KC: gathered channels (GEMM K), N: output channels, BMN: B operand MN-major.
+template <typename T, int KC, int N, bool BMN>
+__global__ void __launch_bounds__(kThreads, 1)
+conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x, MapView mv, T *__restrict__ y,
+               int32_t *d_status) {
+    using C = Cfg<N>;
+    constexpr int NS = C::kStages;
+    constexpr int KBLK = KC / 64;
+    constexpr uint32_t idesc = make_idesc<T, N, BMN>();
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + NS * C::kStage);
+    uint64_t *empty = full + NS;
+    uint64_t *accfull = empty + NS;
+    uint64_t *accempty = accfull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accempty + 2);
+    __shared__ int s_abort;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int s = 0; s < NS; ++s) {
+            ptx::mbar_init(&full[s], kProdWarps * 32 + 1);
+            ptx::mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            ptx::mbar_init(&accfull[a], 1);
+            ptx::mbar_init(&accempty[a], kEpiWarps * 32);
+        }
+        s_abort = 0;
+        ptx::fence_mbar_init();
+        ptx::fence_proxy_async_smem();
+        ptx::tma_prefetch(&wmap);
+    }
+    if (warp == 0) {
+        ptx::tmem_alloc(tmem_slot, C::kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    int32_t bad = 0;
+
+    if (warp < kProdWarps) {
+        // ------------------------------------------------------------ gather + TMA
+        uint32_t it = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < mv.ntiles && ok; t += gridDim.x) {
+            const uint32_t tm = mv.tile_mask_at(t);
+            const int64_t my_row = t * kM + tid;
+            const int j_own = my_row < mv.n_out ? __ldg(mv.perm + my_row) : -1;
+            for (uint32_t m = tm; m && ok; m &= m - 1) {
+                const int k = __ffs(m) - 1;
+                int src_own = j_own >= 0 ? mv.neighbour(k, j_own) : -1;
+                if (src_own >= mv.n_in) {
+                    bad |= LAT_ERR_BAD_MAP;
+                    src_own = -1;
+                }
+                for (int kb = 0; kb < KBLK; ++kb) {
+                    const uint32_t s = it % NS;
+                    if (!ptx::mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, kWaitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *As = smem + s * C::kStage;
+                    uint8_t *Bs = As + kABytes;
+                    if (tid == 0) {
+                        ptx::mbar_arrive_expect_tx(&full[s], C::kBBytes);
+#pragma unroll
+                        for (int nb = 0; nb < N / 64; ++nb) {
+                            if constexpr (BMN)  // rows k*KC + 64kb.., columns 64nb..
+                                ptx::tma_load_2d(Bs + nb * 8192, &wmap, &full[s], 64 * nb, k * KC + 64 * kb);
+                            else                // rows k*N + 64nb.., columns 64kb..
+                                ptx::tma_load_2d(Bs + nb * 8192, &wmap, &full[s], 64 * kb, k * N + 64 * nb);
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int rl = 4 * i + (lane >> 3);
+                        const int row = warp * 32 + rl;
+                        const int chunk = lane & 7;
+                        const int src = __shfl_sync(0xFFFFFFFFu, src_own, rl);
+                        const T *gp = src >= 0 ? x + int64_t(src) * KC + kb * 64 + chunk * 8 : x;
+                        ptx::cp_async16(As + row * 128 + ((chunk ^ (row & 7)) << 4), gp, src >= 0 ? 16u : 0u);
+                    }
+                    ptx::cp_async_commit();
+                    if (it >= kLag) {
+                        ptx::cp_async_wait<kLag>();
+                        ptx::fence_proxy_async_smem();
+                        ptx::mbar_arrive(&full[(it - kLag) % NS]);
+                    }
+                    ++it;
+                }
+            }
+        }
+        ptx::cp_async_wait<0>();
+        ptx::fence_proxy_async_smem();
+        for (uint32_t d = (it > kLag ? it - kLag : 0); d < it; ++d) ptx::mbar_arrive(&full[d % NS]);
+        if (!ok) s_abort = 1;
+    } else if (warp < kMmaWarp) {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;
+        uint32_t ta = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < mv.ntiles && ok; t += gridDim.x) {
+            const uint32_t tm = mv.tile_mask_at(t);
+            const int64_t grow = t * kM + q * 32 + lane;
+            const int j = grow < mv.n_out ? __ldg(mv.perm + grow) : -1;
+            T *yr = j >= 0 ? y + int64_t(j) * N : nullptr;
+            if (!tm) {  // no neighbour anywhere in the tile: zeros
+                if (yr)
+#pragma unroll
+                    for (int c = 0; c < N; c += 8) *reinterpret_cast<uint4 *>(yr + c) = make_uint4(0, 0, 0, 0);
+                continue;
+            }
+            const uint32_t a = ta & 1;
+            if (!ptx::mbar_wait(&accfull[a], (ta >> 1) & 1, kWaitNs)) {
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + a * N;
+#pragma unroll
+            for (int c0 = 0; c0 < N; c0 += 32) {
+                uint32_t v0[16], v1[16];
+                ptx::tmem_ld16(taddr + c0, v0);
+                ptx::tmem_ld16(taddr + c0 + 16, v1);
+                ptx::tmem_wait_ld();
+                if (yr) {
+                    uint4 o[4];
+                    uint32_t *op = reinterpret_cast<uint32_t *>(o);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        op[e] = pack2(__uint_as_float(v0[2 * e]), __uint_as_float(v0[2 * e + 1]), T{});
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        op[8 + e] = pack2(__uint_as_float(v1[2 * e]), __uint_as_float(v1[2 * e + 1]), T{});
+                    uint4 *dst = reinterpret_cast<uint4 *>(yr + c0);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dst[e] = o[e];
+                }
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&accempty[a]);
+            ++ta;
+        }
+        if (!ok) s_abort = 1;
+    } else if (lane == 0) {
+        // ------------------------------------------------------------ MMA issue
+        uint32_t it = 0, ta = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < mv.ntiles && ok; t += gridDim.x) {
+            const uint32_t tm = mv.tile_mask_at(t);
+            if (!tm) continue;
+            const uint32_t a = ta & 1;
+            if (!ptx::mbar_wait(&accempty[a], ((ta >> 1) & 1) ^ 1, kWaitNs)) {
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            const uint32_t dcol = tmem_base + a * N;
+            uint32_t acc = 0;
+            for (uint32_t m = tm; m && ok; m &= m - 1) {
+                for (int kb = 0; kb < KBLK; ++kb) {
+                    const uint32_t s = it % NS;
+                    if (!ptx::mbar_wait(&full[s], (it / NS) & 1, kWaitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t as = ptx::smem_u32(smem + s * C::kStage);
+                    const uint32_t bs = as + kABytes;
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t ad = ptx::desc_sw128(as + ks * 32, 16, 1024);
+                        const uint64_t bd = BMN ? ptx::desc_sw128(bs + ks * 2048, 8192, 1024)
+                                                : ptx::desc_sw128(bs + ks * 32, 16, 1024);
+                        ptx::umma_f16(dcol, ad, bd, idesc, acc);
+                        acc = 1;
+                    }
+                    ptx::umma_commit(&empty[s]);
+                    ++it;
+                }
+            }
+            if (!ok) break;
+            ptx::umma_commit(&accfull[a]);
+            ++ta;
+        }
+        if (!ok) s_abort = 1;
+    }
+
+    __syncthreads();
+    if (s_abort) {
+        bad |= (tid == 0) ? LAT_ERR_TIMEOUT : 0;
+        __nanosleep(1000000);  // let in-flight async copies / MMAs land before TMEM is released
+    }
+    if (bad) flag(d_status, bad);
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
+// ----------------------------------------------------------------------------- host side
+using EncodeFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+static EncodeFn encode_fn() {
+    static EncodeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeFn>(p);
+    });
+    return fn;
+}
+
+// Weights (k3, wrows, wcols) row-major viewed as a 2D (k3*wrows) x wcols tensor, 64 x 64 boxes, 128-byte swizzle.
+static bool make_weight_map(CUtensorMap *map, const void *w, bool bf16, int k3, int wrows, int wcols) {
+    EncodeFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cuuint64_t(wcols), cuuint64_t(k3) * wrows};
+    const cuuint64_t strides[1] = {cuuint64_t(wcols) * 2};
+    const cuuint32_t box[2] = {64, 64};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+               const_cast<void *>(w), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T, int KC, int N, bool BMN>
+static lat_status launch(const void *x, const void *w, int k3, const MapView &mv, void *y, int32_t *d_status,
+                         cudaStream_t s) {
+    using C = Cfg<N>;
+    CUtensorMap map;
+    // forward: W[k] is (KC x N); data gradient: W[k] is (N x KC)
+    if (!make_weight_map(&map, w, is_bf16<T>(), k3, BMN ? KC : N, BMN ? N : KC)) return LAT_ERR_CUDA;
+    auto kern = conv_tc_kernel<T, KC, N, BMN>;
+    LAT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::kSmem)));
+    const int64_t grid = std::min<int64_t>(mv.ntiles, num_sms());
+    kern<<<unsigned(grid), kThreads, C::kSmem, s>>>(map, static_cast<const T *>(x), mv, static_cast<T *>(y),
+                                                    d_status);
+    LAT_CUDA_TRY(cudaGetLastError());
+    return LAT_OK;
+}
+
+template <typename T, bool BMN>
+static lat_status dispatch(int kc, int n, const void *x, const void *w, int k3, const MapView &mv, void *y,
+                           int32_t *d_status, cudaStream_t s) {
+    if (kc == 64 && n == 64) return launch<T, 64, 64, BMN>(x, w, k3, mv, y, d_status, s);
+    if (kc == 64 && n == 128) return launch<T, 64, 128, BMN>(x, w, k3, mv, y, d_status, s);
+    if (kc == 128 && n == 64) return launch<T, 128, 64, BMN>(x, w, k3, mv, y, d_status, s);
+    if (kc == 128 && n == 128) return launch<T, 128, 128, BMN>(x, w, k3, mv, y, d_status, s);
+    return LAT_ERR_UNSUPPORTED;
+}
+
+}  // namespace tc
+
+bool conv_tc_supported(int kc, int n) { return (kc == 64 || kc == 128) && (n == 64 || n == 128); }
+
+// Forward (wt = false): gathered x (cin) x W[k] (cin x cout).  Data gradient (wt = true):
+// gathered dy (kc = cout) x W[k]^T, producing n = cin channels.
+lat_status launch_conv_tc(bool bf16, const void *x, int kc, const void *w, int n, int k3, const MapView &mv, bool wt,
+                          void *y, int32_t *d_status, cudaStream_t s) {
+    if (mv.ntiles == 0) return LAT_OK;
+    if (bf16)
+        return wt ? tc::dispatch<__nv_bfloat16, false>(kc, n, x, w, k3, mv, y, d_status, s)
+                  : tc::dispatch<__nv_bfloat16, true>(kc, n, x, w, k3, mv, y, d_status, s);
+    return wt ? tc::dispatch<__half, false>(kc, n, x, w, k3, mv, y, d_status, s)
+              : tc::dispatch<__half, true>(kc, n, x, w, k3, mv, y, d_status, s);
+}
+
+}  // namespace lat

@@ -164,3 +164,23 @@ def test_training_step_full_workload():
     assert_close(y.double().cpu().numpy(), oracle.conv_fwd(x64, w64, ref_nbr), dtype, "fwd")
     assert_close(dx.double().cpu().numpy(), oracle.conv_dgrad(g64, w64, ref_nbr, len(coords)), dtype, "dgrad")
     assert_close(dw.double().cpu().numpy(), oracle.conv_wgrad(x64, g64, ref_nbr), dtype, "wgrad")
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
+def test_transposed_fwd_with_rows_without_neighbours(dtype):
+    """K < stride on one axis: two thirds of the fine rows have no coarse neighbour, so
+    whole 128-row tiles have an empty offset set and must be written as zeros."""
+    rng = np.random.default_rng(23)
+    coords = rand_coords(rng, 2500, -9, 9, 2)
+    ks, st_, pd = (3, 2, 1), (2, 1, 3), (0, 1, 0)
+    c = _dev(coords)
+    g = scv.strided_geom(ks, st_, pd)
+    coarse = scv.downsample(c, g).contiguous()
+    rc = coarse.cpu().numpy()
+    up = scv.kernel_map(scv.hash_table(coarse), len(rc), c, scv.transposed_geom(ks, st_, pd))
+    ref_up = oracle.kmap(rc, coords, ks, st_, pd, oracle.TRANSPOSED)
+    assert (ref_up < 0).all(1).sum() >= 256
+    x, x64 = feats(len(rc), 64, dtype, seed=29)
+    w, w64 = weights(6, 64, 64, dtype, seed=29)
+    z = scv.conv_fwd(x, w, up, out=torch.full((len(coords), 64), 3.0, dtype=dtype, device="cuda"))
+    assert_close(z.double().cpu().numpy(), oracle.conv_fwd(x64, w64, ref_up), dtype, "transposed fwd")
