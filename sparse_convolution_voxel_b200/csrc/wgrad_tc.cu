@@ -1,0 +1,342 @@
+// tcgen05 per-offset weight gradient: dW[k] = sum over pairs (i, j) of offset k of
+// x[i]^T dy[j]  (fp16 / bf16 in, fp32 accumulate in TMEM, fp32 out).
+//
+// Per offset this is a GEMM with M = Cin, N = Cout and the pairs as the
+// reduction dimension.  The pairs of each offset (grouped and ordered by the
+// kernel-map query) are cut into fixed chunks of kChunk pairs; one persistent
+// CTA per SM takes chunks round-robin.  For every 64-pair block of a chunk,
+// four gather warps copy the 64 x rows and 64 dy rows with 16-byte cp.async
+// into 128-byte swizzled MN-major tiles (rows of the gathered operands are
+// the reduction dimension, channels are contiguous), and one thread issues 4
+// tcgen05.mma (K = 16 pairs each) into a TMEM accumulator.  Four epilogue
+// warps write the chunk's fp32 partial; a second kernel sums the partials of
+// each offset in chunk order.  No atomics, so dW is deterministic.
+#include "common.cuh"
+#include "conv_common.cuh"
+#include "tc_ptx.cuh"
+
+namespace lat {
+namespace wtc {
+
+constexpr int kKP = 64;            // pairs per stage (GEMM K block)
+constexpr int kChunk = 2048;       // pairs per work unit
+constexpr int kProdWarps = 4, kEpiWarps = 4;
+constexpr int kMmaWarp = kProdWarps + kEpiWarps;
+constexpr int kThreads = (kMmaWarp + 1) * 32;
+constexpr int kLag = 3;
+constexpr int kStages = 6;
+constexpr uint64_t kWaitNs = 2000000000ull;
+
+template <int M, int N>
+struct Cfg {
+    static constexpr uint32_t kABytes = uint32_t(M) * 128;  // 64 pairs x M channels x 2 bytes
+    static constexpr uint32_t kBBytes = uint32_t(N) * 128;
+    static constexpr uint32_t kStage = kABytes + kBBytes;
+    static constexpr uint32_t kSmem = kStages * kStage + 256 + 1024;
+    static constexpr uint32_t kTmemCols = 2 * N;
+};
+
+template <typename T> constexpr bool is_bf16() { return !std::is_same<T, __half>::value; }
+
+// kind::f16, fp32 D, A and B MN-major, M x N
+template <typename T, int M, int N>
+__host__ __device__ constexpr uint32_t make_idesc() {
+    return (1u << 4) | ((is_bf16<T>() ? 1u : 0u) << 7) | ((is_bf16<T>() ? 1u : 0u) << 10) | (1u << 15) |
+           (1u << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
+// Unit u covers pairs [lo, hi) of offset k; returns false past the last unit.
+__device__ __forceinline__ void unit_range(const int32_t *unit_base, const int64_t *pair_off, int64_t capacity,
+                                           int k3, int32_t u, int &k, int64_t &lo, int64_t &hi) {
+    k = 0;
+    while (k + 1 < k3 && unit_base[k + 1] <= u) ++k;
+    const int64_t base = min(pair_off[k], capacity);
+    lo = base + int64_t(u - unit_base[k]) * kChunk;
+    hi = min(lo + kChunk, min(pair_off[k + 1], capacity));
+}
+
+template <typename T, int M, int N>
+__global__ void __launch_bounds__(kThreads, 1)
+wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t *__restrict__ pair_off,
+                const int32_t *__restrict__ pair_in, const int32_t *__restrict__ pair_out, int64_t capacity, int k3,
+                int64_t n_in, int64_t n_out, const int32_t *__restrict__ unit_base, float *__restrict__ partial,
+                int32_t *d_status) {
+    using C = Cfg<M, N>;
+    constexpr int NS = kStages;
+    constexpr uint32_t idesc = make_idesc<T, M, N>();
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + NS * C::kStage);
+    uint64_t *empty = full + NS;
+    uint64_t *accfull = empty + NS;
+    uint64_t *accempty = accfull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accempty + 2);
+    __shared__ int s_abort;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int32_t units = unit_base[k3];
+    if (tid == 0) {
+        for (int s = 0; s < NS; ++s) {
+            ptx::mbar_init(&full[s], kProdWarps * 32);
+            ptx::mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            ptx::mbar_init(&accfull[a], 1);
+            ptx::mbar_init(&accempty[a], kEpiWarps * 32);
+        }
+        s_abort = 0;
+        ptx::fence_mbar_init();
+        ptx::fence_proxy_async_smem();
+    }
+    if (warp == 0) {
+        ptx::tmem_alloc(tmem_slot, C::kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    int32_t bad = 0;
+
+    if (warp < kProdWarps) {
+        // ------------------------------------------------------------ gather x and dy rows
+        uint32_t it = 0;
+        bool ok = true;
+        const int g = lane >> 3, c = lane & 7;
+        for (int32_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            int k;
+            int64_t lo, hi;
+            unit_range(unit_base, pair_off, capacity, k3, u, k, lo, hi);
+            for (int64_t p0 = lo; p0 < hi; p0 += kKP) {
+                // lanes 0..15 fetch the indices of this warp's 16 pairs
+                const int64_t mp = p0 + warp * 16 + (lane & 15);
+                int si = -1, sj = -1;
+                if (lane < 16 && mp < hi) {
+                    si = __ldg(pair_in + mp);
+                    sj = __ldg(pair_out + mp);
+                    if (si < 0 || si >= n_in || sj < 0 || sj >= n_out) {
+                        bad |= LAT_ERR_BAD_MAP;
+                        si = sj = -1;
+                    }
+                }
+                const uint32_t s = it % NS;
+                if (!ptx::mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, kWaitNs)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *As = smem + s * C::kStage;
+                uint8_t *Bs = As + C::kABytes;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int pl = 4 * i + g;           // pair within this warp's 16
+                    const int p = warp * 16 + pl;       // pair within the 64-pair block (K index)
+                    const int ii = __shfl_sync(0xFFFFFFFFu, si, pl);
+                    const int jj = __shfl_sync(0xFFFFFFFFu, sj, pl);
+                    const uint32_t off = (p >> 3) * 1024 + (p & 7) * 128 + ((c ^ (p & 7)) << 4);
+#pragma unroll
+                    for (int mb = 0; mb < M / 64; ++mb) {
+                        const T *src = ii >= 0 ? x + int64_t(ii) * M + mb * 64 + c * 8 : x;
+                        ptx::cp_async16(As + mb * 8192 + off, src, ii >= 0 ? 16u : 0u);
+                    }
+#pragma unroll
+                    for (int nb = 0; nb < N / 64; ++nb) {
+                        const T *src = jj >= 0 ? dy + int64_t(jj) * N + nb * 64 + c * 8 : dy;
+                        ptx::cp_async16(Bs + nb * 8192 + off, src, jj >= 0 ? 16u : 0u);
+                    }
+                }
+                ptx::cp_async_commit();
+                if (it >= kLag) {
+                    ptx::cp_async_wait<kLag>();
+                    ptx::fence_proxy_async_smem();
+                    ptx::mbar_arrive(&full[(it - kLag) % NS]);
+                }
+                ++it;
+            }
+        }
+        ptx::cp_async_wait<0>();
+        ptx::fence_proxy_async_smem();
+        for (uint32_t d = (it > kLag ? it - kLag : 0); d < it; ++d) ptx::mbar_arrive(&full[d % NS]);
+        if (!ok) s_abort = 1;
+    } else if (warp < kMmaWarp) {
+        // ------------------------------------------------------------ epilogue: partial of each unit
+        const int q = warp & 3;
+        // M = 128: lane l of warp q holds row 32q + l; M = 64: lanes 0..15 hold rows 16q + l
+        const int row = M == 128 ? q * 32 + lane : q * 16 + lane;
+        const bool has_row = M == 128 || lane < 16;
+        uint32_t ta = 0;
+        bool ok = true;
+        for (int32_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            int k;
+            int64_t lo, hi;
+            unit_range(unit_base, pair_off, capacity, k3, u, k, lo, hi);
+            float *dst = partial + int64_t(u) * M * N + int64_t(row) * N;
+            if (hi <= lo) {  // cannot happen for a listed unit; keep the partial defined anyway
+                if (has_row)
+                    for (int c0 = 0; c0 < N; c0 += 4) *reinterpret_cast<float4 *>(dst + c0) = make_float4(0, 0, 0, 0);
+                continue;
+            }
+            const uint32_t a = ta & 1;
+            if (!ptx::mbar_wait(&accfull[a], (ta >> 1) & 1, kWaitNs)) {
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + a * N;
+#pragma unroll
+            for (int c0 = 0; c0 < N; c0 += 32) {
+                uint32_t v0[16], v1[16];
+                ptx::tmem_ld16(taddr + c0, v0);
+                ptx::tmem_ld16(taddr + c0 + 16, v1);
+                ptx::tmem_wait_ld();
+                if (has_row) {
+                    float4 *d4 = reinterpret_cast<float4 *>(dst + c0);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        d4[e] = make_float4(__uint_as_float(v0[4 * e]), __uint_as_float(v0[4 * e + 1]),
+                                            __uint_as_float(v0[4 * e + 2]), __uint_as_float(v0[4 * e + 3]));
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        d4[4 + e] = make_float4(__uint_as_float(v1[4 * e]), __uint_as_float(v1[4 * e + 1]),
+                                                __uint_as_float(v1[4 * e + 2]), __uint_as_float(v1[4 * e + 3]));
+                }
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&accempty[a]);
+            ++ta;
+        }
+        if (!ok) s_abort = 1;
+    } else if (lane == 0) {
+        // ------------------------------------------------------------ MMA issue
+        uint32_t it = 0, ta = 0;
+        bool ok = true;
+        for (int32_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            int k;
+            int64_t lo, hi;
+            unit_range(unit_base, pair_off, capacity, k3, u, k, lo, hi);
+            if (hi <= lo) continue;
+            const uint32_t a = ta & 1;
+            if (!ptx::mbar_wait(&accempty[a], ((ta >> 1) & 1) ^ 1, kWaitNs)) {
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            const uint32_t dcol = tmem_base + a * N;
+            uint32_t acc = 0;
+            for (int64_t p0 = lo; p0 < hi; p0 += kKP) {
+                const uint32_t s = it % NS;
+                if (!ptx::mbar_wait(&full[s], (it / NS) & 1, kWaitNs)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t as = ptx::smem_u32(smem + s * C::kStage);
+                const uint32_t bs = as + C::kABytes;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t ad = ptx::desc_sw128(as + ks * 2048, 8192, 1024);
+                    const uint64_t bd = ptx::desc_sw128(bs + ks * 2048, 8192, 1024);
+                    ptx::umma_f16(dcol, ad, bd, idesc, acc);
+                    acc = 1;
+                }
+                ptx::umma_commit(&empty[s]);
+                ++it;
+            }
+            if (!ok) break;
+            ptx::umma_commit(&accfull[a]);
+            ++ta;
+        }
+        if (!ok) s_abort = 1;
+    }
+
+    __syncthreads();
+    if (s_abort) {
+        bad |= (tid == 0) ? LAT_ERR_TIMEOUT : 0;
+        __nanosleep(1000000);
+    }
+    if (bad) flag(d_status, bad);
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
+__global__ void wgrad_tc_units_kernel(const int64_t *__restrict__ pair_off, int k3, int64_t capacity,
+                                      int32_t *__restrict__ unit_base) {
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    int32_t u = 0;
+    for (int k = 0; k < k3; ++k) {
+        unit_base[k] = u;
+        const int64_t lo = min(pair_off[k], capacity), hi = min(pair_off[k + 1], capacity);
+        u += int32_t((hi - lo + kChunk - 1) / kChunk);
+    }
+    unit_base[k3] = u;
+}
+
+__global__ void wgrad_tc_reduce_kernel(const float *__restrict__ partial, const int32_t *__restrict__ unit_base,
+                                       int k3, int nelem, float *__restrict__ dw) {
+    const int k = blockIdx.y;
+    const int el = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
+    if (k >= k3 || el >= nelem) return;
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int32_t u = unit_base[k]; u < unit_base[k + 1]; ++u) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(partial + int64_t(u) * nelem + el));
+        s.x += v.x;
+        s.y += v.y;
+        s.z += v.z;
+        s.w += v.w;
+    }
+    *reinterpret_cast<float4 *>(dw + int64_t(k) * nelem + el) = s;
+}
+
+template <typename T, int M, int N>
+static lat_status launch(const void *x, const void *dy, const lat_kmap *map, float *dw, void *ws, int32_t *d_status,
+                         cudaStream_t s) {
+    using C = Cfg<M, N>;
+    const int64_t units_max = (map->pair_capacity + kChunk - 1) / kChunk + map->k3;
+    Carver cv(ws);
+    int32_t *unit_base = cv.take<int32_t>(size_t(map->k3) + 1);
+    float *partial = cv.take<float>(size_t(units_max) * M * N);
+    wgrad_tc_units_kernel<<<1, 32, 0, s>>>(map->pair_off, map->k3, map->pair_capacity, unit_base);
+    LAT_CUDA_TRY(cudaGetLastError());
+    auto kern = wgrad_tc_kernel<T, M, N>;
+    LAT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::kSmem)));
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(units_max, num_sms()));
+    kern<<<unsigned(grid), kThreads, C::kSmem, s>>>(static_cast<const T *>(x), static_cast<const T *>(dy),
+                                                    map->pair_off, map->pair_in, map->pair_out, map->pair_capacity,
+                                                    map->k3, map->n_in, map->n_out, unit_base, partial, d_status);
+    LAT_CUDA_TRY(cudaGetLastError());
+    const int nelem = M * N;
+    dim3 rg((nelem / 4 + 255) / 256, map->k3);
+    wgrad_tc_reduce_kernel<<<rg, 256, 0, s>>>(partial, unit_base, map->k3, nelem, dw);
+    LAT_CUDA_TRY(cudaGetLastError());
+    return LAT_OK;
+}
+
+}  // namespace wtc
+
+bool wgrad_tc_supported(int cin, int cout) { return (cin == 64 || cin == 128) && (cout == 64 || cout == 128); }
+
+size_t wgrad_tc_ws_bytes(int cin, int cout, const lat_kmap *map) {
+    const int64_t units_max = (map->pair_capacity + wtc::kChunk - 1) / wtc::kChunk + map->k3;
+    Carver cv(nullptr);
+    cv.take<int32_t>(size_t(map->k3) + 1);
+    cv.take<float>(size_t(units_max) * cin * cout);
+    return align_up(cv.used, 256);
+}
+
+lat_status launch_wgrad_tc(bool bf16, const void *x, int cin, const void *dy, int cout, const lat_kmap *map, float *dw,
+                           void *ws, int32_t *d_status, cudaStream_t s) {
+#define LAT_WTC(T, M, N) \
+    if (cin == M && cout == N) return wtc::launch<T, M, N>(x, dy, map, dw, ws, d_status, s);
+    if (bf16) {
+        LAT_WTC(__nv_bfloat16, 64, 64) LAT_WTC(__nv_bfloat16, 64, 128) LAT_WTC(__nv_bfloat16, 128, 64)
+        LAT_WTC(__nv_bfloat16, 128, 128)
+    } else {
+        LAT_WTC(__half, 64, 64) LAT_WTC(__half, 64, 128) LAT_WTC(__half, 128, 64) LAT_WTC(__half, 128, 128)
+    }
+#undef LAT_WTC
+    return LAT_ERR_UNSUPPORTED;
+}
+
+}  // namespace lat
