@@ -6,7 +6,8 @@ SubmConv3d workload (batch 2 x 100k voxels in a 1440x1440x41 grid, fp16,
 
   hash build -> submanifold kernel map (probe, pairs, mask sort, tile masks)
   -> SubmConv3d fwd 64->64 -> dgrad -> per-offset wgrad
-  -> strided support (k=2 s=2) -> strided + transposed kernel maps
+  -> strided support (k=2 s=2, with each voxel's coarse row)
+  -> strided + transposed kernel maps from those parent rows
   -> strided Conv3d fwd 64->128 -> ConvTranspose3d fwd 128->64.
 
 value = effective TFLOP/s of the step (sum over the five convolution passes
@@ -24,7 +25,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -93,15 +93,16 @@ class Pipeline:
         self.z = torch.empty((n, CIN), dtype=torch.half, device=dev)
         self.g_sub, self.g_down, self.g_up = scv.subm_geom(3), scv.strided_geom(2, 2, 0), scv.transposed_geom(2, 2, 0)
         # the coarse support size is fixed for a fixed input: size the coarse buffers once
+        self.parent = torch.empty(n, dtype=torch.int32, device=dev)
         self.nc = scv.lat_downsample_coords(self.d["coords"], self.g_down, self.coarse_buf,
-                                            self.ws.get(scv.lat_downsample_ws_bytes(n, self.g_down)), self.status)
+                                            self.ws.get(scv.lat_downsample_ws_bytes(n, self.g_down)), self.status,
+                                            parent=self.parent)
         nc = self.nc
-        self.ctable = torch.empty(scv.lat_hash_bytes(nc, 2.0) // 8, dtype=torch.int64, device=dev)
         self.km_down = scv.KernelMap(n, nc, 8, dev)
         self.km_up = scv.KernelMap(nc, n, 8, dev)
         self.yc = torch.empty((nc, CMID), dtype=torch.half, device=dev)
         self.ws_bytes = max(scv.lat_kmap_ws_bytes(n, 27), scv.lat_kmap_ws_bytes(n, 8),
-                            scv.lat_downsample_ws_bytes(n, self.g_down),
+                            scv.lat_downsample_ws_bytes(n, self.g_down), scv.lat_kmap_from_parent_ws_bytes(n, nc, 8),
                             scv.lat_sconv_ws_bytes(2, CIN, CIN, self.km.c, torch.half),
                             scv.lat_sconv_ws_bytes(0, CIN, CIN, self.km.c, torch.half),
                             scv.lat_sconv_ws_bytes(1, CIN, CIN, self.km.c, torch.half),
@@ -125,13 +126,10 @@ class Pipeline:
         rec(4)
         scv.lat_sconv_wgrad(d["x"], d["g"], self.km.c, self.dw, self.wsb, s)
         rec(5)
-        nc = scv.lat_downsample_coords(d["coords"], self.g_down, self.coarse_buf, self.wsb, s)
+        nc = scv.lat_downsample_coords(d["coords"], self.g_down, self.coarse_buf, self.wsb, s, parent=self.parent)
         assert nc == self.nc
-        coarse = self.coarse_buf[:nc]
         rec(6)
-        scv.lat_kmap_query(self.table, coarse, self.g_down, self.km_down.c, self.wsb, s)
-        scv.lat_hash_build(coarse, self.ctable, s)
-        scv.lat_kmap_query(self.ctable, d["coords"], self.g_up, self.km_up.c, self.wsb, s)
+        scv.lat_kmap_from_parent(d["coords"], self.parent, self.g_down, self.km_down.c, self.km_up.c, self.wsb, s)
         rec(7)
         scv.lat_sconv_fwd(d["x"], d["wd"], self.km_down.c, self.yc, self.wsb, s)
         rec(8)
@@ -167,55 +165,68 @@ def flush_l2(buf: torch.Tensor):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+    """SM clock and throttle reasons sampled through NVML every ~2 ms while the
+    timed region runs (read-only queries; nothing is changed on the GPU)."""
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv") if os.path.isdir(
-            os.path.join(ROOT, "gpurun_out")) else f"/tmp/lattice_clocks_{os.getpid()}.csv"
+    NAMES = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+             "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+             "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+             "sw_power_cap": "nvmlClocksEventReasonSwPowerCap"}
+
+    def __init__(self, device: torch.device, period_s: float = 0.002):
+        import threading
+        self.period = period_s
+        self.samples = []
+        self.stop = threading.Event()
+        self.thread = None
+        self.handle = None
+        self.max_mhz = None
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nv = nv
+            props = torch.cuda.get_device_properties(device)
+            try:
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                self.handle = nv.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.handle = nv.nvmlDeviceGetHandleByIndex(device.index or 0)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM)
+        except Exception:
+            self.handle = None
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)))
+            except Exception:
+                pass
+            time.sleep(self.period)
 
     def __enter__(self):
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-        try:
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=self.fh, stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+        import threading
+        if self.handle is not None:
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.fh.close()
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
 
     def summary(self) -> dict:
-        if self.proc is None or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            f = [t.strip() for t in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for nm, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if self.handle is None or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"], "samples": 0}
+        reasons = set()
+        for _, r in self.samples:
+            for name, attr in self.NAMES.items():
+                if r & getattr(self.nv, attr):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(c for c, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.samples), "source": "nvml"}
 
 
 def count_launches(pipe: Pipeline) -> int:
@@ -305,6 +316,85 @@ def config_dict(n, world):
             "l2": "flushed (256 MB write) before every timed step"}
 
 
+# --------------------------------------------------------------------------- single-op mode (profiling)
+def run_only(args):
+    """Run one op of the path repeatedly on a named workload (used for ncu captures)."""
+    import sparse_convolution_voxel_b200 as scv
+    from sparse_convolution_voxel_b200 import build as b
+    if not os.path.exists(scv.LIB_PATH):
+        b.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = synthetic.WORKLOADS[args.workload]
+    dt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[wl.dtype]
+    k3 = int(np.prod(wl.ksize))
+    coords = torch.from_numpy(wl.coords()).to(dev)
+    n = coords.shape[0]
+    cin, cout = wl.cin, wl.cout
+    x = torch.from_numpy(synthetic.features(n, cin, wl.seed)).to(dt).to(dev)
+    g = torch.from_numpy(synthetic.features(n, cout, wl.seed, 1)).to(dt).to(dev)
+    w = torch.from_numpy(synthetic.weights(k3, cin, cout, wl.seed)).to(dt).to(dev)
+    st = scv.new_status(dev)
+    ws = scv.Workspace(dev)
+    geom = scv.subm_geom(wl.ksize)
+    table = scv.hash_table(coords, 2.0, st)
+    km = scv.kernel_map(table, n, coords, geom, ws, st)
+    y = torch.empty((n, cout), dtype=dt, device=dev)
+    dx = torch.empty((n, cin), dtype=dt, device=dev)
+    dw = torch.empty((k3, cin, cout), dtype=torch.float32, device=dev)
+    coarse = torch.empty((n * 8, 4), dtype=torch.int32, device=dev)
+    parent = torch.empty(n, dtype=torch.int32, device=dev)
+    wsb = ws.get(max(scv.lat_kmap_ws_bytes(n, k3), scv.lat_sconv_ws_bytes(2, cin, cout, km.c, dt),
+                     scv.lat_downsample_ws_bytes(n, scv.strided_geom(2, 2, 0))))
+    torch.cuda.synchronize()
+    P = int(km.pair_off[k3].item())
+    e = dt.itemsize
+    ops = {
+        "hash": (lambda: scv.lat_hash_build(coords, table, st), n * 32),
+        "kmap": (lambda: scv.lat_kmap_query(table, coords, geom, km.c, wsb, st), n * 16 + n * k3 * 4 + n * 4 + 8 * P),
+        "fwd": (lambda: scv.lat_sconv_fwd(x, w, km.c, y, wsb, st), P * cin * e + n * cout * e + w.numel() * e + 8 * P),
+        "dgrad": (lambda: scv.lat_sconv_dgrad(g, w, km.c, True, dx, wsb, st),
+                  P * cout * e + n * cin * e + w.numel() * e + 8 * P),
+        "wgrad": (lambda: scv.lat_sconv_wgrad(x, g, km.c, dw, wsb, st), P * (cin + cout) * e + dw.numel() * 4 + 8 * P),
+        "downsample": (lambda: scv.lat_downsample_coords(coords, scv.strided_geom(2, 2, 0), coarse, wsb, st,
+                                                         parent=parent),
+                       n * 16 * 2),
+    }
+    fn, nbytes = ops[args.only]
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(args.steps):
+        flush_l2(flush)
+        a, bb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        bb.record()
+        torch.cuda.synchronize()
+        ms.append(a.elapsed_time(bb))
+    # host cost of one call, and the device time per call when calls are issued back to back
+    torch.cuda.synchronize()
+    reps = 20
+    h0 = time.perf_counter()
+    a, bb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        fn()
+    bb.record()
+    host_us = (time.perf_counter() - h0) / reps * 1e6
+    torch.cuda.synchronize()
+    b2b_ms = a.elapsed_time(bb) / reps
+    stv = scv.lat_status_fetch(st)
+    t = statistics.median(ms)
+    hbm, _, src = load_peaks()
+    print(json.dumps({"only": args.only, "workload": args.workload, "rows": n, "pairs": P, "ms_median": t,
+                      "ms_min": min(ms), "alg_bytes": nbytes, "achieved_gbs": nbytes / (t * 1e-3) / 1e9,
+                      "frac_hbm": nbytes / (t * 1e-3) / 1e9 / hbm, "peak_source": src, "status": stv,
+                      "host_us_per_call": host_us, "b2b_ms_per_call": b2b_ms}), flush=True)
+
+
 # --------------------------------------------------------------------------- main GPU arm
 def main():
     ap = argparse.ArgumentParser()
@@ -313,6 +403,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["hash", "kmap", "fwd", "dgrad", "wgrad", "downsample"],
+                    help="time a single op of the path on --workload (for profiler captures)")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(synthetic.WORKLOADS))
     ap.add_argument("--lean", action="store_true",
                     help="skip launch counting, the end-to-end pass and the CPU baseline (for profiler runs)")
     args = ap.parse_args()
@@ -320,6 +413,8 @@ def main():
     world, rank, local = dist_env()
     if args.impl == "reference":
         return run_reference(args)
+    if args.only:
+        return run_only(args)
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -353,7 +448,7 @@ def main():
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev) as clk:
         for i in range(args.steps):
             flush_l2(flush)
             pipe.step(evs[i])

@@ -145,7 +145,8 @@ typedef struct {
  */
 
 /* Bytes of a table for n rows: 16 * next_pow2(max(ceil(rsv_ratio*n), 64)).
- * rsv_ratio must be >= 1 (default 2).  Returns 0 on invalid input. */
+ * rsv_ratio must be >= 1 (default 2); at most 2^31 slots.  Returns 0 on
+ * invalid input. */
 size_t lat_hash_bytes(int64_t n, float rsv_ratio);
 
 /* Insert coords[0..n) (int32 (n,4)) into `table` (table_bytes from
@@ -175,15 +176,35 @@ lat_status lat_kmap_query(const void *table, size_t table_bytes, const int32_t *
  * {stride*q + (ix,iy,iz) - pad} holds at least one active input, batch
  * unchanged.  Written to out_coords (int32 (out_capacity, 4)) sorted by packed
  * key, i.e. in canonical (b, x, y, z) order, so the result is deterministic.
- * geom->mode must be LAT_STRIDED.  Synchronises `stream` and writes the row
- * count to *n_out (HOST pointer).  out_capacity >= n_in is enough when
- * ksize == stride and pad == 0; in general n_in * prod(ceil(ksize/stride))
- * bounds the count.  Too small a capacity returns LAT_ERR_CAPACITY with the
- * needed count in *n_out. */
+ * geom->mode must be LAT_STRIDED.  Synchronises `stream` (twice: once for the
+ * coordinate range, which picks a bitmap counting sort when the coarse fields
+ * pack into at most 30 bits, else a radix sort) and writes the row count to
+ * *n_out (HOST pointer).  out_capacity >= n_in is enough when ksize == stride
+ * and pad == 0; in general n_in * prod(ceil(ksize/stride)) bounds the count.
+ * Too small a capacity returns LAT_ERR_CAPACITY with the needed count in
+ * *n_out.  parent (device int32 [n_in], may be NULL) receives the coarse row
+ * of every input row; it needs ksize == stride and pad == 0 (each input then
+ * lies in exactly one window), else LAT_ERR_UNSUPPORTED. */
 size_t lat_downsample_ws_bytes(int64_t n_in, const lat_geom *geom);
 lat_status lat_downsample_coords(const int32_t *coords, int64_t n_in, const lat_geom *geom,
                                  int32_t *out_coords, int64_t out_capacity, int64_t *n_out,
-                                 void *ws, size_t ws_bytes, int32_t *d_status, lat_stream stream);
+                                 int32_t *parent, void *ws, size_t ws_bytes, int32_t *d_status,
+                                 lat_stream stream);
+
+/* Both kernel maps of a strided Conv3d with ksize == stride and pad == 0,
+ * built from the parent rows that lat_downsample_coords reports instead of by
+ * probing: fine row i sits in coarse window parent[i] at offset
+ * k(i) = (o0*Ky + o1)*Kz + o2 with o = fine coordinate mod stride (floor).
+ *   down  LAT_STRIDED map: n_out = coarse rows, n_in = fine rows
+ *         (nbr[k(i)][parent[i]] = i);
+ *   up    LAT_TRANSPOSED map: n_out = fine rows, n_in = coarse rows
+ *         (nbr[k][i] = parent[i] if k == k(i), else -1).
+ * Either map may be NULL.  The caller sets n_in / n_out / k3 of each map; the
+ * results equal what lat_kmap_query returns for the same geometry. */
+size_t lat_kmap_from_parent_ws_bytes(int64_t n_fine, int64_t n_coarse, int32_t k3);
+lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int32_t *parent, const lat_geom *geom,
+                                lat_kmap *down, lat_kmap *up, void *ws, size_t ws_bytes,
+                                int32_t *d_status, lat_stream stream);
 
 /* ------------------------------------------------------------ convolution --
  * y[j] = sum over k with nbr[k][j] >= 0 of x[nbr[k][j]] . W[k]

@@ -18,12 +18,13 @@ import torch
 from ._lib import (  # noqa: F401  (re-exported C entry points and constants)
     EXPORTS, LAT_BF16, LAT_F16, LAT_F32, LAT_OK, LAT_OP_DGRAD, LAT_OP_FWD, LAT_OP_WGRAD, LAT_STRIDED, LAT_SUBM,
     LAT_TILE_ROWS, LAT_TRANSPOSED, LIB_PATH, LatticeError, lat_downsample_coords, lat_downsample_ws_bytes, lat_geom,
-    lat_hash_build, lat_hash_bytes, lat_kmap, lat_kmap_query, lat_kmap_ws_bytes, lat_sconv_dgrad, lat_sconv_fwd,
+    lat_hash_build, lat_hash_bytes, lat_kmap, lat_kmap_from_parent, lat_kmap_from_parent_ws_bytes, lat_kmap_query,
+    lat_kmap_ws_bytes, lat_sconv_dgrad, lat_sconv_fwd,
     lat_sconv_wgrad, lat_sconv_wgrad_static, lat_sconv_ws_bytes, lat_status_fetch, lat_status_string, lat_version, load, make_geom,
 )
 
 __all__ = [
-    "KernelMap", "Workspace", "hash_table", "kernel_map", "downsample", "conv_fwd", "conv_dgrad", "conv_wgrad",
+    "KernelMap", "Workspace", "hash_table", "kernel_map", "downsample", "maps_from_parent", "conv_fwd", "conv_dgrad", "conv_wgrad",
     "subm_geom", "strided_geom", "transposed_geom", "check_status", "new_status",
 ] + EXPORTS
 
@@ -117,17 +118,33 @@ def kernel_map(table: torch.Tensor, n_in: int, out_coords: torch.Tensor, geom: l
 
 
 def downsample(coords: torch.Tensor, geom: lat_geom, ws: Workspace | None = None, d_status=None,
-               capacity: int | None = None, stream=None) -> torch.Tensor:
-    """Coarse support of a strided Conv3d in canonical order (synchronises)."""
+               capacity: int | None = None, stream=None, with_parent: bool = False):
+    """Coarse support of a strided Conv3d in canonical order (synchronises).
+    With with_parent=True also returns the coarse row of every input row."""
     n = coords.shape[0]
     per = 1
     for a in range(3):
         per *= -(-geom.ksize[a] // geom.stride[a])
     cap = n * per if capacity is None else int(capacity)
     out = torch.empty((max(1, cap), 4), dtype=torch.int32, device=coords.device)
+    parent = torch.empty(max(1, n), dtype=torch.int32, device=coords.device) if with_parent else None
     ws = ws or Workspace(coords.device)
-    m = lat_downsample_coords(coords, geom, out, ws.get(lat_downsample_ws_bytes(n, geom)), d_status, stream)
-    return out[:m]
+    m = lat_downsample_coords(coords, geom, out, ws.get(lat_downsample_ws_bytes(n, geom)), d_status, stream,
+                              parent=parent)
+    return (out[:m], parent[:n]) if with_parent else out[:m]
+
+
+def maps_from_parent(fine_coords: torch.Tensor, parent: torch.Tensor, n_coarse: int, geom: lat_geom,
+                     ws: Workspace | None = None, d_status=None, stream=None):
+    """(strided map, transposed map) of a ksize == stride, pad == 0 Conv3d from parent rows."""
+    n = fine_coords.shape[0]
+    k3 = geom.ksize[0] * geom.ksize[1] * geom.ksize[2]
+    down = KernelMap(n, n_coarse, k3, fine_coords.device)
+    up = KernelMap(n_coarse, n, k3, fine_coords.device)
+    ws = ws or Workspace(fine_coords.device)
+    lat_kmap_from_parent(fine_coords, parent, geom, down.c, up.c, ws.get(lat_kmap_from_parent_ws_bytes(n, n_coarse, k3)),
+                         d_status, stream)
+    return down, up
 
 
 def conv_fwd(x, w, kmap: KernelMap, ws: Workspace | None = None, d_status=None, out=None, stream=None):

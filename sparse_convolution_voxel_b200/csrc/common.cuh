@@ -6,6 +6,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "lattice.h"
 
 namespace lat {
@@ -98,6 +100,52 @@ inline int num_sms() {
     return n;
 }
 inline bool pow2(uint64_t v) { return v && !(v & (v - 1)); }
+
+// CTAs of a persistent kernel that can be resident at once on the current device.
+// The kernels are compiled with __launch_bounds__(threads, max_per_sm), so
+// registers admit max_per_sm CTAs; shared memory admits
+// smem_per_sm / (dynamic + static + per-block reserve); tensor memory (512
+// columns per SM) admits 512 / tmem_cols.  (The runtime occupancy query
+// under-reports here, so the limit is computed from the device attributes.)
+// Also raises the kernel's dynamic shared-memory limit and asks for the
+// largest carveout.  Returns 0 on error.
+template <typename K>
+inline int64_t persistent_grid_uncached(K kern, uint32_t smem, int tmem_cols, int max_per_sm) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess) return 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess) return 0;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return 0;
+    int smem_sm = 0, reserve = 0;
+    if (cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&reserve, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
+        return 0;
+    int per_sm = max_per_sm;
+    const size_t per_cta = size_t(smem) + fa.sharedSizeBytes + size_t(reserve);
+    if (int(smem_sm / per_cta) < per_sm) per_sm = int(smem_sm / per_cta);
+    if (tmem_cols > 0 && per_sm > 512 / tmem_cols) per_sm = 512 / tmem_cols;
+    if (per_sm < 1) return 0;
+    return int64_t(per_sm) * num_sms();
+}
+
+// Per-device cache of one kernel's persistent grid; instantiate once per kernel
+// (the Tag makes every kernel's cache distinct).  The first call on a device
+// sets the kernel's attributes there.
+template <typename Tag>
+struct GridCache {
+    template <typename K>
+    static int64_t get(K kern, uint32_t smem, int tmem_cols, int max_per_sm) {
+        constexpr int kMaxDev = 64;
+        static int64_t cached[kMaxDev] = {};
+        static std::mutex mu;
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return 0;
+        std::lock_guard<std::mutex> lock(mu);
+        if (cached[dev] <= 0) cached[dev] = persistent_grid_uncached(kern, smem, tmem_cols, max_per_sm);
+        return cached[dev];
+    }
+};
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Carves consecutive 256-byte aligned sub-buffers out of a caller workspace.

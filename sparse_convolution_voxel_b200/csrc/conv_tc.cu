@@ -39,7 +39,8 @@ constexpr int kProdWarps = 4;    // gather warps
 constexpr int kEpiWarps = 4;     // epilogue warps
 constexpr int kMmaWarp = kProdWarps + kEpiWarps;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
-constexpr int kLag = 3;          // cp.async groups a gather thread keeps in flight
+constexpr int kLag = 2;          // cp.async groups a gather thread keeps in flight
+constexpr int kIdxBatch = 8;     // neighbour indices a gather thread loads at once
 constexpr uint32_t kABytes = kM * 128;  // 128 rows x 64 channels x 2 bytes
 constexpr uint64_t kWaitNs = 2000000000ull;
 
@@ -47,13 +48,15 @@ template <int N>
 struct Cfg {
     static constexpr uint32_t kBBytes = uint32_t(N) * 128;  // 64 K x N (or N x 64) x 2 bytes
     static constexpr uint32_t kStage = kABytes + kBBytes;
-    static constexpr int kStages = N == 64 ? 8 : 6;
+    static constexpr int kStages = N == 64 ? 4 : 3;  // ~96 KB: two CTAs per SM
     static constexpr uint32_t kBarBytes = 256;
     static constexpr uint32_t kSmem = kStages * kStage + kBarBytes + 1024;
     static constexpr uint32_t kTmemCols = 2 * N;
 };
 
 template <typename T> constexpr bool is_bf16() { return sizeof(T) == 2 && !std::is_same<T, __half>::value; }
+
+template <typename T, int KC, int N, bool BMN> struct KernelTag {};  // one launch-config cache per kernel
 
 // Instruction descriptor, kind::f16: fp32 D, A/B fp16 or bf16, A K-major,
 // B MN-major (forward: W[k] is (Cin x Cout), Cout contiguous) or K-major
@@ -75,7 +78,7 @@ __device__ __forceinline__ uint32_t pack2(float a, float b, __nv_bfloat16) {
 
 // KC: gathered channels (GEMM K), N: output channels, BMN: B operand MN-major.
 template <typename T, int KC, int N, bool BMN>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x, MapView mv, T *__restrict__ y,
                int32_t *d_status) {
     using C = Cfg<N>;
@@ -119,53 +122,75 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x
 
     if (warp < kProdWarps) {
         // ------------------------------------------------------------ gather + TMA
+        // Thread tid owns tile row tid: its output row (perm) is fetched one tile
+        // ahead, and the input rows of up to kIdxBatch offsets are fetched together,
+        // so the index loads overlap instead of stalling each copy.
         uint32_t it = 0;
         bool ok = true;
-        for (int64_t t = blockIdx.x; t < mv.ntiles && ok; t += gridDim.x) {
+        int64_t t = blockIdx.x;
+        int j_next = (t < mv.ntiles && t * kM + tid < mv.n_out) ? __ldg(mv.perm + t * kM + tid) : -1;
+        for (; t < mv.ntiles && ok; t += gridDim.x) {
             const uint32_t tm = mv.tile_mask_at(t);
-            const int64_t my_row = t * kM + tid;
-            const int j_own = my_row < mv.n_out ? __ldg(mv.perm + my_row) : -1;
-            for (uint32_t m = tm; m && ok; m &= m - 1) {
-                const int k = __ffs(m) - 1;
-                int src_own = j_own >= 0 ? mv.neighbour(k, j_own) : -1;
-                if (src_own >= mv.n_in) {
-                    bad |= LAT_ERR_BAD_MAP;
-                    src_own = -1;
+            const int j_own = j_next;
+            const int64_t tn = t + gridDim.x;
+            j_next = (tn < mv.ntiles && tn * kM + tid < mv.n_out) ? __ldg(mv.perm + tn * kM + tid) : -1;
+            uint32_t rem = tm;
+            while (rem && ok) {
+                int kk[kIdxBatch], src_b[kIdxBatch];
+#pragma unroll
+                for (int e = 0; e < kIdxBatch; ++e) {
+                    kk[e] = -1;
+                    src_b[e] = -1;
+                    if (rem) {
+                        kk[e] = __ffs(rem) - 1;
+                        rem &= rem - 1;
+                        if (j_own >= 0) src_b[e] = mv.neighbour(kk[e], j_own);
+                    }
                 }
-                for (int kb = 0; kb < KBLK; ++kb) {
-                    const uint32_t s = it % NS;
-                    if (!ptx::mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, kWaitNs)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t *As = smem + s * C::kStage;
-                    uint8_t *Bs = As + kABytes;
-                    if (tid == 0) {
-                        ptx::mbar_arrive_expect_tx(&full[s], C::kBBytes);
 #pragma unroll
-                        for (int nb = 0; nb < N / 64; ++nb) {
-                            if constexpr (BMN)  // rows k*KC + 64kb.., columns 64nb..
-                                ptx::tma_load_2d(Bs + nb * 8192, &wmap, &full[s], 64 * nb, k * KC + 64 * kb);
-                            else                // rows k*N + 64nb.., columns 64kb..
-                                ptx::tma_load_2d(Bs + nb * 8192, &wmap, &full[s], 64 * kb, k * N + 64 * nb);
+                for (int e = 0; e < kIdxBatch; ++e) {
+                    if (kk[e] < 0 || !ok) continue;
+                    const int k = kk[e];
+                    int src_own = src_b[e];
+                    if (src_own >= mv.n_in) {
+                        bad |= LAT_ERR_BAD_MAP;
+                        src_own = -1;
+                    }
+                    for (int kb = 0; kb < KBLK; ++kb) {
+                        const uint32_t s = it % NS;
+                        if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, kWaitNs))) {
+                            ok = false;
+                            break;
                         }
-                    }
+                        uint8_t *As = smem + s * C::kStage;
+                        uint8_t *Bs = As + kABytes;
+                        if (tid == 0) {
+                            ptx::mbar_arrive_expect_tx(&full[s], C::kBBytes);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int rl = 4 * i + (lane >> 3);
-                        const int row = warp * 32 + rl;
-                        const int chunk = lane & 7;
-                        const int src = __shfl_sync(0xFFFFFFFFu, src_own, rl);
-                        const T *gp = src >= 0 ? x + int64_t(src) * KC + kb * 64 + chunk * 8 : x;
-                        ptx::cp_async16(As + row * 128 + ((chunk ^ (row & 7)) << 4), gp, src >= 0 ? 16u : 0u);
+                            for (int nb = 0; nb < N / 64; ++nb) {
+                                if constexpr (BMN)  // rows k*KC + 64kb.., columns 64nb..
+                                    ptx::tma_load_2d(Bs + nb * 8192, &wmap, &full[s], 64 * nb, k * KC + 64 * kb);
+                                else                // rows k*N + 64nb.., columns 64kb..
+                                    ptx::tma_load_2d(Bs + nb * 8192, &wmap, &full[s], 64 * kb, k * N + 64 * nb);
+                            }
+                        }
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int rl = 4 * i + (lane >> 3);
+                            const int row = warp * 32 + rl;
+                            const int chunk = lane & 7;
+                            const int src = __shfl_sync(0xFFFFFFFFu, src_own, rl);
+                            const T *gp = src >= 0 ? x + int64_t(src) * KC + kb * 64 + chunk * 8 : x;
+                            ptx::cp_async16(As + row * 128 + ((chunk ^ (row & 7)) << 4), gp, src >= 0 ? 16u : 0u);
+                        }
+                        ptx::cp_async_commit();
+                        if (it >= kLag) {
+                            ptx::cp_async_wait<kLag>();
+                            ptx::fence_proxy_async_smem();
+                            ptx::mbar_arrive(&full[(it - kLag) % NS]);
+                        }
+                        ++it;
                     }
-                    ptx::cp_async_commit();
-                    if (it >= kLag) {
-                        ptx::cp_async_wait<kLag>();
-                        ptx::fence_proxy_async_smem();
-                        ptx::mbar_arrive(&full[(it - kLag) % NS]);
-                    }
-                    ++it;
                 }
             }
         }
@@ -178,10 +203,14 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x
         const int q = warp & 3;
         uint32_t ta = 0;
         bool ok = true;
-        for (int64_t t = blockIdx.x; t < mv.ntiles && ok; t += gridDim.x) {
+        int64_t t = blockIdx.x;
+        int j_next = (t < mv.ntiles && t * kM + q * 32 + lane < mv.n_out) ? __ldg(mv.perm + t * kM + q * 32 + lane) : -1;
+        for (; t < mv.ntiles && ok; t += gridDim.x) {
             const uint32_t tm = mv.tile_mask_at(t);
-            const int64_t grow = t * kM + q * 32 + lane;
-            const int j = grow < mv.n_out ? __ldg(mv.perm + grow) : -1;
+            const int j = j_next;
+            const int64_t tn = t + gridDim.x;
+            j_next = (tn < mv.ntiles && tn * kM + q * 32 + lane < mv.n_out) ? __ldg(mv.perm + tn * kM + q * 32 + lane)
+                                                                             : -1;
             T *yr = j >= 0 ? y + int64_t(j) * N : nullptr;
             if (!tm) {  // no neighbour anywhere in the tile: zeros
                 if (yr)
@@ -190,7 +219,7 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x
                 continue;
             }
             const uint32_t a = ta & 1;
-            if (!ptx::mbar_wait(&accfull[a], (ta >> 1) & 1, kWaitNs)) {
+            if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(&accfull[a], (ta >> 1) & 1, kWaitNs))) {
                 ok = false;
                 break;
             }
@@ -315,8 +344,8 @@ static lat_status launch(const void *x, const void *w, int k3, const MapView &mv
     // forward: W[k] is (KC x N); data gradient: W[k] is (N x KC)
     if (!make_weight_map(&map, w, is_bf16<T>(), k3, BMN ? KC : N, BMN ? N : KC)) return LAT_ERR_CUDA;
     auto kern = conv_tc_kernel<T, KC, N, BMN>;
-    LAT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::kSmem)));
-    const int64_t grid = std::min<int64_t>(mv.ntiles, num_sms());
+    const int64_t grid = std::min<int64_t>(mv.ntiles, GridCache<KernelTag<T, KC, N, BMN>>::get(kern, C::kSmem, int(C::kTmemCols), 2));
+    if (grid <= 0) return LAT_ERR_CUDA;
     kern<<<unsigned(grid), kThreads, C::kSmem, s>>>(map, static_cast<const T *>(x), mv, static_cast<T *>(y),
                                                     d_status);
     LAT_CUDA_TRY(cudaGetLastError());

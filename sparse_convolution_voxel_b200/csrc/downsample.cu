@@ -5,11 +5,25 @@
 // a strided forward convolution creates a downsampled support.  The coarse
 // support is every q whose window {stride*q + off - pad, off in [0,K)^3}
 // holds an active input.  Each input row proposes the coarse rows whose
-// windows contain it (exactly one when K == stride and pad == 0: floor(p/s)),
-// the packed keys are radix sorted and made unique, so the result is in
-// canonical (b, x, y, z) order and independent of the input row order.
+// windows contain it (exactly one when K == stride and pad == 0: floor(p/s)).
+// The proposals are made unique and put in canonical (b, x, y, z) order, so
+// the result does not depend on the input row order.
+//
+// Two ways to sort + unique, chosen after one pass that finds the range of
+// every coarse field:
+//   * counting sort on a bitmap: when the fields, shifted to start at their
+//     minimum, pack into a key of at most 30 bits and the bitmap is no larger
+//     than max(2^24, 512 bits per proposal), every proposal sets its bit, a
+//     scan of per-1024-bit popcounts gives each set bit its rank, and the
+//     ranks are the sorted unique order;
+//   * otherwise a radix sort of the packed 64-bit keys followed by unique.
+// Both can also report each input's coarse row (its parent) when K == stride
+// and pad == 0.
 #include <cub/device/device_radix_sort.cuh>
+#include <cub/device/device_scan.cuh>
 #include <cub/device/device_select.cuh>
+
+#include <climits>
 
 #include "common.cuh"
 
@@ -21,41 +35,163 @@ struct DownGeom {
     int cands;        // product of per_axis
 };
 
+constexpr int kMaxBitmapBits = 30;
+
+// Candidate coarse rows of every input as packed keys (EMPTY when a candidate
+// does not exist), and the min / max of each coarse field over all candidates
+// (range[0..3] = min b,x,y,z; range[4..7] = max).
 __global__ void __launch_bounds__(256)
 down_candidates_kernel(const int4 *__restrict__ coords, int64_t n, DownGeom g, uint64_t *__restrict__ keys,
-                       int32_t *d_status) {
+                       int *__restrict__ range, int32_t *d_status) {
+    int mn[4] = {INT_MAX, INT_MAX, INT_MAX, INT_MAX}, mx[4] = {INT_MIN, INT_MIN, INT_MIN, INT_MIN};
+    const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+    if (i < n) {
+        const int4 c = __ldg(coords + i);
+        uint64_t self;
+        uint64_t *dst = keys + i * g.cands;
+        if (!pack_key(c.x, c.y, c.z, c.w, self)) {
+            for (int e = 0; e < g.cands; ++e) dst[e] = kEmptyKey;
+            flag(d_status, LAT_ERR_COORD_RANGE);
+        } else {
+            const int p[3] = {c.y, c.z, c.w};
+            int first[3];  // smallest off in [0,K) with (p - off + pad) divisible by s
+#pragma unroll
+            for (int a = 0; a < 3; ++a) first[a] = (p[a] + g.pd[a]) - floordiv(p[a] + g.pd[a], g.st[a]) * g.st[a];
+            int e = 0;
+            for (int u = 0; u < g.per_axis[0]; ++u)
+                for (int v = 0; v < g.per_axis[1]; ++v)
+                    for (int w = 0; w < g.per_axis[2]; ++w, ++e) {
+                        const int off[3] = {first[0] + u * g.st[0], first[1] + v * g.st[1], first[2] + w * g.st[2]};
+                        uint64_t key = kEmptyKey;
+                        if (off[0] < g.ks[0] && off[1] < g.ks[1] && off[2] < g.ks[2]) {
+                            int q[3];
+#pragma unroll
+                            for (int a = 0; a < 3; ++a) q[a] = (p[a] - off[a] + g.pd[a]) / g.st[a];  // exact
+                            if (pack_key(c.x, q[0], q[1], q[2], key)) {
+                                const int f[4] = {c.x, q[0], q[1], q[2]};
+#pragma unroll
+                                for (int a = 0; a < 4; ++a) {
+                                    mn[a] = min(mn[a], f[a]);
+                                    mx[a] = max(mx[a], f[a]);
+                                }
+                            } else {
+                                key = kEmptyKey;
+                            }
+                        }
+                        dst[e] = key;
+                    }
+        }
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        for (int o = 16; o; o >>= 1) {
+            mn[a] = min(mn[a], __shfl_xor_sync(0xFFFFFFFFu, mn[a], o));
+            mx[a] = max(mx[a], __shfl_xor_sync(0xFFFFFFFFu, mx[a], o));
+        }
+    }
+    if ((threadIdx.x & 31) == 0 && mn[0] != INT_MAX) {
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            atomicMin(range + a, mn[a]);
+            atomicMax(range + 4 + a, mx[a]);
+        }
+    }
+}
+
+__global__ void range_init_kernel(int *range) {
+    if (threadIdx.x < 4) range[threadIdx.x] = INT_MAX;
+    else if (threadIdx.x < 8) range[threadIdx.x] = INT_MIN;
+}
+
+// Order-preserving compact key of a coarse row: fields shifted to their minimum, packed.
+struct Compact {
+    int mn[4];
+    int w[4];  // bit widths of b, x, y, z
+    __device__ __forceinline__ uint32_t pack(uint64_t key) const {
+        int4 c;
+        unpack_key(key, c);
+        uint32_t v = uint32_t(c.x - mn[0]);
+        v = (v << w[1]) | uint32_t(c.y - mn[1]);
+        v = (v << w[2]) | uint32_t(c.z - mn[2]);
+        v = (v << w[3]) | uint32_t(c.w - mn[3]);
+        return v;
+    }
+    __device__ __forceinline__ int4 unpack(uint32_t v) const {
+        int4 c;
+        c.w = int(v & ((1u << w[3]) - 1u)) + mn[3];
+        v >>= w[3];
+        c.z = int(v & ((1u << w[2]) - 1u)) + mn[2];
+        v >>= w[2];
+        c.y = int(v & ((1u << w[1]) - 1u)) + mn[1];
+        v >>= w[1];
+        c.x = int(v) + mn[0];
+        return c;
+    }
+};
+
+__global__ void __launch_bounds__(256)
+bitmap_mark_kernel(const uint64_t *__restrict__ keys, int64_t items, Compact cp, uint32_t *__restrict__ bitmap) {
+    const int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+    if (e >= items) return;
+    const uint64_t key = keys[e];
+    if (key == kEmptyKey) return;
+    const uint32_t v = cp.pack(key);
+    atomicOr(bitmap + (v >> 5), 1u << (v & 31));
+}
+
+// set bits per group of 32 words (1024 bits)
+__global__ void __launch_bounds__(256)
+bitmap_count_kernel(const uint32_t *__restrict__ bitmap, int64_t ngroups, int32_t *__restrict__ grp_cnt) {
+    const int64_t gi = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+    if (gi >= ngroups) return;
+    const uint4 *w4 = reinterpret_cast<const uint4 *>(bitmap + gi * 32);
+    int c = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const uint4 v = __ldg(w4 + e);
+        c += __popc(v.x) + __popc(v.y) + __popc(v.z) + __popc(v.w);
+    }
+    grp_cnt[gi] = c;
+}
+
+// Coordinates of the set bits in bit order (= canonical order); also the total count.
+__global__ void __launch_bounds__(256)
+bitmap_emit_kernel(const uint32_t *__restrict__ bitmap, int64_t ngroups, const int32_t *__restrict__ grp_cnt,
+                   const int64_t *__restrict__ grp_off, Compact cp, int4 *__restrict__ out, int64_t capacity,
+                   int64_t *__restrict__ n_out_dev) {
+    const int64_t gi = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+    if (gi >= ngroups) return;
+    if (gi == ngroups - 1) *n_out_dev = grp_off[gi] + grp_cnt[gi];
+    if (grp_cnt[gi] == 0) return;
+    int64_t rank = grp_off[gi];
+    for (int wi = 0; wi < 32; ++wi) {
+        uint32_t word = bitmap[gi * 32 + wi];
+        while (word) {
+            const int b = __ffs(word) - 1;
+            word &= word - 1;
+            if (rank < capacity) out[rank] = cp.unpack(uint32_t(gi * 1024 + wi * 32 + b));
+            ++rank;
+        }
+    }
+}
+
+// Rank of each input's (single) proposal among the set bits: its coarse row.
+__global__ void __launch_bounds__(256)
+bitmap_parent_kernel(const uint64_t *__restrict__ keys, int64_t n, Compact cp, const uint32_t *__restrict__ bitmap,
+                     const int64_t *__restrict__ grp_off, int32_t *__restrict__ parent) {
     const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
     if (i >= n) return;
-    const int4 c = __ldg(coords + i);
-    uint64_t self;
-    uint64_t *dst = keys + i * g.cands;
-    if (!pack_key(c.x, c.y, c.z, c.w, self)) {
-        for (int e = 0; e < g.cands; ++e) dst[e] = kEmptyKey;
-        flag(d_status, LAT_ERR_COORD_RANGE);
+    const uint64_t key = keys[i];
+    if (key == kEmptyKey) {
+        parent[i] = -1;
         return;
     }
-    const int p[3] = {c.y, c.z, c.w};
-    int first[3];  // smallest off in [0,K) with (p - off + pad) divisible by s
-#pragma unroll
-    for (int a = 0; a < 3; ++a) {
-        const int r = (p[a] + g.pd[a]) - floordiv(p[a] + g.pd[a], g.st[a]) * g.st[a];
-        first[a] = r;
-    }
-    int e = 0;
-    for (int u = 0; u < g.per_axis[0]; ++u)
-        for (int v = 0; v < g.per_axis[1]; ++v)
-            for (int w = 0; w < g.per_axis[2]; ++w, ++e) {
-                const int off[3] = {first[0] + u * g.st[0], first[1] + v * g.st[1], first[2] + w * g.st[2]};
-                uint64_t key = kEmptyKey;
-                bool ok = off[0] < g.ks[0] && off[1] < g.ks[1] && off[2] < g.ks[2];
-                if (ok) {
-                    int q[3];
-#pragma unroll
-                    for (int a = 0; a < 3; ++a) q[a] = (p[a] - off[a] + g.pd[a]) / g.st[a];  // exact division
-                    if (!pack_key(c.x, q[0], q[1], q[2], key)) key = kEmptyKey;
-                }
-                dst[e] = key;
-            }
+    const uint32_t v = cp.pack(key);
+    const uint32_t gi = v >> 10, wi = (v >> 5) & 31;
+    int64_t rank = grp_off[gi];
+    for (uint32_t e = 0; e < wi; ++e) rank += __popc(__ldg(bitmap + gi * 32 + e));
+    rank += __popc(__ldg(bitmap + (v >> 5)) & ((1u << (v & 31)) - 1u));
+    parent[i] = int32_t(rank);
 }
 
 // Unpack the unique keys (the last one may be the EMPTY filler) into coordinate rows.
@@ -72,13 +208,21 @@ down_unpack_kernel(const uint64_t *__restrict__ uniq, const int *__restrict__ n_
     out[r] = c;
 }
 
-struct DownWs {
-    uint64_t *keys, *sorted, *uniq;
-    int *n_uniq;
-    int64_t *n_out_dev;
-    void *sort_tmp, *sel_tmp;
-    size_t sort_bytes, sel_bytes, total;
-};
+// Coarse row of each input by binary search in the sorted unique keys.
+__global__ void __launch_bounds__(256)
+sorted_parent_kernel(const uint64_t *__restrict__ keys, int64_t n, const uint64_t *__restrict__ uniq,
+                     const int64_t *__restrict__ n_out_dev, int32_t *__restrict__ parent) {
+    const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+    if (i >= n) return;
+    const uint64_t key = keys[i];
+    int64_t lo = 0, hi = *n_out_dev;
+    while (lo < hi) {
+        const int64_t mid = (lo + hi) >> 1;
+        if (uniq[mid] < key) lo = mid + 1;
+        else hi = mid;
+    }
+    parent[i] = (key != kEmptyKey && lo < *n_out_dev && uniq[lo] == key) ? int32_t(lo) : -1;
+}
 
 static bool down_geom(const lat_geom *geom, DownGeom &g) {
     if (!geom || geom->mode != LAT_STRIDED) return false;
@@ -95,22 +239,67 @@ static bool down_geom(const lat_geom *geom, DownGeom &g) {
     return g.ks[0] * g.ks[1] * g.ks[2] <= 32;
 }
 
-static DownWs carve_down_ws(void *base, int64_t n_items) {
+// Largest bitmap (bits) the counting-sort path may use for `items` proposals.
+static int64_t bitmap_budget_bits(int64_t items) {
+    int64_t b = std::max<int64_t>(int64_t(1) << 24, 512 * items);
+    return std::min<int64_t>(b, int64_t(1) << kMaxBitmapBits);
+}
+
+struct DownWs {
+    uint64_t *keys;
+    int *range;
+    int64_t *n_out_dev;
+    // sort path
+    uint64_t *sorted, *uniq;
+    int *n_uniq;
+    void *sort_tmp, *sel_tmp;
+    size_t sort_bytes, sel_bytes;
+    // bitmap path
+    uint32_t *bitmap;
+    int32_t *grp_cnt;
+    int64_t *grp_off;
+    void *scan_tmp;
+    size_t scan_bytes;
+    int64_t max_groups;
+    size_t total;
+};
+
+static DownWs carve_down_ws(void *base, int64_t items) {
     DownWs w{};
     Carver cv(base);
-    w.keys = cv.take<uint64_t>(size_t(n_items));
-    w.sorted = cv.take<uint64_t>(size_t(n_items));
-    w.uniq = cv.take<uint64_t>(size_t(n_items));
-    w.n_uniq = cv.take<int>(1);
+    w.keys = cv.take<uint64_t>(size_t(items));
+    w.range = cv.take<int>(8);
     w.n_out_dev = cv.take<int64_t>(1);
+    const size_t common = cv.used;
+    // sort path
+    w.sorted = cv.take<uint64_t>(size_t(items));
+    w.uniq = cv.take<uint64_t>(size_t(items));
+    w.n_uniq = cv.take<int>(1);
     cub::DeviceRadixSort::SortKeys(nullptr, w.sort_bytes, (const uint64_t *)nullptr, (uint64_t *)nullptr,
-                                   int(n_items), 0, 64);
+                                   int(items), 0, 64);
     cub::DeviceSelect::Unique(nullptr, w.sel_bytes, (const uint64_t *)nullptr, (uint64_t *)nullptr, (int *)nullptr,
-                              int(n_items));
+                              int(items));
     w.sort_tmp = cv.take<char>(w.sort_bytes);
     w.sel_tmp = cv.take<char>(w.sel_bytes);
-    w.total = align_up(cv.used, 256);
+    const size_t sort_end = cv.used;
+    // bitmap path (overlaps the sort path's buffers)
+    cv.used = common;
+    const int64_t bits = bitmap_budget_bits(items);
+    w.max_groups = std::max<int64_t>(1, bits / 1024);
+    w.bitmap = cv.take<uint32_t>(size_t(w.max_groups) * 32);
+    w.grp_cnt = cv.take<int32_t>(size_t(w.max_groups));
+    w.grp_off = cv.take<int64_t>(size_t(w.max_groups));
+    cub::DeviceScan::ExclusiveSum(nullptr, w.scan_bytes, (const int32_t *)nullptr, (int64_t *)nullptr,
+                                  int(w.max_groups));
+    w.scan_tmp = cv.take<char>(w.scan_bytes);
+    w.total = align_up(std::max(sort_end, cv.used), 256);
     return w;
+}
+
+static int bit_width(int64_t span) {  // bits to hold values 0..span
+    int b = 0;
+    while ((int64_t(1) << b) <= span) ++b;
+    return b;
 }
 
 }  // namespace lat
@@ -120,17 +309,22 @@ extern "C" size_t lat_downsample_ws_bytes(int64_t n_in, const lat_geom *geom) {
     if (n_in < 0 || !lat::down_geom(geom, g)) return 0;
     const int64_t items = n_in * g.cands;
     if (items >= (int64_t(1) << 31)) return 0;
-    return lat::carve_down_ws(nullptr, items).total;
+    return lat::carve_down_ws(nullptr, std::max<int64_t>(items, 1)).total;
 }
 
 extern "C" lat_status lat_downsample_coords(const int32_t *coords, int64_t n_in, const lat_geom *geom,
-                                            int32_t *out_coords, int64_t out_capacity, int64_t *n_out, void *ws,
-                                            size_t ws_bytes, int32_t *d_status, lat_stream stream) {
+                                            int32_t *out_coords, int64_t out_capacity, int64_t *n_out,
+                                            int32_t *parent, void *ws, size_t ws_bytes, int32_t *d_status,
+                                            lat_stream stream) {
     using namespace lat;
     DownGeom g;
     if (!n_out || n_in < 0 || out_capacity < 0 || !down_geom(geom, g)) return LAT_ERR_ARG;
     if (n_in > 0 && (!coords || (out_capacity > 0 && !out_coords))) return LAT_ERR_ARG;
     if (reinterpret_cast<uintptr_t>(coords) % 16 || reinterpret_cast<uintptr_t>(out_coords) % 16) return LAT_ERR_ARG;
+    if (parent) {  // one coarse row per input only when the kernel tiles the stride exactly
+        for (int a = 0; a < 3; ++a)
+            if (g.ks[a] != g.st[a] || g.pd[a] != 0) return LAT_ERR_UNSUPPORTED;
+    }
     const int64_t items = n_in * g.cands;
     if (items >= (int64_t(1) << 31)) return LAT_ERR_UNSUPPORTED;
     *n_out = 0;
@@ -139,17 +333,60 @@ extern "C" lat_status lat_downsample_coords(const int32_t *coords, int64_t n_in,
     if (!ws || ws_bytes < need.total) return LAT_ERR_WORKSPACE;
     DownWs w = carve_down_ws(ws, items);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    down_candidates_kernel<<<unsigned((n_in + 255) / 256), 256, 0, s>>>(reinterpret_cast<const int4 *>(coords), n_in,
-                                                                         g, w.keys, d_status);
+    const unsigned in_blocks = unsigned((n_in + 255) / 256), item_blocks = unsigned((items + 255) / 256);
+
+    range_init_kernel<<<1, 32, 0, s>>>(w.range);
     LAT_CUDA_TRY(cudaGetLastError());
-    size_t b = w.sort_bytes;
-    LAT_CUDA_TRY(cub::DeviceRadixSort::SortKeys(w.sort_tmp, b, w.keys, w.sorted, int(items), 0, 64, s));
-    b = w.sel_bytes;
-    LAT_CUDA_TRY(cub::DeviceSelect::Unique(w.sel_tmp, b, w.sorted, w.uniq, w.n_uniq, int(items), s));
-    down_unpack_kernel<<<unsigned((items + 255) / 256), 256, 0, s>>>(w.uniq, w.n_uniq,
-                                                                     reinterpret_cast<int4 *>(out_coords),
-                                                                     out_capacity, w.n_out_dev);
+    down_candidates_kernel<<<in_blocks, 256, 0, s>>>(reinterpret_cast<const int4 *>(coords), n_in, g, w.keys, w.range,
+                                                     d_status);
     LAT_CUDA_TRY(cudaGetLastError());
+    int range[8];
+    LAT_CUDA_TRY(cudaMemcpyAsync(range, w.range, sizeof(range), cudaMemcpyDeviceToHost, s));
+    LAT_CUDA_TRY(cudaStreamSynchronize(s));
+    if (range[0] == INT_MAX) {  // no coarse row exists
+        if (parent) LAT_CUDA_TRY(cudaMemsetAsync(parent, 0xFF, sizeof(int32_t) * n_in, s));
+        return LAT_OK;
+    }
+    Compact cp;
+    int total_bits = 0;
+    for (int a = 0; a < 4; ++a) {
+        cp.mn[a] = range[a];
+        cp.w[a] = bit_width(int64_t(range[4 + a]) - range[a]);
+        total_bits += cp.w[a];
+    }
+    const int64_t bits = total_bits <= kMaxBitmapBits ? (int64_t(1) << total_bits) : 0;
+    if (total_bits <= kMaxBitmapBits && bits <= bitmap_budget_bits(items)) {
+        // ------------------------------------------------ counting sort on a bitmap
+        const int64_t ngroups = std::max<int64_t>(1, bits / 1024);
+        LAT_CUDA_TRY(cudaMemsetAsync(w.bitmap, 0, sizeof(uint32_t) * size_t(ngroups) * 32, s));
+        bitmap_mark_kernel<<<item_blocks, 256, 0, s>>>(w.keys, items, cp, w.bitmap);
+        LAT_CUDA_TRY(cudaGetLastError());
+        const unsigned gblocks = unsigned((ngroups + 255) / 256);
+        bitmap_count_kernel<<<gblocks, 256, 0, s>>>(w.bitmap, ngroups, w.grp_cnt);
+        LAT_CUDA_TRY(cudaGetLastError());
+        size_t sb = w.scan_bytes;
+        LAT_CUDA_TRY(cub::DeviceScan::ExclusiveSum(w.scan_tmp, sb, w.grp_cnt, w.grp_off, int(ngroups), s));
+        bitmap_emit_kernel<<<gblocks, 256, 0, s>>>(w.bitmap, ngroups, w.grp_cnt, w.grp_off, cp,
+                                                   reinterpret_cast<int4 *>(out_coords), out_capacity, w.n_out_dev);
+        LAT_CUDA_TRY(cudaGetLastError());
+        if (parent) {
+            bitmap_parent_kernel<<<in_blocks, 256, 0, s>>>(w.keys, n_in, cp, w.bitmap, w.grp_off, parent);
+            LAT_CUDA_TRY(cudaGetLastError());
+        }
+    } else {
+        // ------------------------------------------------ radix sort + unique of the packed keys
+        size_t b = w.sort_bytes;
+        LAT_CUDA_TRY(cub::DeviceRadixSort::SortKeys(w.sort_tmp, b, w.keys, w.sorted, int(items), 0, 64, s));
+        b = w.sel_bytes;
+        LAT_CUDA_TRY(cub::DeviceSelect::Unique(w.sel_tmp, b, w.sorted, w.uniq, w.n_uniq, int(items), s));
+        down_unpack_kernel<<<item_blocks, 256, 0, s>>>(w.uniq, w.n_uniq, reinterpret_cast<int4 *>(out_coords),
+                                                       out_capacity, w.n_out_dev);
+        LAT_CUDA_TRY(cudaGetLastError());
+        if (parent) {
+            sorted_parent_kernel<<<in_blocks, 256, 0, s>>>(w.keys, n_in, w.uniq, w.n_out_dev, parent);
+            LAT_CUDA_TRY(cudaGetLastError());
+        }
+    }
     int64_t m = 0;
     LAT_CUDA_TRY(cudaMemcpyAsync(&m, w.n_out_dev, sizeof(int64_t), cudaMemcpyDeviceToHost, s));
     LAT_CUDA_TRY(cudaStreamSynchronize(s));

@@ -49,6 +49,7 @@ extern "C" size_t lat_hash_bytes(int64_t n, float rsv_ratio) {
     double want = double(rsv_ratio) * double(n);
     uint64_t cap = 64;
     while (double(cap) < want) cap <<= 1;
+    if (cap > (uint64_t(1) << 31)) return 0;  // slot indices are 32-bit in the query kernels
     return size_t(cap) * sizeof(lat::Slot);
 }
 
@@ -56,7 +57,8 @@ extern "C" lat_status lat_hash_build(const int32_t *coords, int64_t n, void *tab
                                      int32_t *d_status, lat_stream stream) {
     using namespace lat;
     if (n < 0 || n >= (int64_t(1) << 31) || (n > 0 && !coords) || !table) return LAT_ERR_ARG;
-    if (table_bytes % sizeof(Slot) || !pow2(table_bytes / sizeof(Slot)) || table_bytes / sizeof(Slot) < 64)
+    if (table_bytes % sizeof(Slot) || !pow2(table_bytes / sizeof(Slot)) || table_bytes / sizeof(Slot) < 64 ||
+        table_bytes / sizeof(Slot) > (uint64_t(1) << 31))
         return LAT_ERR_ARG;
     if (reinterpret_cast<uintptr_t>(coords) % 16 || reinterpret_cast<uintptr_t>(table) % 16) return LAT_ERR_ARG;
     const uint64_t cap = table_bytes / sizeof(Slot);

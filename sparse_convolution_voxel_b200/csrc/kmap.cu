@@ -7,8 +7,8 @@
 //   1. probe:  one thread per output row, K^3 probes of the input table;
 //              writes nbr (offset-major, coalesced), mask, and per (offset,
 //              block) hit counts from warp ballots.
-//   2. scan:   one block turns the counts into pair offsets (offset-major,
-//              so pairs come out grouped by offset, rows ascending).
+//   2. scan:   one block per offset turns its per-block counts into offsets
+//              (pairs come out grouped by offset, rows ascending).
 //   3. emit:   re-reads nbr and writes (in, out) pairs at ballot-ranked
 //              positions: deterministic, no atomics.
 //   4. sort:   stable radix sort of output rows by mask -> perm.
@@ -26,7 +26,10 @@ struct Geom {
     int ks[3], st[3], pd[3];
     int mode;
     int k3;
+    signed char off[32][3];  // (ix, iy, iz) of offset k
 };
+
+constexpr int kProbeBatch = 8;  // slot loads a thread keeps in flight
 
 // Input coordinate probed by output row c at offset (ix, iy, iz); false if none.
 __device__ __forceinline__ bool query_coord(const Geom &g, const int4 &c, int ix, int iy, int iz, uint64_t &key) {
@@ -47,6 +50,12 @@ __device__ __forceinline__ bool query_coord(const Geom &g, const int4 &c, int ix
     return pack_key(c.x, p[0], p[1], p[2], key);
 }
 
+// One thread per output row.  Offsets are probed in batches of kProbeBatch:
+// each round loads the current slot of every still-unresolved offset of the
+// batch at once (one 16-byte load per slot), then resolves what it can, so a
+// thread keeps several independent loads in flight instead of walking the
+// probe sequences one after another.  Rounds are bounded by the slot count.
+// For a submanifold map the centre offset is the row itself and is not probed.
 __global__ void __launch_bounds__(kQueryThreads)
 kmap_probe_kernel(const Slot *__restrict__ slots, uint64_t cap_mask, const int4 *__restrict__ out_coords,
                   int64_t n_out, int64_t n_in, Geom g, int32_t *__restrict__ nbr, uint32_t *__restrict__ mask,
@@ -58,21 +67,64 @@ kmap_probe_kernel(const Slot *__restrict__ slots, uint64_t cap_mask, const int4 
     const bool live = j < n_out;
     int4 c = make_int4(0, 0, 0, 0);
     if (live) c = __ldg(out_coords + j);
+    const int centre = g.mode == LAT_SUBM ? g.k3 / 2 : -1;
     uint32_t m = 0;
     int32_t bad = 0;
-    int k = 0;
-    for (int ix = 0; ix < g.ks[0]; ++ix)
-        for (int iy = 0; iy < g.ks[1]; ++iy)
-            for (int iz = 0; iz < g.ks[2]; ++iz, ++k) {
-                int row = -1;
-                uint64_t key;
-                if (live && query_coord(g, c, ix, iy, iz, key)) row = hash_find(slots, cap_mask, key);
-                if (row >= n_in) { bad |= LAT_ERR_BAD_MAP; row = -1; }
-                if (live) nbr[int64_t(k) * n_out + j] = row;
-                const unsigned hits = __ballot_sync(0xFFFFFFFFu, row >= 0);
-                if (row >= 0) m |= 1u << k;
-                if ((threadIdx.x & 31) == 0 && hits) atomicAdd(&s_cnt[k], __popc(hits));
+    for (int k0 = 0; k0 < g.k3; k0 += kProbeBatch) {
+        uint64_t key[kProbeBatch];
+        uint32_t slot[kProbeBatch];  // slot counts are below 2^31 (lat_hash_bytes)
+        int row[kProbeBatch];
+        uint32_t pending = 0;
+#pragma unroll
+        for (int e = 0; e < kProbeBatch; ++e) {
+            const int k = k0 + e;
+            row[e] = -1;
+            key[e] = kEmptyKey;
+            slot[e] = 0;
+            if (!live || k >= g.k3) continue;
+            if (k == centre) {
+                row[e] = int(j);
+            } else if (query_coord(g, c, g.off[k][0], g.off[k][1], g.off[k][2], key[e])) {
+                slot[e] = uint32_t(mix64(key[e]) & cap_mask);
+                pending |= 1u << e;
             }
+        }
+        for (uint64_t round = 0; pending && round <= cap_mask; ++round) {
+            unsigned long long kv[kProbeBatch];
+            uint32_t rv[kProbeBatch];
+#pragma unroll
+            for (int e = 0; e < kProbeBatch; ++e) {
+                if (pending & (1u << e)) {
+                    const ulonglong2 v = __ldg(reinterpret_cast<const ulonglong2 *>(slots + slot[e]));
+                    kv[e] = v.x;
+                    rv[e] = uint32_t(v.y);
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < kProbeBatch; ++e) {
+                if (!(pending & (1u << e))) continue;
+                if (kv[e] == key[e]) {
+                    row[e] = int(rv[e]);
+                    pending &= ~(1u << e);
+                } else if (kv[e] == kEmptyKey) {
+                    pending &= ~(1u << e);
+                } else {
+                    slot[e] = uint32_t((slot[e] + 1) & cap_mask);
+                }
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < kProbeBatch; ++e) {
+            const int k = k0 + e;
+            if (k >= g.k3) break;
+            int r = row[e];
+            if (r >= n_in) { bad |= LAT_ERR_BAD_MAP; r = -1; }
+            if (live) nbr[int64_t(k) * n_out + j] = r;
+            const unsigned hits = __ballot_sync(0xFFFFFFFFu, r >= 0);
+            if (r >= 0) m |= 1u << k;
+            if ((threadIdx.x & 31) == 0 && hits) atomicAdd(&s_cnt[k], __popc(hits));
+        }
+    }
     if (live) {
         mask[j] = m;
         iota[j] = int32_t(j);
@@ -82,38 +134,66 @@ kmap_probe_kernel(const Slot *__restrict__ slots, uint64_t cap_mask, const int4 
     if (threadIdx.x < g.k3) block_counts[int64_t(threadIdx.x) * nblk + blockIdx.x] = s_cnt[threadIdx.x];
 }
 
-// Exclusive scan of block_counts (k-major) -> block_offsets; pair_off[k] = start of offset k.
+// Exclusive scan of the per-block hit counts of one offset (block k scans row k of
+// block_counts) -> block_offsets relative to the offset's first pair, and the
+// offset's total pair count.
 __global__ void __launch_bounds__(1024)
-kmap_scan_kernel(const int32_t *__restrict__ block_counts, int64_t *__restrict__ block_offsets, int64_t len,
-                 int nblk, int k3, int64_t *__restrict__ pair_off) {
-    __shared__ int64_t s_part[1024];
-    const int t = threadIdx.x;
-    const int64_t per = (len + 1023) / 1024;
-    const int64_t lo = min(len, t * per), hi = min(len, lo + per);
-    int64_t sum = 0;
-    for (int64_t e = lo; e < hi; ++e) sum += block_counts[e];
-    s_part[t] = sum;
+kmap_scan_kernel(const int32_t *__restrict__ block_counts, int64_t *__restrict__ block_offsets, int nblk,
+                 int64_t *__restrict__ k_total) {
+    __shared__ int64_t s_warp[32];
+    __shared__ int64_t s_carry;
+    const int k = blockIdx.x;
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const int32_t *row = block_counts + int64_t(k) * nblk;
+    int64_t *orow = block_offsets + int64_t(k) * nblk;
+    if (t == 0) s_carry = 0;
     __syncthreads();
-    for (int d = 1; d < 1024; d <<= 1) {  // Hillis-Steele inclusive scan
-        int64_t v = t >= d ? s_part[t - d] : 0;
+    for (int base = 0; base < nblk; base += 1024) {
+        const int e = base + t;
+        const int64_t v = e < nblk ? row[e] : 0;
+        int64_t incl = v;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int64_t o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+            if (lane >= d) incl += o;
+        }
+        if (lane == 31) s_warp[w] = incl;
         __syncthreads();
-        s_part[t] += v;
+        if (w == 0) {
+            int64_t ws = s_warp[lane];
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int64_t o = __shfl_up_sync(0xFFFFFFFFu, ws, d);
+                if (lane >= d) ws += o;
+            }
+            s_warp[lane] = ws;
+        }
+        __syncthreads();
+        const int64_t excl = s_carry + (w ? s_warp[w - 1] : 0) + incl - v;
+        if (e < nblk) orow[e] = excl;
+        __syncthreads();
+        if (t == 1023) s_carry = excl + v;
         __syncthreads();
     }
-    int64_t run = s_part[t] - sum;
-    for (int64_t e = lo; e < hi; ++e) {
-        block_offsets[e] = run;
-        if (e % nblk == 0) pair_off[e / nblk] = run;
-        run += block_counts[e];
-    }
-    if (t == 1023) pair_off[k3] = s_part[1023];
+    if (t == 0) k_total[k] = s_carry;
 }
 
 __global__ void __launch_bounds__(kQueryThreads)
 kmap_emit_kernel(const int32_t *__restrict__ nbr, int64_t n_out, int k3, const int64_t *__restrict__ block_offsets,
-                 int nblk, int32_t *__restrict__ pair_in, int32_t *__restrict__ pair_out, int64_t capacity,
-                 int32_t *d_status) {
+                 const int64_t *__restrict__ k_total, int nblk, int32_t *__restrict__ pair_in,
+                 int32_t *__restrict__ pair_out, int64_t capacity, int64_t *__restrict__ pair_off, int32_t *d_status) {
     __shared__ int s_warp[32][kQueryWarps];
+    __shared__ int64_t s_kstart[33];
+    if (threadIdx.x == 0) {
+        int64_t run = 0;
+        for (int k = 0; k < k3; ++k) {
+            s_kstart[k] = run;
+            run += k_total[k];
+        }
+        s_kstart[k3] = run;
+        if (blockIdx.x == 0)
+            for (int k = 0; k <= k3; ++k) pair_off[k] = s_kstart[k];
+    }
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t j = blockIdx.x * int64_t(kQueryThreads) + threadIdx.x;
     const bool live = j < n_out;
@@ -128,7 +208,7 @@ kmap_emit_kernel(const int32_t *__restrict__ nbr, int64_t n_out, int k3, const i
         const int row = live ? nbr[int64_t(k) * n_out + j] : -1;
         const unsigned hits = __ballot_sync(0xFFFFFFFFu, row >= 0);
         if (row < 0) continue;
-        int64_t pos = block_offsets[int64_t(k) * nblk + blockIdx.x];
+        int64_t pos = s_kstart[k] + block_offsets[int64_t(k) * nblk + blockIdx.x];
         for (int w = 0; w < warp; ++w) pos += s_warp[k][w];
         pos += __popc(hits & ((1u << lane) - 1u));
         if (pos < capacity) {
@@ -155,9 +235,58 @@ __global__ void tile_mask_kernel(const uint32_t *__restrict__ sorted_mask, int64
     if (lane == 0) tile_mask[t] = m;
 }
 
+// Per-(offset, block) hit counts of a neighbour table that was filled without
+// probing (maps built from parent indices); also writes the identity row order.
+__global__ void __launch_bounds__(kQueryThreads)
+kmap_count_kernel(const int32_t *__restrict__ nbr, int64_t n_out, int k3, int32_t *__restrict__ iota,
+                  int32_t *__restrict__ block_counts, int nblk) {
+    __shared__ int s_cnt[32];
+    if (threadIdx.x < 32) s_cnt[threadIdx.x] = 0;
+    __syncthreads();
+    const int64_t j = blockIdx.x * int64_t(kQueryThreads) + threadIdx.x;
+    const bool live = j < n_out;
+    for (int k = 0; k < k3; ++k) {
+        const int row = live ? nbr[int64_t(k) * n_out + j] : -1;
+        const unsigned hits = __ballot_sync(0xFFFFFFFFu, row >= 0);
+        if ((threadIdx.x & 31) == 0 && hits) atomicAdd(&s_cnt[k], __popc(hits));
+    }
+    if (live) iota[j] = int32_t(j);
+    __syncthreads();
+    if (threadIdx.x < k3) block_counts[int64_t(threadIdx.x) * nblk + blockIdx.x] = s_cnt[threadIdx.x];
+}
+
+// Kernel size == stride, no padding: fine row i lies in exactly one coarse window,
+// parent[i], at offset k(i) = its position inside the window (floor modulo the
+// stride per axis).  Writes the transposed map's rows directly (one neighbour per
+// fine row) and scatters the strided map's entries (the down table must hold -1
+// and the down mask 0 beforehand).
+__global__ void __launch_bounds__(256)
+parent_maps_kernel(const int4 *__restrict__ fine, const int32_t *__restrict__ parent, int64_t n_fine,
+                   int64_t n_coarse, int s0, int s1, int s2, int k3, int32_t *__restrict__ up_nbr,
+                   uint32_t *__restrict__ up_mask, int32_t *__restrict__ down_nbr, uint32_t *__restrict__ down_mask,
+                   int32_t *d_status) {
+    const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+    if (i >= n_fine) return;
+    const int4 c = __ldg(fine + i);
+    const int q = __ldg(parent + i);
+    const int o0 = c.y - floordiv(c.y, s0) * s0, o1 = c.z - floordiv(c.z, s1) * s1, o2 = c.w - floordiv(c.w, s2) * s2;
+    const int k = (o0 * s1 + o1) * s2 + o2;
+    const bool ok = q >= 0 && q < n_coarse;
+    if (!ok) flag(d_status, LAT_ERR_BAD_MAP);
+    if (up_nbr) {
+        for (int kk = 0; kk < k3; ++kk) up_nbr[int64_t(kk) * n_fine + i] = (ok && kk == k) ? q : -1;
+        up_mask[i] = ok ? (1u << k) : 0u;
+    }
+    if (down_nbr && ok) {
+        down_nbr[int64_t(k) * n_coarse + q] = int32_t(i);
+        atomicOr(down_mask + q, 1u << k);
+    }
+}
+
 struct KmapWs {
     int32_t *block_counts;
     int64_t *block_offsets;
+    int64_t *k_total;
     int32_t *iota;
     uint32_t *sorted_mask;
     void *cub_tmp;
@@ -171,6 +300,7 @@ static KmapWs carve_kmap_ws(void *base, int64_t n_out, int k3) {
     Carver cv(base);
     w.block_counts = cv.take<int32_t>(size_t(k3) * nblk);
     w.block_offsets = cv.take<int64_t>(size_t(k3) * nblk);
+    w.k_total = cv.take<int64_t>(size_t(k3));
     w.iota = cv.take<int32_t>(size_t(n_out));
     w.sorted_mask = cv.take<uint32_t>(size_t(n_out));
     size_t cub_bytes = 0;
@@ -180,6 +310,33 @@ static KmapWs carve_kmap_ws(void *base, int64_t n_out, int k3) {
     w.cub_tmp = cv.take<char>(cub_bytes);
     w.total = align_up(cv.used, 256);
     return w;
+}
+
+// Scan the per-block counts, emit the pair lists, sort rows by mask and OR the tile masks.
+static lat_status finish_kmap(lat_kmap *map, int k3, int nblk, KmapWs &w, int32_t *d_status, cudaStream_t s) {
+    const int64_t n_out = map->n_out;
+    kmap_scan_kernel<<<k3, 1024, 0, s>>>(w.block_counts, w.block_offsets, nblk, w.k_total);
+    LAT_CUDA_TRY(cudaGetLastError());
+    kmap_emit_kernel<<<nblk, kQueryThreads, 0, s>>>(map->nbr, n_out, k3, w.block_offsets, w.k_total, nblk,
+                                                     map->pair_in, map->pair_out, map->pair_capacity, map->pair_off,
+                                                     d_status);
+    LAT_CUDA_TRY(cudaGetLastError());
+    size_t cub_bytes = w.cub_bytes;
+    LAT_CUDA_TRY(cub::DeviceRadixSort::SortPairs(w.cub_tmp, cub_bytes, map->mask, w.sorted_mask, w.iota, map->perm,
+                                                 int(n_out), 0, k3, s));
+    const int64_t ntiles = (n_out + LAT_TILE_ROWS - 1) / LAT_TILE_ROWS;
+    tile_mask_kernel<<<unsigned((ntiles + 7) / 8), 256, 0, s>>>(w.sorted_mask, n_out, map->tile_mask, ntiles);
+    LAT_CUDA_TRY(cudaGetLastError());
+    return LAT_OK;
+}
+
+static bool map_buffers_ok(const lat_kmap *map) {
+    if (!map || map->n_out < 0 || map->n_out >= (int64_t(1) << 31) || map->n_in < 0 ||
+        map->n_in >= (int64_t(1) << 31) || map->pair_capacity < 0 || !map->pair_off)
+        return false;
+    if (map->n_out > 0 && (!map->nbr || !map->mask || !map->perm || !map->tile_mask)) return false;
+    if (map->pair_capacity > 0 && (!map->pair_in || !map->pair_out)) return false;
+    return true;
 }
 
 bool geom_ok(const lat_geom *g, int &k3) {
@@ -211,13 +368,12 @@ extern "C" lat_status lat_kmap_query(const void *table, size_t table_bytes, cons
                                      int32_t *d_status, lat_stream stream) {
     using namespace lat;
     int k3 = 0;
-    if (!map || !geom_ok(geom, k3) || map->k3 != k3) return LAT_ERR_ARG;
+    if (!map || !geom_ok(geom, k3) || map->k3 != k3 || !map_buffers_ok(map)) return LAT_ERR_ARG;
     const int64_t n_out = map->n_out, n_in = map->n_in;
-    if (n_out < 0 || n_out >= (int64_t(1) << 31) || n_in < 0 || n_in >= (int64_t(1) << 31)) return LAT_ERR_ARG;
-    if (!table || table_bytes % sizeof(Slot) || !pow2(table_bytes / sizeof(Slot))) return LAT_ERR_ARG;
-    if (map->pair_capacity < 0 || !map->pair_off) return LAT_ERR_ARG;
-    if (n_out > 0 && (!out_coords || !map->nbr || !map->mask || !map->perm || !map->tile_mask)) return LAT_ERR_ARG;
-    if (map->pair_capacity > 0 && (!map->pair_in || !map->pair_out)) return LAT_ERR_ARG;
+    if (!table || table_bytes % sizeof(Slot) || !pow2(table_bytes / sizeof(Slot)) ||
+        table_bytes / sizeof(Slot) > (uint64_t(1) << 31))
+        return LAT_ERR_ARG;
+    if (n_out > 0 && !out_coords) return LAT_ERR_ARG;
     if (reinterpret_cast<uintptr_t>(out_coords) % 16 || reinterpret_cast<uintptr_t>(table) % 16) return LAT_ERR_ARG;
     const KmapWs need = carve_kmap_ws(nullptr, n_out, k3);
     if (ws_bytes < need.total || (need.total && !ws)) return LAT_ERR_WORKSPACE;
@@ -236,22 +392,74 @@ extern "C" lat_status lat_kmap_query(const void *table, size_t table_bytes, cons
     }
     g.mode = geom->mode;
     g.k3 = k3;
+    for (int ix = 0, k = 0; ix < g.ks[0]; ++ix)
+        for (int iy = 0; iy < g.ks[1]; ++iy)
+            for (int iz = 0; iz < g.ks[2]; ++iz, ++k) {
+                g.off[k][0] = static_cast<signed char>(ix);
+                g.off[k][1] = static_cast<signed char>(iy);
+                g.off[k][2] = static_cast<signed char>(iz);
+            }
     const int nblk = int((n_out + kQueryThreads - 1) / kQueryThreads);
     const uint64_t cap_mask = table_bytes / sizeof(Slot) - 1;
     kmap_probe_kernel<<<nblk, kQueryThreads, 0, s>>>(static_cast<const Slot *>(table), cap_mask,
                                                       reinterpret_cast<const int4 *>(out_coords), n_out, n_in, g,
                                                       map->nbr, map->mask, w.iota, w.block_counts, nblk, d_status);
     LAT_CUDA_TRY(cudaGetLastError());
-    kmap_scan_kernel<<<1, 1024, 0, s>>>(w.block_counts, w.block_offsets, int64_t(k3) * nblk, nblk, k3, map->pair_off);
-    LAT_CUDA_TRY(cudaGetLastError());
-    kmap_emit_kernel<<<nblk, kQueryThreads, 0, s>>>(map->nbr, n_out, k3, w.block_offsets, nblk, map->pair_in,
-                                                     map->pair_out, map->pair_capacity, d_status);
-    LAT_CUDA_TRY(cudaGetLastError());
-    size_t cub_bytes = w.cub_bytes;
-    LAT_CUDA_TRY(cub::DeviceRadixSort::SortPairs(w.cub_tmp, cub_bytes, map->mask, w.sorted_mask, w.iota, map->perm,
-                                                 int(n_out), 0, k3, s));
-    const int64_t ntiles = (n_out + LAT_TILE_ROWS - 1) / LAT_TILE_ROWS;
-    tile_mask_kernel<<<unsigned((ntiles + 7) / 8), 256, 0, s>>>(w.sorted_mask, n_out, map->tile_mask, ntiles);
-    LAT_CUDA_TRY(cudaGetLastError());
+    return finish_kmap(map, k3, nblk, w, d_status, s);
+}
+
+extern "C" size_t lat_kmap_from_parent_ws_bytes(int64_t n_fine, int64_t n_coarse, int32_t k3) {
+    if (n_fine < 0 || n_coarse < 0 || n_fine >= (int64_t(1) << 31) || k3 < 1 || k3 > 32) return 0;
+    const int64_t n = n_fine > n_coarse ? n_fine : n_coarse;
+    return lat::carve_kmap_ws(nullptr, n, k3).total;
+}
+
+extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int32_t *parent, const lat_geom *geom,
+                                           lat_kmap *down, lat_kmap *up, void *ws, size_t ws_bytes,
+                                           int32_t *d_status, lat_stream stream) {
+    using namespace lat;
+    int k3 = 0;
+    if (!geom_ok(geom, k3) || geom->mode != LAT_STRIDED) return LAT_ERR_ARG;
+    for (int a = 0; a < 3; ++a)
+        if (geom->ksize[a] != geom->stride[a] || geom->pad[a] != 0) return LAT_ERR_UNSUPPORTED;
+    if (!down && !up) return LAT_ERR_ARG;
+    if ((down && (!map_buffers_ok(down) || down->k3 != k3)) || (up && (!map_buffers_ok(up) || up->k3 != k3)))
+        return LAT_ERR_ARG;
+    const int64_t n_fine = up ? up->n_out : down->n_in;
+    const int64_t n_coarse = up ? up->n_in : down->n_out;
+    if (down && up && (down->n_in != n_fine || down->n_out != n_coarse)) return LAT_ERR_ARG;
+    if (n_fine > 0 && (!fine_coords || !parent)) return LAT_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(fine_coords) % 16) return LAT_ERR_ARG;
+    const size_t need = lat_kmap_from_parent_ws_bytes(n_fine, n_coarse, k3);
+    if (ws_bytes < need || (need && !ws)) return LAT_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (down) {
+        down->mode = LAT_STRIDED;
+        if (n_coarse > 0) {
+            LAT_CUDA_TRY(cudaMemsetAsync(down->nbr, 0xFF, sizeof(int32_t) * size_t(k3) * n_coarse, s));
+            LAT_CUDA_TRY(cudaMemsetAsync(down->mask, 0, sizeof(uint32_t) * size_t(n_coarse), s));
+        }
+    }
+    if (up) up->mode = LAT_TRANSPOSED;
+    if (n_fine > 0) {
+        parent_maps_kernel<<<unsigned((n_fine + 255) / 256), 256, 0, s>>>(
+            reinterpret_cast<const int4 *>(fine_coords), parent, n_fine, n_coarse, geom->stride[0], geom->stride[1],
+            geom->stride[2], k3, up ? up->nbr : nullptr, up ? up->mask : nullptr, down ? down->nbr : nullptr,
+            down ? down->mask : nullptr, d_status);
+        LAT_CUDA_TRY(cudaGetLastError());
+    }
+    for (lat_kmap *map : {down, up}) {
+        if (!map) continue;
+        if (map->n_out == 0) {
+            LAT_CUDA_TRY(cudaMemsetAsync(map->pair_off, 0, sizeof(int64_t) * (k3 + 1), s));
+            continue;
+        }
+        KmapWs w = carve_kmap_ws(ws, map->n_out, k3);
+        const int nblk = int((map->n_out + kQueryThreads - 1) / kQueryThreads);
+        kmap_count_kernel<<<nblk, kQueryThreads, 0, s>>>(map->nbr, map->n_out, k3, w.iota, w.block_counts, nblk);
+        LAT_CUDA_TRY(cudaGetLastError());
+        const lat_status st = finish_kmap(map, k3, nblk, w, d_status, s);
+        if (st != LAT_OK) return st;
+    }
     return LAT_OK;
 }

@@ -23,8 +23,6 @@ constexpr int kChunk = 2048;       // pairs per work unit
 constexpr int kProdWarps = 4, kEpiWarps = 4;
 constexpr int kMmaWarp = kProdWarps + kEpiWarps;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
-constexpr int kLag = 3;
-constexpr int kStages = 6;
 constexpr uint64_t kWaitNs = 2000000000ull;
 
 template <int M, int N>
@@ -32,11 +30,16 @@ struct Cfg {
     static constexpr uint32_t kABytes = uint32_t(M) * 128;  // 64 pairs x M channels x 2 bytes
     static constexpr uint32_t kBBytes = uint32_t(N) * 128;
     static constexpr uint32_t kStage = kABytes + kBBytes;
+    // about 96 KB of stages so that two CTAs share an SM
+    static constexpr int kStages = kStage <= 16384 ? 6 : (kStage <= 24576 ? 4 : 3);
+    static constexpr int kLag = kStages - 1 < 3 ? kStages - 1 : 3;  // cp.async groups in flight per thread
     static constexpr uint32_t kSmem = kStages * kStage + 256 + 1024;
     static constexpr uint32_t kTmemCols = 2 * N;
 };
 
 template <typename T> constexpr bool is_bf16() { return !std::is_same<T, __half>::value; }
+
+template <typename T, int M, int N> struct KernelTag {};  // one launch-config cache per kernel
 
 // kind::f16, fp32 D, A and B MN-major, M x N
 template <typename T, int M, int N>
@@ -56,13 +59,14 @@ __device__ __forceinline__ void unit_range(const int32_t *unit_base, const int64
 }
 
 template <typename T, int M, int N>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t *__restrict__ pair_off,
                 const int32_t *__restrict__ pair_in, const int32_t *__restrict__ pair_out, int64_t capacity, int k3,
                 int64_t n_in, int64_t n_out, const int32_t *__restrict__ unit_base, float *__restrict__ partial,
                 int32_t *d_status) {
     using C = Cfg<M, N>;
-    constexpr int NS = kStages;
+    constexpr int NS = C::kStages;
+    constexpr int kLag = C::kLag;
     constexpr uint32_t idesc = make_idesc<T, M, N>();
 
     extern __shared__ uint8_t smem_raw[];
@@ -108,20 +112,26 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
             int k;
             int64_t lo, hi;
             unit_range(unit_base, pair_off, capacity, k3, u, k, lo, hi);
-            for (int64_t p0 = lo; p0 < hi; p0 += kKP) {
-                // lanes 0..15 fetch the indices of this warp's 16 pairs
+            // lanes 0..15 fetch the indices of this warp's 16 pairs of a block, one block ahead
+            auto fetch = [&](int64_t p0, int &si, int &sj) {
                 const int64_t mp = p0 + warp * 16 + (lane & 15);
-                int si = -1, sj = -1;
+                si = sj = -1;
                 if (lane < 16 && mp < hi) {
                     si = __ldg(pair_in + mp);
                     sj = __ldg(pair_out + mp);
-                    if (si < 0 || si >= n_in || sj < 0 || sj >= n_out) {
-                        bad |= LAT_ERR_BAD_MAP;
-                        si = sj = -1;
-                    }
+                }
+            };
+            int si_n, sj_n;
+            fetch(lo, si_n, sj_n);
+            for (int64_t p0 = lo; p0 < hi; p0 += kKP) {
+                int si = si_n, sj = sj_n;
+                if (p0 + kKP < hi) fetch(p0 + kKP, si_n, sj_n);
+                if (si >= n_in || sj >= n_out || (si < 0) != (sj < 0)) {
+                    bad |= LAT_ERR_BAD_MAP;
+                    si = sj = -1;
                 }
                 const uint32_t s = it % NS;
-                if (!ptx::mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, kWaitNs)) {
+                if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, kWaitNs))) {
                     ok = false;
                     break;
                 }
@@ -177,7 +187,7 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
                 continue;
             }
             const uint32_t a = ta & 1;
-            if (!ptx::mbar_wait(&accfull[a], (ta >> 1) & 1, kWaitNs)) {
+            if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(&accfull[a], (ta >> 1) & 1, kWaitNs))) {
                 ok = false;
                 break;
             }
@@ -300,8 +310,8 @@ static lat_status launch(const void *x, const void *dy, const lat_kmap *map, flo
     wgrad_tc_units_kernel<<<1, 32, 0, s>>>(map->pair_off, map->k3, map->pair_capacity, unit_base);
     LAT_CUDA_TRY(cudaGetLastError());
     auto kern = wgrad_tc_kernel<T, M, N>;
-    LAT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::kSmem)));
-    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(units_max, num_sms()));
+    const int64_t grid = std::min<int64_t>(units_max, GridCache<KernelTag<T, M, N>>::get(kern, C::kSmem, int(C::kTmemCols), 2));
+    if (grid <= 0) return LAT_ERR_CUDA;
     kern<<<unsigned(grid), kThreads, C::kSmem, s>>>(static_cast<const T *>(x), static_cast<const T *>(dy),
                                                     map->pair_off, map->pair_in, map->pair_out, map->pair_capacity,
                                                     map->k3, map->n_in, map->n_out, unit_base, partial, d_status);

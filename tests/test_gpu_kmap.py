@@ -176,3 +176,47 @@ def test_downsample_capacity_error():
     coords = rand_coords(rng, 300, 0, 20)
     with pytest.raises(scv.LatticeError):
         scv.downsample(_dev(coords), scv.strided_geom(2, 2, 0), capacity=10)
+
+
+# --------------------------------------------------------------------------- parents and maps from parents
+@pytest.mark.parametrize("lo,hi", [(-10, 10), (-30000, 30000)])   # bitmap counting sort / radix sort path
+def test_downsample_parent_and_maps_from_parent(lo, hi):
+    rng = np.random.default_rng(abs(lo))
+    if hi - lo > 100:
+        coords = np.unique(rng.integers(lo, hi, (3000, 4)).astype(np.int32), axis=0)
+        coords[:, 0] = rng.integers(0, 3, len(coords))
+        coords = np.unique(coords, axis=0)
+        coords = coords[rng.permutation(len(coords))]
+    else:
+        coords = rand_coords(rng, 1500, lo, hi, 3)
+    c = _dev(coords)
+    g = scv.strided_geom(2, 2, 0)
+    st = scv.new_status()
+    coarse, parent = scv.downsample(c, g, d_status=st, with_parent=True)
+    ref = oracle.downsample(coords, 2, 2, 0)
+    assert np.array_equal(coarse.cpu().numpy(), ref)
+    par = parent.cpu().numpy()
+    assert np.array_equal(ref[par][:, 1:], np.floor_divide(coords[:, 1:], 2))
+    assert np.array_equal(ref[par][:, 0], coords[:, 0])
+    down, up = scv.maps_from_parent(c, parent, len(ref), g, d_status=st)
+    scv.check_status(st)
+    check_kmap(down, oracle.kmap(coords, ref, 2, 2, 0, oracle.STRIDED))
+    check_kmap(up, oracle.kmap(ref, coords, 2, 2, 0, oracle.TRANSPOSED))
+
+
+def test_maps_from_parent_full_workload():
+    coords = synthetic.WORKLOADS["lidar_down_up"].coords()
+    c = _dev(coords)
+    g = scv.strided_geom(2, 2, 0)
+    coarse, parent = scv.downsample(c, g, with_parent=True)
+    ref = oracle.downsample(coords, 2, 2, 0)
+    assert np.array_equal(coarse.cpu().numpy(), ref)
+    down, up = scv.maps_from_parent(c, parent, len(ref), g)
+    check_kmap(down, oracle.kmap(coords, ref, 2, 2, 0, oracle.STRIDED))
+    check_kmap(up, oracle.kmap(ref, coords, 2, 2, 0, oracle.TRANSPOSED))
+
+
+def test_downsample_parent_needs_kernel_equal_stride():
+    coords = rand_coords(np.random.default_rng(0), 100, 0, 8)
+    with pytest.raises(scv.LatticeError):
+        scv.downsample(_dev(coords), scv.strided_geom(3, 2, 1), with_parent=True)
