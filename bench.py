@@ -56,10 +56,28 @@ def load_peaks():
     return 6650.0, 1590.0, "fallback"
 
 
+# --------------------------------------------------------------------------- multi-rank helpers
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Every rank draws its own batch (weak scaling: per-rank work is fixed)."""
+    return base_seed + 1000 * rank
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """The slowest rank's time: all ranks report, the max is the job's time."""
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(flops_per_rank: float, world: int, steps: int, total_ms: float) -> float:
+    """Whole-job effective TFLOP/s: the work of all ranks over the max-over-ranks time."""
+    return flops_per_rank * world * steps / (total_ms * 1e-3) / 1e12
+
+
 # --------------------------------------------------------------------------- inputs
 def make_inputs(rank: int):
     wl = synthetic.WORKLOADS[WORKLOAD]
-    seed = wl.seed + 1000 * rank
+    seed = rank_seed(wl.seed, rank)
     coords = synthetic.lidar(seed=seed, **wl.gen_args)
     n = len(coords)
     x = torch.from_numpy(synthetic.features(n, CIN, seed)).half()
@@ -459,11 +477,9 @@ def main():
     phase_ms = {p: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, p in enumerate(Pipeline.PHASES)}
     total_ms = sum(step_ms)
     if pg:
-        t = torch.tensor([total_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms = max_over_ranks(total_ms, pg, dev)
     flops = pipe.flops()
-    value = flops * world * args.steps / (total_ms * 1e-3) / 1e12
+    value = job_throughput(flops, world, args.steps, total_ms)
     kmap_ms = phase_ms["hash"] + phase_ms["kmap"]
 
     # end to end through the public API: host inputs in, results back to the host

@@ -102,8 +102,12 @@ typedef struct {
  * buffers that lat_kmap_query fills:
  *   nbr       int32  [k3][n_out]  nbr[k*n_out + j] = input row, or -1
  *   mask      uint32 [n_out]      bit k set iff nbr[k*n_out + j] >= 0
- *   perm      int32  [n_out]      output rows sorted by mask (stable: ties keep
- *                                 ascending row order)
+ *   perm      int32  [n_out]      output rows sorted by the grouping key
+ *                                 (min(popcount(mask), 31) << 11) |
+ *                                 ((mask * 0x9E3779B1 mod 2^32) >> 21), stable
+ *                                 (ties keep ascending row order); rows with
+ *                                 equal masks are adjacent.  With k3 <= 8
+ *                                 the key is the mask itself.
  *   tile_mask uint32 [ceil(n_out/LAT_TILE_ROWS)]  OR of mask over each run of
  *                                 LAT_TILE_ROWS consecutive entries of perm
  *   pair_off  int64  [k3 + 1]     pair_off[k] = first pair of offset k
@@ -140,8 +144,9 @@ typedef struct {
  * [0, 65534] and x, y, z in [-32768, 32767]; rows outside are skipped and
  * flag LAT_ERR_COORD_RANGE.  The table is an array of 16-byte slots
  * {uint64 key; int32 row; int32 unused} with a power-of-two slot count; an
- * empty slot holds key 0xFFFF...F.  Keys are placed with the SplitMix64
- * output function and linear probing.
+ * empty slot holds key 0xFFFF...F.  A key's home slot is a 32-bit mix of
+ * the key (its two halves folded, then the MurmurHash3 fmix32 finalizer);
+ * collisions are resolved by linear probing.
  */
 
 /* Bytes of a table for n rows: 16 * next_pow2(max(ceil(rsv_ratio*n), 64)).

@@ -53,8 +53,6 @@ def _load():
             P = ctypes.c_void_p
             i64, i32 = ctypes.c_int64, ctypes.c_int
             lib.orc_version.restype = i32
-            lib.orc_splitmix64.restype = ctypes.c_uint64
-            lib.orc_splitmix64.argtypes = [ctypes.c_uint64]
             lib.orc_pack_key.restype = ctypes.c_uint64
             lib.orc_pack_key.argtypes = [ctypes.c_int32] * 4
             lib.orc_kmap.restype = i32
@@ -96,11 +94,6 @@ class OracleError(RuntimeError):
 
 def max_threads() -> int:
     return _load().orc_max_threads()
-
-
-def splitmix64(z: int) -> int:
-    """SplitMix64 output function (Steele, Lea & Flood 2014)."""
-    return int(_load().orc_splitmix64(ctypes.c_uint64(z & 0xFFFFFFFFFFFFFFFF)))
 
 
 def pack_key(b: int, x: int, y: int, z: int) -> int:

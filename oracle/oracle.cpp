@@ -84,17 +84,6 @@ extern "C" {
 
 int orc_version() { return 1; }
 
-// SplitMix64 output function (Steele, Lea, Flood, "Fast splittable
-// pseudorandom number generators", OOPSLA 2014; constants as published by
-// Vigna for splitmix64).  Exposed so tests can check where the GPU hash
-// table placed each key.
-uint64_t orc_splitmix64(uint64_t z) {
-    z += 0x9E3779B97F4A7C15ull;
-    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
-    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
-    return z ^ (z >> 31);
-}
-
 // Packed key of one coordinate row; returns ~0 if out of range.
 uint64_t orc_pack_key(int32_t b, int32_t x, int32_t y, int32_t z) {
     if (!in_range(b, x, y, z)) return ~uint64_t(0);

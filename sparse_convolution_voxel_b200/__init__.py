@@ -25,7 +25,7 @@ from ._lib import (  # noqa: F401  (re-exported C entry points and constants)
 
 __all__ = [
     "KernelMap", "Workspace", "hash_table", "kernel_map", "downsample", "maps_from_parent", "conv_fwd", "conv_dgrad", "conv_wgrad",
-    "subm_geom", "strided_geom", "transposed_geom", "check_status", "new_status",
+    "subm_geom", "strided_geom", "target_geom", "transposed_geom", "check_status", "new_status",
 ] + EXPORTS
 
 
@@ -36,6 +36,12 @@ def subm_geom(ksize=3):
 
 def strided_geom(ksize=2, stride=2, pad=0):
     return make_geom(ksize, stride, pad, LAT_STRIDED)
+
+
+def target_geom(ksize=3):
+    """TargetConv3d: the stride-1 relation evaluated at caller output coordinates."""
+    ks = (ksize,) * 3 if isinstance(ksize, int) else tuple(ksize)
+    return make_geom(ks, 1, tuple((k - 1) // 2 for k in ks), LAT_STRIDED)
 
 
 def transposed_geom(ksize=2, stride=2, pad=0):

@@ -38,20 +38,25 @@ __device__ __forceinline__ void unpack_key(uint64_t key, int4 &c) {
     c.w = int(key & 0xFFFF) - 32768;
 }
 
-// SplitMix64 output function (Steele, Lea & Flood, OOPSLA 2014): a full-avalanche
-// 64-bit mixer, so consecutive voxels land in unrelated slots.
-__device__ __forceinline__ uint64_t mix64(uint64_t z) {
-    z += 0x9E3779B97F4A7C15ull;
-    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
-    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
-    return z ^ (z >> 31);
+// Slot hash of a packed key: fold the two 32-bit halves (the high half scaled by
+// the 32-bit golden-ratio constant), then the MurmurHash3 32-bit finalizer
+// (Austin Appleby, public domain) for full avalanche, so neighbouring voxels land
+// in unrelated slots.  32-bit arithmetic only: the probe kernels are
+// instruction-bound and slot counts are below 2^31.
+__device__ __forceinline__ uint32_t slot_hash(uint64_t key) {
+    uint32_t h = uint32_t(key) ^ (uint32_t(key >> 32) * 0x9E3779B1u);
+    h ^= h >> 16;
+    h *= 0x85EBCA6Bu;
+    h ^= h >> 13;
+    h *= 0xC2B2AE35u;
+    h ^= h >> 16;
+    return h;
 }
 
 // Look a key up; returns the row or -1.  Probing is bounded by the slot count.
-__device__ __forceinline__ int hash_find(const Slot *__restrict__ slots, uint64_t cap_mask,
-                                         uint64_t key) {
-    uint64_t s = mix64(key) & cap_mask;
-    for (uint64_t probe = 0; probe <= cap_mask; ++probe) {
+__device__ __forceinline__ int hash_find(const Slot *__restrict__ slots, uint32_t cap_mask, uint64_t key) {
+    uint32_t s = slot_hash(key) & cap_mask;
+    for (uint32_t probe = 0; probe <= cap_mask; ++probe) {
         const ulonglong2 v = __ldg(reinterpret_cast<const ulonglong2 *>(slots + s));
         if (v.x == key) return int(unsigned(v.y));
         if (v.x == kEmptyKey) return -1;

@@ -82,18 +82,32 @@ down_candidates_kernel(const int4 *__restrict__ coords, int64_t n, DownGeom g, u
                     }
         }
     }
+    // warp, then block reduction: one set of global atomics per block (all blocks
+    // update the same eight words, so per-warp atomics would serialise)
+    __shared__ int s_mn[8][4], s_mx[8][4];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
         for (int o = 16; o; o >>= 1) {
             mn[a] = min(mn[a], __shfl_xor_sync(0xFFFFFFFFu, mn[a], o));
             mx[a] = max(mx[a], __shfl_xor_sync(0xFFFFFFFFu, mx[a], o));
         }
+        if (lane == 0) {
+            s_mn[warp][a] = mn[a];
+            s_mx[warp][a] = mx[a];
+        }
     }
-    if ((threadIdx.x & 31) == 0 && mn[0] != INT_MAX) {
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-            atomicMin(range + a, mn[a]);
-            atomicMax(range + 4 + a, mx[a]);
+    __syncthreads();
+    if (threadIdx.x < 4) {
+        const int a = threadIdx.x;
+        int bmn = INT_MAX, bmx = INT_MIN;
+        for (int w = 0; w < int(blockDim.x >> 5); ++w) {
+            bmn = min(bmn, s_mn[w][a]);
+            bmx = max(bmx, s_mx[w][a]);
+        }
+        if (bmn != INT_MAX) {
+            atomicMin(range + a, bmn);
+            atomicMax(range + 4 + a, bmx);
         }
     }
 }

@@ -3,7 +3,7 @@
 // Torch Lattice docs, "Migrating from TorchSparse": hashing is one of the CUDA
 // kernels of the library ("What remains familiar") and its capacity knob is
 // torch_lattice.backends.hash_rsv_ratio ("Backend and configuration
-// differences").  Design: 16-byte slots {key, row}, SplitMix64 placement,
+// differences").  Design: 16-byte slots {key, row}, 32-bit mixing hash placement,
 // linear probing bounded by the slot count, 64-bit atomicCAS to claim a slot
 // and an unsigned atomicMin on the row so that duplicates keep the lowest row
 // deterministically.
@@ -12,7 +12,7 @@
 namespace lat {
 
 __global__ void __launch_bounds__(256) hash_insert_kernel(const int4 *__restrict__ coords, int64_t n,
-                                                          Slot *__restrict__ slots, uint64_t cap_mask,
+                                                          Slot *__restrict__ slots, uint32_t cap_mask,
                                                           int32_t *d_status) {
     int32_t bad = 0;
     for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n;
@@ -23,9 +23,9 @@ __global__ void __launch_bounds__(256) hash_insert_kernel(const int4 *__restrict
             bad |= LAT_ERR_COORD_RANGE;
             continue;
         }
-        uint64_t s = mix64(key) & cap_mask;
+        uint32_t s = slot_hash(key) & cap_mask;
         bool placed = false;
-        for (uint64_t probe = 0; probe <= cap_mask; ++probe) {
+        for (uint32_t probe = 0; probe <= cap_mask; ++probe) {
             unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(&slots[s].key);
             if (cur == kEmptyKey)
                 cur = atomicCAS(&slots[s].key, (unsigned long long)kEmptyKey, (unsigned long long)key);
@@ -68,7 +68,7 @@ extern "C" lat_status lat_hash_build(const int32_t *coords, int64_t n, void *tab
     const int threads = 256;
     const int64_t blocks = (n + threads - 1) / threads;
     hash_insert_kernel<<<unsigned(blocks), threads, 0, s>>>(reinterpret_cast<const int4 *>(coords), n,
-                                                             static_cast<Slot *>(table), cap - 1, d_status);
+                                                             static_cast<Slot *>(table), uint32_t(cap - 1), d_status);
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }

@@ -4,14 +4,17 @@
 // and coordinate query are CUDA kernels of the library ("What remains
 // familiar", "Sparse tensor expectations"), and the support semantics come
 // from the "Convolution mapping" table.  Pipeline (all on `stream`):
-//   1. probe:  one thread per output row, K^3 probes of the input table;
-//              writes nbr (offset-major, coalesced), mask, and per (offset,
-//              block) hit counts from warp ballots.
+//   1. probe:  one thread per output row probes the input table (for a
+//              submanifold map only the offsets below the centre, mirroring
+//              each hit); writes nbr (offset-major, coalesced), mask, and per
+//              (offset, block) hit counts from warp ballots (a count pass over
+//              nbr does the last two for submanifold maps).
 //   2. scan:   one block per offset turns its per-block counts into offsets
 //              (pairs come out grouped by offset, rows ascending).
 //   3. emit:   re-reads nbr and writes (in, out) pairs at ballot-ranked
 //              positions: deterministic, no atomics.
-//   4. sort:   stable radix sort of output rows by mask -> perm.
+//   4. sort:   stable 2-pass radix sort of output rows by a 16-bit grouping
+//              key of the mask (neighbour count, mask hash) -> perm.
 //   5. tiles:  OR of masks over each LAT_TILE_ROWS run of perm -> tile_mask.
 #include <cub/device/device_radix_sort.cuh>
 
@@ -27,9 +30,29 @@ struct Geom {
     int mode;
     int k3;
     signed char off[32][3];  // (ix, iy, iz) of offset k
+    // Unit stride on every axis: the probed coordinate is the row's own plus a
+    // fixed vector, so the probed key is the row's key plus a packed delta as long
+    // as no field leaves [0, 65535] (row coordinates within [lo, hi] per axis).
+    int shift;
+    long long delta[32];
+    int lo[3], hi[3];
 };
 
 constexpr int kProbeBatch = 8;  // slot loads a thread keeps in flight
+constexpr int kGroupKeyBits = 16;
+
+// Sort key that groups output rows for the convolution tiles: the number of
+// neighbours (capped at 31) in the top 5 bits, then 11 bits of a multiplicative
+// hash of the mask.  Rows with equal masks share a key; sorting by it keeps the
+// union of masks inside a 128-row tile as small as an exact sort by mask does
+// on the LiDAR- and image-shaped inputs, in 2 radix passes instead of 4.
+// With at most 8 offsets the mask itself is the key (exact, one radix pass).
+__device__ __forceinline__ uint32_t group_key(uint32_t m, int k3) {
+    if (k3 <= 8) return m;
+    const uint32_t pc = min(__popc(m), 31);
+    return (pc << 11) | ((m * 0x9E3779B1u) >> 21);
+}
+inline int group_key_bits(int k3) { return k3 <= 8 ? k3 : kGroupKeyBits; }
 
 // Input coordinate probed by output row c at offset (ix, iy, iz); false if none.
 __device__ __forceinline__ bool query_coord(const Geom &g, const int4 &c, int ix, int iy, int iz, uint64_t &key) {
@@ -55,24 +78,38 @@ __device__ __forceinline__ bool query_coord(const Geom &g, const int4 &c, int ix
 // batch at once (one 16-byte load per slot), then resolves what it can, so a
 // thread keeps several independent loads in flight instead of walking the
 // probe sequences one after another.  Rounds are bounded by the slot count.
-// For a submanifold map the centre offset is the row itself and is not probed.
+//
+// SYM (submanifold maps): the relation is symmetric -- input i sits at offset
+// k of row j exactly when j sits at offset k3-1-k of row i -- so only the
+// offsets below the centre are probed; a hit also writes the mirrored entry
+// (the upper half of nbr must hold -1 beforehand), and the centre is the row
+// itself.  Masks and per-block counts then come from kmap_count_kernel.
+// Otherwise every offset is probed and the mask and counts are produced here.
+template <bool SYM>
 __global__ void __launch_bounds__(kQueryThreads)
-kmap_probe_kernel(const Slot *__restrict__ slots, uint64_t cap_mask, const int4 *__restrict__ out_coords,
+kmap_probe_kernel(const Slot *__restrict__ slots, uint32_t cap_mask, const int4 *__restrict__ out_coords,
                   int64_t n_out, int64_t n_in, Geom g, int32_t *__restrict__ nbr, uint32_t *__restrict__ mask,
-                  int32_t *__restrict__ iota, int32_t *__restrict__ block_counts, int nblk, int32_t *d_status) {
+                  uint32_t *__restrict__ keys, int32_t *__restrict__ iota, int32_t *__restrict__ block_counts, int nblk,
+                  int32_t *d_status) {
     __shared__ int s_cnt[32];
-    if (threadIdx.x < 32) s_cnt[threadIdx.x] = 0;
-    __syncthreads();
+    if (!SYM) {
+        if (threadIdx.x < 32) s_cnt[threadIdx.x] = 0;
+        __syncthreads();
+    }
     const int64_t j = blockIdx.x * int64_t(kQueryThreads) + threadIdx.x;
     const bool live = j < n_out;
     int4 c = make_int4(0, 0, 0, 0);
     if (live) c = __ldg(out_coords + j);
     const int centre = g.mode == LAT_SUBM ? g.k3 / 2 : -1;
+    const int kend = SYM ? centre : g.k3;
+    uint64_t self = 0;
+    const bool fast = live && g.shift && c.y >= g.lo[0] && c.y <= g.hi[0] && c.z >= g.lo[1] && c.z <= g.hi[1] &&
+                      c.w >= g.lo[2] && c.w <= g.hi[2] && pack_key(c.x, c.y, c.z, c.w, self);
     uint32_t m = 0;
     int32_t bad = 0;
-    for (int k0 = 0; k0 < g.k3; k0 += kProbeBatch) {
+    for (int k0 = 0; k0 < kend; k0 += kProbeBatch) {
         uint64_t key[kProbeBatch];
-        uint32_t slot[kProbeBatch];  // slot counts are below 2^31 (lat_hash_bytes)
+        uint32_t slot[kProbeBatch];
         int row[kProbeBatch];
         uint32_t pending = 0;
 #pragma unroll
@@ -81,15 +118,24 @@ kmap_probe_kernel(const Slot *__restrict__ slots, uint64_t cap_mask, const int4 
             row[e] = -1;
             key[e] = kEmptyKey;
             slot[e] = 0;
-            if (!live || k >= g.k3) continue;
+            if (!live || k >= kend) continue;
             if (k == centre) {
                 row[e] = int(j);
-            } else if (query_coord(g, c, g.off[k][0], g.off[k][1], g.off[k][2], key[e])) {
-                slot[e] = uint32_t(mix64(key[e]) & cap_mask);
+                continue;
+            }
+            bool ok;
+            if (fast) {
+                key[e] = self + uint64_t(g.delta[k]);
+                ok = true;
+            } else {
+                ok = query_coord(g, c, g.off[k][0], g.off[k][1], g.off[k][2], key[e]);
+            }
+            if (ok) {
+                slot[e] = slot_hash(key[e]) & cap_mask;
                 pending |= 1u << e;
             }
         }
-        for (uint64_t round = 0; pending && round <= cap_mask; ++round) {
+        for (uint32_t round = 0; pending && round <= cap_mask; ++round) {
             unsigned long long kv[kProbeBatch];
             uint32_t rv[kProbeBatch];
 #pragma unroll
@@ -109,27 +155,36 @@ kmap_probe_kernel(const Slot *__restrict__ slots, uint64_t cap_mask, const int4 
                 } else if (kv[e] == kEmptyKey) {
                     pending &= ~(1u << e);
                 } else {
-                    slot[e] = uint32_t((slot[e] + 1) & cap_mask);
+                    slot[e] = (slot[e] + 1) & cap_mask;
                 }
             }
         }
 #pragma unroll
         for (int e = 0; e < kProbeBatch; ++e) {
             const int k = k0 + e;
-            if (k >= g.k3) break;
+            if (k >= kend) break;
             int r = row[e];
-            if (r >= n_in) { bad |= LAT_ERR_BAD_MAP; r = -1; }
+            if (r >= n_in || (SYM && r >= n_out)) { bad |= LAT_ERR_BAD_MAP; r = -1; }
             if (live) nbr[int64_t(k) * n_out + j] = r;
-            const unsigned hits = __ballot_sync(0xFFFFFFFFu, r >= 0);
-            if (r >= 0) m |= 1u << k;
-            if ((threadIdx.x & 31) == 0 && hits) atomicAdd(&s_cnt[k], __popc(hits));
+            if (SYM) {
+                if (r >= 0) nbr[int64_t(g.k3 - 1 - k) * n_out + r] = int32_t(j);
+            } else {
+                const unsigned hits = __ballot_sync(0xFFFFFFFFu, r >= 0);
+                if (r >= 0) m |= 1u << k;
+                if ((threadIdx.x & 31) == 0 && hits) atomicAdd(&s_cnt[k], __popc(hits));
+            }
         }
+    }
+    if (bad) flag(d_status, bad);
+    if (SYM) {
+        if (live) nbr[int64_t(centre) * n_out + j] = int32_t(j);
+        return;
     }
     if (live) {
         mask[j] = m;
+        keys[j] = group_key(m, g.k3);
         iota[j] = int32_t(j);
     }
-    if (bad) flag(d_status, bad);
     __syncthreads();
     if (threadIdx.x < g.k3) block_counts[int64_t(threadIdx.x) * nblk + blockIdx.x] = s_cnt[threadIdx.x];
 }
@@ -221,15 +276,15 @@ kmap_emit_kernel(const int32_t *__restrict__ nbr, int64_t n_out, int k3, const i
     if (over) flag(d_status, LAT_ERR_CAPACITY);
 }
 
-__global__ void tile_mask_kernel(const uint32_t *__restrict__ sorted_mask, int64_t n, uint32_t *__restrict__ tile_mask,
-                                 int64_t ntiles) {
+__global__ void tile_mask_kernel(const uint32_t *__restrict__ mask, const int32_t *__restrict__ perm, int64_t n,
+                                 uint32_t *__restrict__ tile_mask, int64_t ntiles) {
     const int64_t t = blockIdx.x * int64_t(blockDim.x / 32) + (threadIdx.x >> 5);
     if (t >= ntiles) return;
     const int lane = threadIdx.x & 31;
     uint32_t m = 0;
     for (int r = lane; r < LAT_TILE_ROWS; r += 32) {
         const int64_t e = t * LAT_TILE_ROWS + r;
-        if (e < n) m |= sorted_mask[e];
+        if (e < n) m |= mask[perm[e]];
     }
     for (int o = 16; o; o >>= 1) m |= __shfl_xor_sync(0xFFFFFFFFu, m, o);
     if (lane == 0) tile_mask[t] = m;
@@ -239,18 +294,25 @@ __global__ void tile_mask_kernel(const uint32_t *__restrict__ sorted_mask, int64
 // probing (maps built from parent indices); also writes the identity row order.
 __global__ void __launch_bounds__(kQueryThreads)
 kmap_count_kernel(const int32_t *__restrict__ nbr, int64_t n_out, int k3, int32_t *__restrict__ iota,
-                  int32_t *__restrict__ block_counts, int nblk) {
+                  int32_t *__restrict__ block_counts, int nblk, uint32_t *__restrict__ mask,
+                  uint32_t *__restrict__ keys) {
     __shared__ int s_cnt[32];
     if (threadIdx.x < 32) s_cnt[threadIdx.x] = 0;
     __syncthreads();
     const int64_t j = blockIdx.x * int64_t(kQueryThreads) + threadIdx.x;
     const bool live = j < n_out;
+    uint32_t m = 0;
     for (int k = 0; k < k3; ++k) {
         const int row = live ? nbr[int64_t(k) * n_out + j] : -1;
         const unsigned hits = __ballot_sync(0xFFFFFFFFu, row >= 0);
+        if (row >= 0) m |= 1u << k;
         if ((threadIdx.x & 31) == 0 && hits) atomicAdd(&s_cnt[k], __popc(hits));
     }
-    if (live) iota[j] = int32_t(j);
+    if (live) {
+        iota[j] = int32_t(j);
+        keys[j] = group_key(m, k3);
+        if (mask) mask[j] = m;
+    }
     __syncthreads();
     if (threadIdx.x < k3) block_counts[int64_t(threadIdx.x) * nblk + blockIdx.x] = s_cnt[threadIdx.x];
 }
@@ -288,7 +350,8 @@ struct KmapWs {
     int64_t *block_offsets;
     int64_t *k_total;
     int32_t *iota;
-    uint32_t *sorted_mask;
+    uint32_t *keys;
+    uint32_t *sorted_keys;
     void *cub_tmp;
     size_t cub_bytes;
     size_t total;
@@ -302,7 +365,8 @@ static KmapWs carve_kmap_ws(void *base, int64_t n_out, int k3) {
     w.block_offsets = cv.take<int64_t>(size_t(k3) * nblk);
     w.k_total = cv.take<int64_t>(size_t(k3));
     w.iota = cv.take<int32_t>(size_t(n_out));
-    w.sorted_mask = cv.take<uint32_t>(size_t(n_out));
+    w.keys = cv.take<uint32_t>(size_t(n_out));
+    w.sorted_keys = cv.take<uint32_t>(size_t(n_out));
     size_t cub_bytes = 0;
     cub::DeviceRadixSort::SortPairs(nullptr, cub_bytes, (const uint32_t *)nullptr, (uint32_t *)nullptr,
                                     (const int32_t *)nullptr, (int32_t *)nullptr, int(n_out), 0, 32);
@@ -322,10 +386,10 @@ static lat_status finish_kmap(lat_kmap *map, int k3, int nblk, KmapWs &w, int32_
                                                      d_status);
     LAT_CUDA_TRY(cudaGetLastError());
     size_t cub_bytes = w.cub_bytes;
-    LAT_CUDA_TRY(cub::DeviceRadixSort::SortPairs(w.cub_tmp, cub_bytes, map->mask, w.sorted_mask, w.iota, map->perm,
-                                                 int(n_out), 0, k3, s));
+    LAT_CUDA_TRY(cub::DeviceRadixSort::SortPairs(w.cub_tmp, cub_bytes, w.keys, w.sorted_keys, w.iota, map->perm,
+                                                 int(n_out), 0, group_key_bits(k3), s));
     const int64_t ntiles = (n_out + LAT_TILE_ROWS - 1) / LAT_TILE_ROWS;
-    tile_mask_kernel<<<unsigned((ntiles + 7) / 8), 256, 0, s>>>(w.sorted_mask, n_out, map->tile_mask, ntiles);
+    tile_mask_kernel<<<unsigned((ntiles + 7) / 8), 256, 0, s>>>(map->mask, map->perm, n_out, map->tile_mask, ntiles);
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }
@@ -374,6 +438,7 @@ extern "C" lat_status lat_kmap_query(const void *table, size_t table_bytes, cons
         table_bytes / sizeof(Slot) > (uint64_t(1) << 31))
         return LAT_ERR_ARG;
     if (n_out > 0 && !out_coords) return LAT_ERR_ARG;
+    if (geom->mode == LAT_SUBM && n_in != n_out) return LAT_ERR_ARG;  // the support is preserved
     if (reinterpret_cast<uintptr_t>(out_coords) % 16 || reinterpret_cast<uintptr_t>(table) % 16) return LAT_ERR_ARG;
     const KmapWs need = carve_kmap_ws(nullptr, n_out, k3);
     if (ws_bytes < need.total || (need.total && !ws)) return LAT_ERR_WORKSPACE;
@@ -392,18 +457,47 @@ extern "C" lat_status lat_kmap_query(const void *table, size_t table_bytes, cons
     }
     g.mode = geom->mode;
     g.k3 = k3;
+    // unit stride: probed coordinate = own + sign * (off - pad), sign -1 for the transposed relation
+    g.shift = g.st[0] == 1 && g.st[1] == 1 && g.st[2] == 1;
+    const int sign = g.mode == LAT_TRANSPOSED ? -1 : 1;
+    int dmin[3] = {0, 0, 0}, dmax[3] = {0, 0, 0};
+    for (int a = 0; a < 3; ++a) {
+        const int d0 = sign * (0 - g.pd[a]), d1 = sign * (g.ks[a] - 1 - g.pd[a]);
+        dmin[a] = d0 < d1 ? d0 : d1;
+        dmax[a] = d0 < d1 ? d1 : d0;
+        g.lo[a] = -32768 - dmin[a];
+        g.hi[a] = 32767 - dmax[a];
+    }
     for (int ix = 0, k = 0; ix < g.ks[0]; ++ix)
         for (int iy = 0; iy < g.ks[1]; ++iy)
             for (int iz = 0; iz < g.ks[2]; ++iz, ++k) {
                 g.off[k][0] = static_cast<signed char>(ix);
                 g.off[k][1] = static_cast<signed char>(iy);
                 g.off[k][2] = static_cast<signed char>(iz);
+                const long long dx = sign * (ix - g.pd[0]), dy = sign * (iy - g.pd[1]), dz = sign * (iz - g.pd[2]);
+                g.delta[k] = dx * (1ll << 32) + dy * (1ll << 16) + dz;
             }
     const int nblk = int((n_out + kQueryThreads - 1) / kQueryThreads);
-    const uint64_t cap_mask = table_bytes / sizeof(Slot) - 1;
-    kmap_probe_kernel<<<nblk, kQueryThreads, 0, s>>>(static_cast<const Slot *>(table), cap_mask,
-                                                      reinterpret_cast<const int4 *>(out_coords), n_out, n_in, g,
-                                                      map->nbr, map->mask, w.iota, w.block_counts, nblk, d_status);
+    const uint32_t cap_mask = uint32_t(table_bytes / sizeof(Slot) - 1);
+    const Slot *slots = static_cast<const Slot *>(table);
+    const int4 *oc = reinterpret_cast<const int4 *>(out_coords);
+    if (geom->mode == LAT_SUBM) {
+        // the upper half of the table is filled by mirrored hits only
+        const int centre = k3 / 2;
+        if (centre + 1 < k3)
+            LAT_CUDA_TRY(cudaMemsetAsync(map->nbr + int64_t(centre + 1) * n_out, 0xFF,
+                                         sizeof(int32_t) * size_t(k3 - 1 - centre) * n_out, s));
+        kmap_probe_kernel<true><<<nblk, kQueryThreads, 0, s>>>(slots, cap_mask, oc, n_out, n_in, g, map->nbr,
+                                                               map->mask, w.keys, w.iota, w.block_counts, nblk,
+                                                               d_status);
+        LAT_CUDA_TRY(cudaGetLastError());
+        kmap_count_kernel<<<nblk, kQueryThreads, 0, s>>>(map->nbr, n_out, k3, w.iota, w.block_counts, nblk,
+                                                          map->mask, w.keys);
+    } else {
+        kmap_probe_kernel<false><<<nblk, kQueryThreads, 0, s>>>(slots, cap_mask, oc, n_out, n_in, g, map->nbr,
+                                                                map->mask, w.keys, w.iota, w.block_counts, nblk,
+                                                                d_status);
+    }
     LAT_CUDA_TRY(cudaGetLastError());
     return finish_kmap(map, k3, nblk, w, d_status, s);
 }
@@ -456,7 +550,8 @@ extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int
         }
         KmapWs w = carve_kmap_ws(ws, map->n_out, k3);
         const int nblk = int((map->n_out + kQueryThreads - 1) / kQueryThreads);
-        kmap_count_kernel<<<nblk, kQueryThreads, 0, s>>>(map->nbr, map->n_out, k3, w.iota, w.block_counts, nblk);
+        kmap_count_kernel<<<nblk, kQueryThreads, 0, s>>>(map->nbr, map->n_out, k3, w.iota, w.block_counts, nblk,
+                                                          nullptr, w.keys);
         LAT_CUDA_TRY(cudaGetLastError());
         const lat_status st = finish_kmap(map, k3, nblk, w, d_status, s);
         if (st != LAT_OK) return st;

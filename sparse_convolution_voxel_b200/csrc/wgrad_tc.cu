@@ -48,7 +48,19 @@ __host__ __device__ constexpr uint32_t make_idesc() {
            (1u << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
 
-// Unit u covers pairs [lo, hi) of offset k; returns false past the last unit.
+// First unit of every offset (and the total in ub[k3]): offset k's clamped pairs
+// are cut into ceil(P_k / kChunk) units, numbered in offset order.
+__device__ __forceinline__ void unit_bases(const int64_t *pair_off, int64_t capacity, int k3, int32_t *ub) {
+    int32_t u = 0;
+    for (int k = 0; k < k3; ++k) {
+        ub[k] = u;
+        const int64_t lo = min(pair_off[k], capacity), hi = min(pair_off[k + 1], capacity);
+        u += int32_t((hi - lo + kChunk - 1) / kChunk);
+    }
+    ub[k3] = u;
+}
+
+// Unit u covers pairs [lo, hi) of offset k.
 __device__ __forceinline__ void unit_range(const int32_t *unit_base, const int64_t *pair_off, int64_t capacity,
                                            int k3, int32_t u, int &k, int64_t &lo, int64_t &hi) {
     k = 0;
@@ -62,8 +74,7 @@ template <typename T, int M, int N>
 __global__ void __launch_bounds__(kThreads, 2)
 wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t *__restrict__ pair_off,
                 const int32_t *__restrict__ pair_in, const int32_t *__restrict__ pair_out, int64_t capacity, int k3,
-                int64_t n_in, int64_t n_out, const int32_t *__restrict__ unit_base, float *__restrict__ partial,
-                int32_t *d_status) {
+                int64_t n_in, int64_t n_out, float *__restrict__ partial, int32_t *d_status) {
     using C = Cfg<M, N>;
     constexpr int NS = C::kStages;
     constexpr int kLag = C::kLag;
@@ -77,10 +88,11 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
     uint64_t *accempty = accfull + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accempty + 2);
     __shared__ int s_abort;
+    __shared__ int32_t unit_base[33];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int32_t units = unit_base[k3];
     if (tid == 0) {
+        unit_bases(pair_off, capacity, k3, unit_base);
         for (int s = 0; s < NS; ++s) {
             ptx::mbar_init(&full[s], kProdWarps * 32);
             ptx::mbar_init(&empty[s], 1);
@@ -101,6 +113,7 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    const int32_t units = unit_base[k3];
     int32_t bad = 0;
 
     if (warp < kProdWarps) {
@@ -271,20 +284,11 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
     }
 }
 
-__global__ void wgrad_tc_units_kernel(const int64_t *__restrict__ pair_off, int k3, int64_t capacity,
-                                      int32_t *__restrict__ unit_base) {
-    if (threadIdx.x != 0 || blockIdx.x != 0) return;
-    int32_t u = 0;
-    for (int k = 0; k < k3; ++k) {
-        unit_base[k] = u;
-        const int64_t lo = min(pair_off[k], capacity), hi = min(pair_off[k + 1], capacity);
-        u += int32_t((hi - lo + kChunk - 1) / kChunk);
-    }
-    unit_base[k3] = u;
-}
-
-__global__ void wgrad_tc_reduce_kernel(const float *__restrict__ partial, const int32_t *__restrict__ unit_base,
-                                       int k3, int nelem, float *__restrict__ dw) {
+__global__ void wgrad_tc_reduce_kernel(const float *__restrict__ partial, const int64_t *__restrict__ pair_off,
+                                       int64_t capacity, int k3, int nelem, float *__restrict__ dw) {
+    __shared__ int32_t unit_base[33];
+    if (threadIdx.x == 0) unit_bases(pair_off, capacity, k3, unit_base);
+    __syncthreads();
     const int k = blockIdx.y;
     const int el = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
     if (k >= k3 || el >= nelem) return;
@@ -305,20 +309,17 @@ static lat_status launch(const void *x, const void *dy, const lat_kmap *map, flo
     using C = Cfg<M, N>;
     const int64_t units_max = (map->pair_capacity + kChunk - 1) / kChunk + map->k3;
     Carver cv(ws);
-    int32_t *unit_base = cv.take<int32_t>(size_t(map->k3) + 1);
     float *partial = cv.take<float>(size_t(units_max) * M * N);
-    wgrad_tc_units_kernel<<<1, 32, 0, s>>>(map->pair_off, map->k3, map->pair_capacity, unit_base);
-    LAT_CUDA_TRY(cudaGetLastError());
     auto kern = wgrad_tc_kernel<T, M, N>;
     const int64_t grid = std::min<int64_t>(units_max, GridCache<KernelTag<T, M, N>>::get(kern, C::kSmem, int(C::kTmemCols), 2));
     if (grid <= 0) return LAT_ERR_CUDA;
     kern<<<unsigned(grid), kThreads, C::kSmem, s>>>(static_cast<const T *>(x), static_cast<const T *>(dy),
                                                     map->pair_off, map->pair_in, map->pair_out, map->pair_capacity,
-                                                    map->k3, map->n_in, map->n_out, unit_base, partial, d_status);
+                                                    map->k3, map->n_in, map->n_out, partial, d_status);
     LAT_CUDA_TRY(cudaGetLastError());
     const int nelem = M * N;
     dim3 rg((nelem / 4 + 255) / 256, map->k3);
-    wgrad_tc_reduce_kernel<<<rg, 256, 0, s>>>(partial, unit_base, map->k3, nelem, dw);
+    wgrad_tc_reduce_kernel<<<rg, 256, 0, s>>>(partial, map->pair_off, map->pair_capacity, map->k3, nelem, dw);
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }
@@ -330,7 +331,6 @@ bool wgrad_tc_supported(int cin, int cout) { return (cin == 64 || cin == 128) &&
 size_t wgrad_tc_ws_bytes(int cin, int cout, const lat_kmap *map) {
     const int64_t units_max = (map->pair_capacity + wtc::kChunk - 1) / wtc::kChunk + map->k3;
     Carver cv(nullptr);
-    cv.take<int32_t>(size_t(map->k3) + 1);
     cv.take<float>(size_t(units_max) * cin * cout);
     return align_up(cv.used, 256);
 }

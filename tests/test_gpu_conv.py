@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import synthetic
-from tests.util import TORCH_DT, assert_close, feats, rand_coords, weights
+from tests.util import TORCH_DT, assert_close, check_kmap, feats, rand_coords, weights
 
 pytestmark = pytest.mark.gpu
 
@@ -184,3 +184,19 @@ def test_transposed_fwd_with_rows_without_neighbours(dtype):
     w, w64 = weights(6, 64, 64, dtype, seed=29)
     z = scv.conv_fwd(x, w, up, out=torch.full((len(coords), 64), 3.0, dtype=dtype, device="cuda"))
     assert_close(z.double().cpu().numpy(), oracle.conv_fwd(x64, w64, ref_up), dtype, "transposed fwd")
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.float32])
+def test_target_conv(dtype):
+    """TargetConv3d: a stride-1 strided geometry evaluated at caller coordinates."""
+    rng = np.random.default_rng(43)
+    coords = rand_coords(rng, 1200, -8, 8, 2)
+    targets = rand_coords(rng, 1000, -9, 9, 2)
+    c, tg = _dev(coords), _dev(targets)
+    km = scv.kernel_map(scv.hash_table(c), len(coords), tg, scv.target_geom(3))
+    ref_nbr = oracle.kmap(coords, targets, 3, 1, 1, oracle.STRIDED)
+    check_kmap(km, ref_nbr)
+    x, x64 = feats(len(coords), 64, dtype, seed=47)
+    w, w64 = weights(27, 64, 64, dtype, seed=47)
+    y = scv.conv_fwd(x, w, km)
+    assert_close(y.double().cpu().numpy(), oracle.conv_fwd(x64, w64, ref_nbr), dtype, "target conv")

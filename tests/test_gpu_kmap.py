@@ -21,6 +21,19 @@ def _dev(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
 
+def _slot_hash(key: int) -> int:
+    """The table's placement function (fold of the key halves + MurmurHash3 fmix32),
+    restated here to check where the GPU put every key."""
+    M = 0xFFFFFFFF
+    h = (key & M) ^ (((key >> 32) * 0x9E3779B1) & M)
+    h ^= h >> 16
+    h = (h * 0x85EBCA6B) & M
+    h ^= h >> 13
+    h = (h * 0xC2B2AE35) & M
+    h ^= h >> 16
+    return h
+
+
 def _subm(coords, ks=(3, 3, 3), d_status=None):
     c = _dev(coords)
     table = scv.hash_table(c, 2.0, d_status)
@@ -45,7 +58,7 @@ def test_hash_table_places_every_key_reachably():
     for s in occupied:
         k = int(keys[s])
         assert want[k] == rows[s]
-        home = oracle.splitmix64(k) & (cap - 1)
+        home = _slot_hash(k) & (cap - 1)
         d = (s - home) % cap                       # linear probing: no empty slot between home and s
         assert all(keys[(home + e) % cap] != empty for e in range(d))
 

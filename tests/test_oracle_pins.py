@@ -8,8 +8,7 @@
   backward passes;
 * closed forms and special cases: kernel size 1 equals a dense matmul, an
   isolated voxel sees only the centre weight, adjoint identities, offset
-  symmetry of the submanifold map, one parent per input for k = s;
-* the published SplitMix64 reference sequence.
+  symmetry of the submanifold map, one parent per input for k = s.
 """
 import os
 
@@ -97,14 +96,6 @@ def test_two_voxel_worked_example(golden_dir):
 
 
 # --------------------------------------------------------------------------- key packing + hash fn
-def test_splitmix64_reference_sequence(golden_dir):
-    for line in open(os.path.join(golden_dir, "splitmix64_seed0.txt")):
-        if line.startswith("#") or not line.strip():
-            continue
-        z, out = (int(t, 16) for t in line.split())
-        assert oracle.splitmix64(z) == out
-
-
 def test_packed_key_order_is_lexicographic():
     rng = np.random.default_rng(0)
     rows = np.concatenate([
@@ -345,3 +336,16 @@ def test_support_preserving_counts():
     nbr = oracle.kmap(c, c, 3, 1, 1, SUBM)
     assert nbr.shape[0] == len(c)
     assert len(oracle.downsample(c, 2, 2, 0)) <= len(c)
+
+
+def test_target_conv_matches_dense_conv_at_target_sites():
+    """TargetConv3d ("Convolution mapping": convolution at known output
+    coordinates) = the stride-1 strided relation evaluated at caller targets."""
+    rng = np.random.default_rng(41)
+    c = _rand_coords(rng, 150, 0, 8, batch=2)
+    targets = _rand_coords(rng, 90, 0, 8, batch=2)       # mixes active and inactive sites
+    x = rng.standard_normal((len(c), 3))
+    w = rng.standard_normal((27, 3, 5))
+    y = oracle.conv_fwd(x, w, oracle.kmap(c, targets, 3, 1, 1, STRIDED))
+    dense = torch.nn.functional.conv3d(_densify(c, x, (8, 8, 8), (0, 0, 0)), _dense_weight(w, (3, 3, 3)), padding=1)
+    np.testing.assert_allclose(y, _read(dense, targets, (0, 0, 0)).numpy(), rtol=1e-12, atol=1e-12)

@@ -51,6 +51,15 @@ def u32(a: np.ndarray) -> np.ndarray:
     return np.asarray(a).astype(np.int64) & 0xFFFFFFFF
 
 
+def group_key(mask: np.ndarray, k3: int) -> np.ndarray:
+    """The documented row-grouping key of a neighbour mask (include/lattice.h, lat_kmap.perm)."""
+    m = np.asarray(mask, np.int64) & 0xFFFFFFFF
+    if k3 <= 8:
+        return m
+    pc = np.minimum(np.array([bin(int(v)).count("1") for v in m], np.int64), 31)
+    return (pc << 11) | (((m * 0x9E3779B1) & 0xFFFFFFFF) >> 21)
+
+
 def check_kmap(km, ref_nbr: np.ndarray):
     """Bit-exact comparison of a device KernelMap against the oracle's (n_out, k3) table."""
     import oracle
@@ -66,7 +75,7 @@ def check_kmap(km, ref_nbr: np.ndarray):
     assert np.array_equal(km.pair_in[:P].cpu().numpy(), pin), "pair inputs differ"
     assert np.array_equal(km.pair_out[:P].cpu().numpy(), pout), "pair outputs differ"
     perm = km.perm[:n_out].cpu().numpy()
-    assert np.array_equal(perm, np.argsort(ref_mask, kind="stable")), "perm is not the stable mask sort"
+    assert np.array_equal(perm, np.argsort(group_key(ref_mask, k3), kind="stable")), "perm is not the stable key sort"
     ntiles = (n_out + 127) // 128
     tm = u32(km.tile_mask[:ntiles].cpu().numpy())
     sm = ref_mask[perm] if n_out else ref_mask
