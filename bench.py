@@ -39,6 +39,7 @@ import synthetic  # noqa: E402
 WORKLOAD = "lidar_subm"
 METRIC = "sparse-conv effective TFLOP/s + kmap Mvoxels/s at 1 B200, % of roofline"
 CIN, CMID = 64, 128
+RSV_RATIO = 4.0  # hash slots per voxel (hash_rsv_ratio)
 
 
 def dist_env():
@@ -102,7 +103,7 @@ class Pipeline:
         n = self.n = host["coords"].shape[0]
         self.status = scv.new_status(dev)
         self.ws = scv.Workspace(dev)
-        self.table = torch.empty(scv.lat_hash_bytes(n, 2.0) // 8, dtype=torch.int64, device=dev)
+        self.table = torch.empty(scv.lat_hash_bytes(n, RSV_RATIO) // 8, dtype=torch.int64, device=dev)
         self.km = scv.KernelMap(n, n, 27, dev)
         self.y = torch.empty((n, CIN), dtype=torch.half, device=dev)
         self.dx = torch.empty((n, CIN), dtype=torch.half, device=dev)
@@ -176,6 +177,13 @@ class Pipeline:
             "down_fwd": n * CIN * e + nc * CMID * e + 8 * CIN * CMID * e + 8 * n,
             "up_fwd": n * CMID * e + n * CIN * e + 8 * CIN * CMID * e + 8 * n,
         }
+
+
+# DRAM bytes per launch of a phase from one ncu capture of this workload
+# (profiles/launches_lidar_subm_step.md: the submanifold kmap query, all of its
+# kernels, cache control at ncu's default); None where no capture matches the
+# current kernels.
+PHASE_TRAFFIC = {"kmap": 60.83e6}
 
 
 def flush_l2(buf: torch.Tensor):
@@ -355,7 +363,7 @@ def run_only(args):
     st = scv.new_status(dev)
     ws = scv.Workspace(dev)
     geom = scv.subm_geom(wl.ksize)
-    table = scv.hash_table(coords, 2.0, st)
+    table = scv.hash_table(coords, args.rsv_ratio, st)
     km = scv.kernel_map(table, n, coords, geom, ws, st)
     y = torch.empty((n, cout), dtype=dt, device=dev)
     dx = torch.empty((n, cin), dtype=dt, device=dev)
@@ -407,7 +415,8 @@ def run_only(args):
     stv = scv.lat_status_fetch(st)
     t = statistics.median(ms)
     hbm, _, src = load_peaks()
-    print(json.dumps({"only": args.only, "workload": args.workload, "rows": n, "pairs": P, "ms_median": t,
+    print(json.dumps({"only": args.only, "workload": args.workload, "rsv_ratio": args.rsv_ratio, "rows": n,
+                      "pairs": P, "ms_median": t,
                       "ms_min": min(ms), "alg_bytes": nbytes, "achieved_gbs": nbytes / (t * 1e-3) / 1e9,
                       "frac_hbm": nbytes / (t * 1e-3) / 1e9 / hbm, "peak_source": src, "status": stv,
                       "host_us_per_call": host_us, "b2b_ms_per_call": b2b_ms}), flush=True)
@@ -424,6 +433,7 @@ def main():
     ap.add_argument("--only", choices=["hash", "kmap", "fwd", "dgrad", "wgrad", "downsample"],
                     help="time a single op of the path on --workload (for profiler captures)")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(synthetic.WORKLOADS))
+    ap.add_argument("--rsv-ratio", type=float, default=RSV_RATIO, help="hash table slots per voxel (--only mode)")
     ap.add_argument("--lean", action="store_true",
                     help="skip launch counting, the end-to-end pass and the CPU baseline (for profiler runs)")
     args = ap.parse_args()
@@ -501,7 +511,8 @@ def main():
             "pairs": pipe.pair_count(), "coarse_voxels": pipe.nc,
             "phase_ms": {k: round(v, 4) for k, v in phase_ms.items()},
             "roofline": {"kernel": dominant, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                         "frac": achieved / hbm, "traffic": None, "peak_source": f"{src} hbm_gbs",
+                         "frac": achieved / hbm, "traffic": PHASE_TRAFFIC.get(dominant),
+                         "alg_bytes": pb[dominant], "peak_source": f"{src} hbm_gbs",
                          "per_phase_frac": {p: round(pb[p] / (phase_ms[p] * 1e-3) / 1e9 / hbm, 4) for p in pb}},
             "gpu_launches": None if launches_per_step is None else launches_per_step * args.steps,
             "e2e": e2e,

@@ -150,8 +150,9 @@ typedef struct {
  */
 
 /* Bytes of a table for n rows: 16 * next_pow2(max(ceil(rsv_ratio*n), 64)).
- * rsv_ratio must be >= 1 (default 2); at most 2^31 slots.  Returns 0 on
- * invalid input. */
+ * rsv_ratio must be >= 1; at most 2^31 slots.  The Python helpers use 4: at
+ * a load factor of 1/8..1/4 most probes end at their home slot, which cuts
+ * the query's probe rounds.  Returns 0 on invalid input. */
 size_t lat_hash_bytes(int64_t n, float rsv_ratio);
 
 /* Insert coords[0..n) (int32 (n,4)) into `table` (table_bytes from

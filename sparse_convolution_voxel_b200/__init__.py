@@ -105,7 +105,7 @@ class KernelMap:
         return self.nbr[: self.k3 * self.n_out].view(self.k3, self.n_out).t()
 
 
-def hash_table(coords: torch.Tensor, rsv_ratio: float = 2.0, d_status=None, stream=None) -> torch.Tensor:
+def hash_table(coords: torch.Tensor, rsv_ratio: float = 4.0, d_status=None, stream=None) -> torch.Tensor:
     nbytes = lat_hash_bytes(coords.shape[0], rsv_ratio)
     if nbytes == 0:
         raise LatticeError(1, "lat_hash_bytes")

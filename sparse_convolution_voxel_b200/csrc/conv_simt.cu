@@ -20,8 +20,6 @@
 
 namespace lat {
 
-constexpr int kSimtThreads = 256;
-constexpr int kCoGroup = 8;  // output channels per thread item
 
 template <typename T>
 __device__ __forceinline__ void load8(const T *p, float (&v)[8]);
@@ -68,56 +66,81 @@ __device__ __forceinline__ void store8(T *p, const float (&v)[8]) {
     }
 }
 
-// One tile = LAT_TILE_ROWS rows of perm.  Items (row r, channel group g) are laid
-// out g-major so that a warp holds 32 rows of one channel group: its weight reads
-// are warp-uniform (broadcast) and its feature reads are one row per lane.
+// One block per tile of LAT_TILE_ROWS rows of perm, one thread per row.  For
+// every 32 output channels, each offset of the tile's mask union stages the
+// matching W[k] slice (Cin x 32, fp32) in shared memory; every thread whose row
+// has that neighbour reads its input row (8 channels per vector load) and does
+// 32 FMAs per input channel against warp-uniform (broadcast) weight reads.
 // WT: the weight used at offset k is W[k]^T (data gradient).
+constexpr int kCoChunk = 32;
+
 template <typename T, bool WT>
-__global__ void __launch_bounds__(kSimtThreads)
+__global__ void __launch_bounds__(LAT_TILE_ROWS)
 conv_simt_kernel(const T *__restrict__ x, int cin, const T *__restrict__ w, int cout, MapView mv,
                  T *__restrict__ y, int32_t *d_status) {
-    const int ngroups = cout / kCoGroup;
-    const int items = LAT_TILE_ROWS * ngroups;
-    // weight element (ci, co) of the GEMM at offset k
+    extern __shared__ float s_w[];  // [cin][kCoChunk]
+    const int64_t t = blockIdx.x;
+    const uint32_t tmask = mv.tile_mask_at(t);
+    const int64_t row = t * LAT_TILE_ROWS + threadIdx.x;
+    const int j = row < mv.n_out ? mv.perm[row] : -1;
     const int64_t wk_stride = int64_t(cin) * cout;
     int32_t bad = 0;
-    for (int64_t t = blockIdx.x; t < mv.ntiles; t += gridDim.x) {
-        const uint32_t tmask = mv.tile_mask_at(t);
-        const int64_t row0 = t * LAT_TILE_ROWS;
-        for (int it = threadIdx.x; it < items; it += kSimtThreads) {
-            const int r = it % LAT_TILE_ROWS, g = it / LAT_TILE_ROWS;
-            if (row0 + r >= mv.n_out) continue;
-            const int j = mv.perm[row0 + r];
-            float acc[kCoGroup];
+    for (int co0 = 0; co0 < cout; co0 += kCoChunk) {
+        const int cw = min(kCoChunk, cout - co0);
+        float acc[kCoChunk];
 #pragma unroll
-            for (int c = 0; c < kCoGroup; ++c) acc[c] = 0.f;
-            for (uint32_t m = tmask; m; m &= m - 1) {
-                const int k = __ffs(m) - 1;
-                const int src = mv.neighbour(k, j);
-                if (src < 0) continue;
-                if (src >= mv.n_in) { bad |= LAT_ERR_BAD_MAP; continue; }
-                const T *xr = x + int64_t(src) * cin;
-                const T *wk = w + int64_t(k) * wk_stride;
-                for (int c0 = 0; c0 < cin; c0 += 8) {
-                    float xv[8];
-                    load8<T>(xr + c0, xv);
+        for (int c = 0; c < kCoChunk; ++c) acc[c] = 0.f;
+        for (uint32_t m = tmask; m; m &= m - 1) {
+            const int k = __ffs(m) - 1;
+            int src = j >= 0 ? mv.neighbour(k, j) : -1;
+            if (src >= mv.n_in) {
+                bad |= LAT_ERR_BAD_MAP;
+                src = -1;
+            }
+            const T *wk = w + int64_t(k) * wk_stride;
+            __syncthreads();
+            for (int e = threadIdx.x; e < cin * kCoChunk; e += LAT_TILE_ROWS) {
+                const int ci = e / kCoChunk, c = e % kCoChunk;
+                float v = 0.f;
+                if (c < cw) {
+                    // (ci, co) of the GEMM: W[k][ci][co], or W[k][co][ci] for W^T
+                    v = WT ? Elem<T>::to_f(wk[int64_t(co0 + c) * cin + ci])
+                           : Elem<T>::to_f(wk[int64_t(ci) * cout + co0 + c]);
+                }
+                s_w[e] = v;
+            }
+            __syncthreads();
+            if (src < 0) continue;
+            const T *xr = x + int64_t(src) * cin;
+            for (int c0 = 0; c0 < cin; c0 += 8) {
+                float xv[8];
+                load8<T>(xr + c0, xv);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int ci = c0 + e;
-                        float wv[8];
-                        if constexpr (!WT) {
-                            load8<T>(wk + int64_t(ci) * cout + g * kCoGroup, wv);
-                        } else {  // W^T: element (ci, co) = W[k][co][ci], W[k] is (cout x cin) here
+                for (int e = 0; e < 8; ++e) {
+                    const float4 *wr = reinterpret_cast<const float4 *>(s_w + (c0 + e) * kCoChunk);
 #pragma unroll
-                            for (int c = 0; c < 8; ++c)
-                                wv[c] = Elem<T>::to_f(wk[int64_t(g * kCoGroup + c) * cin + ci]);
-                        }
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) acc[c] = fmaf(xv[e], wv[c], acc[c]);
+                    for (int q = 0; q < kCoChunk / 4; ++q) {
+                        if (4 * q >= cw) break;  // block-uniform: narrow outputs skip the unused columns
+                        const float4 wv = wr[q];
+                        acc[4 * q] = fmaf(xv[e], wv.x, acc[4 * q]);
+                        acc[4 * q + 1] = fmaf(xv[e], wv.y, acc[4 * q + 1]);
+                        acc[4 * q + 2] = fmaf(xv[e], wv.z, acc[4 * q + 2]);
+                        acc[4 * q + 3] = fmaf(xv[e], wv.w, acc[4 * q + 3]);
                     }
                 }
             }
-            store8<T>(y + int64_t(j) * cout + g * kCoGroup, acc);
+        }
+        if (j >= 0) {
+            T *yr = y + int64_t(j) * cout + co0;
+#pragma unroll
+            for (int g = 0; g < kCoChunk / 8; ++g) {
+                if (g * 8 < cw) {
+                    float v[8];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) v[c] = acc[g * 8 + c];
+                    store8<T>(yr + g * 8, v);
+                }
+            }
         }
     }
     if (bad) flag(d_status, bad);
@@ -136,68 +159,95 @@ __global__ void wgrad_units_kernel(const int64_t *__restrict__ pair_off, int k3,
     unit_base[k3] = u;
 }
 
-constexpr int kWgradBatch = 32;
+// One block of 8 warps per (unit, group of slices).  A slice is 256 consecutive
+// elements of the Cin x Cout partial: lane l owns 8 consecutive output channels
+// of one input channel, so for every pair all 32 lanes read the same x row (one
+// value each) and the same dy row (one 32-byte piece each) -- coalesced,
+// broadcast loads -- and do 8 FMAs.  With nslices >= 8 each warp takes one
+// slice over the unit's pairs; with fewer (small Cin x Cout) the warps of a
+// slice split the pairs into parts and add their sums in shared memory in part
+// order.  Pair order and part order are fixed, so each partial is deterministic.
+constexpr int kWgradSlice = 256;
+constexpr int kWgradWarps = 8;
 
 template <typename T>
-__global__ void __launch_bounds__(kSimtThreads)
+__global__ void __launch_bounds__(kWgradWarps * 32)
 wgrad_simt_kernel(const T *__restrict__ x, int cin, const T *__restrict__ dy, int cout, const int64_t *__restrict__ pair_off,
                   const int32_t *__restrict__ pair_in, const int32_t *__restrict__ pair_out, int64_t capacity, int k3,
                   int64_t n_in, int64_t n_out, const int32_t *__restrict__ unit_base, int chunk, float *__restrict__ partial,
                   int32_t *d_status) {
-    extern __shared__ float smem[];
-    float *xs = smem;                       // [kWgradBatch][cin]
-    float *gs = smem + kWgradBatch * cin;   // [kWgradBatch][cout]
+    __shared__ float s_part[kWgradWarps][kWgradSlice];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nelem = cin * cout;
-    const int32_t units = unit_base[k3];
-    int32_t bad = 0;
-    for (int32_t u = blockIdx.x; u < units; u += gridDim.x) {
+    const int nslices = (nelem + kWgradSlice - 1) / kWgradSlice;
+    // warps per slice (parts of the pair range) and slices per block
+    const int parts = nslices >= kWgradWarps ? 1 : (kWgradWarps % nslices == 0 ? kWgradWarps / nslices : 1);
+    const int per_block = kWgradWarps / parts;
+    const int groups = (nslices + per_block - 1) / per_block;
+    const int32_t u = int32_t(blockIdx.x / groups);
+    const int slice = int(blockIdx.x % groups) * per_block + warp / parts;
+    const int part = warp % parts;
+    const bool unit_ok = u < unit_base[k3];
+    const int e0 = slice * kWgradSlice + lane * 8;
+    const bool own = unit_ok && slice < nslices && e0 < nelem;
+    const int ci = own ? e0 / cout : 0, co0 = own ? e0 % cout : 0;
+    int64_t lo = 0, hi = 0;
+    if (unit_ok) {
         int k = 0;
         while (unit_base[k + 1] <= u) ++k;
-        const int64_t lo = min(pair_off[k], capacity) + int64_t(u - unit_base[k]) * chunk;
-        const int64_t hi = min(lo + chunk, min(pair_off[k + 1], capacity));
-        float acc[64];  // up to 256*256/256 elements per thread would not fit; cap nelem/threads at 64
-        const int per = (nelem + kSimtThreads - 1) / kSimtThreads;
+        const int64_t ulo = min(pair_off[k], capacity) + int64_t(u - unit_base[k]) * chunk;
+        const int64_t uhi = min(ulo + chunk, min(pair_off[k + 1], capacity));
+        const int64_t per = (uhi - ulo + parts - 1) / parts;
+        lo = min(uhi, ulo + per * part);
+        hi = min(uhi, lo + per);
+    }
+    float acc[8];
 #pragma unroll
-        for (int e = 0; e < 64; ++e) acc[e] = 0.f;
-        for (int64_t p0 = lo; p0 < hi; p0 += kWgradBatch) {
-            const int np = int(hi - p0 < kWgradBatch ? hi - p0 : int64_t(kWgradBatch));
-            __syncthreads();
-            for (int idx = threadIdx.x; idx < kWgradBatch * (cin + cout); idx += kSimtThreads) {
-                const int p = idx / (cin + cout), c = idx % (cin + cout);
-                float v = 0.f;
-                if (p < np) {
-                    if (c < cin) {
-                        const int i = pair_in[p0 + p];
-                        if (i >= 0 && i < n_in) v = Elem<T>::to_f(x[int64_t(i) * cin + c]);
-                        else bad |= LAT_ERR_BAD_MAP;
-                    } else {
-                        const int j = pair_out[p0 + p];
-                        if (j >= 0 && j < n_out) v = Elem<T>::to_f(dy[int64_t(j) * cout + (c - cin)]);
-                        else bad |= LAT_ERR_BAD_MAP;
+    for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+    int32_t bad = 0;
+    if (own) {
+        for (int64_t p0 = lo; p0 < hi; p0 += 4) {
+            float xv[4], gv[4][8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int64_t p = p0 + q;
+                int i = -1, jj = -1;
+                if (p < hi) {
+                    i = __ldg(pair_in + p);
+                    jj = __ldg(pair_out + p);
+                    if (i < 0 || i >= n_in || jj < 0 || jj >= n_out) {
+                        bad |= LAT_ERR_BAD_MAP;
+                        i = jj = -1;
                     }
                 }
-                if (c < cin) xs[p * cin + c] = v; else gs[p * cout + (c - cin)] = v;
-            }
-            __syncthreads();
+                xv[q] = 0.f;
 #pragma unroll
-            for (int e = 0; e < 64; ++e) {
-                if (e >= per) break;
-                const int el = threadIdx.x + e * kSimtThreads;
-                if (el >= nelem) break;
-                const int ci = el / cout, co = el % cout;
-                float a = acc[e];
-                for (int p = 0; p < np; ++p) a = fmaf(xs[p * cin + ci], gs[p * cout + co], a);
-                acc[e] = a;
+                for (int c = 0; c < 8; ++c) gv[q][c] = 0.f;
+                if (i >= 0) {
+                    xv[q] = Elem<T>::to_f(x[int64_t(i) * cin + ci]);
+                    load8<T>(dy + int64_t(jj) * cout + co0, gv[q]);
+                }
             }
-        }
-        float *dst = partial + int64_t(u) * nelem;
 #pragma unroll
-        for (int e = 0; e < 64; ++e) {
-            if (e >= per) break;
-            const int el = threadIdx.x + e * kSimtThreads;
-            if (el < nelem) dst[el] = acc[e];
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int c = 0; c < 8; ++c) acc[c] = fmaf(xv[q], gv[q][c], acc[c]);
         }
+    }
+    if (parts > 1) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) s_part[warp][lane * 8 + c] = acc[c];
         __syncthreads();
+        if (part == 0 && own) {
+            for (int q = 1; q < parts; ++q)
+#pragma unroll
+                for (int c = 0; c < 8; ++c) acc[c] += s_part[warp + q][lane * 8 + c];
+        }
+    }
+    if (own && part == 0) {
+        float *dst = partial + int64_t(u) * nelem + e0;
+        reinterpret_cast<float4 *>(dst)[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        reinterpret_cast<float4 *>(dst)[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
     if (bad) flag(d_status, bad);
 }
@@ -227,12 +277,13 @@ template <typename T>
 lat_status launch_conv_simt(const void *x, int cin, const void *w, int cout, const MapView &mv, bool wt, void *y,
                             int32_t *d_status, cudaStream_t s) {
     if (mv.ntiles == 0) return LAT_OK;
-    const int64_t grid = std::min<int64_t>(mv.ntiles, int64_t(num_sms()) * 8);
+    if (mv.ntiles >= (int64_t(1) << 31)) return LAT_ERR_UNSUPPORTED;
+    const size_t smem = sizeof(float) * size_t(cin) * kCoChunk;
     if (wt)
-        conv_simt_kernel<T, true><<<unsigned(grid), kSimtThreads, 0, s>>>(
+        conv_simt_kernel<T, true><<<unsigned(mv.ntiles), LAT_TILE_ROWS, smem, s>>>(
             static_cast<const T *>(x), cin, static_cast<const T *>(w), cout, mv, static_cast<T *>(y), d_status);
     else
-        conv_simt_kernel<T, false><<<unsigned(grid), kSimtThreads, 0, s>>>(
+        conv_simt_kernel<T, false><<<unsigned(mv.ntiles), LAT_TILE_ROWS, smem, s>>>(
             static_cast<const T *>(x), cin, static_cast<const T *>(w), cout, mv, static_cast<T *>(y), d_status);
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
@@ -248,16 +299,18 @@ template lat_status launch_conv_simt<__nv_bfloat16>(const void *, int, const voi
 template <typename T>
 lat_status launch_wgrad_simt(const void *x, int cin, const void *dy, int cout, const lat_kmap *map, float *dw,
                              void *ws, int32_t *d_status, cudaStream_t s) {
-    if (cin * cout > 64 * kSimtThreads) return LAT_ERR_UNSUPPORTED;
     const int64_t units_max = (map->pair_capacity + kWgradChunkSimt - 1) / kWgradChunkSimt + map->k3;
     Carver cv(ws);
     int32_t *unit_base = cv.take<int32_t>(size_t(map->k3) + 1);
     float *partial = cv.take<float>(size_t(units_max) * cin * cout);
     wgrad_units_kernel<<<1, 32, 0, s>>>(map->pair_off, map->k3, map->pair_capacity, kWgradChunkSimt, unit_base);
     LAT_CUDA_TRY(cudaGetLastError());
-    const size_t smem = sizeof(float) * kWgradBatch * (cin + cout);
-    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(units_max, int64_t(num_sms()) * 4));
-    wgrad_simt_kernel<T><<<unsigned(grid), kSimtThreads, smem, s>>>(
+    const int64_t nslices = (int64_t(cin) * cout + kWgradSlice - 1) / kWgradSlice;
+    const int64_t parts = nslices >= kWgradWarps ? 1 : (kWgradWarps % nslices == 0 ? kWgradWarps / nslices : 1);
+    const int64_t per_block = kWgradWarps / parts;
+    const int64_t grid = units_max * ((nslices + per_block - 1) / per_block);
+    if (grid >= (int64_t(1) << 31)) return LAT_ERR_UNSUPPORTED;
+    wgrad_simt_kernel<T><<<unsigned(grid), kWgradWarps * 32, 0, s>>>(
         static_cast<const T *>(x), cin, static_cast<const T *>(dy), cout, map->pair_off, map->pair_in, map->pair_out,
         map->pair_capacity, map->k3, map->n_in, map->n_out, unit_base, kWgradChunkSimt, partial, d_status);
     LAT_CUDA_TRY(cudaGetLastError());
