@@ -371,6 +371,7 @@ def run_only(args):
     coarse = torch.empty((n * 8, 4), dtype=torch.int32, device=dev)
     parent = torch.empty(n, dtype=torch.int32, device=dev)
     wsb = ws.get(max(scv.lat_kmap_ws_bytes(n, k3), scv.lat_sconv_ws_bytes(2, cin, cout, km.c, dt),
+                     scv.lat_sconv_ws_bytes(0, cin, cout, km.c, dt), scv.lat_sconv_ws_bytes(1, cin, cout, km.c, dt),
                      scv.lat_downsample_ws_bytes(n, scv.strided_geom(2, 2, 0))))
     torch.cuda.synchronize()
     P = int(km.pair_off[k3].item())

@@ -221,7 +221,12 @@ lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int32_t *paren
  * fixed relation and weight tensor).  cin and cout must be multiples of 8 and
  * at most 256.  fp16 / bf16 with cin, cout in {64, 128} run on the tcgen05
  * tensor cores (fp32 accumulate in TMEM); other shapes and fp32 run on CUDA
- * cores (FFMA, no TF32). */
+ * cores (FFMA, no TF32).
+ * Workspace: the tensor-core forward and data-gradient passes take 256 bytes
+ * (a tile counter, cleared on `stream` before the kernel); the CUDA-core
+ * passes take none.  lat_sconv_ws_bytes gives the size for each op; a call
+ * with less returns LAT_ERR_WORKSPACE.  Two calls must not share a workspace
+ * while both can run (different streams). */
 size_t lat_sconv_ws_bytes(int32_t op, int32_t cin, int32_t cout, const lat_kmap *map,
                           lat_dtype dtype);
 #define LAT_OP_FWD 0

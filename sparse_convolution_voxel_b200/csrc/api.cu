@@ -37,6 +37,9 @@ extern "C" size_t lat_sconv_ws_bytes(int32_t op, int32_t cin, int32_t cout, cons
     if (op == LAT_OP_WGRAD)
         return (dtype != LAT_F32 && lat::wgrad_tc_supported(cin, cout)) ? lat::wgrad_tc_ws_bytes(cin, cout, map)
                                                                         : lat::wgrad_simt_ws_bytes(cin, cout, map);
+    // forward gathers cin channels into cout; the data gradient gathers cout into cin
+    if (op == LAT_OP_FWD) return (dtype != LAT_F32 && lat::conv_tc_supported(cin, cout)) ? lat::conv_tc_ws_bytes() : 0;
+    if (op == LAT_OP_DGRAD) return (dtype != LAT_F32 && lat::conv_tc_supported(cout, cin)) ? lat::conv_tc_ws_bytes() : 0;
     return 0;
 }
 
@@ -44,15 +47,15 @@ extern "C" lat_status lat_sconv_fwd(const void *x, int32_t cin, const void *w, i
                                     void *y, lat_dtype dtype, void *ws, size_t ws_bytes, int32_t *d_status,
                                     lat_stream stream) {
     using namespace lat;
-    (void)ws;
-    (void)ws_bytes;
     if (!map_ok(map) || !chan_ok(cin, dtype) || !chan_ok(cout, dtype)) return LAT_ERR_ARG;
     if (map->n_out > 0 && (!y || !w || (map->n_in > 0 && !x))) return LAT_ERR_ARG;
     if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return LAT_ERR_ARG;
     const MapView mv = make_view(map, false);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (dtype != LAT_F32 && conv_tc_supported(cin, cout))
-        return launch_conv_tc(dtype == LAT_BF16, x, cin, w, cout, map->k3, mv, false, y, d_status, s);
+    if (dtype != LAT_F32 && conv_tc_supported(cin, cout)) {
+        if (!ws || ws_bytes < conv_tc_ws_bytes()) return LAT_ERR_WORKSPACE;
+        return launch_conv_tc(dtype == LAT_BF16, x, cin, w, cout, map->k3, mv, false, y, ws, d_status, s);
+    }
     return by_dtype(dtype, [&](auto t) {
         using T = decltype(t);
         return launch_conv_simt<T>(x, cin, w, cout, mv, false, y, d_status, s);
@@ -63,8 +66,6 @@ extern "C" lat_status lat_sconv_dgrad(const void *dy, int32_t cout, const void *
                                       int32_t flip_offsets, void *dx, lat_dtype dtype, void *ws, size_t ws_bytes,
                                       int32_t *d_status, lat_stream stream) {
     using namespace lat;
-    (void)ws;
-    (void)ws_bytes;
     if (!map_ok(map) || !chan_ok(cin, dtype) || !chan_ok(cout, dtype)) return LAT_ERR_ARG;
     if (flip_offsets && map->n_in != map->n_out) return LAT_ERR_ARG;
     if (map->n_out > 0 && (!dx || !w || (map->n_in > 0 && !dy))) return LAT_ERR_ARG;
@@ -72,8 +73,10 @@ extern "C" lat_status lat_sconv_dgrad(const void *dy, int32_t cout, const void *
     const MapView mv = make_view(map, flip_offsets != 0);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // the pass gathers dy rows (cout channels) and produces dx rows (cin channels) with W[k]^T
-    if (dtype != LAT_F32 && conv_tc_supported(cout, cin))
-        return launch_conv_tc(dtype == LAT_BF16, dy, cout, w, cin, map->k3, mv, true, dx, d_status, s);
+    if (dtype != LAT_F32 && conv_tc_supported(cout, cin)) {
+        if (!ws || ws_bytes < conv_tc_ws_bytes()) return LAT_ERR_WORKSPACE;
+        return launch_conv_tc(dtype == LAT_BF16, dy, cout, w, cin, map->k3, mv, true, dx, ws, d_status, s);
+    }
     return by_dtype(dtype, [&](auto t) {
         using T = decltype(t);
         return launch_conv_simt<T>(dy, cout, w, cin, mv, true, dx, d_status, s);

@@ -25,6 +25,10 @@ struct MapView {
         const uint32_t m = tile_mask[t];
         return flip ? (__brev(m) >> (32 - k3)) : m;
     }
+    __device__ __forceinline__ const int32_t *neighbour_ptr(int k, int64_t j) const {
+        const int kk = flip ? (k3 - 1 - k) : k;
+        return nbr + int64_t(kk) * n_out + j;
+    }
     __device__ __forceinline__ int neighbour(int k, int64_t j) const {
         const int kk = flip ? (k3 - 1 - k) : k;
         return __ldg(nbr + int64_t(kk) * n_out + j);
@@ -57,7 +61,8 @@ bool wgrad_tc_supported(int cin, int cout);
 size_t wgrad_tc_ws_bytes(int cin, int cout, const lat_kmap *map);
 lat_status launch_wgrad_tc(bool bf16, const void *x, int cin, const void *dy, int cout, const lat_kmap *map, float *dw,
                            void *ws, int32_t *d_status, cudaStream_t s);
+size_t conv_tc_ws_bytes();
 lat_status launch_conv_tc(bool bf16, const void *x, int kc, const void *w, int n, int k3, const MapView &mv, bool wt,
-                          void *y, int32_t *d_status, cudaStream_t s);
+                          void *y, void *ws, int32_t *d_status, cudaStream_t s);
 
 }  // namespace lat

@@ -3,11 +3,14 @@
 // Output-stationary implicit GEMM (TorchSparse++ abstract: implicit GEMM
 // overlaps computation and memory access; the migration page's "Backend and
 // configuration differences" requires every dataflow to give the same result
-// for a fixed relation and weight tensor).  One persistent CTA per SM walks
-// 128-row tiles of the mask-sorted output order; for every offset in a
-// tile's mask union and every 64-channel K block it
+// for a fixed relation and weight tensor).  Persistent CTAs (two per SM) take
+// 128-row tiles of the mask-sorted output order from a device-wide counter,
+// heaviest tiles first; for every offset in a tile's mask union and every
+// 64-channel K block a CTA
 //   - gathers the 128 neighbour rows with 16-byte cp.async into a 128-byte
-//     swizzled K-major tile (absent neighbours are zero-filled, no read),
+//     swizzled K-major tile (absent neighbours are zero-filled, no read);
+//     each gather thread's copies arrive on the stage barrier by themselves
+//     (cp.async.mbarrier.arrive.noinc), so the thread never waits for them,
 //   - loads the W[k] slab with TMA (128-byte swizzle, no multicast),
 //   - issues 4 tcgen05.mma (M=128, N=Cout, K=16) into a TMEM accumulator.
 // Epilogue warps read the accumulator with tcgen05.ld, round once to the
@@ -15,8 +18,12 @@
 // accumulator is double buffered in TMEM so the epilogue of tile t overlaps
 // the main loop of tile t+1.
 //
-// Roles (288 threads): warps 0-3 gather (thread 0 also issues TMA), warps 4-7
-// epilogue (warp w reads TMEM lanes 32*(w%4)..+31), warp 8 lane 0 issues MMAs.
+// Roles (320 threads): warps 0-3 gather (thread 0 also issues TMA), warps 4-7
+// epilogue (warp w reads TMEM lanes 32*(w%4)..+31), warp 8 lane 0 issues MMAs,
+// warp 9 claims tiles and publishes (tile, mask union, output rows) in a ring
+// of shared-memory entries that the other roles read in order.  The rows are
+// sorted by neighbour count (ascending), so walking the tiles backwards hands
+// out the long tiles first and the one-offset tiles fill the gaps.
 // Every mbarrier wait is bounded; a wait that gives up flags LAT_ERR_TIMEOUT
 // and the CTA drains and exits, releasing its TMEM.
 //
@@ -38,20 +45,45 @@ constexpr int kM = 128;          // tile rows = MMA M
 constexpr int kProdWarps = 4;    // gather warps
 constexpr int kEpiWarps = 4;     // epilogue warps
 constexpr int kMmaWarp = kProdWarps + kEpiWarps;
-constexpr int kThreads = (kMmaWarp + 1) * 32;
-constexpr int kLag = 2;          // cp.async groups a gather thread keeps in flight
-constexpr int kIdxBatch = 8;     // neighbour indices a gather thread loads at once
+constexpr int kSchedWarp = kMmaWarp + 1;
+constexpr int kThreads = (kSchedWarp + 1) * 32;
+constexpr int kRing = 8;         // tile entries in flight between the scheduler and the other roles
+constexpr int kItems = 16;       // (tile, offset) items in flight between the scheduler and the gather warps
 constexpr uint32_t kABytes = kM * 128;  // 128 rows x 64 channels x 2 bytes
 constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+// One claimed tile as the scheduler publishes it.
+struct TileEntry {
+    int32_t tile;      // tile index, -1 = no more tiles for this CTA
+    uint32_t mask;     // union of the tile rows' offset masks (flipped for a flipped map)
+    int32_t pad[2];
+    int32_t rows[kM];  // output row of every tile row, -1 past n_out
+};
+
+// One (tile, offset) item: the offset and the source row of every tile row,
+// as the scheduler warp publishes it for the gather warps.
+struct ItemEntry {
+    int32_t k;         // offset, -1 = no more items for this CTA
+    int32_t pad[3];
+    int32_t src[kM];   // input row gathered into each tile row, -1 = none (zero row)
+};
 
 template <int N>
 struct Cfg {
     static constexpr uint32_t kBBytes = uint32_t(N) * 128;  // 64 K x N (or N x 64) x 2 bytes
     static constexpr uint32_t kStage = kABytes + kBBytes;
-    static constexpr int kStages = N == 64 ? 4 : 3;  // ~96 KB: two CTAs per SM
-    static constexpr uint32_t kBarBytes = 256;
-    static constexpr uint32_t kSmem = kStages * kStage + kBarBytes + 1024;
+    static constexpr int kStages = N == 64 ? 4 : 3;  // ~100 KB: two CTAs per SM
+    static constexpr uint32_t kRingOff = kStages * kStage;
+    static constexpr uint32_t kItemOff = kRingOff + kRing * sizeof(TileEntry);
+    static constexpr uint32_t kBarOff = kItemOff + kItems * sizeof(ItemEntry);
+    static constexpr uint32_t kBarBytes = 1024;
+    static constexpr uint32_t kSmem = kBarOff + kBarBytes + 1024;
     static constexpr uint32_t kTmemCols = 2 * N;
+    // the scheduler can run ahead of the slowest reader (the epilogue) by at
+    // most stages + 2 tiles; the ring must be deeper than that
+    static_assert(kRing >= kStages + 3, "tile ring too shallow");
+    static_assert((2 * kStages + 4 + 2 * kRing + 2 * kItems) * 8 + 4 <= kBarBytes, "barrier area");
 };
 
 template <typename T> constexpr bool is_bf16() { return sizeof(T) == 2 && !std::is_same<T, __half>::value; }
@@ -77,10 +109,11 @@ __device__ __forceinline__ uint32_t pack2(float a, float b, __nv_bfloat16) {
 }
 
 // KC: gathered channels (GEMM K), N: output channels, BMN: B operand MN-major.
+// tile_counter: zero at launch; CTAs claim tiles past the first gridDim.x from it.
 template <typename T, int KC, int N, bool BMN>
 __global__ void __launch_bounds__(kThreads, 2)
 conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x, MapView mv, T *__restrict__ y,
-               int32_t *d_status) {
+               int32_t *tile_counter, int32_t *d_status) {
     using C = Cfg<N>;
     constexpr int NS = C::kStages;
     constexpr int KBLK = KC / 64;
@@ -88,22 +121,37 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + NS * C::kStage);
+    TileEntry *ring = reinterpret_cast<TileEntry *>(smem + C::kRingOff);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
     uint64_t *empty = full + NS;
     uint64_t *accfull = empty + NS;
     uint64_t *accempty = accfull + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accempty + 2);
+    uint64_t *ring_full = accempty + 2;
+    uint64_t *ring_empty = ring_full + kRing;
+    uint64_t *item_full = ring_empty + kRing;
+    uint64_t *item_empty = item_full + kItems;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(item_empty + kItems);
+    ItemEntry *items = reinterpret_cast<ItemEntry *>(smem + C::kItemOff);
     __shared__ int s_abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
+            // 128 gather threads' copy completions + the weight thread's expect_tx
             ptx::mbar_init(&full[s], kProdWarps * 32 + 1);
             ptx::mbar_init(&empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
             ptx::mbar_init(&accfull[a], 1);
             ptx::mbar_init(&accempty[a], kEpiWarps * 32);
+        }
+        for (int r = 0; r < kRing; ++r) {
+            ptx::mbar_init(&ring_full[r], 32);
+            ptx::mbar_init(&ring_empty[r], 1 + kEpiWarps * 32);  // MMA thread + epilogue threads
+        }
+        for (int r = 0; r < kItems; ++r) {
+            ptx::mbar_init(&item_full[r], 64);  // 32 index-copy completions + 32 plain arrivals
+            ptx::mbar_init(&item_empty[r], kProdWarps * 32);
         }
         s_abort = 0;
         ptx::fence_mbar_init();
@@ -122,95 +170,73 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x
 
     if (warp < kProdWarps) {
         // ------------------------------------------------------------ gather + TMA
-        // Thread tid owns tile row tid: its output row (perm) is fetched one tile
-        // ahead, and the input rows of up to kIdxBatch offsets are fetched together,
-        // so the index loads overlap instead of stalling each copy.
+        // Thread tid owns tile row tid; its source row of every item comes
+        // from the item ring, so no global index load sits on this path.
         uint32_t it = 0;
         bool ok = true;
-        int64_t t = blockIdx.x;
-        int j_next = (t < mv.ntiles && t * kM + tid < mv.n_out) ? __ldg(mv.perm + t * kM + tid) : -1;
-        for (; t < mv.ntiles && ok; t += gridDim.x) {
-            const uint32_t tm = mv.tile_mask_at(t);
-            const int j_own = j_next;
-            const int64_t tn = t + gridDim.x;
-            j_next = (tn < mv.ntiles && tn * kM + tid < mv.n_out) ? __ldg(mv.perm + tn * kM + tid) : -1;
-            uint32_t rem = tm;
-            while (rem && ok) {
-                int kk[kIdxBatch], src_b[kIdxBatch];
+        for (int ii = 0; ok; ++ii) {
+            const int r = ii % kItems;
+            if (!__all_sync(kFull, ptx::mbar_wait(&item_full[r], (ii / kItems) & 1, kWaitNs))) {
+                ok = false;
+                break;
+            }
+            const int k = items[r].k;
+            int src_own = items[r].src[tid];
+            ptx::mbar_arrive(&item_empty[r]);
+            if (k < 0) break;
+            if (src_own >= mv.n_in) {
+                bad |= LAT_ERR_BAD_MAP;
+                src_own = -1;
+            }
+            for (int kb = 0; kb < KBLK; ++kb) {
+                const uint32_t s = it % NS;
+                if (!__all_sync(kFull, ptx::mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, kWaitNs))) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *As = smem + s * C::kStage;
+                uint8_t *Bs = As + kABytes;
+                if (tid == 0) {
+                    ptx::mbar_arrive_expect_tx(&full[s], C::kBBytes);
 #pragma unroll
-                for (int e = 0; e < kIdxBatch; ++e) {
-                    kk[e] = -1;
-                    src_b[e] = -1;
-                    if (rem) {
-                        kk[e] = __ffs(rem) - 1;
-                        rem &= rem - 1;
-                        if (j_own >= 0) src_b[e] = mv.neighbour(kk[e], j_own);
+                    for (int nb = 0; nb < N / 64; ++nb) {
+                        if constexpr (BMN)  // rows k*KC + 64kb.., columns 64nb..
+                            ptx::tma_load_2d(Bs + nb * 8192, &wmap, &full[s], 64 * nb, k * KC + 64 * kb);
+                        else                // rows k*N + 64nb.., columns 64kb..
+                            ptx::tma_load_2d(Bs + nb * 8192, &wmap, &full[s], 64 * kb, k * N + 64 * nb);
                     }
                 }
 #pragma unroll
-                for (int e = 0; e < kIdxBatch; ++e) {
-                    if (kk[e] < 0 || !ok) continue;
-                    const int k = kk[e];
-                    int src_own = src_b[e];
-                    if (src_own >= mv.n_in) {
-                        bad |= LAT_ERR_BAD_MAP;
-                        src_own = -1;
-                    }
-                    for (int kb = 0; kb < KBLK; ++kb) {
-                        const uint32_t s = it % NS;
-                        if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, kWaitNs))) {
-                            ok = false;
-                            break;
-                        }
-                        uint8_t *As = smem + s * C::kStage;
-                        uint8_t *Bs = As + kABytes;
-                        if (tid == 0) {
-                            ptx::mbar_arrive_expect_tx(&full[s], C::kBBytes);
-#pragma unroll
-                            for (int nb = 0; nb < N / 64; ++nb) {
-                                if constexpr (BMN)  // rows k*KC + 64kb.., columns 64nb..
-                                    ptx::tma_load_2d(Bs + nb * 8192, &wmap, &full[s], 64 * nb, k * KC + 64 * kb);
-                                else                // rows k*N + 64nb.., columns 64kb..
-                                    ptx::tma_load_2d(Bs + nb * 8192, &wmap, &full[s], 64 * kb, k * N + 64 * nb);
-                            }
-                        }
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int rl = 4 * i + (lane >> 3);
-                            const int row = warp * 32 + rl;
-                            const int chunk = lane & 7;
-                            const int src = __shfl_sync(0xFFFFFFFFu, src_own, rl);
-                            const T *gp = src >= 0 ? x + int64_t(src) * KC + kb * 64 + chunk * 8 : x;
-                            ptx::cp_async16(As + row * 128 + ((chunk ^ (row & 7)) << 4), gp, src >= 0 ? 16u : 0u);
-                        }
-                        ptx::cp_async_commit();
-                        if (it >= kLag) {
-                            ptx::cp_async_wait<kLag>();
-                            ptx::fence_proxy_async_smem();
-                            ptx::mbar_arrive(&full[(it - kLag) % NS]);
-                        }
-                        ++it;
-                    }
+                for (int i = 0; i < 8; ++i) {
+                    const int rl = 4 * i + (lane >> 3);
+                    const int row = warp * 32 + rl;
+                    const int chunk = lane & 7;
+                    const int src = __shfl_sync(kFull, src_own, rl);
+                    const T *gp = src >= 0 ? x + int64_t(src) * KC + kb * 64 + chunk * 8 : x;
+                    ptx::cp_async16(As + row * 128 + ((chunk ^ (row & 7)) << 4), gp, src >= 0 ? 16u : 0u);
                 }
+                ptx::cp_async_arrive_noinc(&full[s]);
+                ++it;
             }
         }
         ptx::cp_async_wait<0>();
-        ptx::fence_proxy_async_smem();
-        for (uint32_t d = (it > kLag ? it - kLag : 0); d < it; ++d) ptx::mbar_arrive(&full[d % NS]);
         if (!ok) s_abort = 1;
     } else if (warp < kMmaWarp) {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;
         uint32_t ta = 0;
         bool ok = true;
-        int64_t t = blockIdx.x;
-        int j_next = (t < mv.ntiles && t * kM + q * 32 + lane < mv.n_out) ? __ldg(mv.perm + t * kM + q * 32 + lane) : -1;
-        for (; t < mv.ntiles && ok; t += gridDim.x) {
-            const uint32_t tm = mv.tile_mask_at(t);
-            const int j = j_next;
-            const int64_t tn = t + gridDim.x;
-            j_next = (tn < mv.ntiles && tn * kM + q * 32 + lane < mv.n_out) ? __ldg(mv.perm + tn * kM + q * 32 + lane)
-                                                                             : -1;
+        for (int ri = 0; ok; ++ri) {
+            const int r = ri % kRing;
+            if (!__all_sync(kFull, ptx::mbar_wait(&ring_full[r], (ri / kRing) & 1, kWaitNs))) {
+                ok = false;
+                break;
+            }
+            const int t = ring[r].tile;
+            const uint32_t tm = ring[r].mask;
+            const int j = t >= 0 ? ring[r].rows[q * 32 + lane] : -1;
+            ptx::mbar_arrive(&ring_empty[r]);
+            if (t < 0) break;
             T *yr = j >= 0 ? y + int64_t(j) * N : nullptr;
             if (!tm) {  // no neighbour anywhere in the tile: zeros
                 if (yr)
@@ -219,7 +245,7 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x
                 continue;
             }
             const uint32_t a = ta & 1;
-            if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(&accfull[a], (ta >> 1) & 1, kWaitNs))) {
+            if (!__all_sync(kFull, ptx::mbar_wait(&accfull[a], (ta >> 1) & 1, kWaitNs))) {
                 ok = false;
                 break;
             }
@@ -250,47 +276,149 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x
             ++ta;
         }
         if (!ok) s_abort = 1;
-    } else if (lane == 0) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issue
-        uint32_t it = 0, ta = 0;
+        if (lane == 0) {
+            uint32_t it = 0, ta = 0;
+            bool ok = true;
+            for (int ri = 0; ok; ++ri) {
+                const int r = ri % kRing;
+                if (!ptx::mbar_wait(&ring_full[r], (ri / kRing) & 1, kWaitNs)) {
+                    ok = false;
+                    break;
+                }
+                const int t = ring[r].tile;
+                const uint32_t tm = ring[r].mask;
+                ptx::mbar_arrive(&ring_empty[r]);
+                if (t < 0) break;
+                if (!tm) continue;
+                const uint32_t a = ta & 1;
+                if (!ptx::mbar_wait(&accempty[a], ((ta >> 1) & 1) ^ 1, kWaitNs)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t dcol = tmem_base + a * N;
+                uint32_t acc = 0;
+                for (uint32_t m = tm; m && ok; m &= m - 1) {
+                    for (int kb = 0; kb < KBLK; ++kb) {
+                        const uint32_t s = it % NS;
+                        if (!ptx::mbar_wait(&full[s], (it / NS) & 1, kWaitNs)) {
+                            ok = false;
+                            break;
+                        }
+                        ptx::tc_fence_after();
+                        // the gathered rows were written by cp.async (generic proxy);
+                        // order them before the tensor core's async-proxy reads
+                        ptx::fence_proxy_async_smem();
+                        const uint32_t as = ptx::smem_u32(smem + s * C::kStage);
+                        const uint32_t bs = as + kABytes;
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks) {
+                            const uint64_t ad = ptx::desc_sw128(as + ks * 32, 16, 1024);
+                            const uint64_t bd = BMN ? ptx::desc_sw128(bs + ks * 2048, 8192, 1024)
+                                                    : ptx::desc_sw128(bs + ks * 32, 16, 1024);
+                            ptx::umma_f16(dcol, ad, bd, idesc, acc);
+                            acc = 1;
+                        }
+                        ptx::umma_commit(&empty[s]);
+                        ++it;
+                    }
+                }
+                if (!ok) break;
+                ptx::umma_commit(&accfull[a]);
+                ++ta;
+            }
+            if (!ok) s_abort = 1;
+        }
+    } else {
+        // ------------------------------------------------------------ tile scheduler + neighbour indices
+        // Claim order q = 0, 1, ...: q < gridDim.x is CTA q's first tile, later q
+        // come from the counter; tile = ntiles-1-q (heaviest first).  The mask and
+        // output rows of a tile are loaded two tiles ahead; the neighbour indices
+        // are copied into the item ring with cp.async, whose completion the item
+        // barrier tracks, so this warp never waits for index data.
         bool ok = true;
-        for (int64_t t = blockIdx.x; t < mv.ntiles && ok; t += gridDim.x) {
-            const uint32_t tm = mv.tile_mask_at(t);
-            if (!tm) continue;
-            const uint32_t a = ta & 1;
-            if (!ptx::mbar_wait(&accempty[a], ((ta >> 1) & 1) ^ 1, kWaitNs)) {
+        int ii = 0;  // items published
+        auto fetch = [&](int64_t q, int64_t &t, uint32_t &tm, int (&rows)[4]) {
+            t = q < mv.ntiles ? mv.ntiles - 1 - q : -1;
+            tm = t >= 0 ? mv.tile_mask_at(t) : 0u;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int64_t row = t * kM + e * 32 + lane;
+                rows[e] = (t >= 0 && row < mv.n_out) ? __ldg(mv.perm + row) : -1;
+            }
+        };
+        auto push_item = [&](int k, const int (&rows)[4]) -> bool {
+            const int r = ii % kItems;
+            if (!__all_sync(kFull, ptx::mbar_wait(&item_empty[r], ((ii / kItems) & 1) ^ 1, kWaitNs))) return false;
+            if (lane == 0) items[r].k = k;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                int32_t *dst = &items[r].src[e * 32 + lane];
+                if (k >= 0 && rows[e] >= 0)
+                    ptx::cp_async4(dst, mv.neighbour_ptr(k, rows[e]));
+                else
+                    *dst = -1;
+            }
+            ptx::cp_async_arrive_noinc(&item_full[r]);
+            ptx::mbar_arrive(&item_full[r]);
+            ++ii;
+            return true;
+        };
+        // tile 0 is static; the claim for tile 1 is in flight while tile 0's rows load
+        int claimed = lane == 0 ? atomicAdd(tile_counter, 1) : 0;
+        int64_t t_c, t_n;
+        uint32_t m_c, m_n;
+        int r_c[4], r_n[4];
+        fetch(blockIdx.x, t_c, m_c, r_c);
+        if (t_c >= 0) {
+            fetch(int64_t(gridDim.x) + __shfl_sync(kFull, claimed, 0), t_n, m_n, r_n);
+            if (lane == 0) claimed = atomicAdd(tile_counter, 1);
+        } else {
+            t_n = -1;
+            m_n = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) r_n[e] = -1;
+        }
+        for (int i = 0; ok; ++i) {
+            // publish tile i for the MMA and epilogue roles
+            const int r = i % kRing;
+            if (!__all_sync(kFull, ptx::mbar_wait(&ring_empty[r], ((i / kRing) & 1) ^ 1, kWaitNs))) {
                 ok = false;
                 break;
             }
-            ptx::tc_fence_after();
-            const uint32_t dcol = tmem_base + a * N;
-            uint32_t acc = 0;
-            for (uint32_t m = tm; m && ok; m &= m - 1) {
-                for (int kb = 0; kb < KBLK; ++kb) {
-                    const uint32_t s = it % NS;
-                    if (!ptx::mbar_wait(&full[s], (it / NS) & 1, kWaitNs)) {
-                        ok = false;
-                        break;
-                    }
-                    ptx::tc_fence_after();
-                    const uint32_t as = ptx::smem_u32(smem + s * C::kStage);
-                    const uint32_t bs = as + kABytes;
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t ad = ptx::desc_sw128(as + ks * 32, 16, 1024);
-                        const uint64_t bd = BMN ? ptx::desc_sw128(bs + ks * 2048, 8192, 1024)
-                                                : ptx::desc_sw128(bs + ks * 32, 16, 1024);
-                        ptx::umma_f16(dcol, ad, bd, idesc, acc);
-                        acc = 1;
-                    }
-                    ptx::umma_commit(&empty[s]);
-                    ++it;
-                }
+            for (int e = 0; e < 4; ++e) ring[r].rows[e * 32 + lane] = r_c[e];
+            if (lane == 0) {
+                ring[r].tile = int32_t(t_c);
+                ring[r].mask = m_c;
             }
-            if (!ok) break;
-            ptx::umma_commit(&accfull[a]);
-            ++ta;
+            ptx::mbar_arrive(&ring_full[r]);
+            if (t_c < 0) {
+                ok = push_item(-1, r_c);  // end of this CTA's items
+                break;
+            }
+            for (uint32_t m = m_c; m && ok; m &= m - 1) ok = push_item(__ffs(m) - 1, r_c);
+            // start loading tile i+2 (its claim was issued one tile ago)
+            int64_t t_nn = -1;
+            uint32_t m_nn = 0;
+            int r_nn[4] = {-1, -1, -1, -1};
+            if (t_n >= 0) {
+                fetch(int64_t(gridDim.x) + __shfl_sync(kFull, claimed, 0), t_nn, m_nn, r_nn);
+                if (lane == 0) claimed = atomicAdd(tile_counter, 1);
+            }
+            t_c = t_n;
+            m_c = m_n;
+            t_n = t_nn;
+            m_n = m_nn;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                r_c[e] = r_n[e];
+                r_n[e] = r_nn[e];
+            }
         }
+        ptx::cp_async_wait<0>();
         if (!ok) s_abort = 1;
     }
 
@@ -337,8 +465,8 @@ static bool make_weight_map(CUtensorMap *map, const void *w, bool bf16, int k3, 
 }
 
 template <typename T, int KC, int N, bool BMN>
-static lat_status launch(const void *x, const void *w, int k3, const MapView &mv, void *y, int32_t *d_status,
-                         cudaStream_t s) {
+static lat_status launch(const void *x, const void *w, int k3, const MapView &mv, void *y, int32_t *counter,
+                         int32_t *d_status, cudaStream_t s) {
     using C = Cfg<N>;
     CUtensorMap map;
     // forward: W[k] is (KC x N); data gradient: W[k] is (N x KC)
@@ -346,19 +474,20 @@ static lat_status launch(const void *x, const void *w, int k3, const MapView &mv
     auto kern = conv_tc_kernel<T, KC, N, BMN>;
     const int64_t grid = std::min<int64_t>(mv.ntiles, GridCache<KernelTag<T, KC, N, BMN>>::get(kern, C::kSmem, int(C::kTmemCols), 2));
     if (grid <= 0) return LAT_ERR_CUDA;
+    LAT_CUDA_TRY(cudaMemsetAsync(counter, 0, sizeof(int32_t), s));
     kern<<<unsigned(grid), kThreads, C::kSmem, s>>>(map, static_cast<const T *>(x), mv, static_cast<T *>(y),
-                                                    d_status);
+                                                    counter, d_status);
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }
 
 template <typename T, bool BMN>
 static lat_status dispatch(int kc, int n, const void *x, const void *w, int k3, const MapView &mv, void *y,
-                           int32_t *d_status, cudaStream_t s) {
-    if (kc == 64 && n == 64) return launch<T, 64, 64, BMN>(x, w, k3, mv, y, d_status, s);
-    if (kc == 64 && n == 128) return launch<T, 64, 128, BMN>(x, w, k3, mv, y, d_status, s);
-    if (kc == 128 && n == 64) return launch<T, 128, 64, BMN>(x, w, k3, mv, y, d_status, s);
-    if (kc == 128 && n == 128) return launch<T, 128, 128, BMN>(x, w, k3, mv, y, d_status, s);
+                           int32_t *counter, int32_t *d_status, cudaStream_t s) {
+    if (kc == 64 && n == 64) return launch<T, 64, 64, BMN>(x, w, k3, mv, y, counter, d_status, s);
+    if (kc == 64 && n == 128) return launch<T, 64, 128, BMN>(x, w, k3, mv, y, counter, d_status, s);
+    if (kc == 128 && n == 64) return launch<T, 128, 64, BMN>(x, w, k3, mv, y, counter, d_status, s);
+    if (kc == 128 && n == 128) return launch<T, 128, 128, BMN>(x, w, k3, mv, y, counter, d_status, s);
     return LAT_ERR_UNSUPPORTED;
 }
 
@@ -366,16 +495,20 @@ static lat_status dispatch(int kc, int n, const void *x, const void *w, int k3, 
 
 bool conv_tc_supported(int kc, int n) { return (kc == 64 || kc == 128) && (n == 64 || n == 128); }
 
+size_t conv_tc_ws_bytes() { return 256; }
+
 // Forward (wt = false): gathered x (cin) x W[k] (cin x cout).  Data gradient (wt = true):
-// gathered dy (kc = cout) x W[k]^T, producing n = cin channels.
+// gathered dy (kc = cout) x W[k]^T, producing n = cin channels.  ws: conv_tc_ws_bytes()
+// bytes of scratch (the tile counter).
 lat_status launch_conv_tc(bool bf16, const void *x, int kc, const void *w, int n, int k3, const MapView &mv, bool wt,
-                          void *y, int32_t *d_status, cudaStream_t s) {
+                          void *y, void *ws, int32_t *d_status, cudaStream_t s) {
     if (mv.ntiles == 0) return LAT_OK;
+    int32_t *counter = static_cast<int32_t *>(ws);
     if (bf16)
-        return wt ? tc::dispatch<__nv_bfloat16, false>(kc, n, x, w, k3, mv, y, d_status, s)
-                  : tc::dispatch<__nv_bfloat16, true>(kc, n, x, w, k3, mv, y, d_status, s);
-    return wt ? tc::dispatch<__half, false>(kc, n, x, w, k3, mv, y, d_status, s)
-              : tc::dispatch<__half, true>(kc, n, x, w, k3, mv, y, d_status, s);
+        return wt ? tc::dispatch<__nv_bfloat16, false>(kc, n, x, w, k3, mv, y, counter, d_status, s)
+                  : tc::dispatch<__nv_bfloat16, true>(kc, n, x, w, k3, mv, y, counter, d_status, s);
+    return wt ? tc::dispatch<__half, false>(kc, n, x, w, k3, mv, y, counter, d_status, s)
+              : tc::dispatch<__half, true>(kc, n, x, w, k3, mv, y, counter, d_status, s);
 }
 
 }  // namespace lat

@@ -71,3 +71,20 @@ def test_host_argument_checks_return_without_gpu(lib):
     km.k3 = 27
     # channel counts must be multiples of 8
     assert lib.lat_sconv_fwd(P(16), 12, P(16), 16, ctypes.byref(km), P(16), 0, None, 0, None, None) == 1
+
+
+def test_conv_workspace_query_and_check_without_gpu(lib):
+    """Tensor-core fwd / dgrad need the 256-byte tile-counter workspace; the
+    CUDA-core shapes need none; too little workspace fails before any launch."""
+    P = ctypes.c_void_p
+    km = _lib.lat_kmap()
+    km.k3, km.n_out, km.n_in = 27, 10, 10
+    km.nbr, km.perm, km.tile_mask = P(16), P(16), P(16)
+    f32, f16 = 0, 1
+    assert lib.lat_sconv_ws_bytes(0, 64, 64, ctypes.byref(km), f16) == 256
+    assert lib.lat_sconv_ws_bytes(1, 64, 128, ctypes.byref(km), f16) == 256
+    assert lib.lat_sconv_ws_bytes(0, 64, 64, ctypes.byref(km), f32) == 0
+    assert lib.lat_sconv_ws_bytes(0, 16, 32, ctypes.byref(km), f16) == 0
+    assert lib.lat_sconv_fwd(P(16), 64, P(16), 64, ctypes.byref(km), P(16), f16, None, 0, None, None) == 128
+    assert lib.lat_sconv_fwd(P(16), 64, P(16), 64, ctypes.byref(km), P(16), f16, P(256), 16, None, None) == 128
+    assert lib.lat_sconv_dgrad(P(16), 128, P(16), 64, ctypes.byref(km), 1, P(16), f16, None, 0, None, None) == 128
