@@ -48,7 +48,8 @@ constexpr int kMmaWarp = kProdWarps + kEpiWarps;
 constexpr int kSchedWarp = kMmaWarp + 1;
 constexpr int kThreads = (kSchedWarp + 1) * 32;
 constexpr int kRing = 8;         // tile entries in flight between the scheduler and the other roles
-constexpr int kItems = 16;       // (tile, offset) items in flight between the scheduler and the gather warps
+constexpr int kItems = 14;       // (tile, offset) items in flight between the scheduler and the gather warps
+constexpr uint32_t kStgBytes = kEpiWarps * 32 * 32;  // per epilogue warp: 32 rows x 16 output channels
 constexpr uint32_t kABytes = kM * 128;  // 128 rows x 64 channels x 2 bytes
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr unsigned kFull = 0xFFFFFFFFu;
@@ -76,14 +77,17 @@ struct Cfg {
     static constexpr int kStages = N == 64 ? 4 : 3;  // ~100 KB: two CTAs per SM
     static constexpr uint32_t kRingOff = kStages * kStage;
     static constexpr uint32_t kItemOff = kRingOff + kRing * sizeof(TileEntry);
-    static constexpr uint32_t kBarOff = kItemOff + kItems * sizeof(ItemEntry);
-    static constexpr uint32_t kBarBytes = 1024;
+    static constexpr uint32_t kStgOff = kItemOff + kItems * sizeof(ItemEntry);
+    static constexpr uint32_t kBarOff = kStgOff + kStgBytes;
+    static constexpr uint32_t kBarBytes = 512;
     static constexpr uint32_t kSmem = kBarOff + kBarBytes + 1024;
     static constexpr uint32_t kTmemCols = 2 * N;
     // the scheduler can run ahead of the slowest reader (the epilogue) by at
     // most stages + 2 tiles; the ring must be deeper than that
     static_assert(kRing >= kStages + 3, "tile ring too shallow");
     static_assert((2 * kStages + 4 + 2 * kRing + 2 * kItems) * 8 + 4 <= kBarBytes, "barrier area");
+    // two CTAs per SM: 228 KB of shared memory per SM, 1 KB reserved per CTA, 16 B static
+    static_assert(2 * (kSmem + 16 + 1024) <= 228 * 1024, "two CTAs per SM");
 };
 
 template <typename T> constexpr bool is_bf16() { return sizeof(T) == 2 && !std::is_same<T, __half>::value; }
@@ -251,25 +255,43 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x
             }
             ptx::tc_fence_after();
             const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + a * N;
+            // Coalesced write-back: each 16-channel slice of the warp's 32 rows goes
+            // through a 1 KB staging buffer (32 B per row, the two 16-byte halves
+            // swapped on every other group of 4 rows against bank conflicts), then
+            // lane pairs write whole 32-byte sectors of one row.
+            uint8_t *stg = smem + C::kStgOff + q * 1024;
+            auto write_slice = [&](const uint32_t (&v)[16], int col) {
+                uint4 o0, o1;
+                o0.x = pack2(__uint_as_float(v[0]), __uint_as_float(v[1]), T{});
+                o0.y = pack2(__uint_as_float(v[2]), __uint_as_float(v[3]), T{});
+                o0.z = pack2(__uint_as_float(v[4]), __uint_as_float(v[5]), T{});
+                o0.w = pack2(__uint_as_float(v[6]), __uint_as_float(v[7]), T{});
+                o1.x = pack2(__uint_as_float(v[8]), __uint_as_float(v[9]), T{});
+                o1.y = pack2(__uint_as_float(v[10]), __uint_as_float(v[11]), T{});
+                o1.z = pack2(__uint_as_float(v[12]), __uint_as_float(v[13]), T{});
+                o1.w = pack2(__uint_as_float(v[14]), __uint_as_float(v[15]), T{});
+                const int sw = (lane >> 2) & 1;
+                *reinterpret_cast<uint4 *>(stg + lane * 32 + 16 * sw) = o0;
+                *reinterpret_cast<uint4 *>(stg + lane * 32 + 16 * (sw ^ 1)) = o1;
+                __syncwarp();
+#pragma unroll
+                for (int g = 0; g < 2; ++g) {
+                    const int rr = 16 * g + (lane >> 1), hc = lane & 1;
+                    const uint4 val =
+                        *reinterpret_cast<const uint4 *>(stg + rr * 32 + 16 * (hc ^ ((rr >> 2) & 1)));
+                    const int jr = __shfl_sync(kFull, j, rr);
+                    if (jr >= 0) *reinterpret_cast<uint4 *>(y + int64_t(jr) * N + col + 8 * hc) = val;
+                }
+                __syncwarp();
+            };
 #pragma unroll
             for (int c0 = 0; c0 < N; c0 += 32) {
                 uint32_t v0[16], v1[16];
                 ptx::tmem_ld16(taddr + c0, v0);
                 ptx::tmem_ld16(taddr + c0 + 16, v1);
                 ptx::tmem_wait_ld();
-                if (yr) {
-                    uint4 o[4];
-                    uint32_t *op = reinterpret_cast<uint32_t *>(o);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        op[e] = pack2(__uint_as_float(v0[2 * e]), __uint_as_float(v0[2 * e + 1]), T{});
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        op[8 + e] = pack2(__uint_as_float(v1[2 * e]), __uint_as_float(v1[2 * e + 1]), T{});
-                    uint4 *dst = reinterpret_cast<uint4 *>(yr + c0);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) dst[e] = o[e];
-                }
+                write_slice(v0, c0);
+                write_slice(v1, c0 + 16);
             }
             ptx::tc_fence_before();
             ptx::mbar_arrive(&accempty[a]);
@@ -366,56 +388,57 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x
             ++ii;
             return true;
         };
-        // tile 0 is static; the claim for tile 1 is in flight while tile 0's rows load
+        // kLook slots of (tile, mask, rows) rotate through the loop: slot s is
+        // published, its items pushed, and it is refilled with the tile kLook
+        // places later, so every row load has kLook-1 tiles of time to land.
+        // The loop over slots is unrolled; no register holding a load in
+        // flight is moved.  Tile 0 is static, tiles 1 and 2 come from one
+        // claim of two, later tiles from single claims issued one tile ahead.
+        constexpr int kLook = 3;
+        int64_t ts[kLook];
+        uint32_t ms[kLook];
+        int rs[kLook][4];
+        int pair = lane == 0 ? atomicAdd(tile_counter, 2) : 0;
         int claimed = lane == 0 ? atomicAdd(tile_counter, 1) : 0;
-        int64_t t_c, t_n;
-        uint32_t m_c, m_n;
-        int r_c[4], r_n[4];
-        fetch(blockIdx.x, t_c, m_c, r_c);
-        if (t_c >= 0) {
-            fetch(int64_t(gridDim.x) + __shfl_sync(kFull, claimed, 0), t_n, m_n, r_n);
-            if (lane == 0) claimed = atomicAdd(tile_counter, 1);
-        } else {
-            t_n = -1;
-            m_n = 0;
+        fetch(blockIdx.x, ts[0], ms[0], rs[0]);
+        const int64_t q1 = int64_t(gridDim.x) + __shfl_sync(kFull, pair, 0);
+        fetch(ts[0] >= 0 ? q1 : mv.ntiles, ts[1], ms[1], rs[1]);
+        fetch(ts[1] >= 0 ? q1 + 1 : mv.ntiles, ts[2], ms[2], rs[2]);
+        bool more = ts[2] >= 0;  // the last fetched tile exists, so later claims may too
+        int i = 0;               // tiles published
+        bool done = false;
+        while (ok && !done) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) r_n[e] = -1;
-        }
-        for (int i = 0; ok; ++i) {
-            // publish tile i for the MMA and epilogue roles
-            const int r = i % kRing;
-            if (!__all_sync(kFull, ptx::mbar_wait(&ring_empty[r], ((i / kRing) & 1) ^ 1, kWaitNs))) {
-                ok = false;
-                break;
-            }
+            for (int sl = 0; sl < kLook; ++sl) {
+                if (done || !ok) break;
+                // publish tile i for the MMA and epilogue roles
+                const int r = i % kRing;
+                if (!__all_sync(kFull, ptx::mbar_wait(&ring_empty[r], ((i / kRing) & 1) ^ 1, kWaitNs))) {
+                    ok = false;
+                    break;
+                }
 #pragma unroll
-            for (int e = 0; e < 4; ++e) ring[r].rows[e * 32 + lane] = r_c[e];
-            if (lane == 0) {
-                ring[r].tile = int32_t(t_c);
-                ring[r].mask = m_c;
-            }
-            ptx::mbar_arrive(&ring_full[r]);
-            if (t_c < 0) {
-                ok = push_item(-1, r_c);  // end of this CTA's items
-                break;
-            }
-            for (uint32_t m = m_c; m && ok; m &= m - 1) ok = push_item(__ffs(m) - 1, r_c);
-            // start loading tile i+2 (its claim was issued one tile ago)
-            int64_t t_nn = -1;
-            uint32_t m_nn = 0;
-            int r_nn[4] = {-1, -1, -1, -1};
-            if (t_n >= 0) {
-                fetch(int64_t(gridDim.x) + __shfl_sync(kFull, claimed, 0), t_nn, m_nn, r_nn);
-                if (lane == 0) claimed = atomicAdd(tile_counter, 1);
-            }
-            t_c = t_n;
-            m_c = m_n;
-            t_n = t_nn;
-            m_n = m_nn;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                r_c[e] = r_n[e];
-                r_n[e] = r_nn[e];
+                for (int e = 0; e < 4; ++e) ring[r].rows[e * 32 + lane] = rs[sl][e];
+                if (lane == 0) {
+                    ring[r].tile = int32_t(ts[sl]);
+                    ring[r].mask = ms[sl];
+                }
+                ptx::mbar_arrive(&ring_full[r]);
+                ++i;
+                if (ts[sl] < 0) {
+                    ok = push_item(-1, rs[sl]);  // end of this CTA's items
+                    done = true;
+                    break;
+                }
+                for (uint32_t m = ms[sl]; m && ok; m &= m - 1) ok = push_item(__ffs(m) - 1, rs[sl]);
+                // refill the slot with the tile kLook places later
+                int64_t q = mv.ntiles;
+                if (more) {
+                    q = int64_t(gridDim.x) + __shfl_sync(kFull, claimed, 0);
+                    if (lane == 0) claimed = atomicAdd(tile_counter, 1);
+                }
+                fetch(q, ts[sl], ms[sl], rs[sl]);
+                more = more && q < mv.ntiles;
             }
         }
         ptx::cp_async_wait<0>();
