@@ -142,11 +142,15 @@ typedef struct {
  * Key packing: key = b<<48 | (x+2^15)<<32 | (y+2^15)<<16 | (z+2^15), so the
  * unsigned key order is the lexicographic (b, x, y, z) order.  b must lie in
  * [0, 65534] and x, y, z in [-32768, 32767]; rows outside are skipped and
- * flag LAT_ERR_COORD_RANGE.  The table is an array of 16-byte slots
- * {uint64 key; int32 row; int32 unused} with a power-of-two slot count; an
- * empty slot holds key 0xFFFF...F.  A key's home slot is a 32-bit mix of
- * the key (its two halves folded, then the MurmurHash3 fmix32 finalizer);
- * collisions are resolved by linear probing.
+ * flag LAT_ERR_COORD_RANGE.  The table holds a power-of-two number of
+ * slots, 16 bytes of table each, stored as 64-byte groups of 4 slots
+ * {uint64 key[4]; uint32 row[4]; uint32 unused[4]}: slot s is entry s % 4
+ * of group s / 4.  An empty slot holds key 0xFFFF...F.  A key's home slot is
+ * a 32-bit mix of the key (its two halves folded, then the MurmurHash3
+ * fmix32 finalizer) masked to the slot count; its probe sequence starts at
+ * the first slot of the home slot's group and runs over consecutive slots
+ * (linear probing), so a lookup reads whole groups.  The table must be
+ * 64-byte aligned.
  */
 
 /* Bytes of a table for n rows: 16 * next_pow2(max(ceil(rsv_ratio*n), 64)).

@@ -14,12 +14,18 @@ namespace lat {
 
 constexpr uint64_t kEmptyKey = ~0ull;
 
-// One hash slot: 16 bytes so a single vector load resolves a probe.
-struct __align__(16) Slot {
-    unsigned long long key;
-    unsigned int row;  // unsigned so atomicMin keeps the lowest row; 0xFFFFFFFF = none
-    unsigned int unused;
+// The table is an array of 64-byte groups of 4 slots, keys first: one probe
+// round reads a group's 4 keys with two 16-byte loads, and the row of a
+// matching slot with one more load.  Slot s is entry s % 4 of group s / 4;
+// the table size is counted in slots (16 bytes of table each).
+constexpr int kGroupSlots = 4;
+constexpr size_t kSlotBytes = 16;
+struct __align__(64) SlotGroup {
+    unsigned long long key[kGroupSlots];
+    unsigned int row[kGroupSlots];  // unsigned so atomicMin keeps the lowest row; 0xFFFFFFFF = none
+    unsigned int unused[kGroupSlots];
 };
+static_assert(sizeof(SlotGroup) == kGroupSlots * kSlotBytes, "slot group layout");
 
 // Packed key of (b, x, y, z); returns false when a field is outside the key range.
 __device__ __forceinline__ bool pack_key(int b, int x, int y, int z, uint64_t &key) {
@@ -53,13 +59,19 @@ __device__ __forceinline__ uint32_t slot_hash(uint64_t key) {
     return h;
 }
 
+// First slot of a key's probe sequence: its home slot (hash & cap_mask) rounded
+// down to the start of the home group.  Probing then runs over consecutive slots.
+__device__ __forceinline__ uint32_t probe_start(uint64_t key, uint32_t cap_mask) {
+    return slot_hash(key) & cap_mask & ~uint32_t(kGroupSlots - 1);
+}
+
 // Look a key up; returns the row or -1.  Probing is bounded by the slot count.
-__device__ __forceinline__ int hash_find(const Slot *__restrict__ slots, uint32_t cap_mask, uint64_t key) {
-    uint32_t s = slot_hash(key) & cap_mask;
+__device__ __forceinline__ int hash_find(const SlotGroup *__restrict__ groups, uint32_t cap_mask, uint64_t key) {
+    uint32_t s = probe_start(key, cap_mask);
     for (uint32_t probe = 0; probe <= cap_mask; ++probe) {
-        const ulonglong2 v = __ldg(reinterpret_cast<const ulonglong2 *>(slots + s));
-        if (v.x == key) return int(unsigned(v.y));
-        if (v.x == kEmptyKey) return -1;
+        const uint64_t k = __ldg(&groups[s / kGroupSlots].key[s % kGroupSlots]);
+        if (k == key) return int(__ldg(&groups[s / kGroupSlots].row[s % kGroupSlots]));
+        if (k == kEmptyKey) return -1;
         s = (s + 1) & cap_mask;
     }
     return -1;

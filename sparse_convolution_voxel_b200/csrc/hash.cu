@@ -3,16 +3,17 @@
 // Torch Lattice docs, "Migrating from TorchSparse": hashing is one of the CUDA
 // kernels of the library ("What remains familiar") and its capacity knob is
 // torch_lattice.backends.hash_rsv_ratio ("Backend and configuration
-// differences").  Design: 16-byte slots {key, row}, 32-bit mixing hash placement,
-// linear probing bounded by the slot count, 64-bit atomicCAS to claim a slot
-// and an unsigned atomicMin on the row so that duplicates keep the lowest row
-// deterministically.
+// differences").  Design: 64-byte groups of 4 slots (4 keys, then 4 rows),
+// 32-bit mixing hash placement, probing from the start of the home group over
+// consecutive slots (bounded by the slot count), 64-bit atomicCAS to claim a
+// slot and an unsigned atomicMin on the row so that duplicates keep the lowest
+// row deterministically.
 #include "common.cuh"
 
 namespace lat {
 
 __global__ void __launch_bounds__(256) hash_insert_kernel(const int4 *__restrict__ coords, int64_t n,
-                                                          Slot *__restrict__ slots, uint32_t cap_mask,
+                                                          SlotGroup *__restrict__ groups, uint32_t cap_mask,
                                                           int32_t *d_status) {
     int32_t bad = 0;
     for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n;
@@ -23,14 +24,14 @@ __global__ void __launch_bounds__(256) hash_insert_kernel(const int4 *__restrict
             bad |= LAT_ERR_COORD_RANGE;
             continue;
         }
-        uint32_t s = slot_hash(key) & cap_mask;
+        uint32_t s = probe_start(key, cap_mask);
         bool placed = false;
         for (uint32_t probe = 0; probe <= cap_mask; ++probe) {
-            unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(&slots[s].key);
-            if (cur == kEmptyKey)
-                cur = atomicCAS(&slots[s].key, (unsigned long long)kEmptyKey, (unsigned long long)key);
+            unsigned long long *kp = &groups[s / kGroupSlots].key[s % kGroupSlots];
+            unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(kp);
+            if (cur == kEmptyKey) cur = atomicCAS(kp, (unsigned long long)kEmptyKey, (unsigned long long)key);
             if (cur == kEmptyKey || cur == key) {
-                atomicMin(&slots[s].row, unsigned(i));
+                atomicMin(&groups[s / kGroupSlots].row[s % kGroupSlots], unsigned(i));
                 if (cur == key) bad |= LAT_ERR_DUPLICATE;
                 placed = true;
                 break;
@@ -50,25 +51,25 @@ extern "C" size_t lat_hash_bytes(int64_t n, float rsv_ratio) {
     uint64_t cap = 64;
     while (double(cap) < want) cap <<= 1;
     if (cap > (uint64_t(1) << 31)) return 0;  // slot indices are 32-bit in the query kernels
-    return size_t(cap) * sizeof(lat::Slot);
+    return size_t(cap) * lat::kSlotBytes;
 }
 
 extern "C" lat_status lat_hash_build(const int32_t *coords, int64_t n, void *table, size_t table_bytes,
                                      int32_t *d_status, lat_stream stream) {
     using namespace lat;
     if (n < 0 || n >= (int64_t(1) << 31) || (n > 0 && !coords) || !table) return LAT_ERR_ARG;
-    if (table_bytes % sizeof(Slot) || !pow2(table_bytes / sizeof(Slot)) || table_bytes / sizeof(Slot) < 64 ||
-        table_bytes / sizeof(Slot) > (uint64_t(1) << 31))
+    if (table_bytes % kSlotBytes || !pow2(table_bytes / kSlotBytes) || table_bytes / kSlotBytes < 64 ||
+        table_bytes / kSlotBytes > (uint64_t(1) << 31))
         return LAT_ERR_ARG;
-    if (reinterpret_cast<uintptr_t>(coords) % 16 || reinterpret_cast<uintptr_t>(table) % 16) return LAT_ERR_ARG;
-    const uint64_t cap = table_bytes / sizeof(Slot);
+    if (reinterpret_cast<uintptr_t>(coords) % 16 || reinterpret_cast<uintptr_t>(table) % 64) return LAT_ERR_ARG;
+    const uint64_t cap = table_bytes / kSlotBytes;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     LAT_CUDA_TRY(cudaMemsetAsync(table, 0xFF, table_bytes, s));
     if (n == 0) return LAT_OK;
     const int threads = 256;
     const int64_t blocks = (n + threads - 1) / threads;
     hash_insert_kernel<<<unsigned(blocks), threads, 0, s>>>(reinterpret_cast<const int4 *>(coords), n,
-                                                             static_cast<Slot *>(table), uint32_t(cap - 1), d_status);
+                                                             static_cast<SlotGroup *>(table), uint32_t(cap - 1), d_status);
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }

@@ -7,17 +7,18 @@
 //   1. probe:  one thread per output row probes the input table (for a
 //              submanifold map only the offsets below the centre, mirroring
 //              each hit); writes nbr (offset-major, coalesced), mask, and per
-//              (offset, block) hit counts from warp ballots (a count pass over
-//              nbr does the last two for submanifold maps).
+//              (offset, block) hit counts from warp ballots (for submanifold
+//              maps the masks are ORed in atomically and a count pass over the
+//              masks gives the counts).
 //   2. scan:   one block per offset turns its per-block counts into offsets
 //              (pairs come out grouped by offset, rows ascending).
-//   3. emit:   re-reads nbr and writes (in, out) pairs at ballot-ranked
-//              positions: deterministic, no atomics.
-//   4. sort:   stable 2-pass radix sort of output rows by a 16-bit grouping
-//              key of the mask (neighbour count, mask hash) -> perm.
-//   5. tiles:  OR of masks over each LAT_TILE_ROWS run of perm -> tile_mask.
-#include <cub/device/device_radix_sort.cuh>
-
+//   3. emit:   walks the masks and writes (in, out) pairs at ballot-ranked
+//              positions, reading nbr only where a bit is set:
+//              deterministic, no atomics.
+//   4. sort:   stable LSD radix sort (8-bit digits: 2 passes for the 16-bit
+//              grouping key of the mask -- neighbour count, mask hash --, 1
+//              pass when k3 <= 8) of the output rows -> perm; the last pass
+//              ORs the masks of each LAT_TILE_ROWS run of perm -> tile_mask.
 #include "common.cuh"
 
 namespace lat {
@@ -54,6 +55,34 @@ __device__ __forceinline__ uint32_t group_key(uint32_t m, int k3) {
 }
 inline int group_key_bits(int k3) { return k3 <= 8 ? k3 : kGroupKeyBits; }
 
+// ----------------------------------------------------------------------------- row sort
+// Stable LSD radix sort of the row grouping keys (8-bit digits, one pass per
+// digit) producing perm.  The input of a pass is cut into tiles of kSortTile
+// rows; hist[d * ntile + b] counts digit d in tile b.  The first pass's
+// histogram is accumulated by the kernel that computes the keys
+// (sort_hist_add), each pass's scatter accumulates the next pass's histogram;
+// one block per digit scans that digit's per-tile counts, and every scatter
+// block scans the 256 digit totals, which together give the first output
+// position of every (digit, tile).  Within a tile, rows keep their order (ranks from warp
+// match + per-warp digit counts), so the result is the stable sort: perm equals
+// the stable argsort of the keys, deterministic.  The last pass also ORs every
+// row's mask into its tile of LAT_TILE_ROWS output positions.
+constexpr int kSortThreads = 256;
+constexpr int kSortRounds = 8;
+constexpr int kSortTile = kSortThreads * kSortRounds;
+constexpr int kSortWarps = kSortThreads / 32;
+
+// Adds the lowest digit of this lane's key to the first pass's histogram.  Every
+// lane of the warp calls it; the warp's rows lie in one sort tile.
+__device__ __forceinline__ void sort_hist_add(uint32_t key, bool live, int64_t j, int32_t *__restrict__ hist,
+                                              int ntile) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t d = key & 255u;
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, live ? d : 256u + lane);
+    if (live && (peers & ((1u << lane) - 1u)) == 0)
+        atomicAdd(hist + int64_t(d) * ntile + j / kSortTile, int(__popc(peers)));
+}
+
 // Input coordinate probed by output row c at offset (ix, iy, iz); false if none.
 __device__ __forceinline__ bool query_coord(const Geom &g, const int4 &c, int ix, int iy, int iz, uint64_t &key) {
     int p[3];
@@ -74,23 +103,26 @@ __device__ __forceinline__ bool query_coord(const Geom &g, const int4 &c, int ix
 }
 
 // One thread per output row.  Offsets are probed in batches of kProbeBatch:
-// each round loads the current slot of every still-unresolved offset of the
-// batch at once (one 16-byte load per slot), then resolves what it can, so a
-// thread keeps several independent loads in flight instead of walking the
-// probe sequences one after another.  Rounds are bounded by the slot count.
+// each round loads the 4 keys of the current slot group of every unresolved
+// offset of the batch at once (two 16-byte loads per group), then resolves
+// what it can (a match, or an empty slot before it, ends the probe); the rows
+// of the matches are loaded together after the rounds.  At the table's load
+// factor nearly every probe ends inside its home group, so a batch takes about
+// one round.  Rounds are bounded by the group count.
 //
 // SYM (submanifold maps): the relation is symmetric -- input i sits at offset
 // k of row j exactly when j sits at offset k3-1-k of row i -- so only the
 // offsets below the centre are probed; a hit also writes the mirrored entry
-// (the upper half of nbr must hold -1 beforehand), and the centre is the row
-// itself.  Masks and per-block counts then come from kmap_count_kernel.
+// (the upper half of nbr must hold -1 beforehand) and ORs the mirrored bit into
+// the other row's mask (masks must hold 0 beforehand), and the centre is the
+// row itself.  Keys and per-block counts then come from kmap_count_kernel.
 // Otherwise every offset is probed and the mask and counts are produced here.
 template <bool SYM>
 __global__ void __launch_bounds__(kQueryThreads)
-kmap_probe_kernel(const Slot *__restrict__ slots, uint32_t cap_mask, const int4 *__restrict__ out_coords,
+kmap_probe_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const int4 *__restrict__ out_coords,
                   int64_t n_out, int64_t n_in, Geom g, int32_t *__restrict__ nbr, uint32_t *__restrict__ mask,
-                  uint32_t *__restrict__ keys, int32_t *__restrict__ iota, int32_t *__restrict__ block_counts, int nblk,
-                  int32_t *d_status) {
+                  uint32_t *__restrict__ keys, int32_t *__restrict__ hist, int ntile, int32_t *__restrict__ block_counts,
+                  int nblk, int32_t *d_status) {
     __shared__ int s_cnt[32];
     if (!SYM) {
         if (threadIdx.x < 32) s_cnt[threadIdx.x] = 0;
@@ -109,13 +141,15 @@ kmap_probe_kernel(const Slot *__restrict__ slots, uint32_t cap_mask, const int4 
     int32_t bad = 0;
     for (int k0 = 0; k0 < kend; k0 += kProbeBatch) {
         uint64_t key[kProbeBatch];
-        uint32_t slot[kProbeBatch];
+        uint32_t slot[kProbeBatch];  // first slot of the group probed next
+        int hit[kProbeBatch];        // slot of the match, -1 = none
         int row[kProbeBatch];
         uint32_t pending = 0;
 #pragma unroll
         for (int e = 0; e < kProbeBatch; ++e) {
             const int k = k0 + e;
             row[e] = -1;
+            hit[e] = -1;
             key[e] = kEmptyKey;
             slot[e] = 0;
             if (!live || k >= kend) continue;
@@ -131,34 +165,47 @@ kmap_probe_kernel(const Slot *__restrict__ slots, uint32_t cap_mask, const int4 
                 ok = query_coord(g, c, g.off[k][0], g.off[k][1], g.off[k][2], key[e]);
             }
             if (ok) {
-                slot[e] = slot_hash(key[e]) & cap_mask;
+                slot[e] = probe_start(key[e], cap_mask);
                 pending |= 1u << e;
             }
         }
-        for (uint32_t round = 0; pending && round <= cap_mask; ++round) {
-            unsigned long long kv[kProbeBatch];
-            uint32_t rv[kProbeBatch];
+        for (uint32_t round = 0; pending && round <= cap_mask / kGroupSlots; ++round) {
+            ulonglong2 ka[kProbeBatch], kb[kProbeBatch];
 #pragma unroll
             for (int e = 0; e < kProbeBatch; ++e) {
                 if (pending & (1u << e)) {
-                    const ulonglong2 v = __ldg(reinterpret_cast<const ulonglong2 *>(slots + slot[e]));
-                    kv[e] = v.x;
-                    rv[e] = uint32_t(v.y);
+                    const SlotGroup *gp = groups + slot[e] / kGroupSlots;
+                    ka[e] = __ldg(reinterpret_cast<const ulonglong2 *>(gp->key));
+                    kb[e] = __ldg(reinterpret_cast<const ulonglong2 *>(gp->key + 2));
                 }
             }
 #pragma unroll
             for (int e = 0; e < kProbeBatch; ++e) {
                 if (!(pending & (1u << e))) continue;
-                if (kv[e] == key[e]) {
-                    row[e] = int(rv[e]);
+                const uint64_t k4[kGroupSlots] = {ka[e].x, ka[e].y, kb[e].x, kb[e].y};
+                int found = -1;
+                bool stop = false;
+#pragma unroll
+                for (int i = 0; i < kGroupSlots; ++i) {
+                    if (stop) continue;
+                    if (k4[i] == key[e]) {
+                        found = i;
+                        stop = true;
+                    } else if (k4[i] == kEmptyKey) {
+                        stop = true;
+                    }
+                }
+                if (stop) {
                     pending &= ~(1u << e);
-                } else if (kv[e] == kEmptyKey) {
-                    pending &= ~(1u << e);
+                    if (found >= 0) hit[e] = int(slot[e]) + found;
                 } else {
-                    slot[e] = (slot[e] + 1) & cap_mask;
+                    slot[e] = (slot[e] + kGroupSlots) & cap_mask;
                 }
             }
         }
+#pragma unroll
+        for (int e = 0; e < kProbeBatch; ++e)
+            if (hit[e] >= 0) row[e] = int(__ldg(&groups[hit[e] / kGroupSlots].row[hit[e] % kGroupSlots]));
 #pragma unroll
         for (int e = 0; e < kProbeBatch; ++e) {
             const int k = k0 + e;
@@ -167,7 +214,11 @@ kmap_probe_kernel(const Slot *__restrict__ slots, uint32_t cap_mask, const int4 
             if (r >= n_in || (SYM && r >= n_out)) { bad |= LAT_ERR_BAD_MAP; r = -1; }
             if (live) nbr[int64_t(k) * n_out + j] = r;
             if (SYM) {
-                if (r >= 0) nbr[int64_t(g.k3 - 1 - k) * n_out + r] = int32_t(j);
+                if (r >= 0) {
+                    nbr[int64_t(g.k3 - 1 - k) * n_out + r] = int32_t(j);
+                    m |= 1u << k;
+                    atomicOr(mask + r, 1u << (g.k3 - 1 - k));
+                }
             } else {
                 const unsigned hits = __ballot_sync(0xFFFFFFFFu, r >= 0);
                 if (r >= 0) m |= 1u << k;
@@ -177,14 +228,18 @@ kmap_probe_kernel(const Slot *__restrict__ slots, uint32_t cap_mask, const int4 
     }
     if (bad) flag(d_status, bad);
     if (SYM) {
-        if (live) nbr[int64_t(centre) * n_out + j] = int32_t(j);
+        if (live) {
+            nbr[int64_t(centre) * n_out + j] = int32_t(j);
+            atomicOr(mask + j, m | (1u << centre));  // mirrored hits of other rows OR in concurrently
+        }
         return;
     }
+    const uint32_t key = group_key(m, g.k3);
     if (live) {
         mask[j] = m;
-        keys[j] = group_key(m, g.k3);
-        iota[j] = int32_t(j);
+        keys[j] = key;
     }
+    sort_hist_add(key, live, j, hist, ntile);
     __syncthreads();
     if (threadIdx.x < g.k3) block_counts[int64_t(threadIdx.x) * nblk + blockIdx.x] = s_cnt[threadIdx.x];
 }
@@ -233,41 +288,57 @@ kmap_scan_kernel(const int32_t *__restrict__ block_counts, int64_t *__restrict__
     if (t == 0) k_total[k] = s_carry;
 }
 
+// Pairs of every offset at ballot-ranked positions.  The offsets a row has
+// come from its mask; nbr is read only where a bit is set.
 __global__ void __launch_bounds__(kQueryThreads)
-kmap_emit_kernel(const int32_t *__restrict__ nbr, int64_t n_out, int k3, const int64_t *__restrict__ block_offsets,
-                 const int64_t *__restrict__ k_total, int nblk, int32_t *__restrict__ pair_in,
-                 int32_t *__restrict__ pair_out, int64_t capacity, int64_t *__restrict__ pair_off, int32_t *d_status) {
-    __shared__ int s_warp[32][kQueryWarps];
-    __shared__ int64_t s_kstart[33];
-    if (threadIdx.x == 0) {
-        int64_t run = 0;
-        for (int k = 0; k < k3; ++k) {
-            s_kstart[k] = run;
-            run += k_total[k];
-        }
-        s_kstart[k3] = run;
-        if (blockIdx.x == 0)
-            for (int k = 0; k <= k3; ++k) pair_off[k] = s_kstart[k];
-    }
+kmap_emit_kernel(const int32_t *__restrict__ nbr, const uint32_t *__restrict__ mask, int64_t n_out, int k3,
+                 const int64_t *__restrict__ block_offsets, const int64_t *__restrict__ k_total, int nblk,
+                 int32_t *__restrict__ pair_in, int32_t *__restrict__ pair_out, int64_t capacity,
+                 int64_t *__restrict__ pair_off, int32_t *d_status) {
+    __shared__ int s_warp[32][kQueryWarps];  // per (offset, warp): hits, then the exclusive prefix over warps
+    __shared__ int64_t s_base[32];           // first pair of (offset, this block)
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (warp == 0) {
+        // offset starts = exclusive scan of the per-offset totals, all loads in parallel
+        const int64_t tot = lane < k3 ? k_total[lane] : 0;
+        const int64_t bo = lane < k3 ? block_offsets[int64_t(lane) * nblk + blockIdx.x] : 0;
+        int64_t incl = tot;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int64_t o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+            if (lane >= d) incl += o;
+        }
+        if (lane < k3) s_base[lane] = incl - tot + bo;
+        if (blockIdx.x == 0) {
+            if (lane < k3) pair_off[lane] = incl - tot;
+            const int64_t all = __shfl_sync(0xFFFFFFFFu, incl, k3 - 1);
+            if (lane == 0) pair_off[k3] = all;
+        }
+    }
     const int64_t j = blockIdx.x * int64_t(kQueryThreads) + threadIdx.x;
-    const bool live = j < n_out;
+    const uint32_t m = j < n_out ? __ldg(mask + j) : 0u;
     for (int k = 0; k < k3; ++k) {
-        const int row = live ? nbr[int64_t(k) * n_out + j] : -1;
-        const unsigned hits = __ballot_sync(0xFFFFFFFFu, row >= 0);
+        const unsigned hits = __ballot_sync(0xFFFFFFFFu, (m >> k) & 1u);
         if (lane == 0) s_warp[k][warp] = __popc(hits);
+    }
+    __syncthreads();
+    if (threadIdx.x < k3) {
+        int run = 0;
+#pragma unroll
+        for (int w = 0; w < kQueryWarps; ++w) {
+            const int c = s_warp[threadIdx.x][w];
+            s_warp[threadIdx.x][w] = run;
+            run += c;
+        }
     }
     __syncthreads();
     bool over = false;
     for (int k = 0; k < k3; ++k) {
-        const int row = live ? nbr[int64_t(k) * n_out + j] : -1;
-        const unsigned hits = __ballot_sync(0xFFFFFFFFu, row >= 0);
-        if (row < 0) continue;
-        int64_t pos = s_kstart[k] + block_offsets[int64_t(k) * nblk + blockIdx.x];
-        for (int w = 0; w < warp; ++w) pos += s_warp[k][w];
-        pos += __popc(hits & ((1u << lane) - 1u));
+        const unsigned hits = __ballot_sync(0xFFFFFFFFu, (m >> k) & 1u);
+        if (!((m >> k) & 1u)) continue;
+        const int64_t pos = s_base[k] + s_warp[k][warp] + __popc(hits & ((1u << lane) - 1u));
         if (pos < capacity) {
-            pair_in[pos] = row;
+            pair_in[pos] = __ldg(nbr + int64_t(k) * n_out + j);
             pair_out[pos] = int32_t(j);
         } else {
             over = true;
@@ -276,43 +347,151 @@ kmap_emit_kernel(const int32_t *__restrict__ nbr, int64_t n_out, int k3, const i
     if (over) flag(d_status, LAT_ERR_CAPACITY);
 }
 
-__global__ void tile_mask_kernel(const uint32_t *__restrict__ mask, const int32_t *__restrict__ perm, int64_t n,
-                                 uint32_t *__restrict__ tile_mask, int64_t ntiles) {
-    const int64_t t = blockIdx.x * int64_t(blockDim.x / 32) + (threadIdx.x >> 5);
-    if (t >= ntiles) return;
-    const int lane = threadIdx.x & 31;
-    uint32_t m = 0;
-    for (int r = lane; r < LAT_TILE_ROWS; r += 32) {
-        const int64_t e = t * LAT_TILE_ROWS + r;
-        if (e < n) m |= mask[perm[e]];
+// Block d: exclusive scan, in place, of digit d's per-tile counts
+// hist[d * ntile + 0 .. ntile), and the digit's total into totals[d].
+__global__ void __launch_bounds__(256)
+sort_rowscan_kernel(int32_t *__restrict__ hist, int ntile, int32_t *__restrict__ totals) {
+    __shared__ int s_warp[8];
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    int32_t *row = hist + int64_t(blockIdx.x) * ntile;
+    int carry = 0;
+    for (int base = 0; base < ntile; base += 256) {
+        const int i = base + t;
+        const int v = i < ntile ? row[i] : 0;
+        int incl = v;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+            if (lane >= d) incl += o;
+        }
+        if (lane == 31) s_warp[w] = incl;
+        __syncthreads();
+        int before = 0, all = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int x = s_warp[q];
+            before += q < w ? x : 0;
+            all += x;
+        }
+        if (i < ntile) row[i] = carry + before + incl - v;
+        carry += all;
+        __syncthreads();
     }
-    for (int o = 16; o; o >>= 1) m |= __shfl_xor_sync(0xFFFFFFFFu, m, o);
-    if (lane == 0) tile_mask[t] = m;
+    if (t == 0) totals[blockIdx.x] = carry;
 }
 
-// Per-(offset, block) hit counts of a neighbour table that was filled without
-// probing (maps built from parent indices); also writes the identity row order.
+// One pass: scatter the rows of tile blockIdx.x by digit (key >> shift) & 255 to
+// the positions `off` gives.  vals_in == nullptr means the identity (row e).
+// LAST: write perm and OR masks into tile_mask; otherwise write the keys and
+// rows for the next pass and count its digit per output tile into hist_next.
+// All loads of the tile are issued before the first round.
+template <bool LAST>
+__global__ void __launch_bounds__(kSortThreads)
+sort_scatter_kernel(const uint32_t *__restrict__ keys_in, const int32_t *__restrict__ vals_in, int64_t n, int shift,
+                    const int32_t *__restrict__ off, const int32_t *__restrict__ totals, int ntile,
+                    uint32_t *__restrict__ keys_out,
+                    int32_t *__restrict__ vals_out, int32_t *__restrict__ hist_next,
+                    const uint32_t *__restrict__ mask, uint32_t *__restrict__ tile_mask) {
+    __shared__ int s_cnt[2][kSortWarps][256];
+    __shared__ int s_run[256];
+    __shared__ int s_wsum[kSortWarps];
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const unsigned lt = (1u << lane) - 1u;
+    const int b = blockIdx.x;
+    // first output position of digit t: exclusive scan of the digit totals
+    const int tot = totals[t];  // kSortThreads == 256 digits
+    const int off_b = off[int64_t(t) * ntile + b];
+    uint32_t key[kSortRounds], mk[kSortRounds];
+    int32_t val[kSortRounds];
+#pragma unroll
+    for (int r = 0; r < kSortRounds; ++r) {
+        const int64_t e = int64_t(b) * kSortTile + r * kSortThreads + t;
+        key[r] = 0;
+        val[r] = -1;
+        if (e < n) {
+            key[r] = __ldg(keys_in + e);
+            val[r] = vals_in ? __ldg(vals_in + e) : int32_t(e);
+        }
+    }
+    if (LAST) {
+#pragma unroll
+        for (int r = 0; r < kSortRounds; ++r) mk[r] = val[r] >= 0 ? __ldg(mask + val[r]) : 0u;
+    }
+    for (int i = t; i < 2 * kSortWarps * 256; i += kSortThreads) (&s_cnt[0][0][0])[i] = 0;
+    int incl = tot;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += o;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    int base = incl - tot;
+    for (int q = 0; q < warp; ++q) base += s_wsum[q];
+    s_run[t] = base + off_b;
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < kSortRounds; ++r) {
+        const int p = r & 1;
+        const bool live = val[r] >= 0;
+        const uint32_t d = (key[r] >> shift) & 255u;
+        const unsigned peers = __match_any_sync(0xFFFFFFFFu, live ? d : 256u + lane);
+        const bool leader = live && (peers & lt) == 0;
+        if (leader) s_cnt[p][warp][d] = __popc(peers);
+        __syncthreads();
+        int64_t dst = 0;
+        if (live) {
+            int pre = s_run[d] + __popc(peers & lt);
+            for (int w = 0; w < warp; ++w) pre += s_cnt[p][w][d];
+            dst = pre;
+        }
+        __syncthreads();
+        // digit t: advance its running position and clear this round's counts
+        int add = 0;
+#pragma unroll
+        for (int w = 0; w < kSortWarps; ++w) {
+            add += s_cnt[p][w][t];
+            s_cnt[p][w][t] = 0;
+        }
+        s_run[t] += add;
+        if (LAST) {
+            if (live) vals_out[dst] = val[r];
+            // one atomic per (warp, output tile)
+            const uint32_t tile = live ? uint32_t(dst / LAT_TILE_ROWS) : (0x80000000u | lane);
+            const unsigned tp = __match_any_sync(0xFFFFFFFFu, tile);
+            const uint32_t m_or = __reduce_or_sync(tp, mk[r]);
+            if (live && (tp & lt) == 0) atomicOr(tile_mask + dst / LAT_TILE_ROWS, m_or);
+        } else {
+            if (live) {
+                keys_out[dst] = key[r];
+                vals_out[dst] = val[r];
+            }
+            const uint32_t d2 = (key[r] >> (shift + 8)) & 255u;
+            const uint32_t tag = live ? ((d2 << 20) | uint32_t(dst / kSortTile)) : (0x80000000u | lane);
+            const unsigned p2 = __match_any_sync(0xFFFFFFFFu, tag);
+            if (live && (p2 & lt) == 0) atomicAdd(hist_next + int64_t(d2) * ntile + dst / kSortTile, int(__popc(p2)));
+        }
+    }
+}
+
+// Per-(offset, block) hit counts, grouping keys and the first sort pass's
+// histogram from the masks (submanifold probes and maps built from parent indices).
 __global__ void __launch_bounds__(kQueryThreads)
-kmap_count_kernel(const int32_t *__restrict__ nbr, int64_t n_out, int k3, int32_t *__restrict__ iota,
-                  int32_t *__restrict__ block_counts, int nblk, uint32_t *__restrict__ mask,
-                  uint32_t *__restrict__ keys) {
+kmap_count_kernel(const uint32_t *__restrict__ mask, int64_t n_out, int k3, int32_t *__restrict__ block_counts,
+                  int nblk, uint32_t *__restrict__ keys, int32_t *__restrict__ hist, int ntile) {
     __shared__ int s_cnt[32];
     if (threadIdx.x < 32) s_cnt[threadIdx.x] = 0;
     __syncthreads();
     const int64_t j = blockIdx.x * int64_t(kQueryThreads) + threadIdx.x;
     const bool live = j < n_out;
-    uint32_t m = 0;
+    const uint32_t m = live ? __ldg(mask + j) : 0u;
     for (int k = 0; k < k3; ++k) {
-        const int row = live ? nbr[int64_t(k) * n_out + j] : -1;
-        const unsigned hits = __ballot_sync(0xFFFFFFFFu, row >= 0);
-        if (row >= 0) m |= 1u << k;
+        const unsigned hits = __ballot_sync(0xFFFFFFFFu, (m >> k) & 1u);
         if ((threadIdx.x & 31) == 0 && hits) atomicAdd(&s_cnt[k], __popc(hits));
     }
-    if (live) {
-        iota[j] = int32_t(j);
-        keys[j] = group_key(m, k3);
-        if (mask) mask[j] = m;
-    }
+    const uint32_t key = group_key(m, k3);
+    if (live) keys[j] = key;
+    sort_hist_add(key, live, j, hist, ntile);
     __syncthreads();
     if (threadIdx.x < k3) block_counts[int64_t(threadIdx.x) * nblk + blockIdx.x] = s_cnt[threadIdx.x];
 }
@@ -349,47 +528,66 @@ struct KmapWs {
     int32_t *block_counts;
     int64_t *block_offsets;
     int64_t *k_total;
-    int32_t *iota;
     uint32_t *keys;
-    uint32_t *sorted_keys;
-    void *cub_tmp;
-    size_t cub_bytes;
+    uint32_t *keys_tmp;
+    int32_t *vals_tmp;
+    int32_t *hist;    // two histograms of 256 x ntile, cleared before the keys are computed
+    int32_t *totals;  // per-digit totals of each pass
+    int ntile;
+    size_t hist_bytes;
     size_t total;
 };
 
 static KmapWs carve_kmap_ws(void *base, int64_t n_out, int k3) {
     KmapWs w{};
     const int nblk = int((n_out + kQueryThreads - 1) / kQueryThreads);
+    w.ntile = int((n_out + kSortTile - 1) / kSortTile);
     Carver cv(base);
     w.block_counts = cv.take<int32_t>(size_t(k3) * nblk);
     w.block_offsets = cv.take<int64_t>(size_t(k3) * nblk);
     w.k_total = cv.take<int64_t>(size_t(k3));
-    w.iota = cv.take<int32_t>(size_t(n_out));
     w.keys = cv.take<uint32_t>(size_t(n_out));
-    w.sorted_keys = cv.take<uint32_t>(size_t(n_out));
-    size_t cub_bytes = 0;
-    cub::DeviceRadixSort::SortPairs(nullptr, cub_bytes, (const uint32_t *)nullptr, (uint32_t *)nullptr,
-                                    (const int32_t *)nullptr, (int32_t *)nullptr, int(n_out), 0, 32);
-    w.cub_bytes = cub_bytes;
-    w.cub_tmp = cv.take<char>(cub_bytes);
+    w.keys_tmp = cv.take<uint32_t>(size_t(n_out));
+    w.vals_tmp = cv.take<int32_t>(size_t(n_out));
+    w.hist_bytes = sizeof(int32_t) * 2 * 256 * size_t(w.ntile);
+    w.hist = cv.take<int32_t>(2 * 256 * size_t(w.ntile));
+    w.totals = cv.take<int32_t>(2 * 256);
     w.total = align_up(cv.used, 256);
     return w;
 }
 
-// Scan the per-block counts, emit the pair lists, sort rows by mask and OR the tile masks.
+// Scan the per-block counts, emit the pair lists, sort the rows by grouping key
+// (perm) and OR the tile masks.  The keys and the first sort histogram are in w.
 static lat_status finish_kmap(lat_kmap *map, int k3, int nblk, KmapWs &w, int32_t *d_status, cudaStream_t s) {
     const int64_t n_out = map->n_out;
     kmap_scan_kernel<<<k3, 1024, 0, s>>>(w.block_counts, w.block_offsets, nblk, w.k_total);
     LAT_CUDA_TRY(cudaGetLastError());
-    kmap_emit_kernel<<<nblk, kQueryThreads, 0, s>>>(map->nbr, n_out, k3, w.block_offsets, w.k_total, nblk,
+    kmap_emit_kernel<<<nblk, kQueryThreads, 0, s>>>(map->nbr, map->mask, n_out, k3, w.block_offsets, w.k_total, nblk,
                                                      map->pair_in, map->pair_out, map->pair_capacity, map->pair_off,
                                                      d_status);
     LAT_CUDA_TRY(cudaGetLastError());
-    size_t cub_bytes = w.cub_bytes;
-    LAT_CUDA_TRY(cub::DeviceRadixSort::SortPairs(w.cub_tmp, cub_bytes, w.keys, w.sorted_keys, w.iota, map->perm,
-                                                 int(n_out), 0, group_key_bits(k3), s));
     const int64_t ntiles = (n_out + LAT_TILE_ROWS - 1) / LAT_TILE_ROWS;
-    tile_mask_kernel<<<unsigned((ntiles + 7) / 8), 256, 0, s>>>(map->mask, map->perm, n_out, map->tile_mask, ntiles);
+    LAT_CUDA_TRY(cudaMemsetAsync(map->tile_mask, 0, sizeof(uint32_t) * size_t(ntiles), s));
+    const int64_t hsize = 256 * int64_t(w.ntile);
+    int32_t *h1 = w.hist, *h2 = w.hist + hsize;
+    int32_t *t1 = w.totals, *t2 = w.totals + 256;
+    sort_rowscan_kernel<<<256, 256, 0, s>>>(h1, w.ntile, t1);
+    LAT_CUDA_TRY(cudaGetLastError());
+    if (group_key_bits(k3) <= 8) {
+        sort_scatter_kernel<true><<<w.ntile, kSortThreads, 0, s>>>(w.keys, nullptr, n_out, 0, h1, t1, w.ntile,
+                                                                    nullptr, map->perm, nullptr, map->mask,
+                                                                    map->tile_mask);
+        LAT_CUDA_TRY(cudaGetLastError());
+        return LAT_OK;
+    }
+    sort_scatter_kernel<false><<<w.ntile, kSortThreads, 0, s>>>(w.keys, nullptr, n_out, 0, h1, t1, w.ntile,
+                                                                 w.keys_tmp, w.vals_tmp, h2, nullptr, nullptr);
+    LAT_CUDA_TRY(cudaGetLastError());
+    sort_rowscan_kernel<<<256, 256, 0, s>>>(h2, w.ntile, t2);
+    LAT_CUDA_TRY(cudaGetLastError());
+    sort_scatter_kernel<true><<<w.ntile, kSortThreads, 0, s>>>(w.keys_tmp, w.vals_tmp, n_out, 8, h2, t2, w.ntile,
+                                                                nullptr, map->perm, nullptr, map->mask,
+                                                                map->tile_mask);
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }
@@ -434,12 +632,12 @@ extern "C" lat_status lat_kmap_query(const void *table, size_t table_bytes, cons
     int k3 = 0;
     if (!map || !geom_ok(geom, k3) || map->k3 != k3 || !map_buffers_ok(map)) return LAT_ERR_ARG;
     const int64_t n_out = map->n_out, n_in = map->n_in;
-    if (!table || table_bytes % sizeof(Slot) || !pow2(table_bytes / sizeof(Slot)) ||
-        table_bytes / sizeof(Slot) > (uint64_t(1) << 31))
+    if (!table || table_bytes % kSlotBytes || !pow2(table_bytes / kSlotBytes) || table_bytes / kSlotBytes < 64 ||
+        table_bytes / kSlotBytes > (uint64_t(1) << 31))
         return LAT_ERR_ARG;
     if (n_out > 0 && !out_coords) return LAT_ERR_ARG;
     if (geom->mode == LAT_SUBM && n_in != n_out) return LAT_ERR_ARG;  // the support is preserved
-    if (reinterpret_cast<uintptr_t>(out_coords) % 16 || reinterpret_cast<uintptr_t>(table) % 16) return LAT_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(out_coords) % 16 || reinterpret_cast<uintptr_t>(table) % 64) return LAT_ERR_ARG;
     const KmapWs need = carve_kmap_ws(nullptr, n_out, k3);
     if (ws_bytes < need.total || (need.total && !ws)) return LAT_ERR_WORKSPACE;
     map->mode = geom->mode;
@@ -478,8 +676,9 @@ extern "C" lat_status lat_kmap_query(const void *table, size_t table_bytes, cons
                 g.delta[k] = dx * (1ll << 32) + dy * (1ll << 16) + dz;
             }
     const int nblk = int((n_out + kQueryThreads - 1) / kQueryThreads);
-    const uint32_t cap_mask = uint32_t(table_bytes / sizeof(Slot) - 1);
-    const Slot *slots = static_cast<const Slot *>(table);
+    LAT_CUDA_TRY(cudaMemsetAsync(w.hist, 0, w.hist_bytes, s));
+    const uint32_t cap_mask = uint32_t(table_bytes / kSlotBytes - 1);
+    const SlotGroup *slots = static_cast<const SlotGroup *>(table);
     const int4 *oc = reinterpret_cast<const int4 *>(out_coords);
     if (geom->mode == LAT_SUBM) {
         // the upper half of the table is filled by mirrored hits only
@@ -487,16 +686,17 @@ extern "C" lat_status lat_kmap_query(const void *table, size_t table_bytes, cons
         if (centre + 1 < k3)
             LAT_CUDA_TRY(cudaMemsetAsync(map->nbr + int64_t(centre + 1) * n_out, 0xFF,
                                          sizeof(int32_t) * size_t(k3 - 1 - centre) * n_out, s));
+        LAT_CUDA_TRY(cudaMemsetAsync(map->mask, 0, sizeof(uint32_t) * size_t(n_out), s));
         kmap_probe_kernel<true><<<nblk, kQueryThreads, 0, s>>>(slots, cap_mask, oc, n_out, n_in, g, map->nbr,
-                                                               map->mask, w.keys, w.iota, w.block_counts, nblk,
-                                                               d_status);
+                                                               map->mask, w.keys, w.hist, w.ntile, w.block_counts,
+                                                               nblk, d_status);
         LAT_CUDA_TRY(cudaGetLastError());
-        kmap_count_kernel<<<nblk, kQueryThreads, 0, s>>>(map->nbr, n_out, k3, w.iota, w.block_counts, nblk,
-                                                          map->mask, w.keys);
+        kmap_count_kernel<<<nblk, kQueryThreads, 0, s>>>(map->mask, n_out, k3, w.block_counts, nblk, w.keys, w.hist,
+                                                          w.ntile);
     } else {
         kmap_probe_kernel<false><<<nblk, kQueryThreads, 0, s>>>(slots, cap_mask, oc, n_out, n_in, g, map->nbr,
-                                                                map->mask, w.keys, w.iota, w.block_counts, nblk,
-                                                                d_status);
+                                                                map->mask, w.keys, w.hist, w.ntile, w.block_counts,
+                                                                nblk, d_status);
     }
     LAT_CUDA_TRY(cudaGetLastError());
     return finish_kmap(map, k3, nblk, w, d_status, s);
@@ -550,8 +750,9 @@ extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int
         }
         KmapWs w = carve_kmap_ws(ws, map->n_out, k3);
         const int nblk = int((map->n_out + kQueryThreads - 1) / kQueryThreads);
-        kmap_count_kernel<<<nblk, kQueryThreads, 0, s>>>(map->nbr, map->n_out, k3, w.iota, w.block_counts, nblk,
-                                                          nullptr, w.keys);
+        LAT_CUDA_TRY(cudaMemsetAsync(w.hist, 0, w.hist_bytes, s));
+        kmap_count_kernel<<<nblk, kQueryThreads, 0, s>>>(map->mask, map->n_out, k3, w.block_counts, nblk, w.keys,
+                                                          w.hist, w.ntile);
         LAT_CUDA_TRY(cudaGetLastError());
         const lat_status st = finish_kmap(map, k3, nblk, w, d_status, s);
         if (st != LAT_OK) return st;

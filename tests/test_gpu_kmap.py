@@ -34,6 +34,14 @@ def _slot_hash(key: int) -> int:
     return h
 
 
+def _table_slots(table):
+    """(key, row) of every slot of a table of 64-byte groups {key[4], row[4], unused[4]}."""
+    g = table.cpu().numpy().view(np.uint8).reshape(-1, 64)
+    keys = np.ascontiguousarray(g[:, :32]).view(np.uint64).reshape(-1)
+    rows = np.ascontiguousarray(g[:, 32:48]).view(np.uint32).reshape(-1).astype(np.int64)
+    return keys, rows
+
+
 def _subm(coords, ks=(3, 3, 3), d_status=None):
     c = _dev(coords)
     table = scv.hash_table(c, 2.0, d_status)
@@ -48,8 +56,7 @@ def test_hash_table_places_every_key_reachably():
     st = scv.new_status()
     table = scv.hash_table(_dev(coords), 2.0, st)
     scv.check_status(st)
-    t = table.cpu().numpy().view(np.uint64).reshape(-1, 2)
-    keys, rows = t[:, 0], (t[:, 1] & np.uint64(0xFFFFFFFF)).astype(np.int64)
+    keys, rows = _table_slots(table)
     cap = len(keys)
     empty = np.uint64(0xFFFFFFFFFFFFFFFF)
     occupied = np.nonzero(keys != empty)[0]
@@ -58,9 +65,9 @@ def test_hash_table_places_every_key_reachably():
     for s in occupied:
         k = int(keys[s])
         assert want[k] == rows[s]
-        home = _slot_hash(k) & (cap - 1)
-        d = (s - home) % cap                       # linear probing: no empty slot between home and s
-        assert all(keys[(home + e) % cap] != empty for e in range(d))
+        start = _slot_hash(k) & (cap - 1) & ~3     # probing starts at the home slot's 4-slot group
+        d = (s - start) % cap                      # linear probing: no empty slot between start and s
+        assert all(keys[(start + e) % cap] != empty for e in range(d))
 
 
 def test_hash_flags_duplicates_and_keeps_lowest_row():
@@ -68,9 +75,9 @@ def test_hash_flags_duplicates_and_keeps_lowest_row():
     st = scv.new_status()
     table = scv.hash_table(_dev(coords), 2.0, st)
     assert scv.lat_status_fetch(st) & 4
-    t = table.cpu().numpy().view(np.uint64).reshape(-1, 2)
+    keys, rows = _table_slots(table)
     k = np.uint64(oracle.pack_key(0, 1, 2, 3))
-    assert int(t[t[:, 0] == k, 1][0] & np.uint64(0xFFFFFFFF)) == 0
+    assert int(rows[keys == k][0]) == 0
 
 
 def test_hash_flags_out_of_range_coordinates():
