@@ -9,8 +9,9 @@
 // The proposals are made unique and put in canonical (b, x, y, z) order, so
 // the result does not depend on the input row order.
 //
-// Two ways to sort + unique, chosen after one pass that finds the range of
-// every coarse field:
+// Two ways to sort + unique; one pass finds the range of every coarse field
+// and the first is launched right behind it (its kernels read the range on
+// the device), the second runs only when the first reports it did not apply:
 //   * counting sort on a bitmap: when the fields, shifted to start at their
 //     minimum, pack into a key of at most 30 bits and the bitmap is no larger
 //     than max(2^24, 512 bits per proposal), every proposal sets its bit, a
@@ -20,7 +21,6 @@
 // Both can also report each input's coarse row (its parent) when K == stride
 // and pad == 0.
 #include <cub/device/device_radix_sort.cuh>
-#include <cub/device/device_scan.cuh>
 #include <cub/device/device_select.cuh>
 
 #include <climits>
@@ -143,56 +143,168 @@ struct Compact {
     }
 };
 
+// Bitmap plan from the device-side field ranges: the compact layout, the
+// group count (1024 bits per group), whether the bitmap path applies (ok) and
+// whether there is no coarse row at all (empty).  Every bitmap kernel derives
+// it itself, so the host does not wait for the range pass.
+struct Plan {
+    Compact cp;
+    int64_t ngroups;
+    bool ok, empty;
+};
+__device__ __forceinline__ Plan make_plan(const int *__restrict__ range, int64_t budget_bits) {
+    Plan p;
+    p.empty = __ldg(range) == INT_MAX;
+    int total = 0;
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        const int lo = __ldg(range + a), hi = __ldg(range + 4 + a);
+        const int64_t span = p.empty ? 0 : int64_t(hi) - lo;
+        p.cp.mn[a] = lo;
+        p.cp.w[a] = span > 0 ? 64 - __clzll(span) : 0;
+        total += p.cp.w[a];
+    }
+    p.ok = !p.empty && total <= kMaxBitmapBits && (int64_t(1) << total) <= budget_bits;
+    p.ngroups = p.ok ? max(int64_t(1), (int64_t(1) << total) / 1024) : 0;
+    return p;
+}
+
 __global__ void __launch_bounds__(256)
-bitmap_mark_kernel(const uint64_t *__restrict__ keys, int64_t items, Compact cp, uint32_t *__restrict__ bitmap) {
+bitmap_zero_kernel(const int *__restrict__ range, int64_t budget_bits, uint4 *__restrict__ bitmap) {
+    const Plan p = make_plan(range, budget_bits);
+    const int64_t n4 = p.ngroups * 8;  // 32 words per group
+    for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < n4; e += int64_t(gridDim.x) * blockDim.x)
+        bitmap[e] = make_uint4(0, 0, 0, 0);
+}
+
+__global__ void __launch_bounds__(256)
+bitmap_mark_kernel(const uint64_t *__restrict__ keys, int64_t items, const int *__restrict__ range,
+                   int64_t budget_bits, uint32_t *__restrict__ bitmap) {
     const int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
     if (e >= items) return;
+    const Plan p = make_plan(range, budget_bits);
+    if (!p.ok) return;
     const uint64_t key = keys[e];
     if (key == kEmptyKey) return;
-    const uint32_t v = cp.pack(key);
+    const uint32_t v = p.cp.pack(key);
     atomicOr(bitmap + (v >> 5), 1u << (v & 31));
 }
 
-// set bits per group of 32 words (1024 bits)
+// Set bits per group of 32 words (1024 bits), and per block of 256 groups.
 __global__ void __launch_bounds__(256)
-bitmap_count_kernel(const uint32_t *__restrict__ bitmap, int64_t ngroups, int32_t *__restrict__ grp_cnt) {
+bitmap_count_kernel(const uint32_t *__restrict__ bitmap, const int *__restrict__ range, int64_t budget_bits,
+                    int32_t *__restrict__ grp_cnt, int32_t *__restrict__ blk_cnt) {
+    __shared__ int s_warp[8];
+    const Plan p = make_plan(range, budget_bits);
+    if (int64_t(blockIdx.x) * 256 >= p.ngroups) return;
     const int64_t gi = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
-    if (gi >= ngroups) return;
-    const uint4 *w4 = reinterpret_cast<const uint4 *>(bitmap + gi * 32);
     int c = 0;
+    if (gi < p.ngroups) {
+        const uint4 *w4 = reinterpret_cast<const uint4 *>(bitmap + gi * 32);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        const uint4 v = __ldg(w4 + e);
-        c += __popc(v.x) + __popc(v.y) + __popc(v.z) + __popc(v.w);
+        for (int e = 0; e < 8; ++e) {
+            const uint4 v = __ldg(w4 + e);
+            c += __popc(v.x) + __popc(v.y) + __popc(v.z) + __popc(v.w);
+        }
+        grp_cnt[gi] = c;
     }
-    grp_cnt[gi] = c;
+    int sum = c;
+    for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+    if ((threadIdx.x & 31) == 0) s_warp[threadIdx.x >> 5] = sum;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int t = 0;
+        for (int w = 0; w < 8; ++w) t += s_warp[w];
+        blk_cnt[blockIdx.x] = t;
+    }
 }
 
-// Coordinates of the set bits in bit order (= canonical order); also the total count.
+// Exclusive scan of the per-block counts (one block), the coarse row count, and
+// whether the bitmap path produced the result (path_ok; 0 = use the sort path).
+__global__ void __launch_bounds__(1024)
+bitmap_blockscan_kernel(const int *__restrict__ range, int64_t budget_bits, const int32_t *__restrict__ blk_cnt,
+                        int64_t *__restrict__ blk_off, int64_t *__restrict__ n_out_dev, int *__restrict__ path_ok) {
+    __shared__ int64_t s_warp[32];
+    const Plan p = make_plan(range, budget_bits);
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const int64_t nblk = (p.ngroups + 255) / 256;
+    const int64_t per = (nblk + 1023) / 1024;
+    const int64_t b0 = min(nblk, t * per), b1 = min(nblk, b0 + per);
+    int64_t sum = 0;
+    for (int64_t i = b0; i < b1; ++i) sum += blk_cnt[i];
+    int64_t incl = sum;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int64_t o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += o;
+    }
+    if (lane == 31) s_warp[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+        int64_t x = s_warp[lane];
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int64_t o = __shfl_up_sync(0xFFFFFFFFu, x, d);
+            if (lane >= d) x += o;
+        }
+        s_warp[lane] = x;
+    }
+    __syncthreads();
+    int64_t run = (w ? s_warp[w - 1] : 0) + incl - sum;
+    for (int64_t i = b0; i < b1; ++i) {
+        blk_off[i] = run;
+        run += blk_cnt[i];
+    }
+    if (t == 0) {
+        *n_out_dev = p.ok ? s_warp[31] : 0;
+        *path_ok = (p.ok || p.empty) ? 1 : 0;
+    }
+}
+
+// Coordinates of the set bits in bit order (= canonical order); each group's
+// first rank (grp_off) for the parent pass.
 __global__ void __launch_bounds__(256)
-bitmap_emit_kernel(const uint32_t *__restrict__ bitmap, int64_t ngroups, const int32_t *__restrict__ grp_cnt,
-                   const int64_t *__restrict__ grp_off, Compact cp, int4 *__restrict__ out, int64_t capacity,
-                   int64_t *__restrict__ n_out_dev) {
+bitmap_emit_kernel(const uint32_t *__restrict__ bitmap, const int *__restrict__ range, int64_t budget_bits,
+                   const int32_t *__restrict__ grp_cnt, const int64_t *__restrict__ blk_off,
+                   int64_t *__restrict__ grp_off, int4 *__restrict__ out, int64_t capacity) {
+    __shared__ int s_warp[8];
+    const Plan p = make_plan(range, budget_bits);
+    if (int64_t(blockIdx.x) * 256 >= p.ngroups) return;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int64_t gi = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
-    if (gi >= ngroups) return;
-    if (gi == ngroups - 1) *n_out_dev = grp_off[gi] + grp_cnt[gi];
-    if (grp_cnt[gi] == 0) return;
-    int64_t rank = grp_off[gi];
+    const int c = gi < p.ngroups ? grp_cnt[gi] : 0;
+    int incl = c;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += o;
+    }
+    if (lane == 31) s_warp[w] = incl;
+    __syncthreads();
+    int before = 0;
+    for (int q = 0; q < w; ++q) before += s_warp[q];
+    if (gi >= p.ngroups) return;
+    int64_t rank = blk_off[blockIdx.x] + before + incl - c;
+    grp_off[gi] = rank;
+    if (c == 0) return;
     for (int wi = 0; wi < 32; ++wi) {
         uint32_t word = bitmap[gi * 32 + wi];
         while (word) {
             const int b = __ffs(word) - 1;
             word &= word - 1;
-            if (rank < capacity) out[rank] = cp.unpack(uint32_t(gi * 1024 + wi * 32 + b));
+            if (rank < capacity) out[rank] = p.cp.unpack(uint32_t(gi * 1024 + wi * 32 + b));
             ++rank;
         }
     }
 }
 
 // Rank of each input's (single) proposal among the set bits: its coarse row.
+// Inputs without a coarse row get -1; nothing else is written when the bitmap
+// path does not apply (the sort path fills parent then).
 __global__ void __launch_bounds__(256)
-bitmap_parent_kernel(const uint64_t *__restrict__ keys, int64_t n, Compact cp, const uint32_t *__restrict__ bitmap,
-                     const int64_t *__restrict__ grp_off, int32_t *__restrict__ parent) {
+bitmap_parent_kernel(const uint64_t *__restrict__ keys, int64_t n, const int *__restrict__ range,
+                     int64_t budget_bits, const uint32_t *__restrict__ bitmap, const int64_t *__restrict__ grp_off,
+                     int32_t *__restrict__ parent) {
     const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
     if (i >= n) return;
     const uint64_t key = keys[i];
@@ -200,7 +312,9 @@ bitmap_parent_kernel(const uint64_t *__restrict__ keys, int64_t n, Compact cp, c
         parent[i] = -1;
         return;
     }
-    const uint32_t v = cp.pack(key);
+    const Plan p = make_plan(range, budget_bits);
+    if (!p.ok) return;
+    const uint32_t v = p.cp.pack(key);
     const uint32_t gi = v >> 10, wi = (v >> 5) & 31;
     int64_t rank = grp_off[gi];
     for (uint32_t e = 0; e < wi; ++e) rank += __popc(__ldg(bitmap + gi * 32 + e));
@@ -272,8 +386,9 @@ struct DownWs {
     uint32_t *bitmap;
     int32_t *grp_cnt;
     int64_t *grp_off;
-    void *scan_tmp;
-    size_t scan_bytes;
+    int32_t *blk_cnt;
+    int64_t *blk_off;
+    int *path_ok;
     int64_t max_groups;
     size_t total;
 };
@@ -284,6 +399,7 @@ static DownWs carve_down_ws(void *base, int64_t items) {
     w.keys = cv.take<uint64_t>(size_t(items));
     w.range = cv.take<int>(8);
     w.n_out_dev = cv.take<int64_t>(1);
+    w.path_ok = cv.take<int>(1);
     const size_t common = cv.used;
     // sort path
     w.sorted = cv.take<uint64_t>(size_t(items));
@@ -303,17 +419,11 @@ static DownWs carve_down_ws(void *base, int64_t items) {
     w.bitmap = cv.take<uint32_t>(size_t(w.max_groups) * 32);
     w.grp_cnt = cv.take<int32_t>(size_t(w.max_groups));
     w.grp_off = cv.take<int64_t>(size_t(w.max_groups));
-    cub::DeviceScan::ExclusiveSum(nullptr, w.scan_bytes, (const int32_t *)nullptr, (int64_t *)nullptr,
-                                  int(w.max_groups));
-    w.scan_tmp = cv.take<char>(w.scan_bytes);
+    const int64_t max_blk = (w.max_groups + 255) / 256;
+    w.blk_cnt = cv.take<int32_t>(size_t(max_blk));
+    w.blk_off = cv.take<int64_t>(size_t(max_blk));
     w.total = align_up(std::max(sort_end, cv.used), 256);
     return w;
-}
-
-static int bit_width(int64_t span) {  // bits to hold values 0..span
-    int b = 0;
-    while ((int64_t(1) << b) <= span) ++b;
-    return b;
 }
 
 }  // namespace lat
@@ -354,40 +464,40 @@ extern "C" lat_status lat_downsample_coords(const int32_t *coords, int64_t n_in,
     down_candidates_kernel<<<in_blocks, 256, 0, s>>>(reinterpret_cast<const int4 *>(coords), n_in, g, w.keys, w.range,
                                                      d_status);
     LAT_CUDA_TRY(cudaGetLastError());
-    int range[8];
-    LAT_CUDA_TRY(cudaMemcpyAsync(range, w.range, sizeof(range), cudaMemcpyDeviceToHost, s));
+    // ---------------------------------------------------- counting sort on a bitmap
+    // Launched without waiting for the range: every kernel derives the plan on
+    // the device, grids cover the largest bitmap the budget allows, and the
+    // result says whether the path applied (else the sort path below runs).
+    const int64_t budget = bitmap_budget_bits(items);
+    const unsigned gblocks = unsigned((w.max_groups + 255) / 256);
+    const unsigned zblocks = unsigned(std::min<int64_t>((w.max_groups * 8 + 255) / 256, int64_t(num_sms()) * 8));
+    bitmap_zero_kernel<<<zblocks, 256, 0, s>>>(w.range, budget, reinterpret_cast<uint4 *>(w.bitmap));
+    LAT_CUDA_TRY(cudaGetLastError());
+    bitmap_mark_kernel<<<item_blocks, 256, 0, s>>>(w.keys, items, w.range, budget, w.bitmap);
+    LAT_CUDA_TRY(cudaGetLastError());
+    bitmap_count_kernel<<<gblocks, 256, 0, s>>>(w.bitmap, w.range, budget, w.grp_cnt, w.blk_cnt);
+    LAT_CUDA_TRY(cudaGetLastError());
+    bitmap_blockscan_kernel<<<1, 1024, 0, s>>>(w.range, budget, w.blk_cnt, w.blk_off, w.n_out_dev, w.path_ok);
+    LAT_CUDA_TRY(cudaGetLastError());
+    bitmap_emit_kernel<<<gblocks, 256, 0, s>>>(w.bitmap, w.range, budget, w.grp_cnt, w.blk_off, w.grp_off,
+                                               reinterpret_cast<int4 *>(out_coords), out_capacity);
+    LAT_CUDA_TRY(cudaGetLastError());
+    if (parent) {
+        bitmap_parent_kernel<<<in_blocks, 256, 0, s>>>(w.keys, n_in, w.range, budget, w.bitmap, w.grp_off, parent);
+        LAT_CUDA_TRY(cudaGetLastError());
+    }
+    struct {
+        int64_t m;
+        int ok;
+    } res{0, 0};
+    LAT_CUDA_TRY(cudaMemcpyAsync(&res.m, w.n_out_dev, sizeof(int64_t), cudaMemcpyDeviceToHost, s));
+    LAT_CUDA_TRY(cudaMemcpyAsync(&res.ok, w.path_ok, sizeof(int), cudaMemcpyDeviceToHost, s));
     LAT_CUDA_TRY(cudaStreamSynchronize(s));
-    if (range[0] == INT_MAX) {  // no coarse row exists
-        if (parent) LAT_CUDA_TRY(cudaMemsetAsync(parent, 0xFF, sizeof(int32_t) * n_in, s));
-        return LAT_OK;
+    if (res.ok) {
+        *n_out = res.m;
+        return res.m > out_capacity ? LAT_ERR_CAPACITY : LAT_OK;
     }
-    Compact cp;
-    int total_bits = 0;
-    for (int a = 0; a < 4; ++a) {
-        cp.mn[a] = range[a];
-        cp.w[a] = bit_width(int64_t(range[4 + a]) - range[a]);
-        total_bits += cp.w[a];
-    }
-    const int64_t bits = total_bits <= kMaxBitmapBits ? (int64_t(1) << total_bits) : 0;
-    if (total_bits <= kMaxBitmapBits && bits <= bitmap_budget_bits(items)) {
-        // ------------------------------------------------ counting sort on a bitmap
-        const int64_t ngroups = std::max<int64_t>(1, bits / 1024);
-        LAT_CUDA_TRY(cudaMemsetAsync(w.bitmap, 0, sizeof(uint32_t) * size_t(ngroups) * 32, s));
-        bitmap_mark_kernel<<<item_blocks, 256, 0, s>>>(w.keys, items, cp, w.bitmap);
-        LAT_CUDA_TRY(cudaGetLastError());
-        const unsigned gblocks = unsigned((ngroups + 255) / 256);
-        bitmap_count_kernel<<<gblocks, 256, 0, s>>>(w.bitmap, ngroups, w.grp_cnt);
-        LAT_CUDA_TRY(cudaGetLastError());
-        size_t sb = w.scan_bytes;
-        LAT_CUDA_TRY(cub::DeviceScan::ExclusiveSum(w.scan_tmp, sb, w.grp_cnt, w.grp_off, int(ngroups), s));
-        bitmap_emit_kernel<<<gblocks, 256, 0, s>>>(w.bitmap, ngroups, w.grp_cnt, w.grp_off, cp,
-                                                   reinterpret_cast<int4 *>(out_coords), out_capacity, w.n_out_dev);
-        LAT_CUDA_TRY(cudaGetLastError());
-        if (parent) {
-            bitmap_parent_kernel<<<in_blocks, 256, 0, s>>>(w.keys, n_in, cp, w.bitmap, w.grp_off, parent);
-            LAT_CUDA_TRY(cudaGetLastError());
-        }
-    } else {
+    {
         // ------------------------------------------------ radix sort + unique of the packed keys
         size_t b = w.sort_bytes;
         LAT_CUDA_TRY(cub::DeviceRadixSort::SortKeys(w.sort_tmp, b, w.keys, w.sorted, int(items), 0, 64, s));

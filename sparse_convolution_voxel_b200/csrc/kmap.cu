@@ -68,8 +68,9 @@ inline int group_key_bits(int k3) { return k3 <= 8 ? k3 : kGroupKeyBits; }
 // the stable argsort of the keys, deterministic.  The last pass also ORs every
 // row's mask into its tile of LAT_TILE_ROWS output positions.
 constexpr int kSortThreads = 256;
-constexpr int kSortRounds = 8;
+constexpr int kSortRounds = 2;
 constexpr int kSortTile = kSortThreads * kSortRounds;
+static_assert(kSortTile >= 512, "next-pass tag packs the output tile in 22 bits");
 constexpr int kSortWarps = kSortThreads / 32;
 
 // Adds the lowest digit of this lane's key to the first pass's histogram.  Every
@@ -467,7 +468,8 @@ sort_scatter_kernel(const uint32_t *__restrict__ keys_in, const int32_t *__restr
                 vals_out[dst] = val[r];
             }
             const uint32_t d2 = (key[r] >> (shift + 8)) & 255u;
-            const uint32_t tag = live ? ((d2 << 20) | uint32_t(dst / kSortTile)) : (0x80000000u | lane);
+            // output tile < 2^31 / kSortTile <= 2^22, digit < 2^8: the tag fits in 30 bits
+            const uint32_t tag = live ? ((d2 << 22) | uint32_t(dst / kSortTile)) : (0x80000000u | lane);
             const unsigned p2 = __match_any_sync(0xFFFFFFFFu, tag);
             if (live && (p2 & lt) == 0) atomicAdd(hist_next + int64_t(d2) * ntile + dst / kSortTile, int(__popc(p2)));
         }
