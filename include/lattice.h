@@ -255,8 +255,10 @@ lat_status lat_sconv_dgrad(const void *dy, int32_t cout, const void *w, int32_t 
 
 /* Per-offset weight gradient: dW[k] = sum over pairs (i, j) of offset k of
  * x[i]^T dy[j], fp32 (k3, cin, cout), from the forward map's pair lists.
- * Deterministic: fixed chunks of pairs, each reduced into a partial in fp32,
- * partials summed in a fixed order (no atomics). */
+ * Deterministic: the pairs are cut into chunks whose size depends only on
+ * the pair count, each chunk is reduced into an fp32 partial, and the
+ * partials are summed in a fixed order (no atomics), so the bits do not
+ * depend on timing or on the number of SMs. */
 lat_status lat_sconv_wgrad(const void *x, int32_t cin, const void *dy, int32_t cout,
                            const lat_kmap *map, float *dw, lat_dtype dtype, void *ws,
                            size_t ws_bytes, int32_t *d_status, lat_stream stream);
@@ -268,9 +270,12 @@ lat_status lat_sconv_wgrad(const void *x, int32_t cin, const void *dy, int32_t c
  * that runs while a stream is captured into a CUDA graph without memory
  * nodes, real-time loops that must not allocate (cudaMalloc / cudaFree can
  * synchronise the whole device) once running, or hosts whose device
- * allocator belongs to another runtime.  This entry point computes the same
- * dW as lat_sconv_wgrad (same kernels, same chunking, same summation order)
- * but takes no `ws`: its scratch is one static device array of
+ * allocator belongs to another runtime.  This entry point computes dW with
+ * the CUDA-core weight-gradient kernels (those lat_sconv_wgrad runs for fp32
+ * and for the shapes the tensor cores do not take; same chunking, same
+ * summation order, so the same bits there; for the tensor-core shapes of
+ * lat_sconv_wgrad the two agree within fp32 rounding, not bit for bit) and
+ * takes no `ws`: its scratch is one static device array of
  * LAT_WGRAD_STATIC_SCRATCH_BYTES (32 MiB) inside the library, which every
  * GPU that loads the library keeps until the process exits.  It allocates
  * nothing and calls no allocating routine.

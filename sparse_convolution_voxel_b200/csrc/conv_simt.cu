@@ -147,16 +147,24 @@ conv_simt_kernel(const T *__restrict__ x, int cin, const T *__restrict__ w, int 
 }
 
 // Work units of the weight gradient: fixed chunks of kWgradChunk pairs inside one offset.
+// First unit of every offset and the total (unit_base[k3]); one warp, lane k
+// handles offset k (k3 <= 32): offset k's clamped pairs make ceil(P_k / chunk) units.
 __global__ void wgrad_units_kernel(const int64_t *__restrict__ pair_off, int k3, int64_t capacity, int chunk,
                                    int32_t *__restrict__ unit_base) {
-    if (threadIdx.x != 0 || blockIdx.x != 0) return;
-    int32_t u = 0;
-    for (int k = 0; k < k3; ++k) {
-        unit_base[k] = u;
-        const int64_t lo = min(pair_off[k], capacity), hi = min(pair_off[k + 1], capacity);
-        u += int32_t((hi - lo + chunk - 1) / chunk);
+    const int lane = threadIdx.x & 31;
+    const int64_t P = min(pair_off[k3], capacity);
+    const int64_t lo = lane < k3 ? min(pair_off[lane], capacity) : P;
+    const int64_t up = __shfl_down_sync(0xFFFFFFFFu, lo, 1);
+    const int64_t hi = lane == 31 ? P : up;
+    const int32_t units = lane < k3 ? int32_t((hi - lo + chunk - 1) / chunk) : 0;
+    int32_t incl = units;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += o;
     }
-    unit_base[k3] = u;
+    if (lane < k3) unit_base[lane] = incl - units;
+    if (lane == 31) unit_base[k3] = incl;
 }
 
 // One block of 8 warps per (unit, group of slices).  A slice is 256 consecutive

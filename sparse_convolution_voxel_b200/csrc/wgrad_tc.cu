@@ -3,14 +3,18 @@
 //
 // Per offset this is a GEMM with M = Cin, N = Cout and the pairs as the
 // reduction dimension.  The pairs of each offset (grouped and ordered by the
-// kernel-map query) are cut into fixed chunks of kChunk pairs; one persistent
-// CTA per SM takes chunks round-robin.  For every 64-pair block of a chunk,
-// four gather warps copy the 64 x rows and 64 dy rows with 16-byte cp.async
-// into 128-byte swizzled MN-major tiles (rows of the gathered operands are
-// the reduction dimension, channels are contiguous), and one thread issues 4
-// tcgen05.mma (K = 16 pairs each) into a TMEM accumulator.  Four epilogue
-// warps write the chunk's fp32 partial; a second kernel sums the partials of
-// each offset in chunk order.  No atomics, so dW is deterministic.
+// kernel-map query) are cut into chunks whose size depends only on the total
+// pair count P (chunk_pairs: about kTargetUnits chunks in all, whatever the
+// GPU); persistent CTAs (two per SM) take chunks round-robin.  For every
+// 64-pair block of a chunk, four gather warps copy the 64 x rows and 64 dy
+// rows with 16-byte cp.async into 128-byte swizzled MN-major tiles (rows of
+// the gathered operands are the reduction dimension, channels are
+// contiguous); the copies arrive on the stage barrier by themselves
+// (cp.async.mbarrier.arrive.noinc), and one thread issues 4 tcgen05.mma
+// (K = 16 pairs each) into a TMEM accumulator.  Four epilogue warps write the
+// chunk's fp32 partial; a second kernel sums the partials of each offset in a
+// fixed order (32 interleaved lanes over the chunks, then the lanes in order).
+// No atomics, so dW is deterministic and does not depend on the SM count.
 #include "common.cuh"
 #include "conv_common.cuh"
 #include "tc_ptx.cuh"
@@ -19,7 +23,8 @@ namespace lat {
 namespace wtc {
 
 constexpr int kKP = 64;            // pairs per stage (GEMM K block)
-constexpr int kChunk = 2048;       // pairs per work unit
+constexpr int kTargetUnits = 448;  // chunks of all offsets together, about
+constexpr int kMinChunk = 256;     // pairs per chunk at least
 constexpr int kProdWarps = 4, kEpiWarps = 4;
 constexpr int kMmaWarp = kProdWarps + kEpiWarps;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
@@ -32,7 +37,6 @@ struct Cfg {
     static constexpr uint32_t kStage = kABytes + kBBytes;
     // about 96 KB of stages so that two CTAs share an SM
     static constexpr int kStages = kStage <= 16384 ? 6 : (kStage <= 24576 ? 4 : 3);
-    static constexpr int kLag = kStages - 1 < 3 ? kStages - 1 : 3;  // cp.async groups in flight per thread
     static constexpr uint32_t kSmem = kStages * kStage + 256 + 1024;
     static constexpr uint32_t kTmemCols = 2 * N;
 };
@@ -48,26 +52,48 @@ __host__ __device__ constexpr uint32_t make_idesc() {
            (1u << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
 
+// Pairs per chunk for P pairs in all: at least kMinChunk, a multiple of 64, and
+// large enough that the chunks of all offsets number at most kTargetUnits + k3.
+__host__ __device__ __forceinline__ int64_t chunk_pairs(int64_t P) {
+    const int64_t c = (P + kTargetUnits - 1) / kTargetUnits;
+    const int64_t r = (c + 63) / 64 * 64;
+    return r > kMinChunk ? r : kMinChunk;
+}
+
 // First unit of every offset (and the total in ub[k3]): offset k's clamped pairs
-// are cut into ceil(P_k / kChunk) units, numbered in offset order.
+// are cut into ceil(P_k / chunk) units, numbered in offset order; ub[k3 + 1] =
+// chunk.  Called by one full warp (lane k handles offset k, k3 <= 32).
 __device__ __forceinline__ void unit_bases(const int64_t *pair_off, int64_t capacity, int k3, int32_t *ub) {
-    int32_t u = 0;
-    for (int k = 0; k < k3; ++k) {
-        ub[k] = u;
-        const int64_t lo = min(pair_off[k], capacity), hi = min(pair_off[k + 1], capacity);
-        u += int32_t((hi - lo + kChunk - 1) / kChunk);
+    const int lane = threadIdx.x & 31;
+    const int64_t P = min(pair_off[k3], capacity);
+    const int64_t chunk = chunk_pairs(P);
+    const int64_t lo = lane < k3 ? min(pair_off[lane], capacity) : P;
+    const int64_t up = __shfl_down_sync(0xFFFFFFFFu, lo, 1);
+    const int64_t hi = lane == 31 ? P : up;  // offset k ends where offset k+1 starts (P after the last)
+    const int32_t units = lane < k3 ? int32_t((hi - lo + chunk - 1) / chunk) : 0;
+    int32_t incl = units;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += o;
     }
-    ub[k3] = u;
+    if (lane < k3) ub[lane] = incl - units;
+    const int32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+    if (lane == 0) {
+        ub[k3] = total;
+        ub[k3 + 1] = int32_t(chunk);
+    }
 }
 
 // Unit u covers pairs [lo, hi) of offset k.
 __device__ __forceinline__ void unit_range(const int32_t *unit_base, const int64_t *pair_off, int64_t capacity,
                                            int k3, int32_t u, int &k, int64_t &lo, int64_t &hi) {
+    const int64_t chunk = unit_base[k3 + 1];
     k = 0;
     while (k + 1 < k3 && unit_base[k + 1] <= u) ++k;
     const int64_t base = min(pair_off[k], capacity);
-    lo = base + int64_t(u - unit_base[k]) * kChunk;
-    hi = min(lo + kChunk, min(pair_off[k + 1], capacity));
+    lo = base + int64_t(u - unit_base[k]) * chunk;
+    hi = min(lo + chunk, min(pair_off[k + 1], capacity));
 }
 
 template <typename T, int M, int N>
@@ -77,7 +103,6 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
                 int64_t n_in, int64_t n_out, float *__restrict__ partial, int32_t *d_status) {
     using C = Cfg<M, N>;
     constexpr int NS = C::kStages;
-    constexpr int kLag = C::kLag;
     constexpr uint32_t idesc = make_idesc<T, M, N>();
 
     extern __shared__ uint8_t smem_raw[];
@@ -88,11 +113,11 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
     uint64_t *accempty = accfull + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accempty + 2);
     __shared__ int s_abort;
-    __shared__ int32_t unit_base[33];
+    __shared__ int32_t unit_base[34];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (warp == 1) unit_bases(pair_off, capacity, k3, unit_base);
     if (tid == 0) {
-        unit_bases(pair_off, capacity, k3, unit_base);
         for (int s = 0; s < NS; ++s) {
             ptx::mbar_init(&full[s], kProdWarps * 32);
             ptx::mbar_init(&empty[s], 1);
@@ -168,18 +193,11 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
                         ptx::cp_async16(Bs + nb * 8192 + off, src, jj >= 0 ? 16u : 0u);
                     }
                 }
-                ptx::cp_async_commit();
-                if (it >= kLag) {
-                    ptx::cp_async_wait<kLag>();
-                    ptx::fence_proxy_async_smem();
-                    ptx::mbar_arrive(&full[(it - kLag) % NS]);
-                }
+                ptx::cp_async_arrive_noinc(&full[s]);
                 ++it;
             }
         }
         ptx::cp_async_wait<0>();
-        ptx::fence_proxy_async_smem();
-        for (uint32_t d = (it > kLag ? it - kLag : 0); d < it; ++d) ptx::mbar_arrive(&full[d % NS]);
         if (!ok) s_abort = 1;
     } else if (warp < kMmaWarp) {
         // ------------------------------------------------------------ epilogue: partial of each unit
@@ -253,6 +271,9 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
                     break;
                 }
                 ptx::tc_fence_after();
+                // the gathered rows were written by cp.async (generic proxy);
+                // order them before the tensor core's async-proxy reads
+                ptx::fence_proxy_async_smem();
                 const uint32_t as = ptx::smem_u32(smem + s * C::kStage);
                 const uint32_t bs = as + C::kABytes;
 #pragma unroll
@@ -284,30 +305,51 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
     }
 }
 
-__global__ void wgrad_tc_reduce_kernel(const float *__restrict__ partial, const int64_t *__restrict__ pair_off,
-                                       int64_t capacity, int k3, int nelem, float *__restrict__ dw) {
-    __shared__ int32_t unit_base[33];
-    if (threadIdx.x == 0) unit_bases(pair_off, capacity, k3, unit_base);
+// dW[k] = sum of offset k's chunk partials.  Block (x, k): 32 unit lanes x 8
+// groups of 4 elements; lane l sums chunks l, l+32, ... in order, then lane 0
+// adds the 32 lane sums in order -- a fixed order whatever the timing.
+constexpr int kRedLanes = 32;
+__global__ void __launch_bounds__(256)
+wgrad_tc_reduce_kernel(const float *__restrict__ partial, const int64_t *__restrict__ pair_off, int64_t capacity,
+                       int k3, int nelem, float *__restrict__ dw) {
+    __shared__ int32_t unit_base[34];
+    __shared__ float4 s_part[kRedLanes][8];
+    if (threadIdx.x < 32) unit_bases(pair_off, capacity, k3, unit_base);
     __syncthreads();
     const int k = blockIdx.y;
-    const int el = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
-    if (k >= k3 || el >= nelem) return;
-    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int32_t u = unit_base[k]; u < unit_base[k + 1]; ++u) {
-        const float4 v = __ldg(reinterpret_cast<const float4 *>(partial + int64_t(u) * nelem + el));
-        s.x += v.x;
-        s.y += v.y;
-        s.z += v.z;
-        s.w += v.w;
+    const int g = threadIdx.x & 7, l = threadIdx.x >> 3;
+    const int el = (blockIdx.x * 8 + g) * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (el < nelem) {
+#pragma unroll 4
+        for (int32_t u = unit_base[k] + l; u < unit_base[k + 1]; u += kRedLanes) {
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(partial + int64_t(u) * nelem + el));
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
+        }
     }
-    *reinterpret_cast<float4 *>(dw + int64_t(k) * nelem + el) = s;
+    s_part[l][g] = acc;
+    __syncthreads();
+    if (l == 0 && el < nelem) {
+        float4 t = s_part[0][g];
+        for (int q = 1; q < kRedLanes; ++q) {
+            const float4 v = s_part[q][g];
+            t.x += v.x;
+            t.y += v.y;
+            t.z += v.z;
+            t.w += v.w;
+        }
+        *reinterpret_cast<float4 *>(dw + int64_t(k) * nelem + el) = t;
+    }
 }
 
 template <typename T, int M, int N>
 static lat_status launch(const void *x, const void *dy, const lat_kmap *map, float *dw, void *ws, int32_t *d_status,
                          cudaStream_t s) {
     using C = Cfg<M, N>;
-    const int64_t units_max = (map->pair_capacity + kChunk - 1) / kChunk + map->k3;
+    const int64_t units_max = int64_t(kTargetUnits) + map->k3;
     Carver cv(ws);
     float *partial = cv.take<float>(size_t(units_max) * M * N);
     auto kern = wgrad_tc_kernel<T, M, N>;
@@ -318,7 +360,7 @@ static lat_status launch(const void *x, const void *dy, const lat_kmap *map, flo
                                                     map->k3, map->n_in, map->n_out, partial, d_status);
     LAT_CUDA_TRY(cudaGetLastError());
     const int nelem = M * N;
-    dim3 rg((nelem / 4 + 255) / 256, map->k3);
+    dim3 rg((nelem + 31) / 32, map->k3);
     wgrad_tc_reduce_kernel<<<rg, 256, 0, s>>>(partial, map->pair_off, map->pair_capacity, map->k3, nelem, dw);
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
@@ -329,7 +371,7 @@ static lat_status launch(const void *x, const void *dy, const lat_kmap *map, flo
 bool wgrad_tc_supported(int cin, int cout) { return (cin == 64 || cin == 128) && (cout == 64 || cout == 128); }
 
 size_t wgrad_tc_ws_bytes(int cin, int cout, const lat_kmap *map) {
-    const int64_t units_max = (map->pair_capacity + wtc::kChunk - 1) / wtc::kChunk + map->k3;
+    const int64_t units_max = int64_t(wtc::kTargetUnits) + map->k3;
     Carver cv(nullptr);
     cv.take<float>(size_t(units_max) * cin * cout);
     return align_up(cv.used, 256);
