@@ -93,7 +93,10 @@ def make_inputs(rank: int):
 class Pipeline:
     """Preallocated buffers + the sequence of C-ABI calls of one step."""
 
-    PHASES = ["hash", "kmap", "fwd", "dgrad", "wgrad", "downsample", "down_maps", "down_fwd", "up_fwd"]
+    # The coarse support is enqueued right after the kernel map (it needs only the
+    # coordinates) and its row count is read after the submanifold passes are
+    # enqueued, so the GPU runs those while the host waits for the count.
+    PHASES = ["hash", "kmap", "downsample", "fwd", "dgrad", "wgrad", "down_maps", "down_fwd", "up_fwd"]
 
     def __init__(self, host: dict, dev: torch.device):
         import sparse_convolution_voxel_b200 as scv
@@ -128,6 +131,8 @@ class Pipeline:
                             scv.lat_sconv_ws_bytes(0, CIN, CMID, self.km_down.c, torch.half),
                             scv.lat_sconv_ws_bytes(0, CMID, CIN, self.km_up.c, torch.half))
         self.wsb = self.ws.get(self.ws_bytes)
+        self.nc_host = torch.empty(1, dtype=torch.int64, pin_memory=True)
+        self.nc_ready = torch.cuda.Event()
         self.pairs = None
 
     def step(self, ev=None):
@@ -139,13 +144,20 @@ class Pipeline:
         rec(1)
         scv.lat_kmap_query(self.table, d["coords"], self.g_sub, self.km.c, self.wsb, s)
         rec(2)
-        scv.lat_sconv_fwd(d["x"], d["w"], self.km.c, self.y, self.wsb, s)
+        # coarse support (one stream: the passes below reuse the workspace only after it has run)
+        scv.lat_downsample_coords_async(d["coords"], self.g_down, self.coarse_buf, self.wsb, self.nc_host, s,
+                                        parent=self.parent)
+        self.nc_ready.record()
         rec(3)
-        scv.lat_sconv_dgrad(d["g"], d["w"], self.km.c, True, self.dx, self.wsb, s)
+        scv.lat_sconv_fwd(d["x"], d["w"], self.km.c, self.y, self.wsb, s)
         rec(4)
-        scv.lat_sconv_wgrad(d["x"], d["g"], self.km.c, self.dw, self.wsb, s)
+        scv.lat_sconv_dgrad(d["g"], d["w"], self.km.c, True, self.dx, self.wsb, s)
         rec(5)
-        nc = scv.lat_downsample_coords(d["coords"], self.g_down, self.coarse_buf, self.wsb, s, parent=self.parent)
+        scv.lat_sconv_wgrad(d["x"], d["g"], self.km.c, self.dw, self.wsb, s)
+        self.nc_ready.synchronize()
+        nc = int(self.nc_host[0])
+        if nc < 0:  # coarse fields too wide for the bitmap: blocking radix-sort path
+            nc = scv.lat_downsample_coords(d["coords"], self.g_down, self.coarse_buf, self.wsb, s, parent=self.parent)
         assert nc == self.nc
         rec(6)
         scv.lat_kmap_from_parent(d["coords"], self.parent, self.g_down, self.km_down.c, self.km_up.c, self.wsb, s)

@@ -186,10 +186,12 @@ lat_status lat_kmap_query(const void *table, size_t table_bytes, const int32_t *
  * {stride*q + (ix,iy,iz) - pad} holds at least one active input, batch
  * unchanged.  Written to out_coords (int32 (out_capacity, 4)) sorted by packed
  * key, i.e. in canonical (b, x, y, z) order, so the result is deterministic.
- * geom->mode must be LAT_STRIDED.  Synchronises `stream` (twice: once for the
- * coordinate range, which picks a bitmap counting sort when the coarse fields
- * pack into at most 30 bits, else a radix sort) and writes the row count to
- * *n_out (HOST pointer).  out_capacity >= n_in is enough when ksize == stride
+ * geom->mode must be LAT_STRIDED.  A bitmap counting sort runs when the
+ * coarse fields, shifted to their minimum, pack into at most 30 bits (and the
+ * bitmap fits the budget of max(2^24, 512 bits per candidate)); otherwise a
+ * radix sort of the packed keys.  Synchronises `stream` once (twice when the
+ * radix sort is needed) and writes the row count to *n_out (HOST pointer).
+ * out_capacity >= n_in is enough when ksize == stride
  * and pad == 0; in general n_in * prod(ceil(ksize/stride)) bounds the count.
  * Too small a capacity returns LAT_ERR_CAPACITY with the needed count in
  * *n_out.  parent (device int32 [n_in], may be NULL) receives the coarse row
@@ -200,6 +202,19 @@ lat_status lat_downsample_coords(const int32_t *coords, int64_t n_in, const lat_
                                  int32_t *out_coords, int64_t out_capacity, int64_t *n_out,
                                  int32_t *parent, void *ws, size_t ws_bytes, int32_t *d_status,
                                  lat_stream stream);
+
+/* The same support without waiting: enqueues the bitmap counting sort and a
+ * copy of the row count into *n_out_host, then returns.  n_out_host should be
+ * pinned host memory (cudaHostAlloc), else the copy may synchronise.  Once
+ * `stream` has passed this point (an event recorded after the call), *n_out_host
+ * holds the row count, or -1 when the coarse fields do not fit the bitmap:
+ * then call lat_downsample_coords with the same arguments.  Rows beyond
+ * out_capacity are not written; a count above out_capacity means the buffer
+ * was too small.  out_coords, parent and ws must stay untouched until then. */
+lat_status lat_downsample_coords_async(const int32_t *coords, int64_t n_in, const lat_geom *geom,
+                                       int32_t *out_coords, int64_t out_capacity, int64_t *n_out_host,
+                                       int32_t *parent, void *ws, size_t ws_bytes, int32_t *d_status,
+                                       lat_stream stream);
 
 /* Both kernel maps of a strided Conv3d with ksize == stride and pad == 0,
  * built from the parent rows that lat_downsample_coords reports instead of by

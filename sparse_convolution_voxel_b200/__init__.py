@@ -17,14 +17,14 @@ import torch
 
 from ._lib import (  # noqa: F401  (re-exported C entry points and constants)
     EXPORTS, LAT_BF16, LAT_F16, LAT_F32, LAT_OK, LAT_OP_DGRAD, LAT_OP_FWD, LAT_OP_WGRAD, LAT_STRIDED, LAT_SUBM,
-    LAT_TILE_ROWS, LAT_TRANSPOSED, LIB_PATH, LatticeError, lat_downsample_coords, lat_downsample_ws_bytes, lat_geom,
+    LAT_TILE_ROWS, LAT_TRANSPOSED, LIB_PATH, LatticeError, lat_downsample_coords, lat_downsample_coords_async, lat_downsample_ws_bytes, lat_geom,
     lat_hash_build, lat_hash_bytes, lat_kmap, lat_kmap_from_parent, lat_kmap_from_parent_ws_bytes, lat_kmap_query,
     lat_kmap_ws_bytes, lat_sconv_dgrad, lat_sconv_fwd,
     lat_sconv_wgrad, lat_sconv_wgrad_static, lat_sconv_ws_bytes, lat_status_fetch, lat_status_string, lat_version, load, make_geom,
 )
 
 __all__ = [
-    "KernelMap", "Workspace", "hash_table", "kernel_map", "downsample", "maps_from_parent", "conv_fwd", "conv_dgrad", "conv_wgrad",
+    "KernelMap", "Workspace", "hash_table", "kernel_map", "downsample", "downsample_async", "PendingDownsample", "maps_from_parent", "conv_fwd", "conv_dgrad", "conv_wgrad",
     "subm_geom", "strided_geom", "target_geom", "transposed_geom", "check_status", "new_status",
 ] + EXPORTS
 
@@ -121,6 +121,51 @@ def kernel_map(table: torch.Tensor, n_in: int, out_coords: torch.Tensor, geom: l
     ws = ws or Workspace(out_coords.device)
     lat_kmap_query(table, out_coords, geom, km.c, ws.get(lat_kmap_ws_bytes(km.n_out, k3)), d_status, stream)
     return km
+
+
+class PendingDownsample:
+    """A downsample enqueued by downsample_async; result() waits for the coarse row count."""
+
+    def __init__(self, coords, geom, out, parent, host, event, ws_t, d_status, stream):
+        self._args = (coords, geom, out, parent, ws_t, d_status, stream)
+        self._host, self._event = host, event
+
+    def count(self) -> int:
+        """Coarse row count (waits for the stream to pass the downsample)."""
+        coords, geom, out, parent, ws_t, d_status, stream = self._args
+        self._event.synchronize()
+        m = int(self._host[0])
+        if m < 0:  # coarse fields too wide for the bitmap: the blocking radix-sort path
+            m = lat_downsample_coords(coords, geom, out, ws_t, d_status, stream, parent=parent)
+            self._host[0] = m
+        elif m > out.shape[0]:
+            raise LatticeError(16, "lat_downsample_coords_async")
+        return m
+
+    def result(self):
+        """(coarse coords, parent) like downsample(..., with_parent=True), or the coords alone."""
+        m = self.count()
+        coords, _, out, parent, _, _, _ = self._args
+        return (out[:m], parent[:coords.shape[0]]) if parent is not None else out[:m]
+
+
+def downsample_async(coords: torch.Tensor, geom: lat_geom, ws: Workspace | None = None, d_status=None,
+                     capacity: int | None = None, stream=None, with_parent: bool = False) -> PendingDownsample:
+    """Enqueue the coarse support (and parents) without waiting for the row count."""
+    n = coords.shape[0]
+    per = 1
+    for a in range(3):
+        per *= -(-geom.ksize[a] // geom.stride[a])
+    cap = n * per if capacity is None else int(capacity)
+    out = torch.empty((max(1, cap), 4), dtype=torch.int32, device=coords.device)
+    parent = torch.empty(max(1, n), dtype=torch.int32, device=coords.device) if with_parent else None
+    ws = ws or Workspace(coords.device)
+    ws_t = ws.get(lat_downsample_ws_bytes(n, geom))
+    host = torch.empty(1, dtype=torch.int64, pin_memory=True)
+    lat_downsample_coords_async(coords, geom, out, ws_t, host, d_status, stream, parent=parent)
+    event = torch.cuda.Event()
+    event.record(stream if stream is not None else torch.cuda.current_stream())
+    return PendingDownsample(coords, geom, out, parent, host, event, ws_t, d_status, stream)
 
 
 def downsample(coords: torch.Tensor, geom: lat_geom, ws: Workspace | None = None, d_status=None,

@@ -31,7 +31,8 @@ STATUS_BITS = {
 # every symbol include/lattice.h declares
 EXPORTS = [
     "lat_hash_bytes", "lat_hash_build", "lat_kmap_ws_bytes", "lat_kmap_query",
-    "lat_downsample_ws_bytes", "lat_downsample_coords", "lat_kmap_from_parent_ws_bytes", "lat_kmap_from_parent",
+    "lat_downsample_ws_bytes", "lat_downsample_coords", "lat_downsample_coords_async", "lat_kmap_from_parent_ws_bytes",
+    "lat_kmap_from_parent",
     "lat_sconv_ws_bytes", "lat_sconv_fwd",
     "lat_sconv_dgrad", "lat_sconv_wgrad", "lat_sconv_wgrad_static", "lat_status_fetch", "lat_status_string", "lat_version",
 ]
@@ -77,6 +78,7 @@ def load() -> ctypes.CDLL:
         "lat_kmap_query": (I32, [P, SZ, P, G, K, P, SZ, P, P]),
         "lat_downsample_ws_bytes": (SZ, [I64, G]),
         "lat_downsample_coords": (I32, [P, I64, G, P, I64, ctypes.POINTER(I64), P, P, SZ, P, P]),
+        "lat_downsample_coords_async": (I32, [P, I64, G, P, I64, P, P, P, SZ, P, P]),
         "lat_kmap_from_parent_ws_bytes": (SZ, [I64, I64, I32]),
         "lat_kmap_from_parent": (I32, [P, P, G, K, K, P, SZ, P, P]),
         "lat_sconv_ws_bytes": (SZ, [I32, I32, I32, K, I32]),
@@ -166,6 +168,19 @@ def lat_downsample_coords(coords: torch.Tensor, geom: lat_geom, out_coords: torc
                                       _stream(stream))
     _check(rc, "lat_downsample_coords")
     return int(n.value)
+
+
+def lat_downsample_coords_async(coords: torch.Tensor, geom: lat_geom, out_coords: torch.Tensor,
+                                ws: torch.Tensor | None, n_out_host: torch.Tensor, d_status: torch.Tensor | None = None,
+                                stream=None, parent: torch.Tensor | None = None) -> None:
+    """Enqueue the downsample; n_out_host (pinned host int64[1]) receives the count (-1: use the blocking call)."""
+    if n_out_host.device.type != "cpu" or n_out_host.dtype != torch.int64 or n_out_host.numel() < 1:
+        raise ValueError("n_out_host must be a host int64 tensor")
+    rc = load().lat_downsample_coords_async(_ptr(coords), coords.shape[0], ctypes.byref(geom), _ptr(out_coords),
+                                            out_coords.shape[0], ctypes.c_void_p(n_out_host.data_ptr()), _ptr(parent),
+                                            _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                                            _ptr(d_status), _stream(stream))
+    _check(rc, "lat_downsample_coords_async")
 
 
 def lat_kmap_from_parent_ws_bytes(n_fine: int, n_coarse: int, k3: int) -> int:

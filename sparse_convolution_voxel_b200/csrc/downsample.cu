@@ -219,11 +219,11 @@ bitmap_count_kernel(const uint32_t *__restrict__ bitmap, const int *__restrict__
     }
 }
 
-// Exclusive scan of the per-block counts (one block), the coarse row count, and
-// whether the bitmap path produced the result (path_ok; 0 = use the sort path).
+// Exclusive scan of the per-block counts (one block) and the coarse row count,
+// or -1 when the bitmap path does not apply (the sort path must run).
 __global__ void __launch_bounds__(1024)
 bitmap_blockscan_kernel(const int *__restrict__ range, int64_t budget_bits, const int32_t *__restrict__ blk_cnt,
-                        int64_t *__restrict__ blk_off, int64_t *__restrict__ n_out_dev, int *__restrict__ path_ok) {
+                        int64_t *__restrict__ blk_off, int64_t *__restrict__ n_out_dev) {
     __shared__ int64_t s_warp[32];
     const Plan p = make_plan(range, budget_bits);
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
@@ -255,10 +255,7 @@ bitmap_blockscan_kernel(const int *__restrict__ range, int64_t budget_bits, cons
         blk_off[i] = run;
         run += blk_cnt[i];
     }
-    if (t == 0) {
-        *n_out_dev = p.ok ? s_warp[31] : 0;
-        *path_ok = (p.ok || p.empty) ? 1 : 0;
-    }
+    if (t == 0) *n_out_dev = p.ok ? s_warp[31] : (p.empty ? 0 : -1);
 }
 
 // Coordinates of the set bits in bit order (= canonical order); each group's
@@ -388,7 +385,6 @@ struct DownWs {
     int64_t *grp_off;
     int32_t *blk_cnt;
     int64_t *blk_off;
-    int *path_ok;
     int64_t max_groups;
     size_t total;
 };
@@ -399,7 +395,6 @@ static DownWs carve_down_ws(void *base, int64_t items) {
     w.keys = cv.take<uint64_t>(size_t(items));
     w.range = cv.take<int>(8);
     w.n_out_dev = cv.take<int64_t>(1);
-    w.path_ok = cv.take<int>(1);
     const size_t common = cv.used;
     // sort path
     w.sorted = cv.take<uint64_t>(size_t(items));
@@ -436,38 +431,44 @@ extern "C" size_t lat_downsample_ws_bytes(int64_t n_in, const lat_geom *geom) {
     return lat::carve_down_ws(nullptr, std::max<int64_t>(items, 1)).total;
 }
 
-extern "C" lat_status lat_downsample_coords(const int32_t *coords, int64_t n_in, const lat_geom *geom,
-                                            int32_t *out_coords, int64_t out_capacity, int64_t *n_out,
-                                            int32_t *parent, void *ws, size_t ws_bytes, int32_t *d_status,
-                                            lat_stream stream) {
-    using namespace lat;
-    DownGeom g;
-    if (!n_out || n_in < 0 || out_capacity < 0 || !down_geom(geom, g)) return LAT_ERR_ARG;
+namespace lat {
+
+// Checks shared by both entry points; fills g, w, items.  LAT_OK with items == 0
+// means there is nothing to do (no input row).
+static lat_status down_prepare(const int32_t *coords, int64_t n_in, const lat_geom *geom, int32_t *out_coords,
+                               int64_t out_capacity, int32_t *parent, void *ws, size_t ws_bytes, DownGeom &g,
+                               DownWs &w, int64_t &items) {
+    items = 0;
+    if (n_in < 0 || out_capacity < 0 || !down_geom(geom, g)) return LAT_ERR_ARG;
     if (n_in > 0 && (!coords || (out_capacity > 0 && !out_coords))) return LAT_ERR_ARG;
     if (reinterpret_cast<uintptr_t>(coords) % 16 || reinterpret_cast<uintptr_t>(out_coords) % 16) return LAT_ERR_ARG;
     if (parent) {  // one coarse row per input only when the kernel tiles the stride exactly
         for (int a = 0; a < 3; ++a)
             if (g.ks[a] != g.st[a] || g.pd[a] != 0) return LAT_ERR_UNSUPPORTED;
     }
-    const int64_t items = n_in * g.cands;
-    if (items >= (int64_t(1) << 31)) return LAT_ERR_UNSUPPORTED;
-    *n_out = 0;
+    const int64_t n_items = n_in * g.cands;
+    if (n_items >= (int64_t(1) << 31)) return LAT_ERR_UNSUPPORTED;
     if (n_in == 0) return LAT_OK;
-    const DownWs need = carve_down_ws(nullptr, items);
+    const DownWs need = carve_down_ws(nullptr, n_items);
     if (!ws || ws_bytes < need.total) return LAT_ERR_WORKSPACE;
-    DownWs w = carve_down_ws(ws, items);
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const unsigned in_blocks = unsigned((n_in + 255) / 256), item_blocks = unsigned((items + 255) / 256);
+    w = carve_down_ws(ws, n_items);
+    items = n_items;
+    return LAT_OK;
+}
 
+// Range pass and the bitmap counting-sort path, launched without waiting for
+// the range: every kernel derives the plan on the device, grids cover the
+// largest bitmap the budget allows, and w.n_out_dev ends up holding the coarse
+// row count, or -1 when the path did not apply.
+static lat_status enqueue_bitmap_path(const int32_t *coords, int64_t n_in, const DownGeom &g, int64_t items,
+                                      int32_t *out_coords, int64_t out_capacity, int32_t *parent, const DownWs &w,
+                                      int32_t *d_status, cudaStream_t s) {
+    const unsigned in_blocks = unsigned((n_in + 255) / 256), item_blocks = unsigned((items + 255) / 256);
     range_init_kernel<<<1, 32, 0, s>>>(w.range);
     LAT_CUDA_TRY(cudaGetLastError());
     down_candidates_kernel<<<in_blocks, 256, 0, s>>>(reinterpret_cast<const int4 *>(coords), n_in, g, w.keys, w.range,
                                                      d_status);
     LAT_CUDA_TRY(cudaGetLastError());
-    // ---------------------------------------------------- counting sort on a bitmap
-    // Launched without waiting for the range: every kernel derives the plan on
-    // the device, grids cover the largest bitmap the budget allows, and the
-    // result says whether the path applied (else the sort path below runs).
     const int64_t budget = bitmap_budget_bits(items);
     const unsigned gblocks = unsigned((w.max_groups + 255) / 256);
     const unsigned zblocks = unsigned(std::min<int64_t>((w.max_groups * 8 + 255) / 256, int64_t(num_sms()) * 8));
@@ -477,7 +478,7 @@ extern "C" lat_status lat_downsample_coords(const int32_t *coords, int64_t n_in,
     LAT_CUDA_TRY(cudaGetLastError());
     bitmap_count_kernel<<<gblocks, 256, 0, s>>>(w.bitmap, w.range, budget, w.grp_cnt, w.blk_cnt);
     LAT_CUDA_TRY(cudaGetLastError());
-    bitmap_blockscan_kernel<<<1, 1024, 0, s>>>(w.range, budget, w.blk_cnt, w.blk_off, w.n_out_dev, w.path_ok);
+    bitmap_blockscan_kernel<<<1, 1024, 0, s>>>(w.range, budget, w.blk_cnt, w.blk_off, w.n_out_dev);
     LAT_CUDA_TRY(cudaGetLastError());
     bitmap_emit_kernel<<<gblocks, 256, 0, s>>>(w.bitmap, w.range, budget, w.grp_cnt, w.blk_off, w.grp_off,
                                                reinterpret_cast<int4 *>(out_coords), out_capacity);
@@ -486,18 +487,32 @@ extern "C" lat_status lat_downsample_coords(const int32_t *coords, int64_t n_in,
         bitmap_parent_kernel<<<in_blocks, 256, 0, s>>>(w.keys, n_in, w.range, budget, w.bitmap, w.grp_off, parent);
         LAT_CUDA_TRY(cudaGetLastError());
     }
-    struct {
-        int64_t m;
-        int ok;
-    } res{0, 0};
-    LAT_CUDA_TRY(cudaMemcpyAsync(&res.m, w.n_out_dev, sizeof(int64_t), cudaMemcpyDeviceToHost, s));
-    LAT_CUDA_TRY(cudaMemcpyAsync(&res.ok, w.path_ok, sizeof(int), cudaMemcpyDeviceToHost, s));
+    return LAT_OK;
+}
+
+}  // namespace lat
+
+extern "C" lat_status lat_downsample_coords(const int32_t *coords, int64_t n_in, const lat_geom *geom,
+                                            int32_t *out_coords, int64_t out_capacity, int64_t *n_out,
+                                            int32_t *parent, void *ws, size_t ws_bytes, int32_t *d_status,
+                                            lat_stream stream) {
+    using namespace lat;
+    if (!n_out) return LAT_ERR_ARG;
+    DownGeom g;
+    DownWs w;
+    int64_t items = 0;
+    const lat_status st = down_prepare(coords, n_in, geom, out_coords, out_capacity, parent, ws, ws_bytes, g, w, items);
+    if (st != LAT_OK) return st;
+    *n_out = 0;
+    if (items == 0) return LAT_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const unsigned in_blocks = unsigned((n_in + 255) / 256), item_blocks = unsigned((items + 255) / 256);
+    const lat_status eq = enqueue_bitmap_path(coords, n_in, g, items, out_coords, out_capacity, parent, w, d_status, s);
+    if (eq != LAT_OK) return eq;
+    int64_t m = 0;
+    LAT_CUDA_TRY(cudaMemcpyAsync(&m, w.n_out_dev, sizeof(int64_t), cudaMemcpyDeviceToHost, s));
     LAT_CUDA_TRY(cudaStreamSynchronize(s));
-    if (res.ok) {
-        *n_out = res.m;
-        return res.m > out_capacity ? LAT_ERR_CAPACITY : LAT_OK;
-    }
-    {
+    if (m < 0) {
         // ------------------------------------------------ radix sort + unique of the packed keys
         size_t b = w.sort_bytes;
         LAT_CUDA_TRY(cub::DeviceRadixSort::SortKeys(w.sort_tmp, b, w.keys, w.sorted, int(items), 0, 64, s));
@@ -510,10 +525,31 @@ extern "C" lat_status lat_downsample_coords(const int32_t *coords, int64_t n_in,
             sorted_parent_kernel<<<in_blocks, 256, 0, s>>>(w.keys, n_in, w.uniq, w.n_out_dev, parent);
             LAT_CUDA_TRY(cudaGetLastError());
         }
+        LAT_CUDA_TRY(cudaMemcpyAsync(&m, w.n_out_dev, sizeof(int64_t), cudaMemcpyDeviceToHost, s));
+        LAT_CUDA_TRY(cudaStreamSynchronize(s));
     }
-    int64_t m = 0;
-    LAT_CUDA_TRY(cudaMemcpyAsync(&m, w.n_out_dev, sizeof(int64_t), cudaMemcpyDeviceToHost, s));
-    LAT_CUDA_TRY(cudaStreamSynchronize(s));
     *n_out = m;
     return m > out_capacity ? LAT_ERR_CAPACITY : LAT_OK;
+}
+
+extern "C" lat_status lat_downsample_coords_async(const int32_t *coords, int64_t n_in, const lat_geom *geom,
+                                                  int32_t *out_coords, int64_t out_capacity, int64_t *n_out_host,
+                                                  int32_t *parent, void *ws, size_t ws_bytes, int32_t *d_status,
+                                                  lat_stream stream) {
+    using namespace lat;
+    if (!n_out_host) return LAT_ERR_ARG;
+    DownGeom g;
+    DownWs w;
+    int64_t items = 0;
+    const lat_status st = down_prepare(coords, n_in, geom, out_coords, out_capacity, parent, ws, ws_bytes, g, w, items);
+    if (st != LAT_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (items == 0) {
+        *n_out_host = 0;
+        return LAT_OK;
+    }
+    const lat_status eq = enqueue_bitmap_path(coords, n_in, g, items, out_coords, out_capacity, parent, w, d_status, s);
+    if (eq != LAT_OK) return eq;
+    LAT_CUDA_TRY(cudaMemcpyAsync(n_out_host, w.n_out_dev, sizeof(int64_t), cudaMemcpyDeviceToHost, s));
+    return LAT_OK;
 }

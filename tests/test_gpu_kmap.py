@@ -224,6 +224,35 @@ def test_downsample_parent_and_maps_from_parent(lo, hi):
     check_kmap(up, oracle.kmap(ref, coords, 2, 2, 0, oracle.TRANSPOSED))
 
 
+@pytest.mark.parametrize("lo,hi", [(-10, 10), (-30000, 30000)])   # bitmap path / blocking radix-sort fallback
+def test_downsample_async_matches_blocking(lo, hi):
+    rng = np.random.default_rng(7 + abs(lo))
+    if hi - lo > 100:
+        coords = np.unique(rng.integers(lo, hi, (2000, 4)).astype(np.int32), axis=0)
+        coords[:, 0] = rng.integers(0, 2, len(coords))
+        coords = np.unique(coords, axis=0)
+        coords = coords[rng.permutation(len(coords))]
+    else:
+        coords = rand_coords(rng, 1200, lo, hi, 2)
+    c = _dev(coords)
+    g = scv.strided_geom(2, 2, 0)
+    st = scv.new_status()
+    pending = scv.downsample_async(c, g, d_status=st, with_parent=True)
+    raw = int(pending._host[0]) if pending._event.query() else None
+    coarse, parent = pending.result()
+    ref = oracle.downsample(coords, 2, 2, 0)
+    assert np.array_equal(coarse.cpu().numpy(), ref)
+    par = parent.cpu().numpy()
+    assert np.array_equal(ref[par][:, 1:], np.floor_divide(coords[:, 1:], 2))
+    scv.check_status(st)
+    if raw is not None:   # the enqueued count is the row count on the bitmap path, -1 when the fallback ran
+        assert raw == (len(ref) if hi - lo <= 100 else -1)
+    # a count above the capacity is reported (on either path), not written past the buffer
+    small = scv.downsample_async(c, g, capacity=max(1, len(ref) // 2))
+    with pytest.raises(scv.LatticeError):
+        small.count()
+
+
 def test_maps_from_parent_full_workload():
     coords = synthetic.WORKLOADS["lidar_down_up"].coords()
     c = _dev(coords)
