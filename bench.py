@@ -192,10 +192,10 @@ class Pipeline:
 
 
 # DRAM bytes per launch of a phase from one ncu capture of this workload
-# (profiles/launches_lidar_subm_step.md: the submanifold kmap query, all of its
-# kernels, cache control at ncu's default); None where no capture matches the
-# current kernels.
-PHASE_TRAFFIC = {"kmap": 60.83e6}
+# (profiles/launches_lidar_subm_step.md: the submanifold kmap query, its 8
+# kernels summed, caches not flushed between kernels); None where no capture
+# matches the current kernels.
+PHASE_TRAFFIC = {"kmap": 21.0e6}
 
 
 def flush_l2(buf: torch.Tensor):
