@@ -284,8 +284,15 @@ bitmap_emit_kernel(const uint32_t *__restrict__ bitmap, const int *__restrict__ 
     int64_t rank = blk_off[blockIdx.x] + before + incl - c;
     grp_off[gi] = rank;
     if (c == 0) return;
+    // the group's 32 words in 8 vector loads, then its set bits in order
+    uint4 g4[8];
+    const uint4 *w4 = reinterpret_cast<const uint4 *>(bitmap + gi * 32);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) g4[e] = __ldg(w4 + e);
+#pragma unroll
     for (int wi = 0; wi < 32; ++wi) {
-        uint32_t word = bitmap[gi * 32 + wi];
+        const uint4 &q = g4[wi / 4];
+        uint32_t word = (wi & 3) == 0 ? q.x : (wi & 3) == 1 ? q.y : (wi & 3) == 2 ? q.z : q.w;
         while (word) {
             const int b = __ffs(word) - 1;
             word &= word - 1;
@@ -313,9 +320,19 @@ bitmap_parent_kernel(const uint64_t *__restrict__ keys, int64_t n, const int *__
     if (!p.ok) return;
     const uint32_t v = p.cp.pack(key);
     const uint32_t gi = v >> 10, wi = (v >> 5) & 31;
+    // bits of the group before v: whole words below wi, then the low bits of word wi
+    uint4 g4[8];
+    const uint4 *w4 = reinterpret_cast<const uint4 *>(bitmap + int64_t(gi) * 32);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) g4[e] = __ldg(w4 + e);
     int64_t rank = grp_off[gi];
-    for (uint32_t e = 0; e < wi; ++e) rank += __popc(__ldg(bitmap + gi * 32 + e));
-    rank += __popc(__ldg(bitmap + (v >> 5)) & ((1u << (v & 31)) - 1u));
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        const uint4 &q = g4[e / 4];
+        const uint32_t word = (e & 3) == 0 ? q.x : (e & 3) == 1 ? q.y : (e & 3) == 2 ? q.z : q.w;
+        const uint32_t keep = uint32_t(e) < wi ? 0xFFFFFFFFu : (uint32_t(e) == wi ? (1u << (v & 31)) - 1u : 0u);
+        rank += __popc(word & keep);
+    }
     parent[i] = int32_t(rank);
 }
 
