@@ -381,6 +381,19 @@ sort_rowscan_kernel(int32_t *__restrict__ hist, int ntile, int32_t *__restrict__
     if (t == 0) totals[blockIdx.x] = carry;
 }
 
+// Pair lists written by the last sort pass when every row has at most one
+// neighbour and the key is the one-hot mask (transposed maps from parents with
+// K^3 <= 8): then the sorted order is the canonical pair order.  src == nullptr
+// means no pairs here.
+struct PairOut {
+    const int32_t *src;  // the neighbour of each row
+    int32_t *in, *out;
+    int64_t capacity;
+    int64_t *off;
+    int k3;
+    int32_t *status;
+};
+
 // One pass: scatter the rows of tile blockIdx.x by digit (key >> shift) & 255 to
 // the positions `off` gives.  vals_in == nullptr means the identity (row e).
 // LAST: write perm and OR masks into tile_mask; otherwise write the keys and
@@ -392,7 +405,7 @@ sort_scatter_kernel(const uint32_t *__restrict__ keys_in, const int32_t *__restr
                     const int32_t *__restrict__ off, const int32_t *__restrict__ totals, int ntile,
                     uint32_t *__restrict__ keys_out,
                     int32_t *__restrict__ vals_out, int32_t *__restrict__ hist_next,
-                    const uint32_t *__restrict__ mask, uint32_t *__restrict__ tile_mask) {
+                    const uint32_t *__restrict__ mask, uint32_t *__restrict__ tile_mask, PairOut po) {
     __shared__ int s_cnt[2][kSortWarps][256];
     __shared__ int s_run[256];
     __shared__ int s_wsum[kSortWarps];
@@ -430,6 +443,14 @@ sort_scatter_kernel(const uint32_t *__restrict__ keys_in, const int32_t *__restr
     int base = incl - tot;
     for (int q = 0; q < warp; ++q) base += s_wsum[q];
     s_run[t] = base + off_b;
+    // one neighbour per row (po.src): rows of key 0 have none and sort first;
+    // offset k's pairs are the rows of key 1 << k, in sorted order
+    const int zero = po.src ? __ldg(totals) : 0;
+    if (LAST && po.src && b == 0) {
+        if (t > 0 && (t & (t - 1)) == 0 && __ffs(t) - 1 < po.k3) po.off[__ffs(t) - 1] = base - zero;
+        if (t == 255) po.off[po.k3] = base + tot - zero;
+    }
+    bool over = false;
     __syncthreads();
 #pragma unroll
     for (int r = 0; r < kSortRounds; ++r) {
@@ -457,6 +478,15 @@ sort_scatter_kernel(const uint32_t *__restrict__ keys_in, const int32_t *__restr
         s_run[t] += add;
         if (LAST) {
             if (live) vals_out[dst] = val[r];
+            if (po.src && live && key[r] != 0) {
+                const int64_t pos = dst - zero;
+                if (pos < po.capacity) {
+                    po.in[pos] = __ldg(po.src + val[r]);
+                    po.out[pos] = val[r];
+                } else {
+                    over = true;
+                }
+            }
             // one atomic per (warp, output tile)
             const uint32_t tile = live ? uint32_t(dst / LAT_TILE_ROWS) : (0x80000000u | lane);
             const unsigned tp = __match_any_sync(0xFFFFFFFFu, tile);
@@ -474,6 +504,7 @@ sort_scatter_kernel(const uint32_t *__restrict__ keys_in, const int32_t *__restr
             if (live && (p2 & lt) == 0) atomicAdd(hist_next + int64_t(d2) * ntile + dst / kSortTile, int(__popc(p2)));
         }
     }
+    if (over) flag(po.status, LAT_ERR_CAPACITY);
 }
 
 // Per-(offset, block) hit counts, grouping keys and the first sort pass's
@@ -507,22 +538,33 @@ __global__ void __launch_bounds__(256)
 parent_maps_kernel(const int4 *__restrict__ fine, const int32_t *__restrict__ parent, int64_t n_fine,
                    int64_t n_coarse, int s0, int s1, int s2, int k3, int32_t *__restrict__ up_nbr,
                    uint32_t *__restrict__ up_mask, int32_t *__restrict__ down_nbr, uint32_t *__restrict__ down_mask,
-                   int32_t *d_status) {
+                   uint32_t *__restrict__ up_keys, int32_t *__restrict__ up_hist, int up_ntile, int32_t *d_status) {
     const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
-    if (i >= n_fine) return;
-    const int4 c = __ldg(fine + i);
-    const int q = __ldg(parent + i);
-    const int o0 = c.y - floordiv(c.y, s0) * s0, o1 = c.z - floordiv(c.z, s1) * s1, o2 = c.w - floordiv(c.w, s2) * s2;
-    const int k = (o0 * s1 + o1) * s2 + o2;
-    const bool ok = q >= 0 && q < n_coarse;
-    if (!ok) flag(d_status, LAT_ERR_BAD_MAP);
-    if (up_nbr) {
-        for (int kk = 0; kk < k3; ++kk) up_nbr[int64_t(kk) * n_fine + i] = (ok && kk == k) ? q : -1;
-        up_mask[i] = ok ? (1u << k) : 0u;
+    const bool live = i < n_fine;
+    uint32_t m = 0;
+    if (live) {
+        const int4 c = __ldg(fine + i);
+        const int q = __ldg(parent + i);
+        const int o0 = c.y - floordiv(c.y, s0) * s0, o1 = c.z - floordiv(c.z, s1) * s1,
+                  o2 = c.w - floordiv(c.w, s2) * s2;
+        const int k = (o0 * s1 + o1) * s2 + o2;
+        const bool ok = q >= 0 && q < n_coarse;
+        if (!ok) flag(d_status, LAT_ERR_BAD_MAP);
+        m = ok ? (1u << k) : 0u;
+        if (up_nbr) {
+            for (int kk = 0; kk < k3; ++kk) up_nbr[int64_t(kk) * n_fine + i] = (ok && kk == k) ? q : -1;
+            up_mask[i] = m;
+        }
+        if (down_nbr && ok) {
+            down_nbr[int64_t(k) * n_coarse + q] = int32_t(i);
+            atomicOr(down_mask + q, 1u << k);
+        }
     }
-    if (down_nbr && ok) {
-        down_nbr[int64_t(k) * n_coarse + q] = int32_t(i);
-        atomicOr(down_mask + q, 1u << k);
+    // transposed map with K^3 <= 8: the grouping key is the mask, and its first
+    // sort histogram is built here (every lane of the warp takes part)
+    if (up_keys) {
+        if (live) up_keys[i] = m;
+        sort_hist_add(m, live, i, up_hist, up_ntile);
     }
 }
 
@@ -578,18 +620,18 @@ static lat_status finish_kmap(lat_kmap *map, int k3, int nblk, KmapWs &w, int32_
     if (group_key_bits(k3) <= 8) {
         sort_scatter_kernel<true><<<w.ntile, kSortThreads, 0, s>>>(w.keys, nullptr, n_out, 0, h1, t1, w.ntile,
                                                                     nullptr, map->perm, nullptr, map->mask,
-                                                                    map->tile_mask);
+                                                                    map->tile_mask, PairOut{});
         LAT_CUDA_TRY(cudaGetLastError());
         return LAT_OK;
     }
     sort_scatter_kernel<false><<<w.ntile, kSortThreads, 0, s>>>(w.keys, nullptr, n_out, 0, h1, t1, w.ntile,
-                                                                 w.keys_tmp, w.vals_tmp, h2, nullptr, nullptr);
+                                                                 w.keys_tmp, w.vals_tmp, h2, nullptr, nullptr, PairOut{});
     LAT_CUDA_TRY(cudaGetLastError());
     sort_rowscan_kernel<<<256, 256, 0, s>>>(h2, w.ntile, t2);
     LAT_CUDA_TRY(cudaGetLastError());
     sort_scatter_kernel<true><<<w.ntile, kSortThreads, 0, s>>>(w.keys_tmp, w.vals_tmp, n_out, 8, h2, t2, w.ntile,
                                                                 nullptr, map->perm, nullptr, map->mask,
-                                                                map->tile_mask);
+                                                                map->tile_mask, PairOut{});
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }
@@ -706,8 +748,9 @@ extern "C" lat_status lat_kmap_query(const void *table, size_t table_bytes, cons
 
 extern "C" size_t lat_kmap_from_parent_ws_bytes(int64_t n_fine, int64_t n_coarse, int32_t k3) {
     if (n_fine < 0 || n_coarse < 0 || n_fine >= (int64_t(1) << 31) || k3 < 1 || k3 > 32) return 0;
-    const int64_t n = n_fine > n_coarse ? n_fine : n_coarse;
-    return lat::carve_kmap_ws(nullptr, n, k3).total;
+    // the strided map's workspace, then the transposed map's (its keys are built
+    // before the strided map is finished)
+    return lat::carve_kmap_ws(nullptr, n_coarse, k3).total + lat::carve_kmap_ws(nullptr, n_fine, k3).total;
 }
 
 extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int32_t *parent, const lat_geom *geom,
@@ -737,11 +780,17 @@ extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int
         }
     }
     if (up) up->mode = LAT_TRANSPOSED;
+    KmapWs w_down = carve_kmap_ws(ws, n_coarse, k3);
+    KmapWs w_up = carve_kmap_ws(static_cast<char *>(ws) + w_down.total, n_fine, k3);
+    // transposed map with K^3 <= 8: every fine row has one neighbour (its parent)
+    // and its key is the one-hot mask, so the row sort alone yields the pairs
+    const bool up_direct = up && n_fine > 0 && group_key_bits(k3) <= 8;
+    if (up_direct) LAT_CUDA_TRY(cudaMemsetAsync(w_up.hist, 0, w_up.hist_bytes, s));
     if (n_fine > 0) {
         parent_maps_kernel<<<unsigned((n_fine + 255) / 256), 256, 0, s>>>(
             reinterpret_cast<const int4 *>(fine_coords), parent, n_fine, n_coarse, geom->stride[0], geom->stride[1],
             geom->stride[2], k3, up ? up->nbr : nullptr, up ? up->mask : nullptr, down ? down->nbr : nullptr,
-            down ? down->mask : nullptr, d_status);
+            down ? down->mask : nullptr, up_direct ? w_up.keys : nullptr, w_up.hist, w_up.ntile, d_status);
         LAT_CUDA_TRY(cudaGetLastError());
     }
     for (lat_kmap *map : {down, up}) {
@@ -750,7 +799,19 @@ extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int
             LAT_CUDA_TRY(cudaMemsetAsync(map->pair_off, 0, sizeof(int64_t) * (k3 + 1), s));
             continue;
         }
-        KmapWs w = carve_kmap_ws(ws, map->n_out, k3);
+        KmapWs &w = map == down ? w_down : w_up;
+        if (map == up && up_direct) {
+            const int64_t ntiles = (map->n_out + LAT_TILE_ROWS - 1) / LAT_TILE_ROWS;
+            LAT_CUDA_TRY(cudaMemsetAsync(map->tile_mask, 0, sizeof(uint32_t) * size_t(ntiles), s));
+            sort_rowscan_kernel<<<256, 256, 0, s>>>(w.hist, w.ntile, w.totals);
+            LAT_CUDA_TRY(cudaGetLastError());
+            const PairOut po{parent, map->pair_in, map->pair_out, map->pair_capacity, map->pair_off, k3, d_status};
+            sort_scatter_kernel<true><<<w.ntile, kSortThreads, 0, s>>>(w.keys, nullptr, map->n_out, 0, w.hist,
+                                                                        w.totals, w.ntile, nullptr, map->perm, nullptr,
+                                                                        map->mask, map->tile_mask, po);
+            LAT_CUDA_TRY(cudaGetLastError());
+            continue;
+        }
         const int nblk = int((map->n_out + kQueryThreads - 1) / kQueryThreads);
         LAT_CUDA_TRY(cudaMemsetAsync(w.hist, 0, w.hist_bytes, s));
         kmap_count_kernel<<<nblk, kQueryThreads, 0, s>>>(map->mask, map->n_out, k3, w.block_counts, nblk, w.keys,
