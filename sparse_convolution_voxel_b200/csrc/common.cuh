@@ -118,6 +118,41 @@ inline int num_sms() {
 }
 inline bool pow2(uint64_t v) { return v && !(v & (v - 1)); }
 
+// A side stream for independent chains of small kernels inside one entry
+// point: fork() makes it wait for everything enqueued on `s` so far, join()
+// makes `s` wait for everything enqueued on it since.  One side stream and one
+// pair of events per host thread and device, created on first use (make that
+// first call outside a stream capture); the event fork / join also works while
+// `s` is being captured into a graph.
+struct SideStream {
+    cudaStream_t side = nullptr;
+    cudaEvent_t fork_ev = nullptr, join_ev = nullptr;
+};
+inline cudaError_t side_stream(SideStream *&out) {
+    constexpr int kMaxDev = 64;
+    thread_local SideStream per_dev[kMaxDev];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+    SideStream &ss = per_dev[dev];
+    if (!ss.side) {
+        if ((e = cudaStreamCreateWithFlags(&ss.side, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        if ((e = cudaEventCreateWithFlags(&ss.fork_ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+        if ((e = cudaEventCreateWithFlags(&ss.join_ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+    }
+    out = &ss;
+    return cudaSuccess;
+}
+inline cudaError_t side_fork(SideStream &ss, cudaStream_t s) {
+    cudaError_t e = cudaEventRecord(ss.fork_ev, s);
+    return e == cudaSuccess ? cudaStreamWaitEvent(ss.side, ss.fork_ev, 0) : e;
+}
+inline cudaError_t side_join(SideStream &ss, cudaStream_t s) {
+    cudaError_t e = cudaEventRecord(ss.join_ev, ss.side);
+    return e == cudaSuccess ? cudaStreamWaitEvent(s, ss.join_ev, 0) : e;
+}
+
 // CTAs of a persistent kernel that can be resident at once on the current device.
 // The kernels are compiled with __launch_bounds__(threads, max_per_sm), so
 // registers admit max_per_sm CTAs; shared memory admits

@@ -600,16 +600,34 @@ static KmapWs carve_kmap_ws(void *base, int64_t n_out, int k3) {
     return w;
 }
 
+static lat_status sort_rows(lat_kmap *map, int k3, KmapWs &w, cudaStream_t s);
+
 // Scan the per-block counts, emit the pair lists, sort the rows by grouping key
 // (perm) and OR the tile masks.  The keys and the first sort histogram are in w.
-static lat_status finish_kmap(lat_kmap *map, int k3, int nblk, KmapWs &w, int32_t *d_status, cudaStream_t s) {
+// The pair chain (scan, emit) and the sort chain are independent: with a side
+// stream the pair chain runs on it, concurrently with the sort on `s`.
+static lat_status finish_kmap(lat_kmap *map, int k3, int nblk, KmapWs &w, int32_t *d_status, cudaStream_t s,
+                              SideStream *side) {
     const int64_t n_out = map->n_out;
-    kmap_scan_kernel<<<k3, 1024, 0, s>>>(w.block_counts, w.block_offsets, nblk, w.k_total);
+    cudaStream_t ps = s;
+    if (side) {
+        LAT_CUDA_TRY(side_fork(*side, s));
+        ps = side->side;
+    }
+    kmap_scan_kernel<<<k3, 1024, 0, ps>>>(w.block_counts, w.block_offsets, nblk, w.k_total);
     LAT_CUDA_TRY(cudaGetLastError());
-    kmap_emit_kernel<<<nblk, kQueryThreads, 0, s>>>(map->nbr, map->mask, n_out, k3, w.block_offsets, w.k_total, nblk,
-                                                     map->pair_in, map->pair_out, map->pair_capacity, map->pair_off,
-                                                     d_status);
+    kmap_emit_kernel<<<nblk, kQueryThreads, 0, ps>>>(map->nbr, map->mask, n_out, k3, w.block_offsets, w.k_total,
+                                                      nblk, map->pair_in, map->pair_out, map->pair_capacity,
+                                                      map->pair_off, d_status);
     LAT_CUDA_TRY(cudaGetLastError());
+    const lat_status st = sort_rows(map, k3, w, s);
+    if (side) LAT_CUDA_TRY(side_join(*side, s));
+    return st;
+}
+
+// Stable row sort by grouping key -> perm, tile masks ORed by the last pass.
+static lat_status sort_rows(lat_kmap *map, int k3, KmapWs &w, cudaStream_t s) {
+    const int64_t n_out = map->n_out;
     const int64_t ntiles = (n_out + LAT_TILE_ROWS - 1) / LAT_TILE_ROWS;
     LAT_CUDA_TRY(cudaMemsetAsync(map->tile_mask, 0, sizeof(uint32_t) * size_t(ntiles), s));
     const int64_t hsize = 256 * int64_t(w.ntile);
@@ -743,7 +761,9 @@ extern "C" lat_status lat_kmap_query(const void *table, size_t table_bytes, cons
                                                                 nblk, d_status);
     }
     LAT_CUDA_TRY(cudaGetLastError());
-    return finish_kmap(map, k3, nblk, w, d_status, s);
+    SideStream *side = nullptr;
+    LAT_CUDA_TRY(side_stream(side));
+    return finish_kmap(map, k3, nblk, w, d_status, s, side);
 }
 
 extern "C" size_t lat_kmap_from_parent_ws_bytes(int64_t n_fine, int64_t n_coarse, int32_t k3) {
@@ -793,8 +813,17 @@ extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int
             down ? down->mask : nullptr, up_direct ? w_up.keys : nullptr, w_up.hist, w_up.ntile, d_status);
         LAT_CUDA_TRY(cudaGetLastError());
     }
+    // the two maps are independent once the parent scatter is done: the
+    // transposed one is finished on a side stream, concurrently with the other
+    SideStream *side = nullptr;
+    if (down && up) {
+        LAT_CUDA_TRY(side_stream(side));
+        LAT_CUDA_TRY(side_fork(*side, s));
+    }
+    const cudaStream_t main_s = s;
     for (lat_kmap *map : {down, up}) {
         if (!map) continue;
+        const cudaStream_t s = (side && map == up) ? side->side : main_s;
         if (map->n_out == 0) {
             LAT_CUDA_TRY(cudaMemsetAsync(map->pair_off, 0, sizeof(int64_t) * (k3 + 1), s));
             continue;
@@ -817,8 +846,9 @@ extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int
         kmap_count_kernel<<<nblk, kQueryThreads, 0, s>>>(map->mask, map->n_out, k3, w.block_counts, nblk, w.keys,
                                                           w.hist, w.ntile);
         LAT_CUDA_TRY(cudaGetLastError());
-        const lat_status st = finish_kmap(map, k3, nblk, w, d_status, s);
+        const lat_status st = finish_kmap(map, k3, nblk, w, d_status, s, nullptr);
         if (st != LAT_OK) return st;
     }
+    if (side) LAT_CUDA_TRY(side_join(*side, main_s));
     return LAT_OK;
 }
