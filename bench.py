@@ -203,15 +203,16 @@ def flush_l2(buf: torch.Tensor):
 
 
 class ClockSampler:
-    """SM clock and throttle reasons sampled through NVML every ~2 ms while the
-    timed region runs (read-only queries; nothing is changed on the GPU)."""
+    """SM clock and throttle reasons sampled through NVML every ~0.5 ms while the
+    timed region runs, plus one sample as it starts and one as it ends
+    (read-only queries; nothing is changed on the GPU)."""
 
     NAMES = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
              "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
              "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
              "sw_power_cap": "nvmlClocksEventReasonSwPowerCap"}
 
-    def __init__(self, device: torch.device, period_s: float = 0.002):
+    def __init__(self, device: torch.device, period_s: float = 0.0005):
         import threading
         self.period = period_s
         self.samples = []
@@ -233,22 +234,31 @@ class ClockSampler:
         except Exception:
             self.handle = None
 
-    def _run(self):
+    def _sample(self):
         nv = self.nv
+        try:
+            self.samples.append((nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM),
+                                 nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)))
+        except Exception:
+            pass
+
+    def _run(self):
         while not self.stop.is_set():
-            try:
-                self.samples.append((nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM),
-                                     nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)))
-            except Exception:
-                pass
+            self._sample()
             time.sleep(self.period)
 
     def __enter__(self):
         import threading
         if self.handle is not None:
+            self._sample()
             self.thread = threading.Thread(target=self._run, daemon=True)
             self.thread.start()
         return self
+
+    def mark_end(self):
+        """A last sample while the timed work may still be running on the GPU."""
+        if self.handle is not None:
+            self._sample()
 
     def __exit__(self, *exc):
         if self.thread is not None:
@@ -439,7 +449,7 @@ def run_only(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -493,6 +503,7 @@ def main():
         for i in range(args.steps):
             flush_l2(flush)
             pipe.step(evs[i])
+        clk.mark_end()
         torch.cuda.synchronize()
     if pg:
         pg.barrier()
