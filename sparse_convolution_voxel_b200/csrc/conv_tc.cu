@@ -389,28 +389,60 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x
             return true;
         };
         // kLook slots of (tile, mask, rows) rotate through the loop: slot s is
-        // published, its items pushed, and it is refilled with the tile kLook
-        // places later, so every row load has kLook-1 tiles of time to land.
-        // The loop over slots is unrolled; no register holding a load in
-        // flight is moved.  Tile 0 is static, tiles 1 and 2 come from one
-        // claim of two, later tiles from single claims issued one tile ahead.
+        // published, its items pushed, and refilled with a later tile, so each
+        // row load has up to kLook-1 tiles of time to land.  The loop over
+        // slots is unrolled; no register holding a load in flight is moved.
+        // Tile 0 is static; the other slots are first filled once tile 0's
+        // items are pushed, so a CTA holding a long tile does not take light
+        // tiles early.  Positions come from the counter in batches while the
+        // tiles being published are light (at most 2 offsets): 4 while more than
+        // 8 tiles per CTA remain, 2 above 2, else 1 (one tile at a time near the
+        // end keeps the CTAs balanced); the next batch is claimed when the
+        // current one is handed out.
         constexpr int kLook = 3;
+        constexpr int64_t kUnfetched = -2;
         int64_t ts[kLook];
         uint32_t ms[kLook];
         int rs[kLook][4];
-        int pair = lane == 0 ? atomicAdd(tile_counter, 2) : 0;
-        int claimed = lane == 0 ? atomicAdd(tile_counter, 1) : 0;
+        bool more = true;      // the counter may still hold tiles
+        int64_t bq = 0;        // next position of the current batch
+        int bn = 0;            // positions left in it
+        int claim_raw = 0;     // lane 0: result of the claim in flight
+        int claim_size = 0;    // its size; 0 = none in flight
+        int size_hint = 1;
+        int64_t last_q = blockIdx.x;  // last position handed out
+        auto issue_claim = [&]() {
+            if (lane == 0) claim_raw = atomicAdd(tile_counter, size_hint);
+            claim_size = size_hint;
+        };
+        auto next_q = [&]() -> int64_t {
+            if (!more) return mv.ntiles;
+            if (bn == 0) {
+                if (claim_size == 0) issue_claim();
+                bq = int64_t(gridDim.x) + __shfl_sync(kFull, claim_raw, 0);
+                bn = claim_size;
+                claim_size = 0;
+            }
+            const int64_t q = bq++;
+            --bn;
+            last_q = q;
+            if (q >= mv.ntiles) {
+                more = false;
+                return mv.ntiles;
+            }
+            if (bn == 0) issue_claim();  // the next batch, while this one is used
+            return q;
+        };
         fetch(blockIdx.x, ts[0], ms[0], rs[0]);
-        const int64_t q1 = int64_t(gridDim.x) + __shfl_sync(kFull, pair, 0);
-        fetch(ts[0] >= 0 ? q1 : mv.ntiles, ts[1], ms[1], rs[1]);
-        fetch(ts[1] >= 0 ? q1 + 1 : mv.ntiles, ts[2], ms[2], rs[2]);
-        bool more = ts[2] >= 0;  // the last fetched tile exists, so later claims may too
-        int i = 0;               // tiles published
+#pragma unroll
+        for (int sl = 1; sl < kLook; ++sl) ts[sl] = kUnfetched;
+        int i = 0;  // tiles published
         bool done = false;
         while (ok && !done) {
 #pragma unroll
             for (int sl = 0; sl < kLook; ++sl) {
                 if (done || !ok) break;
+                if (ts[sl] == kUnfetched) fetch(next_q(), ts[sl], ms[sl], rs[sl]);
                 // publish tile i for the MMA and epilogue roles
                 const int r = i % kRing;
                 if (!__all_sync(kFull, ptx::mbar_wait(&ring_empty[r], ((i / kRing) & 1) ^ 1, kWaitNs))) {
@@ -431,14 +463,17 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x
                     break;
                 }
                 for (uint32_t m = ms[sl]; m && ok; m &= m - 1) ok = push_item(__ffs(m) - 1, rs[sl]);
-                // refill the slot with the tile kLook places later
-                int64_t q = mv.ntiles;
-                if (more) {
-                    q = int64_t(gridDim.x) + __shfl_sync(kFull, claimed, 0);
-                    if (lane == 0) claimed = atomicAdd(tile_counter, 1);
+                {
+                    const int64_t left = mv.ntiles - last_q, g = gridDim.x;
+                    size_hint = __popc(ms[sl]) > 2 ? 1 : (left > 8 * g ? 4 : (left > 2 * g ? 2 : 1));
                 }
-                fetch(q, ts[sl], ms[sl], rs[sl]);
-                more = more && q < mv.ntiles;
+                // refill: slots still unfetched come first (publish order), then this one
+#pragma unroll
+                for (int d = 1; d < kLook; ++d) {
+                    const int o = (sl + d) % kLook;
+                    if (ts[o] == kUnfetched) fetch(next_q(), ts[o], ms[o], rs[o]);
+                }
+                fetch(next_q(), ts[sl], ms[sl], rs[sl]);
             }
         }
         ptx::cp_async_wait<0>();
