@@ -270,10 +270,11 @@ lat_status lat_sconv_dgrad(const void *dy, int32_t cout, const void *w, int32_t 
 
 /* Per-offset weight gradient: dW[k] = sum over pairs (i, j) of offset k of
  * x[i]^T dy[j], fp32 (k3, cin, cout), from the forward map's pair lists.
- * Deterministic: the pairs are cut into chunks whose size depends only on
- * the pair count, each chunk is reduced into an fp32 partial, and the
- * partials are summed in a fixed order (no atomics), so the bits do not
- * depend on timing or on the number of SMs. */
+ * Deterministic: the pair list is cut into a fixed number of equal
+ * contiguous shares (fixed chunks on the CUDA-core path), each share is
+ * reduced into fp32 partials (one per offset it meets), and the partials are
+ * summed in a fixed order (no atomics), so the bits do not depend on timing
+ * or on the number of SMs. */
 lat_status lat_sconv_wgrad(const void *x, int32_t cin, const void *dy, int32_t cout,
                            const lat_kmap *map, float *dw, lat_dtype dtype, void *ws,
                            size_t ws_bytes, int32_t *d_status, lat_stream stream);

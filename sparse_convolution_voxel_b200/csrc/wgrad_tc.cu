@@ -2,18 +2,21 @@
 // x[i]^T dy[j]  (fp16 / bf16 in, fp32 accumulate in TMEM, fp32 out).
 //
 // Per offset this is a GEMM with M = Cin, N = Cout and the pairs as the
-// reduction dimension.  The pairs of each offset (grouped and ordered by the
-// kernel-map query) are cut into chunks whose size depends only on the total
-// pair count P (chunk_pairs: about kTargetUnits chunks in all, whatever the
-// GPU); persistent CTAs (two per SM) take chunks round-robin.  For every
-// 64-pair block of a chunk, four gather warps copy the 64 x rows and 64 dy
+// reduction dimension.  The pair list (grouped by offset by the kernel-map
+// query) is cut into kWorkers equal contiguous shares -- a constant, so the
+// cut does not depend on the GPU -- and persistent CTAs (two per SM) take the
+// shares round-robin.  A share is processed as segments, its intersections
+// with the offsets' pair ranges; a segment accumulates in TMEM and ends in one
+// fp32 partial, stored at slot share + offset (unique: shares and offsets are
+// both in pair order).  For every 64-pair block of a segment, four gather
+// warps copy the 64 x rows and 64 dy
 // rows with 16-byte cp.async into 128-byte swizzled MN-major tiles (rows of
 // the gathered operands are the reduction dimension, channels are
 // contiguous); the copies arrive on the stage barrier by themselves
 // (cp.async.mbarrier.arrive.noinc), and one thread issues 4 tcgen05.mma
 // (K = 16 pairs each) into a TMEM accumulator.  Four epilogue warps write the
-// chunk's fp32 partial; a second kernel sums the partials of each offset in a
-// fixed order (32 interleaved lanes over the chunks, then the lanes in order).
+// segment's fp32 partial; a second kernel sums the partials of each offset in a
+// fixed order (32 interleaved lanes over the shares, then the lanes in order).
 // No atomics, so dW is deterministic and does not depend on the SM count.
 #include "common.cuh"
 #include "conv_common.cuh"
@@ -23,8 +26,7 @@ namespace lat {
 namespace wtc {
 
 constexpr int kKP = 64;            // pairs per stage (GEMM K block)
-constexpr int kTargetUnits = 448;  // chunks of all offsets together, about
-constexpr int kMinChunk = 256;     // pairs per chunk at least
+constexpr int kWorkers = 296;      // equal shares of the pair list (two per B200 SM)
 constexpr int kProdWarps = 4, kEpiWarps = 4;
 constexpr int kMmaWarp = kProdWarps + kEpiWarps;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
@@ -52,55 +54,67 @@ __host__ __device__ constexpr uint32_t make_idesc() {
            (1u << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
 
-// Pairs per chunk for P pairs in all: at least kMinChunk, a multiple of 64, and
-// large enough that the chunks of all offsets number at most kTargetUnits + k3.
-__host__ __device__ __forceinline__ int64_t chunk_pairs(int64_t P) {
-    const int64_t c = (P + kTargetUnits - 1) / kTargetUnits;
-    const int64_t r = (c + 63) / 64 * 64;
-    return r > kMinChunk ? r : kMinChunk;
+// Clamped pair offsets of the k3 offsets (off[k3] = P) into shared memory; one warp.
+__device__ __forceinline__ void load_offsets(const int64_t *pair_off, int64_t capacity, int k3, int64_t *off) {
+    for (int e = threadIdx.x & 31; e <= k3; e += 32) off[e] = min(pair_off[e], capacity);
 }
 
-// First unit of every offset (and the total in ub[k3]): offset k's clamped pairs
-// are cut into ceil(P_k / chunk) units, numbered in offset order; ub[k3 + 1] =
-// chunk.  Called by one full warp (lane k handles offset k, k3 <= 32).
-__device__ __forceinline__ void unit_bases(const int64_t *pair_off, int64_t capacity, int k3, int32_t *ub) {
-    const int lane = threadIdx.x & 31;
-    const int64_t P = min(pair_off[k3], capacity);
-    const int64_t chunk = chunk_pairs(P);
-    const int64_t lo = lane < k3 ? min(pair_off[lane], capacity) : P;
-    const int64_t up = __shfl_down_sync(0xFFFFFFFFu, lo, 1);
-    const int64_t hi = lane == 31 ? P : up;  // offset k ends where offset k+1 starts (P after the last)
-    const int32_t units = lane < k3 ? int32_t((hi - lo + chunk - 1) / chunk) : 0;
-    int32_t incl = units;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const int32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-        if (lane >= d) incl += o;
+// Share v of the pair list: pairs [P v / kWorkers, P (v+1) / kWorkers).
+__device__ __forceinline__ int64_t share_lo(int64_t P, int v) { return P * v / kWorkers; }
+
+// The share holding pair `pair` (largest v with share_lo(P, v) <= pair); a binary
+// search, so only divisions by the constant kWorkers.
+__device__ __forceinline__ int share_of(int64_t P, int64_t pair) {
+    int lo = 0, hi = kWorkers - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (share_lo(P, mid) <= pair) lo = mid;
+        else hi = mid - 1;
     }
-    if (lane < k3) ub[lane] = incl - units;
-    const int32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
-    if (lane == 0) {
-        ub[k3] = total;
-        ub[k3 + 1] = int32_t(chunk);
-    }
+    return lo;
 }
 
-// Unit u covers pairs [lo, hi) of offset k.
-__device__ __forceinline__ void unit_range(const int32_t *unit_base, const int64_t *pair_off, int64_t capacity,
-                                           int k3, int32_t u, int &k, int64_t &lo, int64_t &hi) {
-    const int64_t chunk = unit_base[k3 + 1];
-    k = 0;
-    while (k + 1 < k3 && unit_base[k + 1] <= u) ++k;
-    const int64_t base = min(pair_off[k], capacity);
-    lo = base + int64_t(u - unit_base[k]) * chunk;
-    hi = min(lo + chunk, min(pair_off[k + 1], capacity));
-}
+// The segments of this CTA's shares, in order: share v = blockIdx.x, +gridDim.x,
+// ..., and within a share the offsets its range meets.  Every role walks the
+// same sequence.
+struct Segments {
+    const int64_t *off;
+    int k3;
+    int64_t P;
+    int v, k;
+    int64_t hv;
+    __device__ Segments(const int64_t *o, int k3_) : off(o), k3(k3_), P(o[k3_]), v(int(blockIdx.x) - int(gridDim.x)),
+                                                   k(k3_), hv(0) {}
+    // next segment: offset ko, pairs [lo, hi), partial slot
+    __device__ bool next(int &ko, int64_t &lo, int64_t &hi, int &slot) {
+        for (;;) {
+            while (k < k3 && off[k] < hv) {
+                const int64_t a = max(share_lo(P, v), off[k]), b = min(hv, off[k + 1]);
+                const int kk = k++;
+                if (a < b) {
+                    ko = kk;
+                    lo = a;
+                    hi = b;
+                    slot = v + kk;
+                    return true;
+                }
+            }
+            v += gridDim.x;
+            if (v >= kWorkers) return false;
+            const int64_t wl = share_lo(P, v);
+            hv = share_lo(P, v + 1);
+            k = 0;
+            while (k < k3 && off[k + 1] <= wl) ++k;
+        }
+    }
+};
 
 template <typename T, int M, int N>
 __global__ void __launch_bounds__(kThreads, 2)
 wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t *__restrict__ pair_off,
                 const int32_t *__restrict__ pair_in, const int32_t *__restrict__ pair_out, int64_t capacity, int k3,
-                int64_t n_in, int64_t n_out, float *__restrict__ partial, int32_t *d_status) {
+                int64_t n_in, int64_t n_out, float *__restrict__ partial, int32_t *__restrict__ ranges,
+                int32_t *d_status) {
     using C = Cfg<M, N>;
     constexpr int NS = C::kStages;
     constexpr uint32_t idesc = make_idesc<T, M, N>();
@@ -113,10 +127,19 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
     uint64_t *accempty = accfull + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accempty + 2);
     __shared__ int s_abort;
-    __shared__ int32_t unit_base[34];
+    __shared__ int64_t s_off[33];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (warp == 1) unit_bases(pair_off, capacity, k3, unit_base);
+    if (warp == 1) {
+        load_offsets(pair_off, capacity, k3, s_off);
+        __syncwarp();
+        if (blockIdx.x == 0 && lane < k3) {
+            // for the reduce: the shares meeting offset lane's pairs [a, b)
+            const int64_t P = s_off[k3], a = s_off[lane], b = s_off[lane + 1];
+            ranges[2 * lane] = a < b ? share_of(P, a) : 0;
+            ranges[2 * lane + 1] = a < b ? share_of(P, b - 1) : -1;
+        }
+    }
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
             ptx::mbar_init(&full[s], kProdWarps * 32);
@@ -138,7 +161,6 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int32_t units = unit_base[k3];
     int32_t bad = 0;
 
     if (warp < kProdWarps) {
@@ -146,10 +168,10 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
         uint32_t it = 0;
         bool ok = true;
         const int g = lane >> 3, c = lane & 7;
-        for (int32_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
-            int k;
-            int64_t lo, hi;
-            unit_range(unit_base, pair_off, capacity, k3, u, k, lo, hi);
+        Segments seg(s_off, k3);
+        int k, slot;
+        int64_t lo, hi;
+        while (ok && seg.next(k, lo, hi, slot)) {
             // lanes 0..15 fetch the indices of this warp's 16 pairs of a block, one block ahead
             auto fetch = [&](int64_t p0, int &si, int &sj) {
                 const int64_t mp = p0 + warp * 16 + (lane & 15);
@@ -207,11 +229,11 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
         const bool has_row = M == 128 || lane < 16;
         uint32_t ta = 0;
         bool ok = true;
-        for (int32_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
-            int k;
-            int64_t lo, hi;
-            unit_range(unit_base, pair_off, capacity, k3, u, k, lo, hi);
-            float *dst = partial + int64_t(u) * M * N + int64_t(row) * N;
+        Segments seg(s_off, k3);
+        int k, slot;
+        int64_t lo, hi;
+        while (ok && seg.next(k, lo, hi, slot)) {
+            float *dst = partial + int64_t(slot) * M * N + int64_t(row) * N;
             if (hi <= lo) {  // cannot happen for a listed unit; keep the partial defined anyway
                 if (has_row)
                     for (int c0 = 0; c0 < N; c0 += 4) *reinterpret_cast<float4 *>(dst + c0) = make_float4(0, 0, 0, 0);
@@ -251,11 +273,10 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
         // ------------------------------------------------------------ MMA issue
         uint32_t it = 0, ta = 0;
         bool ok = true;
-        for (int32_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
-            int k;
-            int64_t lo, hi;
-            unit_range(unit_base, pair_off, capacity, k3, u, k, lo, hi);
-            if (hi <= lo) continue;
+        Segments seg(s_off, k3);
+        int k, slot;
+        int64_t lo, hi;
+        while (ok && seg.next(k, lo, hi, slot)) {
             const uint32_t a = ta & 1;
             if (!ptx::mbar_wait(&accempty[a], ((ta >> 1) & 1) ^ 1, kWaitNs)) {
                 ok = false;
@@ -305,29 +326,28 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
     }
 }
 
-// dW[k] = sum of offset k's chunk partials.  Block (x, k): 32 unit lanes x 8
-// groups of 4 elements; lane l sums chunks l, l+32, ... in order, then lane 0
-// adds the 32 lane sums in order -- a fixed order whatever the timing.
+// dW[k] = sum of offset k's partials, one per share v0..v1 that meets offset k
+// (slot share + k; ranges from the main kernel).  Block (x, k): 32 lanes x 8 groups of 4 elements; lane l sums
+// shares v0+l, v0+l+32, ... in order, then lane 0 adds the 32 lane sums in
+// order -- a fixed order whatever the timing.  Offsets without pairs get 0.
 constexpr int kRedLanes = 32;
 __global__ void __launch_bounds__(256)
-wgrad_tc_reduce_kernel(const float *__restrict__ partial, const int64_t *__restrict__ pair_off, int64_t capacity,
-                       int k3, int nelem, float *__restrict__ dw) {
-    __shared__ int32_t unit_base[34];
+wgrad_tc_reduce_kernel(const float *__restrict__ partial, const int32_t *__restrict__ ranges, int nelem,
+                       float *__restrict__ dw) {
     __shared__ float4 s_part[kRedLanes][8];
-    if (threadIdx.x < 32) unit_bases(pair_off, capacity, k3, unit_base);
-    __syncthreads();
     const int k = blockIdx.y;
+    const int v0 = __ldg(ranges + 2 * k), v1 = __ldg(ranges + 2 * k + 1);
     const int g = threadIdx.x & 7, l = threadIdx.x >> 3;
     const int el = (blockIdx.x * 8 + g) * 4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (el < nelem) {
 #pragma unroll 4
-        for (int32_t u = unit_base[k] + l; u < unit_base[k + 1]; u += kRedLanes) {
-            const float4 v = __ldg(reinterpret_cast<const float4 *>(partial + int64_t(u) * nelem + el));
-            acc.x += v.x;
-            acc.y += v.y;
-            acc.z += v.z;
-            acc.w += v.w;
+        for (int v = v0 + l; v <= v1; v += kRedLanes) {
+            const float4 x = __ldg(reinterpret_cast<const float4 *>(partial + int64_t(v + k) * nelem + el));
+            acc.x += x.x;
+            acc.y += x.y;
+            acc.z += x.z;
+            acc.w += x.w;
         }
     }
     s_part[l][g] = acc;
@@ -335,11 +355,11 @@ wgrad_tc_reduce_kernel(const float *__restrict__ partial, const int64_t *__restr
     if (l == 0 && el < nelem) {
         float4 t = s_part[0][g];
         for (int q = 1; q < kRedLanes; ++q) {
-            const float4 v = s_part[q][g];
-            t.x += v.x;
-            t.y += v.y;
-            t.z += v.z;
-            t.w += v.w;
+            const float4 x = s_part[q][g];
+            t.x += x.x;
+            t.y += x.y;
+            t.z += x.z;
+            t.w += x.w;
         }
         *reinterpret_cast<float4 *>(dw + int64_t(k) * nelem + el) = t;
     }
@@ -349,19 +369,20 @@ template <typename T, int M, int N>
 static lat_status launch(const void *x, const void *dy, const lat_kmap *map, float *dw, void *ws, int32_t *d_status,
                          cudaStream_t s) {
     using C = Cfg<M, N>;
-    const int64_t units_max = int64_t(kTargetUnits) + map->k3;
+    const int64_t units_max = int64_t(kWorkers) + map->k3;
     Carver cv(ws);
     float *partial = cv.take<float>(size_t(units_max) * M * N);
+    int32_t *ranges = cv.take<int32_t>(64);
     auto kern = wgrad_tc_kernel<T, M, N>;
-    const int64_t grid = std::min<int64_t>(units_max, GridCache<KernelTag<T, M, N>>::get(kern, C::kSmem, int(C::kTmemCols), 2));
+    const int64_t grid = std::min<int64_t>(kWorkers, GridCache<KernelTag<T, M, N>>::get(kern, C::kSmem, int(C::kTmemCols), 2));
     if (grid <= 0) return LAT_ERR_CUDA;
     kern<<<unsigned(grid), kThreads, C::kSmem, s>>>(static_cast<const T *>(x), static_cast<const T *>(dy),
                                                     map->pair_off, map->pair_in, map->pair_out, map->pair_capacity,
-                                                    map->k3, map->n_in, map->n_out, partial, d_status);
+                                                    map->k3, map->n_in, map->n_out, partial, ranges, d_status);
     LAT_CUDA_TRY(cudaGetLastError());
     const int nelem = M * N;
     dim3 rg((nelem + 31) / 32, map->k3);
-    wgrad_tc_reduce_kernel<<<rg, 256, 0, s>>>(partial, map->pair_off, map->pair_capacity, map->k3, nelem, dw);
+    wgrad_tc_reduce_kernel<<<rg, 256, 0, s>>>(partial, ranges, nelem, dw);
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }
@@ -371,9 +392,10 @@ static lat_status launch(const void *x, const void *dy, const lat_kmap *map, flo
 bool wgrad_tc_supported(int cin, int cout) { return (cin == 64 || cin == 128) && (cout == 64 || cout == 128); }
 
 size_t wgrad_tc_ws_bytes(int cin, int cout, const lat_kmap *map) {
-    const int64_t units_max = int64_t(wtc::kTargetUnits) + map->k3;
+    const int64_t units_max = int64_t(wtc::kWorkers) + map->k3;
     Carver cv(nullptr);
     cv.take<float>(size_t(units_max) * cin * cout);
+    cv.take<int32_t>(64);
     return align_up(cv.used, 256);
 }
 
