@@ -195,7 +195,7 @@ class Pipeline:
 # (profiles/launches_lidar_subm_step.md: the submanifold kmap query, its 8
 # kernels summed, caches not flushed between kernels); None where no capture
 # matches the current kernels.
-PHASE_TRAFFIC = {"kmap": 21.0e6}
+PHASE_TRAFFIC = {"kmap": 20.2e6}
 
 
 def flush_l2(buf: torch.Tensor):
