@@ -23,8 +23,9 @@
  *     allocates or frees memory and keeps no state between calls except
  *     per-device kernel attributes set on first use.
  *   - Work is enqueued on `stream` (NULL = legacy default stream) and is
- *     asynchronous, except lat_downsample_coords and lat_status_fetch,
- *     which synchronise `stream` because they return a device-computed value.
+ *     asynchronous, except lat_downsample_coords, lat_upsample_coords and
+ *     lat_status_fetch, which synchronise `stream` because they return a
+ *     device-computed value.
  *   - Argument errors are detected on the host and returned synchronously;
  *     nothing is enqueued then.  Errors found by a kernel (range, duplicate,
  *     table full, capacity, malformed map) are OR-ed into the caller's int32
@@ -215,6 +216,22 @@ lat_status lat_downsample_coords_async(const int32_t *coords, int64_t n_in, cons
                                        int32_t *out_coords, int64_t out_capacity, int64_t *n_out_host,
                                        int32_t *parent, void *ws, size_t ws_bytes, int32_t *d_status,
                                        lat_stream stream);
+
+/* Output support of a GenerativeConvTranspose3d (migration page, "Convolution
+ * mapping": a generative transposed convolution creates its output support):
+ * every fine coordinate s*q + (ix,iy,iz) - pad for an input (coarse) row q and
+ * offset (ix,iy,iz) in [0,K)^3, batch unchanged, made unique and written to
+ * out_coords in canonical (b, x, y, z) order.  geom->mode must be
+ * LAT_TRANSPOSED (the geometry the transposed map of the same conv uses).
+ * Generated coordinates outside the packable key range are dropped and flag
+ * LAT_ERR_COORD_RANGE.  out_capacity >= n_in * K^3 always suffices.  Same
+ * algorithm, synchronisation and errors as lat_downsample_coords (no parents).
+ * The convolution then runs on lat_kmap_query(table of the input rows,
+ * out_coords, LAT_TRANSPOSED geom). */
+size_t lat_upsample_ws_bytes(int64_t n_in, const lat_geom *geom);
+lat_status lat_upsample_coords(const int32_t *coords, int64_t n_in, const lat_geom *geom,
+                               int32_t *out_coords, int64_t out_capacity, int64_t *n_out, void *ws,
+                               size_t ws_bytes, int32_t *d_status, lat_stream stream);
 
 /* Both kernel maps of a strided Conv3d with ksize == stride and pad == 0,
  * built from the parent rows that lat_downsample_coords reports instead of by

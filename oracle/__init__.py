@@ -59,6 +59,8 @@ def _load():
             lib.orc_kmap.argtypes = [P, i64, P, i64, P, P, P, i32, P, i32]
             lib.orc_downsample.restype = i64
             lib.orc_downsample.argtypes = [P, i64, P, P, P, P, i64]
+            lib.orc_upsample.restype = i64
+            lib.orc_upsample.argtypes = [P, i64, P, P, P, P, i64]
             lib.orc_conv_fwd.restype = None
             lib.orc_conv_fwd.argtypes = [P, i64, i32, P, i32, P, i64, i32, P, i32]
             lib.orc_conv_dgrad.restype = None
@@ -134,6 +136,19 @@ def downsample(coords, ksize, stride, pad=0) -> np.ndarray:
     m = _load().orc_downsample(_ptr(c), len(c), _ptr(ks), _ptr(st), _ptr(pd), _ptr(out), cap)
     if m < 0:
         raise OracleError("downsample failed")
+    return out[:m].copy()
+
+
+def upsample(coords, ksize, stride, pad=0) -> np.ndarray:
+    """Support generated by a transposed convolution (GenerativeConvTranspose3d):
+    every s*q + off - pad, sorted by packed key ("Convolution mapping")."""
+    c = _i32(coords).reshape(-1, 4)
+    ks, st, pd = _triple(ksize), _triple(stride), _triple(pad)
+    cap = max(1, len(c) * int(np.prod(ks)))
+    out = np.empty((cap, 4), np.int32)
+    m = _load().orc_upsample(_ptr(c), len(c), _ptr(ks), _ptr(st), _ptr(pd), _ptr(out), cap)
+    if m < 0:
+        raise OracleError("upsample failed")
     return out[:m].copy()
 
 

@@ -175,6 +175,34 @@ int64_t orc_downsample(const int32_t* coords, int64_t n, const int32_t* ksize,
     return m;
 }
 
+// Support generated by a transposed convolution: every s*q + off - pad for an
+// input (coarse) row q and off in [0,K)^3, batch unchanged, in range only,
+// sorted by packed key (migration page, "Convolution mapping": generative
+// transposed convolutions create their output support).
+int64_t orc_upsample(const int32_t* coords, int64_t n, const int32_t* ksize,
+                     const int32_t* stride, const int32_t* pad, int32_t* out, int64_t capacity) {
+    for (int a = 0; a < 3; ++a)
+        if (ksize[a] < 1 || stride[a] < 1) return -1;
+    std::set<uint64_t> support;
+    for (int64_t i = 0; i < n; ++i) {
+        const int32_t* c = coords + 4 * i;
+        if (!in_range(c[0], c[1], c[2], c[3])) return -1;
+        for (int ix = 0; ix < ksize[0]; ++ix)
+            for (int iy = 0; iy < ksize[1]; ++iy)
+                for (int iz = 0; iz < ksize[2]; ++iz) {
+                    const int off[3] = {ix, iy, iz};
+                    int64_t p[3];
+                    for (int a = 0; a < 3; ++a) p[a] = int64_t(stride[a]) * c[a + 1] + off[a] - pad[a];
+                    if (in_range(c[0], p[0], p[1], p[2])) support.insert(pack(c[0], p[0], p[1], p[2]));
+                }
+    }
+    const int64_t m = int64_t(support.size());
+    if (m > capacity) return -m - 2;
+    int64_t r = 0;
+    for (uint64_t key : support) unpack(key, out + 4 * r++);
+    return m;
+}
+
 // y[j] = sum over k ascending with i = nbr[j][k] >= 0 of x[i] . W[k]
 // x: [n_in][cin], w: [k3][cin][cout], y: [n_out][cout]; all fp64.
 void orc_conv_fwd(const double* x, int64_t n_in, int cin, const double* w, int cout,

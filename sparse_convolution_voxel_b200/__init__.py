@@ -18,13 +18,15 @@ import torch
 from ._lib import (  # noqa: F401  (re-exported C entry points and constants)
     EXPORTS, LAT_BF16, LAT_F16, LAT_F32, LAT_OK, LAT_OP_DGRAD, LAT_OP_FWD, LAT_OP_WGRAD, LAT_STRIDED, LAT_SUBM,
     LAT_TILE_ROWS, LAT_TRANSPOSED, LIB_PATH, LatticeError, lat_downsample_coords, lat_downsample_coords_async, lat_downsample_ws_bytes, lat_geom,
+    lat_upsample_coords, lat_upsample_ws_bytes,
     lat_hash_build, lat_hash_bytes, lat_kmap, lat_kmap_from_parent, lat_kmap_from_parent_ws_bytes, lat_kmap_query,
     lat_kmap_ws_bytes, lat_sconv_dgrad, lat_sconv_fwd,
     lat_sconv_wgrad, lat_sconv_wgrad_static, lat_sconv_ws_bytes, lat_status_fetch, lat_status_string, lat_version, load, make_geom,
 )
 
 __all__ = [
-    "KernelMap", "Workspace", "hash_table", "kernel_map", "downsample", "downsample_async", "PendingDownsample", "maps_from_parent", "conv_fwd", "conv_dgrad", "conv_wgrad",
+    "KernelMap", "Workspace", "hash_table", "kernel_map", "downsample", "downsample_async", "PendingDownsample",
+    "upsample", "maps_from_parent", "conv_fwd", "conv_dgrad", "conv_wgrad",
     "subm_geom", "strided_geom", "target_geom", "transposed_geom", "check_status", "new_status",
 ] + EXPORTS
 
@@ -121,6 +123,19 @@ def kernel_map(table: torch.Tensor, n_in: int, out_coords: torch.Tensor, geom: l
     ws = ws or Workspace(out_coords.device)
     lat_kmap_query(table, out_coords, geom, km.c, ws.get(lat_kmap_ws_bytes(km.n_out, k3)), d_status, stream)
     return km
+
+
+def upsample(coords: torch.Tensor, geom: lat_geom, ws: Workspace | None = None, d_status=None,
+             capacity: int | None = None, stream=None) -> torch.Tensor:
+    """Support a GenerativeConvTranspose3d generates from `coords` (geom: LAT_TRANSPOSED),
+    in canonical order (synchronises)."""
+    n = coords.shape[0]
+    k3 = geom.ksize[0] * geom.ksize[1] * geom.ksize[2]
+    cap = n * k3 if capacity is None else int(capacity)
+    out = torch.empty((max(1, cap), 4), dtype=torch.int32, device=coords.device)
+    ws = ws or Workspace(coords.device)
+    m = lat_upsample_coords(coords, geom, out, ws.get(lat_upsample_ws_bytes(n, geom)), d_status, stream)
+    return out[:m]
 
 
 class PendingDownsample:

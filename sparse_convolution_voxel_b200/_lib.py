@@ -31,7 +31,8 @@ STATUS_BITS = {
 # every symbol include/lattice.h declares
 EXPORTS = [
     "lat_hash_bytes", "lat_hash_build", "lat_kmap_ws_bytes", "lat_kmap_query",
-    "lat_downsample_ws_bytes", "lat_downsample_coords", "lat_downsample_coords_async", "lat_kmap_from_parent_ws_bytes",
+    "lat_downsample_ws_bytes", "lat_downsample_coords", "lat_downsample_coords_async", "lat_upsample_ws_bytes",
+    "lat_upsample_coords", "lat_kmap_from_parent_ws_bytes",
     "lat_kmap_from_parent",
     "lat_sconv_ws_bytes", "lat_sconv_fwd",
     "lat_sconv_dgrad", "lat_sconv_wgrad", "lat_sconv_wgrad_static", "lat_status_fetch", "lat_status_string", "lat_version",
@@ -79,6 +80,8 @@ def load() -> ctypes.CDLL:
         "lat_downsample_ws_bytes": (SZ, [I64, G]),
         "lat_downsample_coords": (I32, [P, I64, G, P, I64, ctypes.POINTER(I64), P, P, SZ, P, P]),
         "lat_downsample_coords_async": (I32, [P, I64, G, P, I64, P, P, P, SZ, P, P]),
+        "lat_upsample_ws_bytes": (SZ, [I64, G]),
+        "lat_upsample_coords": (I32, [P, I64, G, P, I64, ctypes.POINTER(I64), P, SZ, P, P]),
         "lat_kmap_from_parent_ws_bytes": (SZ, [I64, I64, I32]),
         "lat_kmap_from_parent": (I32, [P, P, G, K, K, P, SZ, P, P]),
         "lat_sconv_ws_bytes": (SZ, [I32, I32, I32, K, I32]),
@@ -181,6 +184,21 @@ def lat_downsample_coords_async(coords: torch.Tensor, geom: lat_geom, out_coords
                                             _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                                             _ptr(d_status), _stream(stream))
     _check(rc, "lat_downsample_coords_async")
+
+
+def lat_upsample_ws_bytes(n_in: int, geom: lat_geom) -> int:
+    return int(load().lat_upsample_ws_bytes(int(n_in), ctypes.byref(geom)))
+
+
+def lat_upsample_coords(coords: torch.Tensor, geom: lat_geom, out_coords: torch.Tensor, ws: torch.Tensor | None,
+                        d_status: torch.Tensor | None = None, stream=None) -> int:
+    n = ctypes.c_int64(0)
+    rc = load().lat_upsample_coords(_ptr(coords), coords.shape[0], ctypes.byref(geom), _ptr(out_coords),
+                                    out_coords.shape[0], ctypes.byref(n), _ptr(ws),
+                                    0 if ws is None else ws.numel() * ws.element_size(), _ptr(d_status),
+                                    _stream(stream))
+    _check(rc, "lat_upsample_coords")
+    return int(n.value)
 
 
 def lat_kmap_from_parent_ws_bytes(n_fine: int, n_coarse: int, k3: int) -> int:

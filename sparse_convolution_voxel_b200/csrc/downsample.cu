@@ -31,8 +31,9 @@ namespace lat {
 
 struct DownGeom {
     int ks[3], st[3], pd[3];
-    int per_axis[3];  // ceil(K/s): candidate offsets per axis
+    int per_axis[3];  // candidate offsets per axis: ceil(K/s), or K when generating
     int cands;        // product of per_axis
+    int up;           // 1: support of a generative transposed conv (every s*q + off - pad)
 };
 
 constexpr int kMaxBitmapBits = 30;
@@ -52,6 +53,33 @@ down_candidates_kernel(const int4 *__restrict__ coords, int64_t n, DownGeom g, u
         if (!pack_key(c.x, c.y, c.z, c.w, self)) {
             for (int e = 0; e < g.cands; ++e) dst[e] = kEmptyKey;
             flag(d_status, LAT_ERR_COORD_RANGE);
+        } else if (g.up) {
+            // generated fine rows s*q + off - pad of coarse row q, off in [0,K)^3
+            int e = 0;
+            bool lost = false;
+            for (int u = 0; u < g.ks[0]; ++u)
+                for (int v = 0; v < g.ks[1]; ++v)
+                    for (int w = 0; w < g.ks[2]; ++w, ++e) {
+                        const int64_t f[3] = {int64_t(g.st[0]) * c.y + u - g.pd[0],
+                                              int64_t(g.st[1]) * c.z + v - g.pd[1],
+                                              int64_t(g.st[2]) * c.w + w - g.pd[2]};
+                        uint64_t key = kEmptyKey;
+                        const bool fits = f[0] >= -32768 && f[0] <= 32767 && f[1] >= -32768 && f[1] <= 32767 &&
+                                          f[2] >= -32768 && f[2] <= 32767;
+                        if (fits && pack_key(c.x, int(f[0]), int(f[1]), int(f[2]), key)) {
+                            const int fv[4] = {c.x, int(f[0]), int(f[1]), int(f[2])};
+#pragma unroll
+                            for (int a = 0; a < 4; ++a) {
+                                mn[a] = min(mn[a], fv[a]);
+                                mx[a] = max(mx[a], fv[a]);
+                            }
+                        } else {
+                            key = kEmptyKey;
+                            lost = true;
+                        }
+                        dst[e] = key;
+                    }
+            if (lost) flag(d_status, LAT_ERR_COORD_RANGE);
         } else {
             const int p[3] = {c.y, c.z, c.w};
             int first[3];  // smallest off in [0,K) with (p - off + pad) divisible by s
@@ -366,8 +394,11 @@ sorted_parent_kernel(const uint64_t *__restrict__ keys, int64_t n, const uint64_
     parent[i] = (key != kEmptyKey && lo < *n_out_dev && uniq[lo] == key) ? int32_t(lo) : -1;
 }
 
-static bool down_geom(const lat_geom *geom, DownGeom &g) {
-    if (!geom || geom->mode != LAT_STRIDED) return false;
+// up = false: the support of a strided / generative Conv3d (geom->mode LAT_STRIDED);
+// up = true: the support a GenerativeConvTranspose3d generates (LAT_TRANSPOSED).
+static bool down_geom(const lat_geom *geom, DownGeom &g, bool up = false) {
+    if (!geom || geom->mode != (up ? LAT_TRANSPOSED : LAT_STRIDED)) return false;
+    g.up = up ? 1 : 0;
     g.cands = 1;
     for (int a = 0; a < 3; ++a) {
         if (geom->ksize[a] < 1 || geom->stride[a] < 1 || geom->pad[a] < 0 || geom->pad[a] >= geom->ksize[a] + 32768)
@@ -375,7 +406,7 @@ static bool down_geom(const lat_geom *geom, DownGeom &g) {
         g.ks[a] = geom->ksize[a];
         g.st[a] = geom->stride[a];
         g.pd[a] = geom->pad[a];
-        g.per_axis[a] = (geom->ksize[a] + geom->stride[a] - 1) / geom->stride[a];
+        g.per_axis[a] = up ? geom->ksize[a] : (geom->ksize[a] + geom->stride[a] - 1) / geom->stride[a];
         g.cands *= g.per_axis[a];
     }
     return g.ks[0] * g.ks[1] * g.ks[2] <= 32;
@@ -454,9 +485,9 @@ namespace lat {
 // means there is nothing to do (no input row).
 static lat_status down_prepare(const int32_t *coords, int64_t n_in, const lat_geom *geom, int32_t *out_coords,
                                int64_t out_capacity, int32_t *parent, void *ws, size_t ws_bytes, DownGeom &g,
-                               DownWs &w, int64_t &items) {
+                               DownWs &w, int64_t &items, bool up = false) {
     items = 0;
-    if (n_in < 0 || out_capacity < 0 || !down_geom(geom, g)) return LAT_ERR_ARG;
+    if (n_in < 0 || out_capacity < 0 || !down_geom(geom, g, up)) return LAT_ERR_ARG;
     if (n_in > 0 && (!coords || (out_capacity > 0 && !out_coords))) return LAT_ERR_ARG;
     if (reinterpret_cast<uintptr_t>(coords) % 16 || reinterpret_cast<uintptr_t>(out_coords) % 16) return LAT_ERR_ARG;
     if (parent) {  // one coarse row per input only when the kernel tiles the stride exactly
@@ -509,16 +540,16 @@ static lat_status enqueue_bitmap_path(const int32_t *coords, int64_t n_in, const
 
 }  // namespace lat
 
-extern "C" lat_status lat_downsample_coords(const int32_t *coords, int64_t n_in, const lat_geom *geom,
-                                            int32_t *out_coords, int64_t out_capacity, int64_t *n_out,
-                                            int32_t *parent, void *ws, size_t ws_bytes, int32_t *d_status,
-                                            lat_stream stream) {
-    using namespace lat;
+namespace lat {
+static lat_status support_blocking(const int32_t *coords, int64_t n_in, const lat_geom *geom, int32_t *out_coords,
+                                   int64_t out_capacity, int64_t *n_out, int32_t *parent, void *ws, size_t ws_bytes,
+                                   int32_t *d_status, lat_stream stream, bool up) {
     if (!n_out) return LAT_ERR_ARG;
     DownGeom g;
     DownWs w;
     int64_t items = 0;
-    const lat_status st = down_prepare(coords, n_in, geom, out_coords, out_capacity, parent, ws, ws_bytes, g, w, items);
+    const lat_status st =
+        down_prepare(coords, n_in, geom, out_coords, out_capacity, parent, ws, ws_bytes, g, w, items, up);
     if (st != LAT_OK) return st;
     *n_out = 0;
     if (items == 0) return LAT_OK;
@@ -547,6 +578,30 @@ extern "C" lat_status lat_downsample_coords(const int32_t *coords, int64_t n_in,
     }
     *n_out = m;
     return m > out_capacity ? LAT_ERR_CAPACITY : LAT_OK;
+}
+}  // namespace lat
+
+extern "C" lat_status lat_downsample_coords(const int32_t *coords, int64_t n_in, const lat_geom *geom,
+                                            int32_t *out_coords, int64_t out_capacity, int64_t *n_out,
+                                            int32_t *parent, void *ws, size_t ws_bytes, int32_t *d_status,
+                                            lat_stream stream) {
+    return lat::support_blocking(coords, n_in, geom, out_coords, out_capacity, n_out, parent, ws, ws_bytes, d_status,
+                                 stream, false);
+}
+
+extern "C" size_t lat_upsample_ws_bytes(int64_t n_in, const lat_geom *geom) {
+    lat::DownGeom g;
+    if (n_in < 0 || !lat::down_geom(geom, g, true)) return 0;
+    const int64_t items = n_in * g.cands;
+    if (items >= (int64_t(1) << 31)) return 0;
+    return lat::carve_down_ws(nullptr, std::max<int64_t>(items, 1)).total;
+}
+
+extern "C" lat_status lat_upsample_coords(const int32_t *coords, int64_t n_in, const lat_geom *geom,
+                                          int32_t *out_coords, int64_t out_capacity, int64_t *n_out, void *ws,
+                                          size_t ws_bytes, int32_t *d_status, lat_stream stream) {
+    return lat::support_blocking(coords, n_in, geom, out_coords, out_capacity, n_out, nullptr, ws, ws_bytes,
+                                 d_status, stream, true);
 }
 
 extern "C" lat_status lat_downsample_coords_async(const int32_t *coords, int64_t n_in, const lat_geom *geom,

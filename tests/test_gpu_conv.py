@@ -200,3 +200,78 @@ def test_target_conv(dtype):
     w, w64 = weights(27, 64, 64, dtype, seed=47)
     y = scv.conv_fwd(x, w, km)
     assert_close(y.double().cpu().numpy(), oracle.conv_fwd(x64, w64, ref_nbr), dtype, "target conv")
+
+
+# --------------------------------------------------------------------------- generative stride-1 Conv3d
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float16])
+@pytest.mark.parametrize("ks", [3, (3, 3, 1)])
+def test_generative_stride1_conv(dtype, ks):
+    """A stride-1 Conv3d that is not submanifold grows the support by its
+    footprint (migration page, "Convolution mapping": generative convs create a
+    new support): support = every q whose window holds an input, then the
+    strided relation, forward and data gradient against the oracle."""
+    rng = np.random.default_rng(23)
+    coords = rand_coords(rng, 700, -8, 8, 2)
+    if ks != 3:
+        coords[:, 3] = 0
+        coords = np.unique(coords, axis=0)
+        coords = coords[rng.permutation(len(coords))]
+    pad = (1, 1, 1) if ks == 3 else (1, 1, 0)
+    g = scv.strided_geom(ks, 1, pad)
+    c = _dev(coords)
+    st = scv.new_status()
+    grown = scv.downsample(c, g, d_status=st).contiguous()
+    ref_grown = oracle.downsample(coords, ks, 1, pad)
+    assert np.array_equal(grown.cpu().numpy(), ref_grown)
+    assert len(ref_grown) > len(coords)              # the support grew
+    km = scv.kernel_map(scv.hash_table(c, 2.0, st), len(coords), grown, g, d_status=st)
+    ref_nbr = oracle.kmap(coords, ref_grown, ks, 1, pad, oracle.STRIDED)
+    check_kmap(km, ref_nbr)
+    k3 = ref_nbr.shape[1]
+    cin, cout = (16, 32) if dtype == torch.float32 else (64, 64)
+    x, x64 = feats(len(coords), cin, dtype, seed=9)
+    w, w64 = weights(k3, cin, cout, dtype, seed=9)
+    y = scv.conv_fwd(x, w, km, d_status=st)
+    assert_close(y.double().cpu().numpy(), oracle.conv_fwd(x64, w64, ref_nbr), dtype, "generative fwd")
+    # data gradient through the opposite relation (grown rows -> input rows)
+    gy, gy64 = feats(len(ref_grown), cout, dtype, seed=9, stream=1)
+    back = scv.kernel_map(scv.hash_table(grown, 2.0, st), len(ref_grown), c, scv.transposed_geom(ks, 1, pad),
+                          d_status=st)
+    dx = scv.conv_dgrad(gy, w, back, flip_offsets=False, d_status=st)
+    scv.check_status(st)
+    assert_close(dx.double().cpu().numpy(), oracle.conv_dgrad(gy64, w64, ref_nbr, len(coords)), dtype,
+                 "generative dgrad")
+
+
+# --------------------------------------------------------------------------- GenerativeConvTranspose3d
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("ks,st_,pd", [(2, 2, 0), (3, 2, 1)])
+def test_generative_transposed_conv(dtype, ks, st_, pd):
+    """GenerativeConvTranspose3d: generated fine support, the transposed relation
+    from the coarse table to it, forward and data gradient against the oracle."""
+    rng = np.random.default_rng(41 + ks)
+    coarse = rand_coords(rng, 400, -6, 6, 2)
+    c = _dev(coarse)
+    g = scv.transposed_geom(ks, st_, pd)
+    st = scv.new_status()
+    fine = scv.upsample(c, g, d_status=st).contiguous()
+    ref_fine = oracle.upsample(coarse, ks, st_, pd)
+    assert np.array_equal(fine.cpu().numpy(), ref_fine)
+    km = scv.kernel_map(scv.hash_table(c, 2.0, st), len(coarse), fine, g, d_status=st)
+    ref_nbr = oracle.kmap(coarse, ref_fine, ks, st_, pd, oracle.TRANSPOSED)
+    check_kmap(km, ref_nbr)
+    assert np.all((ref_nbr >= 0).any(1))             # every generated row has a source
+    k3 = ref_nbr.shape[1]
+    cin, cout = (128, 64) if dtype == torch.bfloat16 else (32, 16)
+    x, x64 = feats(len(coarse), cin, dtype, seed=13)
+    w, w64 = weights(k3, cin, cout, dtype, seed=13)
+    y = scv.conv_fwd(x, w, km, d_status=st)
+    assert_close(y.double().cpu().numpy(), oracle.conv_fwd(x64, w64, ref_nbr), dtype, "generative transposed fwd")
+    # data gradient back to the coarse rows through the strided relation
+    gy, gy64 = feats(len(ref_fine), cout, dtype, seed=13, stream=1)
+    back = scv.kernel_map(scv.hash_table(fine, 2.0, st), len(ref_fine), c, scv.strided_geom(ks, st_, pd),
+                          d_status=st)
+    dx = scv.conv_dgrad(gy, w, back, flip_offsets=False, d_status=st)
+    scv.check_status(st)
+    assert_close(dx.double().cpu().numpy(), oracle.conv_dgrad(gy64, w64, ref_nbr, len(coarse)), dtype,
+                 "generative transposed dgrad")

@@ -269,3 +269,32 @@ def test_downsample_parent_needs_kernel_equal_stride():
     coords = rand_coords(np.random.default_rng(0), 100, 0, 8)
     with pytest.raises(scv.LatticeError):
         scv.downsample(_dev(coords), scv.strided_geom(3, 2, 1), with_parent=True)
+
+
+# --------------------------------------------------------------------------- generative transposed support
+@pytest.mark.parametrize("ks,st_,pd,lo,hi", [((2, 2, 2), (2, 2, 2), (0, 0, 0), -10, 10),
+                                             ((3, 3, 3), (2, 2, 2), (1, 1, 1), -10, 10),
+                                             ((3, 2, 1), (2, 1, 3), (1, 0, 0), -10, 10),
+                                             ((2, 2, 2), (2, 2, 2), (0, 0, 0), -10000, 10000)])  # radix-sort path
+def test_upsample_matches_oracle(ks, st_, pd, lo, hi):
+    rng = np.random.default_rng(31 + abs(lo))
+    if hi - lo > 100:
+        coords = np.unique(rng.integers(lo, hi, (800, 4)).astype(np.int32), axis=0)
+        coords[:, 0] = rng.integers(0, 2, len(coords))
+        coords = np.unique(coords, axis=0)
+        coords = coords[rng.permutation(len(coords))]
+    else:
+        coords = rand_coords(rng, 500, lo, hi, 2)
+    st = scv.new_status()
+    g = scv.transposed_geom(ks, st_, pd)
+    fine = scv.upsample(_dev(coords), g, d_status=st)
+    scv.check_status(st)
+    assert np.array_equal(fine.cpu().numpy(), oracle.upsample(coords, ks, st_, pd))
+
+
+def test_upsample_errors():
+    coords = rand_coords(np.random.default_rng(4), 200, 0, 10)
+    with pytest.raises(scv.LatticeError):            # needs the transposed geometry
+        scv.upsample(_dev(coords), scv.strided_geom(2, 2, 0))
+    with pytest.raises(scv.LatticeError):            # undersized output buffer
+        scv.upsample(_dev(coords), scv.transposed_geom(2, 2, 0), capacity=100)

@@ -349,3 +349,43 @@ def test_target_conv_matches_dense_conv_at_target_sites():
     y = oracle.conv_fwd(x, w, oracle.kmap(c, targets, 3, 1, 1, STRIDED))
     dense = torch.nn.functional.conv3d(_densify(c, x, (8, 8, 8), (0, 0, 0)), _dense_weight(w, (3, 3, 3)), padding=1)
     np.testing.assert_allclose(y, _read(dense, targets, (0, 0, 0)).numpy(), rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- generative transposed conv
+_UP_GEOMS = [((2, 2, 2), (2, 2, 2), (0, 0, 0)), ((3, 3, 3), (2, 2, 2), (1, 1, 1)),
+             ((3, 2, 1), (2, 1, 3), (1, 0, 0))]
+
+
+@pytest.mark.parametrize("ks,st,pd", _UP_GEOMS)
+def test_upsample_support_equals_nonzero_dense_transposed_conv(ks, st, pd):
+    """Generated support = where a dense conv_transpose3d of the occupancy grid
+    with an all-ones kernel is nonzero (input index i <-> coordinate i + origin,
+    output index o <-> coordinate o + s*origin - pad)."""
+    rng = np.random.default_rng(sum(ks) + 7 * sum(st))
+    c = _rand_coords(rng, 60, -3, 5, batch=2)
+    origin = np.array([-3, -3, -3])
+    occ = _densify(c, np.ones((len(c), 1)), (8, 8, 8), tuple(origin))
+    out = torch.nn.functional.conv_transpose3d(occ, torch.ones((1, 1) + ks, dtype=torch.float64), stride=st)
+    nz = torch.nonzero(out[:, 0] > 0).numpy().astype(np.int64)
+    nz[:, 1:] += np.array(st) * origin - np.array(pd)
+    nz = nz[np.lexsort(nz.T[::-1])].astype(np.int32)
+    assert np.array_equal(oracle.upsample(c, ks, st, pd), nz)
+
+
+@pytest.mark.parametrize("ks,st,pd", _UP_GEOMS)
+def test_generative_transposed_conv_matches_dense_conv_transpose3d(ks, st, pd):
+    """GenerativeConvTranspose3d forward on the generated support (transposed
+    relation from the input table) = dense conv_transpose3d read at every
+    generated site."""
+    rng = np.random.default_rng(5 + sum(pd))
+    c = _rand_coords(rng, 40, -3, 5, batch=2)
+    gen = oracle.upsample(c, ks, st, pd)
+    k3, cin, cout = int(np.prod(ks)), 3, 4
+    x = rng.standard_normal((len(c), cin))
+    w = rng.standard_normal((k3, cin, cout))
+    y = oracle.conv_fwd(x, w, oracle.kmap(c, gen, ks, st, pd, TRANSPOSED))
+    wd = torch.as_tensor(w).reshape(ks[0], ks[1], ks[2], cin, cout).permute(3, 4, 0, 1, 2)
+    origin = np.array([-3, -3, -3])
+    dense = torch.nn.functional.conv_transpose3d(_densify(c, x, (8, 8, 8), tuple(origin)), wd, stride=st)
+    read_origin = tuple(np.array(st) * origin - np.array(pd))
+    np.testing.assert_allclose(y, _read(dense, gen, read_origin).numpy(), rtol=1e-12, atol=1e-12)
