@@ -392,9 +392,14 @@ def run_only(args):
     dw = torch.empty((k3, cin, cout), dtype=torch.float32, device=dev)
     coarse = torch.empty((n * 8, 4), dtype=torch.int32, device=dev)
     parent = torch.empty(n, dtype=torch.int32, device=dev)
+    g_up = scv.transposed_geom(2, 2, 0)
     wsb = ws.get(max(scv.lat_kmap_ws_bytes(n, k3), scv.lat_sconv_ws_bytes(2, cin, cout, km.c, dt),
                      scv.lat_sconv_ws_bytes(0, cin, cout, km.c, dt), scv.lat_sconv_ws_bytes(1, cin, cout, km.c, dt),
-                     scv.lat_downsample_ws_bytes(n, scv.strided_geom(2, 2, 0))))
+                     scv.lat_downsample_ws_bytes(n, scv.strided_geom(2, 2, 0)), scv.lat_upsample_ws_bytes(n, g_up)))
+    # generative decoder step: the k2s2 transposed support of the coarse support
+    coarse_c = scv.downsample(coords, scv.strided_geom(2, 2, 0), ws).contiguous() if args.only == "upsample" else coords
+    fine_buf = torch.empty((coarse_c.shape[0] * 8, 4), dtype=torch.int32, device=dev)
+    n_fine = scv.lat_upsample_coords(coarse_c, g_up, fine_buf, wsb, st) if args.only == "upsample" else 0
     torch.cuda.synchronize()
     P = int(km.pair_off[k3].item())
     e = dt.itemsize
@@ -408,6 +413,8 @@ def run_only(args):
         "downsample": (lambda: scv.lat_downsample_coords(coords, scv.strided_geom(2, 2, 0), coarse, wsb, st,
                                                          parent=parent),
                        n * 16 * 2),
+        "upsample": (lambda: scv.lat_upsample_coords(coarse_c, g_up, fine_buf, wsb, st),
+                     coarse_c.shape[0] * 16 + n_fine * 16),
     }
     fn, nbytes = ops[args.only]
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
@@ -453,7 +460,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["hash", "kmap", "fwd", "dgrad", "wgrad", "downsample"],
+    ap.add_argument("--only", choices=["hash", "kmap", "fwd", "dgrad", "wgrad", "downsample", "upsample"],
                     help="time a single op of the path on --workload (for profiler captures)")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(synthetic.WORKLOADS))
     ap.add_argument("--rsv-ratio", type=float, default=RSV_RATIO, help="hash table slots per voxel (--only mode)")
