@@ -67,6 +67,10 @@ def _load():
             lib.orc_conv_dgrad.argtypes = [P, i64, i32, P, i32, P, i32, P, i64, i32]
             lib.orc_conv_wgrad.restype = None
             lib.orc_conv_wgrad.argtypes = [P, i32, P, i32, P, i64, i32, P, i32]
+            lib.orc_pool.restype = None
+            lib.orc_pool.argtypes = [P, i64, i32, P, i64, i32, i32, P]
+            lib.orc_to_dense.restype = i64
+            lib.orc_to_dense.argtypes = [P, i64, P, i32, P, P, i32, P]
             lib.orc_max_threads.restype = i32
             _lib = lib
     return _lib
@@ -197,3 +201,25 @@ def conv_wgrad(x, dy, nbr, nthreads=0) -> np.ndarray:
     _load().orc_conv_wgrad(_ptr(x), x.shape[1], _ptr(dy), dy.shape[1], _ptr(nbr), len(nbr), k3,
                            _ptr(dw), int(nthreads))
     return dw
+
+
+POOL_MAX, POOL_AVG = 0, 1
+
+
+def pool(x, nbr, op=POOL_MAX) -> np.ndarray:
+    """Max (op 0) or mean (op 1) of x over each output row's neighbours; 0 if none.  fp64."""
+    x, nbr = _f64(x), _i32(nbr)
+    n_out, k3 = nbr.shape
+    y = np.empty((n_out, x.shape[1]), np.float64)
+    _load().orc_pool(_ptr(x), len(x), x.shape[1], _ptr(nbr), n_out, k3, int(op), _ptr(y))
+    return y
+
+
+def to_dense(coords, feats, origin, shape, batch):
+    """(grid [batch, sx, sy, sz, C] fp64, number of rows outside the box)."""
+    coords, feats = _i32(coords).reshape(-1, 4), _f64(feats)
+    o, sh = _triple(origin), _triple(shape)
+    grid = np.empty((int(batch), int(sh[0]), int(sh[1]), int(sh[2]), feats.shape[1]), np.float64)
+    outside = _load().orc_to_dense(_ptr(coords), len(coords), _ptr(feats), feats.shape[1], _ptr(o), _ptr(sh),
+                                   int(batch), _ptr(grid))
+    return grid, int(outside)

@@ -25,6 +25,10 @@
 //     differences"); TorchSparse++'s abstract names gather-GEMM-scatter as the
 //     simple dataflow.  So the plain sum is the definition the fast path must
 //     reproduce up to rounding order.
+//   * Pooling and dense materialization are listed among the library's
+//     kernels ("What remains familiar") with no formula: pooling here is the
+//     max or mean over the same relation, dense materialization the scatter
+//     of each row into a zeroed grid.
 //
 // Readings where the pages are silent (each is listed in the design notes):
 //   * cross-correlation: y(q) = sum_k x(in(q,k)) * W[k], as dense conv3d;
@@ -36,6 +40,7 @@
 //   * packed key (b<<48)|(x+2^15)<<32|(y+2^15)<<16|(z+2^15), so unsigned key
 //     order equals lexicographic (b,x,y,z) order; b must lie in [0, 65534],
 //     x,y,z in [-32768, 32767].
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <cmath>
@@ -292,6 +297,57 @@ void orc_conv_wgrad(const double* x, int cin, const double* dy, int cout, const 
             for (int co = 0; co < cout; ++co) row[co] += xv * g[co];
         }
     }
+}
+
+// Sparse pooling over a relation (migration page, "What remains familiar":
+// pooling is one of the library's kernels; no formula is given, so the plain
+// reading): y[j][c] = max, or mean, of x[i][c] over the rows i = nbr[j][k] >= 0,
+// k ascending; 0 for a row with no neighbour.  op 0 = max, 1 = mean.  fp64.
+void orc_pool(const double* x, int64_t n_in, int c, const int32_t* nbr, int64_t n_out, int k3,
+              int op, double* y) {
+    (void)n_in;
+    for (int64_t j = 0; j < n_out; ++j) {
+        double* yj = y + j * c;
+        int count = 0;
+        for (int k = 0; k < k3; ++k) {
+            const int32_t i = nbr[j * k3 + k];
+            if (i < 0) continue;
+            const double* xi = x + int64_t(i) * c;
+            for (int ch = 0; ch < c; ++ch) {
+                if (count == 0) yj[ch] = xi[ch];
+                else if (op == 0) yj[ch] = std::max(yj[ch], xi[ch]);
+                else yj[ch] += xi[ch];
+            }
+            ++count;
+        }
+        for (int ch = 0; ch < c; ++ch) {
+            if (count == 0) yj[ch] = 0.0;
+            else if (op == 1) yj[ch] /= count;
+        }
+    }
+}
+
+// Dense materialization (same passage): out[b][x-ox][y-oy][z-oz][ch] =
+// feats[i][ch] for every row i = (b,x,y,z) inside the box, 0 elsewhere.
+// Returns the number of rows that fall outside the box (they are skipped).
+int64_t orc_to_dense(const int32_t* coords, int64_t n, const double* feats, int c, const int32_t* origin,
+                     const int32_t* shape, int batch, double* out) {
+    const int64_t cells = int64_t(batch) * shape[0] * shape[1] * shape[2];
+    std::memset(out, 0, sizeof(double) * size_t(cells) * c);
+    int64_t outside = 0;
+    for (int64_t i = 0; i < n; ++i) {
+        const int32_t* q = coords + 4 * i;
+        int64_t rel[3];
+        bool inside = q[0] >= 0 && q[0] < batch;
+        for (int a = 0; a < 3; ++a) {
+            rel[a] = int64_t(q[a + 1]) - origin[a];
+            inside = inside && rel[a] >= 0 && rel[a] < shape[a];
+        }
+        if (!inside) { ++outside; continue; }
+        const int64_t cell = ((int64_t(q[0]) * shape[0] + rel[0]) * shape[1] + rel[1]) * shape[2] + rel[2];
+        std::memcpy(out + cell * c, feats + i * c, sizeof(double) * c);
+    }
+    return outside;
 }
 
 int orc_max_threads() { return omp_get_max_threads(); }

@@ -389,3 +389,78 @@ def test_generative_transposed_conv_matches_dense_conv_transpose3d(ks, st, pd):
     dense = torch.nn.functional.conv_transpose3d(_densify(c, x, (8, 8, 8), tuple(origin)), wd, stride=st)
     read_origin = tuple(np.array(st) * origin - np.array(pd))
     np.testing.assert_allclose(y, _read(dense, gen, read_origin).numpy(), rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- pooling / dense grids
+_POOL_GEOMS = [(3, 1, 1, SUBM), (2, 2, 0, STRIDED), (3, 2, 1, STRIDED), ((3, 3, 1), 1, (1, 1, 0), SUBM)]
+
+
+def _pool_case(rng, ks, st, pd, mode):
+    c = _rand_coords(rng, 150, 0, 8, batch=2)
+    out = c if mode == SUBM else oracle.downsample(c, ks, st, pd)
+    x = rng.standard_normal((len(c), 5)) - 2.0          # mostly negative: a stray 0 would win a max
+    return c, out, x, oracle.kmap(c, out, ks, st, pd, mode)
+
+
+@pytest.mark.parametrize("ks,st,pd,mode", _POOL_GEOMS)
+def test_max_pool_matches_dense_max_pool3d(ks, st, pd, mode):
+    """Max over active neighbours = dense max_pool3d of a grid that holds -inf
+    at every inactive cell (torch pads with -inf too), read at the outputs."""
+    rng = np.random.default_rng(31 + st)
+    c, out, x, nbr = _pool_case(rng, ks, st, pd, mode)
+    grid = _densify(c, x, (10, 10, 10), (0, 0, 0))
+    occ = _densify(c, np.ones((len(c), 1)), (10, 10, 10), (0, 0, 0))
+    grid = torch.where(occ > 0, grid, torch.tensor(-np.inf, dtype=torch.float64))
+    ksz = (ks,) * 3 if np.isscalar(ks) else ks
+    pad = (pd,) * 3 if np.isscalar(pd) else pd
+    dense = torch.nn.functional.max_pool3d(grid, ksz, stride=st, padding=pad)
+    np.testing.assert_array_equal(oracle.pool(x, nbr, oracle.POOL_MAX), _read(dense, out, (0, 0, 0)).numpy())
+
+
+@pytest.mark.parametrize("ks,st,pd,mode", _POOL_GEOMS)
+def test_avg_pool_is_dense_window_sum_over_active_count(ks, st, pd, mode):
+    """Mean over active neighbours = (window sum of the zero-filled grid) /
+    (window sum of the occupancy grid): two dense avg_pool3d with divisor 1."""
+    rng = np.random.default_rng(47 + st)
+    c, out, x, nbr = _pool_case(rng, ks, st, pd, mode)
+    ksz = (ks,) * 3 if np.isscalar(ks) else ks
+    pad = (pd,) * 3 if np.isscalar(pd) else pd
+    sums = [torch.nn.functional.avg_pool3d(_densify(c, v, (10, 10, 10), (0, 0, 0)), ksz, stride=st, padding=pad,
+                                           count_include_pad=True, divisor_override=1)
+            for v in (x, np.ones((len(c), 1)))]
+    ref = (_read(sums[0], out, (0, 0, 0)) / _read(sums[1], out, (0, 0, 0))).numpy()
+    np.testing.assert_allclose(oracle.pool(x, nbr, oracle.POOL_AVG), ref, rtol=1e-13, atol=1e-13)
+
+
+def test_pool_of_row_without_neighbours_is_zero_and_k1_is_identity():
+    c = np.array([[0, 0, 0, 0], [0, 1, 0, 0]], np.int32)
+    far = np.array([[0, 9, 9, 9], [1, 0, 0, 0], [0, 0, 0, 0]], np.int32)
+    x = np.array([[-3.0, 4.0], [-1.0, 2.0]])
+    nbr = oracle.kmap(c, far, 3, 1, 1, STRIDED)
+    for op in (oracle.POOL_MAX, oracle.POOL_AVG):
+        y = oracle.pool(x, nbr, op)
+        assert np.all(y[:2] == 0.0)
+    np.testing.assert_array_equal(oracle.pool(x, nbr, oracle.POOL_MAX)[2], [-1.0, 4.0])
+    np.testing.assert_array_equal(oracle.pool(x, nbr, oracle.POOL_AVG)[2], [-2.0, 3.0])
+    rng = np.random.default_rng(3)
+    cc = _rand_coords(rng, 40, -5, 5, batch=2)
+    xx = rng.standard_normal((len(cc), 3))
+    for op in (oracle.POOL_MAX, oracle.POOL_AVG):
+        np.testing.assert_array_equal(oracle.pool(xx, oracle.kmap(cc, cc, 1, 1, 0, SUBM), op), xx)
+
+
+def test_to_dense_matches_sparse_coo_to_dense():
+    """Scatter into the box = torch's sparse COO tensor densified, shifted by the origin;
+    rows outside the box are dropped and counted."""
+    rng = np.random.default_rng(11)
+    c = _rand_coords(rng, 80, -4, 6, batch=3)
+    x = rng.standard_normal((len(c), 4))
+    origin, shape, batch = (-2, -4, -3), (7, 8, 9), 2
+    grid, outside = oracle.to_dense(c, x, origin, shape, batch)
+    rel = c.astype(np.int64) - np.array((0,) + origin)
+    inside = (rel[:, 0] < batch) & np.all(rel[:, 1:] >= 0, 1) & np.all(rel[:, 1:] < np.array(shape), 1)
+    assert outside == int((~inside).sum()) > 0
+    ref = torch.sparse_coo_tensor(torch.as_tensor(rel[inside].T), torch.as_tensor(x[inside]),
+                                  (batch,) + shape + (4,), check_invariants=True).to_dense()
+    np.testing.assert_array_equal(grid, ref.numpy())
+    assert np.count_nonzero(np.any(grid != 0, axis=-1)) == int(inside.sum())
