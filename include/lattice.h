@@ -330,6 +330,44 @@ lat_status lat_sconv_wgrad_static(const void *x, int32_t cin, const void *dy, in
                                   const lat_kmap *map, float *dw, lat_dtype dtype,
                                   int32_t *d_status, lat_stream stream);
 
+/* ------------------------------------------- pooling and dense grids --- */
+
+typedef enum { LAT_POOL_MAX = 0, LAT_POOL_AVG = 1 } lat_pool_op;
+
+/* Sparse pooling over a kernel map ("What remains familiar" of the
+ * migration page: pooling is one of the library's CUDA kernels; the pages
+ * give no formula, so the plain reading is taken).  For every output row j:
+ *   y[j][c] = max  over { x[nbr[k*n_out + j]][c] : bit k of mask[j] set }
+ *   y[j][c] = mean over the same set (fp32 sum in ascending k, divided by
+ *             the number of neighbours)
+ * and y[j] = 0 where mask[j] == 0.  The map is any map lat_kmap_query or
+ * lat_kmap_from_parent built (SUBM, strided or transposed geometry); only
+ * nbr and mask are read, with map->n_in / n_out / k3 giving the sizes.
+ *   x  device [n_in][c] of dtype; y device [n_out][c] of dtype (no overlap
+ *      with x).  Both 16-byte aligned; c a multiple of 8 and >= 8.
+ *   Arithmetic is fp32; each output is rounded once to dtype.
+ *   op is lat_pool_op.  Host checks return LAT_ERR_ARG; a row index outside
+ *   [0, n_in) in the map sets LAT_ERR_BAD_MAP at d_status (may be NULL) and
+ *   is skipped.  Asynchronous on `stream`; allocates nothing. */
+lat_status lat_sparse_pool(const void *x, int32_t c, const lat_kmap *map, int32_t op, void *y,
+                           lat_dtype dtype, int32_t *d_status, lat_stream stream);
+
+/* Dense materialization (same passage): write the sparse tensor into a
+ * zero-filled channels-last grid out[batch][shape[0]][shape[1]][shape[2]][c]
+ * of dtype covering x in [origin[0], origin[0]+shape[0]) and likewise for
+ * y and z, batches 0..batch-1.  Row i lands in cell
+ * (b, x-origin[0], y-origin[1], z-origin[2]) of coords[i] = (b,x,y,z); a row
+ * outside the box is skipped and sets LAT_ERR_COORD_RANGE at d_status.
+ * Coordinates are expected unique (as after hashing); with duplicates one
+ * of the rows wins, which one is unspecified.
+ *   coords device int32 [n][4], 16-byte aligned; feats device [n][c];
+ *   origin, shape host int32[3]; out device, 16-byte aligned,
+ *   batch*shape[0]*shape[1]*shape[2]*c elements.  c a multiple of 8.
+ * Enqueues a memset of `out` and one scatter kernel on `stream`. */
+lat_status lat_to_dense(const int32_t *coords, int64_t n, const void *feats, int32_t c, lat_dtype dtype,
+                        const int32_t *origin, const int32_t *shape, int32_t batch, void *out,
+                        int32_t *d_status, lat_stream stream);
+
 /* ---------------------------------------------------------------- misc --- */
 
 /* Synchronise `stream`, then return the status word at d_status (device). */

@@ -17,16 +17,16 @@ import torch
 
 from ._lib import (  # noqa: F401  (re-exported C entry points and constants)
     EXPORTS, LAT_BF16, LAT_F16, LAT_F32, LAT_OK, LAT_OP_DGRAD, LAT_OP_FWD, LAT_OP_WGRAD, LAT_STRIDED, LAT_SUBM,
-    LAT_TILE_ROWS, LAT_TRANSPOSED, LIB_PATH, LatticeError, lat_downsample_coords, lat_downsample_coords_async, lat_downsample_ws_bytes, lat_geom,
+    LAT_POOL_AVG, LAT_POOL_MAX, LAT_TILE_ROWS, LAT_TRANSPOSED, LIB_PATH, LatticeError, lat_downsample_coords, lat_downsample_coords_async, lat_downsample_ws_bytes, lat_geom,
     lat_upsample_coords, lat_upsample_ws_bytes,
     lat_hash_build, lat_hash_bytes, lat_kmap, lat_kmap_from_parent, lat_kmap_from_parent_ws_bytes, lat_kmap_query,
-    lat_kmap_ws_bytes, lat_sconv_dgrad, lat_sconv_fwd,
+    lat_kmap_ws_bytes, lat_sconv_dgrad, lat_sconv_fwd, lat_sparse_pool, lat_to_dense,
     lat_sconv_wgrad, lat_sconv_wgrad_static, lat_sconv_ws_bytes, lat_status_fetch, lat_status_string, lat_version, load, make_geom,
 )
 
 __all__ = [
     "KernelMap", "Workspace", "hash_table", "kernel_map", "downsample", "downsample_async", "PendingDownsample",
-    "upsample", "maps_from_parent", "conv_fwd", "conv_dgrad", "conv_wgrad",
+    "upsample", "maps_from_parent", "conv_fwd", "conv_dgrad", "conv_wgrad", "sparse_pool", "to_dense",
     "subm_geom", "strided_geom", "target_geom", "transposed_geom", "check_status", "new_status",
 ] + EXPORTS
 
@@ -239,3 +239,19 @@ def conv_wgrad(x, dy, kmap: KernelMap, ws: Workspace | None = None, d_status=Non
                     ws.get(lat_sconv_ws_bytes(LAT_OP_WGRAD, x.shape[1], dy.shape[1], kmap.c, x.dtype)), d_status,
                     stream)
     return dw
+
+
+def sparse_pool(x, kmap: KernelMap, op: str = "max", d_status=None, out=None, stream=None):
+    """Max or mean of x over each output row's neighbours in ``kmap`` (0 where it has none)."""
+    code = {"max": LAT_POOL_MAX, "avg": LAT_POOL_AVG, "mean": LAT_POOL_AVG}[op]
+    y = out if out is not None else torch.empty((kmap.n_out, x.shape[1]), dtype=x.dtype, device=x.device)
+    lat_sparse_pool(x, kmap.c, code, y, d_status, stream)
+    return y
+
+
+def to_dense(coords, feats, origin, shape, batch: int, d_status=None, out=None, stream=None):
+    """Channels-last dense grid [batch, shape[0], shape[1], shape[2], C] over the box at ``origin``."""
+    size = (int(batch), int(shape[0]), int(shape[1]), int(shape[2]), feats.shape[1])
+    grid = out if out is not None else torch.empty(size, dtype=feats.dtype, device=feats.device)
+    lat_to_dense(coords, feats, origin, shape, batch, grid, d_status, stream)
+    return grid

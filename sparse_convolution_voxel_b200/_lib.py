@@ -21,6 +21,7 @@ LAT_F32, LAT_F16, LAT_BF16 = 0, 1, 2
 LAT_SUBM, LAT_STRIDED, LAT_TRANSPOSED = 0, 1, 2
 LAT_OP_FWD, LAT_OP_DGRAD, LAT_OP_WGRAD = 0, 1, 2
 LAT_TILE_ROWS = 128
+LAT_POOL_MAX, LAT_POOL_AVG = 0, 1
 
 STATUS_BITS = {
     1: "LAT_ERR_ARG", 2: "LAT_ERR_COORD_RANGE", 4: "LAT_ERR_DUPLICATE", 8: "LAT_ERR_TABLE_FULL",
@@ -35,7 +36,8 @@ EXPORTS = [
     "lat_upsample_coords", "lat_kmap_from_parent_ws_bytes",
     "lat_kmap_from_parent",
     "lat_sconv_ws_bytes", "lat_sconv_fwd",
-    "lat_sconv_dgrad", "lat_sconv_wgrad", "lat_sconv_wgrad_static", "lat_status_fetch", "lat_status_string", "lat_version",
+    "lat_sconv_dgrad", "lat_sconv_wgrad", "lat_sconv_wgrad_static", "lat_sparse_pool", "lat_to_dense",
+    "lat_status_fetch", "lat_status_string", "lat_version",
 ]
 
 
@@ -89,6 +91,8 @@ def load() -> ctypes.CDLL:
         "lat_sconv_dgrad": (I32, [P, I32, P, I32, K, I32, P, I32, P, SZ, P, P]),
         "lat_sconv_wgrad": (I32, [P, I32, P, I32, K, P, I32, P, SZ, P, P]),
         "lat_sconv_wgrad_static": (I32, [P, I32, P, I32, K, P, I32, P, P]),
+        "lat_sparse_pool": (I32, [P, I32, K, I32, P, I32, P, P]),
+        "lat_to_dense": (I32, [P, I64, P, I32, I32, ctypes.POINTER(I32), ctypes.POINTER(I32), I32, P, P, P]),
         "lat_status_fetch": (I32, [P, P]),
         "lat_status_string": (ctypes.c_char_p, [I32]),
         "lat_version": (I32, []),
@@ -253,6 +257,20 @@ def lat_sconv_wgrad_static(x, dy, kmap: lat_kmap, dw, d_status=None, stream=None
     rc = load().lat_sconv_wgrad_static(_ptr(x), x.shape[1], _ptr(dy), dy.shape[1], ctypes.byref(kmap), _ptr(dw),
                                        dtype_code(x.dtype), _ptr(d_status), _stream(stream))
     _check(rc, "lat_sconv_wgrad_static")
+
+
+def lat_sparse_pool(x, kmap: lat_kmap, op: int, y, d_status=None, stream=None):
+    rc = load().lat_sparse_pool(_ptr(x), x.shape[1], ctypes.byref(kmap), int(op), _ptr(y), dtype_code(x.dtype),
+                                _ptr(d_status), _stream(stream))
+    _check(rc, "lat_sparse_pool")
+
+
+def lat_to_dense(coords, feats, origin, shape, batch: int, out, d_status=None, stream=None):
+    o = (ctypes.c_int32 * 3)(*[int(v) for v in origin])
+    sh = (ctypes.c_int32 * 3)(*[int(v) for v in shape])
+    rc = load().lat_to_dense(_ptr(coords), coords.shape[0], _ptr(feats), feats.shape[1], dtype_code(feats.dtype), o,
+                             sh, int(batch), _ptr(out), _ptr(d_status), _stream(stream))
+    _check(rc, "lat_to_dense")
 
 
 def lat_status_fetch(d_status: torch.Tensor, stream=None) -> int:

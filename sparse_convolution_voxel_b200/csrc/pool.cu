@@ -1,0 +1,177 @@
+// Sparse pooling over a kernel map and dense materialization
+// (lat_sparse_pool, lat_to_dense).
+//
+// Torch Lattice docs, "Migrating from TorchSparse", "What remains familiar":
+// pooling and dense conversion are among the library's CUDA kernels.  The
+// pages fix no formula; the plainest reading is taken:
+//   pool:  y[j][c] = max (or mean) over the offsets k with a neighbour of
+//          x[nbr[k][j]][c]; rows with no neighbour get 0.  fp32 arithmetic,
+//          the mean is the sum in offset order divided by the neighbour count,
+//          one rounding to the output type.
+//   dense: a channels-last grid over a caller-given box, zero where no row
+//          lies; every row inside the box writes its features to its cell.
+// Both are memory-bound gathers / scatters on CUDA cores: one thread per (row,
+// 8-channel group), 16-byte (fp16/bf16) or 2 x 16-byte (fp32) accesses.
+#include "common.cuh"
+
+namespace lat {
+
+template <typename T>
+__device__ __forceinline__ void ld8(const T *p, float (&v)[8]) {
+    if constexpr (sizeof(T) == 4) {
+        const float4 a = __ldg(reinterpret_cast<const float4 *>(p));
+        const float4 b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+        const uint4 a = __ldg(reinterpret_cast<const uint4 *>(p));
+        const T *e = reinterpret_cast<const T *>(&a);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) v[c] = Elem<T>::to_f(e[c]);
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ void st8(T *p, const float (&v)[8]) {
+    if constexpr (sizeof(T) == 4) {
+        reinterpret_cast<float4 *>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+        reinterpret_cast<float4 *>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+    } else {
+        uint4 o;
+        T *e = reinterpret_cast<T *>(&o);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) e[c] = Elem<T>::from_f(v[c]);
+        *reinterpret_cast<uint4 *>(p) = o;
+    }
+}
+
+// One thread per (output row, group of 8 channels); the offsets come from the row's mask.
+template <typename T, bool MAX>
+__global__ void __launch_bounds__(256)
+pool_kernel(const T *__restrict__ x, int c, const int32_t *__restrict__ nbr, const uint32_t *__restrict__ mask,
+            int64_t n_in, int64_t n_out, T *__restrict__ y, int32_t *d_status) {
+    const int groups = c / 8;
+    const int64_t gid = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+    const int64_t j = gid / groups;
+    if (j >= n_out) return;
+    const int cg = int(gid - j * groups);
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = MAX ? -INFINITY : 0.f;
+    int cnt = 0;
+    int32_t bad = 0;
+    for (uint32_t m = __ldg(mask + j); m; m &= m - 1) {
+        const int k = __ffs(m) - 1;
+        const int i = __ldg(nbr + int64_t(k) * n_out + j);
+        if (i < 0 || i >= n_in) {
+            bad |= LAT_ERR_BAD_MAP;
+            continue;
+        }
+        float v[8];
+        ld8<T>(x + int64_t(i) * c + cg * 8, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = MAX ? fmaxf(acc[e], v[e]) : acc[e] + v[e];
+        ++cnt;
+    }
+    if (bad) flag(d_status, bad);
+    float out[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) out[e] = cnt == 0 ? 0.f : (MAX ? acc[e] : acc[e] / float(cnt));
+    st8<T>(y + j * c + cg * 8, out);
+}
+
+struct Box {
+    int ox, oy, oz, sx, sy, sz, batch;
+};
+
+// Scatter every row inside the box into its cell of the zeroed channels-last grid.
+template <typename T>
+__global__ void __launch_bounds__(256)
+dense_scatter_kernel(const int4 *__restrict__ coords, int64_t n, const T *__restrict__ feats, int c, Box bx,
+                     T *__restrict__ out, int32_t *d_status) {
+    const int groups = c / 8;
+    const int64_t gid = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+    const int64_t i = gid / groups;
+    if (i >= n) return;
+    const int cg = int(gid - i * groups);
+    const int4 q = __ldg(coords + i);
+    const int x = q.y - bx.ox, y = q.z - bx.oy, z = q.w - bx.oz;
+    if (q.x < 0 || q.x >= bx.batch || x < 0 || x >= bx.sx || y < 0 || y >= bx.sy || z < 0 || z >= bx.sz) {
+        if (cg == 0) flag(d_status, LAT_ERR_COORD_RANGE);
+        return;
+    }
+    const int64_t cell = ((int64_t(q.x) * bx.sx + x) * bx.sy + y) * bx.sz + z;
+    float v[8];
+    ld8<T>(feats + i * c + cg * 8, v);
+    st8<T>(out + cell * c + cg * 8, v);
+}
+
+template <typename T>
+static lat_status launch_pool(const void *x, int c, const lat_kmap *map, int op, void *y, int32_t *d_status,
+                              cudaStream_t s) {
+    const int64_t threads = map->n_out * (c / 8);
+    if (threads == 0) return LAT_OK;
+    const unsigned blocks = unsigned((threads + 255) / 256);
+    if (op == LAT_POOL_MAX)
+        pool_kernel<T, true><<<blocks, 256, 0, s>>>(static_cast<const T *>(x), c, map->nbr, map->mask, map->n_in,
+                                                    map->n_out, static_cast<T *>(y), d_status);
+    else
+        pool_kernel<T, false><<<blocks, 256, 0, s>>>(static_cast<const T *>(x), c, map->nbr, map->mask, map->n_in,
+                                                     map->n_out, static_cast<T *>(y), d_status);
+    LAT_CUDA_TRY(cudaGetLastError());
+    return LAT_OK;
+}
+
+template <typename T>
+static lat_status launch_dense(const int32_t *coords, int64_t n, const void *feats, int c, const Box &bx, void *out,
+                               int32_t *d_status, cudaStream_t s) {
+    const size_t cells = size_t(bx.batch) * bx.sx * bx.sy * bx.sz;
+    LAT_CUDA_TRY(cudaMemsetAsync(out, 0, cells * c * sizeof(T), s));
+    const int64_t threads = n * (c / 8);
+    if (threads == 0) return LAT_OK;
+    dense_scatter_kernel<T><<<unsigned((threads + 255) / 256), 256, 0, s>>>(
+        reinterpret_cast<const int4 *>(coords), n, static_cast<const T *>(feats), c, bx, static_cast<T *>(out),
+        d_status);
+    LAT_CUDA_TRY(cudaGetLastError());
+    return LAT_OK;
+}
+
+static bool aligned16(const void *p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
+
+}  // namespace lat
+
+extern "C" lat_status lat_sparse_pool(const void *x, int32_t c, const lat_kmap *map, int32_t op, void *y,
+                                      lat_dtype dtype, int32_t *d_status, lat_stream stream) {
+    using namespace lat;
+    if (!map || map->k3 < 1 || map->k3 > 32 || map->n_in < 0 || map->n_out < 0) return LAT_ERR_ARG;
+    if (map->n_out >= (int64_t(1) << 31) || map->n_in >= (int64_t(1) << 31)) return LAT_ERR_ARG;
+    if (c < 8 || c % 8 || (op != LAT_POOL_MAX && op != LAT_POOL_AVG)) return LAT_ERR_ARG;
+    if (map->n_out > 0 && (!map->nbr || !map->mask || !y || (map->n_in > 0 && !x))) return LAT_ERR_ARG;
+    if (!aligned16(x) || !aligned16(y)) return LAT_ERR_ARG;
+    if (int64_t(map->n_out) * (c / 8) >= (int64_t(1) << 40)) return LAT_ERR_UNSUPPORTED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    switch (dtype) {
+        case LAT_F32: return launch_pool<float>(x, c, map, op, y, d_status, s);
+        case LAT_F16: return launch_pool<__half>(x, c, map, op, y, d_status, s);
+        case LAT_BF16: return launch_pool<__nv_bfloat16>(x, c, map, op, y, d_status, s);
+    }
+    return LAT_ERR_ARG;
+}
+
+extern "C" lat_status lat_to_dense(const int32_t *coords, int64_t n, const void *feats, int32_t c, lat_dtype dtype,
+                                   const int32_t *origin, const int32_t *shape, int32_t batch, void *out,
+                                   int32_t *d_status, lat_stream stream) {
+    using namespace lat;
+    if (n < 0 || c < 8 || c % 8 || !origin || !shape || batch < 1 || !out) return LAT_ERR_ARG;
+    if (n > 0 && (!coords || !feats)) return LAT_ERR_ARG;
+    for (int a = 0; a < 3; ++a)
+        if (shape[a] < 1) return LAT_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(coords) % 16 || !aligned16(feats) || !aligned16(out)) return LAT_ERR_ARG;
+    const Box bx{origin[0], origin[1], origin[2], shape[0], shape[1], shape[2], batch};
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    switch (dtype) {
+        case LAT_F32: return launch_dense<float>(coords, n, feats, c, bx, out, d_status, s);
+        case LAT_F16: return launch_dense<__half>(coords, n, feats, c, bx, out, d_status, s);
+        case LAT_BF16: return launch_dense<__nv_bfloat16>(coords, n, feats, c, bx, out, d_status, s);
+    }
+    return LAT_ERR_ARG;
+}

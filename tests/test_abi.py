@@ -88,3 +88,28 @@ def test_conv_workspace_query_and_check_without_gpu(lib):
     assert lib.lat_sconv_fwd(P(16), 64, P(16), 64, ctypes.byref(km), P(16), f16, None, 0, None, None) == 128
     assert lib.lat_sconv_fwd(P(16), 64, P(16), 64, ctypes.byref(km), P(16), f16, P(256), 16, None, None) == 128
     assert lib.lat_sconv_dgrad(P(16), 128, P(16), 64, ctypes.byref(km), 1, P(16), f16, None, 0, None, None) == 128
+
+
+def test_pool_and_dense_argument_checks_without_gpu(lib):
+    """Every rejected argument returns LAT_ERR_ARG before anything is enqueued."""
+    P = ctypes.c_void_p
+    km = _lib.lat_kmap()
+    km.k3, km.n_out, km.n_in = 27, 10, 10
+    km.nbr, km.mask = P(16), P(16)
+    ok = (P(16), 16, ctypes.byref(km), 0, P(32), 0, None, None)
+    assert lib.lat_sparse_pool(None, 16, None, 0, P(32), 0, None, None) == 1          # no map
+    assert lib.lat_sparse_pool(P(16), 12, *ok[2:]) == 1                                # C % 8
+    assert lib.lat_sparse_pool(*ok[:3], 2, *ok[4:]) == 1                               # unknown op
+    assert lib.lat_sparse_pool(P(24), *ok[1:]) == 1                                    # x not 16-byte aligned
+    km.k3 = 33
+    assert lib.lat_sparse_pool(*ok) == 1
+    km.k3, km.mask = 27, None
+    assert lib.lat_sparse_pool(*ok) == 1                                               # no mask
+    i3 = ctypes.c_int32 * 3
+    o, sh = i3(0, 0, 0), i3(4, 4, 4)
+    assert lib.lat_to_dense(P(16), 5, P(16), 8, 0, o, sh, 0, P(16), None, None) == 1   # batch 0
+    assert lib.lat_to_dense(P(16), 5, P(16), 8, 0, o, i3(4, 0, 4), 1, P(16), None, None) == 1
+    assert lib.lat_to_dense(P(16), 5, P(16), 10, 0, o, sh, 1, P(16), None, None) == 1  # C % 8
+    assert lib.lat_to_dense(None, 5, P(16), 8, 0, o, sh, 1, P(16), None, None) == 1
+    assert lib.lat_to_dense(P(8), 5, P(16), 8, 0, o, sh, 1, P(16), None, None) == 1    # coords alignment
+    assert lib.lat_to_dense(P(16), 5, P(16), 8, 3, o, sh, 1, P(16), None, None) == 1   # dtype
