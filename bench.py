@@ -375,7 +375,9 @@ def run_only(args):
     torch.cuda.set_device(dev)
     wl = synthetic.WORKLOADS[args.workload]
     dt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[wl.dtype]
-    k3 = int(np.prod(wl.ksize))
+    # even kernels (the down/up workload) have no submanifold form: its subm ops use 3x3x3
+    ksize = wl.ksize if all(k % 2 for k in wl.ksize) else (3, 3, 3)
+    k3 = int(np.prod(ksize))
     coords = torch.from_numpy(wl.coords()).to(dev)
     n = coords.shape[0]
     cin, cout = wl.cin, wl.cout
@@ -384,7 +386,7 @@ def run_only(args):
     w = torch.from_numpy(synthetic.weights(k3, cin, cout, wl.seed)).to(dt).to(dev)
     st = scv.new_status(dev)
     ws = scv.Workspace(dev)
-    geom = scv.subm_geom(wl.ksize)
+    geom = scv.subm_geom(ksize)
     table = scv.hash_table(coords, args.rsv_ratio, st)
     km = scv.kernel_map(table, n, coords, geom, ws, st)
     y = torch.empty((n, cout), dtype=dt, device=dev)
@@ -415,7 +417,27 @@ def run_only(args):
                        n * 16 * 2),
         "upsample": (lambda: scv.lat_upsample_coords(coarse_c, g_up, fine_buf, wsb, st),
                      coarse_c.shape[0] * 16 + n_fine * 16),
+        # pooling: x read once, y written once, the mask and every used neighbour index
+        "pool_max": (lambda: scv.lat_sparse_pool(x, km.c, scv.LAT_POOL_MAX, dx, st), 2 * n * cin * e + 4 * n + 4 * P),
+        "pool_avg": (lambda: scv.lat_sparse_pool(x, km.c, scv.LAT_POOL_AVG, dx, st), 2 * n * cin * e + 4 * n + 4 * P),
     }
+    if args.only == "pool_down":
+        # k2s2 max pooling onto the generated coarse support
+        g_dn = scv.strided_geom(2, 2, 0)
+        coarse_p = scv.downsample(coords, g_dn, ws).contiguous()
+        km_dn = scv.kernel_map(table, n, coarse_p, g_dn, ws, st)
+        y_dn = torch.empty((coarse_p.shape[0], cin), dtype=dt, device=dev)
+        torch.cuda.synchronize()
+        P = int(km_dn.pair_off[8].item())
+        ops["pool_down"] = (lambda: scv.lat_sparse_pool(x, km_dn.c, scv.LAT_POOL_MAX, y_dn, st),
+                            (n + coarse_p.shape[0]) * cin * e + 4 * coarse_p.shape[0] + 4 * P)
+    if args.only == "dense":
+        # dense grid over the coordinates' bounding box: the whole grid written once, rows read once
+        lo, hi = coords.amin(0).tolist(), coords.amax(0).tolist()
+        box = [hi[a + 1] - lo[a + 1] + 1 for a in range(3)]
+        grid = torch.empty((hi[0] + 1, *box, cin), dtype=dt, device=dev)
+        ops["dense"] = (lambda: scv.lat_to_dense(coords, x, lo[1:], box, hi[0] + 1, grid, st),
+                        grid.numel() * e + n * 16 + n * cin * e)
     fn, nbytes = ops[args.only]
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     for _ in range(args.warmup):
@@ -460,7 +482,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["hash", "kmap", "fwd", "dgrad", "wgrad", "downsample", "upsample"],
+    ap.add_argument("--only", choices=["hash", "kmap", "fwd", "dgrad", "wgrad", "downsample", "upsample", "pool_max",
+                                       "pool_avg", "pool_down", "dense"],
                     help="time a single op of the path on --workload (for profiler captures)")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(synthetic.WORKLOADS))
     ap.add_argument("--rsv-ratio", type=float, default=RSV_RATIO, help="hash table slots per voxel (--only mode)")

@@ -11,8 +11,9 @@
  *   - Conv3d, strided  generates a downsampled support;
  *   - ConvTranspose3d  consumes an existing relation back onto a known support;
  * and the hashing, kernel-map construction and coordinate query that feed
- * them ("What remains familiar": CUDA kernels cover sparse convolution,
- * hashing and coordinate query).  Forward, data-gradient and per-offset
+ * them, plus pooling over a relation and dense materialization ("What
+ * remains familiar": CUDA kernels cover sparse convolution, pooling, hashing,
+ * coordinate query and dense materialization).  Forward, data-gradient and per-offset
  * weight-gradient passes are provided, since models train with standard
  * optimizers (same page) and TorchSparse++ targets training as well as
  * inference (TorchSparse++ abstract).
@@ -347,8 +348,8 @@ typedef enum { LAT_POOL_MAX = 0, LAT_POOL_AVG = 1 } lat_pool_op;
  *      with x).  Both 16-byte aligned; c a multiple of 8 and >= 8.
  *   Arithmetic is fp32; each output is rounded once to dtype.
  *   op is lat_pool_op.  Host checks return LAT_ERR_ARG; a row index outside
- *   [0, n_in) in the map sets LAT_ERR_BAD_MAP at d_status (may be NULL) and
- *   is skipped.  Asynchronous on `stream`; allocates nothing. */
+ *   [0, n_in) or a mask bit at or above k3 sets LAT_ERR_BAD_MAP at d_status
+ *   (may be NULL) and that neighbour is skipped.  Asynchronous on `stream`; allocates nothing. */
 lat_status lat_sparse_pool(const void *x, int32_t c, const lat_kmap *map, int32_t op, void *y,
                            lat_dtype dtype, int32_t *d_status, lat_stream stream);
 
