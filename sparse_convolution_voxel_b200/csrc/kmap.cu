@@ -4,12 +4,12 @@
 // and coordinate query are CUDA kernels of the library ("What remains
 // familiar", "Sparse tensor expectations"), and the support semantics come
 // from the "Convolution mapping" table.  Pipeline (all on `stream`):
-//   1. probe:  one thread per output row probes the input table (for a
-//              submanifold map only the offsets below the centre, mirroring
-//              each hit); writes nbr (offset-major, coalesced), mask, and per
-//              (offset, block) hit counts from warp ballots (for submanifold
-//              maps the masks are ORed in atomically and a count pass over the
-//              masks gives the counts).
+//   1. probe:  strided / transposed maps: one thread per output row probes
+//              every offset and writes nbr (offset-major, coalesced), mask and
+//              per (offset, block) hit counts from warp ballots.  Submanifold
+//              maps: one thread per (row, offset below the centre), each hit
+//              mirrored (the relation is symmetric) and ORed into both masks
+//              atomically; a count pass over the masks gives the counts.
 //   2. scan:   one block per offset turns its per-block counts into offsets
 //              (pairs come out grouped by offset, rows ascending).
 //   3. emit:   walks the masks and writes (in, out) pairs at ballot-ranked
@@ -109,32 +109,23 @@ __device__ __forceinline__ bool query_coord(const Geom &g, const int4 &c, int ix
 // what it can (a match, or an empty slot before it, ends the probe); the rows
 // of the matches are loaded together after the rounds.  At the table's load
 // factor nearly every probe ends inside its home group, so a batch takes about
-// one round.  Rounds are bounded by the group count.
-//
-// SYM (submanifold maps): the relation is symmetric -- input i sits at offset
-// k of row j exactly when j sits at offset k3-1-k of row i -- so only the
-// offsets below the centre are probed; a hit also writes the mirrored entry
-// (the upper half of nbr must hold -1 beforehand) and ORs the mirrored bit into
-// the other row's mask (masks must hold 0 beforehand), and the centre is the
-// row itself.  Keys and per-block counts then come from kmap_count_kernel.
-// Otherwise every offset is probed and the mask and counts are produced here.
-template <bool SYM>
+// one round.  Rounds are bounded by the group count.  Strided and transposed
+// maps (submanifold maps use kmap_probe_sym_kernel): every offset is probed and
+// the mask, grouping key, first sort histogram and per-block counts are
+// produced here.
 __global__ void __launch_bounds__(kQueryThreads)
 kmap_probe_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const int4 *__restrict__ out_coords,
                   int64_t n_out, int64_t n_in, Geom g, int32_t *__restrict__ nbr, uint32_t *__restrict__ mask,
                   uint32_t *__restrict__ keys, int32_t *__restrict__ hist, int ntile, int32_t *__restrict__ block_counts,
                   int nblk, int32_t *d_status) {
     __shared__ int s_cnt[32];
-    if (!SYM) {
-        if (threadIdx.x < 32) s_cnt[threadIdx.x] = 0;
-        __syncthreads();
-    }
+    if (threadIdx.x < 32) s_cnt[threadIdx.x] = 0;
+    __syncthreads();
     const int64_t j = blockIdx.x * int64_t(kQueryThreads) + threadIdx.x;
     const bool live = j < n_out;
     int4 c = make_int4(0, 0, 0, 0);
     if (live) c = __ldg(out_coords + j);
-    const int centre = g.mode == LAT_SUBM ? g.k3 / 2 : -1;
-    const int kend = SYM ? centre : g.k3;
+    const int kend = g.k3;
     uint64_t self = 0;
     const bool fast = live && g.shift && c.y >= g.lo[0] && c.y <= g.hi[0] && c.z >= g.lo[1] && c.z <= g.hi[1] &&
                       c.w >= g.lo[2] && c.w <= g.hi[2] && pack_key(c.x, c.y, c.z, c.w, self);
@@ -154,10 +145,6 @@ kmap_probe_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const
             key[e] = kEmptyKey;
             slot[e] = 0;
             if (!live || k >= kend) continue;
-            if (k == centre) {
-                row[e] = int(j);
-                continue;
-            }
             bool ok;
             if (fast) {
                 key[e] = self + uint64_t(g.delta[k]);
@@ -212,29 +199,14 @@ kmap_probe_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const
             const int k = k0 + e;
             if (k >= kend) break;
             int r = row[e];
-            if (r >= n_in || (SYM && r >= n_out)) { bad |= LAT_ERR_BAD_MAP; r = -1; }
+            if (r >= n_in) { bad |= LAT_ERR_BAD_MAP; r = -1; }
             if (live) nbr[int64_t(k) * n_out + j] = r;
-            if (SYM) {
-                if (r >= 0) {
-                    nbr[int64_t(g.k3 - 1 - k) * n_out + r] = int32_t(j);
-                    m |= 1u << k;
-                    atomicOr(mask + r, 1u << (g.k3 - 1 - k));
-                }
-            } else {
-                const unsigned hits = __ballot_sync(0xFFFFFFFFu, r >= 0);
-                if (r >= 0) m |= 1u << k;
-                if ((threadIdx.x & 31) == 0 && hits) atomicAdd(&s_cnt[k], __popc(hits));
-            }
+            const unsigned hits = __ballot_sync(0xFFFFFFFFu, r >= 0);
+            if (r >= 0) m |= 1u << k;
+            if ((threadIdx.x & 31) == 0 && hits) atomicAdd(&s_cnt[k], __popc(hits));
         }
     }
     if (bad) flag(d_status, bad);
-    if (SYM) {
-        if (live) {
-            nbr[int64_t(centre) * n_out + j] = int32_t(j);
-            atomicOr(mask + j, m | (1u << centre));  // mirrored hits of other rows OR in concurrently
-        }
-        return;
-    }
     const uint32_t key = group_key(m, g.k3);
     if (live) {
         mask[j] = m;
@@ -243,6 +215,86 @@ kmap_probe_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const
     sort_hist_add(key, live, j, hist, ntile);
     __syncthreads();
     if (threadIdx.x < g.k3) block_counts[int64_t(threadIdx.x) * nblk + blockIdx.x] = s_cnt[threadIdx.x];
+}
+
+// Submanifold map, step 0: the centre row of nbr (every row is its own centre
+// neighbour), -1 in every offset above the centre (filled by mirrored hits
+// only), and masks holding just the centre bit.  One thread per row; all stores
+// coalesced.
+__global__ void __launch_bounds__(kQueryThreads)
+kmap_subm_init_kernel(int64_t n_out, int k3, int32_t *__restrict__ nbr, uint32_t *__restrict__ mask) {
+    const int64_t j = blockIdx.x * int64_t(kQueryThreads) + threadIdx.x;
+    if (j >= n_out) return;
+    const int centre = k3 / 2;
+    nbr[int64_t(centre) * n_out + j] = int32_t(j);
+    for (int k = centre + 1; k < k3; ++k) nbr[int64_t(k) * n_out + j] = -1;
+    mask[j] = 1u << centre;
+}
+
+// Submanifold map, step 1: one thread per (offset k below the centre, row j);
+// blockIdx.y is the offset, so a warp probes one offset for 32 consecutive rows
+// (coalesced coordinate loads and nbr stores, a uniform key delta).  A probe
+// reads its home group's 4 keys with two 16-byte loads and walks on to the next
+// group only when all 4 slots hold other keys (bounded by the group count).
+// A hit at row r also writes the mirrored entry nbr[k3-1-k][r] = j (the
+// relation is symmetric) and ORs both bits into the masks.  Far fewer
+// instructions per lookup than looping over the offsets inside one thread,
+// and about 30 registers, so every SM runs its full complement of warps.
+__global__ void __launch_bounds__(kQueryThreads)
+kmap_probe_sym_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const int4 *__restrict__ out_coords,
+                      int64_t n_out, Geom g, int32_t *__restrict__ nbr, uint32_t *__restrict__ mask,
+                      int32_t *d_status) {
+    const int k = blockIdx.y;
+    const int64_t j = blockIdx.x * int64_t(kQueryThreads) + threadIdx.x;
+    if (j >= n_out) return;
+    const int4 c = __ldg(out_coords + j);
+    uint64_t key = 0;
+    bool ok;
+    if (g.shift && c.y >= g.lo[0] && c.y <= g.hi[0] && c.z >= g.lo[1] && c.z <= g.hi[1] && c.w >= g.lo[2] &&
+        c.w <= g.hi[2] && pack_key(c.x, c.y, c.z, c.w, key)) {
+        key += uint64_t(g.delta[k]);
+        ok = true;
+    } else {
+        ok = query_coord(g, c, g.off[k][0], g.off[k][1], g.off[k][2], key);
+    }
+    int r = -1;
+    if (ok) {
+        uint32_t slot = probe_start(key, cap_mask);
+        for (uint32_t round = 0; round <= cap_mask / kGroupSlots; ++round) {
+            const SlotGroup *gp = groups + slot / kGroupSlots;
+            const ulonglong2 a = __ldg(reinterpret_cast<const ulonglong2 *>(gp->key));
+            const ulonglong2 b = __ldg(reinterpret_cast<const ulonglong2 *>(gp->key + 2));
+            const uint64_t k4[kGroupSlots] = {a.x, a.y, b.x, b.y};
+            int found = -1;
+            bool stop = false;
+#pragma unroll
+            for (int i = 0; i < kGroupSlots; ++i) {
+                if (stop) continue;
+                if (k4[i] == key) {
+                    found = i;
+                    stop = true;
+                } else if (k4[i] == kEmptyKey) {
+                    stop = true;
+                }
+            }
+            if (stop) {
+                if (found >= 0) r = int(__ldg(&gp->row[found]));
+                break;
+            }
+            slot = (slot + kGroupSlots) & cap_mask;
+        }
+    }
+    if (r >= n_out) {
+        flag(d_status, LAT_ERR_BAD_MAP);
+        r = -1;
+    }
+    nbr[int64_t(k) * n_out + j] = r;
+    if (r >= 0) {
+        const int km = g.k3 - 1 - k;
+        nbr[int64_t(km) * n_out + r] = int32_t(j);
+        atomicOr(mask + j, 1u << k);
+        atomicOr(mask + r, 1u << km);
+    }
 }
 
 // Exclusive scan of the per-block hit counts of one offset (block k scans row k of
@@ -745,18 +797,17 @@ extern "C" lat_status lat_kmap_query(const void *table, size_t table_bytes, cons
     if (geom->mode == LAT_SUBM) {
         // the upper half of the table is filled by mirrored hits only
         const int centre = k3 / 2;
-        if (centre + 1 < k3)
-            LAT_CUDA_TRY(cudaMemsetAsync(map->nbr + int64_t(centre + 1) * n_out, 0xFF,
-                                         sizeof(int32_t) * size_t(k3 - 1 - centre) * n_out, s));
-        LAT_CUDA_TRY(cudaMemsetAsync(map->mask, 0, sizeof(uint32_t) * size_t(n_out), s));
-        kmap_probe_kernel<true><<<nblk, kQueryThreads, 0, s>>>(slots, cap_mask, oc, n_out, n_in, g, map->nbr,
-                                                               map->mask, w.keys, w.hist, w.ntile, w.block_counts,
-                                                               nblk, d_status);
+        kmap_subm_init_kernel<<<nblk, kQueryThreads, 0, s>>>(n_out, k3, map->nbr, map->mask);
         LAT_CUDA_TRY(cudaGetLastError());
+        if (centre > 0) {
+            kmap_probe_sym_kernel<<<dim3(unsigned(nblk), unsigned(centre)), kQueryThreads, 0, s>>>(
+                slots, cap_mask, oc, n_out, g, map->nbr, map->mask, d_status);
+            LAT_CUDA_TRY(cudaGetLastError());
+        }
         kmap_count_kernel<<<nblk, kQueryThreads, 0, s>>>(map->mask, n_out, k3, w.block_counts, nblk, w.keys, w.hist,
                                                           w.ntile);
     } else {
-        kmap_probe_kernel<false><<<nblk, kQueryThreads, 0, s>>>(slots, cap_mask, oc, n_out, n_in, g, map->nbr,
+        kmap_probe_kernel<<<nblk, kQueryThreads, 0, s>>>(slots, cap_mask, oc, n_out, n_in, g, map->nbr,
                                                                 map->mask, w.keys, w.hist, w.ntile, w.block_counts,
                                                                 nblk, d_status);
     }
