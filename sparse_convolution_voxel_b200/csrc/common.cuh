@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include <mutex>
+#include <utility>
 
 #include "lattice.h"
 
@@ -77,6 +78,19 @@ __device__ __forceinline__ int hash_find(const SlotGroup *__restrict__ groups, u
     return -1;
 }
 
+// Programmatic dependent launch.  Kernels started with launch_pdl may be
+// scheduled while the previous kernel on the stream is still running:
+// pdl_wait() blocks until that grid has completed and its memory is visible,
+// and must come before the first global access; pdl_trigger() lets the next
+// grid on the stream be scheduled now (its blocks then sit in their own
+// pdl_wait()).  Both are no-ops for a kernel launched the ordinary way.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_enter() {
+    pdl_wait();
+    pdl_trigger();
+}
+
 __device__ __forceinline__ void flag(int32_t *d_status, int32_t bits) {
     if (d_status) atomicOr(d_status, bits);
 }
@@ -117,6 +131,45 @@ inline int num_sms() {
     return n;
 }
 inline bool pow2(uint64_t v) { return v && !(v & (v - 1)); }
+
+// launch_pdl: launch with programmatic stream serialization: the kernel may be scheduled
+// as soon as the previous kernel on `s` has triggered (every kernel of the
+// library calls pdl_enter() first), so its launch latency overlaps that
+// kernel's tail instead of following it.  Ordering is unchanged: the kernel's
+// pdl_wait() returns only once the previous grid has completed.
+template <typename... P, typename... A>
+inline cudaError_t launch_pdl(void (*kern)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, A &&...args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
+}
+
+// Fills n 32-bit words at p with v: a kernel rather than cudaMemsetAsync, so
+// that it joins the programmatic launch chain of the kernels around it.
+template <int = 0>
+__global__ void __launch_bounds__(256) fill_u32_kernel(uint32_t *__restrict__ p, int64_t n, uint32_t v) {
+    pdl_enter();
+    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+    const int64_t i0 = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+    const int64_t n4 = reinterpret_cast<uintptr_t>(p) % 16 == 0 ? n / 4 : 0;
+    const uint4 v4 = make_uint4(v, v, v, v);
+    for (int64_t i = i0; i < n4; i += stride) reinterpret_cast<uint4 *>(p)[i] = v4;
+    for (int64_t i = 4 * n4 + i0; i < n; i += stride) p[i] = v;
+}
+inline cudaError_t fill_u32(void *p, int64_t n, uint32_t v, cudaStream_t s) {
+    if (n <= 0) return cudaSuccess;
+    const int64_t want = (n / 4 + 255) / 256 + 1, cap = int64_t(num_sms()) * 8;
+    return launch_pdl(fill_u32_kernel<0>, dim3(unsigned(want < cap ? want : cap)), dim3(256), 0, s,
+                      static_cast<uint32_t *>(p), n, v);
+}
 
 // A side stream for independent chains of small kernels inside one entry
 // point: fork() makes it wait for everything enqueued on `s` so far, join()

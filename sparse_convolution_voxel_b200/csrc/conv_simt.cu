@@ -78,6 +78,7 @@ template <typename T, bool WT>
 __global__ void __launch_bounds__(LAT_TILE_ROWS)
 conv_simt_kernel(const T *__restrict__ x, int cin, const T *__restrict__ w, int cout, MapView mv,
                  T *__restrict__ y, int32_t *d_status) {
+    pdl_enter();
     extern __shared__ float s_w[];  // [cin][kCoChunk]
     const int64_t t = blockIdx.x;
     const uint32_t tmask = mv.tile_mask_at(t);
@@ -151,6 +152,7 @@ conv_simt_kernel(const T *__restrict__ x, int cin, const T *__restrict__ w, int 
 // handles offset k (k3 <= 32): offset k's clamped pairs make ceil(P_k / chunk) units.
 __global__ void wgrad_units_kernel(const int64_t *__restrict__ pair_off, int k3, int64_t capacity, int chunk,
                                    int32_t *__restrict__ unit_base) {
+    pdl_enter();
     const int lane = threadIdx.x & 31;
     const int64_t P = min(pair_off[k3], capacity);
     const int64_t lo = lane < k3 ? min(pair_off[lane], capacity) : P;
@@ -184,6 +186,7 @@ wgrad_simt_kernel(const T *__restrict__ x, int cin, const T *__restrict__ dy, in
                   const int32_t *__restrict__ pair_in, const int32_t *__restrict__ pair_out, int64_t capacity, int k3,
                   int64_t n_in, int64_t n_out, const int32_t *__restrict__ unit_base, int chunk, float *__restrict__ partial,
                   int32_t *d_status) {
+    pdl_enter();
     __shared__ float s_part[kWgradWarps][kWgradSlice];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nelem = cin * cout;
@@ -262,6 +265,7 @@ wgrad_simt_kernel(const T *__restrict__ x, int cin, const T *__restrict__ dy, in
 
 __global__ void wgrad_reduce_kernel(const float *__restrict__ partial, const int32_t *__restrict__ unit_base, int k3,
                                     int nelem, float *__restrict__ dw) {
+    pdl_enter();
     const int k = blockIdx.y;
     const int el = blockIdx.x * blockDim.x + threadIdx.x;
     if (k >= k3 || el >= nelem) return;
@@ -288,11 +292,13 @@ lat_status launch_conv_simt(const void *x, int cin, const void *w, int cout, con
     if (mv.ntiles >= (int64_t(1) << 31)) return LAT_ERR_UNSUPPORTED;
     const size_t smem = sizeof(float) * size_t(cin) * kCoChunk;
     if (wt)
-        conv_simt_kernel<T, true><<<unsigned(mv.ntiles), LAT_TILE_ROWS, smem, s>>>(
-            static_cast<const T *>(x), cin, static_cast<const T *>(w), cout, mv, static_cast<T *>(y), d_status);
+        LAT_CUDA_TRY(launch_pdl(conv_simt_kernel<T, true>, dim3(unsigned(mv.ntiles)), dim3(LAT_TILE_ROWS), smem, s,
+                                static_cast<const T *>(x), cin, static_cast<const T *>(w), cout, mv,
+                                static_cast<T *>(y), d_status));
     else
-        conv_simt_kernel<T, false><<<unsigned(mv.ntiles), LAT_TILE_ROWS, smem, s>>>(
-            static_cast<const T *>(x), cin, static_cast<const T *>(w), cout, mv, static_cast<T *>(y), d_status);
+        LAT_CUDA_TRY(launch_pdl(conv_simt_kernel<T, false>, dim3(unsigned(mv.ntiles)), dim3(LAT_TILE_ROWS), smem, s,
+                                static_cast<const T *>(x), cin, static_cast<const T *>(w), cout, mv,
+                                static_cast<T *>(y), d_status));
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }
@@ -311,20 +317,22 @@ lat_status launch_wgrad_simt(const void *x, int cin, const void *dy, int cout, c
     Carver cv(ws);
     int32_t *unit_base = cv.take<int32_t>(size_t(map->k3) + 1);
     float *partial = cv.take<float>(size_t(units_max) * cin * cout);
-    wgrad_units_kernel<<<1, 32, 0, s>>>(map->pair_off, map->k3, map->pair_capacity, kWgradChunkSimt, unit_base);
+    LAT_CUDA_TRY(launch_pdl(wgrad_units_kernel, dim3(1), dim3(32), 0, s, map->pair_off, map->k3, map->pair_capacity,
+                            kWgradChunkSimt, unit_base));
     LAT_CUDA_TRY(cudaGetLastError());
     const int64_t nslices = (int64_t(cin) * cout + kWgradSlice - 1) / kWgradSlice;
     const int64_t parts = nslices >= kWgradWarps ? 1 : (kWgradWarps % nslices == 0 ? kWgradWarps / nslices : 1);
     const int64_t per_block = kWgradWarps / parts;
     const int64_t grid = units_max * ((nslices + per_block - 1) / per_block);
     if (grid >= (int64_t(1) << 31)) return LAT_ERR_UNSUPPORTED;
-    wgrad_simt_kernel<T><<<unsigned(grid), kWgradWarps * 32, 0, s>>>(
-        static_cast<const T *>(x), cin, static_cast<const T *>(dy), cout, map->pair_off, map->pair_in, map->pair_out,
-        map->pair_capacity, map->k3, map->n_in, map->n_out, unit_base, kWgradChunkSimt, partial, d_status);
+    LAT_CUDA_TRY(launch_pdl(wgrad_simt_kernel<T>, dim3(unsigned(grid)), dim3(kWgradWarps * 32), 0, s,
+                            static_cast<const T *>(x), cin, static_cast<const T *>(dy), cout, map->pair_off,
+                            map->pair_in, map->pair_out, map->pair_capacity, map->k3, map->n_in, map->n_out, unit_base,
+                            kWgradChunkSimt, partial, d_status));
     LAT_CUDA_TRY(cudaGetLastError());
     const int nelem = cin * cout;
     dim3 rg((nelem + 255) / 256, map->k3);
-    wgrad_reduce_kernel<<<rg, 256, 0, s>>>(partial, unit_base, map->k3, nelem, dw);
+    LAT_CUDA_TRY(launch_pdl(wgrad_reduce_kernel, dim3(rg), dim3(256), 0, s, partial, unit_base, map->k3, nelem, dw));
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }

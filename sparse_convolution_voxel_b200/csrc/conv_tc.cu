@@ -118,6 +118,7 @@ template <typename T, int KC, int N, bool BMN>
 __global__ void __launch_bounds__(kThreads, 2)
 conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x, MapView mv, T *__restrict__ y,
                int32_t *tile_counter, int32_t *d_status) {
+    pdl_enter();
     using C = Cfg<N>;
     constexpr int NS = C::kStages;
     constexpr int KBLK = KC / 64;
@@ -532,9 +533,9 @@ static lat_status launch(const void *x, const void *w, int k3, const MapView &mv
     auto kern = conv_tc_kernel<T, KC, N, BMN>;
     const int64_t grid = std::min<int64_t>(mv.ntiles, GridCache<KernelTag<T, KC, N, BMN>>::get(kern, C::kSmem, int(C::kTmemCols), 2));
     if (grid <= 0) return LAT_ERR_CUDA;
-    LAT_CUDA_TRY(cudaMemsetAsync(counter, 0, sizeof(int32_t), s));
-    kern<<<unsigned(grid), kThreads, C::kSmem, s>>>(map, static_cast<const T *>(x), mv, static_cast<T *>(y),
-                                                    counter, d_status);
+    LAT_CUDA_TRY(fill_u32(counter, 1, 0u, s));
+    LAT_CUDA_TRY(launch_pdl(kern, dim3(unsigned(grid)), dim3(kThreads), C::kSmem, s, map, static_cast<const T *>(x),
+                            mv, static_cast<T *>(y), counter, d_status));
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }

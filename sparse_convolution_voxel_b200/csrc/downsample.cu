@@ -44,6 +44,7 @@ constexpr int kMaxBitmapBits = 30;
 __global__ void __launch_bounds__(256)
 down_candidates_kernel(const int4 *__restrict__ coords, int64_t n, DownGeom g, uint64_t *__restrict__ keys,
                        int *__restrict__ range, int32_t *d_status) {
+    pdl_enter();
     int mn[4] = {INT_MAX, INT_MAX, INT_MAX, INT_MAX}, mx[4] = {INT_MIN, INT_MIN, INT_MIN, INT_MIN};
     const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
     if (i < n) {
@@ -141,6 +142,7 @@ down_candidates_kernel(const int4 *__restrict__ coords, int64_t n, DownGeom g, u
 }
 
 __global__ void range_init_kernel(int *range) {
+    pdl_enter();
     if (threadIdx.x < 4) range[threadIdx.x] = INT_MAX;
     else if (threadIdx.x < 8) range[threadIdx.x] = INT_MIN;
 }
@@ -199,6 +201,7 @@ __device__ __forceinline__ Plan make_plan(const int *__restrict__ range, int64_t
 
 __global__ void __launch_bounds__(256)
 bitmap_zero_kernel(const int *__restrict__ range, int64_t budget_bits, uint4 *__restrict__ bitmap) {
+    pdl_enter();
     const Plan p = make_plan(range, budget_bits);
     const int64_t n4 = p.ngroups * 8;  // 32 words per group
     for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < n4; e += int64_t(gridDim.x) * blockDim.x)
@@ -208,6 +211,7 @@ bitmap_zero_kernel(const int *__restrict__ range, int64_t budget_bits, uint4 *__
 __global__ void __launch_bounds__(256)
 bitmap_mark_kernel(const uint64_t *__restrict__ keys, int64_t items, const int *__restrict__ range,
                    int64_t budget_bits, uint32_t *__restrict__ bitmap) {
+    pdl_enter();
     const int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
     if (e >= items) return;
     const Plan p = make_plan(range, budget_bits);
@@ -222,6 +226,7 @@ bitmap_mark_kernel(const uint64_t *__restrict__ keys, int64_t items, const int *
 __global__ void __launch_bounds__(256)
 bitmap_count_kernel(const uint32_t *__restrict__ bitmap, const int *__restrict__ range, int64_t budget_bits,
                     int32_t *__restrict__ grp_cnt, int32_t *__restrict__ blk_cnt) {
+    pdl_enter();
     __shared__ int s_warp[8];
     const Plan p = make_plan(range, budget_bits);
     if (int64_t(blockIdx.x) * 256 >= p.ngroups) return;
@@ -252,6 +257,7 @@ bitmap_count_kernel(const uint32_t *__restrict__ bitmap, const int *__restrict__
 __global__ void __launch_bounds__(1024)
 bitmap_blockscan_kernel(const int *__restrict__ range, int64_t budget_bits, const int32_t *__restrict__ blk_cnt,
                         int64_t *__restrict__ blk_off, int64_t *__restrict__ n_out_dev) {
+    pdl_enter();
     __shared__ int64_t s_warp[32];
     const Plan p = make_plan(range, budget_bits);
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
@@ -292,6 +298,7 @@ __global__ void __launch_bounds__(256)
 bitmap_emit_kernel(const uint32_t *__restrict__ bitmap, const int *__restrict__ range, int64_t budget_bits,
                    const int32_t *__restrict__ grp_cnt, const int64_t *__restrict__ blk_off,
                    int64_t *__restrict__ grp_off, int4 *__restrict__ out, int64_t capacity) {
+    pdl_enter();
     __shared__ int s_warp[8];
     const Plan p = make_plan(range, budget_bits);
     if (int64_t(blockIdx.x) * 256 >= p.ngroups) return;
@@ -337,6 +344,7 @@ __global__ void __launch_bounds__(256)
 bitmap_parent_kernel(const uint64_t *__restrict__ keys, int64_t n, const int *__restrict__ range,
                      int64_t budget_bits, const uint32_t *__restrict__ bitmap, const int64_t *__restrict__ grp_off,
                      int32_t *__restrict__ parent) {
+    pdl_enter();
     const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
     if (i >= n) return;
     const uint64_t key = keys[i];
@@ -368,6 +376,7 @@ bitmap_parent_kernel(const uint64_t *__restrict__ keys, int64_t n, const int *__
 __global__ void __launch_bounds__(256)
 down_unpack_kernel(const uint64_t *__restrict__ uniq, const int *__restrict__ n_uniq, int4 *__restrict__ out,
                    int64_t capacity, int64_t *__restrict__ n_out_dev) {
+    pdl_enter();
     const int64_t r = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
     int64_t m = *n_uniq;
     if (m > 0 && uniq[m - 1] == kEmptyKey) --m;
@@ -382,6 +391,7 @@ down_unpack_kernel(const uint64_t *__restrict__ uniq, const int *__restrict__ n_
 __global__ void __launch_bounds__(256)
 sorted_parent_kernel(const uint64_t *__restrict__ keys, int64_t n, const uint64_t *__restrict__ uniq,
                      const int64_t *__restrict__ n_out_dev, int32_t *__restrict__ parent) {
+    pdl_enter();
     const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
     if (i >= n) return;
     const uint64_t key = keys[i];
@@ -512,27 +522,32 @@ static lat_status enqueue_bitmap_path(const int32_t *coords, int64_t n_in, const
                                       int32_t *out_coords, int64_t out_capacity, int32_t *parent, const DownWs &w,
                                       int32_t *d_status, cudaStream_t s) {
     const unsigned in_blocks = unsigned((n_in + 255) / 256), item_blocks = unsigned((items + 255) / 256);
-    range_init_kernel<<<1, 32, 0, s>>>(w.range);
+    LAT_CUDA_TRY(launch_pdl(range_init_kernel, dim3(1), dim3(32), 0, s, w.range));
     LAT_CUDA_TRY(cudaGetLastError());
-    down_candidates_kernel<<<in_blocks, 256, 0, s>>>(reinterpret_cast<const int4 *>(coords), n_in, g, w.keys, w.range,
-                                                     d_status);
+    LAT_CUDA_TRY(launch_pdl(down_candidates_kernel, dim3(in_blocks), dim3(256), 0, s,
+                            reinterpret_cast<const int4 *>(coords), n_in, g, w.keys, w.range, d_status));
     LAT_CUDA_TRY(cudaGetLastError());
     const int64_t budget = bitmap_budget_bits(items);
     const unsigned gblocks = unsigned((w.max_groups + 255) / 256);
     const unsigned zblocks = unsigned(std::min<int64_t>((w.max_groups * 8 + 255) / 256, int64_t(num_sms()) * 8));
-    bitmap_zero_kernel<<<zblocks, 256, 0, s>>>(w.range, budget, reinterpret_cast<uint4 *>(w.bitmap));
+    LAT_CUDA_TRY(launch_pdl(bitmap_zero_kernel, dim3(zblocks), dim3(256), 0, s, w.range, budget,
+                            reinterpret_cast<uint4 *>(w.bitmap)));
     LAT_CUDA_TRY(cudaGetLastError());
-    bitmap_mark_kernel<<<item_blocks, 256, 0, s>>>(w.keys, items, w.range, budget, w.bitmap);
+    LAT_CUDA_TRY(launch_pdl(bitmap_mark_kernel, dim3(item_blocks), dim3(256), 0, s, w.keys, items, w.range, budget,
+                            w.bitmap));
     LAT_CUDA_TRY(cudaGetLastError());
-    bitmap_count_kernel<<<gblocks, 256, 0, s>>>(w.bitmap, w.range, budget, w.grp_cnt, w.blk_cnt);
+    LAT_CUDA_TRY(launch_pdl(bitmap_count_kernel, dim3(gblocks), dim3(256), 0, s, w.bitmap, w.range, budget, w.grp_cnt,
+                            w.blk_cnt));
     LAT_CUDA_TRY(cudaGetLastError());
-    bitmap_blockscan_kernel<<<1, 1024, 0, s>>>(w.range, budget, w.blk_cnt, w.blk_off, w.n_out_dev);
+    LAT_CUDA_TRY(launch_pdl(bitmap_blockscan_kernel, dim3(1), dim3(1024), 0, s, w.range, budget, w.blk_cnt, w.blk_off,
+                            w.n_out_dev));
     LAT_CUDA_TRY(cudaGetLastError());
-    bitmap_emit_kernel<<<gblocks, 256, 0, s>>>(w.bitmap, w.range, budget, w.grp_cnt, w.blk_off, w.grp_off,
-                                               reinterpret_cast<int4 *>(out_coords), out_capacity);
+    LAT_CUDA_TRY(launch_pdl(bitmap_emit_kernel, dim3(gblocks), dim3(256), 0, s, w.bitmap, w.range, budget, w.grp_cnt,
+                            w.blk_off, w.grp_off, reinterpret_cast<int4 *>(out_coords), out_capacity));
     LAT_CUDA_TRY(cudaGetLastError());
     if (parent) {
-        bitmap_parent_kernel<<<in_blocks, 256, 0, s>>>(w.keys, n_in, w.range, budget, w.bitmap, w.grp_off, parent);
+        LAT_CUDA_TRY(launch_pdl(bitmap_parent_kernel, dim3(in_blocks), dim3(256), 0, s, w.keys, n_in, w.range, budget,
+                                w.bitmap, w.grp_off, parent));
         LAT_CUDA_TRY(cudaGetLastError());
     }
     return LAT_OK;
@@ -566,11 +581,12 @@ static lat_status support_blocking(const int32_t *coords, int64_t n_in, const la
         LAT_CUDA_TRY(cub::DeviceRadixSort::SortKeys(w.sort_tmp, b, w.keys, w.sorted, int(items), 0, 64, s));
         b = w.sel_bytes;
         LAT_CUDA_TRY(cub::DeviceSelect::Unique(w.sel_tmp, b, w.sorted, w.uniq, w.n_uniq, int(items), s));
-        down_unpack_kernel<<<item_blocks, 256, 0, s>>>(w.uniq, w.n_uniq, reinterpret_cast<int4 *>(out_coords),
-                                                       out_capacity, w.n_out_dev);
+        LAT_CUDA_TRY(launch_pdl(down_unpack_kernel, dim3(item_blocks), dim3(256), 0, s, w.uniq, w.n_uniq,
+                                reinterpret_cast<int4 *>(out_coords), out_capacity, w.n_out_dev));
         LAT_CUDA_TRY(cudaGetLastError());
         if (parent) {
-            sorted_parent_kernel<<<in_blocks, 256, 0, s>>>(w.keys, n_in, w.uniq, w.n_out_dev, parent);
+            LAT_CUDA_TRY(launch_pdl(sorted_parent_kernel, dim3(in_blocks), dim3(256), 0, s, w.keys, n_in, w.uniq,
+                                    w.n_out_dev, parent));
             LAT_CUDA_TRY(cudaGetLastError());
         }
         LAT_CUDA_TRY(cudaMemcpyAsync(&m, w.n_out_dev, sizeof(int64_t), cudaMemcpyDeviceToHost, s));

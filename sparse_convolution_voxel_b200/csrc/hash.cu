@@ -15,6 +15,7 @@ namespace lat {
 __global__ void __launch_bounds__(256) hash_insert_kernel(const int4 *__restrict__ coords, int64_t n,
                                                           SlotGroup *__restrict__ groups, uint32_t cap_mask,
                                                           int32_t *d_status) {
+    pdl_enter();
     int32_t bad = 0;
     for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n;
          i += int64_t(gridDim.x) * blockDim.x) {
@@ -68,8 +69,9 @@ extern "C" lat_status lat_hash_build(const int32_t *coords, int64_t n, void *tab
     if (n == 0) return LAT_OK;
     const int threads = 256;
     const int64_t blocks = (n + threads - 1) / threads;
-    hash_insert_kernel<<<unsigned(blocks), threads, 0, s>>>(reinterpret_cast<const int4 *>(coords), n,
-                                                             static_cast<SlotGroup *>(table), uint32_t(cap - 1), d_status);
+    LAT_CUDA_TRY(launch_pdl(hash_insert_kernel, dim3(unsigned(blocks)), dim3(threads), 0, s,
+                            reinterpret_cast<const int4 *>(coords), n, static_cast<SlotGroup *>(table),
+                            uint32_t(cap - 1), d_status));
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }

@@ -118,6 +118,7 @@ kmap_probe_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const
                   int64_t n_out, int64_t n_in, Geom g, int32_t *__restrict__ nbr, uint32_t *__restrict__ mask,
                   uint32_t *__restrict__ keys, int32_t *__restrict__ hist, int ntile, int32_t *__restrict__ block_counts,
                   int nblk, int32_t *d_status) {
+    pdl_enter();
     __shared__ int s_cnt[32];
     if (threadIdx.x < 32) s_cnt[threadIdx.x] = 0;
     __syncthreads();
@@ -223,6 +224,7 @@ kmap_probe_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const
 // coalesced.
 __global__ void __launch_bounds__(kQueryThreads)
 kmap_subm_init_kernel(int64_t n_out, int k3, int32_t *__restrict__ nbr, uint32_t *__restrict__ mask) {
+    pdl_enter();
     const int64_t j = blockIdx.x * int64_t(kQueryThreads) + threadIdx.x;
     if (j >= n_out) return;
     const int centre = k3 / 2;
@@ -244,6 +246,7 @@ __global__ void __launch_bounds__(kQueryThreads)
 kmap_probe_sym_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const int4 *__restrict__ out_coords,
                       int64_t n_out, Geom g, int32_t *__restrict__ nbr, uint32_t *__restrict__ mask,
                       int32_t *d_status) {
+    pdl_enter();
     const int k = blockIdx.y;
     const int64_t j = blockIdx.x * int64_t(kQueryThreads) + threadIdx.x;
     if (j >= n_out) return;
@@ -303,6 +306,7 @@ kmap_probe_sym_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, c
 __global__ void __launch_bounds__(1024)
 kmap_scan_kernel(const int32_t *__restrict__ block_counts, int64_t *__restrict__ block_offsets, int nblk,
                  int64_t *__restrict__ k_total) {
+    pdl_enter();
     __shared__ int64_t s_warp[32];
     __shared__ int64_t s_carry;
     const int k = blockIdx.x;
@@ -348,6 +352,7 @@ kmap_emit_kernel(const int32_t *__restrict__ nbr, const uint32_t *__restrict__ m
                  const int64_t *__restrict__ block_offsets, const int64_t *__restrict__ k_total, int nblk,
                  int32_t *__restrict__ pair_in, int32_t *__restrict__ pair_out, int64_t capacity,
                  int64_t *__restrict__ pair_off, int32_t *d_status) {
+    pdl_enter();
     __shared__ int s_warp[32][kQueryWarps];  // per (offset, warp): hits, then the exclusive prefix over warps
     __shared__ int64_t s_base[32];           // first pair of (offset, this block)
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -404,6 +409,7 @@ kmap_emit_kernel(const int32_t *__restrict__ nbr, const uint32_t *__restrict__ m
 // hist[d * ntile + 0 .. ntile), and the digit's total into totals[d].
 __global__ void __launch_bounds__(256)
 sort_rowscan_kernel(int32_t *__restrict__ hist, int ntile, int32_t *__restrict__ totals) {
+    pdl_enter();
     __shared__ int s_warp[8];
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
     int32_t *row = hist + int64_t(blockIdx.x) * ntile;
@@ -458,6 +464,7 @@ sort_scatter_kernel(const uint32_t *__restrict__ keys_in, const int32_t *__restr
                     uint32_t *__restrict__ keys_out,
                     int32_t *__restrict__ vals_out, int32_t *__restrict__ hist_next,
                     const uint32_t *__restrict__ mask, uint32_t *__restrict__ tile_mask, PairOut po) {
+    pdl_enter();
     __shared__ int s_cnt[2][kSortWarps][256];
     __shared__ int s_run[256];
     __shared__ int s_wsum[kSortWarps];
@@ -564,6 +571,7 @@ sort_scatter_kernel(const uint32_t *__restrict__ keys_in, const int32_t *__restr
 __global__ void __launch_bounds__(kQueryThreads)
 kmap_count_kernel(const uint32_t *__restrict__ mask, int64_t n_out, int k3, int32_t *__restrict__ block_counts,
                   int nblk, uint32_t *__restrict__ keys, int32_t *__restrict__ hist, int ntile) {
+    pdl_enter();
     __shared__ int s_cnt[32];
     if (threadIdx.x < 32) s_cnt[threadIdx.x] = 0;
     __syncthreads();
@@ -591,6 +599,7 @@ parent_maps_kernel(const int4 *__restrict__ fine, const int32_t *__restrict__ pa
                    int64_t n_coarse, int s0, int s1, int s2, int k3, int32_t *__restrict__ up_nbr,
                    uint32_t *__restrict__ up_mask, int32_t *__restrict__ down_nbr, uint32_t *__restrict__ down_mask,
                    uint32_t *__restrict__ up_keys, int32_t *__restrict__ up_hist, int up_ntile, int32_t *d_status) {
+    pdl_enter();
     const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
     const bool live = i < n_fine;
     uint32_t m = 0;
@@ -666,11 +675,12 @@ static lat_status finish_kmap(lat_kmap *map, int k3, int nblk, KmapWs &w, int32_
         LAT_CUDA_TRY(side_fork(*side, s));
         ps = side->side;
     }
-    kmap_scan_kernel<<<k3, 1024, 0, ps>>>(w.block_counts, w.block_offsets, nblk, w.k_total);
+    LAT_CUDA_TRY(launch_pdl(kmap_scan_kernel, dim3(k3), dim3(1024), 0, ps, w.block_counts, w.block_offsets, nblk,
+                            w.k_total));
     LAT_CUDA_TRY(cudaGetLastError());
-    kmap_emit_kernel<<<nblk, kQueryThreads, 0, ps>>>(map->nbr, map->mask, n_out, k3, w.block_offsets, w.k_total,
-                                                      nblk, map->pair_in, map->pair_out, map->pair_capacity,
-                                                      map->pair_off, d_status);
+    LAT_CUDA_TRY(launch_pdl(kmap_emit_kernel, dim3(nblk), dim3(kQueryThreads), 0, ps, map->nbr, map->mask, n_out, k3,
+                            w.block_offsets, w.k_total, nblk, map->pair_in, map->pair_out, map->pair_capacity,
+                            map->pair_off, d_status));
     LAT_CUDA_TRY(cudaGetLastError());
     const lat_status st = sort_rows(map, k3, w, s);
     if (side) LAT_CUDA_TRY(side_join(*side, s));
@@ -681,27 +691,27 @@ static lat_status finish_kmap(lat_kmap *map, int k3, int nblk, KmapWs &w, int32_
 static lat_status sort_rows(lat_kmap *map, int k3, KmapWs &w, cudaStream_t s) {
     const int64_t n_out = map->n_out;
     const int64_t ntiles = (n_out + LAT_TILE_ROWS - 1) / LAT_TILE_ROWS;
-    LAT_CUDA_TRY(cudaMemsetAsync(map->tile_mask, 0, sizeof(uint32_t) * size_t(ntiles), s));
+    LAT_CUDA_TRY(fill_u32(map->tile_mask, ntiles, 0u, s));
     const int64_t hsize = 256 * int64_t(w.ntile);
     int32_t *h1 = w.hist, *h2 = w.hist + hsize;
     int32_t *t1 = w.totals, *t2 = w.totals + 256;
-    sort_rowscan_kernel<<<256, 256, 0, s>>>(h1, w.ntile, t1);
+    LAT_CUDA_TRY(launch_pdl(sort_rowscan_kernel, dim3(256), dim3(256), 0, s, h1, w.ntile, t1));
     LAT_CUDA_TRY(cudaGetLastError());
     if (group_key_bits(k3) <= 8) {
-        sort_scatter_kernel<true><<<w.ntile, kSortThreads, 0, s>>>(w.keys, nullptr, n_out, 0, h1, t1, w.ntile,
-                                                                    nullptr, map->perm, nullptr, map->mask,
-                                                                    map->tile_mask, PairOut{});
+        LAT_CUDA_TRY(launch_pdl(sort_scatter_kernel<true>, dim3(w.ntile), dim3(kSortThreads), 0, s, w.keys, nullptr,
+                                n_out, 0, h1, t1, w.ntile, nullptr, map->perm, nullptr, map->mask, map->tile_mask,
+                                PairOut{}));
         LAT_CUDA_TRY(cudaGetLastError());
         return LAT_OK;
     }
-    sort_scatter_kernel<false><<<w.ntile, kSortThreads, 0, s>>>(w.keys, nullptr, n_out, 0, h1, t1, w.ntile,
-                                                                 w.keys_tmp, w.vals_tmp, h2, nullptr, nullptr, PairOut{});
+    LAT_CUDA_TRY(launch_pdl(sort_scatter_kernel<false>, dim3(w.ntile), dim3(kSortThreads), 0, s, w.keys, nullptr,
+                            n_out, 0, h1, t1, w.ntile, w.keys_tmp, w.vals_tmp, h2, nullptr, nullptr, PairOut{}));
     LAT_CUDA_TRY(cudaGetLastError());
-    sort_rowscan_kernel<<<256, 256, 0, s>>>(h2, w.ntile, t2);
+    LAT_CUDA_TRY(launch_pdl(sort_rowscan_kernel, dim3(256), dim3(256), 0, s, h2, w.ntile, t2));
     LAT_CUDA_TRY(cudaGetLastError());
-    sort_scatter_kernel<true><<<w.ntile, kSortThreads, 0, s>>>(w.keys_tmp, w.vals_tmp, n_out, 8, h2, t2, w.ntile,
-                                                                nullptr, map->perm, nullptr, map->mask,
-                                                                map->tile_mask, PairOut{});
+    LAT_CUDA_TRY(launch_pdl(sort_scatter_kernel<true>, dim3(w.ntile), dim3(kSortThreads), 0, s, w.keys_tmp, w.vals_tmp,
+                            n_out, 8, h2, t2, w.ntile, nullptr, map->perm, nullptr, map->mask, map->tile_mask,
+                            PairOut{}));
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }
@@ -790,26 +800,26 @@ extern "C" lat_status lat_kmap_query(const void *table, size_t table_bytes, cons
                 g.delta[k] = dx * (1ll << 32) + dy * (1ll << 16) + dz;
             }
     const int nblk = int((n_out + kQueryThreads - 1) / kQueryThreads);
-    LAT_CUDA_TRY(cudaMemsetAsync(w.hist, 0, w.hist_bytes, s));
+    LAT_CUDA_TRY(fill_u32(w.hist, int64_t(w.hist_bytes / 4), 0u, s));
     const uint32_t cap_mask = uint32_t(table_bytes / kSlotBytes - 1);
     const SlotGroup *slots = static_cast<const SlotGroup *>(table);
     const int4 *oc = reinterpret_cast<const int4 *>(out_coords);
     if (geom->mode == LAT_SUBM) {
         // the upper half of the table is filled by mirrored hits only
         const int centre = k3 / 2;
-        kmap_subm_init_kernel<<<nblk, kQueryThreads, 0, s>>>(n_out, k3, map->nbr, map->mask);
+        LAT_CUDA_TRY(launch_pdl(kmap_subm_init_kernel, dim3(nblk), dim3(kQueryThreads), 0, s, n_out, k3, map->nbr,
+                                map->mask));
         LAT_CUDA_TRY(cudaGetLastError());
         if (centre > 0) {
-            kmap_probe_sym_kernel<<<dim3(unsigned(nblk), unsigned(centre)), kQueryThreads, 0, s>>>(
-                slots, cap_mask, oc, n_out, g, map->nbr, map->mask, d_status);
+            LAT_CUDA_TRY(launch_pdl(kmap_probe_sym_kernel, dim3(unsigned(nblk), unsigned(centre)), dim3(kQueryThreads),
+                                    0, s, slots, cap_mask, oc, n_out, g, map->nbr, map->mask, d_status));
             LAT_CUDA_TRY(cudaGetLastError());
         }
-        kmap_count_kernel<<<nblk, kQueryThreads, 0, s>>>(map->mask, n_out, k3, w.block_counts, nblk, w.keys, w.hist,
-                                                          w.ntile);
+        LAT_CUDA_TRY(launch_pdl(kmap_count_kernel, dim3(nblk), dim3(kQueryThreads), 0, s, map->mask, n_out, k3,
+                                w.block_counts, nblk, w.keys, w.hist, w.ntile));
     } else {
-        kmap_probe_kernel<<<nblk, kQueryThreads, 0, s>>>(slots, cap_mask, oc, n_out, n_in, g, map->nbr,
-                                                                map->mask, w.keys, w.hist, w.ntile, w.block_counts,
-                                                                nblk, d_status);
+        LAT_CUDA_TRY(launch_pdl(kmap_probe_kernel, dim3(nblk), dim3(kQueryThreads), 0, s, slots, cap_mask, oc, n_out,
+                                n_in, g, map->nbr, map->mask, w.keys, w.hist, w.ntile, w.block_counts, nblk, d_status));
     }
     LAT_CUDA_TRY(cudaGetLastError());
     SideStream *side = nullptr;
@@ -846,8 +856,8 @@ extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int
     if (down) {
         down->mode = LAT_STRIDED;
         if (n_coarse > 0) {
-            LAT_CUDA_TRY(cudaMemsetAsync(down->nbr, 0xFF, sizeof(int32_t) * size_t(k3) * n_coarse, s));
-            LAT_CUDA_TRY(cudaMemsetAsync(down->mask, 0, sizeof(uint32_t) * size_t(n_coarse), s));
+            LAT_CUDA_TRY(fill_u32(down->nbr, int64_t(k3) * n_coarse, ~0u, s));
+            LAT_CUDA_TRY(fill_u32(down->mask, n_coarse, 0u, s));
         }
     }
     if (up) up->mode = LAT_TRANSPOSED;
@@ -856,12 +866,13 @@ extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int
     // transposed map with K^3 <= 8: every fine row has one neighbour (its parent)
     // and its key is the one-hot mask, so the row sort alone yields the pairs
     const bool up_direct = up && n_fine > 0 && group_key_bits(k3) <= 8;
-    if (up_direct) LAT_CUDA_TRY(cudaMemsetAsync(w_up.hist, 0, w_up.hist_bytes, s));
+    if (up_direct) LAT_CUDA_TRY(fill_u32(w_up.hist, int64_t(w_up.hist_bytes / 4), 0u, s));
     if (n_fine > 0) {
-        parent_maps_kernel<<<unsigned((n_fine + 255) / 256), 256, 0, s>>>(
-            reinterpret_cast<const int4 *>(fine_coords), parent, n_fine, n_coarse, geom->stride[0], geom->stride[1],
-            geom->stride[2], k3, up ? up->nbr : nullptr, up ? up->mask : nullptr, down ? down->nbr : nullptr,
-            down ? down->mask : nullptr, up_direct ? w_up.keys : nullptr, w_up.hist, w_up.ntile, d_status);
+        LAT_CUDA_TRY(launch_pdl(parent_maps_kernel, dim3(unsigned((n_fine + 255) / 256)), dim3(256), 0, s,
+                                reinterpret_cast<const int4 *>(fine_coords), parent, n_fine, n_coarse, geom->stride[0],
+                                geom->stride[1], geom->stride[2], k3, up ? up->nbr : nullptr, up ? up->mask : nullptr,
+                                down ? down->nbr : nullptr, down ? down->mask : nullptr,
+                                up_direct ? w_up.keys : nullptr, w_up.hist, w_up.ntile, d_status));
         LAT_CUDA_TRY(cudaGetLastError());
     }
     // the two maps are independent once the parent scatter is done: the
@@ -882,20 +893,20 @@ extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int
         KmapWs &w = map == down ? w_down : w_up;
         if (map == up && up_direct) {
             const int64_t ntiles = (map->n_out + LAT_TILE_ROWS - 1) / LAT_TILE_ROWS;
-            LAT_CUDA_TRY(cudaMemsetAsync(map->tile_mask, 0, sizeof(uint32_t) * size_t(ntiles), s));
-            sort_rowscan_kernel<<<256, 256, 0, s>>>(w.hist, w.ntile, w.totals);
+            LAT_CUDA_TRY(fill_u32(map->tile_mask, ntiles, 0u, s));
+            LAT_CUDA_TRY(launch_pdl(sort_rowscan_kernel, dim3(256), dim3(256), 0, s, w.hist, w.ntile, w.totals));
             LAT_CUDA_TRY(cudaGetLastError());
             const PairOut po{parent, map->pair_in, map->pair_out, map->pair_capacity, map->pair_off, k3, d_status};
-            sort_scatter_kernel<true><<<w.ntile, kSortThreads, 0, s>>>(w.keys, nullptr, map->n_out, 0, w.hist,
-                                                                        w.totals, w.ntile, nullptr, map->perm, nullptr,
-                                                                        map->mask, map->tile_mask, po);
+            LAT_CUDA_TRY(launch_pdl(sort_scatter_kernel<true>, dim3(w.ntile), dim3(kSortThreads), 0, s, w.keys,
+                                    nullptr, map->n_out, 0, w.hist, w.totals, w.ntile, nullptr, map->perm, nullptr,
+                                    map->mask, map->tile_mask, po));
             LAT_CUDA_TRY(cudaGetLastError());
             continue;
         }
         const int nblk = int((map->n_out + kQueryThreads - 1) / kQueryThreads);
-        LAT_CUDA_TRY(cudaMemsetAsync(w.hist, 0, w.hist_bytes, s));
-        kmap_count_kernel<<<nblk, kQueryThreads, 0, s>>>(map->mask, map->n_out, k3, w.block_counts, nblk, w.keys,
-                                                          w.hist, w.ntile);
+        LAT_CUDA_TRY(fill_u32(w.hist, int64_t(w.hist_bytes / 4), 0u, s));
+        LAT_CUDA_TRY(launch_pdl(kmap_count_kernel, dim3(nblk), dim3(kQueryThreads), 0, s, map->mask, map->n_out, k3,
+                                w.block_counts, nblk, w.keys, w.hist, w.ntile));
         LAT_CUDA_TRY(cudaGetLastError());
         const lat_status st = finish_kmap(map, k3, nblk, w, d_status, s, nullptr);
         if (st != LAT_OK) return st;

@@ -58,6 +58,7 @@ template <typename T, bool MAX>
 __global__ void __launch_bounds__(256)
 pool_kernel(const T *__restrict__ x, int c, const int32_t *__restrict__ nbr, const uint32_t *__restrict__ mask,
             int k3, int64_t n_in, int64_t n_out, T *__restrict__ y, int32_t *d_status) {
+    pdl_enter();
     const int groups = c / 8;
     const int64_t gid = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
     const int64_t j = gid / groups;
@@ -116,6 +117,7 @@ template <typename T>
 __global__ void __launch_bounds__(256)
 dense_scatter_kernel(const int4 *__restrict__ coords, int64_t n, const T *__restrict__ feats, int c, Box bx,
                      T *__restrict__ out, int32_t *d_status) {
+    pdl_enter();
     const int groups = c / 8;
     const int64_t gid = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
     const int64_t i = gid / groups;
@@ -141,11 +143,11 @@ static lat_status launch_pool(const void *x, int c, const lat_kmap *map, int op,
     if (threads == 0) return LAT_OK;
     const unsigned blocks = unsigned((threads + 255) / 256);
     if (op == LAT_POOL_MAX)
-        pool_kernel<T, true><<<blocks, 256, 0, s>>>(static_cast<const T *>(x), c, map->nbr, map->mask, map->k3, map->n_in,
-                                                    map->n_out, static_cast<T *>(y), d_status);
+        LAT_CUDA_TRY(launch_pdl(pool_kernel<T, true>, dim3(blocks), dim3(256), 0, s, static_cast<const T *>(x), c,
+                                map->nbr, map->mask, map->k3, map->n_in, map->n_out, static_cast<T *>(y), d_status));
     else
-        pool_kernel<T, false><<<blocks, 256, 0, s>>>(static_cast<const T *>(x), c, map->nbr, map->mask, map->k3, map->n_in,
-                                                     map->n_out, static_cast<T *>(y), d_status);
+        LAT_CUDA_TRY(launch_pdl(pool_kernel<T, false>, dim3(blocks), dim3(256), 0, s, static_cast<const T *>(x), c,
+                                map->nbr, map->mask, map->k3, map->n_in, map->n_out, static_cast<T *>(y), d_status));
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }
@@ -157,9 +159,9 @@ static lat_status launch_dense(const int32_t *coords, int64_t n, const void *fea
     LAT_CUDA_TRY(cudaMemsetAsync(out, 0, cells * c * sizeof(T), s));
     const int64_t threads = n * (c / 8);
     if (threads == 0) return LAT_OK;
-    dense_scatter_kernel<T><<<unsigned((threads + 255) / 256), 256, 0, s>>>(
-        reinterpret_cast<const int4 *>(coords), n, static_cast<const T *>(feats), c, bx, static_cast<T *>(out),
-        d_status);
+    LAT_CUDA_TRY(launch_pdl(dense_scatter_kernel<T>, dim3(unsigned((threads + 255) / 256)), dim3(256), 0, s,
+                            reinterpret_cast<const int4 *>(coords), n, static_cast<const T *>(feats), c, bx,
+                            static_cast<T *>(out), d_status));
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }

@@ -115,6 +115,7 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
                 const int32_t *__restrict__ pair_in, const int32_t *__restrict__ pair_out, int64_t capacity, int k3,
                 int64_t n_in, int64_t n_out, float *__restrict__ partial, int32_t *__restrict__ ranges,
                 int32_t *d_status) {
+    pdl_enter();
     using C = Cfg<M, N>;
     constexpr int NS = C::kStages;
     constexpr uint32_t idesc = make_idesc<T, M, N>();
@@ -334,6 +335,7 @@ constexpr int kRedLanes = 32;
 __global__ void __launch_bounds__(256)
 wgrad_tc_reduce_kernel(const float *__restrict__ partial, const int32_t *__restrict__ ranges, int nelem,
                        float *__restrict__ dw) {
+    pdl_enter();
     __shared__ float4 s_part[kRedLanes][8];
     const int k = blockIdx.y;
     const int v0 = __ldg(ranges + 2 * k), v1 = __ldg(ranges + 2 * k + 1);
@@ -376,13 +378,13 @@ static lat_status launch(const void *x, const void *dy, const lat_kmap *map, flo
     auto kern = wgrad_tc_kernel<T, M, N>;
     const int64_t grid = std::min<int64_t>(kWorkers, GridCache<KernelTag<T, M, N>>::get(kern, C::kSmem, int(C::kTmemCols), 2));
     if (grid <= 0) return LAT_ERR_CUDA;
-    kern<<<unsigned(grid), kThreads, C::kSmem, s>>>(static_cast<const T *>(x), static_cast<const T *>(dy),
-                                                    map->pair_off, map->pair_in, map->pair_out, map->pair_capacity,
-                                                    map->k3, map->n_in, map->n_out, partial, ranges, d_status);
+    LAT_CUDA_TRY(launch_pdl(kern, dim3(unsigned(grid)), dim3(kThreads), C::kSmem, s, static_cast<const T *>(x),
+                            static_cast<const T *>(dy), map->pair_off, map->pair_in, map->pair_out, map->pair_capacity,
+                            map->k3, map->n_in, map->n_out, partial, ranges, d_status));
     LAT_CUDA_TRY(cudaGetLastError());
     const int nelem = M * N;
     dim3 rg((nelem + 31) / 32, map->k3);
-    wgrad_tc_reduce_kernel<<<rg, 256, 0, s>>>(partial, ranges, nelem, dw);
+    LAT_CUDA_TRY(launch_pdl(wgrad_tc_reduce_kernel, dim3(rg), dim3(256), 0, s, partial, ranges, nelem, dw));
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }
