@@ -151,8 +151,11 @@ typedef struct {
  * a 32-bit mix of the key (its two halves folded, then the MurmurHash3
  * fmix32 finalizer) masked to the slot count; its probe sequence starts at
  * the first slot of the home slot's group and runs over consecutive slots
- * (linear probing), so a lookup reads whole groups.  The table must be
- * 64-byte aligned.
+ * (linear probing), so a lookup reads whole groups.  A key is stored within
+ * 4096 slots of the start of its home group (anywhere in a smaller table);
+ * an insert that finds no free slot in that window flags
+ * LAT_ERR_TABLE_FULL (only a table filled close to capacity gets there), and
+ * a lookup stops after the window.  The table must be 64-byte aligned.
  */
 
 /* Bytes of a table for n rows: 16 * next_pow2(max(ceil(rsv_ratio*n), 64)).
@@ -163,7 +166,8 @@ size_t lat_hash_bytes(int64_t n, float rsv_ratio);
 
 /* Insert coords[0..n) (int32 (n,4)) into `table` (table_bytes from
  * lat_hash_bytes; clears it first).  A duplicate coordinate keeps the lowest
- * row and flags LAT_ERR_DUPLICATE; a full table flags LAT_ERR_TABLE_FULL. */
+ * row and flags LAT_ERR_DUPLICATE; a key with no free slot in its probe
+ * window flags LAT_ERR_TABLE_FULL. */
 lat_status lat_hash_build(const int32_t *coords, int64_t n, void *table, size_t table_bytes,
                           int32_t *d_status, lat_stream stream);
 

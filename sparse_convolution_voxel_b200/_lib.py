@@ -114,9 +114,19 @@ def _ptr(t: torch.Tensor | None):
     return ctypes.c_void_p(t.data_ptr())
 
 
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+_cur_dev = getattr(torch._C, "_cuda_getDevice", None)
+
+
 def _stream(stream=None):
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return ctypes.c_void_p(s.cuda_stream)
+    """The CUDA stream handle: `stream` (a torch.cuda.Stream or a raw handle), else
+    the current stream of the current device (read without building a Stream object,
+    which costs a few microseconds per call)."""
+    if stream is None:
+        if _raw_stream is not None and _cur_dev is not None:
+            return ctypes.c_void_p(_raw_stream(_cur_dev()))
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream if isinstance(stream, int) else stream.cuda_stream)
 
 
 def _check(rc: int, where: str):
@@ -124,8 +134,11 @@ def _check(rc: int, where: str):
         raise LatticeError(rc, where)
 
 
+_DTYPE_CODE = {torch.float32: LAT_F32, torch.float16: LAT_F16, torch.bfloat16: LAT_BF16}
+
+
 def dtype_code(dt: torch.dtype) -> int:
-    return {torch.float32: LAT_F32, torch.float16: LAT_F16, torch.bfloat16: LAT_BF16}[dt]
+    return _DTYPE_CODE[dt]
 
 
 def make_geom(ksize, stride=1, pad=0, mode=LAT_SUBM) -> lat_geom:

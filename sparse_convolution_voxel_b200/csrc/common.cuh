@@ -62,21 +62,22 @@ __device__ __forceinline__ uint32_t slot_hash(uint64_t key) {
 
 // First slot of a key's probe sequence: its home slot (hash & cap_mask) rounded
 // down to the start of the home group.  Probing then runs over consecutive slots.
+// A key is stored within this many slots of the start of its home group (or
+// anywhere, for a smaller table): inserts that find no free slot in that
+// window flag LAT_ERR_TABLE_FULL, so lookups stop after it.  At the load
+// factors lat_hash_bytes gives (1/8 to 1/2 for ratios 2 to 8) probe
+// sequences are a few slots long; only a table filled close to capacity
+// reaches the limit.  It also bounds the work of a lookup in a table that
+// lat_hash_build did not fill.
+constexpr uint32_t kMaxProbeSlots = 4096;
+__device__ __forceinline__ uint32_t probe_window(uint32_t cap_mask) {
+    return cap_mask < kMaxProbeSlots - 1 ? cap_mask + 1 : kMaxProbeSlots;
+}
+
 __device__ __forceinline__ uint32_t probe_start(uint64_t key, uint32_t cap_mask) {
     return slot_hash(key) & cap_mask & ~uint32_t(kGroupSlots - 1);
 }
 
-// Look a key up; returns the row or -1.  Probing is bounded by the slot count.
-__device__ __forceinline__ int hash_find(const SlotGroup *__restrict__ groups, uint32_t cap_mask, uint64_t key) {
-    uint32_t s = probe_start(key, cap_mask);
-    for (uint32_t probe = 0; probe <= cap_mask; ++probe) {
-        const uint64_t k = __ldg(&groups[s / kGroupSlots].key[s % kGroupSlots]);
-        if (k == key) return int(__ldg(&groups[s / kGroupSlots].row[s % kGroupSlots]));
-        if (k == kEmptyKey) return -1;
-        s = (s + 1) & cap_mask;
-    }
-    return -1;
-}
 
 // Programmatic dependent launch.  Kernels started with launch_pdl may be
 // scheduled while the previous kernel on the stream is still running:
@@ -125,10 +126,18 @@ template <> struct Elem<__nv_bfloat16> {
     } while (0)
 
 namespace lat {
+// SM count of the current device (looked up once per device).
 inline int num_sms() {
-    int dev = 0, n = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n;
+    constexpr int kMaxDev = 64;
+    static int cached[kMaxDev] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return 148;
+    if (cached[dev] <= 0) {
+        int n = 148;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n;
+    }
+    return cached[dev];
 }
 inline bool pow2(uint64_t v) { return v && !(v & (v - 1)); }
 
@@ -169,6 +178,46 @@ inline cudaError_t fill_u32(void *p, int64_t n, uint32_t v, cudaStream_t s) {
     const int64_t want = (n / 4 + 255) / 256 + 1, cap = int64_t(num_sms()) * 8;
     return launch_pdl(fill_u32_kernel<0>, dim3(unsigned(want < cap ? want : cap)), dim3(256), 0, s,
                       static_cast<uint32_t *>(p), n, v);
+}
+
+// Up to kMaxFills regions of 32-bit words, each filled with its own value by
+// one launch (fill_list): the zero / -1 initialisations an entry point needs
+// cost one kernel instead of one each.
+constexpr int kMaxFills = 6;
+struct FillList {
+    uint32_t *p[kMaxFills];
+    int64_t n[kMaxFills];
+    uint32_t v[kMaxFills];
+    int count = 0;
+    void add(void *ptr, int64_t words, uint32_t value) {
+        if (words <= 0 || count >= kMaxFills) return;
+        p[count] = static_cast<uint32_t *>(ptr);
+        n[count] = words;
+        v[count] = value;
+        ++count;
+    }
+};
+template <int = 0>
+__global__ void __launch_bounds__(256) fill_list_kernel(FillList f) {
+    pdl_enter();
+    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+    const int64_t i0 = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+    for (int r = 0; r < f.count; ++r) {
+        uint32_t *p = f.p[r];
+        const int64_t n = f.n[r];
+        const uint32_t v = f.v[r];
+        const int64_t n4 = reinterpret_cast<uintptr_t>(p) % 16 == 0 ? n / 4 : 0;
+        const uint4 v4 = make_uint4(v, v, v, v);
+        for (int64_t i = i0; i < n4; i += stride) reinterpret_cast<uint4 *>(p)[i] = v4;
+        for (int64_t i = 4 * n4 + i0; i < n; i += stride) p[i] = v;
+    }
+}
+inline cudaError_t fill_list(const FillList &f, cudaStream_t s) {
+    if (f.count == 0) return cudaSuccess;
+    int64_t words = 0;
+    for (int r = 0; r < f.count; ++r) words = f.n[r] > words ? f.n[r] : words;
+    const int64_t want = (words / 4 + 255) / 256 + 1, cap = int64_t(num_sms()) * 8;
+    return launch_pdl(fill_list_kernel<0>, dim3(unsigned(want < cap ? want : cap)), dim3(256), 0, s, f);
 }
 
 // A side stream for independent chains of small kernels inside one entry

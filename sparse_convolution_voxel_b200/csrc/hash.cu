@@ -5,7 +5,7 @@
 // torch_lattice.backends.hash_rsv_ratio ("Backend and configuration
 // differences").  Design: 64-byte groups of 4 slots (4 keys, then 4 rows),
 // 32-bit mixing hash placement, probing from the start of the home group over
-// consecutive slots (bounded by the slot count), 64-bit atomicCAS to claim a
+// consecutive slots (at most kMaxProbeSlots of them), 64-bit atomicCAS to claim a
 // slot and an unsigned atomicMin on the row so that duplicates keep the lowest
 // row deterministically.
 #include "common.cuh"
@@ -27,7 +27,8 @@ __global__ void __launch_bounds__(256) hash_insert_kernel(const int4 *__restrict
         }
         uint32_t s = probe_start(key, cap_mask);
         bool placed = false;
-        for (uint32_t probe = 0; probe <= cap_mask; ++probe) {
+        const uint32_t window = probe_window(cap_mask);
+        for (uint32_t probe = 0; probe < window; ++probe) {
             unsigned long long *kp = &groups[s / kGroupSlots].key[s % kGroupSlots];
             unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(kp);
             if (cur == kEmptyKey) cur = atomicCAS(kp, (unsigned long long)kEmptyKey, (unsigned long long)key);

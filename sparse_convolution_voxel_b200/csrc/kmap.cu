@@ -109,7 +109,7 @@ __device__ __forceinline__ bool query_coord(const Geom &g, const int4 &c, int ix
 // what it can (a match, or an empty slot before it, ends the probe); the rows
 // of the matches are loaded together after the rounds.  At the table's load
 // factor nearly every probe ends inside its home group, so a batch takes about
-// one round.  Rounds are bounded by the group count.  Strided and transposed
+// one round.  Rounds are bounded by the probe window (kMaxProbeSlots).  Strided and transposed
 // maps (submanifold maps use kmap_probe_sym_kernel): every offset is probed and
 // the mask, grouping key, first sort histogram and per-block counts are
 // produced here.
@@ -158,7 +158,7 @@ kmap_probe_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const
                 pending |= 1u << e;
             }
         }
-        for (uint32_t round = 0; pending && round <= cap_mask / kGroupSlots; ++round) {
+        for (uint32_t round = 0; pending && round < probe_window(cap_mask) / kGroupSlots; ++round) {
             ulonglong2 ka[kProbeBatch], kb[kProbeBatch];
 #pragma unroll
             for (int e = 0; e < kProbeBatch; ++e) {
@@ -220,12 +220,18 @@ kmap_probe_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const
 
 // Submanifold map, step 0: the centre row of nbr (every row is its own centre
 // neighbour), -1 in every offset above the centre (filled by mirrored hits
-// only), and masks holding just the centre bit.  One thread per row; all stores
-// coalesced.
+// only), masks holding just the centre bit, and zeroed sort histograms and
+// tile masks.  One thread per row; all stores coalesced.
 __global__ void __launch_bounds__(kQueryThreads)
-kmap_subm_init_kernel(int64_t n_out, int k3, int32_t *__restrict__ nbr, uint32_t *__restrict__ mask) {
+kmap_subm_init_kernel(int64_t n_out, int k3, int32_t *__restrict__ nbr, uint32_t *__restrict__ mask,
+                      int32_t *__restrict__ hist, int64_t hist_words, uint32_t *__restrict__ tile_mask,
+                      int64_t ntiles) {
     pdl_enter();
     const int64_t j = blockIdx.x * int64_t(kQueryThreads) + threadIdx.x;
+    // the row sort's digit histograms and the tile masks start at zero
+    const int64_t stride = int64_t(gridDim.x) * kQueryThreads;
+    for (int64_t i = j; i < hist_words; i += stride) hist[i] = 0;
+    for (int64_t i = j; i < ntiles; i += stride) tile_mask[i] = 0;
     if (j >= n_out) return;
     const int centre = k3 / 2;
     nbr[int64_t(centre) * n_out + j] = int32_t(j);
@@ -237,7 +243,7 @@ kmap_subm_init_kernel(int64_t n_out, int k3, int32_t *__restrict__ nbr, uint32_t
 // blockIdx.y is the offset, so a warp probes one offset for 32 consecutive rows
 // (coalesced coordinate loads and nbr stores, a uniform key delta).  A probe
 // reads its home group's 4 keys with two 16-byte loads and walks on to the next
-// group only when all 4 slots hold other keys (bounded by the group count).
+// group only when all 4 slots hold other keys (bounded by the probe window).
 // A hit at row r also writes the mirrored entry nbr[k3-1-k][r] = j (the
 // relation is symmetric) and ORs both bits into the masks.  Far fewer
 // instructions per lookup than looping over the offsets inside one thread,
@@ -263,7 +269,7 @@ kmap_probe_sym_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, c
     int r = -1;
     if (ok) {
         uint32_t slot = probe_start(key, cap_mask);
-        for (uint32_t round = 0; round <= cap_mask / kGroupSlots; ++round) {
+        for (uint32_t round = 0; round < probe_window(cap_mask) / kGroupSlots; ++round) {
             const SlotGroup *gp = groups + slot / kGroupSlots;
             const ulonglong2 a = __ldg(reinterpret_cast<const ulonglong2 *>(gp->key));
             const ulonglong2 b = __ldg(reinterpret_cast<const ulonglong2 *>(gp->key + 2));
@@ -687,11 +693,10 @@ static lat_status finish_kmap(lat_kmap *map, int k3, int nblk, KmapWs &w, int32_
     return st;
 }
 
-// Stable row sort by grouping key -> perm, tile masks ORed by the last pass.
+// Stable row sort by grouping key -> perm, tile masks ORed by the last pass
+// (map->tile_mask must hold zeros beforehand).
 static lat_status sort_rows(lat_kmap *map, int k3, KmapWs &w, cudaStream_t s) {
     const int64_t n_out = map->n_out;
-    const int64_t ntiles = (n_out + LAT_TILE_ROWS - 1) / LAT_TILE_ROWS;
-    LAT_CUDA_TRY(fill_u32(map->tile_mask, ntiles, 0u, s));
     const int64_t hsize = 256 * int64_t(w.ntile);
     int32_t *h1 = w.hist, *h2 = w.hist + hsize;
     int32_t *t1 = w.totals, *t2 = w.totals + 256;
@@ -800,7 +805,7 @@ extern "C" lat_status lat_kmap_query(const void *table, size_t table_bytes, cons
                 g.delta[k] = dx * (1ll << 32) + dy * (1ll << 16) + dz;
             }
     const int nblk = int((n_out + kQueryThreads - 1) / kQueryThreads);
-    LAT_CUDA_TRY(fill_u32(w.hist, int64_t(w.hist_bytes / 4), 0u, s));
+    const int64_t ntiles = (n_out + LAT_TILE_ROWS - 1) / LAT_TILE_ROWS;
     const uint32_t cap_mask = uint32_t(table_bytes / kSlotBytes - 1);
     const SlotGroup *slots = static_cast<const SlotGroup *>(table);
     const int4 *oc = reinterpret_cast<const int4 *>(out_coords);
@@ -808,7 +813,7 @@ extern "C" lat_status lat_kmap_query(const void *table, size_t table_bytes, cons
         // the upper half of the table is filled by mirrored hits only
         const int centre = k3 / 2;
         LAT_CUDA_TRY(launch_pdl(kmap_subm_init_kernel, dim3(nblk), dim3(kQueryThreads), 0, s, n_out, k3, map->nbr,
-                                map->mask));
+                                map->mask, w.hist, int64_t(w.hist_bytes / 4), map->tile_mask, ntiles));
         LAT_CUDA_TRY(cudaGetLastError());
         if (centre > 0) {
             LAT_CUDA_TRY(launch_pdl(kmap_probe_sym_kernel, dim3(unsigned(nblk), unsigned(centre)), dim3(kQueryThreads),
@@ -818,6 +823,10 @@ extern "C" lat_status lat_kmap_query(const void *table, size_t table_bytes, cons
         LAT_CUDA_TRY(launch_pdl(kmap_count_kernel, dim3(nblk), dim3(kQueryThreads), 0, s, map->mask, n_out, k3,
                                 w.block_counts, nblk, w.keys, w.hist, w.ntile));
     } else {
+        FillList f;
+        f.add(w.hist, int64_t(w.hist_bytes / 4), 0u);
+        f.add(map->tile_mask, ntiles, 0u);
+        LAT_CUDA_TRY(fill_list(f, s));
         LAT_CUDA_TRY(launch_pdl(kmap_probe_kernel, dim3(nblk), dim3(kQueryThreads), 0, s, slots, cap_mask, oc, n_out,
                                 n_in, g, map->nbr, map->mask, w.keys, w.hist, w.ntile, w.block_counts, nblk, d_status));
     }
@@ -853,20 +862,28 @@ extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int
     const size_t need = lat_kmap_from_parent_ws_bytes(n_fine, n_coarse, k3);
     if (ws_bytes < need || (need && !ws)) return LAT_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (down) {
-        down->mode = LAT_STRIDED;
-        if (n_coarse > 0) {
-            LAT_CUDA_TRY(fill_u32(down->nbr, int64_t(k3) * n_coarse, ~0u, s));
-            LAT_CUDA_TRY(fill_u32(down->mask, n_coarse, 0u, s));
-        }
-    }
+    if (down) down->mode = LAT_STRIDED;
     if (up) up->mode = LAT_TRANSPOSED;
     KmapWs w_down = carve_kmap_ws(ws, n_coarse, k3);
     KmapWs w_up = carve_kmap_ws(static_cast<char *>(ws) + w_down.total, n_fine, k3);
     // transposed map with K^3 <= 8: every fine row has one neighbour (its parent)
     // and its key is the one-hot mask, so the row sort alone yields the pairs
     const bool up_direct = up && n_fine > 0 && group_key_bits(k3) <= 8;
-    if (up_direct) LAT_CUDA_TRY(fill_u32(w_up.hist, int64_t(w_up.hist_bytes / 4), 0u, s));
+    // every initialisation both maps need, in one launch: the strided map's
+    // table (-1) and masks (0, both filled by the parent scatter), and each
+    // map's sort histograms and tile masks
+    FillList f;
+    if (down && n_coarse > 0) {
+        f.add(down->nbr, int64_t(k3) * n_coarse, ~0u);
+        f.add(down->mask, n_coarse, 0u);
+        f.add(w_down.hist, int64_t(w_down.hist_bytes / 4), 0u);
+        f.add(down->tile_mask, (n_coarse + LAT_TILE_ROWS - 1) / LAT_TILE_ROWS, 0u);
+    }
+    if (up && n_fine > 0) {
+        f.add(w_up.hist, int64_t(w_up.hist_bytes / 4), 0u);
+        f.add(up->tile_mask, (n_fine + LAT_TILE_ROWS - 1) / LAT_TILE_ROWS, 0u);
+    }
+    LAT_CUDA_TRY(fill_list(f, s));
     if (n_fine > 0) {
         LAT_CUDA_TRY(launch_pdl(parent_maps_kernel, dim3(unsigned((n_fine + 255) / 256)), dim3(256), 0, s,
                                 reinterpret_cast<const int4 *>(fine_coords), parent, n_fine, n_coarse, geom->stride[0],
@@ -892,8 +909,6 @@ extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int
         }
         KmapWs &w = map == down ? w_down : w_up;
         if (map == up && up_direct) {
-            const int64_t ntiles = (map->n_out + LAT_TILE_ROWS - 1) / LAT_TILE_ROWS;
-            LAT_CUDA_TRY(fill_u32(map->tile_mask, ntiles, 0u, s));
             LAT_CUDA_TRY(launch_pdl(sort_rowscan_kernel, dim3(256), dim3(256), 0, s, w.hist, w.ntile, w.totals));
             LAT_CUDA_TRY(cudaGetLastError());
             const PairOut po{parent, map->pair_in, map->pair_out, map->pair_capacity, map->pair_off, k3, d_status};
@@ -904,7 +919,6 @@ extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int
             continue;
         }
         const int nblk = int((map->n_out + kQueryThreads - 1) / kQueryThreads);
-        LAT_CUDA_TRY(fill_u32(w.hist, int64_t(w.hist_bytes / 4), 0u, s));
         LAT_CUDA_TRY(launch_pdl(kmap_count_kernel, dim3(nblk), dim3(kQueryThreads), 0, s, map->mask, map->n_out, k3,
                                 w.block_counts, nblk, w.keys, w.hist, w.ntile));
         LAT_CUDA_TRY(cudaGetLastError());
