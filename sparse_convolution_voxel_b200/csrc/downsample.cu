@@ -141,10 +141,13 @@ down_candidates_kernel(const int4 *__restrict__ coords, int64_t n, DownGeom g, u
     }
 }
 
+// range[0..3] = INT_MAX, range[4..7] = INT_MIN (the candidates pass reduces into
+// them), range[8] = 0 (the count pass's arrival counter).
 __global__ void range_init_kernel(int *range) {
     pdl_enter();
     if (threadIdx.x < 4) range[threadIdx.x] = INT_MAX;
     else if (threadIdx.x < 8) range[threadIdx.x] = INT_MIN;
+    else if (threadIdx.x == 8) range[8] = 0;
 }
 
 // Order-preserving compact key of a coarse row: fields shifted to their minimum, packed.
@@ -222,14 +225,29 @@ bitmap_mark_kernel(const uint64_t *__restrict__ keys, int64_t items, const int *
     atomicOr(bitmap + (v >> 5), 1u << (v & 31));
 }
 
-// Set bits per group of 32 words (1024 bits), and per block of 256 groups.
+// Set bits per group of 32 words (1024 bits): grp_cnt, and grp_pre = the
+// exclusive prefix of grp_cnt within each block of 256 groups; blk_cnt = the
+// block's total.  The last block to finish (an arrival counter that the range
+// pass zeroes) scans blk_cnt into blk_off and writes the coarse row count, or
+// -1 when the bitmap path does not apply (0 when there is no row at all), so
+// no separate scan launch is needed.  Blocks past the plan's groups only
+// return; the arrival count is over the blocks that cover groups.
 __global__ void __launch_bounds__(256)
-bitmap_count_kernel(const uint32_t *__restrict__ bitmap, const int *__restrict__ range, int64_t budget_bits,
-                    int32_t *__restrict__ grp_cnt, int32_t *__restrict__ blk_cnt) {
+bitmap_count_kernel(const uint32_t *__restrict__ bitmap, int *__restrict__ range, int64_t budget_bits,
+                    int32_t *__restrict__ grp_cnt, int32_t *__restrict__ grp_pre, int32_t *__restrict__ blk_cnt,
+                    int64_t *__restrict__ blk_off, int64_t *__restrict__ n_out_dev) {
     pdl_enter();
     __shared__ int s_warp[8];
+    __shared__ int64_t s_big[8];
+    __shared__ bool s_last;
     const Plan p = make_plan(range, budget_bits);
-    if (int64_t(blockIdx.x) * 256 >= p.ngroups) return;
+    const int64_t nblk = (p.ngroups + 255) / 256;
+    if (nblk == 0) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) *n_out_dev = p.empty ? 0 : -1;
+        return;
+    }
+    if (int64_t(blockIdx.x) >= nblk) return;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int64_t gi = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
     int c = 0;
     if (gi < p.ngroups) {
@@ -239,72 +257,7 @@ bitmap_count_kernel(const uint32_t *__restrict__ bitmap, const int *__restrict__
             const uint4 v = __ldg(w4 + e);
             c += __popc(v.x) + __popc(v.y) + __popc(v.z) + __popc(v.w);
         }
-        grp_cnt[gi] = c;
     }
-    int sum = c;
-    for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-    if ((threadIdx.x & 31) == 0) s_warp[threadIdx.x >> 5] = sum;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int t = 0;
-        for (int w = 0; w < 8; ++w) t += s_warp[w];
-        blk_cnt[blockIdx.x] = t;
-    }
-}
-
-// Exclusive scan of the per-block counts (one block) and the coarse row count,
-// or -1 when the bitmap path does not apply (the sort path must run).
-__global__ void __launch_bounds__(1024)
-bitmap_blockscan_kernel(const int *__restrict__ range, int64_t budget_bits, const int32_t *__restrict__ blk_cnt,
-                        int64_t *__restrict__ blk_off, int64_t *__restrict__ n_out_dev) {
-    pdl_enter();
-    __shared__ int64_t s_warp[32];
-    const Plan p = make_plan(range, budget_bits);
-    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
-    const int64_t nblk = (p.ngroups + 255) / 256;
-    const int64_t per = (nblk + 1023) / 1024;
-    const int64_t b0 = min(nblk, t * per), b1 = min(nblk, b0 + per);
-    int64_t sum = 0;
-    for (int64_t i = b0; i < b1; ++i) sum += blk_cnt[i];
-    int64_t incl = sum;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const int64_t o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-        if (lane >= d) incl += o;
-    }
-    if (lane == 31) s_warp[w] = incl;
-    __syncthreads();
-    if (w == 0) {
-        int64_t x = s_warp[lane];
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const int64_t o = __shfl_up_sync(0xFFFFFFFFu, x, d);
-            if (lane >= d) x += o;
-        }
-        s_warp[lane] = x;
-    }
-    __syncthreads();
-    int64_t run = (w ? s_warp[w - 1] : 0) + incl - sum;
-    for (int64_t i = b0; i < b1; ++i) {
-        blk_off[i] = run;
-        run += blk_cnt[i];
-    }
-    if (t == 0) *n_out_dev = p.ok ? s_warp[31] : (p.empty ? 0 : -1);
-}
-
-// Coordinates of the set bits in bit order (= canonical order); each group's
-// first rank (grp_off) for the parent pass.
-__global__ void __launch_bounds__(256)
-bitmap_emit_kernel(const uint32_t *__restrict__ bitmap, const int *__restrict__ range, int64_t budget_bits,
-                   const int32_t *__restrict__ grp_cnt, const int64_t *__restrict__ blk_off,
-                   int64_t *__restrict__ grp_off, int4 *__restrict__ out, int64_t capacity) {
-    pdl_enter();
-    __shared__ int s_warp[8];
-    const Plan p = make_plan(range, budget_bits);
-    if (int64_t(blockIdx.x) * 256 >= p.ngroups) return;
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const int64_t gi = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
-    const int c = gi < p.ngroups ? grp_cnt[gi] : 0;
     int incl = c;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -315,60 +268,107 @@ bitmap_emit_kernel(const uint32_t *__restrict__ bitmap, const int *__restrict__ 
     __syncthreads();
     int before = 0;
     for (int q = 0; q < w; ++q) before += s_warp[q];
-    if (gi >= p.ngroups) return;
-    int64_t rank = blk_off[blockIdx.x] + before + incl - c;
-    grp_off[gi] = rank;
-    if (c == 0) return;
-    // the group's 32 words in 8 vector loads, then its set bits in order
-    uint4 g4[8];
-    const uint4 *w4 = reinterpret_cast<const uint4 *>(bitmap + gi * 32);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) g4[e] = __ldg(w4 + e);
-#pragma unroll
-    for (int wi = 0; wi < 32; ++wi) {
-        const uint4 &q = g4[wi / 4];
-        uint32_t word = (wi & 3) == 0 ? q.x : (wi & 3) == 1 ? q.y : (wi & 3) == 2 ? q.z : q.w;
-        while (word) {
-            const int b = __ffs(word) - 1;
-            word &= word - 1;
-            if (rank < capacity) out[rank] = p.cp.unpack(uint32_t(gi * 1024 + wi * 32 + b));
-            ++rank;
-        }
+    if (gi < p.ngroups) {
+        grp_cnt[gi] = c;
+        grp_pre[gi] = before + incl - c;
     }
+    if (threadIdx.x == 0) {
+        int t = 0;
+        for (int q = 0; q < 8; ++q) t += s_warp[q];
+        blk_cnt[blockIdx.x] = t;
+        __threadfence();
+        s_last = atomicAdd(range + 8, 1) == int(nblk - 1);
+    }
+    __syncthreads();
+    if (!s_last) return;
+    // last block: exclusive scan of the block totals (each thread a run of them)
+    __threadfence();
+    const int64_t per = (nblk + 255) / 256;
+    const int64_t b0 = min(nblk, threadIdx.x * per), b1 = min(nblk, b0 + per);
+    int64_t sum = 0;
+    for (int64_t i = b0; i < b1; ++i) sum += __ldcg(blk_cnt + i);
+    int64_t inc = sum;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int64_t o = __shfl_up_sync(0xFFFFFFFFu, inc, d);
+        if (lane >= d) inc += o;
+    }
+    if (lane == 31) s_big[w] = inc;
+    __syncthreads();
+    int64_t run = inc - sum;
+    for (int q = 0; q < w; ++q) run += s_big[q];
+    for (int64_t i = b0; i < b1; ++i) {
+        blk_off[i] = run;
+        run += __ldcg(blk_cnt + i);
+    }
+    if (threadIdx.x == 255) *n_out_dev = run;
 }
 
-// Rank of each input's (single) proposal among the set bits: its coarse row.
-// Inputs without a coarse row get -1; nothing else is written when the bitmap
-// path does not apply (the sort path fills parent then).
+// Two roles in one launch, both reading only the count pass's results:
+//   blocks [0, emit_blocks): warps walk the 1024-bit groups (grid-stride, 32
+//     groups at a time, skipping empty ones); per group each lane takes one word: a warp scan of the word popcounts gives every set bit its
+//     rank = blk_off + grp_pre + the bits before it, and the lane writes the
+//     coordinates of its bits (bit order = canonical order);
+//   the remaining blocks: one thread per input, its (single) proposal's rank
+//     among the set bits = its coarse row (parent); -1 for an input without
+//     one.  Nothing is written when the bitmap path does not apply.
 __global__ void __launch_bounds__(256)
-bitmap_parent_kernel(const uint64_t *__restrict__ keys, int64_t n, const int *__restrict__ range,
-                     int64_t budget_bits, const uint32_t *__restrict__ bitmap, const int64_t *__restrict__ grp_off,
-                     int32_t *__restrict__ parent) {
+bitmap_emit_kernel(const uint32_t *__restrict__ bitmap, const int *__restrict__ range, int64_t budget_bits,
+                   const int32_t *__restrict__ grp_cnt, const int32_t *__restrict__ grp_pre,
+                   const int64_t *__restrict__ blk_off, int4 *__restrict__ out, int64_t capacity, int emit_blocks,
+                   const uint64_t *__restrict__ keys, int64_t n_in, int32_t *__restrict__ parent) {
     pdl_enter();
-    const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
-    if (i >= n) return;
+    const Plan p = make_plan(range, budget_bits);
+    if (!p.ok) return;
+    const int lane = threadIdx.x & 31;
+    if (int(blockIdx.x) < emit_blocks) {
+        // a warp takes 32 consecutive groups at a time: one coalesced load of their
+        // counts, then only the non-empty ones (most groups of a sparse bitmap are empty)
+        const int64_t nwarps = int64_t(emit_blocks) * (blockDim.x >> 5);
+        const int64_t nchunks = (p.ngroups + 31) / 32;
+        for (int64_t ch = blockIdx.x * int64_t(blockDim.x >> 5) + (threadIdx.x >> 5); ch < nchunks; ch += nwarps) {
+            const int64_t gl = ch * 32 + lane;
+            unsigned busy = __ballot_sync(0xFFFFFFFFu, gl < p.ngroups && __ldg(grp_cnt + gl) != 0);
+            while (busy) {
+                const int64_t g = ch * 32 + __ffs(busy) - 1;
+                busy &= busy - 1;
+                uint32_t word = __ldg(bitmap + g * 32 + lane);
+                const int pc = __popc(word);
+                int incl = pc;
+#pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+                    if (lane >= d) incl += o;
+                }
+                int64_t rank = __ldg(blk_off + (g >> 8)) + __ldg(grp_pre + g) + incl - pc;
+                while (word) {
+                    const int b = __ffs(word) - 1;
+                    word &= word - 1;
+                    if (rank < capacity) out[rank] = p.cp.unpack(uint32_t(g * 1024 + lane * 32 + b));
+                    ++rank;
+                }
+            }
+        }
+        return;
+    }
+    const int64_t i = (int64_t(blockIdx.x) - emit_blocks) * blockDim.x + threadIdx.x;
+    if (i >= n_in) return;
     const uint64_t key = keys[i];
     if (key == kEmptyKey) {
         parent[i] = -1;
         return;
     }
-    const Plan p = make_plan(range, budget_bits);
-    if (!p.ok) return;
     const uint32_t v = p.cp.pack(key);
     const uint32_t gi = v >> 10, wi = (v >> 5) & 31;
     // bits of the group before v: whole words below wi, then the low bits of word wi
-    uint4 g4[8];
-    const uint4 *w4 = reinterpret_cast<const uint4 *>(bitmap + int64_t(gi) * 32);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) g4[e] = __ldg(w4 + e);
-    int64_t rank = grp_off[gi];
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-        const uint4 &q = g4[e / 4];
-        const uint32_t word = (e & 3) == 0 ? q.x : (e & 3) == 1 ? q.y : (e & 3) == 2 ? q.z : q.w;
-        const uint32_t keep = uint32_t(e) < wi ? 0xFFFFFFFFu : (uint32_t(e) == wi ? (1u << (v & 31)) - 1u : 0u);
-        rank += __popc(word & keep);
+    const uint32_t *gw = bitmap + int64_t(gi) * 32;
+    int64_t rank = __ldg(blk_off + (gi >> 8)) + __ldg(grp_pre + gi);
+    for (uint32_t e = 0; e < (wi & ~3u); e += 4) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4 *>(gw + e));
+        rank += __popc(q.x) + __popc(q.y) + __popc(q.z) + __popc(q.w);
     }
+    for (uint32_t e = wi & ~3u; e < wi; ++e) rank += __popc(__ldg(gw + e));
+    rank += __popc(__ldg(gw + wi) & ((1u << (v & 31)) - 1u));
     parent[i] = int32_t(rank);
 }
 
@@ -440,7 +440,7 @@ struct DownWs {
     // bitmap path
     uint32_t *bitmap;
     int32_t *grp_cnt;
-    int64_t *grp_off;
+    int32_t *grp_pre;
     int32_t *blk_cnt;
     int64_t *blk_off;
     int64_t max_groups;
@@ -451,7 +451,7 @@ static DownWs carve_down_ws(void *base, int64_t items) {
     DownWs w{};
     Carver cv(base);
     w.keys = cv.take<uint64_t>(size_t(items));
-    w.range = cv.take<int>(8);
+    w.range = cv.take<int>(16);
     w.n_out_dev = cv.take<int64_t>(1);
     const size_t common = cv.used;
     // sort path
@@ -471,7 +471,7 @@ static DownWs carve_down_ws(void *base, int64_t items) {
     w.max_groups = std::max<int64_t>(1, bits / 1024);
     w.bitmap = cv.take<uint32_t>(size_t(w.max_groups) * 32);
     w.grp_cnt = cv.take<int32_t>(size_t(w.max_groups));
-    w.grp_off = cv.take<int64_t>(size_t(w.max_groups));
+    w.grp_pre = cv.take<int32_t>(size_t(w.max_groups));
     const int64_t max_blk = (w.max_groups + 255) / 256;
     w.blk_cnt = cv.take<int32_t>(size_t(max_blk));
     w.blk_off = cv.take<int64_t>(size_t(max_blk));
@@ -537,19 +537,14 @@ static lat_status enqueue_bitmap_path(const int32_t *coords, int64_t n_in, const
                             w.bitmap));
     LAT_CUDA_TRY(cudaGetLastError());
     LAT_CUDA_TRY(launch_pdl(bitmap_count_kernel, dim3(gblocks), dim3(256), 0, s, w.bitmap, w.range, budget, w.grp_cnt,
-                            w.blk_cnt));
+                            w.grp_pre, w.blk_cnt, w.blk_off, w.n_out_dev));
     LAT_CUDA_TRY(cudaGetLastError());
-    LAT_CUDA_TRY(launch_pdl(bitmap_blockscan_kernel, dim3(1), dim3(1024), 0, s, w.range, budget, w.blk_cnt, w.blk_off,
-                            w.n_out_dev));
+    const int emit_blocks = int(std::min<int64_t>((w.max_groups + 255) / 256, int64_t(num_sms()) * 8));
+    const unsigned parent_blocks = parent ? in_blocks : 0u;
+    LAT_CUDA_TRY(launch_pdl(bitmap_emit_kernel, dim3(unsigned(emit_blocks) + parent_blocks), dim3(256), 0, s, w.bitmap,
+                            w.range, budget, w.grp_cnt, w.grp_pre, w.blk_off, reinterpret_cast<int4 *>(out_coords),
+                            out_capacity, emit_blocks, w.keys, parent ? n_in : int64_t(0), parent));
     LAT_CUDA_TRY(cudaGetLastError());
-    LAT_CUDA_TRY(launch_pdl(bitmap_emit_kernel, dim3(gblocks), dim3(256), 0, s, w.bitmap, w.range, budget, w.grp_cnt,
-                            w.blk_off, w.grp_off, reinterpret_cast<int4 *>(out_coords), out_capacity));
-    LAT_CUDA_TRY(cudaGetLastError());
-    if (parent) {
-        LAT_CUDA_TRY(launch_pdl(bitmap_parent_kernel, dim3(in_blocks), dim3(256), 0, s, w.keys, n_in, w.range, budget,
-                                w.bitmap, w.grp_off, parent));
-        LAT_CUDA_TRY(cudaGetLastError());
-    }
     return LAT_OK;
 }
 
