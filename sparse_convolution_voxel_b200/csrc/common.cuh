@@ -202,7 +202,9 @@ __global__ void __launch_bounds__(256) fill_list_kernel(FillList f) {
     pdl_enter();
     const int64_t stride = int64_t(gridDim.x) * blockDim.x;
     const int64_t i0 = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
-    for (int r = 0; r < f.count; ++r) {
+#pragma unroll
+    for (int r = 0; r < kMaxFills; ++r) {
+        if (r >= f.count) break;
         uint32_t *p = f.p[r];
         const int64_t n = f.n[r];
         const uint32_t v = f.v[r];
