@@ -104,8 +104,9 @@ class Pipeline:
     and joined back at the end.  Each chain has its own workspace.  Many of the
     kernels are short or latency-bound, so the two chains fill each other's
     gaps on the GPU.  The host enqueues the coarse support first, then the
-    kernel map and the forward pass, then reads the coarse row count (ready by
-    then) and enqueues the rest of both chains."""
+    kernel map and the forward pass, then reads the coarse row count and
+    enqueues the rest of both chains interleaved; the second chain's stream has
+    the higher priority (it waits on the host for the count halfway through)."""
 
     MAIN_PHASES = ["hash", "kmap", "fwd", "dgrad", "wgrad"]
     SIDE_PHASES = ["downsample", "down_maps", "down_fwd", "up_fwd"]
@@ -120,7 +121,10 @@ class Pipeline:
         self.status = scv.new_status(dev)
         self.ws = scv.Workspace(dev)
         self.ws_side = scv.Workspace(dev)
-        self.side = torch.cuda.Stream(dev)
+        # the second chain waits on the host for the coarse row count halfway through,
+        # so its kernels get the higher stream priority: its first half finishes
+        # sooner and its second half is enqueued sooner
+        self.side = torch.cuda.Stream(dev, priority=torch.cuda.Stream.priority_range()[1])
         self.forked, self.joined = torch.cuda.Event(), torch.cuda.Event()
         self.table = torch.empty(scv.lat_hash_bytes(n, RSV_RATIO) // 8, dtype=torch.int64, device=dev)
         self.km = scv.KernelMap(n, n, 27, dev)
@@ -188,19 +192,19 @@ class Pipeline:
         scv.lat_kmap_from_parent(d["coords"], self.parent, self.g_down, self.km_down.c, self.km_up.c, self.wsb_side, s,
                                  stream=side)
         rec("down_maps", 1, side)
+        rec("dgrad", 0, main)
+        scv.lat_sconv_dgrad(d["g"], d["w"], self.km.c, True, self.dx, self.wsb, s)
+        rec("dgrad", 1, main)
         rec("down_fwd", 0, side)
         scv.lat_sconv_fwd(d["x"], d["wd"], self.km_down.c, self.yc, self.wsb_side, s, stream=side)
         rec("down_fwd", 1, side)
+        rec("wgrad", 0, main)
+        scv.lat_sconv_wgrad(d["x"], d["g"], self.km.c, self.dw, self.wsb, s)
+        rec("wgrad", 1, main)
         rec("up_fwd", 0, side)
         scv.lat_sconv_fwd(self.yc, d["wu"], self.km_up.c, self.z, self.wsb_side, s, stream=side)
         rec("up_fwd", 1, side)
         self.joined.record(side)
-        rec("dgrad", 0, main)
-        scv.lat_sconv_dgrad(d["g"], d["w"], self.km.c, True, self.dx, self.wsb, s)
-        rec("dgrad", 1, main)
-        rec("wgrad", 0, main)
-        scv.lat_sconv_wgrad(d["x"], d["g"], self.km.c, self.dw, self.wsb, s)
-        rec("wgrad", 1, main)
         main.wait_event(self.joined)
 
     def pair_count(self) -> int:
