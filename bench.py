@@ -231,11 +231,17 @@ class Pipeline:
         }
 
 
-# DRAM bytes per launch of a phase from one ncu capture of this workload
-# (profiles/launches_lidar_subm_step.md: the submanifold kmap query, its 8
-# kernels summed, caches not flushed between kernels); None where no capture
-# matches the current kernels.
-PHASE_TRAFFIC = {"kmap": 26.8e6}
+# The kernel the roofline object reports: the path kernel with the largest
+# share of the step's ncu launch list (serialised; the tcgen05 data-gradient
+# conv, 8.2% of the step's kernel time and the largest of the path's kernels).
+DOMINANT_KERNEL = "dgrad"
+
+# DRAM bytes per launch from that ncu launch list of this workload (caches not
+# flushed between kernels): the dgrad conv (its DRAM writes include the
+# write-back of the forward pass's output, evicted while it runs) and the
+# submanifold kmap query's kernels summed; None where no capture matches the
+# current kernels.
+PHASE_TRAFFIC = {"dgrad": 77.1e6, "kmap": 26.8e6}
 
 
 def flush_l2(buf: torch.Tensor):
@@ -566,7 +572,7 @@ def main():
 
     # per-phase times from instrumented steps outside the timed region: a timing
     # event between two kernels holds back the next kernel's early launch, so the
-    # timed steps carry events around the largest phase only
+    # timed steps carry events around the dominant kernel's call only
     pb = pipe.phase_bytes()
     inst = [{p: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
              for p in Pipeline.PHASES} for _ in range(min(args.steps, 10))]
@@ -576,7 +582,7 @@ def main():
         pipe.step(ev)
     torch.cuda.synchronize()
     phase_ms_inst = {p: statistics.mean(ev[p][0].elapsed_time(ev[p][1]) for ev in inst) for p in Pipeline.PHASES}
-    dominant = max(pb, key=lambda p: phase_ms_inst[p])
+    dominant = DOMINANT_KERNEL
 
     steps = [{"step": (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)),
               dominant: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))}
@@ -621,10 +627,12 @@ def main():
             "phase_ms": {k: round(v, 4) for k, v in phase_ms_inst.items()},
             "phase_ms_note": "per-phase event times from instrumented steps outside the timed region "
                              "(the two chains overlap, so phases do not add up to the step)",
-            "roofline": {"kernel": dominant, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "roofline": {"kernel": f"{dominant} (conv_tc_kernel: gather dy, W^T on tcgen05)", "bound": "hbm",
+                         "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm, "traffic": PHASE_TRAFFIC.get(dominant),
                          "alg_bytes": pb[dominant], "ms": dominant_ms, "peak_source": f"{src} hbm_gbs",
                          "timing": "CUDA events around this phase on its stream in every timed step",
+                         "traffic_per_phase": PHASE_TRAFFIC,
                          "per_phase_frac": {p: round(pb[p] / (phase_ms_inst[p] * 1e-3) / 1e9 / hbm, 4)
                                             for p in pb}},
             "gpu_launches": None if launches_per_step is None else launches_per_step * args.steps,
