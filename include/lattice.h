@@ -118,7 +118,9 @@ typedef struct {
  * Pairs are grouped by offset (ascending k) and, within an offset, sorted by
  * ascending output row, so the lists are deterministic.  n_in, n_out and k3
  * are set by the caller before lat_kmap_query; mode records the geometry's
- * mode (written by the query).
+ * mode (written by the query).  In a LAT_SUBM map the centre offset K^3/2
+ * maps every row to itself (nbr[centre*n_out + j] == j); the convolution
+ * passes rely on that and do not read the centre column.
  */
 typedef struct {
     int32_t *nbr;

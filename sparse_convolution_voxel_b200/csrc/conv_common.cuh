@@ -20,6 +20,7 @@ struct MapView {
     int64_t ntiles;
     int k3;
     int flip;
+    int centre;  // submanifold maps: the centre offset, whose neighbour of row j is j itself; else -1
 
     __device__ __forceinline__ uint32_t tile_mask_at(int64_t t) const {
         const uint32_t m = tile_mask[t];
@@ -30,6 +31,7 @@ struct MapView {
         return nbr + int64_t(kk) * n_out + j;
     }
     __device__ __forceinline__ int neighbour(int k, int64_t j) const {
+        if (k == centre) return int(j);
         const int kk = flip ? (k3 - 1 - k) : k;
         return __ldg(nbr + int64_t(kk) * n_out + j);
     }
@@ -45,6 +47,9 @@ inline MapView make_view(const lat_kmap *m, bool flip) {
     v.ntiles = (m->n_out + LAT_TILE_ROWS - 1) / LAT_TILE_ROWS;
     v.k3 = m->k3;
     v.flip = flip ? 1 : 0;
+    // a submanifold query writes nbr[centre][j] = j (the row itself; flipping maps the
+    // centre to itself), so the kernels need not load that column
+    v.centre = (m->mode == LAT_SUBM && m->n_in == m->n_out) ? m->k3 / 2 : -1;
     return v;
 }
 

@@ -379,7 +379,9 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 int32_t *dst = &items[r].src[e * 32 + lane];
-                if (k >= 0 && rows[e] >= 0)
+                if (k >= 0 && k == mv.centre)
+                    *dst = rows[e];  // submanifold centre: every row is its own neighbour
+                else if (k >= 0 && rows[e] >= 0)
                     ptx::cp_async4(dst, mv.neighbour_ptr(k, rows[e]));
                 else
                     *dst = -1;
