@@ -525,13 +525,44 @@ static bool make_weight_map(CUtensorMap *map, const void *w, bool bf16, int k3, 
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The weight tensor map of (w, shape, type), remembered per host thread for the
+// last few weight tensors: encoding one is a driver call on every launch
+// otherwise.  A map holds only the address, sizes and strides, so reusing it
+// for the same (address, shape, type) is exact whatever the buffer holds.
+static bool weight_map(CUtensorMap *map, const void *w, bool bf16, int k3, int wrows, int wcols) {
+    struct Entry {
+        const void *w = nullptr;
+        int k3 = 0, rows = 0, cols = 0;
+        bool bf16 = false;
+        CUtensorMap map;
+    };
+    constexpr int kEntries = 8;
+    thread_local Entry cache[kEntries];
+    thread_local int next = 0;
+    for (const Entry &e : cache)
+        if (e.w == w && e.k3 == k3 && e.rows == wrows && e.cols == wcols && e.bf16 == bf16) {
+            *map = e.map;
+            return true;
+        }
+    if (!make_weight_map(map, w, bf16, k3, wrows, wcols)) return false;
+    Entry &e = cache[next];
+    next = (next + 1) % kEntries;
+    e.w = w;
+    e.k3 = k3;
+    e.rows = wrows;
+    e.cols = wcols;
+    e.bf16 = bf16;
+    e.map = *map;
+    return true;
+}
+
 template <typename T, int KC, int N, bool BMN>
 static lat_status launch(const void *x, const void *w, int k3, const MapView &mv, void *y, int32_t *counter,
                          int32_t *d_status, cudaStream_t s) {
     using C = Cfg<N>;
     CUtensorMap map;
     // forward: W[k] is (KC x N); data gradient: W[k] is (N x KC)
-    if (!make_weight_map(&map, w, is_bf16<T>(), k3, BMN ? KC : N, BMN ? N : KC)) return LAT_ERR_CUDA;
+    if (!weight_map(&map, w, is_bf16<T>(), k3, BMN ? KC : N, BMN ? N : KC)) return LAT_ERR_CUDA;
     auto kern = conv_tc_kernel<T, KC, N, BMN>;
     const int64_t grid = std::min<int64_t>(mv.ntiles, GridCache<KernelTag<T, KC, N, BMN>>::get(kern, C::kSmem, int(C::kTmemCols), 2));
     if (grid <= 0) return LAT_ERR_CUDA;
