@@ -351,7 +351,7 @@ typedef enum { LAT_POOL_MAX = 0, LAT_POOL_AVG = 1 } lat_pool_op;
  * lat_kmap_from_parent built (SUBM, strided or transposed geometry); only
  * nbr and mask are read, with map->n_in / n_out / k3 giving the sizes.
  *   x  device [n_in][c] of dtype; y device [n_out][c] of dtype (no overlap
- *      with x).  Both 16-byte aligned; c a multiple of 8 and >= 8.
+ *      with x).  Both 16-byte aligned; c a multiple of 8 in [8, 2048].
  *   Arithmetic is fp32; each output is rounded once to dtype.
  *   op is lat_pool_op.  Host checks return LAT_ERR_ARG; a row index outside
  *   [0, n_in) or a mask bit at or above k3 sets LAT_ERR_BAD_MAP at d_status
@@ -369,7 +369,8 @@ lat_status lat_sparse_pool(const void *x, int32_t c, const lat_kmap *map, int32_
  * of the rows wins, which one is unspecified.
  *   coords device int32 [n][4], 16-byte aligned; feats device [n][c];
  *   origin, shape host int32[3]; out device, 16-byte aligned,
- *   batch*shape[0]*shape[1]*shape[2]*c elements.  c a multiple of 8.
+ *   batch*shape[0]*shape[1]*shape[2]*c elements.  c a multiple of 8 in
+ *   [8, 2048]; n < 2^31.
  * Enqueues a memset of `out` and one scatter kernel on `stream`. */
 lat_status lat_to_dense(const int32_t *coords, int64_t n, const void *feats, int32_t c, lat_dtype dtype,
                         const int32_t *origin, const int32_t *shape, int32_t batch, void *out,

@@ -11,7 +11,8 @@
 //   dense: a channels-last grid over a caller-given box, zero where no row
 //          lies; every row inside the box writes its features to its cell.
 // Both are memory-bound gathers / scatters on CUDA cores: one thread per (row,
-// 8-channel group), 16-byte (fp16/bf16) or 2 x 16-byte (fp32) accesses.
+// 8-channel group) -- a 2D block, so no thread divides its index -- with
+// 16-byte (fp16/bf16) or 2 x 16-byte (fp32) accesses.
 #include "common.cuh"
 
 namespace lat {
@@ -59,11 +60,10 @@ __global__ void __launch_bounds__(256)
 pool_kernel(const T *__restrict__ x, int c, const int32_t *__restrict__ nbr, const uint32_t *__restrict__ mask,
             int k3, int64_t n_in, int64_t n_out, T *__restrict__ y, int32_t *d_status) {
     pdl_enter();
-    const int groups = c / 8;
-    const int64_t gid = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
-    const int64_t j = gid / groups;
+    // threadIdx.x = 8-channel group, threadIdx.y = row of the block
+    const int64_t j = blockIdx.x * int64_t(blockDim.y) + threadIdx.y;
     if (j >= n_out) return;
-    const int cg = int(gid - j * groups);
+    const int cg = threadIdx.x;
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = MAX ? -INFINITY : 0.f;
@@ -118,11 +118,9 @@ __global__ void __launch_bounds__(256)
 dense_scatter_kernel(const int4 *__restrict__ coords, int64_t n, const T *__restrict__ feats, int c, Box bx,
                      T *__restrict__ out, int32_t *d_status) {
     pdl_enter();
-    const int groups = c / 8;
-    const int64_t gid = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
-    const int64_t i = gid / groups;
+    const int64_t i = blockIdx.x * int64_t(blockDim.y) + threadIdx.y;
     if (i >= n) return;
-    const int cg = int(gid - i * groups);
+    const int cg = threadIdx.x;
     const int4 q = __ldg(coords + i);
     const int x = q.y - bx.ox, y = q.z - bx.oy, z = q.w - bx.oz;
     if (q.x < 0 || q.x >= bx.batch || x < 0 || x >= bx.sx || y < 0 || y >= bx.sy || z < 0 || z >= bx.sz) {
@@ -136,17 +134,24 @@ dense_scatter_kernel(const int4 *__restrict__ coords, int64_t n, const T *__rest
     for (int h = 0; h < int(sizeof(T) / 2); ++h) reinterpret_cast<uint4 *>(out + cell * c + cg * 8)[h] = v.v[h];
 }
 
+// Thread block of the pooling / dense kernels: x = the row's 8-channel groups
+// (c / 8 <= 256), y = rows, about 256 threads.
+static dim3 rows_block(int c) {
+    const int groups = c / 8;
+    return dim3(unsigned(groups), unsigned(groups >= 256 ? 1 : 256 / groups));
+}
+
 template <typename T>
 static lat_status launch_pool(const void *x, int c, const lat_kmap *map, int op, void *y, int32_t *d_status,
                               cudaStream_t s) {
-    const int64_t threads = map->n_out * (c / 8);
-    if (threads == 0) return LAT_OK;
-    const unsigned blocks = unsigned((threads + 255) / 256);
+    if (map->n_out == 0) return LAT_OK;
+    const dim3 block = rows_block(c);
+    const dim3 blocks(unsigned((map->n_out + block.y - 1) / block.y));
     if (op == LAT_POOL_MAX)
-        LAT_CUDA_TRY(launch_pdl(pool_kernel<T, true>, dim3(blocks), dim3(256), 0, s, static_cast<const T *>(x), c,
+        LAT_CUDA_TRY(launch_pdl(pool_kernel<T, true>, blocks, block, 0, s, static_cast<const T *>(x), c,
                                 map->nbr, map->mask, map->k3, map->n_in, map->n_out, static_cast<T *>(y), d_status));
     else
-        LAT_CUDA_TRY(launch_pdl(pool_kernel<T, false>, dim3(blocks), dim3(256), 0, s, static_cast<const T *>(x), c,
+        LAT_CUDA_TRY(launch_pdl(pool_kernel<T, false>, blocks, block, 0, s, static_cast<const T *>(x), c,
                                 map->nbr, map->mask, map->k3, map->n_in, map->n_out, static_cast<T *>(y), d_status));
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
@@ -157,9 +162,9 @@ static lat_status launch_dense(const int32_t *coords, int64_t n, const void *fea
                                int32_t *d_status, cudaStream_t s) {
     const size_t cells = size_t(bx.batch) * bx.sx * bx.sy * bx.sz;
     LAT_CUDA_TRY(cudaMemsetAsync(out, 0, cells * c * sizeof(T), s));
-    const int64_t threads = n * (c / 8);
-    if (threads == 0) return LAT_OK;
-    LAT_CUDA_TRY(launch_pdl(dense_scatter_kernel<T>, dim3(unsigned((threads + 255) / 256)), dim3(256), 0, s,
+    if (n == 0) return LAT_OK;
+    const dim3 block = rows_block(c);
+    LAT_CUDA_TRY(launch_pdl(dense_scatter_kernel<T>, dim3(unsigned((n + block.y - 1) / block.y)), block, 0, s,
                             reinterpret_cast<const int4 *>(coords), n, static_cast<const T *>(feats), c, bx,
                             static_cast<T *>(out), d_status));
     LAT_CUDA_TRY(cudaGetLastError());
@@ -175,10 +180,9 @@ extern "C" lat_status lat_sparse_pool(const void *x, int32_t c, const lat_kmap *
     using namespace lat;
     if (!map || map->k3 < 1 || map->k3 > 32 || map->n_in < 0 || map->n_out < 0) return LAT_ERR_ARG;
     if (map->n_out >= (int64_t(1) << 31) || map->n_in >= (int64_t(1) << 31)) return LAT_ERR_ARG;
-    if (c < 8 || c % 8 || (op != LAT_POOL_MAX && op != LAT_POOL_AVG)) return LAT_ERR_ARG;
+    if (c < 8 || c % 8 || c > 2048 || (op != LAT_POOL_MAX && op != LAT_POOL_AVG)) return LAT_ERR_ARG;
     if (map->n_out > 0 && (!map->nbr || !map->mask || !y || (map->n_in > 0 && !x))) return LAT_ERR_ARG;
     if (!aligned16(x) || !aligned16(y)) return LAT_ERR_ARG;
-    if (int64_t(map->n_out) * (c / 8) >= (int64_t(1) << 40)) return LAT_ERR_UNSUPPORTED;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     switch (dtype) {
         case LAT_F32: return launch_pool<float>(x, c, map, op, y, d_status, s);
@@ -192,7 +196,8 @@ extern "C" lat_status lat_to_dense(const int32_t *coords, int64_t n, const void 
                                    const int32_t *origin, const int32_t *shape, int32_t batch, void *out,
                                    int32_t *d_status, lat_stream stream) {
     using namespace lat;
-    if (n < 0 || c < 8 || c % 8 || !origin || !shape || batch < 1 || !out) return LAT_ERR_ARG;
+    if (n < 0 || n >= (int64_t(1) << 31) || c < 8 || c % 8 || c > 2048 || !origin || !shape || batch < 1 || !out)
+        return LAT_ERR_ARG;
     if (n > 0 && (!coords || !feats)) return LAT_ERR_ARG;
     for (int a = 0; a < 3; ++a)
         if (shape[a] < 1) return LAT_ERR_ARG;
