@@ -147,6 +147,73 @@ conv_simt_kernel(const T *__restrict__ x, int cin, const T *__restrict__ w, int 
     if (bad) flag(d_status, bad);
 }
 
+// Small problems (too few 128-row tiles to fill the GPU): one warp per output
+// row, lane k takes offset k, so a row's offsets are gathered in parallel
+// instead of one after another.  The block stages W transposed as
+// s_w[ci][co][k] (lanes read consecutive words: no bank conflicts); each lane
+// forms x[nbr[k][j]] . W[k] for the row's cout outputs and the warp sums the
+// offsets with a fixed xor-butterfly (deterministic).  Needs k3 <= 32,
+// cout <= 32 and cin * cout * 32 floats of shared memory.
+constexpr int kRowsPerBlock = 8;
+
+template <typename T, bool WT>
+__global__ void __launch_bounds__(kRowsPerBlock * 32)
+conv_rows_kernel(const T *__restrict__ x, int cin, const T *__restrict__ w, int cout, MapView mv,
+                 T *__restrict__ y, int32_t *d_status) {
+    pdl_enter();
+    extern __shared__ float s_w[];  // [cin][cout][32]
+    const int lane = threadIdx.x & 31;
+    for (int e = threadIdx.x; e < cin * cout * 32; e += blockDim.x) {
+        const int k = e & 31, co = (e >> 5) % cout, ci = (e >> 5) / cout;
+        float v = 0.f;
+        if (k < mv.k3) {
+            // (ci, co) of the GEMM: W[k][ci][co], or W[k][co][ci] for W^T
+            const T *wk = w + int64_t(k) * cin * cout;
+            v = WT ? Elem<T>::to_f(wk[int64_t(co) * cin + ci]) : Elem<T>::to_f(wk[int64_t(ci) * cout + co]);
+        }
+        s_w[e] = v;
+    }
+    __syncthreads();
+    const int64_t j = blockIdx.x * int64_t(kRowsPerBlock) + (threadIdx.x >> 5);
+    if (j >= mv.n_out) return;
+    int32_t bad = 0;
+    float acc[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) acc[c] = 0.f;
+    int src = lane < mv.k3 ? mv.neighbour(lane, j) : -1;
+    if (src >= mv.n_in) {
+        bad |= LAT_ERR_BAD_MAP;
+        src = -1;
+    }
+    if (src >= 0) {
+        const T *xr = x + int64_t(src) * cin;
+        for (int c0 = 0; c0 < cin; c0 += 8) {
+            float xv[8];
+            load8<T>(xr + c0, xv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float *wr = s_w + ((c0 + e) * cout) * 32 + lane;
+#pragma unroll
+                for (int co = 0; co < 32; ++co)
+                    if (co < cout) acc[co] = fmaf(xv[e], wr[co * 32], acc[co]);
+            }
+        }
+    }
+#pragma unroll
+    for (int co = 0; co < 32; ++co) {
+        if (co >= cout) break;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) acc[co] += __shfl_xor_sync(0xFFFFFFFFu, acc[co], o);
+    }
+    // lane co writes output channel co (every lane holds every total)
+    float mine = 0.f;
+#pragma unroll
+    for (int co = 0; co < 32; ++co)
+        if (co == lane) mine = acc[co];
+    if (lane < cout) y[j * cout + lane] = Elem<T>::from_f(mine);
+    if (bad) flag(d_status, bad);
+}
+
 // Work units of the weight gradient: fixed chunks of kWgradChunk pairs inside one offset.
 // First unit of every offset and the total (unit_base[k3]); one warp, lane k
 // handles offset k (k3 <= 32): offset k's clamped pairs make ceil(P_k / chunk) units.
@@ -290,6 +357,22 @@ lat_status launch_conv_simt(const void *x, int cin, const void *w, int cout, con
                             int32_t *d_status, cudaStream_t s) {
     if (mv.ntiles == 0) return LAT_OK;
     if (mv.ntiles >= (int64_t(1) << 31)) return LAT_ERR_UNSUPPORTED;
+    // too few tiles to fill the GPU: one warp per row, offsets across the lanes
+    const size_t rows_smem = sizeof(float) * size_t(cin) * size_t(cout) * 32;
+    if (mv.ntiles < 2 * int64_t(num_sms()) && mv.k3 <= 32 && cout <= 32 && rows_smem <= 96 * 1024) {
+        const dim3 grid(unsigned((mv.n_out + kRowsPerBlock - 1) / kRowsPerBlock)), block(kRowsPerBlock * 32);
+        auto go = [&](auto kern) -> cudaError_t {
+            if (rows_smem > 48 * 1024) {
+                const cudaError_t e =
+                    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(rows_smem));
+                if (e != cudaSuccess) return e;
+            }
+            return launch_pdl(kern, grid, block, rows_smem, s, static_cast<const T *>(x), cin,
+                              static_cast<const T *>(w), cout, mv, static_cast<T *>(y), d_status);
+        };
+        LAT_CUDA_TRY(wt ? go(conv_rows_kernel<T, true>) : go(conv_rows_kernel<T, false>));
+        return LAT_OK;
+    }
     const size_t smem = sizeof(float) * size_t(cin) * kCoChunk;
     if (wt)
         LAT_CUDA_TRY(launch_pdl(conv_simt_kernel<T, true>, dim3(unsigned(mv.ntiles)), dim3(LAT_TILE_ROWS), smem, s,
