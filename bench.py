@@ -232,16 +232,14 @@ class Pipeline:
 
 
 # The kernel the roofline object reports: the path kernel with the largest
-# share of the step's ncu launch list (serialised; the tcgen05 data-gradient
-# conv, 8.2% of the step's kernel time and the largest of the path's kernels).
-DOMINANT_KERNEL = "dgrad"
+# share of the step's ncu launch list (serialised; the tcgen05 strided Conv3d
+# 64 -> 128, 7.1% of the step's kernel time, the largest of the path's kernels).
+DOMINANT_KERNEL = "down_fwd"
 
 # DRAM bytes per launch from that ncu launch list of this workload (caches not
-# flushed between kernels): the dgrad conv (its DRAM writes include the
-# write-back of the forward pass's output, evicted while it runs) and the
-# submanifold kmap query's kernels summed; None where no capture matches the
-# current kernels.
-PHASE_TRAFFIC = {"dgrad": 77.1e6, "kmap": 26.8e6}
+# flushed between kernels): the strided conv, and the submanifold kmap query's
+# kernels summed; None where no capture matches the current kernels.
+PHASE_TRAFFIC = {"down_fwd": 71.9e6, "kmap": 26.8e6}
 
 
 def flush_l2(buf: torch.Tensor):
@@ -477,6 +475,18 @@ def run_only(args):
         P = int(km_dn.pair_off[8].item())
         ops["pool_down"] = (lambda: scv.lat_sparse_pool(x, km_dn.c, scv.LAT_POOL_MAX, y_dn, st),
                             (n + coarse_p.shape[0]) * cin * e + 4 * coarse_p.shape[0] + 4 * P)
+    if args.only == "down_fwd":
+        # strided Conv3d k2s2 Cin -> Cout onto the generated coarse support (maps from parents)
+        g_dn = scv.strided_geom(2, 2, 0)
+        coarse_d, par = scv.downsample(coords, g_dn, ws, with_parent=True)
+        ncd = coarse_d.shape[0]
+        km_d, _ = scv.maps_from_parent(coords, par.contiguous(), ncd, g_dn, ws, st)
+        wd = torch.from_numpy(synthetic.weights(8, cin, cout, wl.seed)).to(dt).to(dev)
+        yd = torch.empty((ncd, cout), dtype=dt, device=dev)
+        wsd = torch.empty(max(1, scv.lat_sconv_ws_bytes(0, cin, cout, km_d.c, dt)), dtype=torch.uint8, device=dev)
+        torch.cuda.synchronize()
+        ops["down_fwd"] = (lambda: scv.lat_sconv_fwd(x, wd, km_d.c, yd, wsd, st),
+                           n * cin * e + ncd * cout * e + 8 * cin * cout * e + 8 * n)
     if args.only == "dense":
         # dense grid over the coordinates' bounding box: the whole grid written once, rows read once
         lo, hi = coords.amin(0).tolist(), coords.amax(0).tolist()
@@ -529,7 +539,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["hash", "kmap", "fwd", "dgrad", "wgrad", "downsample", "upsample", "pool_max",
-                                       "pool_avg", "pool_down", "dense"],
+                                       "pool_avg", "pool_down", "dense", "down_fwd"],
                     help="time a single op of the path on --workload (for profiler captures)")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(synthetic.WORKLOADS))
     ap.add_argument("--rsv-ratio", type=float, default=RSV_RATIO, help="hash table slots per voxel (--only mode)")
@@ -627,7 +637,7 @@ def main():
             "phase_ms": {k: round(v, 4) for k, v in phase_ms_inst.items()},
             "phase_ms_note": "per-phase event times from instrumented steps outside the timed region "
                              "(the two chains overlap, so phases do not add up to the step)",
-            "roofline": {"kernel": f"{dominant} (conv_tc_kernel: gather dy, W^T on tcgen05)", "bound": "hbm",
+            "roofline": {"kernel": f"{dominant} (conv_tc_kernel, strided Conv3d 64->128 on tcgen05)", "bound": "hbm",
                          "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm, "traffic": PHASE_TRAFFIC.get(dominant),
                          "alg_bytes": pb[dominant], "ms": dominant_ms, "peak_source": f"{src} hbm_gbs",
