@@ -476,17 +476,19 @@ def run_only(args):
         ops["pool_down"] = (lambda: scv.lat_sparse_pool(x, km_dn.c, scv.LAT_POOL_MAX, y_dn, st),
                             (n + coarse_p.shape[0]) * cin * e + 4 * coarse_p.shape[0] + 4 * P)
     if args.only == "down_fwd":
-        # strided Conv3d k2s2 Cin -> Cout onto the generated coarse support (maps from parents)
+        # strided Conv3d k2s2 Cin -> 2 Cin onto the generated coarse support (maps from
+        # parents): on lidar_subm the bench step's fp16 64 -> 128 down conv
         g_dn = scv.strided_geom(2, 2, 0)
         coarse_d, par = scv.downsample(coords, g_dn, ws, with_parent=True)
         ncd = coarse_d.shape[0]
         km_d, _ = scv.maps_from_parent(coords, par.contiguous(), ncd, g_dn, ws, st)
-        wd = torch.from_numpy(synthetic.weights(8, cin, cout, wl.seed)).to(dt).to(dev)
-        yd = torch.empty((ncd, cout), dtype=dt, device=dev)
-        wsd = torch.empty(max(1, scv.lat_sconv_ws_bytes(0, cin, cout, km_d.c, dt)), dtype=torch.uint8, device=dev)
+        cd = 2 * cin
+        wd = torch.from_numpy(synthetic.weights(8, cin, cd, wl.seed)).to(dt).to(dev)
+        yd = torch.empty((ncd, cd), dtype=dt, device=dev)
+        wsd = torch.empty(max(1, scv.lat_sconv_ws_bytes(0, cin, cd, km_d.c, dt)), dtype=torch.uint8, device=dev)
         torch.cuda.synchronize()
         ops["down_fwd"] = (lambda: scv.lat_sconv_fwd(x, wd, km_d.c, yd, wsd, st),
-                           n * cin * e + ncd * cout * e + 8 * cin * cout * e + 8 * n)
+                           n * cin * e + ncd * cd * e + 8 * cin * cd * e + 8 * n)
     if args.only == "dense":
         # dense grid over the coordinates' bounding box: the whole grid written once, rows read once
         lo, hi = coords.amin(0).tolist(), coords.amax(0).tolist()
