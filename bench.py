@@ -152,6 +152,7 @@ class Pipeline:
                                              scv.lat_sconv_ws_bytes(0, CIN, CMID, self.km_down.c, torch.half),
                                              scv.lat_sconv_ws_bytes(0, CMID, CIN, self.km_up.c, torch.half)))
         self.nc_host = torch.empty(1, dtype=torch.int64, pin_memory=True)
+        self.nc_view = self.nc_host.numpy()  # read without building a tensor each step
         self.nc_ready = torch.cuda.Event()
         self.pairs = None
 
@@ -183,7 +184,7 @@ class Pipeline:
         scv.lat_sconv_fwd(d["x"], d["w"], self.km.c, self.y, self.wsb, s)
         rec("fwd", 1, main)
         self.nc_ready.synchronize()
-        nc = int(self.nc_host[0])
+        nc = int(self.nc_view[0])
         if nc < 0:  # coarse fields too wide for the bitmap: blocking radix-sort path
             nc = scv.lat_downsample_coords(d["coords"], self.g_down, self.coarse_buf, self.wsb_side, s,
                                            stream=side, parent=self.parent)
