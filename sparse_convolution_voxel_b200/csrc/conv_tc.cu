@@ -171,6 +171,7 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    const bool y32 = (reinterpret_cast<uintptr_t>(y) & 31) == 0;  // 256-bit stores of output slices
     int32_t bad = 0;
 
     if (warp < kProdWarps) {
@@ -256,12 +257,22 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x
             }
             ptx::tc_fence_after();
             const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + a * N;
-            // Coalesced write-back: each 16-channel slice of the warp's 32 rows goes
-            // through a 1 KB staging buffer (32 B per row, the two 16-byte halves
-            // swapped on every other group of 4 rows against bank conflicts), then
-            // lane pairs write whole 32-byte sectors of one row.
+            // Write-back of each 16-channel slice (32 B of a row).  With a 32-byte
+            // aligned output every lane stores its own row's slice with one 256-bit
+            // store: a whole 32-byte sector per lane, no staging.  Otherwise the
+            // warp's 32 rows go through a 1 KB staging buffer (the two 16-byte
+            // halves swapped on every other group of 4 rows against bank
+            // conflicts) and lane pairs write whole 32-byte sectors of one row.
             uint8_t *stg = smem + C::kStgOff + q * 1024;
             auto write_slice = [&](const uint32_t (&v)[16], int col) {
+                if (y32) {
+                    uint32_t o[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        o[e] = pack2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]), T{});
+                    if (j >= 0) ptx::st_global_v8(y + int64_t(j) * N + col, o);
+                    return;
+                }
                 uint4 o0, o1;
                 o0.x = pack2(__uint_as_float(v[0]), __uint_as_float(v[1]), T{});
                 o0.y = pack2(__uint_as_float(v[2]), __uint_as_float(v[3]), T{});

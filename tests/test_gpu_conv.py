@@ -275,3 +275,25 @@ def test_generative_transposed_conv(dtype, ks, st_, pd):
     scv.check_status(st)
     assert_close(dx.double().cpu().numpy(), oracle.conv_dgrad(gy64, w64, ref_nbr, len(coarse)), dtype,
                  "generative transposed dgrad")
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("cout", [64, 128])
+def test_tc_fwd_output_16_byte_aligned(dtype, cout):
+    """The tensor-core epilogue stores 32-byte slices when the output is 32-byte
+    aligned and stages them otherwise: an output view 16 bytes into a buffer
+    gives the same bits as an aligned one."""
+    rng = np.random.default_rng(61)
+    coords = rand_coords(rng, 900, -7, 7, 2)
+    km, ref_nbr = _subm_map(coords)
+    x, x64 = feats(len(coords), 64, dtype, seed=61)
+    w, w64 = weights(27, 64, cout, dtype, seed=61)
+    y_al = scv.conv_fwd(x, w, km)
+    flat = torch.full((len(coords) * cout + 8,), 7.0, dtype=dtype, device="cuda")
+    y_off = flat[8:].view(len(coords), cout)
+    assert y_off.data_ptr() % 32 == 16
+    scv.conv_fwd(x, w, km, out=y_off)
+    torch.cuda.synchronize()
+    assert torch.equal(y_al, y_off)
+    assert torch.all(flat[:8] == 7.0)
+    assert_close(y_al.double().cpu().numpy(), oracle.conv_fwd(x64, w64, ref_nbr), dtype, "aligned fwd")
