@@ -234,13 +234,13 @@ class Pipeline:
 
 # The kernel the roofline object reports: the path kernel with the largest
 # share of the step's ncu launch list (serialised; the tcgen05 strided Conv3d
-# 64 -> 128, 7.1% of the step's kernel time, the largest of the path's kernels).
+# 64 -> 128, 6.9% of the step's kernel time, the largest of the path's kernels).
 DOMINANT_KERNEL = "down_fwd"
 
 # DRAM bytes per launch from that ncu launch list of this workload (caches not
 # flushed between kernels): the strided conv, and the submanifold kmap query's
 # kernels summed; None where no capture matches the current kernels.
-PHASE_TRAFFIC = {"down_fwd": 71.9e6, "kmap": 26.8e6}
+PHASE_TRAFFIC = {"down_fwd": 72.3e6, "kmap": 27.2e6}
 
 
 def flush_l2(buf: torch.Tensor):
