@@ -113,3 +113,19 @@ def test_pool_and_dense_argument_checks_without_gpu(lib):
     assert lib.lat_to_dense(None, 5, P(16), 8, 0, o, sh, 1, P(16), None, None) == 1
     assert lib.lat_to_dense(P(8), 5, P(16), 8, 0, o, sh, 1, P(16), None, None) == 1    # coords alignment
     assert lib.lat_to_dense(P(16), 5, P(16), 8, 3, o, sh, 1, P(16), None, None) == 1   # dtype
+
+
+def test_binding_rejects_host_tensors(lib):
+    """The binding only marshals device pointers: a host tensor fails loudly
+    (no CPU fallback) before anything reaches the library."""
+    import torch
+    km = scv.KernelMap.__new__(scv.KernelMap)  # the struct alone; no device buffers needed
+    km.c = _lib.lat_kmap()
+    km.c.k3, km.c.n_out, km.c.n_in = 27, 4, 4
+    x = torch.zeros((4, 16))
+    with pytest.raises(ValueError, match="device tensors"):
+        _lib.lat_sparse_pool(x, km.c, 0, torch.zeros((4, 16)))
+    with pytest.raises(ValueError, match="device tensors"):
+        _lib.lat_sconv_fwd(x, torch.zeros((27, 16, 16)), km.c, torch.zeros((4, 16)))
+    with pytest.raises(ValueError, match="device tensors"):
+        _lib.lat_hash_build(torch.zeros((4, 4), dtype=torch.int32), torch.zeros(64, dtype=torch.int64))
