@@ -460,7 +460,8 @@ def test_to_dense_matches_sparse_coo_to_dense():
     rel = c.astype(np.int64) - np.array((0,) + origin)
     inside = (rel[:, 0] < batch) & np.all(rel[:, 1:] >= 0, 1) & np.all(rel[:, 1:] < np.array(shape), 1)
     assert outside == int((~inside).sum()) > 0
-    ref = torch.sparse_coo_tensor(torch.as_tensor(rel[inside].T), torch.as_tensor(x[inside]),
-                                  (batch,) + shape + (4,), check_invariants=True).to_dense()
+    with torch.sparse.check_sparse_tensor_invariants():
+        ref = torch.sparse_coo_tensor(torch.as_tensor(rel[inside].T), torch.as_tensor(x[inside]),
+                                      (batch,) + shape + (4,)).to_dense()
     np.testing.assert_array_equal(grid, ref.numpy())
     assert np.count_nonzero(np.any(grid != 0, axis=-1)) == int(inside.sum())
