@@ -243,7 +243,10 @@ def conv_wgrad(x, dy, kmap: KernelMap, ws: Workspace | None = None, d_status=Non
 
 def sparse_pool(x, kmap: KernelMap, op: str = "max", d_status=None, out=None, stream=None):
     """Max or mean of x over each output row's neighbours in ``kmap`` (0 where it has none)."""
-    code = {"max": LAT_POOL_MAX, "avg": LAT_POOL_AVG, "mean": LAT_POOL_AVG}[op]
+    codes = {"max": LAT_POOL_MAX, "avg": LAT_POOL_AVG, "mean": LAT_POOL_AVG}
+    if op not in codes:
+        raise ValueError(f"pooling op must be one of {sorted(codes)}, not {op!r}")
+    code = codes[op]
     y = out if out is not None else torch.empty((kmap.n_out, x.shape[1]), dtype=x.dtype, device=x.device)
     lat_sparse_pool(x, kmap.c, code, y, d_status, stream)
     return y

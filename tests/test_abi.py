@@ -129,3 +129,12 @@ def test_binding_rejects_host_tensors(lib):
         _lib.lat_sconv_fwd(x, torch.zeros((27, 16, 16)), km.c, torch.zeros((4, 16)))
     with pytest.raises(ValueError, match="device tensors"):
         _lib.lat_hash_build(torch.zeros((4, 4), dtype=torch.int32), torch.zeros(64, dtype=torch.int64))
+
+
+def test_pool_helper_rejects_unknown_op(lib):
+    import torch
+    km = scv.KernelMap.__new__(scv.KernelMap)
+    km.c = _lib.lat_kmap()
+    km.n_out = 4
+    with pytest.raises(ValueError, match="pooling op"):
+        scv.sparse_pool(torch.zeros((4, 16)), km, "sum", out=torch.zeros((4, 16)))
