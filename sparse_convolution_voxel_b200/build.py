@@ -1,9 +1,11 @@
 """Compile liblattice.so in-tree for sm_100a with nvcc.
 
 Every ``csrc/*.cu`` is compiled to an object under ``_build/`` (in parallel)
-and linked into ``sparse_convolution_voxel_b200/liblattice.so``.  Objects
-are rebuilt when their source, any ``csrc/*.cuh`` or ``include/lattice.h``
-is newer.
+and linked into ``sparse_convolution_voxel_b200/liblattice.so``; the
+measurement kernels under ``measure/`` (device peaks for the benchmark's
+roofline, not part of the library) go into ``measure/libmeasure.so``.
+Objects are rebuilt when their source, any ``csrc/*.cuh`` or
+``include/*.h`` is newer.
 """
 from __future__ import annotations
 
@@ -20,6 +22,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "liblattice.so")
+MEASURE = os.path.join(PKG, "measure")
+MEASURE_LIB = os.path.join(MEASURE, "libmeasure.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
@@ -34,7 +38,7 @@ def nvcc() -> str:
 
 
 def _deps_mtime() -> float:
-    files = glob.glob(os.path.join(CSRC, "*.cuh")) + [os.path.join(INCLUDE, "lattice.h")]
+    files = glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
     return max(os.path.getmtime(f) for f in files)
 
 
@@ -52,18 +56,25 @@ def _compile(src: str, extra: list[str]) -> str:
     return obj
 
 
-def build(verbose: bool = False, extra: list[str] | None = None) -> str:
-    os.makedirs(BUILD, exist_ok=True)
-    srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
-    with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 4)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, extra or []), srcs))
-    if not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+def _link(objs: list[str], lib: str):
+    if not os.path.exists(lib) or os.path.getmtime(lib) < max(os.path.getmtime(o) for o in objs):
+        tmp = lib + f".tmp{os.getpid()}"
         cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", *objs, "-o", tmp, "-lcudart"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stderr}")
-        os.replace(tmp, LIB)
+        os.replace(tmp, lib)
+
+
+def build(verbose: bool = False, extra: list[str] | None = None) -> str:
+    os.makedirs(BUILD, exist_ok=True)
+    srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    msrcs = sorted(glob.glob(os.path.join(MEASURE, "*.cu")))
+    with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 4)) as ex:
+        objs = list(ex.map(lambda s: _compile(s, extra or []), srcs + msrcs))
+    _link(objs[:len(srcs)], LIB)
+    if msrcs:
+        _link(objs[len(srcs):], MEASURE_LIB)
     if verbose:
         print(LIB)
     return LIB

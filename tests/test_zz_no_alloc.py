@@ -13,7 +13,8 @@ import numpy as np
 import pytest
 import torch
 
-from tests.util import assert_close, feats, rand_coords
+import oracle
+from tests.util import assert_close, feats, rand_coords, with_terms
 
 pytestmark = pytest.mark.gpu
 
@@ -28,30 +29,40 @@ def _map(coords):
     return km
 
 
+def _static_wgrad(x, g, km, cin, cout, dtype):
+    dw = torch.full((27, cin, cout), float("nan"), dtype=torch.float32, device="cuda")
+    st = scv.new_status()
+    rc = scv.load().lat_sconv_wgrad_static(ctypes.c_void_p(x.data_ptr()), cin, ctypes.c_void_p(g.data_ptr()), cout,
+                                           ctypes.byref(km.c), ctypes.c_void_p(dw.data_ptr()),
+                                           scv._lib.dtype_code(dtype), ctypes.c_void_p(st.data_ptr()),
+                                           ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0, scv.lat_status_string(rc)
+    scv.check_status(st)
+    return dw
+
+
 @pytest.mark.parametrize("dtype,cin,cout", [(torch.float16, 64, 64), (torch.bfloat16, 128, 128),
-                                            (torch.float32, 16, 32)])
-def test_static_scratch_wgrad_matches_workspace_wgrad_twice(dtype, cin, cout):
+                                            (torch.float32, 16, 32), (torch.float32, 8, 32)])
+def test_static_scratch_wgrad_matches_oracle_twice(dtype, cin, cout):
+    """Two calls in a row, each against the fp64 oracle; on the shapes where
+    lat_sconv_wgrad also runs on the CUDA cores (fp32 here) both entry points
+    run the same kernels in the same order, so their dW must agree bit for bit."""
     scv.load()
     rng = np.random.default_rng(cin + cout)
     coords = rand_coords(rng, 4000, -12, 12, 2)
     km = _map(coords)
-    x, _ = feats(len(coords), cin, dtype, seed=41)
-    g, _ = feats(len(coords), cout, dtype, seed=41, stream=1)
-    ref = scv.conv_wgrad(x, g, km).double().cpu().numpy()
-    lib = scv.load()
+    ref_nbr = oracle.kmap(coords, coords, 3, 1, 1, oracle.SUBM)
+    x, x64 = feats(len(coords), cin, dtype, seed=41)
+    g, g64 = feats(len(coords), cout, dtype, seed=41, stream=1)
+    ref = with_terms(oracle.conv_wgrad, x64, g64, ref_nbr)
     outs = []
     for _ in range(2):
-        dw = torch.full((27, cin, cout), float("nan"), dtype=torch.float32, device="cuda")
-        st = scv.new_status()
-        rc = lib.lat_sconv_wgrad_static(ctypes.c_void_p(x.data_ptr()), cin, ctypes.c_void_p(g.data_ptr()), cout,
-                                        ctypes.byref(km.c), ctypes.c_void_p(dw.data_ptr()),
-                                        scv._lib.dtype_code(dtype), ctypes.c_void_p(st.data_ptr()),
-                                        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
-        assert rc == 0, scv.lat_status_string(rc)
-        scv.check_status(st)
-        outs.append(dw.double().cpu().numpy())
-        assert_close(outs[-1], ref, dtype, "static-scratch wgrad")
-    assert_close(outs[1], outs[0], dtype, "second call")
+        dw = _static_wgrad(x, g, km, cin, cout, dtype)
+        outs.append(dw)
+        assert_close(dw.double().cpu().numpy(), ref, dtype, "static-scratch wgrad")
+    assert torch.equal(outs[0], outs[1]), "the second call differs from the first"
+    if dtype == torch.float32:
+        assert torch.equal(outs[0], scv.conv_wgrad(x, g, km)), "differs from lat_sconv_wgrad on CUDA-core shapes"
 
 
 def test_static_scratch_wgrad_rejects_problems_above_its_limit():

@@ -1,5 +1,9 @@
-"""Shared helpers for the parity tests: seeded inputs, layout conversion, tolerances."""
+"""Shared helpers for the parity tests: seeded inputs, layout conversion, tolerances,
+and the per-element error statistics reported beside every feature check."""
 from __future__ import annotations
+
+import json
+import os
 
 import numpy as np
 import torch
@@ -23,7 +27,46 @@ def weights(k3: int, cin: int, cout: int, dtype: torch.dtype, seed: int, stream:
     return t.to(device), t.double().numpy()
 
 
+# Error statistics of every check made with a reference that carries its terms
+# (see with_terms): kept for the session summary, and appended as JSON lines to
+# the file named by LAT_ERR_REPORT when that variable is set.
+ERROR_LOG: list[dict] = []
+
+
+class _Ref(np.ndarray):
+    """An oracle result that also carries, per element, the sum of the absolute
+    values of the terms summed into it (``terms``)."""
+    terms = None
+
+
+def with_terms(fn, *args, **kw) -> np.ndarray:
+    """fn(*args) (an oracle routine that sums products of its float inputs) with
+    ``.terms`` = the same routine on the absolute values of those inputs, which
+    is, element by element, the sum of |term| over the terms of that element."""
+    ref = np.asarray(fn(*args, **kw), np.float64).view(_Ref)
+    absargs = [np.abs(a) if isinstance(a, np.ndarray) and a.dtype.kind == "f" else a for a in args]
+    ref.terms = np.asarray(fn(*absargs, **kw), np.float64)
+    return ref
+
+
+def error_stats(got: np.ndarray, ref: np.ndarray, terms: np.ndarray) -> dict:
+    """Per-element |got - ref| / sum|terms| over the elements that have a term:
+    median, 99th percentile and maximum (the validation of CUDA results against
+    another backend by percentile error statistics)."""
+    err = np.abs(np.asarray(got, np.float64) - np.asarray(ref, np.float64))
+    sel = terms > 0
+    rel = err[sel] / terms[sel]
+    if rel.size == 0:
+        return {"rel_terms_p50": 0.0, "rel_terms_p99": 0.0, "rel_terms_max": 0.0, "elements": 0}
+    p50, p99 = np.percentile(rel, [50, 99])
+    return {"rel_terms_p50": float(p50), "rel_terms_p99": float(p99), "rel_terms_max": float(rel.max()),
+            "elements": int(rel.size)}
+
+
 def assert_close(got: np.ndarray, ref: np.ndarray, dtype: torch.dtype, what: str = ""):
+    """Normwise check max|got - ref| <= tol(dtype) * max|ref|; when ``ref`` carries
+    its terms (with_terms), the per-element error statistics are recorded too."""
+    terms = getattr(ref, "terms", None)
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     assert got.shape == ref.shape, (got.shape, ref.shape)
@@ -31,6 +74,15 @@ def assert_close(got: np.ndarray, ref: np.ndarray, dtype: torch.dtype, what: str
     scale = max(np.abs(ref).max(initial=0.0), 1e-30)
     err = np.abs(got - ref).max(initial=0.0)
     tol = REL_TOL[dtype]
+    if terms is not None:
+        rec = {"test": os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0], "what": what,
+               "dtype": str(dtype).replace("torch.", ""), "max_err_over_max_ref": float(err / scale), "tol": tol,
+               **error_stats(got, ref, terms)}
+        ERROR_LOG.append(rec)
+        path = os.environ.get("LAT_ERR_REPORT")
+        if path:
+            with open(path, "a") as f:
+                f.write(json.dumps(rec) + "\n")
     assert err <= tol * scale, f"{what}: max|err| {err:.3e} > {tol:g} * max|ref| {scale:.3e}"
     return err / scale
 
