@@ -968,12 +968,13 @@ def main():
     value = job_throughput(flops, world, args.steps, total_ms)
 
     if rank == 0:
-        fp32 = None
-        try:
-            from sparse_convolution_voxel_b200 import measure
-            fp32 = measure.ffma_peak(dev)
-        except Exception as exc:  # the probe library is optional for the headline
-            fp32 = {"error": str(exc)}
+        fp32 = {"skipped": "--lean"}
+        if not args.lean:
+            try:
+                from sparse_convolution_voxel_b200 import measure
+                fp32 = measure.ffma_peak(dev)
+            except Exception as exc:  # the probe library is optional for the headline
+                fp32 = {"error": str(exc)}
         fp32_tflops = fp32.get("tflops")
         rl = roofline_of(layer, pms, peaks, fp32_tflops)
         pb = layer.phase_bytes()

@@ -150,10 +150,13 @@ typedef struct {
  * slots, 16 bytes of table each, stored as 64-byte groups of 4 slots
  * {uint64 key[4]; uint32 row[4]; uint32 unused[4]}: slot s is entry s % 4
  * of group s / 4.  An empty slot holds key 0xFFFF...F.  A key's home slot is
- * a 32-bit mix of the key (its two halves folded, then the MurmurHash3
- * fmix32 finalizer) masked to the slot count; its probe sequence starts at
- * the first slot of the home slot's group and runs over consecutive slots
- * (linear probing), so a lookup reads whole groups.  A key is stored within
+ * a 32-bit mix of its z-brick -- the key with the two low bits of the z
+ * field cleared, so the 4 cells z = 4m..4m+3 of one (b, x, y) column share
+ * it -- (the two halves folded, then the MurmurHash3 fmix32 finalizer)
+ * masked to the slot count; its probe sequence starts at the first slot of
+ * the home slot's group and runs over consecutive slots (linear probing), so
+ * a lookup reads whole groups, and one group read answers the z-neighbours
+ * of a cell that share its brick.  A key is stored within
  * 4096 slots of the start of its home group (anywhere in a smaller table);
  * an insert that finds no free slot in that window flags
  * LAT_ERR_TABLE_FULL (only a table filled close to capacity gets there), and
@@ -295,10 +298,12 @@ lat_status lat_sconv_dgrad(const void *dy, int32_t cout, const void *w, int32_t 
 /* Per-offset weight gradient: dW[k] = sum over pairs (i, j) of offset k of
  * x[i]^T dy[j], fp32 (k3, cin, cout), from the forward map's pair lists.
  * Deterministic: the pair list is cut into a fixed number of equal
- * contiguous shares (fixed chunks on the CUDA-core path), each share is
+ * contiguous shares (296 on the tensor cores; on the CUDA cores 1184 when
+ * cin*cout <= 2048, else 296; never more shares than pairs), each share is
  * reduced into fp32 partials (one per offset it meets), and the partials are
- * summed in a fixed order (no atomics), so the bits do not depend on timing
- * or on the number of SMs. */
+ * summed in a fixed order (no atomics), so the bits do not depend on timing,
+ * on the number of SMs or on pair_capacity.  The scratch holds
+ * (shares + k3) partials of cin*cout fp32, whatever the pair count. */
 lat_status lat_sconv_wgrad(const void *x, int32_t cin, const void *dy, int32_t cout,
                            const lat_kmap *map, float *dw, lat_dtype dtype, void *ws,
                            size_t ws_bytes, int32_t *d_status, lat_stream stream);
@@ -312,21 +317,22 @@ lat_status lat_sconv_wgrad(const void *x, int32_t cin, const void *dy, int32_t c
  * synchronise the whole device) once running, or hosts whose device
  * allocator belongs to another runtime.  This entry point computes dW with
  * the CUDA-core weight-gradient kernels (those lat_sconv_wgrad runs for fp32
- * and for the shapes the tensor cores do not take; same chunking, same
+ * and for the shapes the tensor cores do not take; same shares, same
  * summation order, so the same bits there; for the tensor-core shapes of
  * lat_sconv_wgrad the two agree within fp32 rounding, not bit for bit) and
  * takes no `ws`: its scratch is one static device array of
  * LAT_WGRAD_STATIC_SCRATCH_BYTES (32 MiB) inside the library, which every
  * GPU that loads the library keeps until the process exits.  It allocates
  * nothing and calls no allocating routine.
- *   - Limit: the scratch must hold (k3 + 1) int32 plus
- *     (ceil(pair_capacity / 1024) + k3) fp32 partials of cin*cout; larger
- *     problems return LAT_ERR_WORKSPACE before anything is enqueued (e.g.
- *     cin = cout = 64 allows about 2.07 million pair slots, 128 x 128
- *     about 496 thousand).
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture begins.
+ *   - Limit: the scratch must hold (shares + k3) fp32 partials of cin*cout
+ *     (shares as for lat_sconv_wgrad above); it does not depend on the row
+ *     or pair count.  With k3 = 27 that allows cin*cout up to 25,970 (every
+ *     shape up to 128 x 192); larger shapes return LAT_ERR_WORKSPACE before
+ *     anything is enqueued.
+ *   - The first successful call on each device looks up the array's device
+ *     address (cudaGetSymbolAddress) with that device current and keeps it;
+ *     make that first call before any stream capture begins.  A failed
+ *     lookup returns LAT_ERR_CUDA and is tried again on the next call.
  *   - All calls share the one array and it keeps the last call's contents;
  *     every byte a call reads is written earlier by the same call, so no
  *     clearing is needed.  Calls whose work overlaps on the GPU (different
@@ -386,6 +392,18 @@ const char *lat_status_string(int32_t status);
 
 /* Library ABI version (major*100 + minor). */
 int32_t lat_version(void);
+
+/* Failure detection: limit, in nanoseconds, of every barrier wait in the
+ * tensor-core kernels (the fp16 / bf16 convolution and weight-gradient
+ * passes); 2 s by default.  A wait that runs out flags LAT_ERR_TIMEOUT at
+ * d_status; its CTA then waits (with a separate 1 s limit) for the tensor
+ * memory accelerator loads and MMAs it still has in flight, frees its tensor
+ * memory and exits, so the context stays usable and later calls run
+ * normally.  The outputs of a call that timed out are undefined.  0 makes
+ * every wait that is not already complete give up at once (tests use it to
+ * run the timeout path without faulting or hanging anything).  One
+ * process-wide value, read at each launch; returns the previous one. */
+uint64_t lat_set_wait_limit_ns(uint64_t ns);
 
 #ifdef __cplusplus
 }

@@ -21,7 +21,8 @@ from ._lib import (  # noqa: F401  (re-exported C entry points and constants)
     lat_upsample_coords, lat_upsample_ws_bytes,
     lat_hash_build, lat_hash_bytes, lat_kmap, lat_kmap_from_parent, lat_kmap_from_parent_ws_bytes, lat_kmap_query,
     lat_kmap_ws_bytes, lat_sconv_dgrad, lat_sconv_fwd, lat_sparse_pool, lat_to_dense,
-    lat_sconv_wgrad, lat_sconv_wgrad_static, lat_sconv_ws_bytes, lat_status_fetch, lat_status_string, lat_version, load, make_geom,
+    lat_sconv_wgrad, lat_sconv_wgrad_static, lat_sconv_ws_bytes, lat_set_wait_limit_ns, lat_status_fetch,
+    lat_status_string, lat_version, load, make_geom,
 )
 
 __all__ = [

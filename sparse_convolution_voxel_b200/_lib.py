@@ -37,7 +37,7 @@ EXPORTS = [
     "lat_kmap_from_parent",
     "lat_sconv_ws_bytes", "lat_sconv_fwd",
     "lat_sconv_dgrad", "lat_sconv_wgrad", "lat_sconv_wgrad_static", "lat_sparse_pool", "lat_to_dense",
-    "lat_status_fetch", "lat_status_string", "lat_version",
+    "lat_status_fetch", "lat_status_string", "lat_version", "lat_set_wait_limit_ns",
 ]
 
 
@@ -96,6 +96,7 @@ def load() -> ctypes.CDLL:
         "lat_status_fetch": (I32, [P, P]),
         "lat_status_string": (ctypes.c_char_p, [I32]),
         "lat_version": (I32, []),
+        "lat_set_wait_limit_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -296,3 +297,8 @@ def lat_status_string(status: int) -> str:
 
 def lat_version() -> int:
     return int(load().lat_version())
+
+
+def lat_set_wait_limit_ns(ns: int) -> int:
+    """Limit of every barrier wait in the tensor-core kernels (ns); returns the previous limit."""
+    return int(load().lat_set_wait_limit_ns(int(ns)))

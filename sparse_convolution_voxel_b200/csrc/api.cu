@@ -126,3 +126,5 @@ extern "C" const char *lat_status_string(int32_t status) {
 }
 
 extern "C" int32_t lat_version(void) { return 100; }
+
+extern "C" uint64_t lat_set_wait_limit_ns(uint64_t ns) { return lat::wait_limit_store().exchange(ns); }

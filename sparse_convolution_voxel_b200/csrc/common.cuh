@@ -6,6 +6,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 #include <utility>
 
@@ -74,8 +75,18 @@ __device__ __forceinline__ uint32_t probe_window(uint32_t cap_mask) {
     return cap_mask < kMaxProbeSlots - 1 ? cap_mask + 1 : kMaxProbeSlots;
 }
 
+// The home slot is the hash of the key's z-brick, the key with the low two bits
+// of its z field cleared: the (up to) 4 cells of one z-run share a probe
+// sequence, so a lookup of the z-neighbours of a cell (the 3 offsets of one
+// kernel column) reads one group (two when the run crosses a brick edge).
 __device__ __forceinline__ uint32_t probe_start(uint64_t key, uint32_t cap_mask) {
-    return slot_hash(key) & cap_mask & ~uint32_t(kGroupSlots - 1);
+    return slot_hash(key & ~uint64_t(3)) & cap_mask & ~uint32_t(kGroupSlots - 1);
+}
+
+__device__ __forceinline__ uint64_t ptx_globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
 }
 
 
@@ -140,6 +151,14 @@ inline int num_sms() {
     return cached[dev];
 }
 inline bool pow2(uint64_t v) { return v && !(v & (v - 1)); }
+
+// Limit of every barrier wait in the tensor-core kernels (lat_set_wait_limit_ns):
+// one process-wide value, read when a kernel is launched.
+inline std::atomic<uint64_t> &wait_limit_store() {
+    static std::atomic<uint64_t> v{2000000000ull};
+    return v;
+}
+inline uint64_t wait_limit_ns() { return wait_limit_store().load(std::memory_order_relaxed); }
 
 // launch_pdl: launch with programmatic stream serialization: the kernel may be scheduled
 // as soon as the previous kernel on `s` has triggered (every kernel of the

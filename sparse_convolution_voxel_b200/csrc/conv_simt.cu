@@ -12,9 +12,9 @@
 // kernel computes the data gradient with W[k]^T and, for a submanifold map,
 // the flipped offset (the pair (i, j, k) sits at nbr[k3-1-k][i]).
 //
-// Weight gradient: pairs of each offset are cut into fixed chunks; one block
-// reduces a chunk into an fp32 partial, then the partials of each offset are
-// summed in chunk order, so the result is deterministic.
+// Weight gradient: the pair list is cut into a fixed number of shares; every
+// (share, offset) segment is reduced into one fp32 partial, then the partials
+// of each offset are summed in share order, so the result is deterministic.
 #include "common.cuh"
 #include "conv_common.cuh"
 
@@ -214,142 +214,257 @@ conv_rows_kernel(const T *__restrict__ x, int cin, const T *__restrict__ w, int 
     if (bad) flag(d_status, bad);
 }
 
-// Work units of the weight gradient: fixed chunks of kWgradChunk pairs inside one offset.
-// First unit of every offset and the total (unit_base[k3]); one warp, lane k
-// handles offset k (k3 <= 32): offset k's clamped pairs make ceil(P_k / chunk) units.
-__global__ void wgrad_units_kernel(const int64_t *__restrict__ pair_off, int k3, int64_t capacity, int chunk,
-                                   int32_t *__restrict__ unit_base) {
-    pdl_enter();
-    const int lane = threadIdx.x & 31;
-    const int64_t P = min(pair_off[k3], capacity);
-    const int64_t lo = lane < k3 ? min(pair_off[lane], capacity) : P;
-    const int64_t up = __shfl_down_sync(0xFFFFFFFFu, lo, 1);
-    const int64_t hi = lane == 31 ? P : up;
-    const int32_t units = lane < k3 ? int32_t((hi - lo + chunk - 1) / chunk) : 0;
-    int32_t incl = units;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const int32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-        if (lane >= d) incl += o;
+// ----------------------------------------------------------------------------- weight gradient
+// dW[k] = sum over the pairs (i, j) of offset k of x[i]^T dy[j].  The pair list
+// (grouped by offset) is cut into S equal contiguous shares -- S a constant of
+// the channel counts, so the cut depends on neither the GPU nor the buffer
+// sizes -- and each share into segments, its intersections with the offsets'
+// pair ranges.  A segment's sum is written as one fp32 partial at slot
+// share + offset (unique: shares and offsets are both in pair order, so along
+// the pair list every step moves to a later share or a later offset); a
+// second kernel adds the partials of each offset in share order.  Every sum
+// runs in a fixed order, so dW is deterministic, and the scratch holds
+// (S + k3) partials whatever the pair count.
+constexpr int kSharesLanes = 1184;  // small Cin x Cout (register-tiled kernel)
+constexpr int kSharesSlices = 296;  // large Cin x Cout (slice kernel)
+constexpr int kLanesMaxElems = 2048;  // Cin x Cout handled by the register-tiled kernel (<= 32 8x8 tiles)
+
+// Shares actually used for P pairs: at most S_max, and at most P so that no
+// share is empty (each share writes the partials its slots stand for).
+__device__ __forceinline__ int share_count(int64_t P, int s_max) { return int(min(int64_t(s_max), P)); }
+__device__ __forceinline__ int64_t share_lo(int64_t P, int v, int S) { return P * v / S; }
+
+// The share holding pair `pair` (largest v with share_lo(P, v) <= pair).
+__device__ __forceinline__ int share_of(int64_t P, int64_t pair, int S) {
+    int lo = 0, hi = S - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (share_lo(P, mid, S) <= pair) lo = mid;
+        else hi = mid - 1;
     }
-    if (lane < k3) unit_base[lane] = incl - units;
-    if (lane == 31) unit_base[k3] = incl;
+    return lo;
 }
 
-// One block of 8 warps per (unit, group of slices).  A slice is 256 consecutive
-// elements of the Cin x Cout partial: lane l owns 8 consecutive output channels
-// of one input channel, so for every pair all 32 lanes read the same x row (one
-// value each) and the same dy row (one 32-byte piece each) -- coalesced,
-// broadcast loads -- and do 8 FMAs.  With nslices >= 8 each warp takes one
-// slice over the unit's pairs; with fewer (small Cin x Cout) the warps of a
-// slice split the pairs into parts and add their sums in shared memory in part
-// order.  Pair order and part order are fixed, so each partial is deterministic.
+// Register-tiled weight gradient for Cin x Cout <= 2048: the partial is cut
+// into 8x8 tiles (input channels ci0..ci0+7, output channels co0..co0+7), E of
+// them, and LP = E rounded up to a power of two lanes share one pair: lane
+// (q, t) takes tile t of every PW = 32 / LP-th pair, loads its 8 x values and
+// 8 dy values (16- or 32-byte loads) and does 64 FMAs, so one warp covers PW
+// pairs per step and a block 8 PW.  At the end of a segment the PW lanes of
+// each tile are summed with a fixed butterfly, the 8 warps' sums are added in
+// warp order through shared memory (E x 64 floats per warp), and the result
+// is stored as the segment's partial.  Persistent blocks walk the shares
+// blockIdx.x, + gridDim.x, ...
+template <typename T>
+__global__ void __launch_bounds__(256)
+wgrad_lanes_kernel(const T *__restrict__ x, int cin, const T *__restrict__ dy, int cout,
+                   const int64_t *__restrict__ pair_off, const int32_t *__restrict__ pair_in,
+                   const int32_t *__restrict__ pair_out, int64_t capacity, int k3, int64_t n_in, int64_t n_out,
+                   float *__restrict__ partial, int32_t *d_status) {
+    pdl_enter();
+    extern __shared__ float s_red[];  // [8 warps][E * 64]
+    __shared__ int64_t s_off[33];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int cob = cout / 8, E = (cin / 8) * cob;
+    int LP = 1;
+    while (LP < E) LP <<= 1;
+    const int PW = 32 / LP;
+    const int tq = lane % LP, q = warp * PW + lane / LP, step = 8 * PW;
+    const bool tile_ok = tq < E;
+    const int ci0 = tile_ok ? (tq / cob) * 8 : 0, co0 = tile_ok ? (tq % cob) * 8 : 0;
+    if (threadIdx.x <= k3) s_off[threadIdx.x] = min(pair_off[threadIdx.x], capacity);
+    __syncthreads();
+    const int64_t P = s_off[k3];
+    const int S = share_count(P, kSharesLanes);
+    const int nelem = cin * cout;
+    int32_t bad = 0;
+    for (int v = blockIdx.x; v < S; v += gridDim.x) {
+        int64_t lo = share_lo(P, v, S);
+        const int64_t hi = share_lo(P, v + 1, S);
+        int k = 0;
+        while (k < k3 && s_off[k + 1] <= lo) ++k;
+        while (lo < hi) {
+            const int64_t seg_hi = min(hi, s_off[k + 1]);
+            float acc[8][8];
+#pragma unroll
+            for (int a = 0; a < 8; ++a)
+#pragma unroll
+                for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
+            if (tile_ok) {
+                for (int64_t p0 = lo + q; p0 < seg_hi; p0 += 2 * step) {
+                    float xv[2][8], gv[2][8];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int64_t p = p0 + u * step;
+                        int i = -1, jj = -1;
+                        if (p < seg_hi) {
+                            i = __ldg(pair_in + p);
+                            jj = __ldg(pair_out + p);
+                            if (i < 0 || i >= n_in || jj < 0 || jj >= n_out) {
+                                bad |= LAT_ERR_BAD_MAP;
+                                i = jj = -1;
+                            }
+                        }
+                        if (i >= 0) {
+                            load8<T>(x + int64_t(i) * cin + ci0, xv[u]);
+                            load8<T>(dy + int64_t(jj) * cout + co0, gv[u]);
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) xv[u][c] = gv[u][c] = 0.f;
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 2; ++u)
+#pragma unroll
+                        for (int a = 0; a < 8; ++a)
+#pragma unroll
+                            for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(xv[u][a], gv[u][b], acc[a][b]);
+                }
+            }
+            // lanes of one tile: a fixed butterfly over the pair lanes
+            for (int o = LP; o < 32; o <<= 1)
+#pragma unroll
+                for (int a = 0; a < 8; ++a)
+#pragma unroll
+                    for (int b = 0; b < 8; ++b) acc[a][b] += __shfl_xor_sync(0xFFFFFFFFu, acc[a][b], o);
+            if (lane < LP && tile_ok) {
+                float *dst = s_red + (warp * E + tq) * 64;
+#pragma unroll
+                for (int a = 0; a < 8; ++a)
+#pragma unroll
+                    for (int b = 0; b < 8; b += 4)
+                        *reinterpret_cast<float4 *>(dst + a * 8 + b) =
+                            make_float4(acc[a][b], acc[a][b + 1], acc[a][b + 2], acc[a][b + 3]);
+            }
+            __syncthreads();
+            // the 8 warps' sums in warp order, stored row-major (ci, co) at slot v + k
+            float *out = partial + int64_t(v + k) * nelem;
+            for (int e = threadIdx.x; e < E * 64; e += blockDim.x) {
+                float sum = 0.f;
+#pragma unroll
+                for (int w = 0; w < 8; ++w) sum += s_red[w * E * 64 + e];
+                const int tt = e / 64, a = (e % 64) / 8, b = e % 8;
+                out[((tt / cob) * 8 + a) * cout + (tt % cob) * 8 + b] = sum;
+            }
+            __syncthreads();
+            lo = seg_hi;
+            ++k;
+            while (k < k3 && s_off[k + 1] <= lo) ++k;
+        }
+    }
+    if (bad) flag(d_status, bad);
+}
+
+// Slice weight gradient for Cin x Cout > 2048: a slice is 256 consecutive
+// elements of the Cin x Cout partial; lane l owns 8 consecutive output
+// channels of one input channel, so for every pair all 32 lanes read the same
+// x row (one value each) and the same dy row (one 32-byte piece each) --
+// coalesced, broadcast loads -- and do 8 FMAs.  Block (share v, group of 8
+// slices): each warp takes one slice over every segment of the share, pairs
+// in order, 4 at a time.
 constexpr int kWgradSlice = 256;
 constexpr int kWgradWarps = 8;
 
 template <typename T>
 __global__ void __launch_bounds__(kWgradWarps * 32)
-wgrad_simt_kernel(const T *__restrict__ x, int cin, const T *__restrict__ dy, int cout, const int64_t *__restrict__ pair_off,
-                  const int32_t *__restrict__ pair_in, const int32_t *__restrict__ pair_out, int64_t capacity, int k3,
-                  int64_t n_in, int64_t n_out, const int32_t *__restrict__ unit_base, int chunk, float *__restrict__ partial,
-                  int32_t *d_status) {
+wgrad_slices_kernel(const T *__restrict__ x, int cin, const T *__restrict__ dy, int cout,
+                    const int64_t *__restrict__ pair_off, const int32_t *__restrict__ pair_in,
+                    const int32_t *__restrict__ pair_out, int64_t capacity, int k3, int64_t n_in, int64_t n_out,
+                    float *__restrict__ partial, int32_t *d_status) {
     pdl_enter();
-    __shared__ float s_part[kWgradWarps][kWgradSlice];
+    __shared__ int64_t s_off[33];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nelem = cin * cout;
     const int nslices = (nelem + kWgradSlice - 1) / kWgradSlice;
-    // warps per slice (parts of the pair range) and slices per block
-    const int parts = nslices >= kWgradWarps ? 1 : (kWgradWarps % nslices == 0 ? kWgradWarps / nslices : 1);
-    const int per_block = kWgradWarps / parts;
-    const int groups = (nslices + per_block - 1) / per_block;
-    const int32_t u = int32_t(blockIdx.x / groups);
-    const int slice = int(blockIdx.x % groups) * per_block + warp / parts;
-    const int part = warp % parts;
-    const bool unit_ok = u < unit_base[k3];
+    const int groups = (nslices + kWgradWarps - 1) / kWgradWarps;
+    const int v = blockIdx.x / groups;
+    const int slice = (blockIdx.x % groups) * kWgradWarps + warp;
     const int e0 = slice * kWgradSlice + lane * 8;
-    const bool own = unit_ok && slice < nslices && e0 < nelem;
+    const bool own = slice < nslices && e0 < nelem;
     const int ci = own ? e0 / cout : 0, co0 = own ? e0 % cout : 0;
-    int64_t lo = 0, hi = 0;
-    if (unit_ok) {
-        int k = 0;
-        while (unit_base[k + 1] <= u) ++k;
-        const int64_t ulo = min(pair_off[k], capacity) + int64_t(u - unit_base[k]) * chunk;
-        const int64_t uhi = min(ulo + chunk, min(pair_off[k + 1], capacity));
-        const int64_t per = (uhi - ulo + parts - 1) / parts;
-        lo = min(uhi, ulo + per * part);
-        hi = min(uhi, lo + per);
-    }
-    float acc[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+    if (threadIdx.x <= k3) s_off[threadIdx.x] = min(pair_off[threadIdx.x], capacity);
+    __syncthreads();
+    const int64_t P = s_off[k3];
+    const int S = share_count(P, kSharesSlices);
+    if (v >= S) return;
+    int64_t lo = share_lo(P, v, S);
+    const int64_t hi = share_lo(P, v + 1, S);
+    int k = 0;
+    while (k < k3 && s_off[k + 1] <= lo) ++k;
     int32_t bad = 0;
-    if (own) {
-        for (int64_t p0 = lo; p0 < hi; p0 += 4) {
-            float xv[4], gv[4][8];
+    while (lo < hi) {
+        const int64_t seg_hi = min(hi, s_off[k + 1]);
+        float acc[8];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int64_t p = p0 + q;
-                int i = -1, jj = -1;
-                if (p < hi) {
-                    i = __ldg(pair_in + p);
-                    jj = __ldg(pair_out + p);
-                    if (i < 0 || i >= n_in || jj < 0 || jj >= n_out) {
-                        bad |= LAT_ERR_BAD_MAP;
-                        i = jj = -1;
+        for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+        if (own) {
+            for (int64_t p0 = lo; p0 < seg_hi; p0 += 4) {
+                float xv[4], gv[4][8];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int64_t p = p0 + u;
+                    int i = -1, jj = -1;
+                    if (p < seg_hi) {
+                        i = __ldg(pair_in + p);
+                        jj = __ldg(pair_out + p);
+                        if (i < 0 || i >= n_in || jj < 0 || jj >= n_out) {
+                            bad |= LAT_ERR_BAD_MAP;
+                            i = jj = -1;
+                        }
+                    }
+                    xv[u] = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) gv[u][c] = 0.f;
+                    if (i >= 0) {
+                        xv[u] = Elem<T>::to_f(x[int64_t(i) * cin + ci]);
+                        load8<T>(dy + int64_t(jj) * cout + co0, gv[u]);
                     }
                 }
-                xv[q] = 0.f;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) gv[q][c] = 0.f;
-                if (i >= 0) {
-                    xv[q] = Elem<T>::to_f(x[int64_t(i) * cin + ci]);
-                    load8<T>(dy + int64_t(jj) * cout + co0, gv[q]);
-                }
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) acc[c] = fmaf(xv[u], gv[u][c], acc[c]);
             }
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-#pragma unroll
-                for (int c = 0; c < 8; ++c) acc[c] = fmaf(xv[q], gv[q][c], acc[c]);
+            float *dst = partial + int64_t(v + k) * nelem + e0;
+            reinterpret_cast<float4 *>(dst)[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            reinterpret_cast<float4 *>(dst)[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
         }
-    }
-    if (parts > 1) {
-#pragma unroll
-        for (int c = 0; c < 8; ++c) s_part[warp][lane * 8 + c] = acc[c];
-        __syncthreads();
-        if (part == 0 && own) {
-            for (int q = 1; q < parts; ++q)
-#pragma unroll
-                for (int c = 0; c < 8; ++c) acc[c] += s_part[warp + q][lane * 8 + c];
-        }
-    }
-    if (own && part == 0) {
-        float *dst = partial + int64_t(u) * nelem + e0;
-        reinterpret_cast<float4 *>(dst)[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        reinterpret_cast<float4 *>(dst)[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        lo = seg_hi;
+        ++k;
+        while (k < k3 && s_off[k + 1] <= lo) ++k;
     }
     if (bad) flag(d_status, bad);
 }
 
-__global__ void wgrad_reduce_kernel(const float *__restrict__ partial, const int32_t *__restrict__ unit_base, int k3,
-                                    int nelem, float *__restrict__ dw) {
+// dW[k] = the partials of offset k's segments, added in share order (0 for an
+// offset without pairs).  s_max: the share count the main kernel was given.
+__global__ void wgrad_share_reduce_kernel(const float *__restrict__ partial, const int64_t *__restrict__ pair_off,
+                                          int64_t capacity, int k3, int nelem, int s_max, float *__restrict__ dw) {
     pdl_enter();
+    __shared__ int s_v[2];
     const int k = blockIdx.y;
+    if (threadIdx.x == 0) {
+        const int64_t P = min(pair_off[k3], capacity);
+        const int S = share_count(P, s_max);
+        const int64_t lo = min(pair_off[k], capacity), hi = min(pair_off[k + 1], capacity);
+        s_v[0] = lo < hi ? share_of(P, lo, S) : 0;
+        s_v[1] = lo < hi ? share_of(P, hi - 1, S) : -1;
+    }
+    __syncthreads();
     const int el = blockIdx.x * blockDim.x + threadIdx.x;
     if (k >= k3 || el >= nelem) return;
     float s = 0.f;
-    for (int32_t u = unit_base[k]; u < unit_base[k + 1]; ++u) s += partial[int64_t(u) * nelem + el];
+    for (int v = s_v[0]; v <= s_v[1]; ++v) s += partial[int64_t(v + k) * nelem + el];
     dw[int64_t(k) * nelem + el] = s;
 }
 
 // ----------------------------------------------------------------------------- host side
-constexpr int kWgradChunkSimt = 1024;
+static int wgrad_shares(int cin, int cout) {
+    return int64_t(cin) * cout <= kLanesMaxElems ? kSharesLanes : kSharesSlices;
+}
 
 size_t wgrad_simt_ws_bytes(int cin, int cout, const lat_kmap *map) {
-    const int64_t units = (map->pair_capacity + kWgradChunkSimt - 1) / kWgradChunkSimt + map->k3;
-    Carver cv(nullptr);
-    cv.take<int32_t>(size_t(map->k3) + 1);
-    cv.take<float>(size_t(units) * cin * cout);
-    return align_up(cv.used, 256);
+    return align_up(sizeof(float) * size_t(wgrad_shares(cin, cout) + map->k3) * size_t(cin) * size_t(cout), 256);
 }
 
 template <typename T>
@@ -396,26 +511,31 @@ template lat_status launch_conv_simt<__nv_bfloat16>(const void *, int, const voi
 template <typename T>
 lat_status launch_wgrad_simt(const void *x, int cin, const void *dy, int cout, const lat_kmap *map, float *dw,
                              void *ws, int32_t *d_status, cudaStream_t s) {
-    const int64_t units_max = (map->pair_capacity + kWgradChunkSimt - 1) / kWgradChunkSimt + map->k3;
-    Carver cv(ws);
-    int32_t *unit_base = cv.take<int32_t>(size_t(map->k3) + 1);
-    float *partial = cv.take<float>(size_t(units_max) * cin * cout);
-    LAT_CUDA_TRY(launch_pdl(wgrad_units_kernel, dim3(1), dim3(32), 0, s, map->pair_off, map->k3, map->pair_capacity,
-                            kWgradChunkSimt, unit_base));
-    LAT_CUDA_TRY(cudaGetLastError());
-    const int64_t nslices = (int64_t(cin) * cout + kWgradSlice - 1) / kWgradSlice;
-    const int64_t parts = nslices >= kWgradWarps ? 1 : (kWgradWarps % nslices == 0 ? kWgradWarps / nslices : 1);
-    const int64_t per_block = kWgradWarps / parts;
-    const int64_t grid = units_max * ((nslices + per_block - 1) / per_block);
-    if (grid >= (int64_t(1) << 31)) return LAT_ERR_UNSUPPORTED;
-    LAT_CUDA_TRY(launch_pdl(wgrad_simt_kernel<T>, dim3(unsigned(grid)), dim3(kWgradWarps * 32), 0, s,
-                            static_cast<const T *>(x), cin, static_cast<const T *>(dy), cout, map->pair_off,
-                            map->pair_in, map->pair_out, map->pair_capacity, map->k3, map->n_in, map->n_out, unit_base,
-                            kWgradChunkSimt, partial, d_status));
-    LAT_CUDA_TRY(cudaGetLastError());
+    float *partial = static_cast<float *>(ws);
     const int nelem = cin * cout;
-    dim3 rg((nelem + 255) / 256, map->k3);
-    LAT_CUDA_TRY(launch_pdl(wgrad_reduce_kernel, dim3(rg), dim3(256), 0, s, partial, unit_base, map->k3, nelem, dw));
+    const int S = wgrad_shares(cin, cout);
+    if (nelem <= kLanesMaxElems) {
+        const int E = (cin / 8) * (cout / 8);
+        const size_t smem = sizeof(float) * 8 * size_t(E) * 64;
+        auto kern = wgrad_lanes_kernel<T>;
+        if (smem > 48 * 1024)
+            LAT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+        const int grid = std::min(S, 2 * num_sms());
+        LAT_CUDA_TRY(launch_pdl(kern, dim3(grid), dim3(256), smem, s, static_cast<const T *>(x), cin,
+                                static_cast<const T *>(dy), cout, map->pair_off, map->pair_in, map->pair_out,
+                                map->pair_capacity, map->k3, map->n_in, map->n_out, partial, d_status));
+    } else {
+        const int nslices = (nelem + kWgradSlice - 1) / kWgradSlice;
+        const int groups = (nslices + kWgradWarps - 1) / kWgradWarps;
+        LAT_CUDA_TRY(launch_pdl(wgrad_slices_kernel<T>, dim3(unsigned(S * groups)), dim3(kWgradWarps * 32), 0, s,
+                                static_cast<const T *>(x), cin, static_cast<const T *>(dy), cout, map->pair_off,
+                                map->pair_in, map->pair_out, map->pair_capacity, map->k3, map->n_in, map->n_out,
+                                partial, d_status));
+    }
+    LAT_CUDA_TRY(cudaGetLastError());
+    const dim3 rg((nelem + 255) / 256, map->k3);
+    LAT_CUDA_TRY(launch_pdl(wgrad_share_reduce_kernel, rg, dim3(256), 0, s, partial, map->pair_off, map->pair_capacity,
+                            map->k3, nelem, S, dw));
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }

@@ -24,8 +24,9 @@
 // of shared-memory entries that the other roles read in order.  The rows are
 // sorted by neighbour count (ascending), so walking the tiles backwards hands
 // out the long tiles first and the one-offset tiles fill the gaps.
-// Every mbarrier wait is bounded; a wait that gives up flags LAT_ERR_TIMEOUT
-// and the CTA drains and exits, releasing its TMEM.
+// Every mbarrier wait is bounded (lat_set_wait_limit_ns, 2 s by default); a
+// wait that gives up flags LAT_ERR_TIMEOUT, and the CTA waits for its
+// in-flight TMA loads and MMAs, releases its TMEM and exits.
 //
 // The same kernel computes the data gradient: the gathered operand is dy, the
 // B operand is W[k]^T (K-major view of the same weight slab), and a
@@ -51,8 +52,8 @@ constexpr int kRing = 8;         // tile entries in flight between the scheduler
 constexpr int kItems = 14;       // (tile, offset) items in flight between the scheduler and the gather warps
 constexpr uint32_t kStgBytes = kEpiWarps * 32 * 32;  // per epilogue warp: 32 rows x 16 output channels
 constexpr uint32_t kABytes = kM * 128;  // 128 rows x 64 channels x 2 bytes
-constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr unsigned kFull = 0xFFFFFFFFu;
+constexpr uint64_t kDrainNs = 1000000000ull;  // limit of the waits that drain a CTA that gave up
 
 // One claimed tile as the scheduler publishes it.
 struct TileEntry {
@@ -85,7 +86,7 @@ struct Cfg {
     // the scheduler can run ahead of the slowest reader (the epilogue) by at
     // most stages + 2 tiles; the ring must be deeper than that
     static_assert(kRing >= kStages + 3, "tile ring too shallow");
-    static_assert((2 * kStages + 4 + 2 * kRing + 2 * kItems) * 8 + 4 <= kBarBytes, "barrier area");
+    static_assert((2 * kStages + 4 + 2 * kRing + 2 * kItems + 1) * 8 + 4 <= kBarBytes, "barrier area");
     // two CTAs per SM: 228 KB of shared memory per SM, 1 KB reserved per CTA, 16 B static
     static_assert(2 * (kSmem + 16 + 1024) <= 228 * 1024, "two CTAs per SM");
 };
@@ -114,10 +115,12 @@ __device__ __forceinline__ uint32_t pack2(float a, float b, __nv_bfloat16) {
 
 // KC: gathered channels (GEMM K), N: output channels, BMN: B operand MN-major.
 // tile_counter: zero at launch; CTAs claim tiles past the first gridDim.x from it.
+// wait_ns: how long any one barrier wait may take before the CTA gives up.
 template <typename T, int KC, int N, bool BMN>
 __global__ void __launch_bounds__(kThreads, 2)
 conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x, MapView mv, T *__restrict__ y,
-               int32_t *tile_counter, int32_t *d_status) {
+               int32_t *tile_counter, uint64_t wait_ns, int32_t *d_status) {
+    const uint64_t kWaitNs = wait_ns;
     pdl_enter();
     using C = Cfg<N>;
     constexpr int NS = C::kStages;
@@ -135,7 +138,8 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x
     uint64_t *ring_empty = ring_full + kRing;
     uint64_t *item_full = ring_empty + kRing;
     uint64_t *item_empty = item_full + kItems;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(item_empty + kItems);
+    uint64_t *drain = item_empty + kItems;  // tracks the MMAs still in flight when a CTA gives up
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     ItemEntry *items = reinterpret_cast<ItemEntry *>(smem + C::kItemOff);
     __shared__ int s_abort;
 
@@ -158,6 +162,7 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x
             ptx::mbar_init(&item_full[r], 64);  // 32 index-copy completions + 32 plain arrivals
             ptx::mbar_init(&item_empty[r], kProdWarps * 32);
         }
+        ptx::mbar_init(drain, 1);
         s_abort = 0;
         ptx::fence_mbar_init();
         ptx::fence_proxy_async_smem();
@@ -173,6 +178,7 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x
     const uint32_t tmem_base = *tmem_slot;
     const bool y32 = (reinterpret_cast<uintptr_t>(y) & 31) == 0;  // 256-bit stores of output slices
     int32_t bad = 0;
+    uint32_t stages_issued = 0;  // thread 0: stage fills (each with a weight TMA) issued
 
     if (warp < kProdWarps) {
         // ------------------------------------------------------------ gather + TMA
@@ -226,6 +232,7 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x
             }
         }
         ptx::cp_async_wait<0>();
+        stages_issued = it;
         if (!ok) s_abort = 1;
     } else if (warp < kMmaWarp) {
         // ------------------------------------------------------------ epilogue
@@ -496,8 +503,23 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x
 
     __syncthreads();
     if (s_abort) {
+        // A role gave up: before the CTA releases its TMEM and shared memory,
+        // everything still writing into them must land.  Every thread's
+        // cp.async copies are complete (cp.async.wait_all above); thread 0
+        // waits for the last weight-tile phase of each stage it filled (its TMA
+        // bytes and the gather threads' arrivals), and the MMA thread commits
+        // every MMA it issued to `drain` and waits for it.  These waits have
+        // their own limit, independent of wait_ns.
         bad |= (tid == 0) ? LAT_ERR_TIMEOUT : 0;
-        __nanosleep(1000000);  // let in-flight async copies / MMAs land before TMEM is released
+        if (tid == 0) {
+            for (uint32_t i = stages_issued > NS ? stages_issued - NS : 0; i < stages_issued; ++i)
+                if (!ptx::mbar_wait(&full[i % NS], (i / NS) & 1, kDrainNs)) break;
+        }
+        if (warp == kMmaWarp && lane == 0) {
+            ptx::umma_commit(drain);
+            ptx::mbar_wait(drain, 0, kDrainNs);
+        }
+        __syncthreads();
     }
     if (bad) flag(d_status, bad);
     if (warp == 0) {
@@ -579,7 +601,7 @@ static lat_status launch(const void *x, const void *w, int k3, const MapView &mv
     if (grid <= 0) return LAT_ERR_CUDA;
     LAT_CUDA_TRY(fill_u32(counter, 1, 0u, s));
     LAT_CUDA_TRY(launch_pdl(kern, dim3(unsigned(grid)), dim3(kThreads), C::kSmem, s, map, static_cast<const T *>(x),
-                            mv, static_cast<T *>(y), counter, d_status));
+                            mv, static_cast<T *>(y), counter, wait_limit_ns(), d_status));
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }

@@ -4,7 +4,8 @@
 // kernels of the library ("What remains familiar") and its capacity knob is
 // torch_lattice.backends.hash_rsv_ratio ("Backend and configuration
 // differences").  Design: 64-byte groups of 4 slots (4 keys, then 4 rows),
-// 32-bit mixing hash placement, probing from the start of the home group over
+// 32-bit mixing hash of the key's z-brick (4 consecutive z cells share a home
+// group, see probe_start), probing from the start of the home group over
 // consecutive slots (at most kMaxProbeSlots of them), 64-bit atomicCAS to claim a
 // slot and an unsigned atomicMin on the row so that duplicates keep the lowest
 // row deterministically.
@@ -66,7 +67,9 @@ extern "C" lat_status lat_hash_build(const int32_t *coords, int64_t n, void *tab
     if (reinterpret_cast<uintptr_t>(coords) % 16 || reinterpret_cast<uintptr_t>(table) % 64) return LAT_ERR_ARG;
     const uint64_t cap = table_bytes / kSlotBytes;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    LAT_CUDA_TRY(cudaMemsetAsync(table, 0xFF, table_bytes, s));
+    // all-ones keys mark empty slots; a fill kernel (not a memset) keeps the
+    // clearing in the programmatic launch chain of the kernels around it
+    LAT_CUDA_TRY(fill_u32(table, int64_t(table_bytes / 4), 0xFFFFFFFFu, s));
     if (n == 0) return LAT_OK;
     const int threads = 256;
     const int64_t blocks = (n + threads - 1) / threads;

@@ -1,30 +1,40 @@
-// Kernel-map construction / coordinate query (lat_kmap_ws_bytes, lat_kmap_query).
+// Kernel-map construction / coordinate query (lat_kmap_ws_bytes, lat_kmap_query,
+// lat_kmap_from_parent).
 //
 // Torch Lattice docs, "Migrating from TorchSparse": kernel-map construction
 // and coordinate query are CUDA kernels of the library ("What remains
 // familiar", "Sparse tensor expectations"), and the support semantics come
-// from the "Convolution mapping" table.  Pipeline (all on `stream`):
-//   1. probe:  strided / transposed maps: one thread per output row probes
-//              every offset and writes nbr (offset-major, coalesced), mask and
-//              per (offset, block) hit counts from warp ballots.  Submanifold
-//              maps: one thread per (row, offset below the centre), each hit
-//              mirrored (the relation is symmetric) and ORed into both masks
-//              atomically; a count pass over the masks gives the counts.
-//   2. scan:   one block per offset turns its per-block counts into offsets
-//              (pairs come out grouped by offset, rows ascending).
-//   3. emit:   walks the masks and writes (in, out) pairs at ballot-ranked
-//              positions, reading nbr only where a bit is set:
-//              deterministic, no atomics.
-//   4. sort:   stable LSD radix sort (8-bit digits: 2 passes for the 16-bit
-//              grouping key of the mask -- neighbour count, mask hash --, 1
-//              pass when k3 <= 8) of the output rows -> perm; the last pass
-//              ORs the masks of each LAT_TILE_ROWS run of perm -> tile_mask.
+// from the "Convolution mapping" table.  Pipeline of one map (all on
+// `stream`; four launches for a submanifold map with K^3 > 8):
+//   0. fill:   zeroes the global counters, the sweeps' look-back state and
+//              the tile masks.
+//   1. front end: nbr (offset-major), the neighbour mask and the grouping key
+//              of every output row, plus global totals: hits per offset and
+//              the histograms of both bytes of the key.
+//                submanifold maps:  subm_probe_kernel (one warp per kernel
+//                                   column (ix, iy); one probe of a z-brick
+//                                   answers the column's Kz offsets)
+//                strided/transposed: kmap_probe_kernel (a row per thread)
+//                maps from parents: parent_maps_kernel (+ kmap_count_kernel)
+//   2. sweep 1: the pair lists (grouped by offset, output rows ascending) and
+//              the first stable radix pass of the rows by the key's low byte.
+//   3. sweep 2: the second pass (high byte) -> perm, and the tile masks.
+//              With K^3 <= 8 the key is the mask itself (one byte) and
+//              sweep 1 writes perm and the tile masks directly.
+// The sweeps cut the rows into tiles of kSwTile positions; a tile learns
+// where its rows go from its predecessors' counts by decoupled look-back
+// (Merrill and Garland, "Single-pass Parallel Prefix Scan with Decoupled
+// Look-back", 2016; Adinets and Merrill's one-sweep radix sort uses it once
+// per digit): it publishes its own counts, then walks back over the earlier
+// tiles until it meets one that has published an inclusive prefix.  Tiles
+// are numbered in the order blocks start, so every tile it waits for is
+// already running; every wait is bounded.  Ranks inside a tile keep row
+// order, so the sort is stable and every output is deterministic.
 #include "common.cuh"
 
 namespace lat {
 
 constexpr int kQueryThreads = 256;
-constexpr int kQueryWarps = kQueryThreads / 32;
 
 struct Geom {
     int ks[3], st[3], pd[3];
@@ -53,37 +63,270 @@ __device__ __forceinline__ uint32_t group_key(uint32_t m, int k3) {
     const uint32_t pc = min(__popc(m), 31);
     return (pc << 11) | ((m * 0x9E3779B1u) >> 21);
 }
-inline int group_key_bits(int k3) { return k3 <= 8 ? k3 : kGroupKeyBits; }
+__host__ __device__ inline int group_key_bits(int k3) { return k3 <= 8 ? k3 : kGroupKeyBits; }
 
-// ----------------------------------------------------------------------------- row sort
-// Stable LSD radix sort of the row grouping keys (8-bit digits, one pass per
-// digit) producing perm.  The input of a pass is cut into tiles of kSortTile
-// rows; hist[d * ntile + b] counts digit d in tile b.  The first pass's
-// histogram is accumulated by the kernel that computes the keys
-// (sort_hist_add), each pass's scatter accumulates the next pass's histogram;
-// one block per digit scans that digit's per-tile counts, and every scatter
-// block scans the 256 digit totals, which together give the first output
-// position of every (digit, tile).  Within a tile, rows keep their order (ranks from warp
-// match + per-warp digit counts), so the result is the stable sort: perm equals
-// the stable argsort of the keys, deterministic.  The last pass also ORs every
-// row's mask into its tile of LAT_TILE_ROWS output positions.
-constexpr int kSortThreads = 256;
-constexpr int kSortRounds = 2;
-constexpr int kSortTile = kSortThreads * kSortRounds;
-static_assert(kSortTile >= 512, "next-pass tag packs the output tile in 22 bits");
-constexpr int kSortWarps = kSortThreads / 32;
+// ----------------------------------------------------------------------------- global totals
+// counters[0..255]: histogram of the key's low byte, [256..511]: of its high
+// byte, [512..543]: hits per offset, [544], [545]: tile counters of the two
+// sweeps.  Zero before the front end runs.
+constexpr int kCntHist = 0, kCntOff = 512, kCntTile = 544, kCntWords = 576;
 
-// Adds the lowest digit of this lane's key to the first pass's histogram.  Every
-// lane of the warp calls it; the warp's rows lie in one sort tile.
-__device__ __forceinline__ void sort_hist_add(uint32_t key, bool live, int64_t j, int32_t *__restrict__ hist,
-                                              int ntile) {
+// Shared-memory tallies of one block (s_h: both key-byte histograms, s_o: hits
+// per offset), added to the global counters once at the end of the block.
+struct Tally {
+    int *s_h;  // [512]
+    int *s_o;  // [32]
+};
+
+// Counts one row per lane into the block's tallies; every lane of the warp calls it.
+__device__ __forceinline__ void tally_row(const Tally &ty, uint32_t key, uint32_t m, bool live, bool two) {
     const int lane = threadIdx.x & 31;
-    const uint32_t d = key & 255u;
-    const unsigned peers = __match_any_sync(0xFFFFFFFFu, live ? d : 256u + lane);
-    if (live && (peers & ((1u << lane) - 1u)) == 0)
-        atomicAdd(hist + int64_t(d) * ntile + j / kSortTile, int(__popc(peers)));
+    const uint32_t d0 = key & 255u;
+    unsigned peers = __match_any_sync(0xFFFFFFFFu, live ? d0 : 256u + lane);
+    if (live && (peers & ((1u << lane) - 1u)) == 0) atomicAdd(&ty.s_h[d0], int(__popc(peers)));
+    if (two) {
+        const uint32_t d1 = (key >> 8) & 255u;
+        peers = __match_any_sync(0xFFFFFFFFu, live ? d1 : 256u + lane);
+        if (live && (peers & ((1u << lane) - 1u)) == 0) atomicAdd(&ty.s_h[256 + d1], int(__popc(peers)));
+    }
+    const uint32_t mm = live ? m : 0u;
+    for (uint32_t any = __reduce_or_sync(0xFFFFFFFFu, mm); any; any &= any - 1) {
+        const int k = __ffs(any) - 1;
+        const unsigned hits = __ballot_sync(0xFFFFFFFFu, (mm >> k) & 1u);
+        if (lane == 0) atomicAdd(&ty.s_o[k], int(__popc(hits)));
+    }
 }
 
+__device__ __forceinline__ void tally_clear(const Tally &ty) {
+    for (int i = threadIdx.x; i < 512 + 32; i += blockDim.x) (i < 512 ? ty.s_h[i] : ty.s_o[i - 512]) = 0;
+}
+
+// Adds the block's tallies to the global counters (after a __syncthreads()).
+__device__ __forceinline__ void tally_flush(const Tally &ty, int k3, bool two, int32_t *counters) {
+    for (int i = threadIdx.x; i < 512 + 32; i += blockDim.x) {
+        if (i < 512) {
+            const int v = ty.s_h[i];
+            if (v && (i < 256 || two)) atomicAdd(counters + kCntHist + i, v);
+        } else if (i - 512 < k3) {
+            const int v = ty.s_o[i - 512];
+            if (v) atomicAdd(counters + kCntOff + (i - 512), v);
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------- table lookups
+// The 4 keys of the slot group holding slot s (two 16-byte loads of one sector).
+__device__ __forceinline__ void group_keys(const SlotGroup *groups, uint32_t s, uint64_t (&k4)[kGroupSlots]) {
+    const SlotGroup *gp = groups + s / kGroupSlots;
+    const ulonglong2 a = __ldg(reinterpret_cast<const ulonglong2 *>(gp->key));
+    const ulonglong2 b = __ldg(reinterpret_cast<const ulonglong2 *>(gp->key + 2));
+    k4[0] = a.x;
+    k4[1] = a.y;
+    k4[2] = b.x;
+    k4[3] = b.y;
+}
+
+// Slot of `key` (linear probing from its group start), -1 if absent.
+__device__ __forceinline__ int probe_one(const SlotGroup *groups, uint32_t cap_mask, uint64_t key) {
+    uint32_t slot = probe_start(key, cap_mask);
+    for (uint32_t round = 0; round < probe_window(cap_mask) / kGroupSlots; ++round) {
+        uint64_t k4[kGroupSlots];
+        group_keys(groups, slot, k4);
+#pragma unroll
+        for (int i = 0; i < kGroupSlots; ++i) {
+            if (k4[i] == key) return int(slot) + i;
+            if (k4[i] == kEmptyKey) return -1;
+        }
+        slot = (slot + kGroupSlots) & cap_mask;
+    }
+    return -1;
+}
+
+// Searches one kernel column (b, X, Y) for its KZ targets z_t = zlo + t
+// (t = 0..KZ-1, bit t of `want` set for the ones to look up), given as the
+// column's upper key word col_hi = b<<16 | X field, the Y field and the z
+// field zf0 of target 0.  A slot holds target t iff its upper 48 bits equal
+// the column's and its z field is zf0 + t.  Every key lives in the probe
+// sequence of its z-brick (probe_start ignores the low two bits of the z
+// field), so KZ <= 5 consecutive targets need at most two sequences, A for
+// the first wanted target's brick and B for the last's; both are read at once
+// and each is walked until its targets are found or it shows an empty slot
+// (no key of that brick lies beyond an empty slot of its sequence).  Bounded
+// by the probe window.  slot_of[t] = the slot of target t, or -1.
+template <int KZ>
+__device__ __forceinline__ void probe_column(const SlotGroup *groups, uint32_t cap_mask, uint32_t col_hi,
+                                             uint32_t col_y, int zf0, uint32_t want, int (&slot_of)[KZ]) {
+    static_assert(KZ >= 1 && KZ <= 5, "two z-bricks at most");
+#pragma unroll
+    for (int t = 0; t < KZ; ++t) slot_of[t] = -1;
+    if (!want) return;
+    const int t_lo = __ffs(want) - 1, t_hi = 31 - __clz(want);
+    const uint32_t b_lo = uint32_t(zf0 + t_lo) >> 2, b_hi = uint32_t(zf0 + t_hi) >> 2;
+    const uint64_t colkey = (uint64_t(col_hi) << 32) | (uint64_t(col_y) << 16);
+    uint32_t want_a = 0;
+#pragma unroll
+    for (int t = 0; t < KZ; ++t)
+        if (((want >> t) & 1u) && (uint32_t(zf0 + t) >> 2) == b_lo) want_a |= 1u << t;
+    const uint32_t want_b = want & ~want_a;
+    uint32_t sa = probe_start(colkey | (uint64_t(b_lo) << 2), cap_mask);
+    uint32_t sb = probe_start(colkey | (uint64_t(b_hi) << 2), cap_mask);
+    bool act_a = want_a != 0, act_b = want_b != 0;
+    uint32_t found = 0;
+    auto scan = [&](const uint64_t (&k4)[kGroupSlots], uint32_t s) -> bool {
+        bool empty = false;
+#pragma unroll
+        for (int i = 0; i < kGroupSlots; ++i) {
+            const uint64_t k = k4[i];
+            if (k == kEmptyKey) {
+                empty = true;
+                continue;
+            }
+            if (uint32_t(k >> 32) != col_hi || uint32_t(k >> 16 & 0xFFFFu) != col_y) continue;
+            const int d = int(k & 0xFFFFu) - zf0;
+#pragma unroll
+            for (int t = 0; t < KZ; ++t)
+                if (d == t) slot_of[t] = int(s) + i;
+            if (d >= 0 && d < KZ) found |= 1u << d;
+        }
+        return empty;
+    };
+    for (uint32_t round = 0; (act_a || act_b) && round < probe_window(cap_mask) / kGroupSlots; ++round) {
+        uint64_t ka[kGroupSlots], kb[kGroupSlots];
+        if (act_a) group_keys(groups, sa, ka);
+        if (act_b) group_keys(groups, sb, kb);
+        if (act_a) {
+            const bool e = scan(ka, sa);
+            act_a = !e && (want_a & ~found);
+            sa = (sa + kGroupSlots) & cap_mask;
+        }
+        if (act_b) {
+            const bool e = scan(kb, sb);
+            act_b = !e && (want_b & ~found);
+            sb = (sb + kGroupSlots) & cap_mask;
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < KZ; ++t)
+        if (!((want >> t) & 1u)) slot_of[t] = -1;
+}
+
+// ----------------------------------------------------------------------------- submanifold front end
+struct SubmGeom {
+    int kx, ky, kz;
+    int px, py, pz;  // (K - 1) / 2
+    int k3;
+};
+
+constexpr int kProbeRows = 128;  // output rows per block (four per lane)
+
+// Submanifold map, one launch: block = one warp per kernel column (ix, iy)
+// (warp w = ix * Ky + iy) over kProbeRows rows; the column's offsets are
+// k = w * Kz + iz.  The block's coordinates are staged in shared memory once.
+// A lane takes its rows one at a time: it searches the table for the
+// neighbours at (x + ix - px, y + iy - py, z + iz - pz), iz = 0..Kz-1, in
+// one pass over at most two z-brick sequences (KZ = 1 or 3; KZ = 0 probes
+// each offset on its own, for any Kz), writes those Kz entries of nbr
+// (coalesced: the warp's 32 rows are consecutive) and ballots its hits into
+// shared memory.  The centre offset is the row itself and is not probed.
+// Then each row's mask is gathered from the ballots, and the row's grouping
+// key, the block's hits per offset and its key-byte histograms are computed
+// and added to the global counters.
+template <int KZ>
+__global__ void __launch_bounds__(1024)
+subm_probe_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const int4 *__restrict__ coords, int64_t n,
+                  SubmGeom g, int32_t *__restrict__ nbr, uint32_t *__restrict__ mask, uint32_t *__restrict__ keys,
+                  int32_t *__restrict__ counters, int32_t *d_status) {
+    pdl_enter();
+    __shared__ int4 s_c[kProbeRows];
+    __shared__ uint32_t s_bits[32][kProbeRows / 32];
+    __shared__ int s_h[512], s_o[32];
+    const Tally ty{s_h, s_o};
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nwarp = blockDim.x >> 5;
+    const int64_t row0 = int64_t(blockIdx.x) * kProbeRows;
+    for (int i = tid; i < kProbeRows; i += blockDim.x)
+        s_c[i] = row0 + i < n ? __ldg(coords + row0 + i) : make_int4(-1, 0, 0, 0);
+    for (int i = tid; i < 32 * (kProbeRows / 32); i += blockDim.x) (&s_bits[0][0])[i] = 0u;
+    tally_clear(ty);
+    __syncthreads();
+    const int kz = KZ ? KZ : g.kz;
+    const int dx = w / g.ky - g.px, dy = w % g.ky - g.py;
+    const bool own = dx == 0 && dy == 0;
+    int32_t bad = 0;
+    for (int r = 0; r < kProbeRows / 32; ++r) {
+        const int64_t j = row0 + 32 * r + lane;
+        const bool live = j < n;
+        const int4 c = s_c[32 * r + lane];
+        const int X = c.y + dx, Y = c.z + dy;
+        const bool colok = live && c.x >= 0 && c.x <= 65534 && X >= -32768 && X <= 32767 && Y >= -32768 &&
+                           Y <= 32767 && c.w >= -32768 && c.w <= 32767;
+        const int zf0 = c.w + 32768 - g.pz;  // z field of target iz = 0
+        const uint32_t col_hi = (uint32_t(c.x) << 16) | uint32_t(X + 32768);
+        const uint32_t col_y = uint32_t(Y + 32768);
+        uint32_t want = 0;
+        for (int t = 0; t < kz; ++t)
+            if (colok && zf0 + t >= 0 && zf0 + t <= 65535 && !(own && t == g.pz)) want |= 1u << t;
+        if constexpr (KZ > 0) {
+            int slot_of[KZ];
+            probe_column<KZ>(groups, cap_mask, col_hi, col_y, zf0, want, slot_of);
+            int rr[KZ];
+#pragma unroll
+            for (int t = 0; t < KZ; ++t)
+                rr[t] = slot_of[t] >= 0 ? int(__ldg(&groups[slot_of[t] / kGroupSlots].row[slot_of[t] % kGroupSlots]))
+                                        : -1;
+#pragma unroll
+            for (int t = 0; t < KZ; ++t) {
+                int v = rr[t];
+                if (own && t == g.pz) v = live ? int(j) : -1;
+                if (v >= n) {
+                    bad |= LAT_ERR_BAD_MAP;
+                    v = -1;
+                }
+                const int k = w * KZ + t;
+                if (live) nbr[int64_t(k) * n + j] = v;
+                const unsigned hits = __ballot_sync(0xFFFFFFFFu, v >= 0);
+                if (lane == 0) s_bits[k][r] = hits;
+            }
+        } else {
+            for (int t = 0; t < kz; ++t) {
+                int v = -1;
+                if (own && t == g.pz) {
+                    v = live ? int(j) : -1;
+                } else if ((want >> t) & 1u) {
+                    const uint64_t key = (uint64_t(col_hi) << 32) | (uint64_t(col_y) << 16) | uint64_t(zf0 + t);
+                    const int s = probe_one(groups, cap_mask, key);
+                    v = s >= 0 ? int(__ldg(&groups[s / kGroupSlots].row[s % kGroupSlots])) : -1;
+                }
+                if (v >= n) {
+                    bad |= LAT_ERR_BAD_MAP;
+                    v = -1;
+                }
+                const int k = w * kz + t;
+                if (live) nbr[int64_t(k) * n + j] = v;
+                const unsigned hits = __ballot_sync(0xFFFFFFFFu, v >= 0);
+                if (lane == 0) s_bits[k][r] = hits;
+            }
+        }
+    }
+    if (bad) flag(d_status, bad);
+    __syncthreads();
+    const bool two = group_key_bits(g.k3) > 8;
+    for (int r = w; r < kProbeRows / 32; r += nwarp) {
+        const int64_t j = row0 + 32 * r + lane;
+        const bool live = j < n;
+        uint32_t m = 0;
+        for (int k = 0; k < g.k3; ++k) m |= ((s_bits[k][r] >> lane) & 1u) << k;
+        const uint32_t key = group_key(m, g.k3);
+        if (live) {
+            mask[j] = m;
+            keys[j] = key;
+        }
+        tally_row(ty, key, m, live, two);
+    }
+    __syncthreads();
+    tally_flush(ty, g.k3, two, counters);
+}
+
+// ----------------------------------------------------------------------------- strided / transposed front end
 // Input coordinate probed by output row c at offset (ix, iy, iz); false if none.
 __device__ __forceinline__ bool query_coord(const Geom &g, const int4 &c, int ix, int iy, int iz, uint64_t &key) {
     int p[3];
@@ -109,18 +352,18 @@ __device__ __forceinline__ bool query_coord(const Geom &g, const int4 &c, int ix
 // what it can (a match, or an empty slot before it, ends the probe); the rows
 // of the matches are loaded together after the rounds.  At the table's load
 // factor nearly every probe ends inside its home group, so a batch takes about
-// one round.  Rounds are bounded by the probe window (kMaxProbeSlots).  Strided and transposed
-// maps (submanifold maps use kmap_probe_sym_kernel): every offset is probed and
-// the mask, grouping key, first sort histogram and per-block counts are
+// one round.  Rounds are bounded by the probe window (kMaxProbeSlots).  Strided
+// and transposed maps (and TargetConv3d's stride-1 strided maps): every
+// offset is probed, and the mask, grouping key and global totals are
 // produced here.
 __global__ void __launch_bounds__(kQueryThreads)
 kmap_probe_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const int4 *__restrict__ out_coords,
                   int64_t n_out, int64_t n_in, Geom g, int32_t *__restrict__ nbr, uint32_t *__restrict__ mask,
-                  uint32_t *__restrict__ keys, int32_t *__restrict__ hist, int ntile, int32_t *__restrict__ block_counts,
-                  int nblk, int32_t *d_status) {
+                  uint32_t *__restrict__ keys, int32_t *__restrict__ counters, int32_t *d_status) {
     pdl_enter();
-    __shared__ int s_cnt[32];
-    if (threadIdx.x < 32) s_cnt[threadIdx.x] = 0;
+    __shared__ int s_h[512], s_o[32];
+    const Tally ty{s_h, s_o};
+    tally_clear(ty);
     __syncthreads();
     const int64_t j = blockIdx.x * int64_t(kQueryThreads) + threadIdx.x;
     const bool live = j < n_out;
@@ -200,11 +443,12 @@ kmap_probe_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const
             const int k = k0 + e;
             if (k >= kend) break;
             int r = row[e];
-            if (r >= n_in) { bad |= LAT_ERR_BAD_MAP; r = -1; }
+            if (r >= n_in) {
+                bad |= LAT_ERR_BAD_MAP;
+                r = -1;
+            }
             if (live) nbr[int64_t(k) * n_out + j] = r;
-            const unsigned hits = __ballot_sync(0xFFFFFFFFu, r >= 0);
             if (r >= 0) m |= 1u << k;
-            if ((threadIdx.x & 31) == 0 && hits) atomicAdd(&s_cnt[k], __popc(hits));
         }
     }
     if (bad) flag(d_status, bad);
@@ -213,399 +457,48 @@ kmap_probe_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const
         mask[j] = m;
         keys[j] = key;
     }
-    sort_hist_add(key, live, j, hist, ntile);
+    const bool two = group_key_bits(g.k3) > 8;
+    tally_row(ty, key, m, live, two);
     __syncthreads();
-    if (threadIdx.x < g.k3) block_counts[int64_t(threadIdx.x) * nblk + blockIdx.x] = s_cnt[threadIdx.x];
+    tally_flush(ty, g.k3, two, counters);
 }
 
-// Submanifold map, step 0: the centre row of nbr (every row is its own centre
-// neighbour), -1 in every offset above the centre (filled by mirrored hits
-// only), masks holding just the centre bit, and zeroed sort histograms and
-// tile masks.  One thread per row; all stores coalesced.
+// Grouping keys and global totals from final masks (the strided map of a
+// ksize == stride convolution, whose masks the parent scatter builds).
 __global__ void __launch_bounds__(kQueryThreads)
-kmap_subm_init_kernel(int64_t n_out, int k3, int32_t *__restrict__ nbr, uint32_t *__restrict__ mask,
-                      int32_t *__restrict__ hist, int64_t hist_words, uint32_t *__restrict__ tile_mask,
-                      int64_t ntiles) {
+kmap_count_kernel(const uint32_t *__restrict__ mask, int64_t n_out, int k3, uint32_t *__restrict__ keys,
+                  int32_t *__restrict__ counters) {
     pdl_enter();
-    const int64_t j = blockIdx.x * int64_t(kQueryThreads) + threadIdx.x;
-    // the row sort's digit histograms and the tile masks start at zero
-    const int64_t stride = int64_t(gridDim.x) * kQueryThreads;
-    for (int64_t i = j; i < hist_words; i += stride) hist[i] = 0;
-    for (int64_t i = j; i < ntiles; i += stride) tile_mask[i] = 0;
-    if (j >= n_out) return;
-    const int centre = k3 / 2;
-    nbr[int64_t(centre) * n_out + j] = int32_t(j);
-    for (int k = centre + 1; k < k3; ++k) nbr[int64_t(k) * n_out + j] = -1;
-    mask[j] = 1u << centre;
-}
-
-// Submanifold map, step 1: one thread per (offset k below the centre, row j);
-// blockIdx.y is the offset, so a warp probes one offset for 32 consecutive rows
-// (coalesced coordinate loads and nbr stores, a uniform key delta).  A probe
-// reads its home group's 4 keys with two 16-byte loads and walks on to the next
-// group only when all 4 slots hold other keys (bounded by the probe window).
-// A hit at row r also writes the mirrored entry nbr[k3-1-k][r] = j (the
-// relation is symmetric) and ORs both bits into the masks.  Far fewer
-// instructions per lookup than looping over the offsets inside one thread,
-// and about 30 registers, so every SM runs its full complement of warps.
-__global__ void __launch_bounds__(kQueryThreads)
-kmap_probe_sym_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const int4 *__restrict__ out_coords,
-                      int64_t n_out, Geom g, int32_t *__restrict__ nbr, uint32_t *__restrict__ mask,
-                      int32_t *d_status) {
-    pdl_enter();
-    const int k = blockIdx.y;
-    const int64_t j = blockIdx.x * int64_t(kQueryThreads) + threadIdx.x;
-    if (j >= n_out) return;
-    const int4 c = __ldg(out_coords + j);
-    uint64_t key = 0;
-    bool ok;
-    if (g.shift && c.y >= g.lo[0] && c.y <= g.hi[0] && c.z >= g.lo[1] && c.z <= g.hi[1] && c.w >= g.lo[2] &&
-        c.w <= g.hi[2] && pack_key(c.x, c.y, c.z, c.w, key)) {
-        key += uint64_t(g.delta[k]);
-        ok = true;
-    } else {
-        ok = query_coord(g, c, g.off[k][0], g.off[k][1], g.off[k][2], key);
-    }
-    int r = -1;
-    if (ok) {
-        uint32_t slot = probe_start(key, cap_mask);
-        for (uint32_t round = 0; round < probe_window(cap_mask) / kGroupSlots; ++round) {
-            const SlotGroup *gp = groups + slot / kGroupSlots;
-            const ulonglong2 a = __ldg(reinterpret_cast<const ulonglong2 *>(gp->key));
-            const ulonglong2 b = __ldg(reinterpret_cast<const ulonglong2 *>(gp->key + 2));
-            const uint64_t k4[kGroupSlots] = {a.x, a.y, b.x, b.y};
-            int found = -1;
-            bool stop = false;
-#pragma unroll
-            for (int i = 0; i < kGroupSlots; ++i) {
-                if (stop) continue;
-                if (k4[i] == key) {
-                    found = i;
-                    stop = true;
-                } else if (k4[i] == kEmptyKey) {
-                    stop = true;
-                }
-            }
-            if (stop) {
-                if (found >= 0) r = int(__ldg(&gp->row[found]));
-                break;
-            }
-            slot = (slot + kGroupSlots) & cap_mask;
-        }
-    }
-    if (r >= n_out) {
-        flag(d_status, LAT_ERR_BAD_MAP);
-        r = -1;
-    }
-    nbr[int64_t(k) * n_out + j] = r;
-    if (r >= 0) {
-        const int km = g.k3 - 1 - k;
-        nbr[int64_t(km) * n_out + r] = int32_t(j);
-        atomicOr(mask + j, 1u << k);
-        atomicOr(mask + r, 1u << km);
-    }
-}
-
-// Exclusive scan of the per-block hit counts of one offset (block k scans row k of
-// block_counts) -> block_offsets relative to the offset's first pair, and the
-// offset's total pair count.
-__global__ void __launch_bounds__(1024)
-kmap_scan_kernel(const int32_t *__restrict__ block_counts, int64_t *__restrict__ block_offsets, int nblk,
-                 int64_t *__restrict__ k_total) {
-    pdl_enter();
-    __shared__ int64_t s_warp[32];
-    __shared__ int64_t s_carry;
-    const int k = blockIdx.x;
-    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
-    const int32_t *row = block_counts + int64_t(k) * nblk;
-    int64_t *orow = block_offsets + int64_t(k) * nblk;
-    if (t == 0) s_carry = 0;
-    __syncthreads();
-    for (int base = 0; base < nblk; base += 1024) {
-        const int e = base + t;
-        const int64_t v = e < nblk ? row[e] : 0;
-        int64_t incl = v;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const int64_t o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-            if (lane >= d) incl += o;
-        }
-        if (lane == 31) s_warp[w] = incl;
-        __syncthreads();
-        if (w == 0) {
-            int64_t ws = s_warp[lane];
-#pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                const int64_t o = __shfl_up_sync(0xFFFFFFFFu, ws, d);
-                if (lane >= d) ws += o;
-            }
-            s_warp[lane] = ws;
-        }
-        __syncthreads();
-        const int64_t excl = s_carry + (w ? s_warp[w - 1] : 0) + incl - v;
-        if (e < nblk) orow[e] = excl;
-        __syncthreads();
-        if (t == 1023) s_carry = excl + v;
-        __syncthreads();
-    }
-    if (t == 0) k_total[k] = s_carry;
-}
-
-// Pairs of every offset at ballot-ranked positions.  The offsets a row has
-// come from its mask; nbr is read only where a bit is set.
-__global__ void __launch_bounds__(kQueryThreads)
-kmap_emit_kernel(const int32_t *__restrict__ nbr, const uint32_t *__restrict__ mask, int64_t n_out, int k3,
-                 const int64_t *__restrict__ block_offsets, const int64_t *__restrict__ k_total, int nblk,
-                 int32_t *__restrict__ pair_in, int32_t *__restrict__ pair_out, int64_t capacity,
-                 int64_t *__restrict__ pair_off, int32_t *d_status) {
-    pdl_enter();
-    __shared__ int s_warp[32][kQueryWarps];  // per (offset, warp): hits, then the exclusive prefix over warps
-    __shared__ int64_t s_base[32];           // first pair of (offset, this block)
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (warp == 0) {
-        // offset starts = exclusive scan of the per-offset totals, all loads in parallel
-        const int64_t tot = lane < k3 ? k_total[lane] : 0;
-        const int64_t bo = lane < k3 ? block_offsets[int64_t(lane) * nblk + blockIdx.x] : 0;
-        int64_t incl = tot;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const int64_t o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-            if (lane >= d) incl += o;
-        }
-        if (lane < k3) s_base[lane] = incl - tot + bo;
-        if (blockIdx.x == 0) {
-            if (lane < k3) pair_off[lane] = incl - tot;
-            const int64_t all = __shfl_sync(0xFFFFFFFFu, incl, k3 - 1);
-            if (lane == 0) pair_off[k3] = all;
-        }
-    }
-    const int64_t j = blockIdx.x * int64_t(kQueryThreads) + threadIdx.x;
-    const uint32_t m = j < n_out ? __ldg(mask + j) : 0u;
-    for (int k = 0; k < k3; ++k) {
-        const unsigned hits = __ballot_sync(0xFFFFFFFFu, (m >> k) & 1u);
-        if (lane == 0) s_warp[k][warp] = __popc(hits);
-    }
-    __syncthreads();
-    if (threadIdx.x < k3) {
-        int run = 0;
-#pragma unroll
-        for (int w = 0; w < kQueryWarps; ++w) {
-            const int c = s_warp[threadIdx.x][w];
-            s_warp[threadIdx.x][w] = run;
-            run += c;
-        }
-    }
-    __syncthreads();
-    bool over = false;
-    for (int k = 0; k < k3; ++k) {
-        const unsigned hits = __ballot_sync(0xFFFFFFFFu, (m >> k) & 1u);
-        if (!((m >> k) & 1u)) continue;
-        const int64_t pos = s_base[k] + s_warp[k][warp] + __popc(hits & ((1u << lane) - 1u));
-        if (pos < capacity) {
-            pair_in[pos] = __ldg(nbr + int64_t(k) * n_out + j);
-            pair_out[pos] = int32_t(j);
-        } else {
-            over = true;
-        }
-    }
-    if (over) flag(d_status, LAT_ERR_CAPACITY);
-}
-
-// Block d: exclusive scan, in place, of digit d's per-tile counts
-// hist[d * ntile + 0 .. ntile), and the digit's total into totals[d].
-__global__ void __launch_bounds__(256)
-sort_rowscan_kernel(int32_t *__restrict__ hist, int ntile, int32_t *__restrict__ totals) {
-    pdl_enter();
-    __shared__ int s_warp[8];
-    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
-    int32_t *row = hist + int64_t(blockIdx.x) * ntile;
-    int carry = 0;
-    for (int base = 0; base < ntile; base += 256) {
-        const int i = base + t;
-        const int v = i < ntile ? row[i] : 0;
-        int incl = v;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-            if (lane >= d) incl += o;
-        }
-        if (lane == 31) s_warp[w] = incl;
-        __syncthreads();
-        int before = 0, all = 0;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const int x = s_warp[q];
-            before += q < w ? x : 0;
-            all += x;
-        }
-        if (i < ntile) row[i] = carry + before + incl - v;
-        carry += all;
-        __syncthreads();
-    }
-    if (t == 0) totals[blockIdx.x] = carry;
-}
-
-// Pair lists written by the last sort pass when every row has at most one
-// neighbour and the key is the one-hot mask (transposed maps from parents with
-// K^3 <= 8): then the sorted order is the canonical pair order.  src == nullptr
-// means no pairs here.
-struct PairOut {
-    const int32_t *src;  // the neighbour of each row
-    int32_t *in, *out;
-    int64_t capacity;
-    int64_t *off;
-    int k3;
-    int32_t *status;
-};
-
-// One pass: scatter the rows of tile blockIdx.x by digit (key >> shift) & 255 to
-// the positions `off` gives.  vals_in == nullptr means the identity (row e).
-// LAST: write perm and OR masks into tile_mask; otherwise write the keys and
-// rows for the next pass and count its digit per output tile into hist_next.
-// All loads of the tile are issued before the first round.
-template <bool LAST>
-__global__ void __launch_bounds__(kSortThreads)
-sort_scatter_kernel(const uint32_t *__restrict__ keys_in, const int32_t *__restrict__ vals_in, int64_t n, int shift,
-                    const int32_t *__restrict__ off, const int32_t *__restrict__ totals, int ntile,
-                    uint32_t *__restrict__ keys_out,
-                    int32_t *__restrict__ vals_out, int32_t *__restrict__ hist_next,
-                    const uint32_t *__restrict__ mask, uint32_t *__restrict__ tile_mask, PairOut po) {
-    pdl_enter();
-    __shared__ int s_cnt[2][kSortWarps][256];
-    __shared__ int s_run[256];
-    __shared__ int s_wsum[kSortWarps];
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const unsigned lt = (1u << lane) - 1u;
-    const int b = blockIdx.x;
-    // first output position of digit t: exclusive scan of the digit totals
-    const int tot = totals[t];  // kSortThreads == 256 digits
-    const int off_b = off[int64_t(t) * ntile + b];
-    uint32_t key[kSortRounds], mk[kSortRounds];
-    int32_t val[kSortRounds];
-#pragma unroll
-    for (int r = 0; r < kSortRounds; ++r) {
-        const int64_t e = int64_t(b) * kSortTile + r * kSortThreads + t;
-        key[r] = 0;
-        val[r] = -1;
-        if (e < n) {
-            key[r] = __ldg(keys_in + e);
-            val[r] = vals_in ? __ldg(vals_in + e) : int32_t(e);
-        }
-    }
-    if (LAST) {
-#pragma unroll
-        for (int r = 0; r < kSortRounds; ++r) mk[r] = val[r] >= 0 ? __ldg(mask + val[r]) : 0u;
-    }
-    for (int i = t; i < 2 * kSortWarps * 256; i += kSortThreads) (&s_cnt[0][0][0])[i] = 0;
-    int incl = tot;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-        if (lane >= d) incl += o;
-    }
-    if (lane == 31) s_wsum[warp] = incl;
-    __syncthreads();
-    int base = incl - tot;
-    for (int q = 0; q < warp; ++q) base += s_wsum[q];
-    s_run[t] = base + off_b;
-    // one neighbour per row (po.src): rows of key 0 have none and sort first;
-    // offset k's pairs are the rows of key 1 << k, in sorted order
-    const int zero = po.src ? __ldg(totals) : 0;
-    if (LAST && po.src && b == 0) {
-        if (t > 0 && (t & (t - 1)) == 0 && __ffs(t) - 1 < po.k3) po.off[__ffs(t) - 1] = base - zero;
-        if (t == 255) po.off[po.k3] = base + tot - zero;
-    }
-    bool over = false;
-    __syncthreads();
-#pragma unroll
-    for (int r = 0; r < kSortRounds; ++r) {
-        const int p = r & 1;
-        const bool live = val[r] >= 0;
-        const uint32_t d = (key[r] >> shift) & 255u;
-        const unsigned peers = __match_any_sync(0xFFFFFFFFu, live ? d : 256u + lane);
-        const bool leader = live && (peers & lt) == 0;
-        if (leader) s_cnt[p][warp][d] = __popc(peers);
-        __syncthreads();
-        int64_t dst = 0;
-        if (live) {
-            int pre = s_run[d] + __popc(peers & lt);
-            for (int w = 0; w < warp; ++w) pre += s_cnt[p][w][d];
-            dst = pre;
-        }
-        __syncthreads();
-        // digit t: advance its running position and clear this round's counts
-        int add = 0;
-#pragma unroll
-        for (int w = 0; w < kSortWarps; ++w) {
-            add += s_cnt[p][w][t];
-            s_cnt[p][w][t] = 0;
-        }
-        s_run[t] += add;
-        if (LAST) {
-            if (live) vals_out[dst] = val[r];
-            if (po.src && live && key[r] != 0) {
-                const int64_t pos = dst - zero;
-                if (pos < po.capacity) {
-                    po.in[pos] = __ldg(po.src + val[r]);
-                    po.out[pos] = val[r];
-                } else {
-                    over = true;
-                }
-            }
-            // one atomic per (warp, output tile)
-            const uint32_t tile = live ? uint32_t(dst / LAT_TILE_ROWS) : (0x80000000u | lane);
-            const unsigned tp = __match_any_sync(0xFFFFFFFFu, tile);
-            const uint32_t m_or = __reduce_or_sync(tp, mk[r]);
-            if (live && (tp & lt) == 0) atomicOr(tile_mask + dst / LAT_TILE_ROWS, m_or);
-        } else {
-            if (live) {
-                keys_out[dst] = key[r];
-                vals_out[dst] = val[r];
-            }
-            const uint32_t d2 = (key[r] >> (shift + 8)) & 255u;
-            // output tile < 2^31 / kSortTile <= 2^22, digit < 2^8: the tag fits in 30 bits
-            const uint32_t tag = live ? ((d2 << 22) | uint32_t(dst / kSortTile)) : (0x80000000u | lane);
-            const unsigned p2 = __match_any_sync(0xFFFFFFFFu, tag);
-            if (live && (p2 & lt) == 0) atomicAdd(hist_next + int64_t(d2) * ntile + dst / kSortTile, int(__popc(p2)));
-        }
-    }
-    if (over) flag(po.status, LAT_ERR_CAPACITY);
-}
-
-// Per-(offset, block) hit counts, grouping keys and the first sort pass's
-// histogram from the masks (submanifold probes and maps built from parent indices).
-__global__ void __launch_bounds__(kQueryThreads)
-kmap_count_kernel(const uint32_t *__restrict__ mask, int64_t n_out, int k3, int32_t *__restrict__ block_counts,
-                  int nblk, uint32_t *__restrict__ keys, int32_t *__restrict__ hist, int ntile) {
-    pdl_enter();
-    __shared__ int s_cnt[32];
-    if (threadIdx.x < 32) s_cnt[threadIdx.x] = 0;
+    __shared__ int s_h[512], s_o[32];
+    const Tally ty{s_h, s_o};
+    tally_clear(ty);
     __syncthreads();
     const int64_t j = blockIdx.x * int64_t(kQueryThreads) + threadIdx.x;
     const bool live = j < n_out;
     const uint32_t m = live ? __ldg(mask + j) : 0u;
-    for (int k = 0; k < k3; ++k) {
-        const unsigned hits = __ballot_sync(0xFFFFFFFFu, (m >> k) & 1u);
-        if ((threadIdx.x & 31) == 0 && hits) atomicAdd(&s_cnt[k], __popc(hits));
-    }
     const uint32_t key = group_key(m, k3);
     if (live) keys[j] = key;
-    sort_hist_add(key, live, j, hist, ntile);
+    const bool two = group_key_bits(k3) > 8;
+    tally_row(ty, key, m, live, two);
     __syncthreads();
-    if (threadIdx.x < k3) block_counts[int64_t(threadIdx.x) * nblk + blockIdx.x] = s_cnt[threadIdx.x];
+    tally_flush(ty, k3, two, counters);
 }
 
 // Kernel size == stride, no padding: fine row i lies in exactly one coarse window,
 // parent[i], at offset k(i) = its position inside the window (floor modulo the
-// stride per axis).  Writes the transposed map's rows directly (one neighbour per
-// fine row) and scatters the strided map's entries (the down table must hold -1
-// and the down mask 0 beforehand).
+// stride per axis).  Writes the transposed map's rows directly (one neighbour
+// per fine row), with their grouping keys and totals, and scatters the strided
+// map's entries (its table must hold -1 and its masks 0 beforehand).
 __global__ void __launch_bounds__(256)
 parent_maps_kernel(const int4 *__restrict__ fine, const int32_t *__restrict__ parent, int64_t n_fine,
                    int64_t n_coarse, int s0, int s1, int s2, int k3, int32_t *__restrict__ up_nbr,
-                   uint32_t *__restrict__ up_mask, int32_t *__restrict__ down_nbr, uint32_t *__restrict__ down_mask,
-                   uint32_t *__restrict__ up_keys, int32_t *__restrict__ up_hist, int up_ntile, int32_t *d_status) {
+                   uint32_t *__restrict__ up_mask, uint32_t *__restrict__ up_keys, int32_t *__restrict__ up_counters,
+                   int32_t *__restrict__ down_nbr, uint32_t *__restrict__ down_mask, int32_t *d_status) {
     pdl_enter();
+    __shared__ int s_h[512], s_o[32];
+    const Tally ty{s_h, s_o};
+    if (up_nbr) tally_clear(ty);
+    __syncthreads();
     const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
     const bool live = i < n_fine;
     uint32_t m = 0;
@@ -627,96 +520,335 @@ parent_maps_kernel(const int4 *__restrict__ fine, const int32_t *__restrict__ pa
             atomicOr(down_mask + q, 1u << k);
         }
     }
-    // transposed map with K^3 <= 8: the grouping key is the mask, and its first
-    // sort histogram is built here (every lane of the warp takes part)
-    if (up_keys) {
-        if (live) up_keys[i] = m;
-        sort_hist_add(m, live, i, up_hist, up_ntile);
+    if (up_nbr) {  // block-uniform: every lane of the warp takes part
+        const uint32_t key = group_key(m, k3);
+        if (live) up_keys[i] = key;
+        const bool two = group_key_bits(k3) > 8;
+        tally_row(ty, key, m, live, two);
+        __syncthreads();
+        tally_flush(ty, k3, two, up_counters);
     }
 }
 
+// ----------------------------------------------------------------------------- sweeps
+constexpr int kSwThreads = 512;
+constexpr int kSwWarps = kSwThreads / 32;
+constexpr int kSwRounds = 4;
+constexpr int kSwTile = kSwThreads * kSwRounds;  // rows per tile
+constexpr int kSwChains = 256 + 32;              // look-back chains per tile: 256 digits, then 32 offsets
+constexpr unsigned long long kFlagAgg = 1ull << 32, kFlagPrefix = 2ull << 32;
+constexpr uint64_t kLookbackNs = 1000000000ull;  // a look-back wait gives up after 1 s
+
+__device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_relaxed(unsigned long long *p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+struct Sweep {
+    const uint32_t *keys_in;   // key of each input position
+    const int32_t *vals_in;    // output row of each input position; nullptr = the position itself
+    const uint32_t *masks_in;  // neighbour mask of each input position
+    int64_t n;
+    int shift;                 // this pass's digit: (key >> shift) & 255
+    int32_t *counters;         // global totals (kCnt*); tile counter of this sweep at kCntTile + which
+    int which;                 // 0 = first sweep, 1 = second
+    unsigned long long *status;  // [ntile][kSwChains] look-back words, zero at launch
+    // pair emission (first sweep)
+    const int32_t *nbr;
+    int centre;  // offset whose neighbour of row j is j itself (submanifold), else -1
+    int k3;
+    int32_t *pair_in, *pair_out;
+    int64_t capacity;
+    int64_t *pair_off;
+    // outputs: to the second sweep, or perm and the tile masks
+    uint32_t *keys_out;
+    int32_t *vals_out;
+    uint32_t *masks_out;
+    int32_t *perm;
+    uint32_t *tile_mask;  // zero at launch
+    int32_t *d_status;
+};
+
+// One tile of one radix pass.  EMIT: also write the pair lists (first sweep,
+// rows in input order).  LAST: write perm and OR each row's mask into its
+// LAT_TILE_ROWS output tile; otherwise hand (key, row, mask) to the next
+// sweep at the sorted position.  Positions: the digit's start (exclusive scan
+// of the global digit histogram) + the digit's count in earlier tiles
+// (look-back) + the row's rank among this tile's rows of that digit (warp
+// match, per-warp counts; rounds in row order).  Pair positions likewise per
+// offset.
+template <bool EMIT, bool LAST>
+__global__ void __launch_bounds__(kSwThreads) sweep_kernel(Sweep a) {
+    pdl_enter();
+    __shared__ int s_tile;
+    __shared__ int s_cnt[2][kSwWarps][256];  // per round (double buffered): per-warp digit counts
+    __shared__ int s_run[256];               // next position of each digit
+    __shared__ int s_hist[256];              // this tile's rows per digit
+    __shared__ int s_ocnt[32];               // this tile's pairs per offset
+    __shared__ int s_pw[2][kSwWarps][32];    // per round: per-warp pairs per offset, then their prefix
+    __shared__ long long s_orun[2][32];      // per round: next pair position of each offset
+    __shared__ int s_wsum[8];
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const unsigned lt = (1u << lane) - 1u;
+    if (t == 0) s_tile = atomicAdd(a.counters + kCntTile + a.which, 1);
+    for (int i = t; i < 2 * kSwWarps * 256; i += kSwThreads) (&s_cnt[0][0][0])[i] = 0;
+    if (t < 256) s_hist[t] = 0;
+    if (t < 32) s_ocnt[t] = 0;
+    __syncthreads();
+    const int tile = s_tile;
+    if (int64_t(tile) * kSwTile >= a.n) {  // the tile counter was not cleared: no tile waits for this one
+        if (t == 0) flag(a.d_status, LAT_ERR_BAD_MAP);
+        return;
+    }
+    uint32_t key[kSwRounds], mk[kSwRounds];
+    int32_t val[kSwRounds];
+#pragma unroll
+    for (int r = 0; r < kSwRounds; ++r) {
+        const int64_t e = int64_t(tile) * kSwTile + r * kSwThreads + t;
+        key[r] = 0;
+        mk[r] = 0;
+        val[r] = -1;
+        if (e < a.n) {
+            key[r] = __ldg(a.keys_in + e);
+            val[r] = a.vals_in ? __ldg(a.vals_in + e) : int32_t(e);
+            if (EMIT || LAST) mk[r] = __ldg(a.masks_in + e);
+        }
+    }
+    // this tile's counts
+#pragma unroll
+    for (int r = 0; r < kSwRounds; ++r) {
+        const bool live = val[r] >= 0;
+        const uint32_t d = (key[r] >> a.shift) & 255u;
+        const unsigned peers = __match_any_sync(0xFFFFFFFFu, live ? d : 256u + lane);
+        if (live && (peers & lt) == 0) atomicAdd(&s_hist[d], int(__popc(peers)));
+        if (EMIT) {
+            const uint32_t m = live ? mk[r] : 0u;
+            for (uint32_t any = __reduce_or_sync(0xFFFFFFFFu, m); any; any &= any - 1) {
+                const int k = __ffs(any) - 1;
+                const unsigned hits = __ballot_sync(0xFFFFFFFFu, (m >> k) & 1u);
+                if (lane == 0) atomicAdd(&s_ocnt[k], int(__popc(hits)));
+            }
+        }
+    }
+    __syncthreads();
+    // publish this tile's counts, look back for the earlier tiles', publish the prefix
+    const int nchain = EMIT ? 256 + a.k3 : 256;
+    unsigned long long *st = a.status + int64_t(tile) * kSwChains;
+    int own = 0, excl = 0;
+    if (t < nchain) {
+        own = t < 256 ? s_hist[t] : s_ocnt[t - 256];
+        st_relaxed(st + t, (tile == 0 ? kFlagPrefix : kFlagAgg) | uint32_t(own));
+        if (tile > 0) {
+            bool timed_out = false;
+            uint64_t t0 = 0;
+            int64_t pb = tile - 1;
+            for (uint32_t spin = 0;;) {
+                const unsigned long long v = ld_relaxed(a.status + pb * kSwChains + t);
+                if ((v >> 32) == 0) {  // that tile has not published yet: it is running, wait
+                    if (++spin == 64) t0 = ptx_globaltimer();
+                    if (spin > 64 && (spin & 15) == 0 && ptx_globaltimer() - t0 > kLookbackNs) {
+                        timed_out = true;
+                        break;
+                    }
+                    __nanosleep(64);
+                    continue;
+                }
+                excl += int(uint32_t(v));
+                if ((v >> 32) == 2 || pb == 0) break;
+                --pb;
+            }
+            if (timed_out) flag(a.d_status, LAT_ERR_TIMEOUT);
+            st_relaxed(st + t, kFlagPrefix | uint32_t(excl + own));
+        }
+    }
+    // digit starts: exclusive scan of the global digit histogram
+    if (t < 256) {
+        const int v = a.counters[kCntHist + (a.shift ? 256 : 0) + t];
+        int incl = v;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+            if (lane >= d) incl += o;
+        }
+        if (lane == 31) s_wsum[warp] = incl;
+        s_run[t] = incl - v + excl;  // completed with the earlier warps' sums below
+    }
+    if (EMIT && warp == 8) {  // offset starts: exclusive scan of the per-offset totals
+        const int64_t v = lane < a.k3 ? a.counters[kCntOff + lane] : 0;
+        int64_t incl = v;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int64_t o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+            if (lane >= d) incl += o;
+        }
+        if (lane < a.k3) s_orun[0][lane] = incl - v + excl;
+        if (tile == 0) {
+            if (lane < a.k3) a.pair_off[lane] = incl - v;
+            const int64_t all = __shfl_sync(0xFFFFFFFFu, incl, 31);
+            if (lane == 0) a.pair_off[a.k3] = all;
+        }
+    }
+    __syncthreads();
+    if (t < 256)
+        for (int q = 0; q < warp; ++q) s_run[t] += s_wsum[q];
+    __syncthreads();
+    bool over = false, bad = false;
+#pragma unroll
+    for (int r = 0; r < kSwRounds; ++r) {
+        const int p = r & 1;
+        const bool live = val[r] >= 0;
+        const uint32_t d = (key[r] >> a.shift) & 255u;
+        const unsigned peers = __match_any_sync(0xFFFFFFFFu, live ? d : 256u + lane);
+        if (live && (peers & lt) == 0) s_cnt[p][warp][d] = __popc(peers);
+        const uint32_t m = (EMIT && live) ? mk[r] : 0u;
+        uint32_t any = 0;
+        if (EMIT) {
+            s_pw[p][warp][lane] = 0;
+            __syncwarp();
+            any = __reduce_or_sync(0xFFFFFFFFu, m);
+            for (uint32_t b = any; b; b &= b - 1) {
+                const int k = __ffs(b) - 1;
+                const unsigned hits = __ballot_sync(0xFFFFFFFFu, (m >> k) & 1u);
+                if (lane == 0) s_pw[p][warp][k] = __popc(hits);
+            }
+        }
+        __syncthreads();
+        int64_t dst = 0;
+        bool put = false;
+        if (live) {
+            int pre = s_run[d] + __popc(peers & lt);
+            for (int w = 0; w < warp; ++w) pre += s_cnt[p][w][d];
+            dst = pre;
+            // totals that disagree with the rows (never for maps the front ends built)
+            put = dst >= 0 && dst < a.n;
+            if (!put) bad = true;
+        }
+        if (EMIT && t < a.k3) {  // per offset: exclusive prefix over the warps, and the next round's start
+            int run = 0;
+            for (int w = 0; w < kSwWarps; ++w) {
+                const int c = s_pw[p][w][t];
+                s_pw[p][w][t] = run;
+                run += c;
+            }
+            s_orun[p ^ 1][t] = s_orun[p][t] + run;
+        }
+        __syncthreads();
+        if (t < 256) {  // digit t: advance its position and clear this round's counts
+            int add = 0;
+#pragma unroll
+            for (int w = 0; w < kSwWarps; ++w) {
+                add += s_cnt[p][w][t];
+                s_cnt[p][w][t] = 0;
+            }
+            s_run[t] += add;
+        }
+        if (EMIT) {
+            for (uint32_t b = any; b; b &= b - 1) {
+                const int k = __ffs(b) - 1;
+                const unsigned hits = __ballot_sync(0xFFFFFFFFu, (m >> k) & 1u);
+                if ((m >> k) & 1u) {
+                    const int64_t pos = s_orun[p][k] + s_pw[p][warp][k] + __popc(hits & lt);
+                    if (pos < a.capacity) {
+                        a.pair_in[pos] = k == a.centre ? val[r] : __ldg(a.nbr + int64_t(k) * a.n + val[r]);
+                        a.pair_out[pos] = val[r];
+                    } else {
+                        over = true;
+                    }
+                }
+            }
+        }
+        if (LAST) {
+            if (put) a.perm[dst] = val[r];
+            // one atomic per (warp, output tile)
+            const uint32_t tl = put ? uint32_t(dst / LAT_TILE_ROWS) : (0x80000000u | lane);
+            const unsigned tp = __match_any_sync(0xFFFFFFFFu, tl);
+            const uint32_t m_or = __reduce_or_sync(tp, mk[r]);
+            if (put && (tp & lt) == 0) atomicOr(a.tile_mask + dst / LAT_TILE_ROWS, m_or);
+        } else if (put) {
+            a.keys_out[dst] = key[r];
+            a.vals_out[dst] = val[r];
+            a.masks_out[dst] = mk[r];
+        }
+    }
+    if (over || bad) flag(a.d_status, (over ? LAT_ERR_CAPACITY : 0) | (bad ? LAT_ERR_BAD_MAP : 0));
+}
+
+// ----------------------------------------------------------------------------- workspace and host side
 struct KmapWs {
-    int32_t *block_counts;
-    int64_t *block_offsets;
-    int64_t *k_total;
-    uint32_t *keys;
-    uint32_t *keys_tmp;
+    uint32_t *keys;       // grouping key of every row (front end)
+    uint32_t *keys_tmp;   // rows after the first sweep: key, row, mask
     int32_t *vals_tmp;
-    int32_t *hist;    // two histograms of 256 x ntile, cleared before the keys are computed
-    int32_t *totals;  // per-digit totals of each pass
-    int ntile;
-    size_t hist_bytes;
+    uint32_t *masks_tmp;
+    int32_t *counters;    // kCntWords words, then the look-back words of both sweeps
+    unsigned long long *status[2];
+    int64_t ntile;
+    int64_t zero_words;   // 32-bit words from `counters` on that must be zero before the front end
     size_t total;
 };
 
-static KmapWs carve_kmap_ws(void *base, int64_t n_out, int k3) {
+static KmapWs carve_kmap_ws(void *base, int64_t n_out) {
     KmapWs w{};
-    const int nblk = int((n_out + kQueryThreads - 1) / kQueryThreads);
-    w.ntile = int((n_out + kSortTile - 1) / kSortTile);
+    w.ntile = (n_out + kSwTile - 1) / kSwTile;
     Carver cv(base);
-    w.block_counts = cv.take<int32_t>(size_t(k3) * nblk);
-    w.block_offsets = cv.take<int64_t>(size_t(k3) * nblk);
-    w.k_total = cv.take<int64_t>(size_t(k3));
     w.keys = cv.take<uint32_t>(size_t(n_out));
     w.keys_tmp = cv.take<uint32_t>(size_t(n_out));
     w.vals_tmp = cv.take<int32_t>(size_t(n_out));
-    w.hist_bytes = sizeof(int32_t) * 2 * 256 * size_t(w.ntile);
-    w.hist = cv.take<int32_t>(2 * 256 * size_t(w.ntile));
-    w.totals = cv.take<int32_t>(2 * 256);
+    w.masks_tmp = cv.take<uint32_t>(size_t(n_out));
+    w.counters = cv.take<int32_t>(kCntWords);  // kCntWords * 4 is a multiple of 256: status follows directly
+    static_assert(kCntWords * 4 % 256 == 0, "counters and look-back words are one contiguous zero region");
+    w.status[0] = cv.take<unsigned long long>(size_t(w.ntile) * kSwChains);
+    w.status[1] = cv.take<unsigned long long>(size_t(w.ntile) * kSwChains);
+    w.zero_words = kCntWords + 2 * 2 * w.ntile * kSwChains;
     w.total = align_up(cv.used, 256);
     return w;
 }
 
-static lat_status sort_rows(lat_kmap *map, int k3, KmapWs &w, cudaStream_t s);
-
-// Scan the per-block counts, emit the pair lists, sort the rows by grouping key
-// (perm) and OR the tile masks.  The keys and the first sort histogram are in w.
-// The pair chain (scan, emit) and the sort chain are independent: with a side
-// stream the pair chain runs on it, concurrently with the sort on `s`.
-static lat_status finish_kmap(lat_kmap *map, int k3, int nblk, KmapWs &w, int32_t *d_status, cudaStream_t s,
-                              SideStream *side) {
-    const int64_t n_out = map->n_out;
-    cudaStream_t ps = s;
-    if (side) {
-        LAT_CUDA_TRY(side_fork(*side, s));
-        ps = side->side;
-    }
-    LAT_CUDA_TRY(launch_pdl(kmap_scan_kernel, dim3(k3), dim3(1024), 0, ps, w.block_counts, w.block_offsets, nblk,
-                            w.k_total));
-    LAT_CUDA_TRY(cudaGetLastError());
-    LAT_CUDA_TRY(launch_pdl(kmap_emit_kernel, dim3(nblk), dim3(kQueryThreads), 0, ps, map->nbr, map->mask, n_out, k3,
-                            w.block_offsets, w.k_total, nblk, map->pair_in, map->pair_out, map->pair_capacity,
-                            map->pair_off, d_status));
-    LAT_CUDA_TRY(cudaGetLastError());
-    const lat_status st = sort_rows(map, k3, w, s);
-    if (side) LAT_CUDA_TRY(side_join(*side, s));
-    return st;
-}
-
-// Stable row sort by grouping key -> perm, tile masks ORed by the last pass
-// (map->tile_mask must hold zeros beforehand).
-static lat_status sort_rows(lat_kmap *map, int k3, KmapWs &w, cudaStream_t s) {
-    const int64_t n_out = map->n_out;
-    const int64_t hsize = 256 * int64_t(w.ntile);
-    int32_t *h1 = w.hist, *h2 = w.hist + hsize;
-    int32_t *t1 = w.totals, *t2 = w.totals + 256;
-    LAT_CUDA_TRY(launch_pdl(sort_rowscan_kernel, dim3(256), dim3(256), 0, s, h1, w.ntile, t1));
-    LAT_CUDA_TRY(cudaGetLastError());
+// The sweeps of one map whose front end has written nbr, mask, w.keys and the
+// global totals: pair lists, perm and tile masks.
+static lat_status sweep_map(lat_kmap *map, int k3, const KmapWs &w, int centre, int32_t *d_status, cudaStream_t s) {
+    const int64_t n = map->n_out;
+    Sweep a{};
+    a.keys_in = w.keys;
+    a.vals_in = nullptr;
+    a.masks_in = map->mask;
+    a.n = n;
+    a.shift = 0;
+    a.counters = w.counters;
+    a.which = 0;
+    a.status = w.status[0];
+    a.nbr = map->nbr;
+    a.centre = centre;
+    a.k3 = k3;
+    a.pair_in = map->pair_in;
+    a.pair_out = map->pair_out;
+    a.capacity = map->pair_capacity;
+    a.pair_off = map->pair_off;
+    a.perm = map->perm;
+    a.tile_mask = map->tile_mask;
+    a.d_status = d_status;
+    const dim3 grid(unsigned(w.ntile)), block(kSwThreads);
     if (group_key_bits(k3) <= 8) {
-        LAT_CUDA_TRY(launch_pdl(sort_scatter_kernel<true>, dim3(w.ntile), dim3(kSortThreads), 0, s, w.keys, nullptr,
-                                n_out, 0, h1, t1, w.ntile, nullptr, map->perm, nullptr, map->mask, map->tile_mask,
-                                PairOut{}));
+        LAT_CUDA_TRY(launch_pdl(sweep_kernel<true, true>, grid, block, 0, s, a));
         LAT_CUDA_TRY(cudaGetLastError());
         return LAT_OK;
     }
-    LAT_CUDA_TRY(launch_pdl(sort_scatter_kernel<false>, dim3(w.ntile), dim3(kSortThreads), 0, s, w.keys, nullptr,
-                            n_out, 0, h1, t1, w.ntile, w.keys_tmp, w.vals_tmp, h2, nullptr, nullptr, PairOut{}));
+    a.keys_out = w.keys_tmp;
+    a.vals_out = w.vals_tmp;
+    a.masks_out = w.masks_tmp;
+    LAT_CUDA_TRY(launch_pdl(sweep_kernel<true, false>, grid, block, 0, s, a));
     LAT_CUDA_TRY(cudaGetLastError());
-    LAT_CUDA_TRY(launch_pdl(sort_rowscan_kernel, dim3(256), dim3(256), 0, s, h2, w.ntile, t2));
-    LAT_CUDA_TRY(cudaGetLastError());
-    LAT_CUDA_TRY(launch_pdl(sort_scatter_kernel<true>, dim3(w.ntile), dim3(kSortThreads), 0, s, w.keys_tmp, w.vals_tmp,
-                            n_out, 8, h2, t2, w.ntile, nullptr, map->perm, nullptr, map->mask, map->tile_mask,
-                            PairOut{}));
+    Sweep b = a;
+    b.keys_in = w.keys_tmp;
+    b.vals_in = w.vals_tmp;
+    b.masks_in = w.masks_tmp;
+    b.shift = 8;
+    b.which = 1;
+    b.status = w.status[1];
+    LAT_CUDA_TRY(launch_pdl(sweep_kernel<false, true>, grid, block, 0, s, b));
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }
@@ -751,7 +883,7 @@ bool geom_ok(const lat_geom *g, int &k3) {
 
 extern "C" size_t lat_kmap_ws_bytes(int64_t n_out, int32_t k3) {
     if (n_out < 0 || n_out >= (int64_t(1) << 31) || k3 < 1 || k3 > 32) return 0;
-    return lat::carve_kmap_ws(nullptr, n_out, k3).total;
+    return lat::carve_kmap_ws(nullptr, n_out).total;
 }
 
 extern "C" lat_status lat_kmap_query(const void *table, size_t table_bytes, const int32_t *out_coords,
@@ -767,7 +899,7 @@ extern "C" lat_status lat_kmap_query(const void *table, size_t table_bytes, cons
     if (n_out > 0 && !out_coords) return LAT_ERR_ARG;
     if (geom->mode == LAT_SUBM && n_in != n_out) return LAT_ERR_ARG;  // the support is preserved
     if (reinterpret_cast<uintptr_t>(out_coords) % 16 || reinterpret_cast<uintptr_t>(table) % 64) return LAT_ERR_ARG;
-    const KmapWs need = carve_kmap_ws(nullptr, n_out, k3);
+    const KmapWs need = carve_kmap_ws(nullptr, n_out);
     if (ws_bytes < need.total || (need.total && !ws)) return LAT_ERR_WORKSPACE;
     map->mode = geom->mode;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -775,72 +907,71 @@ extern "C" lat_status lat_kmap_query(const void *table, size_t table_bytes, cons
         LAT_CUDA_TRY(cudaMemsetAsync(map->pair_off, 0, sizeof(int64_t) * (k3 + 1), s));
         return LAT_OK;
     }
-    KmapWs w = carve_kmap_ws(ws, n_out, k3);
-    Geom g{};
-    for (int a = 0; a < 3; ++a) {
-        g.ks[a] = geom->ksize[a];
-        g.st[a] = geom->stride[a];
-        g.pd[a] = geom->pad[a];
-    }
-    g.mode = geom->mode;
-    g.k3 = k3;
-    // unit stride: probed coordinate = own + sign * (off - pad), sign -1 for the transposed relation
-    g.shift = g.st[0] == 1 && g.st[1] == 1 && g.st[2] == 1;
-    const int sign = g.mode == LAT_TRANSPOSED ? -1 : 1;
-    int dmin[3] = {0, 0, 0}, dmax[3] = {0, 0, 0};
-    for (int a = 0; a < 3; ++a) {
-        const int d0 = sign * (0 - g.pd[a]), d1 = sign * (g.ks[a] - 1 - g.pd[a]);
-        dmin[a] = d0 < d1 ? d0 : d1;
-        dmax[a] = d0 < d1 ? d1 : d0;
-        g.lo[a] = -32768 - dmin[a];
-        g.hi[a] = 32767 - dmax[a];
-    }
-    for (int ix = 0, k = 0; ix < g.ks[0]; ++ix)
-        for (int iy = 0; iy < g.ks[1]; ++iy)
-            for (int iz = 0; iz < g.ks[2]; ++iz, ++k) {
-                g.off[k][0] = static_cast<signed char>(ix);
-                g.off[k][1] = static_cast<signed char>(iy);
-                g.off[k][2] = static_cast<signed char>(iz);
-                const long long dx = sign * (ix - g.pd[0]), dy = sign * (iy - g.pd[1]), dz = sign * (iz - g.pd[2]);
-                g.delta[k] = dx * (1ll << 32) + dy * (1ll << 16) + dz;
-            }
-    const int nblk = int((n_out + kQueryThreads - 1) / kQueryThreads);
+    const KmapWs w = carve_kmap_ws(ws, n_out);
     const int64_t ntiles = (n_out + LAT_TILE_ROWS - 1) / LAT_TILE_ROWS;
     const uint32_t cap_mask = uint32_t(table_bytes / kSlotBytes - 1);
     const SlotGroup *slots = static_cast<const SlotGroup *>(table);
     const int4 *oc = reinterpret_cast<const int4 *>(out_coords);
+    FillList f;
+    f.add(w.counters, w.zero_words, 0u);
+    f.add(map->tile_mask, ntiles, 0u);
+    LAT_CUDA_TRY(fill_list(f, s));
+    int centre = -1;
     if (geom->mode == LAT_SUBM) {
-        // the upper half of the table is filled by mirrored hits only
-        const int centre = k3 / 2;
-        LAT_CUDA_TRY(launch_pdl(kmap_subm_init_kernel, dim3(nblk), dim3(kQueryThreads), 0, s, n_out, k3, map->nbr,
-                                map->mask, w.hist, int64_t(w.hist_bytes / 4), map->tile_mask, ntiles));
-        LAT_CUDA_TRY(cudaGetLastError());
-        if (centre > 0) {
-            LAT_CUDA_TRY(launch_pdl(kmap_probe_sym_kernel, dim3(unsigned(nblk), unsigned(centre)), dim3(kQueryThreads),
-                                    0, s, slots, cap_mask, oc, n_out, g, map->nbr, map->mask, d_status));
-            LAT_CUDA_TRY(cudaGetLastError());
-        }
-        LAT_CUDA_TRY(launch_pdl(kmap_count_kernel, dim3(nblk), dim3(kQueryThreads), 0, s, map->mask, n_out, k3,
-                                w.block_counts, nblk, w.keys, w.hist, w.ntile));
+        SubmGeom g{geom->ksize[0], geom->ksize[1], geom->ksize[2], geom->pad[0], geom->pad[1], geom->pad[2], k3};
+        const dim3 grid(unsigned((n_out + kProbeRows - 1) / kProbeRows)), block(32 * g.kx * g.ky);
+        if (g.kz == 3)
+            LAT_CUDA_TRY(launch_pdl(subm_probe_kernel<3>, grid, block, 0, s, slots, cap_mask, oc, n_out, g, map->nbr,
+                                    map->mask, w.keys, w.counters, d_status));
+        else if (g.kz == 1)
+            LAT_CUDA_TRY(launch_pdl(subm_probe_kernel<1>, grid, block, 0, s, slots, cap_mask, oc, n_out, g, map->nbr,
+                                    map->mask, w.keys, w.counters, d_status));
+        else
+            LAT_CUDA_TRY(launch_pdl(subm_probe_kernel<0>, grid, block, 0, s, slots, cap_mask, oc, n_out, g, map->nbr,
+                                    map->mask, w.keys, w.counters, d_status));
+        centre = k3 / 2;
     } else {
-        FillList f;
-        f.add(w.hist, int64_t(w.hist_bytes / 4), 0u);
-        f.add(map->tile_mask, ntiles, 0u);
-        LAT_CUDA_TRY(fill_list(f, s));
+        Geom g{};
+        for (int a = 0; a < 3; ++a) {
+            g.ks[a] = geom->ksize[a];
+            g.st[a] = geom->stride[a];
+            g.pd[a] = geom->pad[a];
+        }
+        g.mode = geom->mode;
+        g.k3 = k3;
+        // unit stride: probed coordinate = own + sign * (off - pad), sign -1 for the transposed relation
+        g.shift = g.st[0] == 1 && g.st[1] == 1 && g.st[2] == 1;
+        const int sign = g.mode == LAT_TRANSPOSED ? -1 : 1;
+        for (int a = 0; a < 3; ++a) {
+            const int d0 = sign * (0 - g.pd[a]), d1 = sign * (g.ks[a] - 1 - g.pd[a]);
+            const int dmin = d0 < d1 ? d0 : d1, dmax = d0 < d1 ? d1 : d0;
+            g.lo[a] = -32768 - dmin;
+            g.hi[a] = 32767 - dmax;
+        }
+        for (int ix = 0, k = 0; ix < g.ks[0]; ++ix)
+            for (int iy = 0; iy < g.ks[1]; ++iy)
+                for (int iz = 0; iz < g.ks[2]; ++iz, ++k) {
+                    g.off[k][0] = static_cast<signed char>(ix);
+                    g.off[k][1] = static_cast<signed char>(iy);
+                    g.off[k][2] = static_cast<signed char>(iz);
+                    const long long dx = sign * (ix - g.pd[0]), dy = sign * (iy - g.pd[1]),
+                                    dz = sign * (iz - g.pd[2]);
+                    g.delta[k] = dx * (1ll << 32) + dy * (1ll << 16) + dz;
+                }
+        const int nblk = int((n_out + kQueryThreads - 1) / kQueryThreads);
         LAT_CUDA_TRY(launch_pdl(kmap_probe_kernel, dim3(nblk), dim3(kQueryThreads), 0, s, slots, cap_mask, oc, n_out,
-                                n_in, g, map->nbr, map->mask, w.keys, w.hist, w.ntile, w.block_counts, nblk, d_status));
+                                n_in, g, map->nbr, map->mask, w.keys, w.counters, d_status));
     }
     LAT_CUDA_TRY(cudaGetLastError());
-    SideStream *side = nullptr;
-    LAT_CUDA_TRY(side_stream(side));
-    return finish_kmap(map, k3, nblk, w, d_status, s, side);
+    return sweep_map(map, k3, w, centre, d_status, s);
 }
 
 extern "C" size_t lat_kmap_from_parent_ws_bytes(int64_t n_fine, int64_t n_coarse, int32_t k3) {
-    if (n_fine < 0 || n_coarse < 0 || n_fine >= (int64_t(1) << 31) || k3 < 1 || k3 > 32) return 0;
-    // the strided map's workspace, then the transposed map's (its keys are built
-    // before the strided map is finished)
-    return lat::carve_kmap_ws(nullptr, n_coarse, k3).total + lat::carve_kmap_ws(nullptr, n_fine, k3).total;
+    if (n_fine < 0 || n_coarse < 0 || n_fine >= (int64_t(1) << 31) || n_coarse >= (int64_t(1) << 31) || k3 < 1 ||
+        k3 > 32)
+        return 0;
+    // the strided map's workspace, then the transposed map's
+    return lat::carve_kmap_ws(nullptr, n_coarse).total + lat::carve_kmap_ws(nullptr, n_fine).total;
 }
 
 extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int32_t *parent, const lat_geom *geom,
@@ -864,23 +995,20 @@ extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (down) down->mode = LAT_STRIDED;
     if (up) up->mode = LAT_TRANSPOSED;
-    KmapWs w_down = carve_kmap_ws(ws, n_coarse, k3);
-    KmapWs w_up = carve_kmap_ws(static_cast<char *>(ws) + w_down.total, n_fine, k3);
-    // transposed map with K^3 <= 8: every fine row has one neighbour (its parent)
-    // and its key is the one-hot mask, so the row sort alone yields the pairs
-    const bool up_direct = up && n_fine > 0 && group_key_bits(k3) <= 8;
+    const KmapWs w_down = carve_kmap_ws(ws, n_coarse);
+    const KmapWs w_up = carve_kmap_ws(static_cast<char *>(ws) + w_down.total, n_fine);
     // every initialisation both maps need, in one launch: the strided map's
     // table (-1) and masks (0, both filled by the parent scatter), and each
-    // map's sort histograms and tile masks
+    // map's counters, look-back words and tile masks
     FillList f;
     if (down && n_coarse > 0) {
         f.add(down->nbr, int64_t(k3) * n_coarse, ~0u);
         f.add(down->mask, n_coarse, 0u);
-        f.add(w_down.hist, int64_t(w_down.hist_bytes / 4), 0u);
+        f.add(w_down.counters, w_down.zero_words, 0u);
         f.add(down->tile_mask, (n_coarse + LAT_TILE_ROWS - 1) / LAT_TILE_ROWS, 0u);
     }
     if (up && n_fine > 0) {
-        f.add(w_up.hist, int64_t(w_up.hist_bytes / 4), 0u);
+        f.add(w_up.counters, w_up.zero_words, 0u);
         f.add(up->tile_mask, (n_fine + LAT_TILE_ROWS - 1) / LAT_TILE_ROWS, 0u);
     }
     LAT_CUDA_TRY(fill_list(f, s));
@@ -888,8 +1016,8 @@ extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int
         LAT_CUDA_TRY(launch_pdl(parent_maps_kernel, dim3(unsigned((n_fine + 255) / 256)), dim3(256), 0, s,
                                 reinterpret_cast<const int4 *>(fine_coords), parent, n_fine, n_coarse, geom->stride[0],
                                 geom->stride[1], geom->stride[2], k3, up ? up->nbr : nullptr, up ? up->mask : nullptr,
-                                down ? down->nbr : nullptr, down ? down->mask : nullptr,
-                                up_direct ? w_up.keys : nullptr, w_up.hist, w_up.ntile, d_status));
+                                up ? w_up.keys : nullptr, w_up.counters, down ? down->nbr : nullptr,
+                                down ? down->mask : nullptr, d_status));
         LAT_CUDA_TRY(cudaGetLastError());
     }
     // the two maps are independent once the parent scatter is done: the
@@ -902,27 +1030,19 @@ extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int
     const cudaStream_t main_s = s;
     for (lat_kmap *map : {down, up}) {
         if (!map) continue;
-        const cudaStream_t s = (side && map == up) ? side->side : main_s;
+        const cudaStream_t ms = (side && map == up) ? side->side : main_s;
         if (map->n_out == 0) {
-            LAT_CUDA_TRY(cudaMemsetAsync(map->pair_off, 0, sizeof(int64_t) * (k3 + 1), s));
+            LAT_CUDA_TRY(cudaMemsetAsync(map->pair_off, 0, sizeof(int64_t) * (k3 + 1), ms));
             continue;
         }
-        KmapWs &w = map == down ? w_down : w_up;
-        if (map == up && up_direct) {
-            LAT_CUDA_TRY(launch_pdl(sort_rowscan_kernel, dim3(256), dim3(256), 0, s, w.hist, w.ntile, w.totals));
+        const KmapWs &w = map == down ? w_down : w_up;
+        if (map == down) {
+            const int nblk = int((map->n_out + kQueryThreads - 1) / kQueryThreads);
+            LAT_CUDA_TRY(launch_pdl(kmap_count_kernel, dim3(nblk), dim3(kQueryThreads), 0, ms, map->mask, map->n_out,
+                                    k3, w.keys, w.counters));
             LAT_CUDA_TRY(cudaGetLastError());
-            const PairOut po{parent, map->pair_in, map->pair_out, map->pair_capacity, map->pair_off, k3, d_status};
-            LAT_CUDA_TRY(launch_pdl(sort_scatter_kernel<true>, dim3(w.ntile), dim3(kSortThreads), 0, s, w.keys,
-                                    nullptr, map->n_out, 0, w.hist, w.totals, w.ntile, nullptr, map->perm, nullptr,
-                                    map->mask, map->tile_mask, po));
-            LAT_CUDA_TRY(cudaGetLastError());
-            continue;
         }
-        const int nblk = int((map->n_out + kQueryThreads - 1) / kQueryThreads);
-        LAT_CUDA_TRY(launch_pdl(kmap_count_kernel, dim3(nblk), dim3(kQueryThreads), 0, s, map->mask, map->n_out, k3,
-                                w.block_counts, nblk, w.keys, w.hist, w.ntile));
-        LAT_CUDA_TRY(cudaGetLastError());
-        const lat_status st = finish_kmap(map, k3, nblk, w, d_status, s, nullptr);
+        const lat_status st = sweep_map(map, k3, w, -1, d_status, ms);
         if (st != LAT_OK) return st;
     }
     if (side) LAT_CUDA_TRY(side_join(*side, main_s));

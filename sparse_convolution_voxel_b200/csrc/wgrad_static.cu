@@ -5,15 +5,16 @@
 // while a stream is being captured into a CUDA graph without memory nodes,
 // real-time loops that forbid cudaMalloc/cudaFree (a device-wide
 // synchronisation) after start-up, or hosts whose allocator is owned by
-// someone else.  This entry point runs the same chunked weight-gradient
-// kernels as lat_sconv_wgrad, but its scratch (chunk table + per-chunk fp32
-// partials) lives in one file-scope __device__ array that every GPU loading
-// the library holds until the process exits.
+// someone else.  This entry point runs the same share-based weight-gradient
+// kernels as lat_sconv_wgrad's CUDA-core path, but its scratch (the fp32
+// partials of every (share, offset) segment) lives in one file-scope
+// __device__ array that every GPU loading the library holds until the
+// process exits.
 //
 // Host code must not pass the array's name to a kernel: on the host it is
-// only a stand-in symbol.  Its device address is fetched once per device
-// with cudaGetSymbolAddress, with that device current, on the first call
-// made on that device.
+// only a stand-in symbol.  Its device address is fetched per device with
+// cudaGetSymbolAddress, with that device current, by the first call on that
+// device that succeeds in looking it up, and kept from then on.
 #include <mutex>
 
 #include "common.cuh"
@@ -25,22 +26,27 @@ namespace {
 static __device__ __align__(256) unsigned char g_wgrad_scratch[LAT_WGRAD_STATIC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_once[kMaxDevices];
-void *g_scratch_addr[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
+std::mutex g_mu;
+void *g_scratch_addr[kMaxDevices];  // nullptr until a lookup on that device succeeded
 
-// Device address of g_wgrad_scratch on the current device (set up on first use).
+// Device address of g_wgrad_scratch on the current device.  Only a successful
+// lookup is kept; a failed one (its error cleared, so that it does not show
+// up in later launch checks) is reported and tried again on the next call.
 cudaError_t static_scratch(void **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::call_once(g_once[dev], [dev] {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_scratch_addr[dev]) {
         void *p = nullptr;
-        g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_wgrad_scratch);
+        e = cudaGetSymbolAddress(&p, g_wgrad_scratch);
+        if (e != cudaSuccess || !p) {
+            cudaGetLastError();
+            return e != cudaSuccess ? e : cudaErrorUnknown;
+        }
         g_scratch_addr[dev] = p;
-    });
-    if (g_scratch_err[dev] != cudaSuccess) return g_scratch_err[dev];
+    }
     *out = g_scratch_addr[dev];
     return cudaSuccess;
 }
@@ -65,7 +71,8 @@ extern "C" lat_status lat_sconv_wgrad_static(const void *x, int32_t cin, const v
     auto a16 = [](const void *p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; };
     if (!a16(x) || !a16(dy) || !a16(dw)) return LAT_ERR_ARG;
     // every byte of scratch this call reads is written earlier in the same call,
-    // so nothing left over from a previous call needs clearing
+    // so nothing left over from a previous call needs clearing; every check
+    // comes before the first launch
     if (wgrad_simt_ws_bytes(cin, cout, map) > size_t(LAT_WGRAD_STATIC_SCRATCH_BYTES)) return LAT_ERR_WORKSPACE;
     void *scratch = nullptr;
     if (static_scratch(&scratch) != cudaSuccess) return LAT_ERR_CUDA;

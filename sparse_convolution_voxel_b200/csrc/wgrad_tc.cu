@@ -3,7 +3,8 @@
 //
 // Per offset this is a GEMM with M = Cin, N = Cout and the pairs as the
 // reduction dimension.  The pair list (grouped by offset by the kernel-map
-// query) is cut into kWorkers equal contiguous shares -- a constant, so the
+// query) is cut into kWorkers equal contiguous shares (fewer when there are
+// fewer pairs than that, so that no share is empty) -- a constant, so the
 // cut does not depend on the GPU -- and persistent CTAs (two per SM) take the
 // shares round-robin.  A share is processed as segments, its intersections
 // with the offsets' pair ranges; a segment accumulates in TMEM and ends in one
@@ -30,7 +31,7 @@ constexpr int kWorkers = 296;      // equal shares of the pair list (two per B20
 constexpr int kProdWarps = 4, kEpiWarps = 4;
 constexpr int kMmaWarp = kProdWarps + kEpiWarps;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
-constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr uint64_t kDrainNs = 1000000000ull;  // limit of the waits that drain a CTA that gave up
 
 template <int M, int N>
 struct Cfg {
@@ -59,13 +60,16 @@ __device__ __forceinline__ void load_offsets(const int64_t *pair_off, int64_t ca
     for (int e = threadIdx.x & 31; e <= k3; e += 32) off[e] = min(pair_off[e], capacity);
 }
 
-// Share v of the pair list: pairs [P v / kWorkers, P (v+1) / kWorkers).
-__device__ __forceinline__ int64_t share_lo(int64_t P, int v) { return P * v / kWorkers; }
+// Shares of a list of P pairs: min(kWorkers, P), so that no share is empty
+// (every share then writes the partials its slots stand for).
+__device__ __forceinline__ int share_count(int64_t P) { return int(min(int64_t(kWorkers), P)); }
 
-// The share holding pair `pair` (largest v with share_lo(P, v) <= pair); a binary
-// search, so only divisions by the constant kWorkers.
+// Share v of the pair list: pairs [P v / S, P (v+1) / S), S = share_count(P).
+__device__ __forceinline__ int64_t share_lo(int64_t P, int v) { return P * v / share_count(P); }
+
+// The share holding pair `pair` (largest v with share_lo(P, v) <= pair); a binary search.
 __device__ __forceinline__ int share_of(int64_t P, int64_t pair) {
-    int lo = 0, hi = kWorkers - 1;
+    int lo = 0, hi = share_count(P) - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (share_lo(P, mid) <= pair) lo = mid;
@@ -100,7 +104,7 @@ struct Segments {
                 }
             }
             v += gridDim.x;
-            if (v >= kWorkers) return false;
+            if (v >= share_count(P)) return false;
             const int64_t wl = share_lo(P, v);
             hv = share_lo(P, v + 1);
             k = 0;
@@ -114,8 +118,9 @@ __global__ void __launch_bounds__(kThreads, 2)
 wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t *__restrict__ pair_off,
                 const int32_t *__restrict__ pair_in, const int32_t *__restrict__ pair_out, int64_t capacity, int k3,
                 int64_t n_in, int64_t n_out, float *__restrict__ partial, int32_t *__restrict__ ranges,
-                int32_t *d_status) {
+                uint64_t wait_ns, int32_t *d_status) {
     pdl_enter();
+    const uint64_t kWaitNs = wait_ns;
     using C = Cfg<M, N>;
     constexpr int NS = C::kStages;
     constexpr uint32_t idesc = make_idesc<T, M, N>();
@@ -126,7 +131,8 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
     uint64_t *empty = full + NS;
     uint64_t *accfull = empty + NS;
     uint64_t *accempty = accfull + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accempty + 2);
+    uint64_t *drain = accempty + 2;  // tracks the MMAs still in flight when a CTA gives up
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     __shared__ int s_abort;
     __shared__ int64_t s_off[33];
 
@@ -150,6 +156,7 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
             ptx::mbar_init(&accfull[a], 1);
             ptx::mbar_init(&accempty[a], kEpiWarps * 32);
         }
+        ptx::mbar_init(drain, 1);
         s_abort = 0;
         ptx::fence_mbar_init();
         ptx::fence_proxy_async_smem();
@@ -317,8 +324,16 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
 
     __syncthreads();
     if (s_abort) {
+        // A role gave up: every thread's cp.async copies are complete
+        // (cp.async.wait_all above); the MMA thread commits every MMA it issued
+        // to `drain` and waits for it (with its own limit) before the TMEM and
+        // shared memory are released.
         bad |= (tid == 0) ? LAT_ERR_TIMEOUT : 0;
-        __nanosleep(1000000);
+        if (warp == kMmaWarp && lane == 0) {
+            ptx::umma_commit(drain);
+            ptx::mbar_wait(drain, 0, kDrainNs);
+        }
+        __syncthreads();
     }
     if (bad) flag(d_status, bad);
     if (warp == 0) {
@@ -380,7 +395,7 @@ static lat_status launch(const void *x, const void *dy, const lat_kmap *map, flo
     if (grid <= 0) return LAT_ERR_CUDA;
     LAT_CUDA_TRY(launch_pdl(kern, dim3(unsigned(grid)), dim3(kThreads), C::kSmem, s, static_cast<const T *>(x),
                             static_cast<const T *>(dy), map->pair_off, map->pair_in, map->pair_out, map->pair_capacity,
-                            map->k3, map->n_in, map->n_out, partial, ranges, d_status));
+                            map->k3, map->n_in, map->n_out, partial, ranges, wait_limit_ns(), d_status));
     LAT_CUDA_TRY(cudaGetLastError());
     const int nelem = M * N;
     dim3 rg((nelem + 31) / 32, map->k3);

@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import synthetic
-from tests.util import TORCH_DT, assert_close, check_kmap, feats, rand_coords, weights
+from tests.util import TORCH_DT, assert_close, check_kmap, feats, rand_coords, weights, with_terms
 
 pytestmark = pytest.mark.gpu
 
@@ -44,7 +44,7 @@ def test_subm_fwd_small(dtype, cin, cout):
     st = scv.new_status()
     y = scv.conv_fwd(x, w, km, d_status=st)
     scv.check_status(st)
-    assert_close(y.double().cpu().numpy(), oracle.conv_fwd(x64, w64, ref_nbr), dtype, "fwd")
+    assert_close(y.double().cpu().numpy(), with_terms(oracle.conv_fwd, x64, w64, ref_nbr), dtype, "fwd")
 
 
 @pytest.mark.parametrize("dtype", DTYPES)
@@ -77,7 +77,7 @@ def test_subm_fwd_full_workloads(name):
     x, x64 = feats(len(coords), wl.cin, dtype, seed=wl.seed)
     w, w64 = weights(k3, wl.cin, wl.cout, dtype, seed=wl.seed)
     y = scv.conv_fwd(x, w, km)
-    assert_close(y.double().cpu().numpy(), oracle.conv_fwd(x64, w64, ref_nbr), dtype, name)
+    assert_close(y.double().cpu().numpy(), with_terms(oracle.conv_fwd, x64, w64, ref_nbr), dtype, name)
 
 
 def test_down_up_full_workload():
@@ -94,12 +94,12 @@ def test_down_up_full_workload():
     wd, wd64 = weights(8, 64, 128, dtype, seed=3)
     wu, wu64 = weights(8, 128, 64, dtype, seed=3, stream=1)
     y = scv.conv_fwd(x, wd, down)
-    ref_y = oracle.conv_fwd(x64, wd64, oracle.kmap(coords, ref_coarse, 2, 2, 0, oracle.STRIDED))
+    ref_y = with_terms(oracle.conv_fwd, x64, wd64, oracle.kmap(coords, ref_coarse, 2, 2, 0, oracle.STRIDED))
     assert_close(y.double().cpu().numpy(), ref_y, dtype, "down")
     # the up pass consumes the GPU's rounded coarse features, as the layer chain would
     y64 = y.double().cpu().numpy()
     z = scv.conv_fwd(y, wu, up)
-    ref_z = oracle.conv_fwd(y64, wu64, oracle.kmap(ref_coarse, coords, 2, 2, 0, oracle.TRANSPOSED))
+    ref_z = with_terms(oracle.conv_fwd, y64, wu64, oracle.kmap(ref_coarse, coords, 2, 2, 0, oracle.TRANSPOSED))
     assert_close(z.double().cpu().numpy(), ref_z, dtype, "up")
 
 
@@ -117,8 +117,9 @@ def test_subm_dgrad_wgrad_small(dtype, cin, cout):
     dx = scv.conv_dgrad(g, w, km, flip_offsets=True, d_status=st)
     dw = scv.conv_wgrad(x, g, km, d_status=st)
     scv.check_status(st)
-    assert_close(dx.double().cpu().numpy(), oracle.conv_dgrad(g64, w64, ref_nbr, len(coords)), dtype, "dgrad")
-    assert_close(dw.double().cpu().numpy(), oracle.conv_wgrad(x64, g64, ref_nbr), dtype, "wgrad")
+    assert_close(dx.double().cpu().numpy(), with_terms(oracle.conv_dgrad, g64, w64, ref_nbr, len(coords)),
+                 dtype, "dgrad")
+    assert_close(dw.double().cpu().numpy(), with_terms(oracle.conv_wgrad, x64, g64, ref_nbr), dtype, "wgrad")
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
@@ -138,16 +139,18 @@ def test_strided_and_transposed_backward(dtype):
     gy, gy64 = feats(len(rc), 128, dtype, seed=9, stream=2)
     # strided Conv3d: dgrad walks the transposed map, wgrad uses the forward pairs
     dx = scv.conv_dgrad(gy, w, up, flip_offsets=False)
-    assert_close(dx.double().cpu().numpy(), oracle.conv_dgrad(gy64, w64, ref_down, len(coords)), dtype, "down dgrad")
+    assert_close(dx.double().cpu().numpy(), with_terms(oracle.conv_dgrad, gy64, w64, ref_down, len(coords)),
+                 dtype, "down dgrad")
     dw = scv.conv_wgrad(x, gy, down)
-    assert_close(dw.double().cpu().numpy(), oracle.conv_wgrad(x64, gy64, ref_down), dtype, "down wgrad")
+    assert_close(dw.double().cpu().numpy(), with_terms(oracle.conv_wgrad, x64, gy64, ref_down), dtype, "down wgrad")
     # ConvTranspose3d: dgrad walks the strided map
     wt, wt64 = weights(8, 128, 64, dtype, seed=9, stream=3)
     gz, gz64 = feats(len(coords), 64, dtype, seed=9, stream=4)
     dyc = scv.conv_dgrad(gz, wt, down, flip_offsets=False)
-    assert_close(dyc.double().cpu().numpy(), oracle.conv_dgrad(gz64, wt64, ref_up, len(rc)), dtype, "up dgrad")
+    assert_close(dyc.double().cpu().numpy(), with_terms(oracle.conv_dgrad, gz64, wt64, ref_up, len(rc)),
+                 dtype, "up dgrad")
     dwt = scv.conv_wgrad(gy, gz, up)
-    assert_close(dwt.double().cpu().numpy(), oracle.conv_wgrad(gy64, gz64, ref_up), dtype, "up wgrad")
+    assert_close(dwt.double().cpu().numpy(), with_terms(oracle.conv_wgrad, gy64, gz64, ref_up), dtype, "up wgrad")
 
 
 def test_training_step_full_workload():
@@ -161,9 +164,10 @@ def test_training_step_full_workload():
     y = scv.conv_fwd(x, w, km)
     dx = scv.conv_dgrad(g, w, km, flip_offsets=True)
     dw = scv.conv_wgrad(x, g, km)
-    assert_close(y.double().cpu().numpy(), oracle.conv_fwd(x64, w64, ref_nbr), dtype, "fwd")
-    assert_close(dx.double().cpu().numpy(), oracle.conv_dgrad(g64, w64, ref_nbr, len(coords)), dtype, "dgrad")
-    assert_close(dw.double().cpu().numpy(), oracle.conv_wgrad(x64, g64, ref_nbr), dtype, "wgrad")
+    assert_close(y.double().cpu().numpy(), with_terms(oracle.conv_fwd, x64, w64, ref_nbr), dtype, "fwd")
+    assert_close(dx.double().cpu().numpy(), with_terms(oracle.conv_dgrad, g64, w64, ref_nbr, len(coords)),
+                 dtype, "dgrad")
+    assert_close(dw.double().cpu().numpy(), with_terms(oracle.conv_wgrad, x64, g64, ref_nbr), dtype, "wgrad")
 
 
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
@@ -183,7 +187,7 @@ def test_transposed_fwd_with_rows_without_neighbours(dtype):
     x, x64 = feats(len(rc), 64, dtype, seed=29)
     w, w64 = weights(6, 64, 64, dtype, seed=29)
     z = scv.conv_fwd(x, w, up, out=torch.full((len(coords), 64), 3.0, dtype=dtype, device="cuda"))
-    assert_close(z.double().cpu().numpy(), oracle.conv_fwd(x64, w64, ref_up), dtype, "transposed fwd")
+    assert_close(z.double().cpu().numpy(), with_terms(oracle.conv_fwd, x64, w64, ref_up), dtype, "transposed fwd")
 
 
 @pytest.mark.parametrize("dtype", [torch.float16, torch.float32])
@@ -199,7 +203,7 @@ def test_target_conv(dtype):
     x, x64 = feats(len(coords), 64, dtype, seed=47)
     w, w64 = weights(27, 64, 64, dtype, seed=47)
     y = scv.conv_fwd(x, w, km)
-    assert_close(y.double().cpu().numpy(), oracle.conv_fwd(x64, w64, ref_nbr), dtype, "target conv")
+    assert_close(y.double().cpu().numpy(), with_terms(oracle.conv_fwd, x64, w64, ref_nbr), dtype, "target conv")
 
 
 # --------------------------------------------------------------------------- generative stride-1 Conv3d
@@ -232,14 +236,14 @@ def test_generative_stride1_conv(dtype, ks):
     x, x64 = feats(len(coords), cin, dtype, seed=9)
     w, w64 = weights(k3, cin, cout, dtype, seed=9)
     y = scv.conv_fwd(x, w, km, d_status=st)
-    assert_close(y.double().cpu().numpy(), oracle.conv_fwd(x64, w64, ref_nbr), dtype, "generative fwd")
+    assert_close(y.double().cpu().numpy(), with_terms(oracle.conv_fwd, x64, w64, ref_nbr), dtype, "generative fwd")
     # data gradient through the opposite relation (grown rows -> input rows)
     gy, gy64 = feats(len(ref_grown), cout, dtype, seed=9, stream=1)
     back = scv.kernel_map(scv.hash_table(grown, 2.0, st), len(ref_grown), c, scv.transposed_geom(ks, 1, pad),
                           d_status=st)
     dx = scv.conv_dgrad(gy, w, back, flip_offsets=False, d_status=st)
     scv.check_status(st)
-    assert_close(dx.double().cpu().numpy(), oracle.conv_dgrad(gy64, w64, ref_nbr, len(coords)), dtype,
+    assert_close(dx.double().cpu().numpy(), with_terms(oracle.conv_dgrad, gy64, w64, ref_nbr, len(coords)), dtype,
                  "generative dgrad")
 
 
@@ -266,14 +270,15 @@ def test_generative_transposed_conv(dtype, ks, st_, pd):
     x, x64 = feats(len(coarse), cin, dtype, seed=13)
     w, w64 = weights(k3, cin, cout, dtype, seed=13)
     y = scv.conv_fwd(x, w, km, d_status=st)
-    assert_close(y.double().cpu().numpy(), oracle.conv_fwd(x64, w64, ref_nbr), dtype, "generative transposed fwd")
+    assert_close(y.double().cpu().numpy(), with_terms(oracle.conv_fwd, x64, w64, ref_nbr),
+                 dtype, "generative transposed fwd")
     # data gradient back to the coarse rows through the strided relation
     gy, gy64 = feats(len(ref_fine), cout, dtype, seed=13, stream=1)
     back = scv.kernel_map(scv.hash_table(fine, 2.0, st), len(ref_fine), c, scv.strided_geom(ks, st_, pd),
                           d_status=st)
     dx = scv.conv_dgrad(gy, w, back, flip_offsets=False, d_status=st)
     scv.check_status(st)
-    assert_close(dx.double().cpu().numpy(), oracle.conv_dgrad(gy64, w64, ref_nbr, len(coarse)), dtype,
+    assert_close(dx.double().cpu().numpy(), with_terms(oracle.conv_dgrad, gy64, w64, ref_nbr, len(coarse)), dtype,
                  "generative transposed dgrad")
 
 
@@ -296,4 +301,4 @@ def test_tc_fwd_output_16_byte_aligned(dtype, cout):
     torch.cuda.synchronize()
     assert torch.equal(y_al, y_off)
     assert torch.all(flat[:8] == 7.0)
-    assert_close(y_al.double().cpu().numpy(), oracle.conv_fwd(x64, w64, ref_nbr), dtype, "aligned fwd")
+    assert_close(y_al.double().cpu().numpy(), with_terms(oracle.conv_fwd, x64, w64, ref_nbr), dtype, "aligned fwd")

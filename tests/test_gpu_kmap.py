@@ -22,9 +22,11 @@ def _dev(a):
 
 
 def _slot_hash(key: int) -> int:
-    """The table's placement function (fold of the key halves + MurmurHash3 fmix32),
+    """The table's placement function (fold of the halves of the key's z-brick, the
+    key with the two low bits of its z field cleared, then MurmurHash3 fmix32),
     restated here to check where the GPU put every key."""
     M = 0xFFFFFFFF
+    key &= ~3
     h = (key & M) ^ (((key >> 32) * 0x9E3779B1) & M)
     h ^= h >> 16
     h = (h * 0x85EBCA6B) & M
@@ -107,6 +109,48 @@ def test_subm_kmap_small_ragged(n, batch, lo, hi):
     check_kmap(km, oracle.kmap(coords, coords, 3, 1, 1, oracle.SUBM))
 
 
+@pytest.mark.parametrize("ratio", [1.0, 2.0, 4.0])
+def test_subm_kmap_dense_cube(ratio):
+    """Every cell of an 11^3 cube in two batches: each z-brick holds 4 keys, so
+    home groups fill up and probes run on into the following groups (at ratio 1
+    the table is 65% full)."""
+    ax = np.arange(-5, 6)
+    g = np.stack(np.meshgrid(ax, ax, ax, indexing="ij"), -1).reshape(-1, 3)
+    coords = np.concatenate([np.c_[np.full(len(g), b), g] for b in range(2)]).astype(np.int32)
+    coords = np.ascontiguousarray(coords[np.random.default_rng(1).permutation(len(coords))])
+    c = _dev(coords)
+    st = scv.new_status()
+    table = scv.hash_table(c, ratio, st)
+    km = scv.kernel_map(table, len(coords), c, scv.subm_geom(3), d_status=st)
+    scv.check_status(st)
+    check_kmap(km, oracle.kmap(coords, coords, 3, 1, 1, oracle.SUBM))
+    keys, rows = _table_slots(table)
+    cap = len(keys)
+    empty = np.uint64(0xFFFFFFFFFFFFFFFF)
+    for s in np.nonzero(keys != empty)[0]:
+        start = _slot_hash(int(keys[s])) & (cap - 1) & ~3
+        d = (s - start) % cap
+        assert all(keys[(start + e) % cap] != empty for e in range(d))
+
+
+def test_subm_kmap_at_the_edges_of_the_key_range():
+    """Rows packed against the key range (x, y, z at -32768 / 32767, batch 0 and
+    65534): neighbours outside the range are absent, never wrapped around."""
+    rows = []
+    for b in (0, 65534):
+        for xs in ((-32768, -32767, -32766), (32765, 32766, 32767)):
+            for zs in ((-32768, -32767, -32766, -32765), (32764, 32765, 32766, 32767)):
+                for x in xs:
+                    for y in (-32768, -32767, 32766, 32767):
+                        for z in zs:
+                            rows.append((b, x, y, z))
+    coords = np.array(rows, np.int32)
+    coords = np.ascontiguousarray(coords[np.random.default_rng(2).permutation(len(coords))])
+    for ks in ((3, 3, 3), (3, 3, 1), (1, 1, 5)):
+        km, _ = _subm(coords, ks)
+        check_kmap(km, oracle.kmap(coords, coords, ks, 1, oracle.subm_pad(ks), oracle.SUBM))
+
+
 def test_subm_kmap_empty():
     coords = np.zeros((0, 4), np.int32)
     km, _ = _subm(coords)
@@ -114,7 +158,8 @@ def test_subm_kmap_empty():
     assert km.pair_off.cpu().numpy().tolist() == [0] * 28
 
 
-@pytest.mark.parametrize("ks", [(5, 3, 1), (1, 1, 1), (3, 3, 1), (5, 5, 1)])
+@pytest.mark.parametrize("ks", [(5, 3, 1), (1, 1, 1), (3, 3, 1), (5, 5, 1), (1, 1, 5), (3, 1, 5), (1, 3, 7),
+                                (1, 5, 3)])
 def test_subm_kmap_other_kernels(ks):
     rng = np.random.default_rng(3)
     coords = rand_coords(rng, 700, -9, 9, 2)

@@ -70,10 +70,13 @@ def test_static_scratch_wgrad_rejects_problems_above_its_limit():
     rng = np.random.default_rng(3)
     coords = rand_coords(rng, 200, 0, 8)
     km = _map(coords)
-    big = scv.lat_kmap.from_buffer_copy(km.c)
-    big.pair_capacity = 3_000_000                     # 64 x 64 partials for 3M pair slots exceed 32 MiB
-    x = torch.zeros((len(coords), 64), dtype=torch.float16, device="cuda")
-    dw = torch.zeros((27, 64, 64), dtype=torch.float32, device="cuda")
-    rc = scv.load().lat_sconv_wgrad_static(ctypes.c_void_p(x.data_ptr()), 64, ctypes.c_void_p(x.data_ptr()), 64,
-                                           ctypes.byref(big), ctypes.c_void_p(dw.data_ptr()), 1, None, None)
+    x = torch.zeros((len(coords), 256), dtype=torch.float16, device="cuda")
+    dw = torch.zeros((27, 256, 256), dtype=torch.float32, device="cuda")
+    # (296 + 27) partials of 256 x 256 fp32 need 84.7 MB, above the 32 MiB array
+    rc = scv.load().lat_sconv_wgrad_static(ctypes.c_void_p(x.data_ptr()), 256, ctypes.c_void_p(x.data_ptr()), 256,
+                                           ctypes.byref(km.c), ctypes.c_void_p(dw.data_ptr()), 1, None, None)
     assert rc == 128                                  # LAT_ERR_WORKSPACE, nothing enqueued
+    # the limit is in channels only: 128 x 192 fits whatever the pair capacity
+    big = scv.lat_kmap.from_buffer_copy(km.c)
+    big.pair_capacity = 50_000_000
+    assert scv.lat_sconv_ws_bytes(2, 128, 192, big, torch.float32) <= 32 << 20
