@@ -5,31 +5,27 @@
 // and coordinate query are CUDA kernels of the library ("What remains
 // familiar", "Sparse tensor expectations"), and the support semantics come
 // from the "Convolution mapping" table.  Pipeline of one map (all on
-// `stream`; four launches for a submanifold map with K^3 > 8):
-//   0. fill:   zeroes the global counters, the sweeps' look-back state and
-//              the tile masks.
+// `stream`):
+//   0. fill:   zeroes the per-tile counts and the tile masks (submanifold maps:
+//              also -1 in the offsets above the centre, centre bit in every mask).
 //   1. front end: nbr (offset-major), the neighbour mask and the grouping key
-//              of every output row, plus global totals: hits per offset and
-//              the histograms of both bytes of the key.
-//                submanifold maps:  subm_probe_kernel (one warp per kernel
-//                                   column (ix, iy); one probe of a z-brick
-//                                   answers the column's Kz offsets)
+//              of every output row, and per tile of kScTile rows the counts of
+//              the key's low byte and of the pairs of every offset.
+//                submanifold: kmap_probe_sym_kernel (one thread per (row,
+//                                   offset below the centre), each hit mirrored
+//                                   into the upper half) + kmap_count_kernel
 //                strided/transposed: kmap_probe_kernel (a row per thread)
 //                maps from parents: parent_maps_kernel (+ kmap_count_kernel)
-//   2. sweep 1: the pair lists (grouped by offset, output rows ascending) and
-//              the first stable radix pass of the rows by the key's low byte.
-//   3. sweep 2: the second pass (high byte) -> perm, and the tile masks.
-//              With K^3 <= 8 the key is the mask itself (one byte) and
-//              sweep 1 writes perm and the tile masks directly.
-// The sweeps cut the rows into tiles of kSwTile positions; a tile learns
-// where its rows go from its predecessors' counts by decoupled look-back
-// (Merrill and Garland, "Single-pass Parallel Prefix Scan with Decoupled
-// Look-back", 2016; Adinets and Merrill's one-sweep radix sort uses it once
-// per digit): it publishes its own counts, then walks back over the earlier
-// tiles until it meets one that has published an inclusive prefix.  Tiles
-// are numbered in the order blocks start, so every tile it waits for is
-// already running; every wait is bounded.  Ranks inside a tile keep row
-// order, so the sort is stable and every output is deterministic.
+//   2. row scan: one block per digit (and per offset) turns its per-tile
+//              counts into tile starts and a total.
+//   3. scatter 1: the pair lists (grouped by offset, output rows ascending)
+//              and the first stable radix pass of the rows by the key's low
+//              byte, counting the high byte per output tile.
+//   4. row scan, 5. scatter 2: the second pass (high byte) -> perm and the
+//              tile masks.  With K^3 <= 8 the key is the mask itself (one
+//              byte) and scatter 1 writes perm and the tile masks directly.
+// Ranks inside a tile keep row order, so the sort is stable and every output
+// is deterministic.
 #include "common.cuh"
 
 namespace lat {
@@ -65,30 +61,30 @@ __device__ __forceinline__ uint32_t group_key(uint32_t m, int k3) {
 }
 __host__ __device__ inline int group_key_bits(int k3) { return k3 <= 8 ? k3 : kGroupKeyBits; }
 
-// ----------------------------------------------------------------------------- global totals
-// counters[0..255]: histogram of the key's low byte, [256..511]: of its high
-// byte, [512..543]: hits per offset, [544], [545]: tile counters of the two
-// sweeps.  Zero before the front end runs.
-constexpr int kCntHist = 0, kCntOff = 512, kCntTile = 544, kCntWords = 576;
+// ----------------------------------------------------------------------------- per-tile counts
+// The scatter passes work on tiles of kScTile rows.  Their first pass needs,
+// per tile, the count of every value of the key's low byte and of the pairs
+// of every offset: chain c (c < 256: digit c, 256 + k: offset k) of tile b at
+// cnt[c * ntile + b].  Front-end blocks cover whole rows of one tile and add
+// their block's counts with one atomic per nonzero value.
+constexpr int kScThreads = 256;
+constexpr int kScWarps = kScThreads / 32;
+constexpr int kScRounds = 2;
+constexpr int kScTile = kScThreads * kScRounds;  // rows per scatter tile
+constexpr int kChains = 256 + 32;
 
-// Shared-memory tallies of one block (s_h: both key-byte histograms, s_o: hits
-// per offset), added to the global counters once at the end of the block.
+// Shared-memory tallies of one block (s_h: the key's low byte, s_o: pairs per offset).
 struct Tally {
-    int *s_h;  // [512]
+    int *s_h;  // [256]
     int *s_o;  // [32]
 };
 
 // Counts one row per lane into the block's tallies; every lane of the warp calls it.
-__device__ __forceinline__ void tally_row(const Tally &ty, uint32_t key, uint32_t m, bool live, bool two) {
+__device__ __forceinline__ void tally_row(const Tally &ty, uint32_t key, uint32_t m, bool live) {
     const int lane = threadIdx.x & 31;
     const uint32_t d0 = key & 255u;
-    unsigned peers = __match_any_sync(0xFFFFFFFFu, live ? d0 : 256u + lane);
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, live ? d0 : 256u + lane);
     if (live && (peers & ((1u << lane) - 1u)) == 0) atomicAdd(&ty.s_h[d0], int(__popc(peers)));
-    if (two) {
-        const uint32_t d1 = (key >> 8) & 255u;
-        peers = __match_any_sync(0xFFFFFFFFu, live ? d1 : 256u + lane);
-        if (live && (peers & ((1u << lane) - 1u)) == 0) atomicAdd(&ty.s_h[256 + d1], int(__popc(peers)));
-    }
     const uint32_t mm = live ? m : 0u;
     for (uint32_t any = __reduce_or_sync(0xFFFFFFFFu, mm); any; any &= any - 1) {
         const int k = __ffs(any) - 1;
@@ -98,19 +94,15 @@ __device__ __forceinline__ void tally_row(const Tally &ty, uint32_t key, uint32_
 }
 
 __device__ __forceinline__ void tally_clear(const Tally &ty) {
-    for (int i = threadIdx.x; i < 512 + 32; i += blockDim.x) (i < 512 ? ty.s_h[i] : ty.s_o[i - 512]) = 0;
+    for (int i = threadIdx.x; i < 256 + 32; i += blockDim.x) (i < 256 ? ty.s_h[i] : ty.s_o[i - 256]) = 0;
 }
 
-// Adds the block's tallies to the global counters (after a __syncthreads()).
-__device__ __forceinline__ void tally_flush(const Tally &ty, int k3, bool two, int32_t *counters) {
-    for (int i = threadIdx.x; i < 512 + 32; i += blockDim.x) {
-        if (i < 512) {
-            const int v = ty.s_h[i];
-            if (v && (i < 256 || two)) atomicAdd(counters + kCntHist + i, v);
-        } else if (i - 512 < k3) {
-            const int v = ty.s_o[i - 512];
-            if (v) atomicAdd(counters + kCntOff + (i - 512), v);
-        }
+// Adds the block's tallies to its tile's counts (after a __syncthreads()).
+__device__ __forceinline__ void tally_flush(const Tally &ty, int k3, int32_t *cnt, int ntile, int64_t first_row) {
+    const int64_t tile = first_row / kScTile;
+    for (int i = threadIdx.x; i < 256 + k3; i += blockDim.x) {
+        const int v = i < 256 ? ty.s_h[i] : ty.s_o[i - 256];
+        if (v) atomicAdd(cnt + int64_t(i) * ntile + tile, v);
     }
 }
 
@@ -142,188 +134,85 @@ __device__ __forceinline__ int probe_one(const SlotGroup *groups, uint32_t cap_m
     return -1;
 }
 
-// Searches one kernel column (b, X, Y) for its KZ targets z_t = zlo + t
-// (t = 0..KZ-1, bit t of `want` set for the ones to look up), given as the
-// column's upper key word col_hi = b<<16 | X field, the Y field and the z
-// field zf0 of target 0.  A slot holds target t iff its upper 48 bits equal
-// the column's and its z field is zf0 + t.  Every key lives in the probe
-// sequence of its z-brick (probe_start ignores the low two bits of the z
-// field), so KZ <= 5 consecutive targets need at most two sequences, A for
-// the first wanted target's brick and B for the last's; both are read at once
-// and each is walked until its targets are found or it shows an empty slot
-// (no key of that brick lies beyond an empty slot of its sequence).  Bounded
-// by the probe window.  slot_of[t] = the slot of target t, or -1.
-template <int KZ>
-__device__ __forceinline__ void probe_column(const SlotGroup *groups, uint32_t cap_mask, uint32_t col_hi,
-                                             uint32_t col_y, int zf0, uint32_t want, int (&slot_of)[KZ]) {
-    static_assert(KZ >= 1 && KZ <= 5, "two z-bricks at most");
-#pragma unroll
-    for (int t = 0; t < KZ; ++t) slot_of[t] = -1;
-    if (!want) return;
-    const int t_lo = __ffs(want) - 1, t_hi = 31 - __clz(want);
-    const uint32_t b_lo = uint32_t(zf0 + t_lo) >> 2, b_hi = uint32_t(zf0 + t_hi) >> 2;
-    const uint64_t colkey = (uint64_t(col_hi) << 32) | (uint64_t(col_y) << 16);
-    uint32_t want_a = 0;
-#pragma unroll
-    for (int t = 0; t < KZ; ++t)
-        if (((want >> t) & 1u) && (uint32_t(zf0 + t) >> 2) == b_lo) want_a |= 1u << t;
-    const uint32_t want_b = want & ~want_a;
-    uint32_t sa = probe_start(colkey | (uint64_t(b_lo) << 2), cap_mask);
-    uint32_t sb = probe_start(colkey | (uint64_t(b_hi) << 2), cap_mask);
-    bool act_a = want_a != 0, act_b = want_b != 0;
-    uint32_t found = 0;
-    auto scan = [&](const uint64_t (&k4)[kGroupSlots], uint32_t s) -> bool {
-        bool empty = false;
-#pragma unroll
-        for (int i = 0; i < kGroupSlots; ++i) {
-            const uint64_t k = k4[i];
-            if (k == kEmptyKey) {
-                empty = true;
-                continue;
-            }
-            if (uint32_t(k >> 32) != col_hi || uint32_t(k >> 16 & 0xFFFFu) != col_y) continue;
-            const int d = int(k & 0xFFFFu) - zf0;
-#pragma unroll
-            for (int t = 0; t < KZ; ++t)
-                if (d == t) slot_of[t] = int(s) + i;
-            if (d >= 0 && d < KZ) found |= 1u << d;
-        }
-        return empty;
-    };
-    for (uint32_t round = 0; (act_a || act_b) && round < probe_window(cap_mask) / kGroupSlots; ++round) {
-        uint64_t ka[kGroupSlots], kb[kGroupSlots];
-        if (act_a) group_keys(groups, sa, ka);
-        if (act_b) group_keys(groups, sb, kb);
-        if (act_a) {
-            const bool e = scan(ka, sa);
-            act_a = !e && (want_a & ~found);
-            sa = (sa + kGroupSlots) & cap_mask;
-        }
-        if (act_b) {
-            const bool e = scan(kb, sb);
-            act_b = !e && (want_b & ~found);
-            sb = (sb + kGroupSlots) & cap_mask;
-        }
-    }
-#pragma unroll
-    for (int t = 0; t < KZ; ++t)
-        if (!((want >> t) & 1u)) slot_of[t] = -1;
-}
+__device__ __forceinline__ bool query_coord(const Geom &g, const int4 &c, int ix, int iy, int iz, uint64_t &key);
 
 // ----------------------------------------------------------------------------- submanifold front end
-struct SubmGeom {
-    int kx, ky, kz;
-    int px, py, pz;  // (K - 1) / 2
-    int k3;
-};
-
-constexpr int kProbeRows = 128;  // output rows per block (four per lane)
-
-// Submanifold map, one launch: block = one warp per kernel column (ix, iy)
-// (warp w = ix * Ky + iy) over kProbeRows rows; the column's offsets are
-// k = w * Kz + iz.  The block's coordinates are staged in shared memory once.
-// A lane takes its rows one at a time: it searches the table for the
-// neighbours at (x + ix - px, y + iy - py, z + iz - pz), iz = 0..Kz-1, in
-// one pass over at most two z-brick sequences (KZ = 1 or 3; KZ = 0 probes
-// each offset on its own, for any Kz), writes those Kz entries of nbr
-// (coalesced: the warp's 32 rows are consecutive) and ballots its hits into
-// shared memory.  The centre offset is the row itself and is not probed.
-// Then each row's mask is gathered from the ballots, and the row's grouping
-// key, the block's hits per offset and its key-byte histograms are computed
-// and added to the global counters.
-template <int KZ>
-__global__ void __launch_bounds__(1024)
-subm_probe_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const int4 *__restrict__ coords, int64_t n,
-                  SubmGeom g, int32_t *__restrict__ nbr, uint32_t *__restrict__ mask, uint32_t *__restrict__ keys,
-                  int32_t *__restrict__ counters, int32_t *d_status) {
+// Submanifold map: one thread per (offset k below the centre, row j);
+// blockIdx.y is the offset, so a warp probes one offset for 32 consecutive rows
+// (coalesced coordinate loads and nbr stores, a uniform key delta).  A probe
+// reads its home group's 4 keys with two 16-byte loads and walks on to the next
+// group only when all 4 slots hold other keys (bounded by the probe window).
+// A hit at row r also writes the mirrored entry nbr[k3-1-k][r] = j (the
+// relation is symmetric) and ORs both bits into the masks.  The fill before
+// it set the offsets above the centre to -1 and every mask to the centre bit;
+// the threads of offset 0 also write the centre column (every row is its own
+// centre neighbour).  Far fewer instructions per lookup than looping over the
+// offsets inside one thread, and about 30 registers, so every SM runs its full
+// complement of warps.
+__global__ void __launch_bounds__(kQueryThreads)
+kmap_probe_sym_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const int4 *__restrict__ out_coords,
+                      int64_t n_out, Geom g, int32_t *__restrict__ nbr, uint32_t *__restrict__ mask,
+                      int32_t *d_status) {
     pdl_enter();
-    __shared__ int4 s_c[kProbeRows];
-    __shared__ uint32_t s_bits[32][kProbeRows / 32];
-    __shared__ int s_h[512], s_o[32];
-    const Tally ty{s_h, s_o};
-    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nwarp = blockDim.x >> 5;
-    const int64_t row0 = int64_t(blockIdx.x) * kProbeRows;
-    for (int i = tid; i < kProbeRows; i += blockDim.x)
-        s_c[i] = row0 + i < n ? __ldg(coords + row0 + i) : make_int4(-1, 0, 0, 0);
-    for (int i = tid; i < 32 * (kProbeRows / 32); i += blockDim.x) (&s_bits[0][0])[i] = 0u;
-    tally_clear(ty);
-    __syncthreads();
-    const int kz = KZ ? KZ : g.kz;
-    const int dx = w / g.ky - g.px, dy = w % g.ky - g.py;
-    const bool own = dx == 0 && dy == 0;
-    int32_t bad = 0;
-    for (int r = 0; r < kProbeRows / 32; ++r) {
-        const int64_t j = row0 + 32 * r + lane;
-        const bool live = j < n;
-        const int4 c = s_c[32 * r + lane];
-        const int X = c.y + dx, Y = c.z + dy;
-        const bool colok = live && c.x >= 0 && c.x <= 65534 && X >= -32768 && X <= 32767 && Y >= -32768 &&
-                           Y <= 32767 && c.w >= -32768 && c.w <= 32767;
-        const int zf0 = c.w + 32768 - g.pz;  // z field of target iz = 0
-        const uint32_t col_hi = (uint32_t(c.x) << 16) | uint32_t(X + 32768);
-        const uint32_t col_y = uint32_t(Y + 32768);
-        uint32_t want = 0;
-        for (int t = 0; t < kz; ++t)
-            if (colok && zf0 + t >= 0 && zf0 + t <= 65535 && !(own && t == g.pz)) want |= 1u << t;
-        if constexpr (KZ > 0) {
-            int slot_of[KZ];
-            probe_column<KZ>(groups, cap_mask, col_hi, col_y, zf0, want, slot_of);
-            int rr[KZ];
+    const int k = blockIdx.y;
+    const int64_t j = blockIdx.x * int64_t(kQueryThreads) + threadIdx.x;
+    if (j >= n_out) return;
+    const int4 c = __ldg(out_coords + j);
+    uint64_t key = 0;
+    bool ok;
+    if (g.shift && c.y >= g.lo[0] && c.y <= g.hi[0] && c.z >= g.lo[1] && c.z <= g.hi[1] && c.w >= g.lo[2] &&
+        c.w <= g.hi[2] && pack_key(c.x, c.y, c.z, c.w, key)) {
+        key += uint64_t(g.delta[k]);
+        ok = true;
+    } else {
+        ok = query_coord(g, c, g.off[k][0], g.off[k][1], g.off[k][2], key);
+    }
+    int r = -1;
+    if (ok) {
+        uint32_t slot = probe_start(key, cap_mask);
+        for (uint32_t round = 0; round < probe_window(cap_mask) / kGroupSlots; ++round) {
+            const SlotGroup *gp = groups + slot / kGroupSlots;
+            const ulonglong2 a = __ldg(reinterpret_cast<const ulonglong2 *>(gp->key));
+            const ulonglong2 b = __ldg(reinterpret_cast<const ulonglong2 *>(gp->key + 2));
+            const uint64_t k4[kGroupSlots] = {a.x, a.y, b.x, b.y};
+            int found = -1;
+            bool stop = false;
 #pragma unroll
-            for (int t = 0; t < KZ; ++t)
-                rr[t] = slot_of[t] >= 0 ? int(__ldg(&groups[slot_of[t] / kGroupSlots].row[slot_of[t] % kGroupSlots]))
-                                        : -1;
-#pragma unroll
-            for (int t = 0; t < KZ; ++t) {
-                int v = rr[t];
-                if (own && t == g.pz) v = live ? int(j) : -1;
-                if (v >= n) {
-                    bad |= LAT_ERR_BAD_MAP;
-                    v = -1;
+            for (int i = 0; i < kGroupSlots; ++i) {
+                if (stop) continue;
+                if (k4[i] == key) {
+                    found = i;
+                    stop = true;
+                } else if (k4[i] == kEmptyKey) {
+                    stop = true;
                 }
-                const int k = w * KZ + t;
-                if (live) nbr[int64_t(k) * n + j] = v;
-                const unsigned hits = __ballot_sync(0xFFFFFFFFu, v >= 0);
-                if (lane == 0) s_bits[k][r] = hits;
             }
-        } else {
-            for (int t = 0; t < kz; ++t) {
-                int v = -1;
-                if (own && t == g.pz) {
-                    v = live ? int(j) : -1;
-                } else if ((want >> t) & 1u) {
-                    const uint64_t key = (uint64_t(col_hi) << 32) | (uint64_t(col_y) << 16) | uint64_t(zf0 + t);
-                    const int s = probe_one(groups, cap_mask, key);
-                    v = s >= 0 ? int(__ldg(&groups[s / kGroupSlots].row[s % kGroupSlots])) : -1;
-                }
-                if (v >= n) {
-                    bad |= LAT_ERR_BAD_MAP;
-                    v = -1;
-                }
-                const int k = w * kz + t;
-                if (live) nbr[int64_t(k) * n + j] = v;
-                const unsigned hits = __ballot_sync(0xFFFFFFFFu, v >= 0);
-                if (lane == 0) s_bits[k][r] = hits;
+            if (stop) {
+                if (found >= 0) r = int(__ldg(&gp->row[found]));
+                break;
             }
+            slot = (slot + kGroupSlots) & cap_mask;
         }
     }
-    if (bad) flag(d_status, bad);
-    __syncthreads();
-    const bool two = group_key_bits(g.k3) > 8;
-    for (int r = w; r < kProbeRows / 32; r += nwarp) {
-        const int64_t j = row0 + 32 * r + lane;
-        const bool live = j < n;
-        uint32_t m = 0;
-        for (int k = 0; k < g.k3; ++k) m |= ((s_bits[k][r] >> lane) & 1u) << k;
-        const uint32_t key = group_key(m, g.k3);
-        if (live) {
-            mask[j] = m;
-            keys[j] = key;
-        }
-        tally_row(ty, key, m, live, two);
+    if (r >= n_out) {
+        flag(d_status, LAT_ERR_BAD_MAP);
+        r = -1;
     }
-    __syncthreads();
-    tally_flush(ty, g.k3, two, counters);
+    nbr[int64_t(k) * n_out + j] = r;
+    if (k == 0) nbr[int64_t(g.k3 / 2) * n_out + j] = int32_t(j);
+    if (r >= 0) {
+        const int km = g.k3 - 1 - k;
+        nbr[int64_t(km) * n_out + r] = int32_t(j);
+        atomicOr(mask + j, 1u << k);
+        atomicOr(mask + r, 1u << km);
+    }
+}
+
+// A submanifold map with a single offset (1x1x1): every row is its own neighbour.
+__global__ void __launch_bounds__(kQueryThreads) kmap_centre_kernel(int64_t n_out, int32_t *__restrict__ nbr) {
+    pdl_enter();
+    const int64_t j = blockIdx.x * int64_t(kQueryThreads) + threadIdx.x;
+    if (j < n_out) nbr[j] = int32_t(j);
 }
 
 // ----------------------------------------------------------------------------- strided / transposed front end
@@ -359,9 +248,9 @@ __device__ __forceinline__ bool query_coord(const Geom &g, const int4 &c, int ix
 __global__ void __launch_bounds__(kQueryThreads)
 kmap_probe_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const int4 *__restrict__ out_coords,
                   int64_t n_out, int64_t n_in, Geom g, int32_t *__restrict__ nbr, uint32_t *__restrict__ mask,
-                  uint32_t *__restrict__ keys, int32_t *__restrict__ counters, int32_t *d_status) {
+                  uint32_t *__restrict__ keys, int32_t *__restrict__ cnt, int ntile, int32_t *d_status) {
     pdl_enter();
-    __shared__ int s_h[512], s_o[32];
+    __shared__ int s_h[256], s_o[32];
     const Tally ty{s_h, s_o};
     tally_clear(ty);
     __syncthreads();
@@ -457,19 +346,18 @@ kmap_probe_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const
         mask[j] = m;
         keys[j] = key;
     }
-    const bool two = group_key_bits(g.k3) > 8;
-    tally_row(ty, key, m, live, two);
+    tally_row(ty, key, m, live);
     __syncthreads();
-    tally_flush(ty, g.k3, two, counters);
+    tally_flush(ty, g.k3, cnt, ntile, blockIdx.x * int64_t(kQueryThreads));
 }
 
 // Grouping keys and global totals from final masks (the strided map of a
 // ksize == stride convolution, whose masks the parent scatter builds).
 __global__ void __launch_bounds__(kQueryThreads)
 kmap_count_kernel(const uint32_t *__restrict__ mask, int64_t n_out, int k3, uint32_t *__restrict__ keys,
-                  int32_t *__restrict__ counters) {
+                  int32_t *__restrict__ cnt, int ntile) {
     pdl_enter();
-    __shared__ int s_h[512], s_o[32];
+    __shared__ int s_h[256], s_o[32];
     const Tally ty{s_h, s_o};
     tally_clear(ty);
     __syncthreads();
@@ -478,10 +366,9 @@ kmap_count_kernel(const uint32_t *__restrict__ mask, int64_t n_out, int k3, uint
     const uint32_t m = live ? __ldg(mask + j) : 0u;
     const uint32_t key = group_key(m, k3);
     if (live) keys[j] = key;
-    const bool two = group_key_bits(k3) > 8;
-    tally_row(ty, key, m, live, two);
+    tally_row(ty, key, m, live);
     __syncthreads();
-    tally_flush(ty, k3, two, counters);
+    tally_flush(ty, k3, cnt, ntile, blockIdx.x * int64_t(kQueryThreads));
 }
 
 // Kernel size == stride, no padding: fine row i lies in exactly one coarse window,
@@ -492,10 +379,10 @@ kmap_count_kernel(const uint32_t *__restrict__ mask, int64_t n_out, int k3, uint
 __global__ void __launch_bounds__(256)
 parent_maps_kernel(const int4 *__restrict__ fine, const int32_t *__restrict__ parent, int64_t n_fine,
                    int64_t n_coarse, int s0, int s1, int s2, int k3, int32_t *__restrict__ up_nbr,
-                   uint32_t *__restrict__ up_mask, uint32_t *__restrict__ up_keys, int32_t *__restrict__ up_counters,
-                   int32_t *__restrict__ down_nbr, uint32_t *__restrict__ down_mask, int32_t *d_status) {
+                   uint32_t *__restrict__ up_mask, uint32_t *__restrict__ up_keys, int32_t *__restrict__ up_cnt,
+                   int up_ntile, int32_t *__restrict__ down_nbr, uint32_t *__restrict__ down_mask, int32_t *d_status) {
     pdl_enter();
-    __shared__ int s_h[512], s_o[32];
+    __shared__ int s_h[256], s_o[32];
     const Tally ty{s_h, s_o};
     if (up_nbr) tally_clear(ty);
     __syncthreads();
@@ -523,92 +410,106 @@ parent_maps_kernel(const int4 *__restrict__ fine, const int32_t *__restrict__ pa
     if (up_nbr) {  // block-uniform: every lane of the warp takes part
         const uint32_t key = group_key(m, k3);
         if (live) up_keys[i] = key;
-        const bool two = group_key_bits(k3) > 8;
-        tally_row(ty, key, m, live, two);
+        tally_row(ty, key, m, live);
         __syncthreads();
-        tally_flush(ty, k3, two, up_counters);
+        tally_flush(ty, k3, up_cnt, up_ntile, blockIdx.x * int64_t(blockDim.x));
     }
 }
 
-// ----------------------------------------------------------------------------- sweeps
-constexpr int kSwThreads = 512;
-constexpr int kSwWarps = kSwThreads / 32;
-constexpr int kSwRounds = 4;
-constexpr int kSwTile = kSwThreads * kSwRounds;  // rows per tile
-constexpr int kSwChains = 256 + 32;              // look-back chains per tile: 256 digits, then 32 offsets
-constexpr unsigned long long kFlagAgg = 1ull << 32, kFlagPrefix = 2ull << 32;
-constexpr uint64_t kLookbackNs = 1000000000ull;  // a look-back wait gives up after 1 s
-
-__device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long *p) {
-    unsigned long long v;
-    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
+// ----------------------------------------------------------------------------- row scan and scatter passes
+// Block c: exclusive scan, in place, of chain c's per-tile counts
+// cnt[c * ntile + 0 .. ntile) (the first row of each tile), and the chain's
+// total into totals[c].
+__global__ void __launch_bounds__(256)
+row_scan_kernel(int32_t *__restrict__ cnt, int ntile, int32_t *__restrict__ totals) {
+    pdl_enter();
+    __shared__ int s_warp[8];
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    int32_t *row = cnt + int64_t(blockIdx.x) * ntile;
+    int carry = 0;
+    for (int base = 0; base < ntile; base += 256) {
+        const int i = base + t;
+        const int v = i < ntile ? row[i] : 0;
+        int incl = v;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+            if (lane >= d) incl += o;
+        }
+        if (lane == 31) s_warp[w] = incl;
+        __syncthreads();
+        int before = 0, all = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int x = s_warp[q];
+            before += q < w ? x : 0;
+            all += x;
+        }
+        if (i < ntile) row[i] = carry + before + incl - v;
+        carry += all;
+        __syncthreads();
+    }
+    if (t == 0) totals[blockIdx.x] = carry;
 }
-__device__ __forceinline__ void st_relaxed(unsigned long long *p, unsigned long long v) {
-    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
 
-struct Sweep {
+struct Scatter {
     const uint32_t *keys_in;   // key of each input position
     const int32_t *vals_in;    // output row of each input position; nullptr = the position itself
     const uint32_t *masks_in;  // neighbour mask of each input position
     int64_t n;
     int shift;                 // this pass's digit: (key >> shift) & 255
-    int32_t *counters;         // global totals (kCnt*); tile counter of this sweep at kCntTile + which
-    int which;                 // 0 = first sweep, 1 = second
-    unsigned long long *status;  // [ntile][kSwChains] look-back words, zero at launch
-    // pair emission (first sweep)
+    const int32_t *cnt;        // chains x tiles: each tile's first position among its chain (row-scanned)
+    const int32_t *totals;     // per chain: 256 digits, then (EMIT) k3 offsets
+    int ntile;
+    // pair emission (first pass)
     const int32_t *nbr;
     int centre;  // offset whose neighbour of row j is j itself (submanifold), else -1
     int k3;
     int32_t *pair_in, *pair_out;
     int64_t capacity;
     int64_t *pair_off;
-    // outputs: to the second sweep, or perm and the tile masks
+    // outputs: to the second pass (with its per-tile counts), or perm and the tile masks
     uint32_t *keys_out;
     int32_t *vals_out;
     uint32_t *masks_out;
+    int32_t *cnt_next;    // [256][ntile], zero at launch
     int32_t *perm;
     uint32_t *tile_mask;  // zero at launch
     int32_t *d_status;
 };
 
-// One tile of one radix pass.  EMIT: also write the pair lists (first sweep,
-// rows in input order).  LAST: write perm and OR each row's mask into its
-// LAT_TILE_ROWS output tile; otherwise hand (key, row, mask) to the next
-// sweep at the sorted position.  Positions: the digit's start (exclusive scan
-// of the global digit histogram) + the digit's count in earlier tiles
-// (look-back) + the row's rank among this tile's rows of that digit (warp
-// match, per-warp counts; rounds in row order).  Pair positions likewise per
-// offset.
+// One tile of one stable radix pass.  EMIT: also write the pair lists (first
+// pass, rows in input order).  LAST: write perm and OR each row's mask into
+// its LAT_TILE_ROWS output tile; otherwise hand (key, row, mask) to the next
+// pass at the sorted position and count the next digit per output tile.
+// Position of a row: its digit's start (exclusive scan of the digit totals)
+// + the tile's start among that digit (row scan) + the row's rank among the
+// tile's rows of that digit (warp match; per round, one thread per digit turns
+// the per-warp counts into per-warp starts with its loads issued together).
+// Pair positions likewise per offset; the pairs' neighbour rows are loaded
+// kEmitBatch at a time before any of them is stored.
+constexpr int kEmitBatch = 4;
+
 template <bool EMIT, bool LAST>
-__global__ void __launch_bounds__(kSwThreads) sweep_kernel(Sweep a) {
-    pdl_enter();
-    __shared__ int s_tile;
-    __shared__ int s_cnt[2][kSwWarps][256];  // per round (double buffered): per-warp digit counts
-    __shared__ int s_run[256];               // next position of each digit
-    __shared__ int s_hist[256];              // this tile's rows per digit
-    __shared__ int s_ocnt[32];               // this tile's pairs per offset
-    __shared__ int s_pw[2][kSwWarps][32];    // per round: per-warp pairs per offset, then their prefix
-    __shared__ long long s_orun[2][32];      // per round: next pair position of each offset
-    __shared__ int s_wsum[8];
+__global__ void __launch_bounds__(kScThreads) scatter_kernel(Scatter a) {
+    pdl_wait();
+    __shared__ int s_cnt[kScWarps][256];        // this round: per-warp rows of each digit
+    __shared__ int s_pre[kScWarps][256];        // this round: first position of each (warp, digit)
+    __shared__ int s_run[256];                  // next position of each digit
+    __shared__ int s_pw[kScWarps][32];          // this round: per-warp pairs of each offset
+    __shared__ unsigned s_ball[kScWarps][32];   // this round: per warp, the lanes with a pair at each offset
+    __shared__ long long s_pwx[kScWarps][32];   // this round: first pair position of each (warp, offset)
+    __shared__ long long s_orun[32];            // next pair position of each offset
+    __shared__ long long s_cbase;               // first pair of the centre offset (submanifold maps)
+    __shared__ int s_wsum[kScWarps];
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const unsigned lt = (1u << lane) - 1u;
-    if (t == 0) s_tile = atomicAdd(a.counters + kCntTile + a.which, 1);
-    for (int i = t; i < 2 * kSwWarps * 256; i += kSwThreads) (&s_cnt[0][0][0])[i] = 0;
-    if (t < 256) s_hist[t] = 0;
-    if (t < 32) s_ocnt[t] = 0;
-    __syncthreads();
-    const int tile = s_tile;
-    if (int64_t(tile) * kSwTile >= a.n) {  // the tile counter was not cleared: no tile waits for this one
-        if (t == 0) flag(a.d_status, LAT_ERR_BAD_MAP);
-        return;
-    }
-    uint32_t key[kSwRounds], mk[kSwRounds];
-    int32_t val[kSwRounds];
+    const int tile = blockIdx.x;
+    uint32_t key[kScRounds], mk[kScRounds];
+    int32_t val[kScRounds];
 #pragma unroll
-    for (int r = 0; r < kSwRounds; ++r) {
-        const int64_t e = int64_t(tile) * kSwTile + r * kSwThreads + t;
+    for (int r = 0; r < kScRounds; ++r) {
+        const int64_t e = int64_t(tile) * kScTile + r * kScThreads + t;
         key[r] = 0;
         mk[r] = 0;
         val[r] = -1;
@@ -618,56 +519,9 @@ __global__ void __launch_bounds__(kSwThreads) sweep_kernel(Sweep a) {
             if (EMIT || LAST) mk[r] = __ldg(a.masks_in + e);
         }
     }
-    // this tile's counts
-#pragma unroll
-    for (int r = 0; r < kSwRounds; ++r) {
-        const bool live = val[r] >= 0;
-        const uint32_t d = (key[r] >> a.shift) & 255u;
-        const unsigned peers = __match_any_sync(0xFFFFFFFFu, live ? d : 256u + lane);
-        if (live && (peers & lt) == 0) atomicAdd(&s_hist[d], int(__popc(peers)));
-        if (EMIT) {
-            const uint32_t m = live ? mk[r] : 0u;
-            for (uint32_t any = __reduce_or_sync(0xFFFFFFFFu, m); any; any &= any - 1) {
-                const int k = __ffs(any) - 1;
-                const unsigned hits = __ballot_sync(0xFFFFFFFFu, (m >> k) & 1u);
-                if (lane == 0) atomicAdd(&s_ocnt[k], int(__popc(hits)));
-            }
-        }
-    }
-    __syncthreads();
-    // publish this tile's counts, look back for the earlier tiles', publish the prefix
-    const int nchain = EMIT ? 256 + a.k3 : 256;
-    unsigned long long *st = a.status + int64_t(tile) * kSwChains;
-    int own = 0, excl = 0;
-    if (t < nchain) {
-        own = t < 256 ? s_hist[t] : s_ocnt[t - 256];
-        st_relaxed(st + t, (tile == 0 ? kFlagPrefix : kFlagAgg) | uint32_t(own));
-        if (tile > 0) {
-            bool timed_out = false;
-            uint64_t t0 = 0;
-            int64_t pb = tile - 1;
-            for (uint32_t spin = 0;;) {
-                const unsigned long long v = ld_relaxed(a.status + pb * kSwChains + t);
-                if ((v >> 32) == 0) {  // that tile has not published yet: it is running, wait
-                    if (++spin == 64) t0 = ptx_globaltimer();
-                    if (spin > 64 && (spin & 15) == 0 && ptx_globaltimer() - t0 > kLookbackNs) {
-                        timed_out = true;
-                        break;
-                    }
-                    __nanosleep(64);
-                    continue;
-                }
-                excl += int(uint32_t(v));
-                if ((v >> 32) == 2 || pb == 0) break;
-                --pb;
-            }
-            if (timed_out) flag(a.d_status, LAT_ERR_TIMEOUT);
-            st_relaxed(st + t, kFlagPrefix | uint32_t(excl + own));
-        }
-    }
-    // digit starts: exclusive scan of the global digit histogram
-    if (t < 256) {
-        const int v = a.counters[kCntHist + (a.shift ? 256 : 0) + t];
+    for (int i = t; i < kScWarps * 256; i += kScThreads) (&s_cnt[0][0])[i] = 0;
+    {  // digit starts: exclusive scan of the digit totals, plus this tile's start
+        const int v = __ldg(a.totals + t);
         int incl = v;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
@@ -675,86 +529,116 @@ __global__ void __launch_bounds__(kSwThreads) sweep_kernel(Sweep a) {
             if (lane >= d) incl += o;
         }
         if (lane == 31) s_wsum[warp] = incl;
-        s_run[t] = incl - v + excl;  // completed with the earlier warps' sums below
+        s_run[t] = incl - v + __ldg(a.cnt + int64_t(t) * a.ntile + tile);  // + the earlier warps' sums below
     }
-    if (EMIT && warp == 8) {  // offset starts: exclusive scan of the per-offset totals
-        const int64_t v = lane < a.k3 ? a.counters[kCntOff + lane] : 0;
+    if (EMIT && warp == 0) {  // offset starts: exclusive scan of the offset totals, plus this tile's start
+        const int64_t v = lane < a.k3 ? __ldg(a.totals + 256 + lane) : 0;
         int64_t incl = v;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
             const int64_t o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
             if (lane >= d) incl += o;
         }
-        if (lane < a.k3) s_orun[0][lane] = incl - v + excl;
+        if (lane < a.k3) s_orun[lane] = incl - v + __ldg(a.cnt + int64_t(256 + lane) * a.ntile + tile);
+        if (a.centre >= 0 && lane == a.centre) s_cbase = incl - v;
         if (tile == 0) {
             if (lane < a.k3) a.pair_off[lane] = incl - v;
             const int64_t all = __shfl_sync(0xFFFFFFFFu, incl, 31);
             if (lane == 0) a.pair_off[a.k3] = all;
         }
     }
+    pdl_trigger();
     __syncthreads();
-    if (t < 256)
-        for (int q = 0; q < warp; ++q) s_run[t] += s_wsum[q];
-    __syncthreads();
+    for (int q = 0; q < warp; ++q) s_run[t] += s_wsum[q];
     bool over = false, bad = false;
 #pragma unroll
-    for (int r = 0; r < kSwRounds; ++r) {
-        const int p = r & 1;
+    for (int r = 0; r < kScRounds; ++r) {
         const bool live = val[r] >= 0;
         const uint32_t d = (key[r] >> a.shift) & 255u;
         const unsigned peers = __match_any_sync(0xFFFFFFFFu, live ? d : 256u + lane);
-        if (live && (peers & lt) == 0) s_cnt[p][warp][d] = __popc(peers);
-        const uint32_t m = (EMIT && live) ? mk[r] : 0u;
-        uint32_t any = 0;
+        if (live && (peers & lt) == 0) s_cnt[warp][d] = __popc(peers);
+        // the centre pair of every row (j, j) sits at a fixed position; the
+        // other offsets are counted per warp, with the lanes that have them
+        const uint32_t cbit = a.centre >= 0 ? 1u << a.centre : 0u;
+        const uint32_t m = (EMIT && live) ? mk[r] & ~cbit : 0u;
         if (EMIT) {
-            s_pw[p][warp][lane] = 0;
+            s_pw[warp][lane] = 0;
             __syncwarp();
-            any = __reduce_or_sync(0xFFFFFFFFu, m);
-            for (uint32_t b = any; b; b &= b - 1) {
+            for (uint32_t b = __reduce_or_sync(0xFFFFFFFFu, m); b; b &= b - 1) {
                 const int k = __ffs(b) - 1;
                 const unsigned hits = __ballot_sync(0xFFFFFFFFu, (m >> k) & 1u);
-                if (lane == 0) s_pw[p][warp][k] = __popc(hits);
+                if (lane == 0) {
+                    s_pw[warp][k] = __popc(hits);
+                    s_ball[warp][k] = hits;
+                }
             }
+        }
+        __syncthreads();
+        {  // digit t: first position of each warp's rows, counts cleared, start advanced
+            int c[kScWarps];
+#pragma unroll
+            for (int w = 0; w < kScWarps; ++w) c[w] = s_cnt[w][t];
+            int run = s_run[t];
+#pragma unroll
+            for (int w = 0; w < kScWarps; ++w) {
+                s_pre[w][t] = run;
+                run += c[w];
+                s_cnt[w][t] = 0;
+            }
+            s_run[t] = run;
+        }
+        if (EMIT && t < a.k3) {  // offset t: the same for the pairs
+            int c[kScWarps];
+#pragma unroll
+            for (int w = 0; w < kScWarps; ++w) c[w] = s_pw[w][t];
+            long long run = s_orun[t];
+#pragma unroll
+            for (int w = 0; w < kScWarps; ++w) {
+                s_pwx[w][t] = run;
+                run += c[w];
+            }
+            s_orun[t] = run;
         }
         __syncthreads();
         int64_t dst = 0;
         bool put = false;
         if (live) {
-            int pre = s_run[d] + __popc(peers & lt);
-            for (int w = 0; w < warp; ++w) pre += s_cnt[p][w][d];
-            dst = pre;
-            // totals that disagree with the rows (never for maps the front ends built)
+            dst = s_pre[warp][d] + __popc(peers & lt);
+            // counts that disagree with the rows (never for maps the front ends built)
             put = dst >= 0 && dst < a.n;
             if (!put) bad = true;
         }
-        if (EMIT && t < a.k3) {  // per offset: exclusive prefix over the warps, and the next round's start
-            int run = 0;
-            for (int w = 0; w < kSwWarps; ++w) {
-                const int c = s_pw[p][w][t];
-                s_pw[p][w][t] = run;
-                run += c;
-            }
-            s_orun[p ^ 1][t] = s_orun[p][t] + run;
-        }
-        __syncthreads();
-        if (t < 256) {  // digit t: advance its position and clear this round's counts
-            int add = 0;
-#pragma unroll
-            for (int w = 0; w < kSwWarps; ++w) {
-                add += s_cnt[p][w][t];
-                s_cnt[p][w][t] = 0;
-            }
-            s_run[t] += add;
-        }
         if (EMIT) {
-            for (uint32_t b = any; b; b &= b - 1) {
-                const int k = __ffs(b) - 1;
-                const unsigned hits = __ballot_sync(0xFFFFFFFFu, (m >> k) & 1u);
-                if ((m >> k) & 1u) {
-                    const int64_t pos = s_orun[p][k] + s_pw[p][warp][k] + __popc(hits & lt);
-                    if (pos < a.capacity) {
-                        a.pair_in[pos] = k == a.centre ? val[r] : __ldg(a.nbr + int64_t(k) * a.n + val[r]);
-                        a.pair_out[pos] = val[r];
+            if (live && (mk[r] & cbit)) {  // centre pair: every row of a submanifold map has it
+                const int64_t pos = s_cbase + val[r];
+                if (pos < a.capacity) {
+                    a.pair_in[pos] = val[r];
+                    a.pair_out[pos] = val[r];
+                } else {
+                    over = true;
+                }
+            }
+            // this lane's other pairs, kEmitBatch neighbour loads in flight at a time
+            for (uint32_t b = m; b;) {
+                int kk[kEmitBatch], vv[kEmitBatch];
+                int64_t pp[kEmitBatch];
+#pragma unroll
+                for (int q = 0; q < kEmitBatch; ++q) {
+                    kk[q] = -1;
+                    if (b) {
+                        const int k = __ffs(b) - 1;
+                        b &= b - 1;
+                        kk[q] = k;
+                        pp[q] = s_pwx[warp][k] + __popc(s_ball[warp][k] & lt);
+                        vv[q] = __ldg(a.nbr + int64_t(k) * a.n + val[r]);
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < kEmitBatch; ++q) {
+                    if (kk[q] < 0) continue;
+                    if (pp[q] < a.capacity) {
+                        a.pair_in[pp[q]] = vv[q];
+                        a.pair_out[pp[q]] = val[r];
                     } else {
                         over = true;
                     }
@@ -768,10 +652,18 @@ __global__ void __launch_bounds__(kSwThreads) sweep_kernel(Sweep a) {
             const unsigned tp = __match_any_sync(0xFFFFFFFFu, tl);
             const uint32_t m_or = __reduce_or_sync(tp, mk[r]);
             if (put && (tp & lt) == 0) atomicOr(a.tile_mask + dst / LAT_TILE_ROWS, m_or);
-        } else if (put) {
-            a.keys_out[dst] = key[r];
-            a.vals_out[dst] = val[r];
-            a.masks_out[dst] = mk[r];
+        } else {
+            if (put) {
+                a.keys_out[dst] = key[r];
+                a.vals_out[dst] = val[r];
+                a.masks_out[dst] = mk[r];
+            }
+            // the next pass's digit per output tile: one atomic per (warp, digit, tile);
+            // output tile < 2^31 / kScTile <= 2^22, digit < 2^8: the tag fits in 30 bits
+            const uint32_t d2 = (key[r] >> (a.shift + 8)) & 255u;
+            const uint32_t tag = put ? ((d2 << 22) | uint32_t(dst / kScTile)) : (0x80000000u | lane);
+            const unsigned p2 = __match_any_sync(0xFFFFFFFFu, tag);
+            if (put && (p2 & lt) == 0) atomicAdd(a.cnt_next + int64_t(d2) * a.ntile + dst / kScTile, int(__popc(p2)));
         }
     }
     if (over || bad) flag(a.d_status, (over ? LAT_ERR_CAPACITY : 0) | (bad ? LAT_ERR_BAD_MAP : 0));
@@ -780,46 +672,46 @@ __global__ void __launch_bounds__(kSwThreads) sweep_kernel(Sweep a) {
 // ----------------------------------------------------------------------------- workspace and host side
 struct KmapWs {
     uint32_t *keys;       // grouping key of every row (front end)
-    uint32_t *keys_tmp;   // rows after the first sweep: key, row, mask
+    uint32_t *keys_tmp;   // rows after the first pass: key, row, mask
     int32_t *vals_tmp;
     uint32_t *masks_tmp;
-    int32_t *counters;    // kCntWords words, then the look-back words of both sweeps
-    unsigned long long *status[2];
-    int64_t ntile;
-    int64_t zero_words;   // 32-bit words from `counters` on that must be zero before the front end
+    int32_t *cnt1;        // [256 + 32][ntile] counts of the first pass (digits, then offsets)
+    int32_t *cnt2;        // [256][ntile] counts of the second pass
+    int32_t *tot1, *tot2;
+    int ntile;
+    int64_t zero_words;   // cnt1 and cnt2 are one contiguous region that must be zero before the front end
     size_t total;
 };
 
 static KmapWs carve_kmap_ws(void *base, int64_t n_out) {
     KmapWs w{};
-    w.ntile = (n_out + kSwTile - 1) / kSwTile;
+    w.ntile = int((n_out + kScTile - 1) / kScTile);
     Carver cv(base);
     w.keys = cv.take<uint32_t>(size_t(n_out));
     w.keys_tmp = cv.take<uint32_t>(size_t(n_out));
     w.vals_tmp = cv.take<int32_t>(size_t(n_out));
     w.masks_tmp = cv.take<uint32_t>(size_t(n_out));
-    w.counters = cv.take<int32_t>(kCntWords);  // kCntWords * 4 is a multiple of 256: status follows directly
-    static_assert(kCntWords * 4 % 256 == 0, "counters and look-back words are one contiguous zero region");
-    w.status[0] = cv.take<unsigned long long>(size_t(w.ntile) * kSwChains);
-    w.status[1] = cv.take<unsigned long long>(size_t(w.ntile) * kSwChains);
-    w.zero_words = kCntWords + 2 * 2 * w.ntile * kSwChains;
+    w.cnt1 = cv.take<int32_t>(size_t(kChains + 256) * w.ntile);
+    w.cnt2 = w.cnt1 ? w.cnt1 + size_t(kChains) * w.ntile : nullptr;
+    w.zero_words = int64_t(kChains + 256) * w.ntile;
+    w.tot1 = cv.take<int32_t>(kChains);
+    w.tot2 = cv.take<int32_t>(256);
     w.total = align_up(cv.used, 256);
     return w;
 }
 
-// The sweeps of one map whose front end has written nbr, mask, w.keys and the
-// global totals: pair lists, perm and tile masks.
-static lat_status sweep_map(lat_kmap *map, int k3, const KmapWs &w, int centre, int32_t *d_status, cudaStream_t s) {
-    const int64_t n = map->n_out;
-    Sweep a{};
+// The passes of one map whose front end has written nbr, mask, w.keys and the
+// first pass's per-tile counts: pair lists, perm and tile masks.
+static lat_status finish_map(lat_kmap *map, int k3, const KmapWs &w, int centre, int32_t *d_status, cudaStream_t s) {
+    Scatter a{};
     a.keys_in = w.keys;
     a.vals_in = nullptr;
     a.masks_in = map->mask;
-    a.n = n;
+    a.n = map->n_out;
     a.shift = 0;
-    a.counters = w.counters;
-    a.which = 0;
-    a.status = w.status[0];
+    a.cnt = w.cnt1;
+    a.totals = w.tot1;
+    a.ntile = w.ntile;
     a.nbr = map->nbr;
     a.centre = centre;
     a.k3 = k3;
@@ -830,25 +722,30 @@ static lat_status sweep_map(lat_kmap *map, int k3, const KmapWs &w, int centre, 
     a.perm = map->perm;
     a.tile_mask = map->tile_mask;
     a.d_status = d_status;
-    const dim3 grid(unsigned(w.ntile)), block(kSwThreads);
+    const dim3 grid(unsigned(w.ntile)), block(kScThreads);
+    LAT_CUDA_TRY(launch_pdl(row_scan_kernel, dim3(256 + k3), dim3(256), 0, s, w.cnt1, w.ntile, w.tot1));
+    LAT_CUDA_TRY(cudaGetLastError());
     if (group_key_bits(k3) <= 8) {
-        LAT_CUDA_TRY(launch_pdl(sweep_kernel<true, true>, grid, block, 0, s, a));
+        LAT_CUDA_TRY(launch_pdl(scatter_kernel<true, true>, grid, block, 0, s, a));
         LAT_CUDA_TRY(cudaGetLastError());
         return LAT_OK;
     }
     a.keys_out = w.keys_tmp;
     a.vals_out = w.vals_tmp;
     a.masks_out = w.masks_tmp;
-    LAT_CUDA_TRY(launch_pdl(sweep_kernel<true, false>, grid, block, 0, s, a));
+    a.cnt_next = w.cnt2;
+    LAT_CUDA_TRY(launch_pdl(scatter_kernel<true, false>, grid, block, 0, s, a));
     LAT_CUDA_TRY(cudaGetLastError());
-    Sweep b = a;
+    LAT_CUDA_TRY(launch_pdl(row_scan_kernel, dim3(256), dim3(256), 0, s, w.cnt2, w.ntile, w.tot2));
+    LAT_CUDA_TRY(cudaGetLastError());
+    Scatter b = a;
     b.keys_in = w.keys_tmp;
     b.vals_in = w.vals_tmp;
     b.masks_in = w.masks_tmp;
     b.shift = 8;
-    b.which = 1;
-    b.status = w.status[1];
-    LAT_CUDA_TRY(launch_pdl(sweep_kernel<false, true>, grid, block, 0, s, b));
+    b.cnt = w.cnt2;
+    b.totals = w.tot2;
+    LAT_CUDA_TRY(launch_pdl(scatter_kernel<false, true>, grid, block, 0, s, b));
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }
@@ -912,58 +809,62 @@ extern "C" lat_status lat_kmap_query(const void *table, size_t table_bytes, cons
     const uint32_t cap_mask = uint32_t(table_bytes / kSlotBytes - 1);
     const SlotGroup *slots = static_cast<const SlotGroup *>(table);
     const int4 *oc = reinterpret_cast<const int4 *>(out_coords);
-    FillList f;
-    f.add(w.counters, w.zero_words, 0u);
-    f.add(map->tile_mask, ntiles, 0u);
-    LAT_CUDA_TRY(fill_list(f, s));
+    Geom g{};
+    for (int a = 0; a < 3; ++a) {
+        g.ks[a] = geom->ksize[a];
+        g.st[a] = geom->stride[a];
+        g.pd[a] = geom->pad[a];
+    }
+    g.mode = geom->mode;
+    g.k3 = k3;
+    // unit stride: probed coordinate = own + sign * (off - pad), sign -1 for the transposed relation
+    g.shift = g.st[0] == 1 && g.st[1] == 1 && g.st[2] == 1;
+    const int sign = g.mode == LAT_TRANSPOSED ? -1 : 1;
+    for (int a = 0; a < 3; ++a) {
+        const int d0 = sign * (0 - g.pd[a]), d1 = sign * (g.ks[a] - 1 - g.pd[a]);
+        const int dmin = d0 < d1 ? d0 : d1, dmax = d0 < d1 ? d1 : d0;
+        g.lo[a] = -32768 - dmin;
+        g.hi[a] = 32767 - dmax;
+    }
+    for (int ix = 0, k = 0; ix < g.ks[0]; ++ix)
+        for (int iy = 0; iy < g.ks[1]; ++iy)
+            for (int iz = 0; iz < g.ks[2]; ++iz, ++k) {
+                g.off[k][0] = static_cast<signed char>(ix);
+                g.off[k][1] = static_cast<signed char>(iy);
+                g.off[k][2] = static_cast<signed char>(iz);
+                const long long dx = sign * (ix - g.pd[0]), dy = sign * (iy - g.pd[1]), dz = sign * (iz - g.pd[2]);
+                g.delta[k] = dx * (1ll << 32) + dy * (1ll << 16) + dz;
+            }
+    const int nblk = int((n_out + kQueryThreads - 1) / kQueryThreads);
     int centre = -1;
     if (geom->mode == LAT_SUBM) {
-        SubmGeom g{geom->ksize[0], geom->ksize[1], geom->ksize[2], geom->pad[0], geom->pad[1], geom->pad[2], k3};
-        const dim3 grid(unsigned((n_out + kProbeRows - 1) / kProbeRows)), block(32 * g.kx * g.ky);
-        if (g.kz == 3)
-            LAT_CUDA_TRY(launch_pdl(subm_probe_kernel<3>, grid, block, 0, s, slots, cap_mask, oc, n_out, g, map->nbr,
-                                    map->mask, w.keys, w.counters, d_status));
-        else if (g.kz == 1)
-            LAT_CUDA_TRY(launch_pdl(subm_probe_kernel<1>, grid, block, 0, s, slots, cap_mask, oc, n_out, g, map->nbr,
-                                    map->mask, w.keys, w.counters, d_status));
-        else
-            LAT_CUDA_TRY(launch_pdl(subm_probe_kernel<0>, grid, block, 0, s, slots, cap_mask, oc, n_out, g, map->nbr,
-                                    map->mask, w.keys, w.counters, d_status));
         centre = k3 / 2;
+        FillList f;
+        f.add(w.cnt1, w.zero_words, 0u);
+        f.add(map->tile_mask, ntiles, 0u);
+        f.add(map->nbr + int64_t(centre + 1) * n_out, int64_t(k3 - 1 - centre) * n_out, ~0u);  // filled by mirrors
+        f.add(map->mask, n_out, 1u << centre);
+        LAT_CUDA_TRY(fill_list(f, s));
+        if (centre > 0) {
+            LAT_CUDA_TRY(launch_pdl(kmap_probe_sym_kernel, dim3(unsigned(nblk), unsigned(centre)), dim3(kQueryThreads),
+                                    0, s, slots, cap_mask, oc, n_out, g, map->nbr, map->mask, d_status));
+        } else {  // 1x1x1: the centre column alone
+            LAT_CUDA_TRY(launch_pdl(kmap_centre_kernel, dim3(unsigned(nblk)), dim3(kQueryThreads), 0, s, n_out,
+                                    map->nbr));
+        }
+        LAT_CUDA_TRY(cudaGetLastError());
+        LAT_CUDA_TRY(launch_pdl(kmap_count_kernel, dim3(nblk), dim3(kQueryThreads), 0, s, map->mask, n_out, k3, w.keys,
+                                w.cnt1, w.ntile));
     } else {
-        Geom g{};
-        for (int a = 0; a < 3; ++a) {
-            g.ks[a] = geom->ksize[a];
-            g.st[a] = geom->stride[a];
-            g.pd[a] = geom->pad[a];
-        }
-        g.mode = geom->mode;
-        g.k3 = k3;
-        // unit stride: probed coordinate = own + sign * (off - pad), sign -1 for the transposed relation
-        g.shift = g.st[0] == 1 && g.st[1] == 1 && g.st[2] == 1;
-        const int sign = g.mode == LAT_TRANSPOSED ? -1 : 1;
-        for (int a = 0; a < 3; ++a) {
-            const int d0 = sign * (0 - g.pd[a]), d1 = sign * (g.ks[a] - 1 - g.pd[a]);
-            const int dmin = d0 < d1 ? d0 : d1, dmax = d0 < d1 ? d1 : d0;
-            g.lo[a] = -32768 - dmin;
-            g.hi[a] = 32767 - dmax;
-        }
-        for (int ix = 0, k = 0; ix < g.ks[0]; ++ix)
-            for (int iy = 0; iy < g.ks[1]; ++iy)
-                for (int iz = 0; iz < g.ks[2]; ++iz, ++k) {
-                    g.off[k][0] = static_cast<signed char>(ix);
-                    g.off[k][1] = static_cast<signed char>(iy);
-                    g.off[k][2] = static_cast<signed char>(iz);
-                    const long long dx = sign * (ix - g.pd[0]), dy = sign * (iy - g.pd[1]),
-                                    dz = sign * (iz - g.pd[2]);
-                    g.delta[k] = dx * (1ll << 32) + dy * (1ll << 16) + dz;
-                }
-        const int nblk = int((n_out + kQueryThreads - 1) / kQueryThreads);
+        FillList f;
+        f.add(w.cnt1, w.zero_words, 0u);
+        f.add(map->tile_mask, ntiles, 0u);
+        LAT_CUDA_TRY(fill_list(f, s));
         LAT_CUDA_TRY(launch_pdl(kmap_probe_kernel, dim3(nblk), dim3(kQueryThreads), 0, s, slots, cap_mask, oc, n_out,
-                                n_in, g, map->nbr, map->mask, w.keys, w.counters, d_status));
+                                n_in, g, map->nbr, map->mask, w.keys, w.cnt1, w.ntile, d_status));
     }
     LAT_CUDA_TRY(cudaGetLastError());
-    return sweep_map(map, k3, w, centre, d_status, s);
+    return finish_map(map, k3, w, centre, d_status, s);
 }
 
 extern "C" size_t lat_kmap_from_parent_ws_bytes(int64_t n_fine, int64_t n_coarse, int32_t k3) {
@@ -999,16 +900,16 @@ extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int
     const KmapWs w_up = carve_kmap_ws(static_cast<char *>(ws) + w_down.total, n_fine);
     // every initialisation both maps need, in one launch: the strided map's
     // table (-1) and masks (0, both filled by the parent scatter), and each
-    // map's counters, look-back words and tile masks
+    // map's per-tile counts and tile masks
     FillList f;
     if (down && n_coarse > 0) {
         f.add(down->nbr, int64_t(k3) * n_coarse, ~0u);
         f.add(down->mask, n_coarse, 0u);
-        f.add(w_down.counters, w_down.zero_words, 0u);
+        f.add(w_down.cnt1, w_down.zero_words, 0u);
         f.add(down->tile_mask, (n_coarse + LAT_TILE_ROWS - 1) / LAT_TILE_ROWS, 0u);
     }
     if (up && n_fine > 0) {
-        f.add(w_up.counters, w_up.zero_words, 0u);
+        f.add(w_up.cnt1, w_up.zero_words, 0u);
         f.add(up->tile_mask, (n_fine + LAT_TILE_ROWS - 1) / LAT_TILE_ROWS, 0u);
     }
     LAT_CUDA_TRY(fill_list(f, s));
@@ -1016,7 +917,7 @@ extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int
         LAT_CUDA_TRY(launch_pdl(parent_maps_kernel, dim3(unsigned((n_fine + 255) / 256)), dim3(256), 0, s,
                                 reinterpret_cast<const int4 *>(fine_coords), parent, n_fine, n_coarse, geom->stride[0],
                                 geom->stride[1], geom->stride[2], k3, up ? up->nbr : nullptr, up ? up->mask : nullptr,
-                                up ? w_up.keys : nullptr, w_up.counters, down ? down->nbr : nullptr,
+                                up ? w_up.keys : nullptr, w_up.cnt1, w_up.ntile, down ? down->nbr : nullptr,
                                 down ? down->mask : nullptr, d_status));
         LAT_CUDA_TRY(cudaGetLastError());
     }
@@ -1039,10 +940,10 @@ extern "C" lat_status lat_kmap_from_parent(const int32_t *fine_coords, const int
         if (map == down) {
             const int nblk = int((map->n_out + kQueryThreads - 1) / kQueryThreads);
             LAT_CUDA_TRY(launch_pdl(kmap_count_kernel, dim3(nblk), dim3(kQueryThreads), 0, ms, map->mask, map->n_out,
-                                    k3, w.keys, w.counters));
+                                    k3, w.keys, w.cnt1, w.ntile));
             LAT_CUDA_TRY(cudaGetLastError());
         }
-        const lat_status st = sweep_map(map, k3, w, -1, d_status, ms);
+        const lat_status st = finish_map(map, k3, w, -1, d_status, ms);
         if (st != LAT_OK) return st;
     }
     if (side) LAT_CUDA_TRY(side_join(*side, main_s));
