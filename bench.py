@@ -891,11 +891,12 @@ def measure_e2e(host: dict, dev: torch.device, steps: int) -> dict:
 # --------------------------------------------------------------------------- main GPU arm
 # The kernel the roofline object reports: the path kernel with the largest
 # share of the headline step's ncu launch list.
-DOMINANT = "wgrad"
-DOMINANT_KERNEL = "wgrad_tc_kernel<bf16, 128, 128> + its ordered partial reduction"
-# DRAM bytes per launch of that phase from an ncu capture of the current
-# kernels (None: no capture matches them).
-PHASE_TRAFFIC = {}
+DOMINANT = "fwd"
+DOMINANT_KERNEL = "conv_tc_kernel<bf16, 128, 128>, forward: gathered x times W[k] on tcgen05"
+# DRAM bytes (read + write) per launch of that phase's kernel from an ncu
+# capture of the current kernel on the same workload (None: no capture
+# matches the kernel as it is).
+PHASE_TRAFFIC = {"fwd": 168_263_680 + 83_786_752}
 
 
 def main():

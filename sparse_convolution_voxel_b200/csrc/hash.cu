@@ -30,9 +30,9 @@ __global__ void __launch_bounds__(256) hash_insert_kernel(const int4 *__restrict
         bool placed = false;
         const uint32_t window = probe_window(cap_mask);
         for (uint32_t probe = 0; probe < window; ++probe) {
+            // the CAS returns the slot's key: empty (now ours), ours (a duplicate) or another key
             unsigned long long *kp = &groups[s / kGroupSlots].key[s % kGroupSlots];
-            unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(kp);
-            if (cur == kEmptyKey) cur = atomicCAS(kp, (unsigned long long)kEmptyKey, (unsigned long long)key);
+            const unsigned long long cur = atomicCAS(kp, (unsigned long long)kEmptyKey, (unsigned long long)key);
             if (cur == kEmptyKey || cur == key) {
                 atomicMin(&groups[s / kGroupSlots].row[s % kGroupSlots], unsigned(i));
                 if (cur == key) bad |= LAT_ERR_DUPLICATE;

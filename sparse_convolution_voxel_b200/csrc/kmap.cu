@@ -419,15 +419,18 @@ parent_maps_kernel(const int4 *__restrict__ fine, const int32_t *__restrict__ pa
 // ----------------------------------------------------------------------------- row scan and scatter passes
 // Block c: exclusive scan, in place, of chain c's per-tile counts
 // cnt[c * ntile + 0 .. ntile) (the first row of each tile), and the chain's
-// total into totals[c].
-__global__ void __launch_bounds__(256)
+// total into totals[c].  1024 threads: one pass covers 1024 tiles (512k rows).
+constexpr int kRowScanThreads = 1024;
+__global__ void __launch_bounds__(kRowScanThreads)
 row_scan_kernel(int32_t *__restrict__ cnt, int ntile, int32_t *__restrict__ totals) {
     pdl_enter();
-    __shared__ int s_warp[8];
+    constexpr int kWarps = kRowScanThreads / 32;
+    __shared__ int s_warp[kWarps];  // per warp: its sum, then the sum of the warps before it
+    __shared__ int s_total;
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
     int32_t *row = cnt + int64_t(blockIdx.x) * ntile;
     int carry = 0;
-    for (int base = 0; base < ntile; base += 256) {
+    for (int base = 0; base < ntile; base += kRowScanThreads) {
         const int i = base + t;
         const int v = i < ntile ? row[i] : 0;
         int incl = v;
@@ -438,15 +441,22 @@ row_scan_kernel(int32_t *__restrict__ cnt, int ntile, int32_t *__restrict__ tota
         }
         if (lane == 31) s_warp[w] = incl;
         __syncthreads();
-        int before = 0, all = 0;
+        if (w == 0) {
+            const int x = s_warp[lane];
+            int wi = x;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const int x = s_warp[q];
-            before += q < w ? x : 0;
-            all += x;
+            for (int d = 1; d < 32; d <<= 1) {
+                const int o = __shfl_up_sync(0xFFFFFFFFu, wi, d);
+                if (lane >= d) wi += o;
+            }
+            s_warp[lane] = wi - x;
         }
+        __syncthreads();
+        const int before = s_warp[w];
         if (i < ntile) row[i] = carry + before + incl - v;
-        carry += all;
+        if (t == kRowScanThreads - 1) s_total = before + incl;
+        __syncthreads();
+        carry += s_total;
         __syncthreads();
     }
     if (t == 0) totals[blockIdx.x] = carry;
@@ -723,7 +733,7 @@ static lat_status finish_map(lat_kmap *map, int k3, const KmapWs &w, int centre,
     a.tile_mask = map->tile_mask;
     a.d_status = d_status;
     const dim3 grid(unsigned(w.ntile)), block(kScThreads);
-    LAT_CUDA_TRY(launch_pdl(row_scan_kernel, dim3(256 + k3), dim3(256), 0, s, w.cnt1, w.ntile, w.tot1));
+    LAT_CUDA_TRY(launch_pdl(row_scan_kernel, dim3(256 + k3), dim3(kRowScanThreads), 0, s, w.cnt1, w.ntile, w.tot1));
     LAT_CUDA_TRY(cudaGetLastError());
     if (group_key_bits(k3) <= 8) {
         LAT_CUDA_TRY(launch_pdl(scatter_kernel<true, true>, grid, block, 0, s, a));
@@ -736,7 +746,7 @@ static lat_status finish_map(lat_kmap *map, int k3, const KmapWs &w, int centre,
     a.cnt_next = w.cnt2;
     LAT_CUDA_TRY(launch_pdl(scatter_kernel<true, false>, grid, block, 0, s, a));
     LAT_CUDA_TRY(cudaGetLastError());
-    LAT_CUDA_TRY(launch_pdl(row_scan_kernel, dim3(256), dim3(256), 0, s, w.cnt2, w.ntile, w.tot2));
+    LAT_CUDA_TRY(launch_pdl(row_scan_kernel, dim3(256), dim3(kRowScanThreads), 0, s, w.cnt2, w.ntile, w.tot2));
     LAT_CUDA_TRY(cudaGetLastError());
     Scatter b = a;
     b.keys_in = w.keys_tmp;
