@@ -970,12 +970,14 @@ def main():
 
     if rank == 0:
         fp32 = {"skipped": "--lean"}
+        rowcopy = {"skipped": "--lean"}
         if not args.lean:
             try:
                 from sparse_convolution_voxel_b200 import measure
                 fp32 = measure.ffma_peak(dev)
+                rowcopy = measure.gather_peak(dev, n=layer.n, row_bytes=layer.cin * layer.dt.itemsize)
             except Exception as exc:  # the probe library is optional for the headline
-                fp32 = {"error": str(exc)}
+                fp32 = rowcopy = {"error": str(exc)}
         fp32_tflops = fp32.get("tflops")
         rl = roofline_of(layer, pms, peaks, fp32_tflops)
         pb = layer.phase_bytes()
@@ -997,11 +999,12 @@ def main():
                          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                          "traffic": PHASE_TRAFFIC.get(DOMINANT), "alg_bytes": pb[DOMINANT], "ms": dominant_ms,
                          "peak_source": f"{peaks['source']} hbm_gbs (burst copy; the kernel is timed inside the step)",
-                         "timing": "CUDA events around this phase on its stream in every timed step"},
+                         "timing": "CUDA events around this phase on its stream in every timed step",
+                         "frac_of_random_row_copy": (achieved / rowcopy["gbs"]) if "gbs" in rowcopy else None},
             "gpu_launches": None if launches_per_step is None else launches_per_step * args.steps,
             "launches_per_step": launches_per_step,
             "clocks": clocks,
-            "peaks": {**peaks, "fp32_ffma": fp32},
+            "peaks": {**peaks, "fp32_ffma": fp32, "random_row_copy": rowcopy},
         }
         del layer
         torch.cuda.empty_cache()

@@ -22,10 +22,12 @@ struct MapView {
     int flip;
     int centre;  // submanifold maps: the centre offset, whose neighbour of row j is j itself; else -1
 
-    __device__ __forceinline__ uint32_t tile_mask_at(int64_t t) const {
-        const uint32_t m = tile_mask[t];
+    // a stored tile mask as this pass sees it (bits past the offset count dropped)
+    __device__ __forceinline__ uint32_t flip_mask(uint32_t m) const {
+        m &= k3 >= 32 ? 0xFFFFFFFFu : ((1u << k3) - 1u);
         return flip ? (__brev(m) >> (32 - k3)) : m;
     }
+    __device__ __forceinline__ uint32_t tile_mask_at(int64_t t) const { return flip_mask(tile_mask[t]); }
     __device__ __forceinline__ const int32_t *neighbour_ptr(int k, int64_t j) const {
         const int kk = flip ? (k3 - 1 - k) : k;
         return nbr + int64_t(kk) * n_out + j;

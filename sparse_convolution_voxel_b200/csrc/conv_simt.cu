@@ -436,10 +436,15 @@ wgrad_slices_kernel(const T *__restrict__ x, int cin, const T *__restrict__ dy, 
     if (bad) flag(d_status, bad);
 }
 
-// dW[k] = the partials of offset k's segments, added in share order (0 for an
-// offset without pairs).  s_max: the share count the main kernel was given.
-__global__ void wgrad_share_reduce_kernel(const float *__restrict__ partial, const int64_t *__restrict__ pair_off,
-                                          int64_t capacity, int k3, int nelem, int s_max, float *__restrict__ dw) {
+// dW[k] = the partials of offset k's segments (0 for an offset without
+// pairs).  s_max: the share count the main kernel was given.  R consecutive
+// lanes (a power of two <= 32) take one element: lane l adds shares v0+l,
+// v0+l+R, ... in order, then an xor butterfly over the R lanes adds the lane
+// sums in a fixed tree.  R depends only on the shapes (wgrad_reduce_lanes), so
+// the order, and the result, is the same on every call.
+__global__ void __launch_bounds__(256)
+wgrad_share_reduce_kernel(const float *__restrict__ partial, const int64_t *__restrict__ pair_off, int64_t capacity,
+                          int k3, int nelem, int s_max, int lanes, float *__restrict__ dw) {
     pdl_enter();
     __shared__ int s_v[2];
     const int k = blockIdx.y;
@@ -451,11 +456,23 @@ __global__ void wgrad_share_reduce_kernel(const float *__restrict__ partial, con
         s_v[1] = lo < hi ? share_of(P, hi - 1, S) : -1;
     }
     __syncthreads();
-    const int el = blockIdx.x * blockDim.x + threadIdx.x;
-    if (k >= k3 || el >= nelem) return;
-    float s = 0.f;
-    for (int v = s_v[0]; v <= s_v[1]; ++v) s += partial[int64_t(v + k) * nelem + el];
-    dw[int64_t(k) * nelem + el] = s;
+    const int l = threadIdx.x & (lanes - 1);
+    const int el = (blockIdx.x * blockDim.x + threadIdx.x) / lanes;
+    float acc = 0.f;
+    if (el < nelem) {
+#pragma unroll 4
+        for (int v = s_v[0] + l; v <= s_v[1]; v += lanes) acc += partial[int64_t(v + k) * nelem + el];
+    }
+    for (int m = 1; m < lanes; m <<= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, m);
+    if (l == 0 && el < nelem) dw[int64_t(k) * nelem + el] = acc;
+}
+
+// Lanes per element of the reduce: about four partials per lane for an
+// offset that meets the average number of shares.
+static int wgrad_reduce_lanes(int s_max, int k3) {
+    int r = 1;
+    while (r < 32 && 8 * r <= s_max / k3) r <<= 1;
+    return r;
 }
 
 // ----------------------------------------------------------------------------- host side
@@ -533,9 +550,10 @@ lat_status launch_wgrad_simt(const void *x, int cin, const void *dy, int cout, c
                                 partial, d_status));
     }
     LAT_CUDA_TRY(cudaGetLastError());
-    const dim3 rg((nelem + 255) / 256, map->k3);
+    const int lanes = wgrad_reduce_lanes(S, map->k3);
+    const dim3 rg(unsigned((int64_t(nelem) * lanes + 255) / 256), map->k3);
     LAT_CUDA_TRY(launch_pdl(wgrad_share_reduce_kernel, rg, dim3(256), 0, s, partial, map->pair_off, map->pair_capacity,
-                            map->k3, nelem, S, dw));
+                            map->k3, nelem, S, lanes, dw));
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }

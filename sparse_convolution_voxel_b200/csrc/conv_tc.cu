@@ -471,7 +471,10 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const T *__restrict__ x
                     break;
                 }
 #pragma unroll
-                for (int e = 0; e < 4; ++e) ring[r].rows[e * 32 + lane] = rs[sl][e];
+                for (int e = 0; e < 4; ++e) {
+                    if (rs[sl][e] >= mv.n_out) rs[sl][e] = -1;  // only a malformed perm has such rows
+                    ring[r].rows[e * 32 + lane] = rs[sl][e];
+                }
                 if (lane == 0) {
                     ring[r].tile = int32_t(ts[sl]);
                     ring[r].mask = ms[sl];

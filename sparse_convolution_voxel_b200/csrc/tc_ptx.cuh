@@ -62,6 +62,8 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
 }
 // Wait for the phase of the given parity to complete; false after `limit_ns`.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+    // a zero limit: one non-blocking test (try_wait may itself block for a while)
+    if (limit_ns == 0) return mbar_test_wait(bar, parity);
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = globaltimer();

@@ -17,7 +17,7 @@
 // (cp.async.mbarrier.arrive.noinc), and one thread issues 4 tcgen05.mma
 // (K = 16 pairs each) into a TMEM accumulator.  Four epilogue warps write the
 // segment's fp32 partial; a second kernel sums the partials of each offset in a
-// fixed order (32 interleaved lanes over the shares, then the lanes in order).
+// fixed order (8 interleaved lanes over the shares, then a fixed xor tree).
 // No atomics, so dW is deterministic and does not depend on the SM count.
 #include "common.cuh"
 #include "conv_common.cuh"
@@ -343,19 +343,22 @@ wgrad_tc_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int64_t
 }
 
 // dW[k] = sum of offset k's partials, one per share v0..v1 that meets offset k
-// (slot share + k; ranges from the main kernel).  Block (x, k): 32 lanes x 8 groups of 4 elements; lane l sums
-// shares v0+l, v0+l+32, ... in order, then lane 0 adds the 32 lane sums in
-// order -- a fixed order whatever the timing.  Offsets without pairs get 0.
-constexpr int kRedLanes = 32;
-__global__ void __launch_bounds__(256)
+// (slot share + k; ranges from the main kernel).  Eight consecutive lanes
+// share a float4 column of dW[k]: lane l sums shares v0+l, v0+l+8, ... in
+// order, then an xor butterfly over the eight lanes adds the lane sums in a
+// fixed tree -- the same order whatever the timing.  Offsets without pairs
+// get 0.
+constexpr int kRedLanes = 8;
+constexpr int kRedThreads = 256;
+constexpr int kRedCols = kRedThreads / kRedLanes;  // float4 columns of dW[k] per block
+__global__ void __launch_bounds__(kRedThreads)
 wgrad_tc_reduce_kernel(const float *__restrict__ partial, const int32_t *__restrict__ ranges, int nelem,
                        float *__restrict__ dw) {
     pdl_enter();
-    __shared__ float4 s_part[kRedLanes][8];
     const int k = blockIdx.y;
     const int v0 = __ldg(ranges + 2 * k), v1 = __ldg(ranges + 2 * k + 1);
-    const int g = threadIdx.x & 7, l = threadIdx.x >> 3;
-    const int el = (blockIdx.x * 8 + g) * 4;
+    const int l = threadIdx.x & (kRedLanes - 1);
+    const int el = (blockIdx.x * kRedCols + threadIdx.x / kRedLanes) * 4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (el < nelem) {
 #pragma unroll 4
@@ -367,19 +370,14 @@ wgrad_tc_reduce_kernel(const float *__restrict__ partial, const int32_t *__restr
             acc.w += x.w;
         }
     }
-    s_part[l][g] = acc;
-    __syncthreads();
-    if (l == 0 && el < nelem) {
-        float4 t = s_part[0][g];
-        for (int q = 1; q < kRedLanes; ++q) {
-            const float4 x = s_part[q][g];
-            t.x += x.x;
-            t.y += x.y;
-            t.z += x.z;
-            t.w += x.w;
-        }
-        *reinterpret_cast<float4 *>(dw + int64_t(k) * nelem + el) = t;
+#pragma unroll
+    for (int m = 1; m < kRedLanes; m <<= 1) {
+        acc.x += __shfl_xor_sync(0xFFFFFFFFu, acc.x, m);
+        acc.y += __shfl_xor_sync(0xFFFFFFFFu, acc.y, m);
+        acc.z += __shfl_xor_sync(0xFFFFFFFFu, acc.z, m);
+        acc.w += __shfl_xor_sync(0xFFFFFFFFu, acc.w, m);
     }
+    if (l == 0 && el < nelem) *reinterpret_cast<float4 *>(dw + int64_t(k) * nelem + el) = acc;
 }
 
 template <typename T, int M, int N>
@@ -398,8 +396,8 @@ static lat_status launch(const void *x, const void *dy, const lat_kmap *map, flo
                             map->k3, map->n_in, map->n_out, partial, ranges, wait_limit_ns(), d_status));
     LAT_CUDA_TRY(cudaGetLastError());
     const int nelem = M * N;
-    dim3 rg((nelem + 31) / 32, map->k3);
-    LAT_CUDA_TRY(launch_pdl(wgrad_tc_reduce_kernel, dim3(rg), dim3(256), 0, s, partial, ranges, nelem, dw));
+    dim3 rg((nelem / 4 + kRedCols - 1) / kRedCols, map->k3);
+    LAT_CUDA_TRY(launch_pdl(wgrad_tc_reduce_kernel, dim3(rg), dim3(kRedThreads), 0, s, partial, ranges, nelem, dw));
     LAT_CUDA_TRY(cudaGetLastError());
     return LAT_OK;
 }

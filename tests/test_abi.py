@@ -37,6 +37,26 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, name), name
 
 
+def test_measure_library_exports_every_declared_symbol(lib):
+    """libmeasure.so (include/lattice_measure.h): the probes bench.py uses for
+    its rooflines; bad arguments return 1 before anything is launched."""
+    from sparse_convolution_voxel_b200 import measure
+    text = open(os.path.join(ROOT, "include", "lattice_measure.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = sorted(set(re.findall(r"\b(lat_[a-z0-9_]+)\s*\(", text)))
+    assert names == ["lat_measure_ffma", "lat_measure_ffma_flops", "lat_measure_gather"]
+    m = measure.load()
+    for name in names:
+        assert hasattr(m, name), name
+    P = ctypes.c_void_p
+    assert m.lat_measure_gather(None, P(16), None, 10, 256, P(16), 8, None) == 1      # no source
+    assert m.lat_measure_gather(P(16), P(16), None, 10, 24, P(16), 8, None) == 1      # row not 16-byte multiple
+    assert m.lat_measure_gather(P(8), P(16), None, 10, 256, P(16), 8, None) == 1      # misaligned source
+    assert m.lat_measure_gather(P(16), P(16), None, 0, 256, P(16), 8, None) == 0      # nothing to copy
+    assert m.lat_measure_ffma(None, 8, 256, 1, 1.0, 0.0, None) == 1
+    assert m.lat_measure_ffma_flops(2, 64, 3) == 2.0 * 64 * 3 * 2 * 64
+
+
 def test_size_queries(lib):
     assert scv.lat_hash_bytes(1000, 2.0) == 16 * 2048
     assert scv.lat_hash_bytes(10, 2.0) == 16 * 64
