@@ -208,6 +208,160 @@ kmap_probe_sym_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, c
     }
 }
 
+// Column form of the submanifold front end.  The offsets below the centre
+// that share (dx, dy) form a run of consecutive z offsets -- a "column" -- and
+// the hash places the 4 cells of a z-brick (z = 4m..4m+3 of one (b, x, y))
+// in one home group, so a column of up to kColMaxCells cells touches at most
+// two bricks: one thread per (row, column) looks up those one or two bricks
+// (a group's 4 keys, two 16-byte loads each) instead of probing every cell,
+// and loads a row only for the cells present.  Outputs, mirror writes and
+// mask bits are exactly those of kmap_probe_sym_kernel.
+constexpr int kColMax = 16;
+constexpr int kColMaxCells = 5;
+struct Col {
+    long long delta;  // key delta of the column's first cell
+    int kbase;        // offset index of that cell; the column's cells are kbase, kbase + 1, ...
+    int n;            // cells, 1..kColMaxCells
+};
+struct Cols {
+    Col c[kColMax];
+    int count;
+};
+
+// Scans the 4 keys of group gi for brick key B (halves bh, bl; bl's low two
+// bits clear): for each key B + d found, sets bit d of occ and puts tag | slot
+// (3 bits) at bits 3d of sel.  Returns whether the group has an empty slot.
+__device__ __forceinline__ bool brick_scan(const SlotGroup *groups, uint32_t gi, uint32_t bh, uint32_t bl,
+                                           uint32_t tag, uint32_t &occ, uint32_t &sel) {
+    const uint4 *gp = reinterpret_cast<const uint4 *>(groups + gi);
+    const uint4 a = __ldg(gp), b = __ldg(gp + 1);  // keys 0, 1 and 2, 3 as (lo, hi) word pairs
+    const uint32_t lo[kGroupSlots] = {a.x, a.z, b.x, b.z};
+    const uint32_t hi[kGroupSlots] = {a.y, a.w, b.y, b.w};
+    bool empty = false;
+#pragma unroll
+    for (int i = 0; i < kGroupSlots; ++i) {
+        const uint32_t d = lo[i] - bl;  // < 4 only for a key of the brick (the high halves must match too)
+        if (hi[i] == bh && d < 4u) {
+            occ |= 1u << d;
+            sel |= (tag | uint32_t(i)) << (3u * d);
+        }
+        empty |= hi[i] == 0xFFFFFFFFu;  // no packed key has an all-ones high half
+    }
+    return empty;
+}
+
+// The present z positions of brick key B (low two bits clear): bit d of occ
+// set if key B + d is in the table; bits 3d of sel give its slot (2 bits) and
+// whether it sits in the home group grp (0) or the next group (4).  Linear
+// probing fills a group's slots in order, so a group with an empty slot, or
+// the 4 cells of the brick found, ends the scan; returns false if the next
+// group is full too and the brick incomplete (the caller then probes cell by
+// cell).
+__device__ __forceinline__ bool brick_lookup(const SlotGroup *groups, uint32_t cap_mask, uint64_t B, uint32_t &occ,
+                                             uint32_t &sel, uint32_t &grp) {
+    grp = probe_start(B, cap_mask) / kGroupSlots;
+    const uint32_t bh = uint32_t(B >> 32), bl = uint32_t(B);
+    occ = 0;
+    sel = 0;
+    if (brick_scan(groups, grp, bh, bl, 0u, occ, sel) || occ == 0xFu) return true;
+    return brick_scan(groups, (grp + 1) & (cap_mask / kGroupSlots), bh, bl, 4u, occ, sel) || occ == 0xFu;
+}
+
+// Row of key `key` (linear probing from its home group), -1 if absent.
+__device__ __forceinline__ int probe_row(const SlotGroup *groups, uint32_t cap_mask, uint64_t key) {
+    const int slot = probe_one(groups, cap_mask, key);
+    return slot < 0 ? -1 : int(__ldg(&groups[slot / kGroupSlots].row[slot % kGroupSlots]));
+}
+
+// One thread per (row j, column blockIdx.y).  Rows whose offsets could leave
+// the key fields, and columns whose brick lookup ends in a full group, take
+// the cells one at a time.  Threads of column 0 also write the centre column.
+__global__ void __launch_bounds__(kQueryThreads)
+kmap_probe_col_kernel(const SlotGroup *__restrict__ groups, uint32_t cap_mask, const int4 *__restrict__ out_coords,
+                      int64_t n_out, Geom g, Cols cols, int32_t *__restrict__ nbr, uint32_t *__restrict__ mask,
+                      int32_t *d_status) {
+    pdl_enter();
+    const Col col = cols.c[blockIdx.y];
+    const int64_t j = blockIdx.x * int64_t(kQueryThreads) + threadIdx.x;
+    if (j >= n_out) return;
+    const int4 c = __ldg(out_coords + j);
+    if (blockIdx.y == 0) nbr[int64_t(g.k3 / 2) * n_out + j] = int32_t(j);
+    int rr[kColMaxCells];
+    uint64_t key = 0;
+    bool fast = g.shift && c.y >= g.lo[0] && c.y <= g.hi[0] && c.z >= g.lo[1] && c.z <= g.hi[1] &&
+                c.w >= g.lo[2] && c.w <= g.hi[2] && pack_key(c.x, c.y, c.z, c.w, key);
+    if (fast) {
+        const uint64_t kc = key + uint64_t(col.delta);  // the column's first cell
+        const uint64_t b1 = kc & ~uint64_t(3);
+        const uint32_t p0 = uint32_t(kc) & 3u;          // its z position within brick b1
+        uint32_t occ, sel, grp, occ2 = 0, sel2 = 0, grp2 = 0;
+        fast = brick_lookup(groups, cap_mask, b1, occ, sel, grp);
+        if (p0 + uint32_t(col.n) > 4u) fast &= brick_lookup(groups, cap_mask, b1 + 4, occ2, sel2, grp2);
+        occ |= occ2 << 4;
+        const uint32_t gmask = cap_mask / kGroupSlots;
+#pragma unroll
+        for (int t = 0; t < kColMaxCells; ++t) {
+            const uint32_t pos = p0 + uint32_t(t);
+            rr[t] = -1;
+            if (t < col.n && fast && ((occ >> pos) & 1u)) {
+                const uint32_t code = pos < 4u ? (sel >> (3u * pos)) : (sel2 >> (3u * (pos - 4u)));
+                const uint32_t gi = ((pos < 4u ? grp : grp2) + (code >> 2 & 1u)) & gmask;
+                rr[t] = int(__ldg(&groups[gi].row[code & 3u]));
+            }
+        }
+    }
+    if (!fast) {
+#pragma unroll
+        for (int t = 0; t < kColMaxCells; ++t) {
+            rr[t] = -1;
+            if (t < col.n) {
+                const int k = col.kbase + t;
+                uint64_t kk;
+                if (query_coord(g, c, g.off[k][0], g.off[k][1], g.off[k][2], kk)) rr[t] = probe_row(groups, cap_mask, kk);
+            }
+        }
+    }
+    uint32_t jbits = 0;
+#pragma unroll
+    for (int t = 0; t < kColMaxCells; ++t) {
+        if (t >= col.n) break;
+        const int k = col.kbase + t;
+        int r = rr[t];
+        if (r >= n_out) {
+            flag(d_status, LAT_ERR_BAD_MAP);
+            r = -1;
+        }
+        nbr[int64_t(k) * n_out + j] = r;
+        if (r >= 0) {
+            const int km = g.k3 - 1 - k;
+            nbr[int64_t(km) * n_out + r] = int32_t(j);
+            atomicOr(mask + r, 1u << km);
+            jbits |= 1u << k;
+        }
+    }
+    if (jbits) atomicOr(mask + j, jbits);
+}
+
+// The columns of a submanifold geometry's lower half (offsets below the
+// centre), in offset order; false if a column has more than kColMaxCells
+// cells (the per-offset kernel then runs).
+static bool subm_columns(const Geom &g, Cols &cols) {
+    const int centre = g.k3 / 2;
+    cols.count = 0;
+    for (int k = 0; k < centre;) {
+        const int ix = g.off[k][0], iy = g.off[k][1];
+        int n = 0;
+        while (k + n < centre && g.off[k + n][0] == ix && g.off[k + n][1] == iy) ++n;
+        if (n > kColMaxCells || cols.count == kColMax) return false;
+        Col &cl = cols.c[cols.count++];
+        cl.delta = g.delta[k];
+        cl.kbase = k;
+        cl.n = n;
+        k += n;
+    }
+    return cols.count > 0;
+}
+
 // A submanifold map with a single offset (1x1x1): every row is its own neighbour.
 __global__ void __launch_bounds__(kQueryThreads) kmap_centre_kernel(int64_t n_out, int32_t *__restrict__ nbr) {
     pdl_enter();
@@ -855,7 +1009,12 @@ extern "C" lat_status lat_kmap_query(const void *table, size_t table_bytes, cons
         f.add(map->nbr + int64_t(centre + 1) * n_out, int64_t(k3 - 1 - centre) * n_out, ~0u);  // filled by mirrors
         f.add(map->mask, n_out, 1u << centre);
         LAT_CUDA_TRY(fill_list(f, s));
-        if (centre > 0) {
+        Cols cols;
+        if (centre > 0 && subm_columns(g, cols)) {
+            LAT_CUDA_TRY(launch_pdl(kmap_probe_col_kernel, dim3(unsigned(nblk), unsigned(cols.count)),
+                                    dim3(kQueryThreads), 0, s, slots, cap_mask, oc, n_out, g, cols, map->nbr, map->mask,
+                                    d_status));
+        } else if (centre > 0) {
             LAT_CUDA_TRY(launch_pdl(kmap_probe_sym_kernel, dim3(unsigned(nblk), unsigned(centre)), dim3(kQueryThreads),
                                     0, s, slots, cap_mask, oc, n_out, g, map->nbr, map->mask, d_status));
         } else {  // 1x1x1: the centre column alone
