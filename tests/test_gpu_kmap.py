@@ -159,8 +159,10 @@ def test_subm_kmap_empty():
 
 
 @pytest.mark.parametrize("ks", [(5, 3, 1), (1, 1, 1), (3, 3, 1), (5, 5, 1), (1, 1, 5), (3, 1, 5), (1, 3, 7),
-                                (1, 5, 3)])
+                                (1, 5, 3), (1, 1, 11), (1, 1, 13)])
 def test_subm_kmap_other_kernels(ks):
+    """(1, 1, 11): a column of five z cells below the centre, the longest the
+    brick lookups take; (1, 1, 13): six, which takes the per-offset probe."""
     rng = np.random.default_rng(3)
     coords = rand_coords(rng, 700, -9, 9, 2)
     km, _ = _subm(coords, ks)
