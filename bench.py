@@ -896,7 +896,7 @@ DOMINANT_KERNEL = "conv_tc_kernel<bf16, 128, 128>, forward: gathered x times W[k
 # DRAM bytes (read + write) per launch of that phase's kernel from an ncu
 # capture of the current kernel on the same workload (None: no capture
 # matches the kernel as it is).
-PHASE_TRAFFIC = {"fwd": 168_263_680 + 83_786_752}
+PHASE_TRAFFIC = {"fwd": 168_960_000 + 83_851_264}
 
 
 def main():
