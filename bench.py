@@ -126,6 +126,7 @@ class SubmLayer:
 
     PHASES = ["hash", "kmap", "fwd", "dgrad", "wgrad"]
     CONV = ["fwd", "dgrad", "wgrad"]
+    SPANS = ["conv_span"]  # forward start to the join of the two gradient streams
 
     def __init__(self, name: str, host: dict, dev: torch.device):
         import sparse_convolution_voxel_b200 as scv
@@ -170,6 +171,7 @@ class SubmLayer:
         rec("kmap", 0)
         scv.lat_kmap_query(self.table, d["coords"], self.geom, self.km.c, self.wsb, s)
         rec("kmap", 1)
+        rec("conv_span", 0)
         rec("fwd", 0)
         scv.lat_sconv_fwd(d["x"], d["w"], self.km.c, self.y, self.wsb, s)
         rec("fwd", 1)
@@ -183,6 +185,7 @@ class SubmLayer:
         scv.lat_sconv_wgrad(d["x"], d["g"], self.km.c, self.dw, self.wsb, s)
         rec("wgrad", 1)
         cur.wait_event(self.ev_dgrad)
+        rec("conv_span", 1)
 
     def outputs(self) -> dict:
         return {"y": self.y, "dx": self.dx, "dw": self.dw}
@@ -460,13 +463,14 @@ def new_events(names) -> dict:
 def phase_times(layer, flush: torch.Tensor, reps: int) -> dict:
     """Mean per-phase event time (ms) over `reps` instrumented steps, L2 flushed
     before each (events between phases; outside any timed region)."""
-    inst = [new_events(layer.PHASES) for _ in range(reps)]
+    names = layer.PHASES + getattr(layer, "SPANS", [])
+    inst = [new_events(names) for _ in range(reps)]
     torch.cuda.synchronize()
     for ev in inst:
         flush_l2(flush)
         layer.step(ev)
     torch.cuda.synchronize()
-    return {p: statistics.mean(ev[p][0].elapsed_time(ev[p][1]) for ev in inst) for p in layer.PHASES}
+    return {p: statistics.mean(ev[p][0].elapsed_time(ev[p][1]) for ev in inst) for p in names}
 
 
 def roofline_of(layer, phase_ms: dict, peaks: dict, fp32_tflops: float | None) -> dict:
@@ -541,14 +545,15 @@ def config_entry(name: str, dev, flush, peaks, fp32_tflops, min_ms: float = 400.
     if st:
         raise layer.scv.LatticeError(st, f"{name}: device status after warm-up")
     pms = phase_times(layer, flush, 10)
-    est = sum(pms.values())
+    est = sum(pms[p] for p in layer.PHASES)
     steps = int(min(2000, max(20, min_ms / max(est, 1e-3))))
     step_ms, _, clocks = time_steps(layer, flush, steps, dev)
     t = statistics.mean(step_ms)
     rl = roofline_of(layer, pms, peaks, fp32_tflops)
     kmap_phases = [p for p in ("hash", "kmap", "downsample", "maps") if p in pms]
     kmap_ms = sum(pms[p] for p in kmap_phases)
-    conv_ms = sum(pms[p] for p in layer.CONV)
+    # the passes' wall span where some of them overlap, else their sum
+    conv_ms = pms.get("conv_span", sum(pms[p] for p in layer.CONV))
     entry = {
         "workload": synthetic.WORKLOADS[name].description, "dtype": synthetic.WORKLOADS[name].dtype,
         "rows": layer.n, "pairs": layer.pair_count(), "steps": steps, "ms_per_step": t,
