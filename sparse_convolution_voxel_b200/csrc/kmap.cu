@@ -11,9 +11,12 @@
 //   1. front end: nbr (offset-major), the neighbour mask and the grouping key
 //              of every output row, and per tile of kScTile rows the counts of
 //              the key's low byte and of the pairs of every offset.
-//                submanifold: kmap_probe_sym_kernel (one thread per (row,
-//                                   offset below the centre), each hit mirrored
-//                                   into the upper half) + kmap_count_kernel
+//                submanifold: kmap_probe_col_kernel (one thread per (row,
+//                                   z-column of offsets below the centre; one or
+//                                   two z-brick group scans per column), each hit
+//                                   mirrored into the upper half; columns of more
+//                                   than kColMaxCells cells: kmap_probe_sym_kernel,
+//                                   one thread per (row, offset)) + kmap_count_kernel
 //                strided/transposed: kmap_probe_kernel (a row per thread)
 //                maps from parents: parent_maps_kernel (+ kmap_count_kernel)
 //   2. row scan: one block per digit (and per offset) turns its per-tile
