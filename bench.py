@@ -154,6 +154,7 @@ class SubmLayer:
         self.wsb_side = self.ws_side.get(scv.lat_sconv_ws_bytes(1, self.cin, self.cout, c, self.dt))
         self.side = torch.cuda.Stream(device=dev, priority=torch.cuda.Stream.priority_range()[1])
         self.ev_fwd, self.ev_dgrad = torch.cuda.Event(), torch.cuda.Event()
+        self.overlap = True  # False: the data gradient on the current stream too (per-pass timing)
         self.pairs = None
 
     def step(self, ev: dict | None = None):
@@ -175,12 +176,13 @@ class SubmLayer:
         rec("fwd", 0)
         scv.lat_sconv_fwd(d["x"], d["w"], self.km.c, self.y, self.wsb, s)
         rec("fwd", 1)
+        dstream = self.side if self.overlap else cur
         self.ev_fwd.record(cur)
-        self.side.wait_event(self.ev_fwd)
-        rec("dgrad", 0, self.side)
-        scv.lat_sconv_dgrad(d["g"], d["w"], self.km.c, True, self.dx, self.wsb_side, s, stream=self.side)
-        rec("dgrad", 1, self.side)
-        self.ev_dgrad.record(self.side)
+        dstream.wait_event(self.ev_fwd)
+        rec("dgrad", 0, dstream)
+        scv.lat_sconv_dgrad(d["g"], d["w"], self.km.c, True, self.dx, self.wsb_side, s, stream=dstream)
+        rec("dgrad", 1, dstream)
+        self.ev_dgrad.record(dstream)
         rec("wgrad", 0)
         scv.lat_sconv_wgrad(d["x"], d["g"], self.km.c, self.dw, self.wsb, s)
         rec("wgrad", 1)
@@ -460,16 +462,25 @@ def new_events(names) -> dict:
     return {p: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for p in names}
 
 
-def phase_times(layer, flush: torch.Tensor, reps: int) -> dict:
+def phase_times(layer, flush: torch.Tensor, reps: int, overlap: bool = False) -> dict:
     """Mean per-phase event time (ms) over `reps` instrumented steps, L2 flushed
-    before each (events between phases; outside any timed region)."""
+    before each (events between phases; outside any timed region).  With
+    overlap=False a layer that runs two passes side by side runs them one
+    after the other, so each phase's time is its own."""
     names = layer.PHASES + getattr(layer, "SPANS", [])
     inst = [new_events(names) for _ in range(reps)]
-    torch.cuda.synchronize()
-    for ev in inst:
-        flush_l2(flush)
-        layer.step(ev)
-    torch.cuda.synchronize()
+    prev = getattr(layer, "overlap", None)
+    if prev is not None:
+        layer.overlap = overlap
+    try:
+        torch.cuda.synchronize()
+        for ev in inst:
+            flush_l2(flush)
+            layer.step(ev)
+        torch.cuda.synchronize()
+    finally:
+        if prev is not None:
+            layer.overlap = prev
     return {p: statistics.mean(ev[p][0].elapsed_time(ev[p][1]) for ev in inst) for p in names}
 
 
@@ -545,6 +556,7 @@ def config_entry(name: str, dev, flush, peaks, fp32_tflops, min_ms: float = 400.
     if st:
         raise layer.scv.LatticeError(st, f"{name}: device status after warm-up")
     pms = phase_times(layer, flush, 10)
+    spans = phase_times(layer, flush, 10, overlap=True) if getattr(layer, "SPANS", None) else {}
     est = sum(pms[p] for p in layer.PHASES)
     steps = int(min(2000, max(20, min_ms / max(est, 1e-3))))
     step_ms, _, clocks = time_steps(layer, flush, steps, dev)
@@ -552,8 +564,8 @@ def config_entry(name: str, dev, flush, peaks, fp32_tflops, min_ms: float = 400.
     rl = roofline_of(layer, pms, peaks, fp32_tflops)
     kmap_phases = [p for p in ("hash", "kmap", "downsample", "maps") if p in pms]
     kmap_ms = sum(pms[p] for p in kmap_phases)
-    # the passes' wall span where some of them overlap, else their sum
-    conv_ms = pms.get("conv_span", sum(pms[p] for p in layer.CONV))
+    # the passes' wall span in the timed schedule (two of them side by side), else their sum
+    conv_ms = spans.get("conv_span", sum(pms[p] for p in layer.CONV))
     entry = {
         "workload": synthetic.WORKLOADS[name].description, "dtype": synthetic.WORKLOADS[name].dtype,
         "rows": layer.n, "pairs": layer.pair_count(), "steps": steps, "ms_per_step": t,
@@ -1011,8 +1023,8 @@ def main():
             "phases": rl["phases"],
             "frac_roofline_step": rl["t_roofline_ms"] / (total_ms / args.steps),
             "phase_note": "per-phase event times from 10 instrumented steps outside the timed region, L2 flushed "
-                          "before each; frac = t_roofline / t per phase; dgrad runs on a second stream beside wgrad, "
-                          "so those two phases overlap",
+                          "before each, the passes one after another (the timed steps run dgrad on a second stream "
+                          "beside wgrad); frac = t_roofline / t per phase",
             "roofline": {"kernel": f"{DOMINANT} ({DOMINANT_KERNEL})", "bound": "hbm", "achieved": achieved,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                          "traffic": PHASE_TRAFFIC.get(DOMINANT), "alg_bytes": pb[DOMINANT], "ms": dominant_ms,
